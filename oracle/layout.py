@@ -1,0 +1,110 @@
+"""Packed (device) weight layouts, written as elementwise index formulas.
+Test infrastructure only: the library's own packer must produce exactly
+these bytes.
+
+The pages say the library turns every format into one standard description
+with the weight, scale and zero point described separately ("Humming:
+open-source kernel library for quantized inference", summary, second
+paragraph).  The concrete device layout is this library's own choice and is
+specified here, one formula per field.
+
+INT4 W4A16, layout version 1 (group size 128):
+  NT = ceil(N / 128) tiles of 128 rows; KB = K / 128 blocks of 128 k.
+  One record per (tile nt, block kb), records in (nt, kb) row-major order,
+  record size REC = 8192 + 256 (+ 128 with zero points) bytes:
+    codes  : byte (c*128 + r)*16 + w*4 + p//2, nibble p%2 (0 = low), where
+             r = n - 128*nt, kk = k - 128*kb, c = kk // 32, w = (kk % 32)//8,
+             e = kk % 8 and p = (e % 2)*4 + e // 2;
+    scale  : fp16 bits, little endian, at byte 8192 + 2*r;
+    zero   : uint8 at byte 8192 + 256 + r (only with zero points).
+  Rows n >= N (tile padding) hold code 0, scale 0 and zero 0.
+  Experts (MoE) are stored one after another, each NT*KB*REC bytes.
+"""
+
+import numpy as np
+
+from . import formats as F
+
+W4_TILE_N = 128
+W4_BLOCK_K = 128
+
+
+def w4a16_record_bytes(has_zero):
+    return 8192 + 256 + (128 if has_zero else 0)
+
+
+def w4a16_packed_bytes(n, k, has_zero, num_experts=1):
+    nt = -(-n // W4_TILE_N)
+    return num_experts * nt * (k // W4_BLOCK_K) * w4a16_record_bytes(has_zero)
+
+
+def w4a16_code_byte_and_nibble(n, k, kdim, has_zero):
+    """Elementwise formula: (byte offset in the expert blob, nibble 0/1) of
+    code q[n, k].  Works on numpy arrays of indices."""
+    n = np.asarray(n, dtype=np.int64)
+    k = np.asarray(k, dtype=np.int64)
+    kb_count = kdim // W4_BLOCK_K
+    rec = w4a16_record_bytes(has_zero)
+    nt, r = n // W4_TILE_N, n % W4_TILE_N
+    kb, kk = k // W4_BLOCK_K, k % W4_BLOCK_K
+    c, w, e = kk // 32, (kk % 32) // 8, kk % 8
+    p = (e % 2) * 4 + e // 2
+    byte = (nt * kb_count + kb) * rec + (c * 128 + r) * 16 + w * 4 + p // 2
+    return byte, p % 2
+
+
+def w4a16_scale_byte(n, kb, kdim, has_zero):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    rec = w4a16_record_bytes(has_zero)
+    nt, r = n // W4_TILE_N, n % W4_TILE_N
+    return (nt * (kdim // W4_BLOCK_K) + kb) * rec + 8192 + 2 * r
+
+
+def w4a16_zero_byte(n, kb, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    rec = w4a16_record_bytes(True)
+    nt, r = n // W4_TILE_N, n % W4_TILE_N
+    return (nt * (kdim // W4_BLOCK_K) + kb) * rec + 8192 + 256 + r
+
+
+def w4a16_pack(qweight, scales, zeros, group=128):
+    """Canonical (int32 [N, K/8], fp16 [N, K/128], uint8 [N, K/128] | None)
+    -> packed uint8 blob, by scattering every element to the position the
+    formulas above give."""
+    assert group == W4_BLOCK_K
+    codes = F.int4_unpack_words(qweight)
+    n, k = codes.shape
+    has_zero = zeros is not None
+    out = np.zeros(w4a16_packed_bytes(n, k, has_zero), dtype=np.uint8)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    byte, nib = w4a16_code_byte_and_nibble(nn.ravel(), kk.ravel(), k, has_zero)
+    vals = codes.ravel().astype(np.uint8) << (4 * nib).astype(np.uint8)
+    np.bitwise_or.at(out, byte, vals)
+    sb = np.asarray(scales, dtype=np.float16).view(np.uint16)
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // group), indexing="ij")
+    off = w4a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    out[off] = (sb.ravel() & 0xFF).astype(np.uint8)
+    out[off + 1] = (sb.ravel() >> 8).astype(np.uint8)
+    if has_zero:
+        zo = w4a16_zero_byte(ng.ravel(), gg.ravel(), k)
+        out[zo] = np.asarray(zeros, dtype=np.uint8).ravel()
+    return out
+
+
+def w4a16_unpack(blob, n, k, has_zero):
+    """Inverse of w4a16_pack: packed blob -> (codes uint8 [N, K],
+    scales fp16 [N, K/128], zeros uint8 [N, K/128] | None)."""
+    blob = np.asarray(blob, dtype=np.uint8)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    byte, nib = w4a16_code_byte_and_nibble(nn.ravel(), kk.ravel(), k, has_zero)
+    codes = ((blob[byte] >> (4 * nib).astype(np.uint8)) & 0xF).reshape(n, k)
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // W4_BLOCK_K), indexing="ij")
+    off = w4a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    sbits = blob[off].astype(np.uint16) | (blob[off + 1].astype(np.uint16) << 8)
+    scales = sbits.reshape(n, k // W4_BLOCK_K).view(np.float16)
+    zeros = None
+    if has_zero:
+        zeros = blob[w4a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // W4_BLOCK_K)
+    return codes.astype(np.uint8), scales, zeros

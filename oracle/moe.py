@@ -1,0 +1,62 @@
+"""MoE routing and expert-sorted permutation (test infrastructure).
+
+The pages name a "Grouped" MoE path ("Humming: open-source kernel library
+for quantized inference", summary, fifth paragraph: the grouped MoE path on
+B300; Humming news page, comparison table row "MoE W4A16, B300, large
+batch").  They do not describe routing; the workload fixes top-8 of 256
+experts from a softmax over router logits, with tokens permuted into
+expert-sorted order and per-expert row offsets.
+
+Readings (the pages are silent):
+  * top-k by probability equals top-k by logit (softmax is monotone), so
+    selection is done on the logits, exactly, without exp rounding;
+  * ties go to the lower expert index; slots within a token are ordered by
+    descending logit (ties: lower index first);
+  * the sorted order is (expert ascending, flattened slot index t*k+j
+    ascending), which is unique and therefore bit-exactly checkable.
+"""
+
+import numpy as np
+
+
+def topk_by_logit(logits, k):
+    """logits fp32 [T, E] -> expert ids int32 [T, k], descending logit,
+    ties to the lower expert index."""
+    l = np.asarray(logits, dtype=np.float32)
+    t, e = l.shape
+    order = np.argsort(-l.astype(np.float64), axis=1, kind="stable")
+    return order[:, :k].astype(np.int32)
+
+
+def softmax_topk_weights(logits, ids):
+    """Softmax probabilities (fp64) of the selected experts, not
+    renormalised.  Reported for completeness; no kernel consumes them."""
+    l = np.asarray(logits, dtype=np.float64)
+    p = np.exp(l - l.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return np.take_along_axis(p, np.asarray(ids, dtype=np.int64), axis=1)
+
+
+def permute(topk_ids, num_experts):
+    """topk ids [T, k] -> (counts [E], offsets [E+1], sorted_src [T*k]).
+
+    counts[e]  = number of slots routed to e;
+    offsets    = exclusive prefix sum of counts, offsets[E] = T*k;
+    sorted_src = flattened slot indices t*k+j ordered by (expert, t*k+j).
+    """
+    ids = np.asarray(topk_ids, dtype=np.int64).ravel()
+    counts = np.bincount(ids, minlength=num_experts).astype(np.int32)
+    offsets = np.zeros(num_experts + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    # explicit (expert, slot) ordering: build buckets slot by slot
+    buckets = [[] for _ in range(num_experts)]
+    for slot, e in enumerate(ids.tolist()):
+        buckets[e].append(slot)
+    sorted_src = np.array([s for b in buckets for s in b], dtype=np.int32)
+    return counts, offsets, sorted_src
+
+
+def gather_rows(a, sorted_src, k):
+    """A_sorted[i] = A[sorted_src[i] // k] (a bit copy of the bf16 row)."""
+    src_tok = np.asarray(sorted_src, dtype=np.int64) // k
+    return np.asarray(a)[src_tok]

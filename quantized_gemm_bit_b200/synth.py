@@ -1,0 +1,79 @@
+"""Seeded synthetic inputs shaped like the method's workloads.
+
+This module only draws random numbers (torch CPU generator, fixed seeds) and
+puts them in the canonical containers the library and the oracle both read.
+It holds none of the method's arithmetic: no dequantization, no GEMM, no
+routing.  The one quantization step it performs (FP8 activations for the
+W4A8-MXFP4 workload) uses torch's own float8_e4m3fn cast, a library routine.
+
+Recipes (one per workload; seed = workload index * 1000 + shape index):
+  * W4A16: qweight int32 [N, K/8] with every bit uniform (= eight uniform
+    uint4 codes per word, packed along K, low nibble first); fp16 scales
+    0.002 + 0.01*|N(0,1)| per (row, group of 128 along K); zero points
+    uniform in [0, 15] (asymmetric) or none (symmetric, zero point 8);
+    activations bf16 N(0,1).
+  * W4A8-MXFP4: FP4 codes uniform over the 16 codes, two per byte (even k
+    low nibble); one E8M0 scale per 32 K with exponent uniform in [-8, -2];
+    activations bf16 N(0,1) widened to fp32, per-token scale amax/448 (fp32),
+    E4M3 codes by torch's cast of x/scale (clamped to +-448).
+  * NVFP4: bf16 N(0,1) draws for both operands; the two-level quantization
+    that turns them into codes is the method's arithmetic and is not done
+    here.
+  * MoE: router logits fp32 N(0,1) [T, E]; activations bf16 N(0,1).
+"""
+
+import torch
+
+
+def _gen(seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def bf16_normal(rows, cols, seed):
+    """bf16 N(0,1) [rows, cols] (torch tensor, CPU)."""
+    g = _gen(seed)
+    return torch.randn(rows, cols, generator=g, dtype=torch.float32).to(torch.bfloat16)
+
+
+def w4a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
+    """Canonical W4A16 weights.  Returns (qweight int32 [.., N, K/8],
+    scales fp16 [.., N, K/G], zeros uint8 [.., N, K/G] or None).  With
+    `experts` set, a leading expert dimension is added."""
+    assert k % group == 0 and k % 8 == 0
+    g = _gen(seed)
+    lead = () if experts is None else (experts,)
+    qweight = torch.randint(-(2 ** 31), 2 ** 31, lead + (n, k // 8), generator=g,
+                            dtype=torch.int64).to(torch.int32)
+    scales = (0.002 + 0.01 * torch.randn(lead + (n, k // group), generator=g).abs()).to(torch.float16)
+    zeros = None
+    if asym:
+        zeros = torch.randint(0, 16, lead + (n, k // group), generator=g, dtype=torch.uint8)
+    return qweight, scales, zeros
+
+
+def mxfp4_weights(n, k, seed=0):
+    """MXFP4 weights: codes uint8 [N, K/2] (two uniform FP4 codes per byte),
+    E8M0 scales uint8 [N, K/32] with exponent uniform in [-8, -2]."""
+    assert k % 32 == 0
+    g = _gen(seed)
+    codes = torch.randint(0, 256, (n, k // 2), generator=g, dtype=torch.uint8)
+    e8m0 = (127 + torch.randint(-8, -1, (n, k // 32), generator=g, dtype=torch.int32)).to(torch.uint8)
+    return codes, e8m0
+
+
+def fp8_activations(m, k, seed=0):
+    """E4M3 activations with a per-token fp32 scale amax/448 (library cast).
+    Returns (codes uint8 [M, K], scale float32 [M])."""
+    x = bf16_normal(m, k, seed).to(torch.float32)
+    amax = x.abs().amax(dim=1)
+    s = amax / 448.0
+    s = torch.where(amax > 0, s, torch.ones_like(s))
+    q = (x / s[:, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8), s.to(torch.float32)
+
+
+def router_logits(t, e, seed=0):
+    g = _gen(seed)
+    return torch.randn(t, e, generator=g, dtype=torch.float32)

@@ -1,0 +1,131 @@
+"""Pins for the oracle's packed-layout formulas and MoE routing."""
+
+import itertools
+
+import numpy as np
+
+from oracle import formats as F
+from oracle import layout as L
+from oracle import moe as R
+from quantized_gemm_bit_b200 import synth
+
+
+def test_w4a16_layout_is_a_bijection():
+    for n, k, asym in ((128, 256, False), (200, 384, True)):
+        nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+        byte, nib = L.w4a16_code_byte_and_nibble(nn.ravel(), kk.ravel(), k, asym)
+        slot = byte * 2 + nib
+        assert len(np.unique(slot)) == n * k
+        total = L.w4a16_packed_bytes(n, k, asym)
+        assert slot.max() < 2 * total
+        # codes, scales and zeros never overlap
+        ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+        sb = L.w4a16_scale_byte(ng.ravel(), gg.ravel(), k, asym)
+        used = set(byte.tolist())
+        assert not (used & set(sb.tolist())) and not (used & set((sb + 1).tolist()))
+        if asym:
+            zb = L.w4a16_zero_byte(ng.ravel(), gg.ravel(), k)
+            assert not (used & set(zb.tolist())) and not (set(zb.tolist()) & set(sb.tolist()))
+
+
+def test_w4a16_pack_unpack_roundtrip():
+    for asym in (False, True):
+        q, s, z = synth.w4a16_weights(136, 256, 128, asym, seed=51)
+        blob = L.w4a16_pack(q.numpy(), s.numpy(), None if z is None else z.numpy())
+        assert blob.size == L.w4a16_packed_bytes(136, 256, asym)
+        codes, s2, z2 = L.w4a16_unpack(blob, 136, 256, asym)
+        assert np.array_equal(codes, F.int4_unpack_words(q.numpy()))
+        assert np.array_equal(s2.view(np.uint16), s.numpy().view(np.uint16))
+        if asym:
+            assert np.array_equal(z2, z.numpy())
+        # padding rows 136..255 of the second tile stay zero
+        nt_bytes = 2 * L.w4a16_record_bytes(asym)
+        rec = L.w4a16_record_bytes(asym)
+        tile1 = blob[nt_bytes:].reshape(2, rec)
+        codes1 = tile1[:, :8192].reshape(2, 4, 128, 16)
+        assert np.all(codes1[:, :, 8:, :] == 0)
+
+
+def test_w4a16_layout_small_hand_example():
+    """Code q[n=1, k=3] (chunk 0, word 0, element 3 -> nibble 5) lands at
+    byte (0*128 + 1)*16 + 0*4 + 2, high nibble; q[0, 33] (chunk 1, word 0,
+    element 1 -> nibble 4) at byte (1*128 + 0)*16 + 2, low nibble."""
+    b, nib = L.w4a16_code_byte_and_nibble(1, 3, 128, False)
+    assert (int(b), int(nib)) == (18, 1)
+    b, nib = L.w4a16_code_byte_and_nibble(0, 33, 128, False)
+    assert (int(b), int(nib)) == (2050, 0)
+
+
+def test_topk_by_logit_brute_force():
+    rng = np.random.default_rng(61)
+    logits = rng.standard_normal((40, 8)).astype(np.float32)
+    logits[3, 2] = logits[3, 5]                          # a tie
+    ids = R.topk_by_logit(logits, 3)
+    for t in range(40):
+        ranked = sorted(range(8), key=lambda e: (-float(logits[t, e]), e))
+        assert list(ids[t]) == ranked[:3]
+
+
+def test_topk_set_invariants_full_size():
+    logits = synth.router_logits(64, 256, seed=3001).numpy()
+    ids = R.topk_by_logit(logits, 8)
+    for t in range(64):
+        sel = set(ids[t].tolist())
+        assert len(sel) == 8
+        rest = [e for e in range(256) if e not in sel]
+        assert logits[t, list(sel)].min() >= logits[t, rest].max()
+
+
+def test_permute_invariants_and_brute_force():
+    rng = np.random.default_rng(62)
+    for t, e, k in ((5, 8, 2), (33, 16, 4), (64, 256, 8)):
+        logits = rng.standard_normal((t, e)).astype(np.float32)
+        ids = R.topk_by_logit(logits, k)
+        counts, off, src = R.permute(ids, e)
+        assert off[0] == 0 and off[-1] == t * k and np.all(np.diff(off) == counts)
+        assert sorted(src.tolist()) == list(range(t * k))
+        flat = ids.ravel()
+        for ex in range(e):
+            seg = src[off[ex]:off[ex + 1]]
+            assert np.all(flat[seg] == ex)
+            assert np.all(np.diff(seg // k) > 0)          # token strictly increasing
+        # brute force: sort all (expert, slot) pairs
+        pairs = sorted((int(flat[s]), s) for s in range(t * k))
+        assert [p[1] for p in pairs] == src.tolist()
+
+
+def test_permute_handles_empty_experts_and_duplicates():
+    ids = np.array([[3, 3], [0, 3]], dtype=np.int32)      # duplicates allowed
+    counts, off, src = R.permute(ids, 5)
+    assert counts.tolist() == [1, 0, 0, 3, 0]
+    assert off.tolist() == [0, 1, 1, 1, 4, 4]
+    assert src.tolist() == [2, 0, 1, 3]
+
+
+def test_gather_rows():
+    a = np.arange(12, dtype=np.uint16).reshape(4, 3)
+    src = np.array([5, 0, 7, 2], dtype=np.int32)
+    out = R.gather_rows(a, src, 2)
+    assert np.array_equal(out, a[[2, 0, 3, 1]])
+
+
+def test_synth_fp8_matches_oracle_quantizer():
+    """The generator's library cast and the oracle's own quantizer agree."""
+    q, s = synth.fp8_activations(16, 512, seed=2000)
+    x = synth.bf16_normal(16, 512, 2000).float().numpy()
+    q2, s2 = F.fp8_per_token_quantize(x)
+    assert np.array_equal(s.numpy(), s2)
+    assert np.array_equal(F.e4m3_decode(q.numpy()), F.e4m3_decode(q2))
+
+
+def test_synth_distributions():
+    q, s, z = synth.w4a16_weights(256, 1024, 128, True, seed=0)
+    codes = F.int4_unpack_words(q.numpy())
+    hist = np.bincount(codes.ravel(), minlength=16) / codes.size
+    assert np.all(np.abs(hist - 1 / 16) < 0.005)
+    sv = s.numpy().astype(np.float64)
+    assert sv.min() >= 0.002 - 1e-6 and abs(sv.mean() - (0.002 + 0.01 * np.sqrt(2 / np.pi))) < 5e-4
+    assert z.numpy().max() == 15 and z.numpy().min() == 0
+    codes, e8 = synth.mxfp4_weights(64, 1024, seed=2)
+    assert set(np.unique(e8.numpy()).tolist()) == set(range(119, 126))
+    assert list(itertools.islice(range(3), 1)) == [0]
