@@ -1,0 +1,220 @@
+/*
+ * hq.h -- C ABI of the B200 (sm_100a) low-bit-weight GEMM library with
+ * fused dequantization.
+ *
+ * What it computes.  A linear layer y = x * W^T whose weights W are stored
+ * in a low-bit format and are dequantized inside the GEMM kernel.  The
+ * method (the Humming quantized-inference kernel library) is described on
+ * news pages only:
+ *   [P-fa]  Humming news page (news.cocoloop.cn, fr), section "Une seule
+ *           bibliotheque pour une longue liste de formats": WnA16 / W8A8 /
+ *           W4A8 / W4A4; INT1..INT8, FP4..FP8, MXFP4, MXINT4, NVFP4; table
+ *           rows "W4A16 dense, petits lots", "W4A8-MXFP4, H200",
+ *           "MoE W4A16, B300, grands lots".
+ *   [P-fa2] "Humming: open-source kernel library for quantized inference"
+ *           (news.ditty.ir), summary paragraph 2 (one standard description
+ *           in which weight, scale, zero point and the other parameters are
+ *           described separately), paragraph 3 (Layer / Compute / Tuning
+ *           configs: shapes+dtype+arch / GEMM type / tile, stages, MMA),
+ *           paragraph 4 (MXFP4 weights converted inside the kernel),
+ *           paragraph 5 (the "Grouped" MoE path).
+ *   [P-pt]  "Ant Group e vLLM lancam a biblioteca open source Humming"
+ *           (aube.news), quantization paragraph (dense and MoE layers).
+ * Element formats follow the public standards the pages name: OCP MX v1.0
+ * (e2m1, E8M0, 32-element blocks), OCP FP8 (E4M3), NVIDIA NVFP4 (e2m1 with
+ * an E4M3 scale per 16 elements and an fp32 tensor scale).
+ *
+ * Conventions shared by every entry point.
+ *   - A (activations) is [M, K] row-major, K contiguous.  W is logically
+ *     [N, K] (K contiguous).  C is [M, N] row-major bf16.
+ *   - The caller owns all memory.  The library never allocates device
+ *     memory, never synchronizes a stream (except hq_check_device_status),
+ *     and launches only on the caller's stream.
+ *   - Arguments are validated on the host before any launch; on failure a
+ *     non-OK status is returned and nothing is launched or written.
+ *   - Errors found on the device (a bounded wait that ran out, offsets that
+ *     are not monotone) are written to the workspace error word and read
+ *     back by hq_check_device_status.
+ *   - Device pointers must be 16-byte aligned; workspaces 256-byte aligned.
+ *   - A workspace must be zero-filled once after allocation; every call
+ *     that completes leaves it zero-filled again (apart from the error word,
+ *     which hq_check_device_status clears).
+ *   - Pointers named *_dev are device pointers; *_host are host pointers.
+ */
+#ifndef HQ_H_
+#define HQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Packed-layout version written by hq_quant_desc_init and checked by every
+ * call taking a descriptor (a descriptor from another layout version is
+ * rejected with HQ_ERR_LAYOUT_VERSION). */
+#define HQ_LAYOUT_VERSION 1
+
+typedef struct CUstream_st* hq_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_INVALID_ARG = 1,
+  HQ_ERR_UNSUPPORTED = 2,
+  HQ_ERR_ALIGNMENT = 3,
+  HQ_ERR_WORKSPACE_TOO_SMALL = 4,
+  HQ_ERR_LAYOUT_VERSION = 5,
+  HQ_ERR_CUDA = 6,
+  HQ_ERR_DEVICE_TIMEOUT = 7,
+  HQ_ERR_DEVICE_BAD_OFFSETS = 8,
+  HQ_ERR_NO_DEVICE = 9
+} hq_status;
+
+typedef enum {
+  HQ_FMT_INT4 = 1,  /* unsigned INT4 codes, fp16 scale + optional uint4 zero point per group of 128 K */
+  HQ_FMT_MXFP4 = 2, /* e2m1 codes, E8M0 scale per 32 K                                             */
+  HQ_FMT_NVFP4 = 3  /* e2m1 codes, E4M3 scale per 16 K, fp32 tensor scale                          */
+} hq_format;
+
+/* Quantization description ([P-fa2] paragraph 2) plus the Layer Config
+ * shape fields ([P-fa2] paragraph 3).  Fill it with hq_quant_desc_init. */
+typedef struct {
+  int32_t layout_version; /* HQ_LAYOUT_VERSION                                         */
+  int32_t fmt;            /* hq_format                                                 */
+  int32_t n;              /* output features (weight rows), per expert                 */
+  int32_t k;              /* input features (reduction length)                         */
+  int32_t group_size;     /* INT4: 128; MXFP4: 32; NVFP4: 16                           */
+  int32_t has_zero_point; /* INT4: 1 = uint4 zero point per group, 0 = symmetric (8)   */
+  int32_t num_experts;    /* 1 = dense layer; >1 = MoE weights stored expert after expert */
+} hq_quant_desc;
+
+/* Execution choices (the Tuning Config of [P-fa2] paragraph 3).  Pass NULL
+ * to let the library's heuristic choose; a zero field also means "choose".
+ *   tile_m   : token tile (the MMA N extent): 16, 32, 64, 128 or 256
+ *   tile_n   : weight rows per tile: 128 (the only value)
+ *   tile_k   : K per pipeline stage: 128 (fixed by the packed layout)
+ *   stages   : shared-memory pipeline depth
+ *   split_k  : number of K splits reduced in the workspace (>= 1)
+ *   cta_group: 1 (one SM per MMA)
+ *   variant  : 0                                                             */
+typedef struct {
+  int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;
+} hq_tuning;
+
+/* Library and layout version. */
+int hq_layout_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hq_status_string(hq_status s);
+
+/* Fill *d.  Returns HQ_ERR_INVALID_ARG / HQ_ERR_UNSUPPORTED for shapes or
+ * formats the library cannot run:
+ *   INT4 : k % 128 == 0, group_size == 128, n >= 1
+ *   MXFP4: k % 128 == 0, group_size == 32, has_zero_point == 0
+ *   NVFP4: k % 256 == 0, group_size == 16, has_zero_point == 0
+ *   num_experts >= 1 (MoE only for INT4). */
+hq_status hq_quant_desc_init(hq_quant_desc* d, int32_t fmt, int32_t n, int32_t k, int32_t group_size,
+                             int32_t has_zero_point, int32_t num_experts);
+
+/* Size in bytes of the packed weight blob for *d (0 if *d is invalid). */
+size_t hq_packed_size(const hq_quant_desc* d);
+
+/* Offline weight packer ([P-fa2] paragraph 2: weight, scale and zero point
+ * described separately -> one device layout).  Host memory in, host memory
+ * out; the caller copies the result to the device.  Canonical inputs,
+ * experts back to back:
+ *   INT4 : codes_host  = int32 [E][N][K/8], element k in bits 4*(k%8)..+3
+ *          scales_host = fp16 bits [E][N][K/128]
+ *          zeros_host  = uint8 [E][N][K/128] (0..15), NULL when symmetric
+ *   MXFP4: codes_host  = uint8 [N][K/2] (even k in the low nibble)
+ *          scales_host = uint8 E8M0 [N][K/32]
+ *   NVFP4: codes_host  = uint8 [N][K/2]; scales_host = uint8 E4M3 [N][K/16];
+ *          global_scale = the fp32 tensor scale of the weights.
+ * The output layout is documented in DESIGN.md ("packed layouts").
+ * Errors: HQ_ERR_INVALID_ARG (NULL pointers, zeros given for a symmetric
+ * descriptor or missing for an asymmetric one, a zero point > 15),
+ * HQ_ERR_WORKSPACE_TOO_SMALL (out_bytes < hq_packed_size). */
+hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
+                          const void* zeros_host, float global_scale, void* out_host, size_t out_bytes);
+
+/* Workspace bytes that hq_gemm_w4a16 (fmt INT4, num_experts 1),
+ * hq_gemm_mxfp4_a8, hq_gemm_nvfp4 or hq_grouped_gemm_moe need for M rows
+ * (total sorted rows for MoE) and the given tuning (NULL = heuristic). */
+size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
+
+/* Dense W4A16 GEMM ([P-fa] table row "W4A16 dense"): C = A * W_hat^T with
+ * W_hat[n,k] = (q[n,k] - z[n,k/128]) * s[n,k/128] dequantized in-kernel.
+ *   d            : INT4 descriptor with num_experts == 1
+ *   packed_w_dev : blob from hq_pack_weights (hq_packed_size bytes)
+ *   a_dev        : bf16 [m][d->k]
+ *   m            : rows of A (m == 0 returns HQ_OK without launching)
+ *   c_dev        : bf16 [m][d->n], written
+ *   ws_dev       : workspace of at least hq_workspace_size bytes */
+hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const void* a_dev, int32_t m,
+                        void* c_dev, const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* W4A8-MXFP4 GEMM ([P-fa] table row "W4A8-MXFP4"; [P-fa2] paragraph 4):
+ * C[m,n] = s_m * sum_k E4M3(a[m,k]) * e2m1(w[n,k]) * 2^(e[n,k/32]-127).
+ *   a_e4m3_dev : uint8 [m][k] E4M3 codes;  a_scale_dev : fp32 [m] */
+hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, const void* a_e4m3_dev,
+                           const float* a_scale_dev, int32_t m, void* c_dev, const hq_tuning* t, void* ws_dev,
+                           size_t ws_bytes, hq_stream_t stream);
+
+/* NVFP4 W4A4 GEMM ([P-fa] format list, W4A4 combination):
+ * C = (g_a * g_w) * sum_k e2m1(a)*sf_a * e2m1(w)*sf_w.
+ *   a_fp4_dev : uint8 [m][k/2] (even k low nibble); a_sf_dev : uint8 E4M3
+ *   [m][k/16]; a_global : fp32 tensor scale of A.  g_w is in the blob. */
+hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const void* a_fp4_dev,
+                        const void* a_sf_dev, float a_global, int32_t m, void* c_dev, const hq_tuning* t,
+                        void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* MoE routing ([P-fa2] paragraph 5, "Grouped" path): top-k experts per
+ * token by router logit (equal to top-k by softmax probability), ties to
+ * the lower expert index, slots in descending logit order.
+ *   logits_dev : fp32 [t][e];  topk_ids_dev : int32 [t][k], written
+ *   1 <= k <= 16, k <= e <= 1024. */
+hq_status hq_moe_topk(const float* logits_dev, int32_t t, int32_t e, int32_t k, int32_t* topk_ids_dev,
+                      hq_stream_t stream);
+
+/* Workspace bytes hq_moe_permute needs. */
+size_t hq_moe_permute_workspace_size(int32_t t, int32_t k, int32_t e);
+
+/* Expert-sorted permutation: expert_offsets = exclusive prefix sum of the
+ * per-expert slot counts ([e+1], offsets[e] = t*k); sorted_src lists the
+ * flattened slots t*k+j ordered by (expert, slot); when a_dev and
+ * a_sorted_dev are both non-NULL, a_sorted[i] = a[sorted_src[i] / k]
+ * (bf16 rows of `hidden` elements).  Ids outside [0, e) set
+ * HQ_ERR_DEVICE_BAD_OFFSETS in the workspace error word. */
+hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int32_t e, int32_t* sorted_src_dev,
+                         int32_t* expert_offsets_dev, const void* a_dev, int32_t hidden, void* a_sorted_dev,
+                         void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* Grouped MoE W4A16 GEMM, one launch for all experts ([P-fa] table row
+ * "MoE W4A16"): for every expert e, rows [off[e], off[e+1]) of A_sorted
+ * times W_hat_e^T.  The tile scheduler reads expert_offsets on the device
+ * (no host synchronization).
+ *   d              : INT4 descriptor, num_experts = e (per-expert n, k)
+ *   packed_w_dev   : blob of all experts from hq_pack_weights
+ *   a_sorted_dev   : bf16 [total_rows][k]
+ *   expert_offsets_dev : int32 [e+1], monotone, offsets[e] == total_rows
+ *   c_sorted_dev   : bf16 [total_rows][n], written */
+hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, const void* a_sorted_dev,
+                              const int32_t* expert_offsets_dev, int32_t total_rows, void* c_sorted_dev,
+                              const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* Synchronizes `stream`, reads the workspace error word, clears it and
+ * returns it (HQ_OK when no device-side error was recorded). */
+hq_status hq_check_device_status(void* ws_dev, hq_stream_t stream);
+
+/* Test hook for the bounded-wait machinery: launches one block that waits
+ * on a barrier nobody arrives on, with a limit of `limit_ns`; the wait runs
+ * out and the kernel writes HQ_ERR_DEVICE_TIMEOUT to the workspace error
+ * word and returns normally.  limit_ns must be <= 100 ms. */
+hq_status hq_debug_timeout_probe(void* ws_dev, uint64_t limit_ns, hq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HQ_H_ */

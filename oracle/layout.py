@@ -108,3 +108,45 @@ def w4a16_unpack(blob, n, k, has_zero):
     if has_zero:
         zeros = blob[w4a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // W4_BLOCK_K)
     return codes.astype(np.uint8), scales, zeros
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 / NVFP4, layout version 1
+#   codes  : [NP][K/2] bytes, row major, even k low nibble (NP = N rounded up
+#            to 128, extra rows zero)
+#   scales : from byte NP*K/2; per (tile nt, group g of 4 scale blocks) a
+#            512-byte block in (nt, g) order; scale of row n, block b sits at
+#            block (nt = n//128, g = b//4), byte (n%32)*16 + ((n%128)//32)*4 + b%4
+#   NVFP4 adds a 16-byte tail holding the fp32 tensor scale.
+# ---------------------------------------------------------------------------
+
+
+def fp4_packed_bytes(n, k, block, with_tail):
+    np_ = -(-n // 128) * 128
+    nt = np_ // 128
+    groups = (k // block) // 4
+    return np_ * k // 2 + nt * groups * 512 + (16 if with_tail else 0)
+
+
+def fp4_scale_byte_np(n, b, k, block, np_rows):
+    n = np.asarray(n, dtype=np.int64)
+    b = np.asarray(b, dtype=np.int64)
+    groups = (k // block) // 4
+    nt, g = n // 128, b // 4
+    return (np_rows * k // 2 + (nt * groups + g) * 512 + (n % 32) * 16 + ((n % 128) // 32) * 4 + b % 4)
+
+
+def fp4_pack(codes_packed, scales, block, global_scale=None):
+    """Canonical (uint8 [N, K/2], uint8 [N, K/block]) -> packed blob."""
+    codes_packed = np.asarray(codes_packed, dtype=np.uint8)
+    scales = np.asarray(scales, dtype=np.uint8)
+    n, kh = codes_packed.shape
+    k = kh * 2
+    np_rows = -(-n // 128) * 128
+    out = np.zeros(fp4_packed_bytes(n, k, block, global_scale is not None), dtype=np.uint8)
+    out[: n * kh] = codes_packed.ravel()
+    nn, bb = np.meshgrid(np.arange(n), np.arange(k // block), indexing="ij")
+    out[fp4_scale_byte_np(nn.ravel(), bb.ravel(), k, block, np_rows)] = scales.ravel()
+    if global_scale is not None:
+        out[-16:-12] = np.frombuffer(np.float32(global_scale).tobytes(), dtype=np.uint8)
+    return out

@@ -1,0 +1,295 @@
+// C-ABI entry points: argument validation, planning and dispatch.
+// Every check happens on the host before any launch; a failing call returns
+// a status and leaves all memory untouched.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "hq_internal.h"
+
+namespace hq {
+
+hq_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HQ_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    DeviceInfo di{};
+    di.device = dev;
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return HQ_ERR_NO_DEVICE;
+    di.num_sms = v;
+    cudaDeviceGetAttribute(&di.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&di.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    di.max_smem_optin = (size_t)v;
+    cache[dev] = di;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  // The kernels are built for sm_100a only.
+  if (out->cc_major != 10 || out->cc_minor != 0) return HQ_ERR_NO_DEVICE;
+  return HQ_OK;
+}
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+hq_status check_desc(const hq_quant_desc* d) {
+  if (!d) return HQ_ERR_INVALID_ARG;
+  if (d->layout_version != HQ_LAYOUT_VERSION) return HQ_ERR_LAYOUT_VERSION;
+  if (d->n < 1 || d->k < 1 || d->num_experts < 1) return HQ_ERR_INVALID_ARG;
+  switch (d->fmt) {
+    case HQ_FMT_INT4:
+      if (d->group_size != 128 || d->k % 128 != 0) return HQ_ERR_UNSUPPORTED;
+      if (d->has_zero_point != 0 && d->has_zero_point != 1) return HQ_ERR_INVALID_ARG;
+      if (d->num_experts > 1024) return HQ_ERR_UNSUPPORTED;
+      return HQ_OK;
+    case HQ_FMT_MXFP4:
+      if (d->group_size != 32 || d->k % 128 != 0 || d->has_zero_point || d->num_experts != 1)
+        return HQ_ERR_UNSUPPORTED;
+      return HQ_OK;
+    case HQ_FMT_NVFP4:
+      if (d->group_size != 16 || d->k % 256 != 0 || d->has_zero_point || d->num_experts != 1)
+        return HQ_ERR_UNSUPPORTED;
+      return HQ_OK;
+    default:
+      return HQ_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace
+
+// Packed size per format (the layouts are written out in hq_pack.cpp).
+size_t packed_size_impl(const hq_quant_desc& d);
+hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scales, const void* zeros, float g,
+                    void* out);
+
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" {
+
+int hq_layout_version(void) { return HQ_LAYOUT_VERSION; }
+
+const char* hq_status_string(hq_status s) {
+  switch (s) {
+    case HQ_OK: return "ok";
+    case HQ_ERR_INVALID_ARG: return "invalid argument";
+    case HQ_ERR_UNSUPPORTED: return "unsupported shape, format or tuning";
+    case HQ_ERR_ALIGNMENT: return "pointer not aligned (16 B for data, 256 B for workspaces)";
+    case HQ_ERR_WORKSPACE_TOO_SMALL: return "buffer or workspace too small";
+    case HQ_ERR_LAYOUT_VERSION: return "descriptor from another packed-layout version";
+    case HQ_ERR_CUDA: return "CUDA runtime or launch error";
+    case HQ_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case HQ_ERR_DEVICE_BAD_OFFSETS: return "expert ids or offsets out of range on the device";
+    case HQ_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+hq_status hq_quant_desc_init(hq_quant_desc* d, int32_t fmt, int32_t n, int32_t k, int32_t group_size,
+                             int32_t has_zero_point, int32_t num_experts) {
+  if (!d) return HQ_ERR_INVALID_ARG;
+  hq_quant_desc t{};
+  t.layout_version = HQ_LAYOUT_VERSION;
+  t.fmt = fmt;
+  t.n = n;
+  t.k = k;
+  t.group_size = group_size;
+  t.has_zero_point = has_zero_point;
+  t.num_experts = num_experts;
+  hq_status st = check_desc(&t);
+  if (st != HQ_OK) return st;
+  *d = t;
+  return HQ_OK;
+}
+
+size_t hq_packed_size(const hq_quant_desc* d) {
+  if (check_desc(d) != HQ_OK) return 0;
+  return packed_size_impl(*d);
+}
+
+hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
+                          const void* zeros_host, float global_scale, void* out_host, size_t out_bytes) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (!codes_host || !scales_host || !out_host) return HQ_ERR_INVALID_ARG;
+  if (d->fmt == HQ_FMT_INT4) {
+    if ((d->has_zero_point != 0) != (zeros_host != nullptr)) return HQ_ERR_INVALID_ARG;
+  } else if (zeros_host) {
+    return HQ_ERR_INVALID_ARG;
+  }
+  if (out_bytes < packed_size_impl(*d)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return pack_impl(*d, codes_host, scales_host, zeros_host, global_scale, out_host);
+}
+
+size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t) {
+  if (check_desc(d) != HQ_OK || m < 0) return 0;
+  if (d->fmt != HQ_FMT_INT4) return sizeof(WsHeader);
+  DeviceInfo dev{};
+  if (device_info(&dev) != HQ_OK) {
+    // no sm_100 device current: size for a 148-SM part so the answer is
+    // still an upper bound the caller can allocate
+    dev.num_sms = 148;
+  }
+  const bool grouped = d->num_experts > 1;
+  W4Config cfg = w4_plan(dev, *d, m < 1 ? 1 : m, grouped, t);
+  return w4_workspace_bytes(*d, m < 1 ? 1 : m, cfg, grouped);
+}
+
+hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const void* a_dev, int32_t m,
+                        void* c_dev, const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (d->fmt != HQ_FMT_INT4 || d->num_experts != 1) return HQ_ERR_INVALID_ARG;
+  if (m < 0) return HQ_ERR_INVALID_ARG;
+  if (m == 0) return HQ_OK;
+  if (!packed_w_dev || !a_dev || !c_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(packed_w_dev, 16) || !aligned(a_dev, 16) || !aligned(c_dev, 16) || !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  if (t) {
+    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
+      return HQ_ERR_UNSUPPORTED;
+    if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 ||
+        (t->cta_group && t->cta_group != 1) || t->variant != 0)
+      return HQ_ERR_UNSUPPORTED;
+  }
+  DeviceInfo dev{};
+  st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  W4Config cfg = w4_plan(dev, *d, m, false, t);
+  if (cfg.stages != w4_stages_for(cfg.ntok)) return HQ_ERR_UNSUPPORTED;
+  if (ws_bytes < w4_workspace_bytes(*d, m, cfg, false)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return w4_launch(*d, cfg, packed_w_dev, a_dev, m, c_dev, nullptr, ws_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, const void* a_sorted_dev,
+                              const int32_t* expert_offsets_dev, int32_t total_rows, void* c_sorted_dev,
+                              const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (d->fmt != HQ_FMT_INT4 || d->num_experts < 2) return HQ_ERR_INVALID_ARG;
+  if (total_rows < 0) return HQ_ERR_INVALID_ARG;
+  if (total_rows == 0) return HQ_OK;
+  if (!packed_w_dev || !a_sorted_dev || !expert_offsets_dev || !c_sorted_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(packed_w_dev, 16) || !aligned(a_sorted_dev, 16) || !aligned(c_sorted_dev, 16) ||
+      !aligned(expert_offsets_dev, 4) || !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  if (t) {
+    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
+      return HQ_ERR_UNSUPPORTED;
+    if (t->split_k > 1 || (t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) ||
+        (t->cta_group && t->cta_group != 1) || t->variant != 0)
+      return HQ_ERR_UNSUPPORTED;
+  }
+  DeviceInfo dev{};
+  st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  W4Config cfg = w4_plan(dev, *d, total_rows, true, t);
+  if (cfg.stages != w4_stages_for(cfg.ntok)) return HQ_ERR_UNSUPPORTED;
+  if (ws_bytes < w4_workspace_bytes(*d, total_rows, cfg, true)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return w4_launch(*d, cfg, packed_w_dev, a_sorted_dev, total_rows, c_sorted_dev, expert_offsets_dev, ws_dev,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, const void* a_e4m3_dev,
+                           const float* a_scale_dev, int32_t m, void* c_dev, const hq_tuning* t, void* ws_dev,
+                           size_t ws_bytes, hq_stream_t stream) {
+  (void)packed_w_dev; (void)a_e4m3_dev; (void)a_scale_dev; (void)c_dev; (void)t; (void)ws_dev; (void)ws_bytes;
+  (void)stream;
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (d->fmt != HQ_FMT_MXFP4 || m < 0) return HQ_ERR_INVALID_ARG;
+  return HQ_ERR_UNSUPPORTED;
+}
+
+hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const void* a_fp4_dev,
+                        const void* a_sf_dev, float a_global, int32_t m, void* c_dev, const hq_tuning* t,
+                        void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
+  (void)packed_w_dev; (void)a_fp4_dev; (void)a_sf_dev; (void)a_global; (void)c_dev; (void)t; (void)ws_dev;
+  (void)ws_bytes; (void)stream;
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (d->fmt != HQ_FMT_NVFP4 || m < 0) return HQ_ERR_INVALID_ARG;
+  return HQ_ERR_UNSUPPORTED;
+}
+
+hq_status hq_moe_topk(const float* logits_dev, int32_t t, int32_t e, int32_t k, int32_t* topk_ids_dev,
+                      hq_stream_t stream) {
+  if (t < 0 || k < 1 || k > 16 || e < k || e > 1024) return HQ_ERR_INVALID_ARG;
+  if (t == 0) return HQ_OK;
+  if (!logits_dev || !topk_ids_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(logits_dev, 4) || !aligned(topk_ids_dev, 4)) return HQ_ERR_ALIGNMENT;
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  return moe_topk_launch(logits_dev, t, e, k, topk_ids_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_moe_permute_workspace_size(int32_t t, int32_t k, int32_t e) {
+  if (t < 0 || k < 1 || e < 1) return 0;
+  return moe_permute_ws_bytes(t, k, e);
+}
+
+hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int32_t e, int32_t* sorted_src_dev,
+                         int32_t* expert_offsets_dev, const void* a_dev, int32_t hidden, void* a_sorted_dev,
+                         void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
+  if (t < 0 || k < 1 || k > 16 || e < 1 || e > 1024) return HQ_ERR_INVALID_ARG;
+  if (!expert_offsets_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (t > 0 && (!topk_ids_dev || !sorted_src_dev)) return HQ_ERR_INVALID_ARG;
+  if ((a_dev == nullptr) != (a_sorted_dev == nullptr)) return HQ_ERR_INVALID_ARG;
+  if (a_dev && (hidden < 1 || hidden % 8 != 0)) return HQ_ERR_INVALID_ARG;
+  if (!aligned(ws_dev, 256) || (a_dev && (!aligned(a_dev, 16) || !aligned(a_sorted_dev, 16))))
+    return HQ_ERR_ALIGNMENT;
+  if (ws_bytes < moe_permute_ws_bytes(t, k, e)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  return moe_permute_launch(topk_ids_dev, t, k, e, sorted_src_dev, expert_offsets_dev, a_dev, hidden, a_sorted_dev,
+                            ws_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_check_device_status(void* ws_dev, hq_stream_t stream) {
+  if (!ws_dev) return HQ_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return HQ_ERR_CUDA;
+  uint32_t err = 0;
+  if (cudaMemcpy(&err, ws_dev, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess) return HQ_ERR_CUDA;
+  if (err != 0) {
+    uint32_t zero = 0;
+    if (cudaMemcpy(ws_dev, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HQ_ERR_CUDA;
+  }
+  return static_cast<hq_status>(err);
+}
+
+hq_status hq_debug_timeout_probe(void* ws_dev, uint64_t limit_ns, hq_stream_t stream) {
+  if (!ws_dev || limit_ns > 100000000ull) return HQ_ERR_INVALID_ARG;
+  if (!aligned(ws_dev, 256)) return HQ_ERR_ALIGNMENT;
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  return debug_timeout_launch(ws_dev, limit_ns, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,63 @@
+// Internal declarations shared by the C-ABI layer and the kernel launchers.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/hq.h"
+
+namespace hq {
+
+// Workspace header: the first 256 bytes of every workspace.
+struct WsHeader {
+  uint32_t err;        // first device-side error (hq_status), 0 = none
+  uint32_t reserved[63];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+constexpr int kTileN = 128;      // weight rows per tile (MMA M)
+constexpr int kBlockK = 128;     // K per packed record / pipeline stage
+constexpr int kW4RecCodes = 8192;
+inline int w4_record_bytes(bool has_zero) { return kW4RecCodes + 256 + (has_zero ? 128 : 0); }
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
+
+// Resolved launch configuration of the W4A16 kernel family.
+struct W4Config {
+  int ntok;     // token tile (MMA N)
+  int stages;
+  int splits;   // split-K factor (dense only)
+  int grid;     // CTAs
+};
+
+struct DeviceInfo {
+  int device;
+  int num_sms;
+  int cc_major, cc_minor;
+  size_t max_smem_optin;
+};
+hq_status device_info(DeviceInfo* out);
+
+// W4A16 (dense or grouped) planning and launch.
+W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t);
+size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bool grouped);
+int w4_stages_for(int ntok);
+hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m,
+                    void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream);
+
+// MoE helpers.
+size_t moe_permute_ws_bytes(int t, int k, int e);
+hq_status moe_topk_launch(const float* logits, int t, int e, int k, int32_t* ids, cudaStream_t s);
+hq_status moe_permute_launch(const int32_t* ids, int t, int k, int e, int32_t* sorted_src, int32_t* offsets,
+                             const void* a, int hidden, void* a_sorted, void* ws, cudaStream_t s);
+
+hq_status debug_timeout_launch(void* ws, uint64_t limit_ns, cudaStream_t s);
+
+// Driver entry point for tensor-map encoding (resolved once).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+}  // namespace hq

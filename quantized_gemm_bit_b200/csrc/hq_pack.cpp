@@ -1,0 +1,182 @@
+// Offline weight packer: canonical (code, scale, zero point) tensors -> the
+// device layout the kernels read.  Host memory in, host memory out.
+//
+// The method keeps weight, scale and zero point as separately described
+// parts of one standard quantization description ("Humming: open-source
+// kernel library for quantized inference", summary paragraph 2); this file
+// fixes how those parts sit in device memory for the B200 kernels.
+//
+// Packed layouts, version 1 (NP = N rounded up to a multiple of 128; rows
+// >= N are zero-filled):
+//
+// INT4 (group 128).  One record per (tile nt of 128 rows, block kb of 128 K),
+// records in (nt, kb) order, expert after expert.  Record bytes:
+//   [0, 8192)      codes: for row r, K-chunk c = kk/32, word w = (kk%32)/8,
+//                  element e = kk%8: byte (c*128 + r)*16 + 4*w holds the
+//                  32-bit word whose nibble p = (e%2)*4 + e/2 is the code.
+//                  (A thread owning row r reads 16 contiguous bytes per
+//                  chunk; nibbles k, k+1 share one 16-bit lane pair.)
+//   [8192, 8448)   fp16 scale of row r at 8192 + 2r
+//   [8448, 8576)   uint4 zero point of row r at 8448 + r (asymmetric only)
+//
+// MXFP4 (E8M0 scale per 32 K).
+//   codes : [NP][K/2] bytes, row major, even k in the low nibble
+//   scales: from byte NP*K/2, one 512-byte block per (tile nt, 128-K group
+//           g) in (nt, g) order; byte l*16 + 4*c + j holds the scale of row
+//           nt*128 + l + 32*c for the 32-K block 4*g + j (l < 32, c < 4,
+//           j < 4).  This is the order tcgen05.cp 32x128b.warpx4 expects.
+//
+// NVFP4 (E4M3 scale per 16 K, fp32 tensor scale).
+//   codes : [NP][K/2] bytes as for MXFP4
+//   scales: from byte NP*K/2, one 512-byte block per (tile nt, 64-K group g)
+//           in (nt, g) order; byte l*16 + 4*c + j = scale of row
+//           nt*128 + l + 32*c for the 16-K block 4*g + j
+//   tail  : 16 bytes; the fp32 tensor scale in the first 4.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "hq_internal.h"
+
+namespace hq {
+
+namespace {
+
+
+template <class F>
+void parallel_for(size_t n, F&& f) {
+  unsigned hw = std::max(1u, std::min(32u, std::thread::hardware_concurrency()));
+  size_t nt = std::min<size_t>(hw, n);
+  if (nt <= 1) {
+    for (size_t i = 0; i < n; ++i) f(i);
+    return;
+  }
+  std::vector<std::thread> th;
+  th.reserve(nt);
+  for (size_t t = 0; t < nt; ++t) {
+    th.emplace_back([&, t]() {
+      for (size_t i = t; i < n; i += nt) f(i);
+    });
+  }
+  for (auto& x : th) x.join();
+}
+
+// Nibble permutation inside one 32-bit word: canonical element e (bits 4e)
+// moves to nibble (e%2)*4 + e/2.
+inline uint32_t permute_word(uint32_t w) {
+  uint32_t out = 0;
+  for (int e = 0; e < 8; ++e) {
+    uint32_t code = (w >> (4 * e)) & 0xF;
+    int p = (e & 1) * 4 + (e >> 1);
+    out |= code << (4 * p);
+  }
+  return out;
+}
+
+hq_status pack_int4(const hq_quant_desc& d, const int32_t* codes, const uint16_t* scales, const uint8_t* zeros,
+                    uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int nt_count = (n + kTileN - 1) / kTileN;
+  const int kb_count = k / kBlockK;
+  const bool hz = zeros != nullptr;
+  const size_t rec = (size_t)w4_record_bytes(hz);
+  const size_t expert_bytes = (size_t)nt_count * kb_count * rec;
+  const size_t kw = (size_t)k / 8;   // canonical words per row
+  const size_t kg = (size_t)k / 128; // groups per row
+  // reject zero points outside 0..15 before writing anything
+  if (hz) {
+    const size_t total = (size_t)d.num_experts * n * kg;
+    for (size_t i = 0; i < total; ++i)
+      if (zeros[i] > 15) return HQ_ERR_INVALID_ARG;
+  }
+  const size_t jobs = (size_t)d.num_experts * nt_count;
+  parallel_for(jobs, [&](size_t job) {
+    const size_t e = job / nt_count;
+    const int nt = (int)(job % nt_count);
+    uint8_t* ebase = out + e * expert_bytes;
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint8_t* r0 = ebase + ((size_t)nt * kb_count + kb) * rec;
+      std::memset(r0, 0, rec);
+      for (int r = 0; r < kTileN; ++r) {
+        const int row = nt * kTileN + r;
+        if (row >= n) break;
+        const int32_t* src = codes + (e * n + row) * kw + (size_t)kb * 16;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(r0 + ((size_t)c * 128 + r) * 16);
+          for (int w = 0; w < 4; ++w) dst[w] = permute_word((uint32_t)src[c * 4 + w]);
+        }
+        const uint16_t s = scales[(e * n + row) * kg + kb];
+        std::memcpy(r0 + kW4RecCodes + 2 * r, &s, 2);
+        if (hz) r0[kW4RecCodes + 256 + r] = zeros[(e * n + row) * kg + kb];
+      }
+    }
+  });
+  return HQ_OK;
+}
+
+// Block-scaled formats: copy codes row by row, then lay out scale blocks.
+hq_status pack_fp4(const hq_quant_desc& d, const uint8_t* codes, const uint8_t* scales, float g, uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int np = (n + kTileN - 1) / kTileN * kTileN;
+  const size_t row_bytes = (size_t)k / 2;
+  const int blk = d.group_size;                   // 32 (MX) or 16 (NV)
+  const int blocks = k / blk;                     // scale entries per row
+  const int groups = blocks / 4;                  // 512-byte chunks per tile
+  const size_t codes_bytes = (size_t)np * row_bytes;
+  std::memset(out, 0, codes_bytes);
+  for (int r = 0; r < n; ++r) std::memcpy(out + (size_t)r * row_bytes, codes + (size_t)r * row_bytes, row_bytes);
+  uint8_t* sf = out + codes_bytes;
+  const int nt_count = np / kTileN;
+  parallel_for((size_t)nt_count, [&](size_t nt) {
+    for (int g4 = 0; g4 < groups; ++g4) {
+      uint8_t* chunk = sf + ((size_t)nt * groups + g4) * 512;
+      for (int l = 0; l < 32; ++l)
+        for (int c = 0; c < 4; ++c)
+          for (int j = 0; j < 4; ++j) {
+            const int row = (int)nt * kTileN + l + 32 * c;
+            chunk[l * 16 + c * 4 + j] = row < n ? scales[(size_t)row * blocks + 4 * g4 + j] : 0;
+          }
+    }
+  });
+  if (d.fmt == HQ_FMT_NVFP4) {
+    uint8_t* tail = sf + (size_t)nt_count * groups * 512;
+    std::memset(tail, 0, 16);
+    std::memcpy(tail, &g, 4);
+  }
+  return HQ_OK;
+}
+
+}  // namespace
+
+size_t packed_size_impl(const hq_quant_desc& d) {
+  const size_t nt = (size_t)(d.n + kTileN - 1) / kTileN;
+  switch (d.fmt) {
+    case HQ_FMT_INT4:
+      return (size_t)d.num_experts * nt * (d.k / kBlockK) * w4_record_bytes(d.has_zero_point != 0);
+    case HQ_FMT_MXFP4:
+      return nt * kTileN * (size_t)d.k / 2 + nt * (d.k / 128) * 512;
+    case HQ_FMT_NVFP4:
+      return nt * kTileN * (size_t)d.k / 2 + nt * (d.k / 64) * 512 + 16;
+    default:
+      return 0;
+  }
+}
+
+hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scales, const void* zeros, float g,
+                    void* out) {
+  switch (d.fmt) {
+    case HQ_FMT_INT4:
+      return pack_int4(d, static_cast<const int32_t*>(codes), static_cast<const uint16_t*>(scales),
+                       static_cast<const uint8_t*>(zeros), static_cast<uint8_t*>(out));
+    case HQ_FMT_MXFP4:
+    case HQ_FMT_NVFP4:
+      return pack_fp4(d, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), g,
+                      static_cast<uint8_t*>(out));
+    default:
+      return HQ_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace hq

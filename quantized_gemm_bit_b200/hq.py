@@ -1,0 +1,223 @@
+"""Thin ctypes binding of the C ABI in include/hq.h (libhq.so).
+
+Argument marshalling only: every function here forwards raw pointers, sizes
+and the caller's CUDA stream to the C entry point of the same name and turns
+a non-OK status into an HQError.  No arithmetic of the method runs in
+Python; if libhq.so is missing the first call raises instead of falling back
+to anything else.
+
+Device arrays are torch CUDA tensors (PyTorch supplies memory and streams);
+host arrays for the packer are numpy arrays or CPU tensors.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhq.so")
+
+HQ_LAYOUT_VERSION = 1
+
+HQ_OK = 0
+HQ_ERR_INVALID_ARG = 1
+HQ_ERR_UNSUPPORTED = 2
+HQ_ERR_ALIGNMENT = 3
+HQ_ERR_WORKSPACE_TOO_SMALL = 4
+HQ_ERR_LAYOUT_VERSION = 5
+HQ_ERR_CUDA = 6
+HQ_ERR_DEVICE_TIMEOUT = 7
+HQ_ERR_DEVICE_BAD_OFFSETS = 8
+HQ_ERR_NO_DEVICE = 9
+
+HQ_FMT_INT4 = 1
+HQ_FMT_MXFP4 = 2
+HQ_FMT_NVFP4 = 3
+
+# Every symbol include/hq.h declares.
+EXPORTS = (
+    "hq_layout_version", "hq_status_string", "hq_quant_desc_init", "hq_packed_size", "hq_pack_weights",
+    "hq_workspace_size", "hq_gemm_w4a16", "hq_gemm_mxfp4_a8", "hq_gemm_nvfp4", "hq_moe_topk",
+    "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_check_device_status",
+    "hq_debug_timeout_probe",
+)
+
+
+class QuantDesc(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in
+                ("layout_version", "fmt", "n", "k", "group_size", "has_zero_point", "num_experts")]
+
+
+class Tuning(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in
+                ("tile_m", "tile_n", "tile_k", "stages", "split_k", "cta_group", "variant")]
+
+
+class HQError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib():
+    """Load libhq.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m quantized_gemm_bit_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int
+        dp = ctypes.POINTER(QuantDesc)
+        tp = ctypes.POINTER(Tuning)
+        sig = {
+            "hq_layout_version": (ctypes.c_int, []),
+            "hq_status_string": (ctypes.c_char_p, [st]),
+            "hq_quant_desc_init": (st, [dp, i32, i32, i32, i32, i32, i32]),
+            "hq_packed_size": (sz, [dp]),
+            "hq_pack_weights": (st, [dp, vp, vp, vp, ctypes.c_float, vp, sz]),
+            "hq_workspace_size": (sz, [dp, i32, tp]),
+            "hq_gemm_w4a16": (st, [dp, vp, vp, i32, vp, tp, vp, sz, vp]),
+            "hq_gemm_mxfp4_a8": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
+            "hq_gemm_nvfp4": (st, [dp, vp, vp, vp, ctypes.c_float, i32, vp, tp, vp, sz, vp]),
+            "hq_moe_topk": (st, [vp, i32, i32, i32, vp, vp]),
+            "hq_moe_permute_workspace_size": (sz, [i32, i32, i32]),
+            "hq_moe_permute": (st, [vp, i32, i32, i32, vp, vp, vp, i32, vp, vp, sz, vp]),
+            "hq_grouped_gemm_moe": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
+            "hq_check_device_status": (st, [vp, vp]),
+            "hq_debug_timeout_probe": (st, [vp, ctypes.c_uint64, vp]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    try:
+        return lib().hq_status_string(int(status)).decode()
+    except RuntimeError:
+        return f"status {status}"
+
+
+def _check(status, where):
+    if status != HQ_OK:
+        raise HQError(status, where)
+
+
+def _ptr(t):
+    """Raw address of a torch tensor / numpy array (None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _tuning(t):
+    if t is None:
+        return None
+    if isinstance(t, Tuning):
+        return ctypes.byref(t)
+    return ctypes.byref(Tuning(**t))
+
+
+def _host(x):
+    if x is None:
+        return None
+    if not isinstance(x, np.ndarray):
+        x = x.contiguous().numpy()
+    return np.ascontiguousarray(x)
+
+
+# ---------------------------------------------------------------- C ABI mirror
+
+def hq_layout_version():
+    return lib().hq_layout_version()
+
+
+def hq_quant_desc_init(fmt, n, k, group_size, has_zero_point=0, num_experts=1):
+    d = QuantDesc()
+    _check(lib().hq_quant_desc_init(ctypes.byref(d), fmt, n, k, group_size, int(has_zero_point), num_experts),
+           "hq_quant_desc_init")
+    return d
+
+
+def hq_packed_size(desc):
+    return lib().hq_packed_size(ctypes.byref(desc))
+
+
+def hq_pack_weights(desc, codes, scales, zeros=None, global_scale=0.0):
+    """Host packer: returns the packed blob as a numpy uint8 array."""
+    codes, scales, zeros = _host(codes), _host(scales), _host(zeros)
+    if scales.dtype == np.float16:
+        scales = scales.view(np.uint16)
+    out = np.empty(hq_packed_size(desc), dtype=np.uint8)
+    _check(lib().hq_pack_weights(ctypes.byref(desc), _ptr(codes), _ptr(scales), _ptr(zeros),
+                                 float(global_scale), _ptr(out), out.nbytes), "hq_pack_weights")
+    return out
+
+
+def hq_workspace_size(desc, m, tuning=None):
+    return lib().hq_workspace_size(ctypes.byref(desc), int(m), _tuning(tuning))
+
+
+def hq_gemm_w4a16(desc, packed_w, a, m, c, ws, tuning=None, stream=None):
+    _check(lib().hq_gemm_w4a16(ctypes.byref(desc), _ptr(packed_w), _ptr(a), int(m), _ptr(c), _tuning(tuning),
+                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "hq_gemm_w4a16")
+
+
+def hq_gemm_mxfp4_a8(desc, packed_w, a_e4m3, a_scale, m, c, ws, tuning=None, stream=None):
+    _check(lib().hq_gemm_mxfp4_a8(ctypes.byref(desc), _ptr(packed_w), _ptr(a_e4m3), _ptr(a_scale), int(m), _ptr(c),
+                                  _tuning(tuning), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hq_gemm_mxfp4_a8")
+
+
+def hq_gemm_nvfp4(desc, packed_w, a_fp4, a_sf, a_global, m, c, ws, tuning=None, stream=None):
+    _check(lib().hq_gemm_nvfp4(ctypes.byref(desc), _ptr(packed_w), _ptr(a_fp4), _ptr(a_sf), float(a_global), int(m),
+                               _ptr(c), _tuning(tuning), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream(stream)), "hq_gemm_nvfp4")
+
+
+def hq_moe_topk(logits, t, e, k, topk_ids, stream=None):
+    _check(lib().hq_moe_topk(_ptr(logits), int(t), int(e), int(k), _ptr(topk_ids), _stream(stream)), "hq_moe_topk")
+
+
+def hq_moe_permute_workspace_size(t, k, e):
+    return lib().hq_moe_permute_workspace_size(int(t), int(k), int(e))
+
+
+def hq_moe_permute(topk_ids, t, k, e, sorted_src, expert_offsets, ws, a=None, hidden=0, a_sorted=None,
+                   stream=None):
+    _check(lib().hq_moe_permute(_ptr(topk_ids), int(t), int(k), int(e), _ptr(sorted_src), _ptr(expert_offsets),
+                                _ptr(a), int(hidden), _ptr(a_sorted), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(stream)), "hq_moe_permute")
+
+
+def hq_grouped_gemm_moe(desc, packed_w, a_sorted, expert_offsets, total_rows, c_sorted, ws, tuning=None,
+                        stream=None):
+    _check(lib().hq_grouped_gemm_moe(ctypes.byref(desc), _ptr(packed_w), _ptr(a_sorted), _ptr(expert_offsets),
+                                     int(total_rows), _ptr(c_sorted), _tuning(tuning), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "hq_grouped_gemm_moe")
+
+
+def hq_check_device_status(ws, stream=None):
+    """Returns the device-side status recorded in the workspace (and clears it)."""
+    return lib().hq_check_device_status(_ptr(ws), _stream(stream))
+
+
+def hq_debug_timeout_probe(ws, limit_ns, stream=None):
+    _check(lib().hq_debug_timeout_probe(_ptr(ws), int(limit_ns), _stream(stream)), "hq_debug_timeout_probe")

@@ -1,0 +1,46 @@
+"""Shared helpers for the GPU parity tests: tolerance checks written out
+from the stated bars, workspace allocation and tile-covering row samples."""
+
+import numpy as np
+import torch
+
+from quantized_gemm_bit_b200 import hq
+
+# GEMM tolerance: relative Frobenius error <= 5e-3 and, per element,
+# |err| <= 1e-2*|ref| + 2e-3*sqrt(K)*rms(ref).
+REL_FRO = 5e-3
+ELEM_REL = 1e-2
+ELEM_ABS = 2e-3
+
+
+def check_gemm(c_bf16, ref, k, what=""):
+    c = c_bf16.float().double().cpu().numpy() if isinstance(c_bf16, torch.Tensor) else np.asarray(c_bf16)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert c.shape == ref.shape, (c.shape, ref.shape)
+    assert np.all(np.isfinite(c)), what
+    err = c - ref
+    nref = np.linalg.norm(ref)
+    rel = np.linalg.norm(err) / nref if nref > 0 else np.linalg.norm(err)
+    rms = np.sqrt(np.mean(ref ** 2))
+    bound = ELEM_REL * np.abs(ref) + ELEM_ABS * np.sqrt(k) * rms
+    worst = np.max(np.abs(err) - bound)
+    assert rel <= REL_FRO, f"{what}: rel Frobenius {rel:.3e}"
+    assert worst <= 0, f"{what}: element bound exceeded by {worst:.3e}"
+    return rel
+
+
+def workspace(nbytes, device="cuda"):
+    # torch's caching allocator returns 512-byte aligned blocks
+    ws = torch.zeros(max(256, nbytes), dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def tile_rows(m, tile, rng, per_tile=2):
+    """First and last row of every `tile`-row tile plus a few random rows."""
+    rows = set()
+    for t0 in range(0, m, tile):
+        t1 = min(m, t0 + tile) - 1
+        rows.update({t0, t1})
+        rows.update(rng.integers(t0, t1 + 1, size=per_tile).tolist())
+    return np.array(sorted(rows))

@@ -1,0 +1,142 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and
+exports every declared symbol, descriptors validate, the packer matches the
+oracle's layout formulas bit for bit, and invalid calls fail before any
+launch."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats as F
+from oracle import layout as L
+from quantized_gemm_bit_b200 import hq, synth
+from quantized_gemm_bit_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build()
+
+
+def test_exports_every_declared_symbol():
+    header = open(os.path.join(ROOT, "include", "hq.h")).read()
+    declared = set(re.findall(r"\b(hq_[a-z0-9_]+)\s*\(", header))
+    assert declared == set(hq.EXPORTS)
+    raw = ctypes.CDLL(hq.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert hq.hq_layout_version() == hq.HQ_LAYOUT_VERSION == 1
+
+
+def test_desc_validation():
+    hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 1024, 1024, 128, 1, 1)
+    for args, code in [((hq.HQ_FMT_INT4, 1024, 1000, 128, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT4, 1024, 1024, 64, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT4, 0, 1024, 128, 0, 1), hq.HQ_ERR_INVALID_ARG),
+                       ((hq.HQ_FMT_MXFP4, 128, 128, 32, 1, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_NVFP4, 128, 128, 16, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((7, 128, 128, 16, 0, 1), hq.HQ_ERR_INVALID_ARG)]:
+        with pytest.raises(hq.HQError) as e:
+            hq.hq_quant_desc_init(*args)
+        assert e.value.status == code
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 128, 128, 128, 0, 1)
+    d.layout_version = 0
+    assert hq.hq_packed_size(d) == 0
+
+
+@pytest.mark.parametrize("n,k,asym,experts", [(256, 384, False, 1), (200, 256, True, 1), (128, 256, False, 3)])
+def test_int4_pack_matches_oracle_layout(n, k, asym, experts):
+    q, s, z = synth.w4a16_weights(n, k, 128, asym, seed=7, experts=experts if experts > 1 else None)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, int(asym), experts)
+    blob = hq.hq_pack_weights(d, q, s, z)
+    assert blob.size == L.w4a16_packed_bytes(n, k, asym, experts)
+    qn, sn = q.numpy(), s.numpy()
+    zn = None if z is None else z.numpy()
+    if experts == 1:
+        ref = L.w4a16_pack(qn, sn, zn)
+    else:
+        ref = np.concatenate([L.w4a16_pack(qn[e], sn[e], None if zn is None else zn[e]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+@pytest.mark.parametrize("fmt,block", [(hq.HQ_FMT_MXFP4, 32), (hq.HQ_FMT_NVFP4, 16)])
+@pytest.mark.parametrize("n", [128, 300])
+def test_fp4_pack_matches_oracle_layout(fmt, block, n):
+    k = 512
+    rng = np.random.default_rng(n)
+    codes = rng.integers(0, 256, size=(n, k // 2), dtype=np.uint8)
+    scales = rng.integers(0, 255, size=(n, k // block), dtype=np.uint8)
+    d = hq.hq_quant_desc_init(fmt, n, k, block, 0, 1)
+    g = 0.125 if fmt == hq.HQ_FMT_NVFP4 else 0.0
+    blob = hq.hq_pack_weights(d, codes, scales, None, g)
+    ref = L.fp4_pack(codes, scales, block, g if fmt == hq.HQ_FMT_NVFP4 else None)
+    assert np.array_equal(blob, ref)
+
+
+def test_fp4_scale_layout_is_a_bijection():
+    n, k, block = 256, 512, 16
+    nn, bb = np.meshgrid(np.arange(n), np.arange(k // block), indexing="ij")
+    off = L.fp4_scale_byte_np(nn.ravel(), bb.ravel(), k, block, 256)
+    assert len(np.unique(off)) == off.size
+    assert off.min() == 256 * k // 2 and off.max() == 256 * k // 2 + off.size - 1
+
+
+def test_pack_rejects_bad_arguments():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 128, 128, 128, 1, 1)
+    q, s, z = synth.w4a16_weights(128, 128, 128, True, seed=1)
+    with pytest.raises(hq.HQError) as e:          # zeros missing for an asymmetric descriptor
+        hq.hq_pack_weights(d, q, s, None)
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
+    zb = z.clone()
+    zb[0, 0] = 16
+    with pytest.raises(hq.HQError) as e:          # zero point out of range
+        hq.hq_pack_weights(d, q, s, zb)
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
+    out = np.empty(10, dtype=np.uint8)
+    st = hq.lib().hq_pack_weights(ctypes.byref(d), q.numpy().ctypes.data, s.numpy().ctypes.data,
+                                  z.numpy().ctypes.data, 0.0, out.ctypes.data, out.nbytes)
+    assert st == hq.HQ_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_gemm_argument_errors_need_no_gpu():
+    L_ = hq.lib()
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 256, 256, 128, 0, 1)
+    # m == 0: nothing to do
+    assert L_.hq_gemm_w4a16(ctypes.byref(d), None, None, 0, None, None, None, 0, None) == hq.HQ_OK
+    # NULL pointers
+    assert L_.hq_gemm_w4a16(ctypes.byref(d), None, None, 4, None, None, None, 0, None) == hq.HQ_ERR_INVALID_ARG
+    # misaligned pointers
+    assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 18, 4, 32, None, 256, 1 << 20, None) == hq.HQ_ERR_ALIGNMENT
+    # wrong format for the entry point
+    d2 = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 256, 256, 32, 0, 1)
+    assert L_.hq_gemm_w4a16(ctypes.byref(d2), 16, 16, 4, 32, None, 256, 1 << 20, None) == hq.HQ_ERR_INVALID_ARG
+    # stale descriptor
+    d.layout_version = 99
+    assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, None, 256, 1 << 20, None) == hq.HQ_ERR_LAYOUT_VERSION
+    # unsupported tuning
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 256, 256, 128, 0, 1)
+    t = hq.Tuning(tile_m=48)
+    assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
+                            None) == hq.HQ_ERR_UNSUPPORTED
+    # routing arguments
+    assert L_.hq_moe_topk(None, 4, 8, 0, None, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_topk(None, 4, 4, 8, None, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_debug_timeout_probe(256, 10 ** 9, None) == hq.HQ_ERR_INVALID_ARG
+
+
+def test_workspace_size_is_deterministic_and_covers_header():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 7168, 18432, 128, 0, 1)
+    a = hq.hq_workspace_size(d, 16)
+    assert a == hq.hq_workspace_size(d, 16) and a >= 256
+    assert hq.hq_workspace_size(d, 4096) >= 256
+
+
+def test_status_strings():
+    for s in range(10):
+        assert hq.status_string(s)

@@ -1,0 +1,133 @@
+"""GPU parity of the dense W4A16 GEMM (through the C ABI) against the fp64
+oracle: full outputs on small shapes that span several tiles and ragged
+tails, sampled rows at the full M-sweep sizes in the bench's launch
+configuration, determinism, guard bands and workspace hygiene."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import check_gemm, tile_rows, workspace
+from oracle import formats as F
+from oracle import gemm as G
+from quantized_gemm_bit_b200 import hq, synth
+from quantized_gemm_bit_b200.build import build
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    build()
+    torch.cuda.init()
+
+
+def _bits(a):
+    return a.view(torch.int16).numpy().view(np.uint16)
+
+
+def make_case(m, n, k, asym, seed):
+    q, s, z = synth.w4a16_weights(n, k, 128, asym, seed)
+    a = synth.bf16_normal(m, k, seed + 1)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, int(asym), 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(DEV)
+    return d, blob, a, (q.numpy(), s.numpy(), None if z is None else z.numpy())
+
+
+def run(d, blob, a, m, tuning=None, c=None):
+    a_d = a.to(DEV)
+    if c is None:
+        c = torch.empty(m, d.n, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, m, tuning))
+    hq.hq_gemm_w4a16(d, blob, a_d, m, c, ws, tuning)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    return c, ws
+
+
+def test_tiny_config_full_output():
+    """W4A16 tiny: M=16, K=N=1024, asymmetric, seed 0."""
+    m, n, k = 16, 1024, 1024
+    d, blob, a, (q, s, z) = make_case(m, n, k, True, 0)
+    c, _ = run(d, blob, a, m)
+    ref = G.w4a16_ref(_bits(a), q, s, z, 128)
+    check_gemm(c, ref, k, "tiny")
+
+
+@pytest.mark.parametrize("m,n,k,asym", [
+    (1, 256, 256, False), (7, 200, 384, True), (17, 384, 1152, False), (100, 128, 512, True),
+    (129, 640, 640, False), (300, 256, 768, True), (513, 384, 256, False),
+])
+def test_ragged_shapes_full_output(m, n, k, asym):
+    d, blob, a, (q, s, z) = make_case(m, n, k, asym, 100 + m)
+    c, _ = run(d, blob, a, m)
+    ref = G.w4a16_ref(_bits(a), q, s, z, 128)
+    check_gemm(c, ref, k, f"m={m} n={n} k={k}")
+
+
+@pytest.mark.parametrize("tile_m", [16, 32, 64, 128, 256])
+def test_every_token_tile(tile_m):
+    m, n, k = 70, 384, 1024
+    d, blob, a, (q, s, z) = make_case(m, n, k, True, 7)
+    c, _ = run(d, blob, a, m, hq.Tuning(tile_m=tile_m))
+    check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"tile_m={tile_m}")
+
+
+@pytest.mark.parametrize("splits", [2, 3, 7])
+def test_split_k_and_determinism(splits):
+    m, n, k = 20, 256, 1792
+    d, blob, a, (q, s, z) = make_case(m, n, k, False, 9)
+    t = hq.Tuning(tile_m=32, split_k=splits)
+    c1, ws = run(d, blob, a, m, t)
+    c2, _ = run(d, blob, a, m, t)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"splits={splits}")
+    # the workspace is left zero-filled (counters reset by the last split)
+    counters = ws[256:256 + 4 * 4 * 2].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
+
+
+def test_guard_bands_untouched():
+    m, n, k = 33, 200, 512
+    d, blob, a, (q, s, z) = make_case(m, n, k, True, 11)
+    # sentinels before and after C in one flat buffer
+    flat = torch.full((m * n + 64,), 7.0, dtype=torch.bfloat16, device=DEV)
+    c = flat[32:32 + m * n].view(m, n)
+    c, _ = run(d, blob, a, m, c=c)
+    assert torch.all(flat[:32] == 7.0) and torch.all(flat[32 + m * n:] == 7.0)
+    check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, "guard")
+
+
+def test_timeout_probe_reports_instead_of_hanging():
+    ws = workspace(256)
+    hq.hq_debug_timeout_probe(ws, 2_000_000)      # 2 ms limit, nobody arrives
+    assert hq.hq_check_device_status(ws) == hq.HQ_ERR_DEVICE_TIMEOUT
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK   # cleared
+
+
+_SWEEP = {}
+
+
+def _sweep_case(k, n):
+    if (k, n) not in _SWEEP:
+        seed = 1000 + (0 if k == 7168 else 1)
+        q, s, z = synth.w4a16_weights(n, k, 128, False, seed)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(DEV)
+        w = G.w4a16_dequant(q.numpy(), s.numpy(), None, 128)
+        _SWEEP[(k, n)] = (d, blob, w)
+    return _SWEEP[(k, n)]
+
+
+@pytest.mark.parametrize("k,n", [(7168, 18432), (18432, 7168)])
+@pytest.mark.parametrize("m", [1, 4, 16, 64, 256, 1024, 4096])
+def test_m_sweep_full_size_sampled_rows(m, k, n):
+    """Full-size M-sweep shapes in the default (heuristic) launch
+    configuration; the oracle evaluates tile-covering sampled rows."""
+    d, blob, w = _sweep_case(k, n)
+    a = synth.bf16_normal(m, k, 1000 + m)
+    c, _ = run(d, blob, a, m)
+    rows = tile_rows(m, 128, np.random.default_rng(m))
+    ref = F.bf16_bits_to_f64(_bits(a)[rows]) @ w.T
+    check_gemm(c[torch.from_numpy(rows).to(DEV)], ref, k, f"sweep m={m} k={k} n={n}")
