@@ -1,0 +1,595 @@
+"""Benchmark of the fused-dequant low-bit GEMM path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload w4a16_sweep|moe|mxfp4|nvfp4]
+
+Default workload (one "step"): the dense W4A16 M-sweep, M in {1, 4, 16, 64,
+256, 1024, 4096} for (K, N) = (7168, 18432) and (18432, 7168), symmetric
+INT4, group 128, fp16 scales, bf16 activations: 14 GEMMs through the C ABI.
+`value` is the sweep's aggregate TFLOP/s (total FLOPs / total time).
+
+Other workloads (--workload): the grouped MoE layer GEMMs (tok/s), the
+W4A8-MXFP4 GEMMs and the NVFP4 W4A4 GEMMs, each printed as its own line.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronize, timed with CUDA events on the launching stream; weight
+blobs rotate over several copies whose total exceeds 3x the L2 size, so
+every GEMM streams its weights from HBM.  Under torchrun every rank runs an
+independent replica (the path has no exchange step) and the time is the
+maximum over ranks.
+
+--impl reference times the CPU oracle (the method's plain fp64 definition)
+on a bounded sample of the same workload on the host cores.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16/FP4 GEMM TFLOP/s and HBM GB/s vs roofline (1 B200), M=1..8192; MoE tok/s"
+SWEEP_M = (1, 4, 16, 64, 256, 1024, 4096)
+SWEEP_KN = ((7168, 18432), (18432, 7168))
+GROUP = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def w4a16_bytes(m, k, n):
+    """Algorithmic bytes of one W4A16 GEMM: packed codes (K*N/2) + fp16
+    scales (2*N*K/128) + bf16 A (2*M*K) + bf16 C (2*M*N), each once."""
+    return k * n // 2 + 2 * n * (k // GROUP) + 2 * m * k + 2 * m * n
+
+
+def w4a16_flops(m, k, n):
+    return 2.0 * m * k * n
+
+
+class Clocks:
+    """Samples nvidia-smi every 50 ms while the timed region runs (the
+    sampler starts half a second early; idle samples below half the peak
+    clock are left out of the median)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)   # let the sampler start before the timed region
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons)}
+        loaded = [x for x in sm if x > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- W4A16 sweep
+
+def setup_w4a16_sweep(l2_bytes):
+    from quantized_gemm_bit_b200 import hq, synth
+    dev = "cuda"
+    shapes = []
+    for si, (k, n) in enumerate(SWEEP_KN):
+        q, s, _ = synth.w4a16_weights(n, k, GROUP, False, seed=1000 + si)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, GROUP, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev)
+        copies = max(2, int(np.ceil(3 * l2_bytes / blob.numel())) + 1)
+        blobs = [blob] + [blob.clone() for _ in range(copies - 1)]
+        acts, outs, wss, host_a, host_c = [], [], [], [], []
+        for m in SWEEP_M:
+            a = synth.bf16_normal(m, k, seed=1000 + m).to(dev)
+            acts.append(a)
+            outs.append(torch.empty(m, n, dtype=torch.bfloat16, device=dev))
+            wss.append(torch.zeros(max(256, hq.hq_workspace_size(d, m)), dtype=torch.uint8, device=dev))
+            host_a.append(a.cpu().pin_memory())
+            host_c.append(torch.empty(m, n, dtype=torch.bfloat16).pin_memory())
+        shapes.append(dict(k=k, n=n, d=d, blobs=blobs, acts=acts, outs=outs, wss=wss, host_a=host_a,
+                           host_c=host_c))
+    return shapes
+
+
+def run_w4a16_sweep(args, rank, world, peaks):
+    from quantized_gemm_bit_b200 import hq
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    shapes = setup_w4a16_sweep(l2)
+    stream = torch.cuda.current_stream()
+    gemms = [(si, mi) for si in range(len(shapes)) for mi in range(len(SWEEP_M))]
+    counter = [0]
+
+    def one_step(events=None, e2e=False):
+        for (si, mi) in gemms:
+            sh = shapes[si]
+            blob = sh["blobs"][counter[0] % len(sh["blobs"])]
+            counter[0] += 1
+            m = SWEEP_M[mi]
+            if e2e:
+                sh["acts"][mi].copy_(sh["host_a"][mi], non_blocking=True)
+            if events is not None:
+                events[(si, mi)][0].append(torch.cuda.Event(enable_timing=True))
+                events[(si, mi)][0][-1].record(stream)
+            hq.hq_gemm_w4a16(sh["d"], blob, sh["acts"][mi], m, sh["outs"][mi], sh["wss"][mi], stream=stream)
+            if events is not None:
+                events[(si, mi)][1].append(torch.cuda.Event(enable_timing=True))
+                events[(si, mi)][1][-1].record(stream)
+            if e2e:
+                sh["host_c"][mi].copy_(sh["outs"][mi], non_blocking=True)
+
+    # correctness guard: the device status must be clean after warm-up
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    for sh in shapes:
+        for ws in sh["wss"]:
+            st = hq.hq_check_device_status(ws)
+            if st != hq.HQ_OK:
+                raise RuntimeError(f"device status after warm-up: {hq.status_string(st)}")
+
+    # ---- device-resident timed region
+    events = {g: ([], []) for g in gemms}
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(torch.cuda.current_device()) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            one_step(events)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+
+    # ---- end-to-end through the C ABI with host buffers (pinned), copies inside
+    for _ in range(max(1, args.warmup // 2)):
+        one_step(e2e=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        one_step(e2e=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+
+    flops_step = sum(w4a16_flops(m, sh["k"], sh["n"]) for sh in shapes for m in SWEEP_M)
+    bytes_step = sum(w4a16_bytes(m, sh["k"], sh["n"]) for sh in shapes for m in SWEEP_M)
+    value = flops_step * args.steps * world / (ms * 1e-3) / 1e12
+    e2e_value = flops_step * args.steps * world / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(m * sh["k"] * 2 for sh in shapes for m in SWEEP_M)
+    d2h = sum(m * sh["n"] * 2 for sh in shapes for m in SWEEP_M)
+
+    sweep = []
+    for (si, mi) in gemms:
+        sh = shapes[si]
+        m = SWEEP_M[mi]
+        st, en = events[(si, mi)]
+        us = statistics.mean(a.elapsed_time(b) for a, b in zip(st, en)) * 1e3
+        fl = w4a16_flops(m, sh["k"], sh["n"])
+        by = w4a16_bytes(m, sh["k"], sh["n"])
+        tf = fl / (us * 1e-6) / 1e12
+        gb = by / (us * 1e-6) / 1e9
+        ridge = peaks["bf16_tflops"] * 1e3 / peaks["hbm_gbs"]        # flop per byte
+        bound = "hbm" if fl / by < ridge else "tensor"
+        frac = gb / peaks["hbm_gbs"] if bound == "hbm" else tf / peaks["bf16_tflops"]
+        sweep.append(dict(m=m, k=sh["k"], n=sh["n"], us=round(us, 2), tflops=round(tf, 1), gbs=round(gb, 1),
+                          bound=bound, frac=round(frac, 3)))
+
+    def roof(entries, bound):
+        # the dominant launch class: time-weighted over the given launches
+        t = sum(e["us"] for e in entries)
+        if bound == "hbm":
+            ach = sum(w4a16_bytes(e["m"], e["k"], e["n"]) for e in entries) / (t * 1e-6) / 1e9
+            return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                        frac=round(ach / peaks["hbm_gbs"], 3), traffic=None,
+                        launches=[f"M={e['m']},K={e['k']},N={e['n']}" for e in entries],
+                        peak_source=f"{peaks['source']} (copy bandwidth, burst)")
+        ach = sum(w4a16_flops(e["m"], e["k"], e["n"]) for e in entries) / (t * 1e-6) / 1e12
+        return dict(bound="tensor", achieved=round(ach, 1), peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                    frac=round(ach / peaks["bf16_tflops"], 3), traffic=None,
+                    launches=[f"M={e['m']},K={e['k']},N={e['n']}" for e in entries],
+                    peak_source=f"{peaks['source']} (cuBLAS bf16 8192^3, burst)")
+
+    big = [e for e in sweep if e["m"] == 4096]
+    small = [e for e in sweep if e["m"] <= 16]
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 x int4 (fp32 accumulate)",
+        "data": "synthetic (seeded; uniform int4 codes, fp16 scales 0.002+0.01|N(0,1)|, bf16 N(0,1) activations)",
+        "config": {
+            "workload": "dense W4A16 M-sweep: M in {1,4,16,64,256,1024,4096} x (K,N) in {(7168,18432),"
+                        "(18432,7168)}, symmetric INT4, group 128",
+            "gemms_per_step": len(gemms),
+            "l2": f"weights rotate over {len(shapes[0]['blobs'])} copies per shape (>3x L2), no flush",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": roof(big, "tensor"),
+        "roofline_small_m": roof(small, "hbm"),
+        "sweep": sweep,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(gemms) * args.steps,
+        "clocks": clocks,
+        "algorithmic_bytes_per_step": bytes_step,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_w4a16(budget_s=args.cpu_budget)
+    return line
+
+
+# ---------------------------------------------------------------- other workloads
+
+FP8_RATIO, FP4_RATIO = 2.0, 4.0   # nominal dense peaks relative to bf16 (4.5 / 9 vs 2.25 PF)
+
+
+def _time_launches(launches, steps, warmup, world):
+    """Run `launches` (list of callables) once per step; returns (total ms
+    over `steps`, per-launch mean microseconds)."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for f in launches:
+            f()
+    torch.cuda.synchronize()
+    ev = [([], []) for _ in launches]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        for i, f in enumerate(launches):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            f()
+            b.record(stream)
+            ev[i][0].append(a)
+            ev[i][1].append(b)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    per = [statistics.mean(a.elapsed_time(b) for a, b in zip(*e)) * 1e3 for e in ev]
+    return ms, per
+
+
+def run_mxfp4(args, rank, world, peaks):
+    """W4A8-MXFP4: M in {16, 256, 4096}, K = N = 7168."""
+    from quantized_gemm_bit_b200 import hq, synth
+    k = n = 7168
+    codes, e8 = synth.mxfp4_weights(n, k, seed=2000)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, n, k, 32, 0, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).cuda()
+    blobs = [blob] + [blob.clone() for _ in range(5)]
+    launches, rows = [], []
+    ctr = [0]
+    for m in (16, 256, 4096):
+        x = synth.bf16_normal(m, k, seed=2000 + m).cuda()
+        q = torch.empty(m, k, dtype=torch.uint8, device="cuda")
+        sc = torch.empty(m, dtype=torch.float32, device="cuda")
+        hq.hq_quantize_fp8_rows(x, m, k, q, sc)
+        c = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(max(256, hq.hq_workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+
+        def f(m=m, q=q, sc=sc, c=c, ws=ws):
+            ctr[0] += 1
+            hq.hq_gemm_mxfp4_a8(d, blobs[ctr[0] % 6], q, sc, m, c, ws)
+        launches.append(f)
+        rows.append(m)
+    ms, per = _time_launches(launches, args.steps, args.warmup, world)
+    peak = peaks["bf16_tflops"] * FP8_RATIO
+    out = []
+    for m, us in zip(rows, per):
+        fl = 2.0 * m * n * k
+        by = n * k // 2 + n * k // 32 + m * k + 4 * m + 2 * m * n
+        out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1), gbs=round(by / us / 1e3, 1),
+                        frac_fp8_peak=round(fl / us / 1e6 / peak, 3), frac_hbm=round(by / us / 1e3 / peaks["hbm_gbs"], 3)))
+    flops = sum(2.0 * m * n * k for m in rows)
+    return {"workload": "W4A8-MXFP4 GEMM, M in {16,256,4096}, K=N=7168", "value": round(flops * args.steps * world
+            / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms / args.steps, 4),
+            "peak_fp8_tflops": round(peak, 1), "peak_source": "measured bf16 x nominal fp8/bf16 ratio 2",
+            "detail": out}
+
+
+def run_nvfp4(args, rank, world, peaks):
+    """NVFP4 W4A4: 8192^3 and M=16384, K=7168, N=18432 (inputs quantized from
+    bf16 N(0,1) draws on the GPU by the library's own quantizer)."""
+    from quantized_gemm_bit_b200 import hq, synth
+    launches, shapes = [], []
+    for si, (m, n, k) in enumerate(((8192, 8192, 8192), (16384, 18432, 7168))):
+        def quant(rows, seed):
+            x = synth.bf16_normal(rows, k, seed).cuda()
+            codes = torch.empty(rows, k // 2, dtype=torch.uint8, device="cuda")
+            sf = torch.empty(rows, k // 16, dtype=torch.uint8, device="cuda")
+            g = torch.empty(1, dtype=torch.float32, device="cuda")
+            wsq = torch.zeros(hq.hq_quantize_nvfp4_workspace_size(rows, k), dtype=torch.uint8, device="cuda")
+            hq.hq_quantize_nvfp4(x, rows, k, codes, sf, g, wsq)
+            return codes, sf, g
+        wc, wsf, wg = quant(n, 4000 + si)
+        ac, asf, ag = quant(m, 4100 + si)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, n, k, 16, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, wc.cpu(), wsf.cpu(), None, float(wg.item()))).cuda()
+        c = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(max(256, hq.hq_workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+        a_g = float(ag.item())
+
+        def f(m=m, d=d, blob=blob, ac=ac, asf=asf, a_g=a_g, c=c, ws=ws):
+            hq.hq_gemm_nvfp4(d, blob, ac, asf, a_g, m, c, ws)
+        launches.append(f)
+        shapes.append((m, n, k))
+    ms, per = _time_launches(launches, args.steps, args.warmup, world)
+    peak = peaks["bf16_tflops"] * FP4_RATIO
+    out = []
+    for (m, n, k), us in zip(shapes, per):
+        fl = 2.0 * m * n * k
+        out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1),
+                        frac_fp4_peak=round(fl / us / 1e6 / peak, 3)))
+    flops = sum(2.0 * m * n * k for m, n, k in shapes)
+    return {"workload": "NVFP4 W4A4 GEMM, 8192^3 and M=16384 K=7168 N=18432", "value": round(
+            flops * args.steps * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms / args.steps, 4), "peak_fp4_tflops": round(peak, 1),
+            "peak_source": "measured bf16 x nominal fp4/bf16 ratio 4", "detail": out}
+
+
+def run_moe(args, rank, world, peaks):
+    """Grouped MoE W4A16: 256 experts, top-8, hidden 7168, gate+up N=4096,
+    down K=2048, T in {64, 1024, 8192}: route + permute + two grouped GEMMs."""
+    from quantized_gemm_bit_b200 import hq, synth
+    E, TOPK, H = 256, 8, 7168
+    mats = {}
+    for name, (n, k, seed) in {"gate_up": (4096, H, 3000), "down": (H, 2048, 3010)}.items():
+        q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=seed, experts=E)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, E)
+        mats[name] = (d, torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).cuda(), n, k)
+        del q, s
+    detail, launches, meta = [], [], []
+    for t in (64, 1024, 8192):
+        logits = synth.router_logits(t, E, seed=3001).cuda()
+        x = synth.bf16_normal(t, H, seed=3002).cuda()
+        xd = synth.bf16_normal(t * TOPK, 2048, seed=3003).cuda()
+        ids = torch.empty(t, TOPK, dtype=torch.int32, device="cuda")
+        src = torch.empty(t * TOPK, dtype=torch.int32, device="cuda")
+        off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        xs = torch.empty(t * TOPK, H, dtype=torch.bfloat16, device="cuda")
+        pws = torch.zeros(hq.hq_moe_permute_workspace_size(t, TOPK, E), dtype=torch.uint8, device="cuda")
+        c1 = torch.empty(t * TOPK, 4096, dtype=torch.bfloat16, device="cuda")
+        c2 = torch.empty(t * TOPK, H, dtype=torch.bfloat16, device="cuda")
+        d1, w1, _, _ = mats["gate_up"]
+        d2, w2, _, _ = mats["down"]
+        ws1 = torch.zeros(max(256, hq.hq_workspace_size(d1, t * TOPK)), dtype=torch.uint8, device="cuda")
+        ws2 = torch.zeros(max(256, hq.hq_workspace_size(d2, t * TOPK)), dtype=torch.uint8, device="cuda")
+
+        def route(t=t, logits=logits, ids=ids, src=src, off=off, x=x, xs=xs, pws=pws):
+            hq.hq_moe_topk(logits, t, E, TOPK, ids)
+            hq.hq_moe_permute(ids, t, TOPK, E, src, off, pws, a=x, hidden=H, a_sorted=xs)
+
+        def g1(t=t, xs=xs, off=off, c1=c1, ws1=ws1):
+            hq.hq_grouped_gemm_moe(d1, w1, xs, off, t * TOPK, c1, ws1)
+
+        def g2(t=t, xd=xd, off=off, c2=c2, ws2=ws2):
+            hq.hq_grouped_gemm_moe(d2, w2, xd, off, t * TOPK, c2, ws2)
+        launches += [route, g1, g2]
+        meta.append((t, off))
+    ms, per = _time_launches(launches, args.steps, args.warmup, world)
+    tok_total, time_total = 0, 0.0
+    for i, (t, off) in enumerate(meta):
+        r_us, g1_us, g2_us = per[3 * i: 3 * i + 3]
+        offs = off.cpu().numpy()
+        active = int((offs[1:] > offs[:-1]).sum())
+        wbytes = active * (4096 * 7168 // 2 + 4096 * 56 * 2 + 7168 * 2048 // 2 + 7168 * 16 * 2)
+        fl = 2.0 * t * TOPK * 7168 * 6144
+        gemm_us = g1_us + g2_us
+        detail.append(dict(tokens=t, active_experts=active, route_permute_us=round(r_us, 2),
+                           gate_up_us=round(g1_us, 2), down_us=round(g2_us, 2),
+                           tok_per_s=round(t / (gemm_us * 1e-6), 1), tflops=round(fl / gemm_us / 1e6, 1),
+                           weight_gbs=round(wbytes / gemm_us / 1e3, 1),
+                           frac_hbm=round(wbytes / gemm_us / 1e3 / peaks["hbm_gbs"], 3)))
+        tok_total += t
+        time_total += gemm_us
+    return {"workload": "grouped MoE W4A16: 256 experts, top-8, hidden 7168, gate+up N=4096, down K=2048, "
+                        "T in {64,1024,8192}", "value": round(tok_total / (time_total * 1e-6), 1), "unit": "tok/s",
+            "ms_per_step": round(ms / args.steps, 4), "detail": detail}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def cpu_baseline_w4a16(budget_s=20.0):
+    """Time the fp64 oracle on a bounded sample of the sweep: for each shape,
+    dequantize W once and multiply 16 activation rows (the M=16 point)."""
+    from oracle import gemm as G
+    from oracle import formats as F
+    from quantized_gemm_bit_b200 import synth
+    flops, secs = 0.0, 0.0
+    for si, (k, n) in enumerate(SWEEP_KN):
+        q, s, _ = synth.w4a16_weights(n, k, GROUP, False, seed=1000 + si)
+        a = synth.bf16_normal(16, k, seed=1016)
+        bits = a.view(torch.int16).numpy().view(np.uint16)
+        t = time.perf_counter()
+        G.w4a16_ref(bits, q.numpy(), s.numpy(), None, GROUP)
+        secs += time.perf_counter() - t
+        flops += w4a16_flops(16, k, n)
+        if secs > budget_s:
+            break
+    cores = torch.get_num_threads()
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": "M=16 rows of both sweep shapes (K,N)=(7168,18432),(18432,7168): full fp64 dequant "
+                      f"of W + fp64 matmul, {secs:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cb = cpu_baseline_w4a16(budget_s=args.cpu_budget)
+    secs = []
+    for _ in range(args.warmup):
+        cpu_baseline_w4a16(budget_s=args.cpu_budget)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        cpu_baseline_w4a16(budget_s=args.cpu_budget)
+    el = time.perf_counter() - t
+    flops = sum(w4a16_flops(16, k, n) for k, n in SWEEP_KN)
+    value = flops * args.steps / el / 1e12
+    secs.append(el)
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "dense W4A16 M-sweep, bounded sample: the M=16 point of both (K,N) shapes",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "nvfp4", "moe"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    rank, world, _ = dist_init()
+    from quantized_gemm_bit_b200.build import build
+    if rank == 0:
+        build()
+    barrier(world)
+    peaks = load_peaks()
+    if args.workload == "w4a16_sweep":
+        line = run_w4a16_sweep(args, rank, world, peaks)
+    else:
+        fn = {"mxfp4": run_mxfp4, "nvfp4": run_nvfp4, "moe": run_moe}[args.workload]
+        line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": True, "scaling": "weak", "data": "synthetic (seeded)"}
+        line.update(fn(args, rank, world, peaks))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -94,8 +94,9 @@ typedef struct {
  *   tile_m   : token tile (the MMA N extent): 16, 32, 64, 128 or 256
  *   tile_n   : weight rows per tile: 128 (the only value)
  *   tile_k   : K per pipeline stage: 128 (fixed by the packed layout)
- *   stages   : shared-memory pipeline depth
- *   split_k  : number of K splits reduced in the workspace (>= 1)
+ *   stages   : 0 (the pipeline depth is fixed per token tile)
+ *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
+ *              splits the whole iteration space evenly when 0)
  *   cta_group: 1 (one SM per MMA)
  *   variant  : 0                                                             */
 typedef struct {
@@ -131,7 +132,8 @@ size_t hq_packed_size(const hq_quant_desc* d);
  *          scales_host = uint8 E8M0 [N][K/32]
  *   NVFP4: codes_host  = uint8 [N][K/2]; scales_host = uint8 E4M3 [N][K/16];
  *          global_scale = the fp32 tensor scale of the weights.
- * The output layout is documented in DESIGN.md ("packed layouts").
+ * The output layout (layout version 1) is spelled out in the header comment
+ * of the packer source, hq_pack.cpp.
  * Errors: HQ_ERR_INVALID_ARG (NULL pointers, zeros given for a symmetric
  * descriptor or missing for an asymmetric one, a zero point > 15),
  * HQ_ERR_WORKSPACE_TOO_SMALL (out_bytes < hq_packed_size). */
@@ -168,6 +170,28 @@ hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, con
 hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const void* a_fp4_dev,
                         const void* a_sf_dev, float a_global, int32_t m, void* c_dev, const hq_tuning* t,
                         void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* Activation quantization for the W4A8 GEMM ([P-fa] W4A8 combination):
+ * per row r, s_r = amax_r / 448 (1 for an all-zero row) and
+ * q[r][k] = RNE_E4M3(x[r][k] / s_r), saturating, every step in fp32 (OCP FP8
+ * rounding); zero results are written as +0.
+ *   x_bf16_dev : bf16 [rows][k], k % 8 == 0;  q_e4m3_dev : uint8 [rows][k];
+ *   scale_dev  : fp32 [rows]. */
+hq_status hq_quantize_fp8_rows(const void* x_bf16_dev, int32_t rows, int32_t k, void* q_e4m3_dev,
+                               float* scale_dev, hq_stream_t stream);
+
+/* Workspace bytes hq_quantize_nvfp4 needs. */
+size_t hq_quantize_nvfp4_workspace_size(int32_t rows, int32_t k);
+
+/* Activation quantization for the W4A4 GEMM ([P-fa] NVFP4 type, W4A4):
+ * g = amax / (448*6) over the whole tensor (1 if all zero);
+ * per 16 contiguous K: sb = RNE_E4M3(amax_block / (6 g)), d = E4M3(sb) * g,
+ * c = RNE_e2m1(x / d) saturating (0 when d == 0); fp32 throughout.
+ *   x_bf16_dev : bf16 [rows][k], k % 16 == 0
+ *   codes_dev  : uint8 [rows][k/2] (even k in the low nibble)
+ *   sf_dev     : uint8 E4M3 [rows][k/16];  global_dev : fp32 [1] (g) */
+hq_status hq_quantize_nvfp4(const void* x_bf16_dev, int32_t rows, int32_t k, void* codes_dev, void* sf_dev,
+                            float* global_dev, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
 
 /* MoE routing ([P-fa2] paragraph 5, "Grouped" path): top-k experts per
  * token by router logit (equal to top-k by softmax probability), ties to

@@ -1,0 +1,512 @@
+// Block-scaled 4-bit GEMMs for sm_100a: W4A8-MXFP4 (e2m1 weights with an
+// E8M0 scale per 32 K, E4M3 activations with a per-token fp32 scale) and
+// W4A4 NVFP4 (e2m1 with an E4M3 scale per 16 K and an fp32 tensor scale on
+// each side).
+//
+// Method: the W4A8-MXFP4 and W4A4 combinations and the MXFP4 / NVFP4 types
+// are listed on the Humming news page (section "one library, many formats",
+// table row "W4A8-MXFP4, H200"); on GPUs without native MXFP4 the library
+// converts the weights inside the kernel ("Humming: open-source kernel
+// library for quantized inference", summary paragraph 4).  B200 has the
+// native block-scaled tensor-core MMA, so here the codes go to the tensor
+// core as they are and the scales ride along in TMEM.
+//
+// B200 design:
+//   * swap-AB, as in the W4A16 kernel: 128 weight rows are the MMA's M side
+//     (A operand), the token tile (16..256) is its N side (B operand); both
+//     staged by TMA with the 128-byte swizzle.  MXFP4 weights use the TMA
+//     type that unpacks 16 four-bit codes into a 16-byte slot, the layout
+//     tcgen05.mma.kind::mxf8f6f4 reads; NVFP4 stays packed for
+//     kind::mxf4nvf4.
+//   * weight scales come from the packed blob, already in the 32x16-byte
+//     order tcgen05.cp .32x128b.warpx4 copies into TMEM; NVFP4 activation
+//     scales are loaded row-major by TMA and reordered in shared memory by
+//     one warp; MXFP4 activations carry no block scale (their E8M0 scale is
+//     1, set once in TMEM) and the per-token fp32 scale is applied in the
+//     epilogue.
+//   * warp roles: 0 producer, 1 MMA issuer (tcgen05.cp of the stage's scales
+//     then its MMAs, in issue order), 2 TMEM allocator, 3 scale reorder
+//     (NVFP4), 4-7 epilogue.  Dense stream-K with the deterministic
+//     last-contributor reduction, as in the W4A16 kernel.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "hq_internal.h"
+#include "ptx.cuh"
+
+namespace hq {
+
+namespace {
+
+constexpr int kBsThreads = 256;
+constexpr int kBsTileN = 128;
+
+enum BsFmt { kMX = 0, kNV = 1 };
+
+template <int FMT, int NTOK>
+struct BsCfg {
+  static constexpr int kKStage = FMT == kNV ? 256 : 128;   // K elements per stage: 128 B per row in SMEM
+  static constexpr int kATile = kBsTileN * 128;            // weights in SMEM
+  // bytes the weight copy moves: NVFP4 loads packed bytes; the MXFP4 load
+  // unpacks 4-bit codes into 16-byte slots and counts the packed bytes
+  static constexpr int kATx = FMT == kNV ? kATile : kBsTileN * 64;
+  static constexpr int kBTile = NTOK * 128;                // activations
+  static constexpr int kSfa = FMT == kNV ? 2048 : 512;     // weight scale chunks per stage
+  static constexpr int kHalves = NTOK > 128 ? 2 : 1;       // 128-row halves of the token tile
+  static constexpr int kSfbRaw = FMT == kNV ? NTOK * 16 : 0;
+  static constexpr int kSfbT = FMT == kNV ? 4 * kHalves * 512 : 0;
+  static constexpr int kStageRaw = kATile + kBTile + kSfa + kSfbRaw + kSfbT;
+  static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
+  static constexpr int kStages = std::min(10, (200 * 1024) / kStage);
+  static constexpr int kAcc = NTOK <= 128 ? 2 : 1;
+  // TMEM columns: accumulators, then per-stage scale slots
+  static constexpr int kSfaCols = FMT == kNV ? 16 : 4;
+  static constexpr int kSfbCols = FMT == kNV ? 16 * kHalves : 0;
+  static constexpr int kSfSlot = kSfaCols + kSfbCols;
+  static constexpr int kSfBase = kAcc * NTOK;
+  static constexpr int kSfbConst = kSfBase + kStages * kSfSlot;   // MXFP4: constant unit scales (8 cols)
+  static_assert(kSfbConst + 8 <= 512, "TMEM budget");
+  static constexpr int kBarBytes = 512;
+  static constexpr size_t kSmem = (size_t)kStages * kStage + 1024 + kBarBytes;
+  static_assert(8 * (3 * kStages + 5) + 16 <= kBarBytes, "barrier area");
+};
+
+struct BsParams {
+  const uint8_t* sf_w;       // weight scale chunks (blob + codes bytes)
+  __nv_bfloat16* c;
+  const float* a_scale;      // MXFP4: per-token scale [m]
+  const float* g_w;          // NVFP4: weight tensor scale (blob tail)
+  float a_global;            // NVFP4: activation tensor scale
+  float* partials;
+  int32_t* counters;
+  uint32_t* err;
+  uint64_t wait_ns;
+  long long total_iters;
+  int m, n, k;
+  int n_tiles, k_stages;
+  int sf_groups;             // 512-byte scale chunks per weight tile (whole K)
+};
+
+template <int FMT, int NTOK>
+__device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, int& nt, int& row0, int& rows,
+                                        int& ks0, int& ks1, int& partial, int& slot) {
+  const long long T = p.total_iters, G = gridDim.x, i = blockIdx.x;
+  const long long beg = sk_start(i, T, G), end = sk_start(i + 1, T, G);
+  const long long kst = p.k_stages;
+  const long long t = beg / kst + idx;
+  const long long x0 = idx == 0 ? beg : t * kst;
+  if (x0 >= end) return false;
+  const long long x1 = min(end, (t + 1) * kst);
+  const int mt = (int)(t / p.n_tiles);
+  tile = (int)t;
+  nt = (int)(t - (long long)mt * p.n_tiles);
+  row0 = mt * NTOK;
+  rows = min(NTOK, p.m - row0);
+  ks0 = (int)(x0 - t * kst);
+  ks1 = (int)(x1 - t * kst);
+  partial = (ks0 != 0 || ks1 != p.k_stages) ? 1 : 0;
+  slot = idx == 0 ? 0 : 1;
+  return true;
+}
+
+template <int FMT, int NTOK>
+__global__ void __launch_bounds__(kBsThreads, 1)
+    blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
+                       const __grid_constant__ CUtensorMap tmap_sfb, const BsParams p) {
+  using C = BsCfg<FMT, NTOK>;
+  constexpr int S = C::kStages;
+  constexpr int ACC = C::kAcc;
+  constexpr uint32_t kTx = C::kATx + C::kBTile + C::kSfa + C::kSfbRaw;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStage);
+  uint64_t* empty = full + S;
+  uint64_t* sfb_ready = empty + S;
+  uint64_t* acc_full = sfb_ready + S;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+
+  auto sA = [&](int s) { return smem + s * C::kStage; };
+  auto sB = [&](int s) { return smem + s * C::kStage + C::kATile; };
+  auto sSfa = [&](int s) { return smem + s * C::kStage + C::kATile + C::kBTile; };
+  auto sSfbRaw = [&](int s) { return sSfa(s) + C::kSfa; };
+  auto sSfbT = [&](int s) { return sSfbRaw(s) + C::kSfbRaw; };
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sfb_ready[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmap_w);
+    prefetch_tensormap(&tmap_a);
+    if (FMT == kNV) prefetch_tensormap(&tmap_sfb);
+  }
+  if (warp == 2) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  if (FMT == kMX && warp >= 4) {
+    // activations carry no block scale: E8M0 127 (= 1.0) in every byte
+    tmem_st_x8(tmem_base + (((warp & 3) * 32) << 16) + C::kSfbConst, 0x7F7F7F7Fu);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  int tile, nt, row0, rows, ks0, ks1, partial, slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!hq_wait(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], kTx);
+          // weights: K coordinate in elements (MXFP4 unpacking type) or bytes (NVFP4)
+          tma_load_2d(sA(s), &tmap_w, FMT == kNV ? ks * 128 : ks * C::kKStage, nt * kBsTileN, &full[s]);
+          tma_load_2d(sB(s), &tmap_a, ks * 128, row0, &full[s]);
+          const int chunks = FMT == kNV ? 4 : 1;
+          const uint8_t* src = p.sf_w + ((size_t)nt * p.sf_groups + (size_t)ks * chunks) * 512;
+          bulk_g2s(sSfa(s), src, C::kSfa, &full[s], pol_w);
+          if (FMT == kNV) tma_load_2d(sSfbRaw(s), &tmap_sfb, ks * 16, row0, &full[s]);
+        }
+      }
+      if (!ok) {
+        const uint32_t first = it > (uint32_t)S ? it - S : 0;
+        for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % S], (j / S) & 1, p.wait_ns, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, uc = 0;
+      bool ok = true;
+      for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
+           ++idx, ++uc) {
+        const int ab = uc % ACC;
+        const uint32_t aph = (uc / ACC) & 1;
+        if (!hq_wait(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
+          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + ab * NTOK;
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          bool got = hq_wait(&full[s], ph, p.wait_ns, s_abort);
+          if (got && FMT == kNV) got = hq_wait(&sfb_ready[s], ph, p.wait_ns, s_abort);
+          if (!got) {
+            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA(s));
+          const uint32_t b_base = smem_u32(sB(s));
+          const uint32_t sf_col = C::kSfBase + s * C::kSfSlot;
+          if (FMT == kNV) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t sfa_t = tmem_base + sf_col + 4 * i;
+              const uint32_t sfb_t = tmem_base + sf_col + 16 + 4 * C::kHalves * i;
+              tmem_cp_sf(sfa_t, smem_desc_sf(smem_u32(sSfa(s)) + 512 * i));
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h)
+                tmem_cp_sf(sfb_t + 4 * h, smem_desc_sf(smem_u32(sSfbT(s)) + 512 * (i * C::kHalves + h)));
+              constexpr uint32_t kId = idesc_block_scaled(1, 1, 0, 128, NTOK, 0, 0);
+              mma_mxf4nvf4(d_tmem, smem_desc_sw128(a_base + 32 * i), smem_desc_sw128(b_base + 32 * i), kId, sfa_t,
+                           sfb_t, (ks > ks0 || i > 0) ? 1u : 0u);
+            }
+          } else {
+            const uint32_t sfa_t = tmem_base + sf_col;
+            tmem_cp_sf(sfa_t, smem_desc_sf(smem_u32(sSfa(s))));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              // byte i of each scale column holds the scale of 32-K block i
+              const uint32_t id = idesc_block_scaled(5, 0, 1, 128, NTOK, (uint32_t)i, 0);
+              mma_mxf8f6f4(d_tmem, smem_desc_sw128(a_base + 32 * i), smem_desc_sw128(b_base + 32 * i), id, sfa_t,
+                           tmem_base + C::kSfbConst, (ks > ks0 || i > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[ab]);
+      }
+      tc_commit(drain);
+      hq_wait(drain, 0, p.wait_ns, nullptr);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ NVFP4 activation-scale reorder
+    if (FMT == kNV) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
+        for (int ks = ks0; ks < ks1; ++ks, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!hq_wait(&full[s], ph, p.wait_ns, s_abort)) {
+            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+            ok = false;
+            break;
+          }
+          // raw: [NTOK rows][16 scale bytes]; chunk (MMA i, half h): byte
+          // l*16 + 4c + j = scale of row h*128 + l + 32c, block 4i + j
+          const uint8_t* raw = sSfbRaw(s);
+          uint8_t* dst = sSfbT(s);
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            uint4 rw[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int row = h * 128 + (int)lane + 32 * c;
+              rw[c] = row < NTOK ? *reinterpret_cast<const uint4*>(raw + row * 16) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t w0 = i == 0 ? rw[0].x : i == 1 ? rw[0].y : i == 2 ? rw[0].z : rw[0].w;
+              const uint32_t w1 = i == 0 ? rw[1].x : i == 1 ? rw[1].y : i == 2 ? rw[1].z : rw[1].w;
+              const uint32_t w2 = i == 0 ? rw[2].x : i == 1 ? rw[2].y : i == 2 ? rw[2].z : rw[2].w;
+              const uint32_t w3 = i == 0 ? rw[3].x : i == 1 ? rw[3].y : i == 2 ? rw[3].z : rw[3].w;
+              *reinterpret_cast<uint4*>(dst + (i * C::kHalves + h) * 512 + lane * 16) = make_uint4(w0, w1, w2, w3);
+            }
+          }
+          fence_proxy_async_smem();  // make the reordered scales visible to tcgen05.cp
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfb_ready[s]);
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3;
+    const int r = (int)(q * 32 + lane);
+    const uint32_t lane_addr = (q * 32) << 16;
+    const float alpha = FMT == kNV ? p.a_global * __ldg(p.g_w) : 1.f;
+    uint32_t uc = 0;
+    for (int idx = 0; bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx, ++uc) {
+      const int ab = uc % ACC;
+      const uint32_t aph = (uc / ACC) & 1;
+      if (!hq_wait(&acc_full[ab], aph, p.wait_ns, s_abort)) {
+        raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const int n = nt * kBsTileN + r;
+      const bool n_ok = n < p.n;
+      float* part = partial ? p.partials + ((size_t)blockIdx.x * 2 + slot) * NTOK * kBsTileN : nullptr;
+#pragma unroll 1
+      for (int j0 = 0; j0 < NTOK; j0 += 16) {
+        uint32_t v[16];
+        tmem_ld_x16(tmem_base + lane_addr + ab * NTOK + j0, v);
+        tmem_wait_ld();
+        if (partial) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(part + (size_t)(j0 + j) * kBsTileN + r, __uint_as_float(v[j]));
+        } else if (n_ok) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (j0 + j < rows) {
+              const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + j0 + j);
+              p.c[(size_t)(row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (partial) {
+        const long long T = p.total_iters, G = gridDim.x, kst = p.k_stages;
+        const long long t0 = (long long)tile * kst;
+        const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kst - 1, T, G);
+        const int cnt = (int)(last - first + 1);
+        __threadfence();
+        __syncwarp();
+        int is_last = 0;
+        if (lane == 0) {
+          __threadfence();
+          is_last = (atomicAdd(p.counters + tile * 4 + q, 1) == cnt - 1);
+          __threadfence();
+        }
+        is_last = __shfl_sync(0xffffffffu, is_last, 0);
+        if (is_last) {
+          __threadfence();
+          for (int j = 0; j < rows; ++j) {
+            float acc = 0.f;
+            for (long long ci = first; ci <= last; ++ci) {
+              const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
+              acc += __ldcg(p.partials + (((size_t)ci * 2 + sl) * NTOK + j) * kBsTileN + r);
+            }
+            const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + j);
+            if (n_ok) p.c[(size_t)(row0 + j) * p.n + n] = __float2bfloat16_rn(acc * sc);
+          }
+          if (lane == 0) p.counters[tile * 4 + q] = 0;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, 512);
+}
+
+template <int FMT, int NTOK>
+hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& msf, const BsParams& p,
+                      int grid, cudaStream_t stream) {
+  auto kern = blockscaled_kernel<FMT, NTOK>;
+  const size_t smem = BsCfg<FMT, NTOK>::kSmem;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  kern<<<grid, kBsThreads, smem, stream>>>(mw, ma, msf, p);
+  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+int bs_tiles(const hq_quant_desc& d, int m, int ntok) {
+  return ((d.n + kBsTileN - 1) / kBsTileN) * ((m + ntok - 1) / ntok);
+}
+
+}  // namespace
+
+BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t) {
+  BsConfig cfg{};
+  int ntok = (t && t->tile_m) ? t->tile_m : 0;
+  if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
+  cfg.ntok = ntok;
+  const int kstage = d.fmt == HQ_FMT_NVFP4 ? 256 : 128;
+  const long long iters = (long long)bs_tiles(d, m, ntok) * (d.k / kstage);
+  long long grid = std::min<long long>(dev.num_sms, std::max<long long>(1, iters / 4));
+  if (t && t->split_k > 0) grid = std::min<long long>((long long)bs_tiles(d, m, ntok) * t->split_k, iters);
+  cfg.grid = (int)std::max<long long>(1, grid);
+  return cfg;
+}
+
+size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg) {
+  const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
+  return sizeof(WsHeader) + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256 +
+         (size_t)cfg.grid * 2 * cfg.ntok * kBsTileN * sizeof(float);
+}
+
+hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* packed, const void* a,
+                    const void* a_sf, const float* a_scale, float a_global, int m, void* c, void* ws,
+                    cudaStream_t stream) {
+  const bool nv = d.fmt == HQ_FMT_NVFP4;
+  const int n_tiles = (d.n + kBsTileN - 1) / kBsTileN;
+  const int np = n_tiles * kBsTileN;
+  const size_t codes_bytes = (size_t)np * d.k / 2;
+  BsParams p{};
+  p.sf_w = static_cast<const uint8_t*>(packed) + codes_bytes;
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.a_scale = a_scale;
+  p.sf_groups = nv ? d.k / 64 : d.k / 128;
+  p.g_w = reinterpret_cast<const float*>(p.sf_w + (size_t)n_tiles * p.sf_groups * 512);
+  p.a_global = a_global;
+  p.err = static_cast<uint32_t*>(ws);
+  p.wait_ns = kDefaultWaitNs;
+  p.m = m;
+  p.n = d.n;
+  p.k = d.k;
+  p.n_tiles = n_tiles;
+  p.k_stages = d.k / (nv ? 256 : 128);
+  const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
+  p.total_iters = (long long)tiles * p.k_stages;
+  uint8_t* base = static_cast<uint8_t*>(ws) + sizeof(WsHeader);
+  p.counters = reinterpret_cast<int32_t*>(base);
+  p.partials = reinterpret_cast<float*>(base + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256);
+
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return HQ_ERR_CUDA;
+  CUtensorMap mw{}, ma{}, msf{};
+  cuuint32_t estr[2] = {1, 1};
+  // weights: codes [NP][K/2] bytes
+  {
+    cuuint64_t dims[2] = {nv ? (cuuint64_t)d.k / 2 : (cuuint64_t)d.k, (cuuint64_t)np};
+    cuuint64_t strides[1] = {(cuuint64_t)d.k / 2};
+    cuuint32_t box[2] = {128, (cuuint32_t)kBsTileN};
+    CUresult cr = enc(&mw, nv ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2,
+                      const_cast<void*>(packed), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
+  }
+  // activations: NVFP4 [M][K/2] bytes, MXFP4 E4M3 [M][K] bytes
+  {
+    const cuuint64_t row_bytes = nv ? (cuuint64_t)d.k / 2 : (cuuint64_t)d.k;
+    cuuint64_t dims[2] = {row_bytes, (cuuint64_t)m};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {128, (cuuint32_t)cfg.ntok};
+    CUresult cr = enc(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
+  }
+  // NVFP4 activation scales: [M][K/16] bytes, 16 per row per stage
+  if (nv) {
+    cuuint64_t dims[2] = {(cuuint64_t)d.k / 16, (cuuint64_t)m};
+    cuuint64_t strides[1] = {(cuuint64_t)d.k / 16};
+    cuuint32_t box[2] = {16, (cuuint32_t)cfg.ntok};
+    CUresult cr = enc(&msf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a_sf), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
+  } else {
+    msf = ma;  // unused
+  }
+
+#define HQ_BS_CASE(F, NT) \
+  case NT: return bs_launch_t<F, NT>(mw, ma, msf, p, cfg.grid, stream);
+  if (nv) {
+    switch (cfg.ntok) {
+      HQ_BS_CASE(kNV, 16) HQ_BS_CASE(kNV, 32) HQ_BS_CASE(kNV, 64) HQ_BS_CASE(kNV, 128) HQ_BS_CASE(kNV, 256)
+      default: return HQ_ERR_UNSUPPORTED;
+    }
+  }
+  switch (cfg.ntok) {
+    HQ_BS_CASE(kMX, 16) HQ_BS_CASE(kMX, 32) HQ_BS_CASE(kMX, 64) HQ_BS_CASE(kMX, 128) HQ_BS_CASE(kMX, 256)
+    default: return HQ_ERR_UNSUPPORTED;
+  }
+#undef HQ_BS_CASE
+}
+
+}  // namespace hq

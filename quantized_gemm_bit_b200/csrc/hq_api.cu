@@ -146,12 +146,15 @@ hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const 
 
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t) {
   if (check_desc(d) != HQ_OK || m < 0) return 0;
-  if (d->fmt != HQ_FMT_INT4) return sizeof(WsHeader);
   DeviceInfo dev{};
   if (device_info(&dev) != HQ_OK) {
     // no sm_100 device current: size for a 148-SM part so the answer is
     // still an upper bound the caller can allocate
     dev.num_sms = 148;
+  }
+  if (d->fmt != HQ_FMT_INT4) {
+    BsConfig cfg = bs_plan(dev, *d, m < 1 ? 1 : m, t);
+    return bs_workspace_bytes(*d, m < 1 ? 1 : m, cfg);
   }
   const bool grouped = d->num_experts > 1;
   W4Config cfg = w4_plan(dev, *d, m < 1 ? 1 : m, grouped, t);
@@ -171,7 +174,7 @@ hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const 
   if (t) {
     if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
       return HQ_ERR_UNSUPPORTED;
-    if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 ||
+    if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
         (t->cta_group && t->cta_group != 1) || t->variant != 0)
       return HQ_ERR_UNSUPPORTED;
   }
@@ -179,7 +182,6 @@ hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const 
   st = device_info(&dev);
   if (st != HQ_OK) return st;
   W4Config cfg = w4_plan(dev, *d, m, false, t);
-  if (cfg.stages != w4_stages_for(cfg.ntok)) return HQ_ERR_UNSUPPORTED;
   if (ws_bytes < w4_workspace_bytes(*d, m, cfg, false)) return HQ_ERR_WORKSPACE_TOO_SMALL;
   return w4_launch(*d, cfg, packed_w_dev, a_dev, m, c_dev, nullptr, ws_dev, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -199,7 +201,7 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
   if (t) {
     if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
       return HQ_ERR_UNSUPPORTED;
-    if (t->split_k > 1 || (t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) ||
+    if (t->split_k > 1 || (t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->stages != 0 ||
         (t->cta_group && t->cta_group != 1) || t->variant != 0)
       return HQ_ERR_UNSUPPORTED;
   }
@@ -207,32 +209,98 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
   st = device_info(&dev);
   if (st != HQ_OK) return st;
   W4Config cfg = w4_plan(dev, *d, total_rows, true, t);
-  if (cfg.stages != w4_stages_for(cfg.ntok)) return HQ_ERR_UNSUPPORTED;
   if (ws_bytes < w4_workspace_bytes(*d, total_rows, cfg, true)) return HQ_ERR_WORKSPACE_TOO_SMALL;
   return w4_launch(*d, cfg, packed_w_dev, a_sorted_dev, total_rows, c_sorted_dev, expert_offsets_dev, ws_dev,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+hq_status check_bs_tuning(const hq_tuning* t) {
+  if (!t) return HQ_OK;
+  if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
+    return HQ_ERR_UNSUPPORTED;
+  if ((t->tile_n && t->tile_n != 128) || t->tile_k || t->split_k < 0 || t->stages != 0 ||
+      (t->cta_group && t->cta_group != 1) || t->variant != 0)
+    return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+}  // namespace
+
 hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, const void* a_e4m3_dev,
                            const float* a_scale_dev, int32_t m, void* c_dev, const hq_tuning* t, void* ws_dev,
                            size_t ws_bytes, hq_stream_t stream) {
-  (void)packed_w_dev; (void)a_e4m3_dev; (void)a_scale_dev; (void)c_dev; (void)t; (void)ws_dev; (void)ws_bytes;
-  (void)stream;
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
   if (d->fmt != HQ_FMT_MXFP4 || m < 0) return HQ_ERR_INVALID_ARG;
-  return HQ_ERR_UNSUPPORTED;
+  if (m == 0) return HQ_OK;
+  if (!packed_w_dev || !a_e4m3_dev || !a_scale_dev || !c_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  // the unpacking weight copy needs a 32-byte aligned blob
+  if (!aligned(packed_w_dev, 256) || !aligned(a_e4m3_dev, 16) || !aligned(a_scale_dev, 4) || !aligned(c_dev, 16) ||
+      !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  st = check_bs_tuning(t);
+  if (st != HQ_OK) return st;
+  DeviceInfo dev{};
+  st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  BsConfig cfg = bs_plan(dev, *d, m, t);
+  if (ws_bytes < bs_workspace_bytes(*d, m, cfg)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return bs_launch(*d, cfg, packed_w_dev, a_e4m3_dev, nullptr, a_scale_dev, 1.f, m, c_dev, ws_dev,
+                   reinterpret_cast<cudaStream_t>(stream));
 }
 
 hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const void* a_fp4_dev,
                         const void* a_sf_dev, float a_global, int32_t m, void* c_dev, const hq_tuning* t,
                         void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
-  (void)packed_w_dev; (void)a_fp4_dev; (void)a_sf_dev; (void)a_global; (void)c_dev; (void)t; (void)ws_dev;
-  (void)ws_bytes; (void)stream;
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
   if (d->fmt != HQ_FMT_NVFP4 || m < 0) return HQ_ERR_INVALID_ARG;
-  return HQ_ERR_UNSUPPORTED;
+  if (m == 0) return HQ_OK;
+  if (!packed_w_dev || !a_fp4_dev || !a_sf_dev || !c_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(packed_w_dev, 256) || !aligned(a_fp4_dev, 16) || !aligned(a_sf_dev, 16) || !aligned(c_dev, 16) ||
+      !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  st = check_bs_tuning(t);
+  if (st != HQ_OK) return st;
+  DeviceInfo dev{};
+  st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  BsConfig cfg = bs_plan(dev, *d, m, t);
+  if (ws_bytes < bs_workspace_bytes(*d, m, cfg)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return bs_launch(*d, cfg, packed_w_dev, a_fp4_dev, a_sf_dev, nullptr, a_global, m, c_dev, ws_dev,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_quantize_fp8_rows(const void* x_bf16_dev, int32_t rows, int32_t k, void* q_e4m3_dev,
+                               float* scale_dev, hq_stream_t stream) {
+  if (rows < 0 || k < 1 || k % 8 != 0) return HQ_ERR_INVALID_ARG;
+  if (rows == 0) return HQ_OK;
+  if (!x_bf16_dev || !q_e4m3_dev || !scale_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x_bf16_dev, 16) || !aligned(q_e4m3_dev, 8) || !aligned(scale_dev, 4)) return HQ_ERR_ALIGNMENT;
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  return fp8_rows_launch(x_bf16_dev, rows, k, q_e4m3_dev, scale_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_quantize_nvfp4_workspace_size(int32_t rows, int32_t k) {
+  if (rows < 0 || k < 1) return 0;
+  return nvfp4_quant_ws_bytes(rows, k);
+}
+
+hq_status hq_quantize_nvfp4(const void* x_bf16_dev, int32_t rows, int32_t k, void* codes_dev, void* sf_dev,
+                            float* global_dev, void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
+  if (rows < 0 || k < 1 || k % 16 != 0) return HQ_ERR_INVALID_ARG;
+  if (rows == 0) return HQ_OK;
+  if (!x_bf16_dev || !codes_dev || !sf_dev || !global_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x_bf16_dev, 16) || !aligned(codes_dev, 8) || !aligned(global_dev, 4) || !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  if (ws_bytes < nvfp4_quant_ws_bytes(rows, k)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  return nvfp4_quant_launch(x_bf16_dev, rows, k, codes_dev, sf_dev, global_dev, ws_dev,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 hq_status hq_moe_topk(const float* logits_dev, int32_t t, int32_t e, int32_t k, int32_t* topk_ids_dev,

@@ -26,8 +26,8 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 // Resolved launch configuration of the W4A16 kernel family.
 struct W4Config {
   int ntok;     // token tile (MMA N)
-  int stages;
-  int splits;   // split-K factor (dense only)
+  int stages;   // unused (pipeline depth is fixed per token tile)
+  int splits;   // unused (dense mode is stream-K over `grid` CTAs)
   int grid;     // CTAs
 };
 
@@ -42,9 +42,24 @@ hq_status device_info(DeviceInfo* out);
 // W4A16 (dense or grouped) planning and launch.
 W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t);
 size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bool grouped);
-int w4_stages_for(int ntok);
 hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m,
                     void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream);
+
+// Block-scaled 4-bit GEMMs (MXFP4 weights x E4M3 activations; NVFP4 x NVFP4).
+struct BsConfig {
+  int ntok;
+  int grid;
+};
+BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t);
+size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg);
+hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* packed, const void* a, const void* a_sf,
+                    const float* a_scale, float a_global, int m, void* c, void* ws, cudaStream_t stream);
+
+// Activation quantizers.
+size_t nvfp4_quant_ws_bytes(int rows, int k);
+hq_status fp8_rows_launch(const void* x, int rows, int k, void* q, float* scale, cudaStream_t s);
+hq_status nvfp4_quant_launch(const void* x, int rows, int k, void* codes, void* sf, float* g, void* ws,
+                             cudaStream_t s);
 
 // MoE helpers.
 size_t moe_permute_ws_bytes(int t, int k, int e);

@@ -201,3 +201,78 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
 }
 
 }  // namespace hq
+
+namespace hq {
+
+// Shared-memory descriptor for a 32-row x 16-byte block without swizzle
+// (rows 16 B apart, 8-row groups 128 B apart): the source of
+// tcgen05.cp .32x128b.warpx4 for block scale factors.
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);   // start address
+  d |= static_cast<uint64_t>(0) << 16;                      // leading byte offset (single 16-B column)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;               // stride byte offset: 8 rows * 16 B
+  d |= static_cast<uint64_t>(1) << 46;                      // descriptor version (sm_100)
+  return d;                                                 // layout: no swizzle (0)
+}
+
+// Copy 32 rows x 128 bits of scale factors from shared memory into TMEM
+// lanes 0..31, replicated into all four 32-lane sub-partitions.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Block-scaled MMAs, A and B from shared memory, scale factors from TMEM.
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor of a block-scaled MMA (fp32 accumulate, K-major A
+// and B).  fmt codes: kind::mxf8f6f4 E4M3 = 0, E2M1 = 5; kind::mxf4nvf4
+// E2M1 = 1.  scale_e8m0: 1 for UE8M0 scales, 0 for UE4M3.  sf_id selects
+// the byte of each 32-bit TMEM scale column the MMA reads.
+__host__ __device__ constexpr uint32_t idesc_block_scaled(uint32_t a_fmt, uint32_t b_fmt, uint32_t scale_e8m0,
+                                                          uint32_t m, uint32_t n, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id << 4) | (a_fmt << 7) | (b_fmt << 10) | ((n >> 3) << 17) | (scale_e8m0 << 23) | ((m >> 4) << 24) |
+         (a_sf_id << 29);
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr), "r"(v)
+      : "memory");
+}
+
+// Stream-K over a dense (tile, k-block) iteration space: CTA i of G owns
+// iterations [start(i), start(i+1)); owner(x) is the CTA holding x.
+__device__ __forceinline__ long long sk_start(long long i, long long T, long long G) { return i * T / G; }
+__device__ __forceinline__ long long sk_owner(long long x, long long T, long long G) {
+  return ((x + 1) * G - 1) / T;
+}
+
+__device__ __forceinline__ void raise_error(uint32_t* err, volatile int* abort_flag, uint32_t code) {
+  atomicCAS(err, 0u, code);
+  *abort_flag = 1;
+}
+
+}  // namespace hq

@@ -46,68 +46,88 @@ struct W4Params {
   const uint8_t* packed;             // expert 0, record (0, 0)
   __nv_bfloat16* c;
   const int32_t* expert_offsets;     // grouped mode only
-  float* partials;
-  int32_t* counters;
+  float* partials;                   // dense: [grid][2][NTOK*128] fp32
+  int32_t* counters;                 // dense: [tiles][4]
   uint32_t* err;
   uint64_t expert_bytes;
   uint64_t wait_ns;
+  long long total_iters;             // dense: tiles * k_blocks
   int m;                             // dense: rows of A; grouped: total sorted rows
   int n;                             // output columns
-  int n_tiles, k_blocks, m_tiles, splits;
+  int n_tiles, k_blocks, m_tiles;
   int num_experts;
   int has_zero;
   int rec_bytes;
   int grouped;
+  int weights_once;                  // each weight tile is read by one CTA
+  int data_parallel;                 // dense: whole tiles per unit, no partials
 };
 
+// One unit of work: a K range of one (expert, token tile, weight tile).
 struct Unit {
   int expert;
   int nt;        // weight tile
   int row0;      // first row of A / C
   int rows;      // valid rows in this tile (<= NTOK)
   int kb0, kb1;  // k-block range
-  int tile;      // dense tile index (split-K bookkeeping)
-  int split;
+  int tile;      // dense tile index
+  int partial;   // 1: other CTAs own the rest of this tile's K range
+  int slot;      // partial slot of this CTA (0: its first unit, 1: its last)
 };
 
 template <int NTOK>
-struct Smem {
-  static constexpr int kATile = NTOK * 256;  // two 64-wide K boxes of NTOK rows x 128 B
-};
-
-__device__ __forceinline__ void raise_error(uint32_t* err, volatile int* abort_flag, uint32_t code) {
-  atomicCAS(err, 0u, code);
-  *abort_flag = 1;
-}
-
-template <int NTOK>
-__device__ __forceinline__ bool decode_unit(const W4Params& p, const int* s_prefix, const int* s_off, int u,
-                                            Unit& x) {
-  if (!p.grouped) {
-    int per_m = p.n_tiles * p.splits;
-    int mt = u / per_m;
-    int rem = u - mt * per_m;
-    x.nt = rem / p.splits;
-    x.split = rem - x.nt * p.splits;
+__device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix, const int* s_off, int total_grouped,
+                                         int idx, Unit& x) {
+  if (!p.grouped && p.data_parallel) {
+    // whole tiles, strided over the persistent CTAs
+    const long long tile = (long long)blockIdx.x + (long long)idx * gridDim.x;
+    if (tile >= (long long)p.m_tiles * p.n_tiles) return false;
+    const int mt = (int)(tile / p.n_tiles);
+    x.tile = (int)tile;
+    x.nt = (int)(tile - (long long)mt * p.n_tiles);
     x.expert = 0;
     x.row0 = mt * NTOK;
     x.rows = min(NTOK, p.m - x.row0);
-    x.kb0 = (int)((long long)x.split * p.k_blocks / p.splits);
-    x.kb1 = (int)((long long)(x.split + 1) * p.k_blocks / p.splits);
-    x.tile = mt * p.n_tiles + x.nt;
+    x.kb0 = 0;
+    x.kb1 = p.k_blocks;
+    x.partial = 0;
+    x.slot = 0;
     return true;
   }
-  // grouped: find the expert e with prefix[e] <= u < prefix[e+1]
-  int lo = 0, hi = p.num_experts;  // invariant: prefix[lo] <= u < prefix[hi]
+  if (!p.grouped) {
+    const long long T = p.total_iters, G = gridDim.x, i = blockIdx.x;
+    const long long beg = sk_start(i, T, G), end = sk_start(i + 1, T, G);
+    const long long kb = p.k_blocks;
+    const long long tile = beg / kb + idx;
+    const long long x0 = idx == 0 ? beg : tile * kb;
+    if (x0 >= end) return false;
+    const long long x1 = min(end, (tile + 1) * kb);
+    const int mt = (int)(tile / p.n_tiles);
+    x.tile = (int)tile;
+    x.nt = (int)(tile - (long long)mt * p.n_tiles);
+    x.expert = 0;
+    x.row0 = mt * NTOK;
+    x.rows = min(NTOK, p.m - x.row0);
+    x.kb0 = (int)(x0 - tile * kb);
+    x.kb1 = (int)(x1 - tile * kb);
+    x.partial = (x.kb0 != 0 || x.kb1 != p.k_blocks) ? 1 : 0;
+    x.slot = idx == 0 ? 0 : 1;
+    return true;
+  }
+  const int u = blockIdx.x + idx * gridDim.x;
+  if (u >= total_grouped) return false;
+  // find the expert e with prefix[e] <= u < prefix[e+1] (empty experts share
+  // their prefix with the next one, so the largest such e has rows)
+  int lo = 0, hi = p.num_experts;
   while (hi - lo > 1) {
-    int mid = (lo + hi) >> 1;
+    const int mid = (lo + hi) >> 1;
     if (s_prefix[mid] <= u) lo = mid; else hi = mid;
   }
-  int e = lo;
-  int rows_e = s_off[e + 1] - s_off[e];
-  int mtiles = (rows_e + NTOK - 1) / NTOK;
-  int local = u - s_prefix[e];
-  int mt = local % mtiles;
+  const int e = lo;
+  const int rows_e = s_off[e + 1] - s_off[e];
+  const int mtiles = (rows_e + NTOK - 1) / NTOK;
+  const int local = u - s_prefix[e];
+  const int mt = local % mtiles;
   x.nt = local / mtiles;
   x.expert = e;
   x.row0 = s_off[e] + mt * NTOK;
@@ -115,43 +135,101 @@ __device__ __forceinline__ bool decode_unit(const W4Params& p, const int* s_pref
   x.kb0 = 0;
   x.kb1 = p.k_blocks;
   x.tile = 0;
-  x.split = 0;
+  x.partial = 0;
+  x.slot = 0;
   return true;
 }
 
-template <int NTOK, int STAGES>
+template <int NTOK>
+struct Cfg {
+  static constexpr int kATile = NTOK * 256;                 // two 64-wide K boxes of NTOK rows x 128 B
+  static constexpr int kSmemStages = NTOK == 16 ? 12 : NTOK == 32 ? 9 : NTOK == 64 ? 6 : NTOK == 128 ? 4 : 3;
+  static constexpr int kTmemStages = NTOK <= 64 ? 6 : NTOK == 128 ? 4 : 3;   // 64 TMEM columns each
+  static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
+  // dequantizing warpgroups; with one accumulator (256 tokens) the epilogue
+  // warpgroup dequantizes too, since the MMA waits for it anyway
+  static constexpr int kDqGroups = NTOK == 128 ? 2 : 3;
+  static constexpr int kBarBytes = 512;
+  static constexpr size_t kSmem = (size_t)kSmemStages * (kATile + kRecMax) + 1024 + kBarBytes +
+                                  2 * (kMaxExperts + 1) * sizeof(int) + 64;
+  static_assert(64 * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
+  static_assert(kTmemStages % kDqGroups == 0 && kSmemStages % kDqGroups == 0,
+                "every SMEM and TMEM stage must always return to the same dequant group");
+  static_assert(8 * (2 * kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
+};
+
+// Dequantize one 128-K block of the packed record for TMEM stage t: thread
+// (warp quarter q, lane) owns weight row r = 32q + lane and writes its 128
+// bf16 weights w = (q - z) * s into TMEM lane r, columns t*64 .. t*64+63
+// (two weights per 32-bit column, even k in the low half).
+__device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
+  uint4 raw[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+  const __half sc = reinterpret_cast<const __half*>(rec + kW4RecCodes)[r];
+  const uint32_t z = has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
+  const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
+  const uint32_t s2 = sbits | (sbits << 16);
+  // bf16(128 + z) is exact; (128 + q) - (128 + z) = q - z is exact in bf16
+  const uint32_t zbits = 0x4300u + z;
+  const uint32_t z2 = zbits | (zbits << 16);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+    uint32_t out[16];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // nibbles of k = 2j and 2j+1 sit at bits 4j and 16+4j: OR-ing them
+        // into the mantissa of bf16 128.0 gives bf16(128 + q)
+        const uint32_t x2 = lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u);
+        out[w * 4 + j] = bf16x2_mul(bf16x2_sub(x2, z2), s2);
+      }
+    }
+    tmem_st_x16(taddr + c * 16, out);
+  }
+}
+
+template <int NTOK>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
-  constexpr int ACC_BUFS = (NTOK <= 128) ? 2 : 1;
-  constexpr int kATile = Smem<NTOK>::kATile;
+  using C = Cfg<NTOK>;
+  constexpr int SS = C::kSmemStages;
+  constexpr int TS = C::kTmemStages;
+  constexpr int ACC = C::kAccBufs;
+  constexpr int NDQ = C::kDqGroups;
+  constexpr int kATile = C::kATile;
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
-  static_assert(64 * STAGES + ACC_BUFS * NTOK <= 512, "TMEM budget");
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                                  // STAGES * kATile
-  uint8_t* sR = smem + STAGES * kATile;                // STAGES * kRecMax
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sR + STAGES * kRecMax);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* aready = bars + 2 * STAGES;
-  uint64_t* acc_full = bars + 3 * STAGES;
+  uint8_t* sA = smem;                               // SS * kATile (activations, 128-byte swizzle)
+  uint8_t* sR = smem + SS * kATile;                 // SS * kRecMax (packed weight records)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sR + SS * kRecMax);
+  uint64_t* empty = full + SS;
+  uint64_t* aready = empty + SS;
+  uint64_t* afree = aready + TS;
+  uint64_t* acc_full = afree + TS;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  int* s_total = const_cast<int*>(reinterpret_cast<volatile int*>(s_abort + 1));
-  int* s_prefix = s_total + 1;                          // [kMaxExperts + 1]
-  int* s_off = s_prefix + (kMaxExperts + 1);           // [kMaxExperts + 1]
+  int* s_total = const_cast<int*>(s_abort + 1);
+  int* s_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);  // [kMaxExperts + 1]
+  int* s_off = s_prefix + (kMaxExperts + 1);                                                   // [kMaxExperts + 1]
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < SS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&aready[s], 8);
+    }
+    for (int t = 0; t < TS; ++t) {
+      mbar_init(&aready[t], 4);
+      mbar_init(&afree[t], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -159,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, 1);
     *s_abort = 0;
+    *s_total = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_a);
@@ -167,11 +246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
 
-  // Unit count: dense is static; grouped builds per-expert tile prefix sums
-  // from the device-resident row offsets.
-  if (!p.grouped) {
-    if (threadIdx.x == 0) *s_total = p.m_tiles * p.n_tiles * p.splits;
-  } else {
+  // Grouped mode: per-expert tile prefix sums from the device-resident row
+  // offsets (no host synchronization).
+  if (p.grouped) {
     const int E = p.num_experts;
     for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = p.expert_offsets[i];
     __syncthreads();
@@ -196,25 +273,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = *s_total;
+  const int total_grouped = *s_total;
 
-  auto a_col = [](int s) -> uint32_t { return (uint32_t)(s * 64); };
-  auto acc_col = [](int b) -> uint32_t { return (uint32_t)(64 * STAGES + b * NTOK); };
+  auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * 64); };
+  auto acc_col = [](int b) -> uint32_t { return (uint32_t)(64 * TS + b * NTOK); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-        Unit x;
-        decode_unit<NTOK>(p, s_prefix, s_off, u, x);
-        const uint8_t* wbase = p.packed + (uint64_t)x.expert * p.expert_bytes +
-                               (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
+      Unit x;
+      for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+        const uint8_t* wbase =
+            p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
         for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
+          const int s = it % SS;
+          const uint32_t ph = (it / SS) & 1;
           if (!hq_wait(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
             raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
             ok = false;
@@ -228,9 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         // let every copy already issued land before the CTA exits
-        uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
-        for (uint32_t j = first; j < it; ++j)
-          hq_wait(&full[j % STAGES], (j / STAGES) & 1, p.wait_ns, nullptr);
+        const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
+        for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -238,11 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, uc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++uc) {
-        Unit x;
-        decode_unit<NTOK>(p, s_prefix, s_off, u, x);
-        const int ab = uc % ACC_BUFS;
-        const uint32_t aph = (uc / ACC_BUFS) & 1;
+      Unit x;
+      for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
+        const int ab = uc % ACC;
+        const uint32_t aph = (uc / ACC) & 1;
         if (!hq_wait(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
           raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
@@ -251,9 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc_col(ab);
         for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!hq_wait(&aready[s], ph, p.wait_ns, s_abort) || !hq_wait(&full[s], ph, p.wait_ns, s_abort)) {
+          const int s = it % SS, t = it % TS;
+          const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
+          if (!hq_wait(&aready[t], ph_t, p.wait_ns, s_abort) || !hq_wait(&full[s], ph_s, p.wait_ns, s_abort)) {
             raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
             ok = false;
             break;
@@ -263,9 +337,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint64_t bdesc = smem_desc_sw128(b_base + (j >> 2) * (NTOK * 128) + (j & 3) * 32);
-            mma_bf16_ts(d_tmem, tmem_base + a_col(s) + j * 8, bdesc, kIdesc, (kb > x.kb0 || j > 0) ? 1u : 0u);
+            mma_bf16_ts(d_tmem, tmem_base + a_col(t) + j * 8, bdesc, kIdesc, (kb > x.kb0 || j > 0) ? 1u : 0u);
           }
           tc_commit(&empty[s]);
+          tc_commit(&afree[t]);
         }
         if (!ok) break;
         tc_commit(&acc_full[ab]);
@@ -274,32 +349,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain);
       hq_wait(drain, 0, p.wait_ns, nullptr);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ epilogue
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ dequantize (+ epilogue in warps 4-7)
     const uint32_t q = warp & 3;
-    const int r = (int)(q * 32 + lane);  // weight row within the tile
+    const int r = (int)(q * 32 + lane);              // weight row within the tile
     const uint32_t lane_addr = (q * 32) << 16;
-    uint32_t uc = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x, ++uc) {
-      Unit x;
-      decode_unit<NTOK>(p, s_prefix, s_off, u, x);
-      const int ab = uc % ACC_BUFS;
-      const uint32_t aph = (uc / ACC_BUFS) & 1;
+    const bool epi = warp < 8;
+    const int dq = warp >= 12 ? 1 : warp >= 8 ? 0 : 2;  // dequant group index (2: epilogue warps)
+    const bool does_dq = dq < NDQ;
+    uint32_t it = 0, uc = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
+      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
+        if (!does_dq || (int)(it % NDQ) != dq) continue;
+        const int s = it % SS, t = it % TS;
+        const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
+        // Both rings are multiples of NDQ deep, so SMEM stage s and TMEM
+        // stage t always come back to this same group: it observes every
+        // phase of the barriers it waits on, one after the other (a parity
+        // wait can only tell adjacent phases apart).
+        if (!hq_wait(&full[s], ph_s, p.wait_ns, s_abort) || !hq_wait(&afree[t], ph_t ^ 1, p.wait_ns, s_abort)) {
+          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        dequant_block(sR + s * kRecMax, r, p.has_zero, tmem_base + lane_addr + a_col(t));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&aready[t]);
+      }
+      if (!ok || !epi) continue;
+
+      // ---- epilogue of this unit (warps 4-7)
+      const int ab = uc % ACC;
+      const uint32_t aph = (uc / ACC) & 1;
       if (!hq_wait(&acc_full[ab], aph, p.wait_ns, s_abort)) {
         raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
         break;
       }
       tc_fence_after();
       const int n = x.nt * kTileN + r;
       const bool n_ok = n < p.n;
-      const bool split = p.splits > 1;
-      float* part = split ? p.partials + ((size_t)(x.tile * p.splits + x.split) * NTOK) * kTileN : nullptr;
+      float* part = x.partial ? p.partials + ((size_t)blockIdx.x * 2 + x.slot) * NTOK * kTileN : nullptr;
 #pragma unroll 1
       for (int j0 = 0; j0 < NTOK; j0 += 16) {
         uint32_t v[16];
         tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0, v);
         tmem_wait_ld();
-        if (split) {
+        if (x.partial) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) __stcg(part + (size_t)(j0 + j) * kTileN + r, __uint_as_float(v[j]));
         } else if (n_ok) {
@@ -313,78 +414,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
-      if (split) {
-        // Each epilogue warp owns 32 rows of the tile and its own counter:
-        // the last split to finish those rows reduces every partial in
-        // split order (deterministic; nobody waits on anybody).
+      if (x.partial) {
+        // Each epilogue warp owns 32 rows of the tile and one counter: the
+        // last contributing CTA reduces every partial in CTA order, so the
+        // result does not depend on arrival order (and nobody waits).
+        const long long T = p.total_iters, G = gridDim.x, kbl = p.k_blocks;
+        const long long t0 = (long long)x.tile * kbl;
+        const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kbl - 1, T, G);
+        const int cnt = (int)(last - first + 1);
         __threadfence();
         __syncwarp();
-        int last = 0;
-        if (lane == 0) last = (atomicAdd(p.counters + x.tile * 4 + q, 1) == p.splits - 1);
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
+        int is_last = 0;
+        if (lane == 0) {
           __threadfence();
-          const float* base = p.partials + (size_t)x.tile * p.splits * NTOK * kTileN;
-          for (int j = 0; j < x.rows; ++j) {
-            float acc = 0.f;
-            for (int sp = 0; sp < p.splits; ++sp) acc += __ldcg(base + ((size_t)sp * NTOK + j) * kTileN + r);
-            if (n_ok) p.c[(size_t)(x.row0 + j) * p.n + n] = __float2bfloat16_rn(acc);
+          is_last = (atomicAdd(p.counters + x.tile * 4 + q, 1) == cnt - 1);
+          __threadfence();
+        }
+        is_last = __shfl_sync(0xffffffffu, is_last, 0);
+        if (is_last) {
+          __threadfence();
+          // 16 token rows at a time, every contributor's loads in flight
+          // together; the sum runs in contributor order
+          for (int j0 = 0; j0 < x.rows; j0 += 16) {
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+            for (long long ci = first; ci <= last; ++ci) {
+              const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
+              const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kTileN + r;
+              float v[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + (size_t)j * kTileN);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[j] += v[j];
+            }
+            if (n_ok) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (j0 + j < x.rows) p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(acc[j]);
+            }
           }
           if (lane == 0) p.counters[x.tile * 4 + q] = 0;  // leave the workspace zeroed
         }
-      }
-    }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ dequantize into TMEM
-    const uint32_t q = warp & 3;
-    const int half = (int)(warp - 8) >> 2;  // chunks {2*half, 2*half+1} of each 128-K block
-    const int r = (int)(q * 32 + lane);
-    const uint32_t lane_addr = (q * 32) << 16;
-    uint32_t it = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-      Unit x;
-      decode_unit<NTOK>(p, s_prefix, s_off, u, x);
-      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        // the TMEM stage s is free once empty[s] completed for the previous
-        // round, which the producer already waited on before refilling s
-        if (!hq_wait(&full[s], ph, p.wait_ns, s_abort)) {
-          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint8_t* rec = sR + s * kRecMax;
-        const __half sc = reinterpret_cast<const __half*>(rec + kW4RecCodes)[r];
-        const uint32_t z = p.has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
-        const __nv_bfloat16 sb = __float2bfloat16_rn(__half2float(sc));
-        const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(sb);
-        const uint32_t s2 = sbits | (sbits << 16);
-        const __nv_bfloat16 zb = __float2bfloat16_rn((float)(128 + z));
-        const uint32_t zbits = (uint32_t)__bfloat16_as_ushort(zb);
-        const uint32_t z2 = zbits | (zbits << 16);
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half * 2 + cc;
-          const uint4 raw = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t out[16];
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t x2 = lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u);  // 128 + q
-              out[w * 4 + j] = bf16x2_mul(bf16x2_sub(x2, z2), s2);
-            }
-          }
-          tmem_st_x16(tmem_base + lane_addr + a_col(s) + c * 16, out);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&aready[s]);
       }
     }
   }
@@ -395,16 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(tmem_base, 512);
 }
 
-template <int NTOK, int STAGES>
-size_t smem_bytes() {
-  return (size_t)STAGES * (Smem<NTOK>::kATile + kRecMax) + 1024 /*align*/ + 256 /*barriers*/ +
-         2 * (kMaxExperts + 1) * sizeof(int) + 64;
-}
-
-template <int NTOK, int STAGES>
+template <int NTOK>
 hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_kernel<NTOK, STAGES>;
-  const size_t smem = smem_bytes<NTOK, STAGES>();
+  auto kern = w4a16_kernel<NTOK>;
+  const size_t smem = Cfg<NTOK>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -417,64 +482,74 @@ hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStre
   return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
-}  // namespace
-
-int w4_stages_for(int ntok) {
-  switch (ntok) {
-    case 16: return 7;
-    case 32: return 7;
-    case 64: return 6;
-    case 128: return 4;
-    default: return 3;
-  }
+int dense_tiles(const hq_quant_desc& d, int m, int ntok) {
+  return ((d.n + kTileN - 1) / kTileN) * ((m + ntok - 1) / ntok);
 }
+
+}  // namespace
 
 W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t) {
   W4Config cfg{};
-  const int n_tiles = (d.n + kTileN - 1) / kTileN;
-  const int k_blocks = d.k / kBlockK;
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) {
     if (grouped) {
       // average rows per expert decides the token tile
-      long long avg = (long long)m / std::max(1, d.num_experts);
+      const long long avg = (long long)m / std::max(1, d.num_experts);
       ntok = avg <= 16 ? 16 : avg <= 32 ? 32 : avg <= 64 ? 64 : 128;
     } else {
       ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
     }
   }
-  cfg.ntok = ntok;
-  cfg.stages = w4_stages_for(ntok);
-  if (t && t->stages) cfg.stages = t->stages;
+  cfg.stages = 0;
+  cfg.splits = 1;
   if (grouped) {
-    cfg.splits = 1;
+    cfg.ntok = ntok;
     cfg.grid = dev.num_sms;
     return cfg;
   }
-  const int m_tiles = (m + ntok - 1) / ntok;
-  const long long tiles = (long long)m_tiles * n_tiles;
-  int splits = 1;
-  if (t && t->split_k) {
-    splits = t->split_k;
-  } else if (tiles < dev.num_sms) {
-    splits = (int)(dev.num_sms / tiles);
-    splits = std::max(1, std::min(splits, k_blocks / 4));
+  // Whole tiles on persistent CTAs (no partial sums) when they fill the SMs
+  // well; the token tile may shrink (down to 64) to make more tiles.
+  // Otherwise stream-K with at most 64 tokens per tile, so the partial sums
+  // of a split tile stay small: every CTA gets an equal share of the
+  // (tile, k-block) space, at least 4 k-blocks each.
+  const bool fixed_tile = t && t->tile_m;
+  auto dp_eff = [&](int nt) {
+    const long long tl = dense_tiles(d, m, nt);
+    const long long waves = (tl + dev.num_sms - 1) / dev.num_sms;
+    return (double)tl / (double)(waves * dev.num_sms);
+  };
+  if (t && t->split_k > 0) {
+    // explicit request: `split_k` CTAs per tile
+    const long long tiles = dense_tiles(d, m, ntok);
+    cfg.ntok = ntok;
+    cfg.splits = t->split_k;
+    cfg.grid = (int)std::max<long long>(1, std::min<long long>(tiles * t->split_k, tiles * (d.k / kBlockK)));
+    return cfg;
   }
-  splits = std::max(1, std::min(splits, k_blocks));
-  cfg.splits = splits;
-  long long units = tiles * splits;
-  cfg.grid = (int)std::min<long long>(units, dev.num_sms);
+  for (int nt = ntok; nt >= (fixed_tile ? ntok : std::min(ntok, 64)); nt /= 2) {
+    if (dp_eff(nt) >= 0.85) {
+      cfg.ntok = nt;
+      cfg.splits = 0;  // data parallel
+      cfg.grid = (int)std::min<long long>(dev.num_sms, dense_tiles(d, m, nt));
+      return cfg;
+    }
+    if (nt == 16) break;
+  }
+  if (!fixed_tile) ntok = std::min(ntok, 64);
+  cfg.ntok = ntok;
+  const long long iters = (long long)dense_tiles(d, m, ntok) * (d.k / kBlockK);
+  long long grid = std::min<long long>(dev.num_sms, std::max<long long>(1, iters / 4));
+  cfg.grid = (int)std::max<long long>(1, grid);
   return cfg;
 }
 
 size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bool grouped) {
   size_t bytes = sizeof(WsHeader);
-  if (grouped || cfg.splits <= 1) return bytes;
-  const int n_tiles = (d.n + kTileN - 1) / kTileN;
-  const int m_tiles = (m + cfg.ntok - 1) / cfg.ntok;
-  const size_t tiles = (size_t)n_tiles * m_tiles;
-  bytes += ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256;           // counters, 4 per tile
-  bytes += tiles * (size_t)cfg.splits * cfg.ntok * kTileN * sizeof(float);  // partials
+  if (grouped) return bytes;
+  if (cfg.splits == 0) return bytes;  // data parallel: no partial sums
+  const size_t tiles = (size_t)dense_tiles(d, m, cfg.ntok);
+  bytes += ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256;                   // counters, 4 per tile
+  bytes += (size_t)cfg.grid * 2 * cfg.ntok * kTileN * sizeof(float);            // partial tiles, 2 per CTA
   return bytes;
 }
 
@@ -494,12 +569,17 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.m = m;
   p.n = d.n;
   p.m_tiles = (m + cfg.ntok - 1) / cfg.ntok;
-  p.splits = cfg.splits;
   p.num_experts = grouped ? d.num_experts : 1;
   p.grouped = grouped ? 1 : 0;
   p.wait_ns = kDefaultWaitNs;
-  if (!grouped && cfg.splits > 1) {
-    const size_t tiles = (size_t)p.n_tiles * p.m_tiles;
+  if (grouped) {
+    // an expert's weight tile is re-read by each of its token tiles
+    p.weights_once = (long long)m <= (long long)cfg.ntok * d.num_experts ? 1 : 0;
+  } else {
+    const size_t tiles = (size_t)dense_tiles(d, m, cfg.ntok);
+    p.total_iters = (long long)tiles * p.k_blocks;
+    p.weights_once = p.m_tiles == 1 ? 1 : 0;
+    p.data_parallel = cfg.splits == 0 ? 1 : 0;
     uint8_t* base = static_cast<uint8_t*>(ws) + sizeof(WsHeader);
     p.counters = reinterpret_cast<int32_t*>(base);
     p.partials = reinterpret_cast<float*>(base + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256);
@@ -518,13 +598,12 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
 
-  const int grid = cfg.grid;
   switch (cfg.ntok) {
-    case 16: return cfg.stages == 7 ? launch_t<16, 7>(map, p, grid, stream) : HQ_ERR_UNSUPPORTED;
-    case 32: return cfg.stages == 7 ? launch_t<32, 7>(map, p, grid, stream) : HQ_ERR_UNSUPPORTED;
-    case 64: return cfg.stages == 6 ? launch_t<64, 6>(map, p, grid, stream) : HQ_ERR_UNSUPPORTED;
-    case 128: return cfg.stages == 4 ? launch_t<128, 4>(map, p, grid, stream) : HQ_ERR_UNSUPPORTED;
-    case 256: return cfg.stages == 3 ? launch_t<256, 3>(map, p, grid, stream) : HQ_ERR_UNSUPPORTED;
+    case 16: return launch_t<16>(map, p, cfg.grid, stream);
+    case 32: return launch_t<32>(map, p, cfg.grid, stream);
+    case 64: return launch_t<64>(map, p, cfg.grid, stream);
+    case 128: return launch_t<128>(map, p, cfg.grid, stream);
+    case 256: return launch_t<256>(map, p, cfg.grid, stream);
     default: return HQ_ERR_UNSUPPORTED;
   }
 }

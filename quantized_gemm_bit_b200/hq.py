@@ -38,7 +38,8 @@ HQ_FMT_NVFP4 = 3
 # Every symbol include/hq.h declares.
 EXPORTS = (
     "hq_layout_version", "hq_status_string", "hq_quant_desc_init", "hq_packed_size", "hq_pack_weights",
-    "hq_workspace_size", "hq_gemm_w4a16", "hq_gemm_mxfp4_a8", "hq_gemm_nvfp4", "hq_moe_topk",
+    "hq_workspace_size", "hq_gemm_w4a16", "hq_gemm_mxfp4_a8", "hq_gemm_nvfp4", "hq_quantize_fp8_rows",
+    "hq_quantize_nvfp4_workspace_size", "hq_quantize_nvfp4", "hq_moe_topk",
     "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_check_device_status",
     "hq_debug_timeout_probe",
 )
@@ -84,6 +85,9 @@ def lib():
             "hq_gemm_w4a16": (st, [dp, vp, vp, i32, vp, tp, vp, sz, vp]),
             "hq_gemm_mxfp4_a8": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
             "hq_gemm_nvfp4": (st, [dp, vp, vp, vp, ctypes.c_float, i32, vp, tp, vp, sz, vp]),
+            "hq_quantize_fp8_rows": (st, [vp, i32, i32, vp, vp, vp]),
+            "hq_quantize_nvfp4_workspace_size": (sz, [i32, i32]),
+            "hq_quantize_nvfp4": (st, [vp, i32, i32, vp, vp, vp, vp, sz, vp]),
             "hq_moe_topk": (st, [vp, i32, i32, i32, vp, vp]),
             "hq_moe_permute_workspace_size": (sz, [i32, i32, i32]),
             "hq_moe_permute": (st, [vp, i32, i32, i32, vp, vp, vp, i32, vp, vp, sz, vp]),
@@ -190,6 +194,20 @@ def hq_gemm_nvfp4(desc, packed_w, a_fp4, a_sf, a_global, m, c, ws, tuning=None, 
     _check(lib().hq_gemm_nvfp4(ctypes.byref(desc), _ptr(packed_w), _ptr(a_fp4), _ptr(a_sf), float(a_global), int(m),
                                _ptr(c), _tuning(tuning), _ptr(ws), ws.numel() * ws.element_size(),
                                _stream(stream)), "hq_gemm_nvfp4")
+
+
+def hq_quantize_fp8_rows(x, rows, k, q, scale, stream=None):
+    _check(lib().hq_quantize_fp8_rows(_ptr(x), int(rows), int(k), _ptr(q), _ptr(scale), _stream(stream)),
+           "hq_quantize_fp8_rows")
+
+
+def hq_quantize_nvfp4_workspace_size(rows, k):
+    return lib().hq_quantize_nvfp4_workspace_size(int(rows), int(k))
+
+
+def hq_quantize_nvfp4(x, rows, k, codes, sf, g, ws, stream=None):
+    _check(lib().hq_quantize_nvfp4(_ptr(x), int(rows), int(k), _ptr(codes), _ptr(sf), _ptr(g), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)), "hq_quantize_nvfp4")
 
 
 def hq_moe_topk(logits, t, e, k, topk_ids, stream=None):

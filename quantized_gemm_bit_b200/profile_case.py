@@ -1,0 +1,76 @@
+"""Run one GEMM configuration a few times through the C ABI, for profilers.
+
+    python -m quantized_gemm_bit_b200.profile_case --kind w4a16 --m 16 --k 7168 --n 18432 --iters 3
+
+Inputs are the seeded synthetic workload tensors; the device status is
+checked at the end (non-zero exit on any error).  Used to capture ncu
+profiles of single kernels on small, self-terminating cases.
+"""
+
+import argparse
+import sys
+
+import torch
+
+from . import hq, synth
+from .build import build
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "moe"])
+    ap.add_argument("--m", type=int, default=16)
+    ap.add_argument("--k", type=int, default=7168)
+    ap.add_argument("--n", type=int, default=18432)
+    ap.add_argument("--experts", type=int, default=256)
+    ap.add_argument("--topk", type=int, default=8)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--asym", action="store_true")
+    ap.add_argument("--tile-m", type=int, default=0)
+    ap.add_argument("--split-k", type=int, default=0)
+    a = ap.parse_args(argv)
+    build()
+    dev = "cuda"
+    tuning = hq.Tuning(tile_m=a.tile_m, split_k=a.split_k) if (a.tile_m or a.split_k) else None
+    if a.kind == "w4a16":
+        q, s, z = synth.w4a16_weights(a.n, a.k, 128, a.asym, seed=1000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, int(a.asym), 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+        x = synth.bf16_normal(a.m, a.k, seed=1001).to(dev)
+        c = torch.empty(a.m, a.n, dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(max(256, hq.hq_workspace_size(d, a.m, tuning)), dtype=torch.uint8, device=dev)
+        for _ in range(a.iters):
+            hq.hq_gemm_w4a16(d, blob, x, a.m, c, ws, tuning)
+    else:
+        t, e, k_top = a.m, a.experts, a.topk
+        q, s, _ = synth.w4a16_weights(a.n, a.k, 128, False, seed=3000, experts=e)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, 0, e)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev)
+        logits = synth.router_logits(t, e, seed=3001).to(dev)
+        x = synth.bf16_normal(t, a.k, seed=3002).to(dev)
+        ids = torch.empty(t, k_top, dtype=torch.int32, device=dev)
+        src = torch.empty(t * k_top, dtype=torch.int32, device=dev)
+        off = torch.empty(e + 1, dtype=torch.int32, device=dev)
+        xs = torch.empty(t * k_top, a.k, dtype=torch.bfloat16, device=dev)
+        c = torch.empty(t * k_top, a.n, dtype=torch.bfloat16, device=dev)
+        pws = torch.zeros(hq.hq_moe_permute_workspace_size(t, k_top, e), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(max(256, hq.hq_workspace_size(d, t * k_top, tuning)), dtype=torch.uint8, device=dev)
+        for _ in range(a.iters):
+            hq.hq_moe_topk(logits, t, e, k_top, ids)
+            hq.hq_moe_permute(ids, t, k_top, e, src, off, pws, a=x, hidden=a.k, a_sorted=xs)
+            hq.hq_grouped_gemm_moe(d, blob, xs, off, t * k_top, c, ws, tuning)
+        st = hq.hq_check_device_status(pws)
+        if st != hq.HQ_OK:
+            print("device status", hq.status_string(st))
+            return 1
+    torch.cuda.synchronize()
+    st = hq.hq_check_device_status(ws)
+    if st != hq.HQ_OK:
+        print("device status", hq.status_string(st))
+        return 1
+    print("ok")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -44,8 +44,7 @@ def w4a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
     assert k % group == 0 and k % 8 == 0
     g = _gen(seed)
     lead = () if experts is None else (experts,)
-    qweight = torch.randint(-(2 ** 31), 2 ** 31, lead + (n, k // 8), generator=g,
-                            dtype=torch.int64).to(torch.int32)
+    qweight = torch.randint(-(2 ** 31), 2 ** 31, lead + (n, k // 8), generator=g, dtype=torch.int32)
     scales = (0.002 + 0.01 * torch.randn(lead + (n, k // group), generator=g).abs()).to(torch.float16)
     zeros = None
     if asym:

@@ -1,0 +1,125 @@
+"""GPU parity of the block-scaled 4-bit GEMMs (through the C ABI) against
+the fp64 oracle: W4A8-MXFP4 (E2M1 weights, E8M0 per 32 K, E4M3 activations
+with per-token scale) and W4A4 NVFP4 (E2M1, E4M3 per 16 K, fp32 tensor
+scales).  Full outputs on small shapes spanning tiles and ragged tails;
+sampled rows and columns at the full workload sizes."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import check_gemm, tile_rows, workspace
+from oracle import formats as F
+from oracle import gemm as G
+from quantized_gemm_bit_b200 import hq, synth
+from quantized_gemm_bit_b200.build import build
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    build()
+    torch.cuda.init()
+
+
+# ---------------------------------------------------------------- MXFP4 x FP8
+
+def mx_case(m, n, k, seed):
+    codes, e8 = synth.mxfp4_weights(n, k, seed=seed)
+    aq, asc = synth.fp8_activations(m, k, seed=seed + 1)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, n, k, 32, 0, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(DEV)
+    return d, blob, aq, asc, codes.numpy(), e8.numpy()
+
+
+def mx_run(d, blob, aq, asc, m, tuning=None):
+    c = torch.empty(m, d.n, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, m, tuning))
+    hq.hq_gemm_mxfp4_a8(d, blob, aq.to(DEV), asc.to(DEV), m, c, ws, tuning)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    return c
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 256, 512), (5, 200, 384), (70, 384, 1024), (300, 256, 640)])
+def test_mxfp4_full_output(m, n, k):
+    d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 200 + m)
+    c = mx_run(d, blob, aq, asc, m)
+    ref = G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8)
+    check_gemm(c, ref, k, f"mxfp4 m={m} n={n} k={k}")
+
+
+@pytest.mark.parametrize("tile_m", [16, 32, 64, 128, 256])
+def test_mxfp4_every_token_tile(tile_m):
+    m, n, k = 90, 256, 1024
+    d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 300)
+    c = mx_run(d, blob, aq, asc, m, hq.Tuning(tile_m=tile_m))
+    check_gemm(c, G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8), k, f"mxfp4 tile_m={tile_m}")
+
+
+@pytest.mark.parametrize("m", [16, 256, 4096])
+def test_mxfp4_full_size(m):
+    """W4A8-MXFP4 workload: K = N = 7168, seeds per shape."""
+    n = k = 7168
+    d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 2000 + m)
+    c = mx_run(d, blob, aq, asc, m)
+    rows = tile_rows(m, 128, np.random.default_rng(m))
+    ref = G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8, rows=rows)
+    check_gemm(c[torch.from_numpy(rows).to(DEV)], ref, k, f"mxfp4 full m={m}")
+
+
+# ---------------------------------------------------------------- NVFP4 W4A4
+
+def nv_quant(rows, k, seed):
+    x = synth.bf16_normal(rows, k, seed).float().numpy()
+    codes, sf, g = F.nvfp4_quantize(x)
+    return F.fp4_pack_bytes(codes), sf, g
+
+
+def nv_case(m, n, k, seed):
+    wp, wsf, wg = nv_quant(n, k, seed)
+    ap, asf, ag = nv_quant(m, k, seed + 1)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, n, k, 16, 0, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, wp, wsf, None, float(wg))).to(DEV)
+    return d, blob, (ap, asf, ag), (wp, wsf, wg)
+
+
+def nv_run(d, blob, act, m, tuning=None):
+    ap, asf, ag = act
+    c = torch.empty(m, d.n, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, m, tuning))
+    hq.hq_gemm_nvfp4(d, blob, torch.from_numpy(ap).to(DEV), torch.from_numpy(asf).to(DEV), float(ag), m, c, ws,
+                     tuning)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    return c
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 256, 512), (7, 200, 768), (130, 384, 1024), (300, 128, 256)])
+def test_nvfp4_full_output(m, n, k):
+    d, blob, act, w = nv_case(m, n, k, 400 + m)
+    c = nv_run(d, blob, act, m)
+    ref = G.nvfp4_ref(*act, *w)
+    check_gemm(c, ref, k, f"nvfp4 m={m} n={n} k={k}")
+
+
+@pytest.mark.parametrize("tile_m", [16, 32, 64, 128, 256])
+def test_nvfp4_every_token_tile(tile_m):
+    m, n, k = 200, 256, 1024
+    d, blob, act, w = nv_case(m, n, k, 500)
+    c = nv_run(d, blob, act, m, hq.Tuning(tile_m=tile_m))
+    check_gemm(c, G.nvfp4_ref(*act, *w), k, f"nvfp4 tile_m={tile_m}")
+
+
+@pytest.mark.parametrize("m,n,k", [(8192, 8192, 8192), (16384, 18432, 7168)])
+def test_nvfp4_full_size(m, n, k):
+    """NVFP4 W4A4 large-batch workload, sampled rows and columns."""
+    d, blob, act, w = nv_case(m, n, k, 4000 + (0 if m == 8192 else 1))
+    c = nv_run(d, blob, act, m)
+    rng = np.random.default_rng(m)
+    rows = tile_rows(m, 256, rng, per_tile=1)
+    cols = np.array(sorted({c0 for nt in range(n // 128)
+                            for c0 in (nt * 128, nt * 128 + 127, nt * 128 + int(rng.integers(0, 128)))}))
+    ref = G.nvfp4_ref(*act, *w, rows=rows, cols=cols)
+    got = c[torch.from_numpy(rows).to(DEV)][:, torch.from_numpy(cols).to(DEV)]
+    check_gemm(got, ref, k, f"nvfp4 full m={m} n={n} k={k}")

@@ -57,7 +57,8 @@ def test_tiny_config_full_output():
 
 @pytest.mark.parametrize("m,n,k,asym", [
     (1, 256, 256, False), (7, 200, 384, True), (17, 384, 1152, False), (100, 128, 512, True),
-    (129, 640, 640, False), (300, 256, 768, True), (513, 384, 256, False),
+    (129, 640, 640, False), (300, 256, 768, True), (513, 384, 256, False), (5, 640, 384, True),
+    (40, 1152, 2560, False),
 ])
 def test_ragged_shapes_full_output(m, n, k, asym):
     d, blob, a, (q, s, z) = make_case(m, n, k, asym, 100 + m)
