@@ -178,20 +178,21 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   int tile, nt, row0, rows, ks0, ks1, partial, slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      uint32_t it = 0;
-      bool ok = true;
-      for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
-        for (int ks = ks0; ks < ks1; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (!hq_wait(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
-            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-            ok = false;
-            break;
-          }
+    // ------------------------------------------------------------ producer (whole warp, one lane issues)
+    const bool leader = elect_one();
+    const uint64_t pol_w = policy_evict_first();
+    uint32_t it = 0;
+    bool ok = true;
+    for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
+      for (int ks = ks0; ks < ks1; ++ks, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        if (leader) {
           mbar_arrive_expect_tx(&full[s], kTx);
           // weights: K coordinate in elements (MXFP4 unpacking type) or bytes (NVFP4)
           tma_load_2d(sA(s), &tmap_w, FMT == kNV ? ks * 128 : ks * C::kKStage, nt * kBsTileN, &full[s]);
@@ -201,42 +202,44 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           bulk_g2s(sSfa(s), src, C::kSfa, &full[s], pol_w);
           if (FMT == kNV) tma_load_2d(sSfbRaw(s), &tmap_sfb, ks * 16, row0, &full[s]);
         }
-      }
-      if (!ok) {
-        const uint32_t first = it > (uint32_t)S ? it - S : 0;
-        for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % S], (j / S) & 1, p.wait_ns, nullptr);
+        __syncwarp();
       }
     }
+    if (!ok && lane == 0) {
+      const uint32_t first = it > (uint32_t)S ? it - S : 0;
+      for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % S], (j / S) & 1, p.wait_ns, nullptr);
+    }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t it = 0, uc = 0;
-      bool ok = true;
-      for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
-           ++idx, ++uc) {
-        const int ab = uc % ACC;
-        const uint32_t aph = (uc / ACC) & 1;
-        if (!hq_wait(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
-          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+    // ------------------------------------------------------------ MMA issuer (whole warp, one fixed lane issues)
+    const bool leader = elect_one();
+    uint32_t it = 0, uc = 0;
+    bool ok = true;
+    for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
+         ++idx, ++uc) {
+      const int ab = uc % ACC;
+      const uint32_t aph = (uc / ACC) & 1;
+      if (!hq_wait_warp(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
+        if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + ab * NTOK;
+      for (int ks = ks0; ks < ks1; ++ks, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        bool got = hq_wait_warp(&full[s], ph, p.wait_ns, s_abort);
+        if (got && FMT == kNV) got = hq_wait_warp(&sfb_ready[s], ph, p.wait_ns, s_abort);
+        if (!got) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * NTOK;
-        for (int ks = ks0; ks < ks1; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          bool got = hq_wait(&full[s], ph, p.wait_ns, s_abort);
-          if (got && FMT == kNV) got = hq_wait(&sfb_ready[s], ph, p.wait_ns, s_abort);
-          if (!got) {
-            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sA(s));
-          const uint32_t b_base = smem_u32(sB(s));
-          const uint32_t sf_col = C::kSfBase + s * C::kSfSlot;
+        const uint32_t a_base = smem_u32(sA(s));
+        const uint32_t b_base = smem_u32(sB(s));
+        const uint32_t sf_col = C::kSfBase + s * C::kSfSlot;
+        if (leader) {
           if (FMT == kNV) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -263,12 +266,17 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           }
           tc_commit(&empty[s]);
         }
-        if (!ok) break;
-        tc_commit(&acc_full[ab]);
+        __syncwarp();
       }
+      if (!ok) break;
+      if (leader) tc_commit(&acc_full[ab]);
+      __syncwarp();
+    }
+    if (leader) {
       tc_commit(drain);
       hq_wait(drain, 0, p.wait_ns, nullptr);
     }
+    __syncwarp();
   } else if (warp == 3) {
     // ------------------------------------------------------------ NVFP4 activation-scale reorder
     if (FMT == kNV) {

@@ -20,6 +20,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 }
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
+
+// One lane of a converged warp (the same lane every time for a full warp).
+// Single-thread issue roles (TMA, tcgen05.mma) run their loops on the whole
+// warp and issue from the elected lane, so addresses and descriptors stay
+// warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
 // ---------------------------------------------------------------- mbarrier
@@ -62,6 +76,13 @@ __device__ __forceinline__ bool hq_wait(uint64_t* bar, uint32_t parity, uint64_t
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
+}
+
+// Bounded wait by every lane of a warp; the verdict of lane 0 is returned to
+// all lanes so the warp never diverges on it.
+__device__ __forceinline__ bool hq_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
+  const bool ok = hq_wait(bar, parity, limit_ns, abort);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 // ---------------------------------------------------------------- copies

@@ -279,61 +279,66 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto acc_col = [](int b) -> uint32_t { return (uint32_t)(64 * TS + b * NTOK); };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_last();
-      uint32_t it = 0;
-      bool ok = true;
-      Unit x;
-      for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
-        const uint8_t* wbase =
-            p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
-        for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
-          const int s = it % SS;
-          const uint32_t ph = (it / SS) & 1;
-          if (!hq_wait(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
-            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-            ok = false;
-            break;
-          }
+    // ------------------------------------------------------------ producer (whole warp, elected lane issues)
+    const bool leader = elect_one();
+    const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_last();
+    uint32_t it = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      const uint8_t* wbase =
+          p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
+      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
+        const int s = it % SS;
+        const uint32_t ph = (it / SS) & 1;
+        if (!hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        if (leader) {
           mbar_arrive_expect_tx(&full[s], (uint32_t)p.rec_bytes + kATile);
           bulk_g2s(sR + s * kRecMax, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)p.rec_bytes, &full[s], pol_w);
           tma_load_2d(sA + s * kATile, &tmap_a, kb * kBlockK, x.row0, &full[s]);
           tma_load_2d(sA + s * kATile + NTOK * 128, &tmap_a, kb * kBlockK + 64, x.row0, &full[s]);
         }
-      }
-      if (!ok) {
-        // let every copy already issued land before the CTA exits
-        const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
-        for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
+        __syncwarp();
       }
     }
+    if (!ok && lane == 0) {
+      // let every copy already issued land before the CTA exits
+      const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
+      for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
+    }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t it = 0, uc = 0;
-      bool ok = true;
-      Unit x;
-      for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
-        const int ab = uc % ACC;
-        const uint32_t aph = (uc / ACC) & 1;
-        if (!hq_wait(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
-          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+    // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
+    // one lane, fixed for the whole kernel, issues every MMA and commit: a
+    // commit tracks the tcgen05 operations of the thread that issues it
+    const bool leader = elect_one();
+    uint32_t it = 0, uc = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
+      const int ab = uc % ACC;
+      const uint32_t aph = (uc / ACC) & 1;
+      if (!hq_wait_warp(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
+        if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc_col(ab);
+      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
+        const int s = it % SS, t = it % TS;
+        const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
+        if (!hq_wait_warp(&aready[t], ph_t, p.wait_ns, s_abort) || !hq_wait_warp(&full[s], ph_s, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc_col(ab);
-        for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
-          const int s = it % SS, t = it % TS;
-          const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
-          if (!hq_wait(&aready[t], ph_t, p.wait_ns, s_abort) || !hq_wait(&full[s], ph_s, p.wait_ns, s_abort)) {
-            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t b_base = smem_u32(sA + s * kATile);
+        const uint32_t b_base = smem_u32(sA + s * kATile);
+        if (leader) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint64_t bdesc = smem_desc_sw128(b_base + (j >> 2) * (NTOK * 128) + (j & 3) * 32);
@@ -342,13 +347,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(&empty[s]);
           tc_commit(&afree[t]);
         }
-        if (!ok) break;
-        tc_commit(&acc_full[ab]);
+        __syncwarp();
       }
-      // make sure no MMA is still running when TMEM is released
+      if (!ok) break;
+      if (leader) tc_commit(&acc_full[ab]);
+      __syncwarp();
+    }
+    // make sure no MMA is still running when TMEM is released
+    if (leader) {
       tc_commit(drain);
       hq_wait(drain, 0, p.wait_ns, nullptr);
     }
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dequantize (+ epilogue in warps 4-7)
     const uint32_t q = warp & 3;
@@ -508,38 +518,40 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
     return cfg;
   }
   // Whole tiles on persistent CTAs (no partial sums) when they fill the SMs
-  // well; the token tile may shrink (down to 64) to make more tiles.
-  // Otherwise stream-K with at most 64 tokens per tile, so the partial sums
-  // of a split tile stay small: every CTA gets an equal share of the
-  // (tile, k-block) space, at least 4 k-blocks each.
-  const bool fixed_tile = t && t->tile_m;
+  // well (a 256-token tile may drop to 128 for that).  Otherwise the K range
+  // is shared: large token tiles (big partial sums) split every tile into
+  // the same number of parts; small ones use stream-K over all SMs (every
+  // CTA an equal share of the (tile, k-block) space, >= 4 k-blocks each).
   auto dp_eff = [&](int nt) {
     const long long tl = dense_tiles(d, m, nt);
     const long long waves = (tl + dev.num_sms - 1) / dev.num_sms;
     return (double)tl / (double)(waves * dev.num_sms);
   };
+  const long long kbs = d.k / kBlockK;
   if (t && t->split_k > 0) {
     // explicit request: `split_k` CTAs per tile
     const long long tiles = dense_tiles(d, m, ntok);
     cfg.ntok = ntok;
     cfg.splits = t->split_k;
-    cfg.grid = (int)std::max<long long>(1, std::min<long long>(tiles * t->split_k, tiles * (d.k / kBlockK)));
+    cfg.grid = (int)std::max<long long>(1, std::min<long long>(tiles * t->split_k, tiles * kbs));
     return cfg;
   }
-  for (int nt = ntok; nt >= (fixed_tile ? ntok : std::min(ntok, 64)); nt /= 2) {
-    if (dp_eff(nt) >= 0.85) {
-      cfg.ntok = nt;
-      cfg.splits = 0;  // data parallel
-      cfg.grid = (int)std::min<long long>(dev.num_sms, dense_tiles(d, m, nt));
-      return cfg;
-    }
-    if (nt == 16) break;
-  }
-  if (!fixed_tile) ntok = std::min(ntok, 64);
+  const bool fixed_tile = t && t->tile_m;
+  if (!fixed_tile && ntok == 256 && dp_eff(256) < 0.85 && dp_eff(128) >= 0.85) ntok = 128;
   cfg.ntok = ntok;
-  const long long iters = (long long)dense_tiles(d, m, ntok) * (d.k / kBlockK);
-  long long grid = std::min<long long>(dev.num_sms, std::max<long long>(1, iters / 4));
-  cfg.grid = (int)std::max<long long>(1, grid);
+  const long long tiles = dense_tiles(d, m, ntok);
+  if (dp_eff(ntok) >= 0.85) {
+    cfg.splits = 0;  // data parallel
+    cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
+    return cfg;
+  }
+  if (ntok >= 128 && tiles * 2 <= dev.num_sms) {
+    cfg.splits = (int)(dev.num_sms / tiles);
+    cfg.grid = (int)std::min<long long>(tiles * cfg.splits, tiles * kbs);
+    return cfg;
+  }
+  cfg.splits = 1;
+  cfg.grid = (int)std::max<long long>(1, std::min<long long>(dev.num_sms, tiles * kbs / 4));
   return cfg;
 }
 
