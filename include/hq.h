@@ -237,6 +237,26 @@ hq_status hq_check_device_status(void* ws_dev, hq_stream_t stream);
  * word and returns normally.  limit_ns must be <= 100 ms. */
 hq_status hq_debug_timeout_probe(void* ws_dev, uint64_t limit_ns, hq_stream_t stream);
 
+/* Dense W4A16 GEMM that allocates nothing (no counterpart in the method's
+ * pages; an addition of this library).  For callers that cannot allocate
+ * device memory where they run the layer -- an engine that plans all memory
+ * up front and forbids allocation on its serving path, or code running inside
+ * another owner's memory pool -- the scratch hq_gemm_w4a16 takes as a
+ * workspace (split-K tile counters and fp32 partial sums) lives here in one
+ * fixed 16 MiB array inside the library, present on every device that loads
+ * it until the process exits.
+ *   Same arguments and result as hq_gemm_w4a16, without ws_dev / ws_bytes.
+ *   A launch plan needing more than 16 MiB of scratch is refused with
+ *   HQ_ERR_WORKSPACE_TOO_SMALL before anything runs (a smaller tile_m in
+ *   `t` needs less).  Each call clears the part of the array that must start
+ *   at zero on its own stream.  All calls share the array: calls that may
+ *   overlap on the GPU (unordered streams) race; calls ordered on one stream
+ *   are safe.  The first call on a device looks up the array's device
+ *   address (cudaGetSymbolAddress), so make it before any stream capture.
+ *   Device-side errors of this entry point are not reported separately. */
+hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* packed_w_dev, const void* a_dev, int32_t m,
+                               void* c_dev, const hq_tuning* t, hq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,7 +41,7 @@ EXPORTS = (
     "hq_workspace_size", "hq_gemm_w4a16", "hq_gemm_mxfp4_a8", "hq_gemm_nvfp4", "hq_quantize_fp8_rows",
     "hq_quantize_nvfp4_workspace_size", "hq_quantize_nvfp4", "hq_moe_topk",
     "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_check_device_status",
-    "hq_debug_timeout_probe",
+    "hq_debug_timeout_probe", "hq_gemm_w4a16_static",
 )
 
 
@@ -94,6 +94,7 @@ def lib():
             "hq_grouped_gemm_moe": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
             "hq_check_device_status": (st, [vp, vp]),
             "hq_debug_timeout_probe": (st, [vp, ctypes.c_uint64, vp]),
+            "hq_gemm_w4a16_static": (st, [dp, vp, vp, i32, vp, tp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -239,3 +240,11 @@ def hq_check_device_status(ws, stream=None):
 
 def hq_debug_timeout_probe(ws, limit_ns, stream=None):
     _check(lib().hq_debug_timeout_probe(_ptr(ws), int(limit_ns), _stream(stream)), "hq_debug_timeout_probe")
+
+
+def hq_gemm_w4a16_static(desc, packed_w, a, m, c, tuning=None, stream=None):
+    """hq_gemm_w4a16 for callers that cannot allocate device memory: the
+    split-K scratch lives in a fixed array inside the library (see
+    include/hq.h for its size and sharing rules)."""
+    _check(lib().hq_gemm_w4a16_static(ctypes.byref(desc), _ptr(packed_w), _ptr(a), int(m), _ptr(c),
+                                      _tuning(tuning), _stream(stream)), "hq_gemm_w4a16_static")
