@@ -86,11 +86,27 @@ struct BsParams {
   int m, n, k;
   int n_tiles, k_stages;
   int sf_groups;             // 512-byte scale chunks per weight tile (whole K)
+  int m_tiles;
+  int data_parallel;         // whole tiles per unit, no partial sums
 };
 
 template <int FMT, int NTOK>
 __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, int& nt, int& row0, int& rows,
                                         int& ks0, int& ks1, int& partial, int& slot) {
+  if (p.data_parallel) {
+    const long long t = (long long)blockIdx.x + (long long)idx * gridDim.x;
+    if (t >= (long long)p.m_tiles * p.n_tiles) return false;
+    const int mt = (int)(t / p.n_tiles);
+    tile = (int)t;
+    nt = (int)(t - (long long)mt * p.n_tiles);
+    row0 = mt * NTOK;
+    rows = min(NTOK, p.m - row0);
+    ks0 = 0;
+    ks1 = p.k_stages;
+    partial = 0;
+    slot = 0;
+    return true;
+  }
   const long long T = p.total_iters, G = gridDim.x, i = blockIdx.x;
   const long long beg = sk_start(i, T, G), end = sk_start(i + 1, T, G);
   const long long kst = p.k_stages;
@@ -373,14 +389,28 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         is_last = __shfl_sync(0xffffffffu, is_last, 0);
         if (is_last) {
           __threadfence();
-          for (int j = 0; j < rows; ++j) {
-            float acc = 0.f;
+          for (int j0 = 0; j0 < rows; j0 += 16) {
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
             for (long long ci = first; ci <= last; ++ci) {
               const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
-              acc += __ldcg(p.partials + (((size_t)ci * 2 + sl) * NTOK + j) * kBsTileN + r);
+              const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kBsTileN + r;
+              float v[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + (size_t)j * kBsTileN);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[j] += v[j];
             }
-            const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + j);
-            if (n_ok) p.c[(size_t)(row0 + j) * p.n + n] = __float2bfloat16_rn(acc * sc);
+            if (n_ok) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                if (j0 + j < rows) {
+                  const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + j0 + j);
+                  p.c[(size_t)(row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(acc[j] * sc);
+                }
+              }
+            }
           }
           if (lane == 0) p.counters[tile * 4 + q] = 0;
         }
@@ -421,16 +451,43 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   BsConfig cfg{};
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
-  cfg.ntok = ntok;
   const int kstage = d.fmt == HQ_FMT_NVFP4 ? 256 : 128;
-  const long long iters = (long long)bs_tiles(d, m, ntok) * (d.k / kstage);
-  long long grid = std::min<long long>(dev.num_sms, std::max<long long>(1, iters / 4));
-  if (t && t->split_k > 0) grid = std::min<long long>((long long)bs_tiles(d, m, ntok) * t->split_k, iters);
-  cfg.grid = (int)std::max<long long>(1, grid);
+  const long long ks = d.k / kstage;
+  auto dp_eff = [&](int nt) {
+    const long long tl = bs_tiles(d, m, nt);
+    const long long waves = (tl + dev.num_sms - 1) / dev.num_sms;
+    return (double)tl / (double)(waves * dev.num_sms);
+  };
+  if (t && t->split_k > 0) {
+    cfg.ntok = ntok;
+    cfg.splits = t->split_k;
+    cfg.grid = (int)std::max<long long>(1, std::min<long long>((long long)bs_tiles(d, m, ntok) * t->split_k,
+                                                                (long long)bs_tiles(d, m, ntok) * ks));
+    return cfg;
+  }
+  // same policy as the W4A16 kernel: whole tiles when they fill the SMs,
+  // an even K split for large token tiles, stream-K otherwise
+  const bool fixed_tile = t && t->tile_m;
+  if (!fixed_tile && ntok == 256 && dp_eff(256) < 0.85 && dp_eff(128) >= 0.85) ntok = 128;
+  cfg.ntok = ntok;
+  const long long tiles = bs_tiles(d, m, ntok);
+  if (dp_eff(ntok) >= 0.85) {
+    cfg.splits = 0;
+    cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
+    return cfg;
+  }
+  if (ntok >= 128 && tiles * 2 <= dev.num_sms) {
+    cfg.splits = (int)(dev.num_sms / tiles);
+    cfg.grid = (int)std::min<long long>(tiles * cfg.splits, tiles * ks);
+    return cfg;
+  }
+  cfg.splits = 1;
+  cfg.grid = (int)std::max<long long>(1, std::min<long long>(dev.num_sms, tiles * ks / 4));
   return cfg;
 }
 
 size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg) {
+  if (cfg.splits == 0) return sizeof(WsHeader);
   const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
   return sizeof(WsHeader) + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256 +
          (size_t)cfg.grid * 2 * cfg.ntok * kBsTileN * sizeof(float);
@@ -459,6 +516,8 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.k_stages = d.k / (nv ? 256 : 128);
   const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
   p.total_iters = (long long)tiles * p.k_stages;
+  p.m_tiles = (m + cfg.ntok - 1) / cfg.ntok;
+  p.data_parallel = cfg.splits == 0 ? 1 : 0;
   uint8_t* base = static_cast<uint8_t*>(ws) + sizeof(WsHeader);
   p.counters = reinterpret_cast<int32_t*>(base);
   p.partials = reinterpret_cast<float*>(base + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256);

@@ -48,6 +48,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
 // Block-scaled 4-bit GEMMs (MXFP4 weights x E4M3 activations; NVFP4 x NVFP4).
 struct BsConfig {
   int ntok;
+  int splits;   // 0: whole tiles per CTA (no partial sums)
   int grid;
 };
 BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t);

@@ -142,17 +142,22 @@ __device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix,
 
 template <int NTOK>
 struct Cfg {
-  static constexpr int kATile = NTOK * 256;                 // two 64-wide K boxes of NTOK rows x 128 B
-  static constexpr int kSmemStages = NTOK == 16 ? 12 : NTOK == 32 ? 9 : NTOK == 64 ? 6 : NTOK == 128 ? 4 : 3;
-  static constexpr int kTmemStages = NTOK <= 64 ? 6 : NTOK == 128 ? 4 : 3;   // 64 TMEM columns each
+  // records (128-K blocks) per pipeline stage: two for the small token tiles,
+  // whose MMAs are cheap, so the per-stage waits and commits are amortized
+  static constexpr int kKps = NTOK <= 64 ? 2 : 1;
+  static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
+  static constexpr int kATile = kKps * kABlock;
+  static constexpr int kRecs = kKps * kRecMax;
+  static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 4 : 3;
+  static constexpr int kTmemStages = NTOK <= 64 ? 3 : NTOK == 128 ? 4 : 3;   // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
   // dequantizing warpgroups; with one accumulator (256 tokens) the epilogue
   // warpgroup dequantizes too, since the MMA waits for it anyway
   static constexpr int kDqGroups = NTOK == 128 ? 2 : 3;
   static constexpr int kBarBytes = 512;
-  static constexpr size_t kSmem = (size_t)kSmemStages * (kATile + kRecMax) + 1024 + kBarBytes +
+  static constexpr size_t kSmem = (size_t)kSmemStages * (kATile + kRecs) + 1024 + kBarBytes +
                                   2 * (kMaxExperts + 1) * sizeof(int) + 64;
-  static_assert(64 * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
+  static_assert(64 * kKps * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
   static_assert(kTmemStages % kDqGroups == 0 && kSmemStages % kDqGroups == 0,
                 "every SMEM and TMEM stage must always return to the same dequant group");
   static_assert(8 * (2 * kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
@@ -200,13 +205,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int ACC = C::kAccBufs;
   constexpr int NDQ = C::kDqGroups;
   constexpr int kATile = C::kATile;
+  constexpr int KPS = C::kKps;
+  constexpr int kRecs = C::kRecs;
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                               // SS * kATile (activations, 128-byte swizzle)
-  uint8_t* sR = smem + SS * kATile;                 // SS * kRecMax (packed weight records)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sR + SS * kRecMax);
+  uint8_t* sR = smem + SS * kATile;                 // SS * kRecs (packed weight records)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sR + SS * kRecs);
   uint64_t* empty = full + SS;
   uint64_t* aready = empty + SS;
   uint64_t* afree = aready + TS;
@@ -275,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *s_tmem;
   const int total_grouped = *s_total;
 
-  auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * 64); };
-  auto acc_col = [](int b) -> uint32_t { return (uint32_t)(64 * TS + b * NTOK); };
+  auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * 64 * KPS); };
+  auto acc_col = [](int b) -> uint32_t { return (uint32_t)(64 * KPS * TS + b * NTOK); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp, elected lane issues)
@@ -288,19 +295,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
       const uint8_t* wbase =
           p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
-      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS;
         const uint32_t ph = (it / SS) & 1;
+        const int nrec = min(KPS, x.kb1 - kb);
         if (!hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         if (leader) {
-          mbar_arrive_expect_tx(&full[s], (uint32_t)p.rec_bytes + kATile);
-          bulk_g2s(sR + s * kRecMax, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)p.rec_bytes, &full[s], pol_w);
-          tma_load_2d(sA + s * kATile, &tmap_a, kb * kBlockK, x.row0, &full[s]);
-          tma_load_2d(sA + s * kATile + NTOK * 128, &tmap_a, kb * kBlockK + 64, x.row0, &full[s]);
+          mbar_arrive_expect_tx(&full[s], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+          for (int r = 0; r < nrec; ++r) {
+            bulk_g2s(sR + s * kRecs + r * kRecMax, wbase + (uint64_t)(kb + r) * p.rec_bytes, (uint32_t)p.rec_bytes,
+                     &full[s], pol_w);
+            uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
+            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, &full[s]);
+            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, &full[s]);
+          }
         }
         __syncwarp();
       }
@@ -328,21 +340,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc_col(ab);
-      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, t = it % TS;
         const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
+        const int nrec = min(KPS, x.kb1 - kb);
         if (!hq_wait_warp(&aready[t], ph_t, p.wait_ns, s_abort) || !hq_wait_warp(&full[s], ph_s, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t b_base = smem_u32(sA + s * kATile);
         if (leader) {
+          // descriptors advance by constants: 32 B per 16-K step inside a
+          // 128-byte swizzle row, one box (NTOK rows) per 64 K
+          const uint64_t b0 = smem_desc_sw128(smem_u32(sA + s * kATile));
+          const uint32_t a0 = tmem_base + a_col(t);
+          for (int r = 0; r < nrec; ++r) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint64_t bdesc = smem_desc_sw128(b_base + (j >> 2) * (NTOK * 128) + (j & 3) * 32);
-            mma_bf16_ts(d_tmem, tmem_base + a_col(t) + j * 8, bdesc, kIdesc, (kb > x.kb0 || j > 0) ? 1u : 0u);
+            for (int j = 0; j < 8; ++j) {
+              const uint64_t bdesc = b0 + (uint64_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
+              mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, kIdesc, (kb + r > x.kb0 || j > 0) ? 1u : 0u);
+            }
           }
           tc_commit(&empty[s]);
           tc_commit(&afree[t]);
@@ -371,8 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     Unit x;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
-      for (int kb = x.kb0; kb < x.kb1; ++kb, ++it) {
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         if (!does_dq || (int)(it % NDQ) != dq) continue;
+        const int nrec = min(KPS, x.kb1 - kb);
         const int s = it % SS, t = it % TS;
         const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
         // Both rings are multiples of NDQ deep, so SMEM stage s and TMEM
@@ -385,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        dequant_block(sR + s * kRecMax, r, p.has_zero, tmem_base + lane_addr + a_col(t));
+        for (int rr = 0; rr < nrec; ++rr)
+          dequant_block(sR + s * kRecs + rr * kRecMax, r, p.has_zero, tmem_base + lane_addr + a_col(t) + rr * 64);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
