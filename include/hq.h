@@ -92,13 +92,19 @@ typedef struct {
 /* Execution choices (the Tuning Config of [P-fa2] paragraph 3).  Pass NULL
  * to let the library's heuristic choose; a zero field also means "choose".
  *   tile_m   : token tile (the MMA N extent): 16, 32, 64, 128 or 256
+ *              (hq_grouped_gemm_moe: 16, 32, 64 or 128)
  *   tile_n   : weight rows per tile: 128 (the only value)
  *   tile_k   : K per pipeline stage: 128 (fixed by the packed layout)
  *   stages   : 0 (the pipeline depth is fixed per token tile)
  *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
  *              splits the whole iteration space evenly when 0)
  *   cta_group: 1 (one SM per MMA)
- *   variant  : 0                                                             */
+ *   variant  : W4A16 / grouped MoE: 0 = token tiles of up to 64 feed the
+ *              exact integers (q - z) to the tensor core and apply each
+ *              group's scale to the fp32 group sums; larger tiles rescale
+ *              the weights to bf16, w = bf16((q - z) * s), and accumulate
+ *              across K in fp32.  1 = the bf16-rescaled weights for every
+ *              tile.  Block-scaled GEMMs: 0.                              */
 typedef struct {
   int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;
 } hq_tuning;

@@ -27,8 +27,11 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 struct W4Config {
   int ntok;     // token tile (MMA N)
   int stages;   // unused (pipeline depth is fixed per token tile)
-  int splits;   // unused (dense mode is stream-K over `grid` CTAs)
+  int splits;   // 0: data parallel (whole tiles); else stream-K / split K
   int grid;     // CTAs
+  int variant;  // 0: exact (q - z) weights + per-group fp32 scaling for tiles
+                //    of <= 64 tokens, bf16-rescaled weights above;
+                // 1: bf16-rescaled weights for every tile
 };
 
 struct DeviceInfo {

@@ -33,112 +33,15 @@
 
 #include "hq_internal.h"
 #include "ptx.cuh"
+#include "w4a16_common.cuh"
 
 namespace hq {
 
+using namespace w4;
+
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kRecMax = 8576;        // packed record with zero points
-constexpr int kMaxExperts = 1024;
-
-struct W4Params {
-  const uint8_t* packed;             // expert 0, record (0, 0)
-  __nv_bfloat16* c;
-  const int32_t* expert_offsets;     // grouped mode only
-  float* partials;                   // dense: [grid][2][NTOK*128] fp32
-  int32_t* counters;                 // dense: [tiles][4]
-  uint32_t* err;
-  uint64_t expert_bytes;
-  uint64_t wait_ns;
-  long long total_iters;             // dense: tiles * k_blocks
-  int m;                             // dense: rows of A; grouped: total sorted rows
-  int n;                             // output columns
-  int n_tiles, k_blocks, m_tiles;
-  int num_experts;
-  int has_zero;
-  int rec_bytes;
-  int grouped;
-  int weights_once;                  // each weight tile is read by one CTA
-  int data_parallel;                 // dense: whole tiles per unit, no partials
-};
-
-// One unit of work: a K range of one (expert, token tile, weight tile).
-struct Unit {
-  int expert;
-  int nt;        // weight tile
-  int row0;      // first row of A / C
-  int rows;      // valid rows in this tile (<= NTOK)
-  int kb0, kb1;  // k-block range
-  int tile;      // dense tile index
-  int partial;   // 1: other CTAs own the rest of this tile's K range
-  int slot;      // partial slot of this CTA (0: its first unit, 1: its last)
-};
-
-template <int NTOK>
-__device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix, const int* s_off, int total_grouped,
-                                         int idx, Unit& x) {
-  if (!p.grouped && p.data_parallel) {
-    // whole tiles, strided over the persistent CTAs
-    const long long tile = (long long)blockIdx.x + (long long)idx * gridDim.x;
-    if (tile >= (long long)p.m_tiles * p.n_tiles) return false;
-    const int mt = (int)(tile / p.n_tiles);
-    x.tile = (int)tile;
-    x.nt = (int)(tile - (long long)mt * p.n_tiles);
-    x.expert = 0;
-    x.row0 = mt * NTOK;
-    x.rows = min(NTOK, p.m - x.row0);
-    x.kb0 = 0;
-    x.kb1 = p.k_blocks;
-    x.partial = 0;
-    x.slot = 0;
-    return true;
-  }
-  if (!p.grouped) {
-    const long long T = p.total_iters, G = gridDim.x, i = blockIdx.x;
-    const long long beg = sk_start(i, T, G), end = sk_start(i + 1, T, G);
-    const long long kb = p.k_blocks;
-    const long long tile = beg / kb + idx;
-    const long long x0 = idx == 0 ? beg : tile * kb;
-    if (x0 >= end) return false;
-    const long long x1 = min(end, (tile + 1) * kb);
-    const int mt = (int)(tile / p.n_tiles);
-    x.tile = (int)tile;
-    x.nt = (int)(tile - (long long)mt * p.n_tiles);
-    x.expert = 0;
-    x.row0 = mt * NTOK;
-    x.rows = min(NTOK, p.m - x.row0);
-    x.kb0 = (int)(x0 - tile * kb);
-    x.kb1 = (int)(x1 - tile * kb);
-    x.partial = (x.kb0 != 0 || x.kb1 != p.k_blocks) ? 1 : 0;
-    x.slot = idx == 0 ? 0 : 1;
-    return true;
-  }
-  const int u = blockIdx.x + idx * gridDim.x;
-  if (u >= total_grouped) return false;
-  // find the expert e with prefix[e] <= u < prefix[e+1] (empty experts share
-  // their prefix with the next one, so the largest such e has rows)
-  int lo = 0, hi = p.num_experts;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (s_prefix[mid] <= u) lo = mid; else hi = mid;
-  }
-  const int e = lo;
-  const int rows_e = s_off[e + 1] - s_off[e];
-  const int mtiles = (rows_e + NTOK - 1) / NTOK;
-  const int local = u - s_prefix[e];
-  const int mt = local % mtiles;
-  x.nt = local / mtiles;
-  x.expert = e;
-  x.row0 = s_off[e] + mt * NTOK;
-  x.rows = min(NTOK, s_off[e + 1] - x.row0);
-  x.kb0 = 0;
-  x.kb1 = p.k_blocks;
-  x.tile = 0;
-  x.partial = 0;
-  x.slot = 0;
-  return true;
-}
+constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 
 template <int NTOK>
 struct Cfg {
@@ -148,19 +51,31 @@ struct Cfg {
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
   static constexpr int kRecs = kKps * kRecMax;
-  static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 4 : 3;
-  static constexpr int kTmemStages = NTOK <= 64 ? 3 : NTOK == 128 ? 4 : 3;   // 64 * kKps TMEM columns each
+  static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;    // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
-  // dequantizing warpgroups; with one accumulator (256 tokens) the epilogue
-  // warpgroup dequantizes too, since the MMA waits for it anyway
-  static constexpr int kDqGroups = NTOK == 128 ? 2 : 3;
+  // dequantizing warpgroups: the epilogue warpgroup joins for small tiles
+  static constexpr int kDqGroups = NTOK <= 64 ? 3 : 2;
+  // full barriers, one per (SMEM stage, dequant group): iteration `it`
+  // uses barrier (it % SS, it % NDQ), so every waiter sees each of its
+  // barrier's phases in order whatever the ring depth
+  static constexpr int kFullBars = kSmemStages * kDqGroups;
+  static constexpr int kFullPeriod = kSmemStages / cgcd(kSmemStages, kDqGroups) * kDqGroups;  // lcm
+  // warp-local transpose buffer for 16-byte output stores (aliases the
+  // expert tables at 256 tokens, a dense-only tile)
+  static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
   static constexpr int kBarBytes = 512;
-  static constexpr size_t kSmem = (size_t)kSmemStages * (kATile + kRecs) + 1024 + kBarBytes +
-                                  2 * (kMaxExperts + 1) * sizeof(int) + 64;
+  // byte offsets from the 1024-aligned base of dynamic shared memory
+  static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
+  static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
+  static constexpr size_t kScrOff = (kTabOff + 2 * (kMaxExperts + 1) * sizeof(int) + 127) / 128 * 128;
+  static constexpr size_t kSmem = 1024 + kScrOff + kEpiScratch;
+  static_assert(kABlock % 1024 == 0 && kRecMax % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
+  static_assert(kEpiScratch != 0 || 2 * (kMaxExperts + 1) * sizeof(int) >= 4 * 2048, "aliased scratch size");
+  static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(64 * kKps * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
-  static_assert(kTmemStages % kDqGroups == 0 && kSmemStages % kDqGroups == 0,
-                "every SMEM and TMEM stage must always return to the same dequant group");
-  static_assert(8 * (2 * kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
+  static_assert(kTmemStages % kDqGroups == 0, "every TMEM stage must always return to the same dequant group");
+  static_assert(8 * (kFullBars + kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
 };
 
 // Dequantize one 128-K block of the packed record for TMEM stage t: thread
@@ -213,8 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                               // SS * kATile (activations, 128-byte swizzle)
   uint8_t* sR = smem + SS * kATile;                 // SS * kRecs (packed weight records)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sR + SS * kRecs);
-  uint64_t* empty = full + SS;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + C::kFullBars;
   uint64_t* aready = empty + SS;
   uint64_t* afree = aready + TS;
   uint64_t* acc_full = afree + TS;
@@ -223,17 +138,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort + 1);
-  int* s_prefix = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::kBarBytes);  // [kMaxExperts + 1]
-  int* s_off = s_prefix + (kMaxExperts + 1);                                                   // [kMaxExperts + 1]
+  int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);  // [kMaxExperts + 1]
+  int* s_off = s_prefix + (kMaxExperts + 1);                    // [kMaxExperts + 1]
+  // 16-byte aligned: read back with 16-byte loads
+  uint16_t* epi_scratch = reinterpret_cast<uint16_t*>(smem + (C::kEpiScratch ? C::kScrOff : C::kTabOff));
+  auto full_bar = [&](uint32_t i) { return &full[(i % SS) * NDQ + (i % NDQ)]; };
+  auto full_par = [](uint32_t i) { return (i / C::kFullPeriod) & 1; };
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
+    for (int s = 0; s < SS; ++s) mbar_init(&empty[s], 1);
+    for (int f = 0; f < C::kFullBars; ++f) mbar_init(&full[f], 1);
     for (int t = 0; t < TS; ++t) {
       mbar_init(&aready[t], 4);
       mbar_init(&afree[t], 1);
@@ -253,29 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
 
-  // Grouped mode: per-expert tile prefix sums from the device-resident row
-  // offsets (no host synchronization).
-  if (p.grouped) {
-    const int E = p.num_experts;
-    for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = p.expert_offsets[i];
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int acc = 0;
-      bool bad = s_off[0] != 0 || s_off[E] != p.m;
-      for (int e = 0; e < E; ++e) {
-        s_prefix[e] = acc;
-        int rows = s_off[e + 1] - s_off[e];
-        if (rows < 0) { bad = true; rows = 0; }
-        acc += ((rows + NTOK - 1) / NTOK) * p.n_tiles;
-      }
-      s_prefix[E] = acc;
-      if (bad) {
-        atomicCAS(p.err, 0u, (uint32_t)HQ_ERR_DEVICE_BAD_OFFSETS);
-        acc = 0;
-      }
-      *s_total = acc;
-    }
-  }
+  if (p.grouped) grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -305,13 +200,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (leader) {
-          mbar_arrive_expect_tx(&full[s], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+          uint64_t* fb = full_bar(it);
+          mbar_arrive_expect_tx(fb, (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
           for (int r = 0; r < nrec; ++r) {
             bulk_g2s(sR + s * kRecs + r * kRecMax, wbase + (uint64_t)(kb + r) * p.rec_bytes, (uint32_t)p.rec_bytes,
-                     &full[s], pol_w);
+                     fb, pol_w);
             uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
-            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, &full[s]);
-            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, &full[s]);
+            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, fb);
+            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, fb);
           }
         }
         __syncwarp();
@@ -320,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && lane == 0) {
       // let every copy already issued land before the CTA exits
       const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
-      for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
+      for (uint32_t j = first; j < it; ++j) hq_wait(full_bar(j), full_par(j), p.wait_ns, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
@@ -342,9 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t d_tmem = tmem_base + acc_col(ab);
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, t = it % TS;
-        const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
+        const uint32_t ph_t = (it / TS) & 1;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp(&aready[t], ph_t, p.wait_ns, s_abort) || !hq_wait_warp(&full[s], ph_s, p.wait_ns, s_abort)) {
+        if (!hq_wait_warp(&aready[t], ph_t, p.wait_ns, s_abort) ||
+            !hq_wait_warp(full_bar(it), full_par(it), p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -393,12 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!does_dq || (int)(it % NDQ) != dq) continue;
         const int nrec = min(KPS, x.kb1 - kb);
         const int s = it % SS, t = it % TS;
-        const uint32_t ph_s = (it / SS) & 1, ph_t = (it / TS) & 1;
-        // Both rings are multiples of NDQ deep, so SMEM stage s and TMEM
-        // stage t always come back to this same group: it observes every
-        // phase of the barriers it waits on, one after the other (a parity
-        // wait can only tell adjacent phases apart).
-        if (!hq_wait(&full[s], ph_s, p.wait_ns, s_abort) || !hq_wait(&afree[t], ph_t ^ 1, p.wait_ns, s_abort)) {
+        const uint32_t ph_t = (it / TS) & 1;
+        // The full barrier of (stage, group) and TMEM stage t (TS % NDQ == 0)
+        // only ever serve this group, so it observes every phase of the
+        // barriers it waits on, one after the other (a parity wait can only
+        // tell adjacent phases apart).
+        if (!hq_wait(full_bar(it), full_par(it), p.wait_ns, s_abort) ||
+            !hq_wait(&afree[t], ph_t ^ 1, p.wait_ns, s_abort)) {
           raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -422,71 +320,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int n = x.nt * kTileN + r;
-      const bool n_ok = n < p.n;
       float* part = x.partial ? p.partials + ((size_t)blockIdx.x * 2 + x.slot) * NTOK * kTileN : nullptr;
+      // batched TMEM loads (EB columns), then fp32 partials or bf16 stores
+      constexpr int EB = NTOK >= 32 ? 32 : 16;
+      uint16_t* sc = epi_scratch + q * 1024;
 #pragma unroll 1
-      for (int j0 = 0; j0 < NTOK; j0 += 16) {
-        uint32_t v[16];
-        tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0, v);
+      for (int j0 = 0; j0 < NTOK; j0 += EB) {
+        uint32_t v0[16], v1[16];
+        tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0, v0);
+        if (EB == 32) tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0 + 16, v1);
         tmem_wait_ld();
-        if (x.partial) {
+        float v[EB];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(part + (size_t)(j0 + j) * kTileN + r, __uint_as_float(v[j]));
-        } else if (n_ok) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j0 + j < x.rows)
-              p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(__uint_as_float(v[j]));
-          }
-        }
+        for (int j = 0; j < EB; ++j) v[j] = __uint_as_float(j < 16 ? v0[j] : v1[j - 16]);
+        store_chunk<EB>(p, x, part, (int)q, (int)lane, j0, v, sc);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
-      if (x.partial) {
-        // Each epilogue warp owns 32 rows of the tile and one counter: the
-        // last contributing CTA reduces every partial in CTA order, so the
-        // result does not depend on arrival order (and nobody waits).
-        const long long T = p.total_iters, G = gridDim.x, kbl = p.k_blocks;
-        const long long t0 = (long long)x.tile * kbl;
-        const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kbl - 1, T, G);
-        const int cnt = (int)(last - first + 1);
-        __threadfence();
-        __syncwarp();
-        int is_last = 0;
-        if (lane == 0) {
-          __threadfence();
-          is_last = (atomicAdd(p.counters + x.tile * 4 + q, 1) == cnt - 1);
-          __threadfence();
-        }
-        is_last = __shfl_sync(0xffffffffu, is_last, 0);
-        if (is_last) {
-          __threadfence();
-          // 16 token rows at a time, every contributor's loads in flight
-          // together; the sum runs in contributor order
-          for (int j0 = 0; j0 < x.rows; j0 += 16) {
-            float acc[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-            for (long long ci = first; ci <= last; ++ci) {
-              const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
-              const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kTileN + r;
-              float v[16];
-#pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + (size_t)j * kTileN);
-#pragma unroll
-              for (int j = 0; j < 16; ++j) acc[j] += v[j];
-            }
-            if (n_ok) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (j0 + j < x.rows) p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(acc[j]);
-            }
-          }
-          if (lane == 0) p.counters[x.tile * 4 + q] = 0;  // leave the workspace zeroed
-        }
-      }
+      if (x.partial) sk_fixup<NTOK>(p, x, (int)q, (int)lane);
     }
   }
 
@@ -532,6 +384,7 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   }
   cfg.stages = 0;
   cfg.splits = 1;
+  cfg.variant = t ? t->variant : 0;
   if (grouped) {
     cfg.ntok = ntok;
     cfg.grid = dev.num_sms;
@@ -630,6 +483,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
 
+  if (cfg.variant == 0 && cfg.ntok <= 64) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
   switch (cfg.ntok) {
     case 16: return launch_t<16>(map, p, cfg.grid, stream);
     case 32: return launch_t<32>(map, p, cfg.grid, stream);

@@ -1,0 +1,241 @@
+// Device code shared by the two W4A16 kernels (w4a16.cu: dequantized and
+// rescaled bf16 weights, fp32 accumulation across K in TMEM; w4a16_small.cu:
+// exact (q - z) weights, per-group fp32 rescaling): the kernel parameters,
+// the unit scheduler (data parallel, stream-K, grouped MoE), the grouped
+// tile table built on the device, the output stores and the stream-K fixup.
+//
+// Method: weights are 4-bit codes with a per-group fp16 scale and an optional
+// uint4 zero point, described separately from the execution choices
+// ("Humming: open-source kernel library for quantized inference", summary
+// paragraph 2); w = (q - z) * s.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "hq_internal.h"
+#include "ptx.cuh"
+
+namespace hq {
+namespace w4 {
+
+constexpr int kThreads = 512;
+constexpr int kRecMax = 8576;        // packed record with zero points
+constexpr int kMaxExperts = 1024;
+
+struct W4Params {
+  const uint8_t* packed;             // expert 0, record (0, 0)
+  __nv_bfloat16* c;
+  const int32_t* expert_offsets;     // grouped mode only
+  float* partials;                   // dense: [grid][2][NTOK*128] fp32
+  int32_t* counters;                 // dense: [tiles][4]
+  uint32_t* err;
+  uint64_t expert_bytes;
+  uint64_t wait_ns;
+  long long total_iters;             // dense: tiles * k_blocks
+  int m;                             // dense: rows of A; grouped: total sorted rows
+  int n;                             // output columns
+  int n_tiles, k_blocks, m_tiles;
+  int num_experts;
+  int has_zero;
+  int rec_bytes;
+  int grouped;
+  int weights_once;                  // each weight tile is read by one CTA
+  int data_parallel;                 // dense: whole tiles per unit, no partials
+};
+
+// One unit of work: a K range of one (expert, token tile, weight tile).
+struct Unit {
+  int expert;
+  int nt;        // weight tile
+  int row0;      // first row of A / C
+  int rows;      // valid rows in this tile (<= NTOK)
+  int kb0, kb1;  // k-block range
+  int tile;      // dense tile index
+  int partial;   // 1: other CTAs own the rest of this tile's K range
+  int slot;      // partial slot of this CTA (0: its first unit, 1: its last)
+};
+
+// Unit `idx` of this CTA, or false when it has no more.  Every role walks
+// the same sequence, so no role needs to hear about units from another.
+template <int NTOK>
+__device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix, const int* s_off, int total_grouped,
+                                         int idx, Unit& x) {
+  if (!p.grouped && p.data_parallel) {
+    // whole tiles, strided over the persistent CTAs
+    const long long tile = (long long)blockIdx.x + (long long)idx * gridDim.x;
+    if (tile >= (long long)p.m_tiles * p.n_tiles) return false;
+    const int mt = (int)(tile / p.n_tiles);
+    x.tile = (int)tile;
+    x.nt = (int)(tile - (long long)mt * p.n_tiles);
+    x.expert = 0;
+    x.row0 = mt * NTOK;
+    x.rows = min(NTOK, p.m - x.row0);
+    x.kb0 = 0;
+    x.kb1 = p.k_blocks;
+    x.partial = 0;
+    x.slot = 0;
+    return true;
+  }
+  if (!p.grouped) {
+    const long long T = p.total_iters, G = gridDim.x, i = blockIdx.x;
+    const long long beg = sk_start(i, T, G), end = sk_start(i + 1, T, G);
+    const long long kb = p.k_blocks;
+    const long long tile = beg / kb + idx;
+    const long long x0 = idx == 0 ? beg : tile * kb;
+    if (x0 >= end) return false;
+    const long long x1 = min(end, (tile + 1) * kb);
+    const int mt = (int)(tile / p.n_tiles);
+    x.tile = (int)tile;
+    x.nt = (int)(tile - (long long)mt * p.n_tiles);
+    x.expert = 0;
+    x.row0 = mt * NTOK;
+    x.rows = min(NTOK, p.m - x.row0);
+    x.kb0 = (int)(x0 - tile * kb);
+    x.kb1 = (int)(x1 - tile * kb);
+    x.partial = (x.kb0 != 0 || x.kb1 != p.k_blocks) ? 1 : 0;
+    x.slot = idx == 0 ? 0 : 1;
+    return true;
+  }
+  const int u = blockIdx.x + idx * gridDim.x;
+  if (u >= total_grouped) return false;
+  // find the expert e with prefix[e] <= u < prefix[e+1] (empty experts share
+  // their prefix with the next one, so the largest such e has rows)
+  int lo = 0, hi = p.num_experts;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_prefix[mid] <= u) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  const int rows_e = s_off[e + 1] - s_off[e];
+  const int mtiles = (rows_e + NTOK - 1) / NTOK;
+  const int local = u - s_prefix[e];
+  const int mt = local % mtiles;
+  x.nt = local / mtiles;
+  x.expert = e;
+  x.row0 = s_off[e] + mt * NTOK;
+  x.rows = min(NTOK, s_off[e + 1] - x.row0);
+  x.kb0 = 0;
+  x.kb1 = p.k_blocks;
+  x.tile = 0;
+  x.partial = 0;
+  x.slot = 0;
+  return true;
+}
+
+// Grouped mode: per-expert tile prefix sums from the device-resident row
+// offsets (no host synchronization).  Called by every thread of the CTA;
+// ends with the table visible to all of them.
+template <int NTOK>
+__device__ __forceinline__ void grouped_tables(const W4Params& p, int* s_off, int* s_prefix, int* s_total) {
+  const int E = p.num_experts;
+  for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = p.expert_offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    bool bad = s_off[0] != 0 || s_off[E] != p.m;
+    for (int e = 0; e < E; ++e) {
+      s_prefix[e] = acc;
+      int rows = s_off[e + 1] - s_off[e];
+      if (rows < 0) { bad = true; rows = 0; }
+      acc += ((rows + NTOK - 1) / NTOK) * p.n_tiles;
+    }
+    s_prefix[E] = acc;
+    if (bad) {
+      atomicCAS(p.err, 0u, (uint32_t)HQ_ERR_DEVICE_BAD_OFFSETS);
+      acc = 0;
+    }
+    *s_total = acc;
+  }
+}
+
+// Writes tokens j0 .. j0+EB-1 of one epilogue warp's 32 weight rows
+// (row n = nt*128 + 32q + lane holds v[j] for token j0+j):
+//   * partial unit: fp32 into this CTA's partial slot (column-major per row);
+//   * whole unit, N % 8 == 0: warp-local transpose through `sc` (32 x EB
+//     bf16) so that each lane writes 16 contiguous bytes of an output row;
+//   * otherwise: one bf16 per (token, row).
+template <int EB>
+__device__ __forceinline__ void store_chunk(const W4Params& p, const Unit& x, float* part, int q, int lane, int j0,
+                                            const float (&v)[EB], uint16_t* sc) {
+  const int r = q * 32 + lane;
+  const int n = x.nt * kTileN + r;
+  if (part) {
+#pragma unroll
+    for (int j = 0; j < EB; ++j) __stcg(part + (size_t)(j0 + j) * kTileN + r, v[j]);
+  } else if ((p.n % 8) == 0) {
+#pragma unroll
+    for (int j = 0; j < EB; ++j) sc[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+    __syncwarp();
+    const int seg = lane & 3;
+    const int n0 = x.nt * kTileN + q * 32 + seg * 8;
+#pragma unroll
+    for (int i = 0; i < EB / 8; ++i) {
+      const int jj = (lane >> 2) + 8 * i;
+      if (j0 + jj < x.rows && n0 < p.n) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sc + jj * 32 + seg * 8);
+        *reinterpret_cast<uint4*>(p.c + (size_t)(x.row0 + j0 + jj) * p.n + n0) = w;
+      }
+    }
+    __syncwarp();
+  } else if (n < p.n) {
+#pragma unroll
+    for (int j = 0; j < EB; ++j) {
+      if (j0 + j < x.rows) p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(v[j]);
+    }
+  }
+}
+
+// Stream-K fixup after a partial unit's fp32 slot has been written: each
+// epilogue warp owns 32 rows of the tile and one counter; the last
+// contributing CTA reduces every partial in CTA order, so the result does
+// not depend on arrival order (and nobody waits).
+template <int NTOK>
+__device__ __forceinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, int lane) {
+  const int r = q * 32 + lane;
+  const int n = x.nt * kTileN + r;
+  const bool n_ok = n < p.n;
+  const long long T = p.total_iters, G = gridDim.x, kbl = p.k_blocks;
+  const long long t0 = (long long)x.tile * kbl;
+  const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kbl - 1, T, G);
+  const int cnt = (int)(last - first + 1);
+  __threadfence();
+  __syncwarp();
+  int is_last = 0;
+  if (lane == 0) {
+    __threadfence();
+    is_last = (atomicAdd(p.counters + x.tile * 4 + q, 1) == cnt - 1);
+    __threadfence();
+  }
+  is_last = __shfl_sync(0xffffffffu, is_last, 0);
+  if (!is_last) return;
+  __threadfence();
+  // 16 token rows at a time, every contributor's loads in flight together;
+  // the sum runs in contributor order
+  for (int j0 = 0; j0 < x.rows; j0 += 16) {
+    float acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+    for (long long ci = first; ci <= last; ++ci) {
+      const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
+      const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kTileN + r;
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + (size_t)j * kTileN);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) acc[j] += v[j];
+    }
+    if (n_ok) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j0 + j < x.rows) p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(acc[j]);
+    }
+  }
+  if (lane == 0) p.counters[x.tile * 4 + q] = 0;  // leave the workspace zeroed
+}
+
+// Host side: launch the small-token-tile kernel (16, 32 or 64 tokens).
+hq_status small_launch(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream);
+
+}  // namespace w4
+}  // namespace hq

@@ -1,0 +1,381 @@
+// W4A16 GEMM for small token tiles (16, 32 or 64 tokens): the
+// weight-bandwidth-bound regime, where the fused dequantization has to keep
+// up with HBM.
+//
+// Method: the weights are 4-bit codes q with a per-group fp16 scale s and an
+// optional uint4 zero point z, w = (q - z) * s ("Humming: open-source kernel
+// library for quantized inference", summary paragraph 2), converted inside
+// the kernel (same page, paragraph 3).  Because the scale is constant over a
+// group of 128 K, the sum over one group factors as
+//     sum_k (q_k - z) s a_k  =  s * sum_k (q_k - z) a_k ,
+// so this kernel feeds the tensor core the exact small integers (q - z) (bf16
+// holds -15..15 exactly) and applies s once per group and output element in
+// fp32.  Compared with rescaling every weight in bf16 this takes one bf16x2
+// multiply per weight pair off the dequantization warps and never rounds s
+// or w to bf16.
+//
+// B200 design:
+//   * swap-AB as in the other W4A16 kernel: 128 weight rows are the MMA's M
+//     side, read from TMEM; the tokens are the N side, TMA-staged in shared
+//     memory with the 128-byte swizzle;
+//   * each pipeline stage holds two 128-K records; its MMAs write one fresh
+//     fp32 tile D_g (128 x NTOK) per group g into a TMEM ring instead of
+//     accumulating across K;
+//   * warps 8-15 unpack codes cooperatively (warp 8+q: the stage's first
+//     record, 12+q: the second, rows 32q..32q+31), so a stage is ready as
+//     soon as possible and a 3-deep TMEM ring lets them run ahead of the MMA;
+//   * warps 4-7 ("scale warps") read s for their 32 rows from the stage in
+//     shared memory, then fold s * D_g into fp32 registers as each D_g
+//     lands, and write the output (or the stream-K partial) when a unit
+//     ends.  The order of the fp32 sum is fixed, so results repeat bit for
+//     bit.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "hq_internal.h"
+#include "ptx.cuh"
+#include "w4a16_common.cuh"
+
+namespace hq {
+namespace w4 {
+
+namespace {
+
+template <int NTOK>
+struct SmallCfg {
+  static constexpr int kKps = 2;                        // records (groups) per stage
+  static constexpr int kABlock = NTOK * 256;            // one record's activations: two 64-K boxes
+  static constexpr int kATile = kKps * kABlock;
+  static constexpr int kRecs = kKps * kRecMax;
+  static constexpr int kSmemStages = NTOK == 16 ? 8 : NTOK == 32 ? 6 : 4;
+  static constexpr int kAStages = NTOK == 64 ? 2 : 3;   // TMEM ring of unpacked weights
+  static constexpr int kDStages = NTOK == 16 ? 4 : 2;   // TMEM ring of per-group results
+  static constexpr int kACols = kKps * 64;              // TMEM columns per weight stage
+  static constexpr int kDCols = kKps * NTOK;            // TMEM columns per result stage
+  static constexpr int kEpiScratch = 4 * 2048;          // warp-local transposes of the output
+  static constexpr int kBarBytes = 512;
+  // byte offsets from the 1024-aligned base of dynamic shared memory
+  static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
+  static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
+  static constexpr size_t kScrOff = (kTabOff + 2 * (kMaxExperts + 1) * sizeof(int) + 127) / 128 * 128;
+  static constexpr size_t kSmem = 1024 + kScrOff + kEpiScratch;
+  static_assert(kABlock % 1024 == 0 && kRecMax % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
+  static_assert(kACols * kAStages + kDCols * kDStages <= 512, "TMEM budget");
+  static_assert(8 * (2 * kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 <= kBarBytes, "barrier area");
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
+
+// Unpack one 128-K block of the packed record into TMEM: thread (warp
+// quarter q, lane) owns weight row r = 32q + lane and writes the 128 exact
+// values bf16(q_k - z) into TMEM lane r, 64 columns from taddr (two weights
+// per 32-bit column, even k in the low half).
+__device__ __forceinline__ void unpack_codes(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
+  uint4 raw[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+  const uint32_t z = has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
+  // bf16(128 + z) is exact, and so is (128 + q) - (128 + z) = q - z
+  const uint32_t zbits = 0x4300u + z;
+  const uint32_t z2 = zbits | (zbits << 16);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+    uint32_t out[16];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // the nibbles of k = 2j and 2j+1 sit at bits 4j and 16+4j: OR-ing
+        // them into the mantissa of bf16 128.0 gives bf16(128 + q)
+        const uint32_t x2 = lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u);
+        out[w * 4 + j] = bf16x2_sub(x2, z2);
+      }
+    }
+    tmem_st_x16(taddr + c * 16, out);
+  }
+}
+
+template <int NTOK>
+__global__ void __launch_bounds__(kThreads, 1)
+    w4a16_small_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
+  using C = SmallCfg<NTOK>;
+  constexpr int SS = C::kSmemStages;
+  constexpr int AS = C::kAStages;
+  constexpr int DS = C::kDStages;
+  constexpr int KPS = C::kKps;
+  constexpr int kATile = C::kATile;
+  constexpr int kRecs = C::kRecs;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                               // SS * kATile (activations, 128-byte swizzle)
+  uint8_t* sR = smem + SS * kATile;                 // SS * kRecs (packed weight records)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + SS;      // MMA commit + the four scale warps
+  uint64_t* aready = empty + SS;    // eight unpacking warps
+  uint64_t* afree = aready + AS;    // MMA commit
+  uint64_t* dfull = afree + AS;     // MMA commit
+  uint64_t* dempty = dfull + DS;    // four scale warps
+  uint64_t* drain = dempty + DS;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_total = const_cast<int*>(s_abort + 1);
+  int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);  // [kMaxExperts + 1]
+  int* s_off = s_prefix + (kMaxExperts + 1);                    // [kMaxExperts + 1]
+  uint16_t* epi_scratch = reinterpret_cast<uint16_t*>(smem + C::kScrOff);  // 16-byte aligned
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 5);
+    }
+    for (int t = 0; t < AS; ++t) {
+      mbar_init(&aready[t], 8);
+      mbar_init(&afree[t], 1);
+    }
+    for (int d = 0; d < DS; ++d) {
+      mbar_init(&dfull[d], 1);
+      mbar_init(&dempty[d], 4);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    *s_total = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_a);
+  if (warp == 2) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (p.grouped) grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total_grouped = *s_total;
+
+  auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * C::kACols); };
+  auto d_col = [](int d) -> uint32_t { return (uint32_t)(AS * C::kACols + d * C::kDCols); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (whole warp, elected lane issues)
+    const bool leader = elect_one();
+    const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_last();
+    uint32_t it = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      const uint8_t* wbase =
+          p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
+        const int s = it % SS;
+        const int nrec = min(KPS, x.kb1 - kb);
+        if (!hq_wait_warp(&empty[s], ((it / SS) & 1) ^ 1, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        if (leader) {
+          mbar_arrive_expect_tx(&full[s], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+          for (int r = 0; r < nrec; ++r) {
+            bulk_g2s(sR + s * kRecs + r * kRecMax, wbase + (uint64_t)(kb + r) * p.rec_bytes, (uint32_t)p.rec_bytes,
+                     &full[s], pol_w);
+            uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
+            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, &full[s]);
+            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, &full[s]);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) {
+      // let every copy already issued land before the CTA exits
+      const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
+      for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
+    // one lane, fixed for the whole kernel, issues every MMA and commit: a
+    // commit tracks the tcgen05 operations of the thread that issues it
+    const bool leader = elect_one();
+    uint32_t it = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
+        const int s = it % SS, t = it % AS, d = it % DS;
+        const int nrec = min(KPS, x.kb1 - kb);
+        if (!hq_wait_warp(&aready[t], (it / AS) & 1, p.wait_ns, s_abort) ||
+            !hq_wait_warp(&full[s], (it / SS) & 1, p.wait_ns, s_abort) ||
+            !hq_wait_warp(&dempty[d], ((it / DS) & 1) ^ 1, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+          // descriptors advance by constants: 32 B per 16-K step inside a
+          // 128-byte swizzle row, one box (NTOK rows) per 64 K
+          const uint64_t b0 = smem_desc_sw128(smem_u32(sA + s * kATile));
+          const uint32_t a0 = tmem_base + a_col(t);
+          const uint32_t d0 = tmem_base + d_col(d);
+          for (int r = 0; r < nrec; ++r) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint64_t bdesc = b0 + (uint64_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
+              mma_bf16_ts(d0 + r * NTOK, a0 + r * 64 + j * 8, bdesc, kIdesc, j > 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&empty[s]);
+          tc_commit(&afree[t]);
+          tc_commit(&dfull[d]);
+        }
+        __syncwarp();
+      }
+    }
+    // make sure no MMA is still running when TMEM is released
+    if (leader) {
+      tc_commit(drain);
+      hq_wait(drain, 0, p.wait_ns, nullptr);
+    }
+    __syncwarp();
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ unpack codes (warps 8-15)
+    const uint32_t q = warp & 3;
+    const int h = (int)(warp - 8) >> 2;               // record of the stage this warp unpacks
+    const int r = (int)(q * 32 + lane);               // weight row within the tile
+    const uint32_t lane_addr = (q * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
+        const int s = it % SS, t = it % AS;
+        const int nrec = min(KPS, x.kb1 - kb);
+        // full[s] cannot move on before this warp's own arrival (through the
+        // MMA it enables) and afree[t] before the MMA it enables: every
+        // phase of both is observed in order
+        if (!hq_wait(&full[s], (it / SS) & 1, p.wait_ns, s_abort) ||
+            !hq_wait(&afree[t], ((it / AS) & 1) ^ 1, p.wait_ns, s_abort)) {
+          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (h < nrec) unpack_codes(sR + s * kRecs + h * kRecMax, r, p.has_zero, tmem_base + lane_addr + a_col(t) + h * 64);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&aready[t]);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ scale warps + epilogue (warps 4-7)
+    const uint32_t q = warp & 3;
+    const int r = (int)(q * 32 + lane);
+    const uint32_t lane_addr = (q * 32) << 16;
+    constexpr int CH = NTOK >= 32 ? 32 : 16;          // TMEM columns per load batch
+    uint32_t it = 0;
+    bool ok = true;
+    Unit x;
+    for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      float acc[NTOK];
+#pragma unroll
+      for (int j = 0; j < NTOK; ++j) acc[j] = 0.f;
+      for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
+        const int s = it % SS, d = it % DS;
+        const int nrec = min(KPS, x.kb1 - kb);
+        if (!hq_wait(&full[s], (it / SS) & 1, p.wait_ns, s_abort)) {
+          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        float sc[KPS];
+#pragma unroll
+        for (int rr = 0; rr < KPS; ++rr)
+          sc[rr] = rr < nrec ? __half2float(reinterpret_cast<const __half*>(sR + s * kRecs + rr * kRecMax +
+                                                                            kW4RecCodes)[r])
+                             : 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (!hq_wait(&dfull[d], (it / DS) & 1, p.wait_ns, s_abort)) {
+          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int rr = 0; rr < KPS; ++rr) {
+          if (rr < nrec) {
+#pragma unroll
+            for (int j0 = 0; j0 < NTOK; j0 += CH) {
+              uint32_t v0[16], v1[16];
+              const uint32_t src = tmem_base + lane_addr + d_col(d) + rr * NTOK + j0;
+              tmem_ld_x16(src, v0);
+              if (CH == 32) tmem_ld_x16(src + 16, v1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < CH; ++j)
+                acc[j0 + j] = fmaf(sc[rr], __uint_as_float(j < 16 ? v0[j] : v1[j - 16]), acc[j0 + j]);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dempty[d]);
+      }
+      if (!ok) break;
+
+      // ---- output of this unit
+      float* part = x.partial ? p.partials + ((size_t)blockIdx.x * 2 + x.slot) * NTOK * kTileN : nullptr;
+      uint16_t* scr = epi_scratch + q * 1024;
+#pragma unroll
+      for (int j0 = 0; j0 < NTOK; j0 += CH) {
+        float v[CH];
+#pragma unroll
+        for (int j = 0; j < CH; ++j) v[j] = acc[j0 + j];
+        store_chunk<CH>(p, x, part, (int)q, (int)lane, j0, v, scr);
+      }
+      if (x.partial) sk_fixup<NTOK>(p, x, (int)q, (int)lane);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tmem_base, 512);
+}
+
+template <int NTOK>
+hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+  auto kern = w4a16_small_kernel<NTOK>;
+  const size_t smem = SmallCfg<NTOK>::kSmem;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  kern<<<grid, kThreads, smem, stream>>>(map, p);
+  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+}  // namespace
+
+hq_status small_launch(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+  switch (ntok) {
+    case 16: return launch_small_t<16>(map, p, grid, stream);
+    case 32: return launch_small_t<32>(map, p, grid, stream);
+    case 64: return launch_small_t<64>(map, p, grid, stream);
+    default: return HQ_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace w4
+}  // namespace hq

@@ -1,6 +1,7 @@
 """Run one GEMM configuration a few times through the C ABI, for profilers.
 
     python -m quantized_gemm_bit_b200.profile_case --kind w4a16 --m 16 --k 7168 --n 18432 --iters 3
+    python -m quantized_gemm_bit_b200.profile_case --kind nvfp4 --m 8192 --k 8192 --n 8192 --iters 2
 
 Inputs are the seeded synthetic workload tensors; the device status is
 checked at the end (non-zero exit on any error).  Used to capture ncu
@@ -18,7 +19,7 @@ from .build import build
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "moe"])
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "moe", "mxfp4", "nvfp4"])
     ap.add_argument("--m", type=int, default=16)
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)
@@ -28,11 +29,43 @@ def main(argv=None):
     ap.add_argument("--asym", action="store_true")
     ap.add_argument("--tile-m", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
+    ap.add_argument("--variant", type=int, default=0)
     a = ap.parse_args(argv)
     build()
     dev = "cuda"
-    tuning = hq.Tuning(tile_m=a.tile_m, split_k=a.split_k) if (a.tile_m or a.split_k) else None
-    if a.kind == "w4a16":
+    tuning = (hq.Tuning(tile_m=a.tile_m, split_k=a.split_k, variant=a.variant)
+              if (a.tile_m or a.split_k or a.variant) else None)
+    if a.kind in ("mxfp4", "nvfp4"):
+        ws = None
+        if a.kind == "mxfp4":
+            codes, e8 = synth.mxfp4_weights(a.n, a.k, seed=2000)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, a.n, a.k, 32, 0, 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(dev)
+            x = synth.bf16_normal(a.m, a.k, seed=2001).to(dev)
+            xq = torch.empty(a.m, a.k, dtype=torch.uint8, device=dev)
+            xs = torch.empty(a.m, dtype=torch.float32, device=dev)
+            hq.hq_quantize_fp8_rows(x, a.m, a.k, xq, xs)
+            run = lambda c, ws: hq.hq_gemm_mxfp4_a8(d, blob, xq, xs, a.m, c, ws, tuning)
+        else:
+            def quant(rows, seed):
+                x = synth.bf16_normal(rows, a.k, seed).to(dev)
+                codes = torch.empty(rows, a.k // 2, dtype=torch.uint8, device=dev)
+                sf = torch.empty(rows, a.k // 16, dtype=torch.uint8, device=dev)
+                g = torch.empty(1, dtype=torch.float32, device=dev)
+                wsq = torch.zeros(hq.hq_quantize_nvfp4_workspace_size(rows, a.k), dtype=torch.uint8, device=dev)
+                hq.hq_quantize_nvfp4(x, rows, a.k, codes, sf, g, wsq)
+                return codes, sf, g
+            wc, wsf, wg = quant(a.n, 4000)
+            ac, asf, ag = quant(a.m, 4100)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, a.n, a.k, 16, 0, 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, wc.cpu(), wsf.cpu(), None, float(wg.item()))).to(dev)
+            a_g = float(ag.item())
+            run = lambda c, ws: hq.hq_gemm_nvfp4(d, blob, ac, asf, a_g, a.m, c, ws, tuning)
+        c = torch.empty(a.m, a.n, dtype=torch.bfloat16, device=dev)
+        ws = torch.zeros(max(256, hq.hq_workspace_size(d, a.m, tuning)), dtype=torch.uint8, device=dev)
+        for _ in range(a.iters):
+            run(c, ws)
+    elif a.kind == "w4a16":
         q, s, z = synth.w4a16_weights(a.n, a.k, 128, a.asym, seed=1000)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, int(a.asym), 1)
         blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)

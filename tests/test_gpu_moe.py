@@ -101,8 +101,8 @@ def _grouped(desc, blob, a_sorted, off, rows, n, tuning=None):
     return c
 
 
-@pytest.mark.parametrize("tile_m", [0, 16, 64, 256])
-def test_grouped_reduced_config_full_output(tile_m):
+@pytest.mark.parametrize("tile_m,variant", [(0, 0), (16, 0), (32, 0), (64, 0), (128, 0), (16, 1), (64, 1)])
+def test_grouped_reduced_config_full_output(tile_m, variant):
     e, n, k, t, topk = 8, 256, 512, 40, 2
     q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=5000, experts=e)
     d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, e)
@@ -113,10 +113,10 @@ def test_grouped_reduced_config_full_output(tile_m):
     a = synth.bf16_normal(t, k, seed=5002)
     src, off, a_sorted, st = gpu_permute(torch.from_numpy(ids).to(DEV), e, a)
     assert st == hq.HQ_OK
-    tuning = hq.Tuning(tile_m=tile_m) if tile_m else None
+    tuning = hq.Tuning(tile_m=tile_m, variant=variant) if (tile_m or variant) else None
     c = _grouped(d, blob, a_sorted, off, t * topk, n, tuning)
     _, ref = G.grouped_w4a16_ref(_bits(a_sorted.cpu()), off.cpu().numpy(), q.numpy(), s.numpy(), None, 128)
-    check_gemm(c, ref, k, f"grouped tile_m={tile_m}")
+    check_gemm(c, ref, k, f"grouped tile_m={tile_m} variant={variant}")
 
 
 def test_grouped_bad_offsets_are_reported():

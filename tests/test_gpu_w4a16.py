@@ -67,19 +67,24 @@ def test_ragged_shapes_full_output(m, n, k, asym):
     check_gemm(c, ref, k, f"m={m} n={n} k={k}")
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("tile_m", [16, 32, 64, 128, 256])
-def test_every_token_tile(tile_m):
+def test_every_token_tile(tile_m, variant):
+    """Every token tile of both kernels: variant 0 feeds exact (q - z) and
+    scales per group in fp32 for tiles <= 64; variant 1 rescales weights to
+    bf16 for every tile."""
     m, n, k = 70, 384, 1024
     d, blob, a, (q, s, z) = make_case(m, n, k, True, 7)
-    c, _ = run(d, blob, a, m, hq.Tuning(tile_m=tile_m))
-    check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"tile_m={tile_m}")
+    c, _ = run(d, blob, a, m, hq.Tuning(tile_m=tile_m, variant=variant))
+    check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"tile_m={tile_m} variant={variant}")
 
 
+@pytest.mark.parametrize("variant", [0, 1])
 @pytest.mark.parametrize("splits", [2, 3, 7])
-def test_split_k_and_determinism(splits):
+def test_split_k_and_determinism(splits, variant):
     m, n, k = 20, 256, 1792
     d, blob, a, (q, s, z) = make_case(m, n, k, False, 9)
-    t = hq.Tuning(tile_m=32, split_k=splits)
+    t = hq.Tuning(tile_m=32, split_k=splits, variant=variant)
     c1, ws = run(d, blob, a, m, t)
     c2, _ = run(d, blob, a, m, t)
     assert torch.equal(c1, c2)
@@ -87,6 +92,18 @@ def test_split_k_and_determinism(splits):
     # the workspace is left zero-filled (counters reset by the last split)
     counters = ws[256:256 + 4 * 4 * 2].view(torch.int32)
     assert int(counters.abs().sum()) == 0
+
+
+@pytest.mark.parametrize("m", [1, 16, 48])
+def test_stream_k_repeats_bit_for_bit(m):
+    """Default plan at a stream-K size (K=N=2048 spread over every SM): two
+    runs give identical bits and match the oracle."""
+    n = k = 2048
+    d, blob, a, (q, s, z) = make_case(m, n, k, True, 13 + m)
+    c1, _ = run(d, blob, a, m)
+    c2, _ = run(d, blob, a, m)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"stream-K m={m}")
 
 
 def test_guard_bands_untouched():
