@@ -172,7 +172,11 @@ hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, con
 /* NVFP4 W4A4 GEMM ([P-fa] format list, W4A4 combination):
  * C = (g_a * g_w) * sum_k e2m1(a)*sf_a * e2m1(w)*sf_w.
  *   a_fp4_dev : uint8 [m][k/2] (even k low nibble); a_sf_dev : uint8 E4M3
- *   [m][k/16]; a_global : fp32 tensor scale of A.  g_w is in the blob. */
+ *   [m][k/16]; a_global : fp32 tensor scale of A.  g_w is in the blob.
+ * Two launches on `stream`: a_sf is first copied into the workspace in the
+ * order the tensor core reads block scales (k/256 chunks of 2 KB per
+ * 128-token slice of each token tile), then the GEMM runs; the workspace
+ * size includes that copy. */
 hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const void* a_fp4_dev,
                         const void* a_sf_dev, float a_global, int32_t m, void* c_dev, const hq_tuning* t,
                         void* ws_dev, size_t ws_bytes, hq_stream_t stream);

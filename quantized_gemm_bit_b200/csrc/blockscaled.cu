@@ -32,6 +32,7 @@
 
 #include <algorithm>
 
+#include "epilogue.cuh"
 #include "hq_internal.h"
 #include "ptx.cuh"
 
@@ -39,8 +40,10 @@ namespace hq {
 
 namespace {
 
-constexpr int kBsThreads = 256;
+constexpr int kBsThreads = 384;    // 12 warps
 constexpr int kBsTileN = 128;
+constexpr int kBsEpiWarps = 8;
+constexpr int kBsEB = 16;          // tokens per transposed output store
 
 enum BsFmt { kMX = 0, kNV = 1 };
 
@@ -53,33 +56,39 @@ struct BsCfg {
   static constexpr int kATx = FMT == kNV ? kATile : kBsTileN * 64;
   static constexpr int kBTile = NTOK * 128;                // activations
   static constexpr int kSfa = FMT == kNV ? 2048 : 512;     // weight scale chunks per stage
-  static constexpr int kHalves = NTOK > 128 ? 2 : 1;       // 128-row halves of the token tile
-  static constexpr int kSfbRaw = FMT == kNV ? NTOK * 16 : 0;
-  static constexpr int kSfbT = FMT == kNV ? 4 * kHalves * 512 : 0;
-  static constexpr int kStageRaw = kATile + kBTile + kSfa + kSfbRaw + kSfbT;
+  static constexpr int kHalves = NTOK > 128 ? 2 : 1;       // 128-token halves of the token tile
+  static constexpr int kSfb = FMT == kNV ? 4 * kHalves * 512 : 0;   // activation scale chunks per stage
+  static constexpr int kStageRaw = kATile + kBTile + kSfa + kSfb;
   static constexpr int kStage = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kStages = std::min(10, (200 * 1024) / kStage);
+  static constexpr int kBarBytes = 512;
+  static constexpr int kScratch = kBsEpiWarps * 32 * kBsEB * 2;   // output transposes
+  static constexpr int kStages = std::min(10, (232448 - 1024 - kBarBytes - kScratch) / kStage);
   static constexpr int kAcc = NTOK <= 128 ? 2 : 1;
+  static constexpr int kCols = NTOK / 2;                   // accumulator columns per epilogue warp
   // TMEM columns: accumulators, then per-stage scale slots
   static constexpr int kSfaCols = FMT == kNV ? 16 : 4;
   static constexpr int kSfbCols = FMT == kNV ? 16 * kHalves : 0;
   static constexpr int kSfSlot = kSfaCols + kSfbCols;
   static constexpr int kSfBase = kAcc * NTOK;
   static constexpr int kSfbConst = kSfBase + kStages * kSfSlot;   // MXFP4: constant unit scales (8 cols)
+  static constexpr size_t kBarOff = (size_t)kStages * kStage;
+  static constexpr size_t kScrOff = kBarOff + kBarBytes;
+  static constexpr size_t kSmem = 1024 + kScrOff + kScratch;
+  static_assert(kStages >= 3, "pipeline depth");
   static_assert(kSfbConst + 8 <= 512, "TMEM budget");
-  static constexpr int kBarBytes = 512;
-  static constexpr size_t kSmem = (size_t)kStages * kStage + 1024 + kBarBytes;
-  static_assert(8 * (3 * kStages + 5) + 16 <= kBarBytes, "barrier area");
+  static_assert(8 * (2 * kStages + 5) + 16 <= kBarBytes, "barrier area");
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct BsParams {
   const uint8_t* sf_w;       // weight scale chunks (blob + codes bytes)
+  const uint8_t* sf_a;       // NVFP4: activation scale chunks, [m_tiles][k_stages][kSfb] (workspace)
   __nv_bfloat16* c;
   const float* a_scale;      // MXFP4: per-token scale [m]
   const float* g_w;          // NVFP4: weight tensor scale (blob tail)
   float a_global;            // NVFP4: activation tensor scale
   float* partials;
-  int32_t* counters;
+  int32_t* counters;         // [tiles][8], one per epilogue warp
   uint32_t* err;
   uint64_t wait_ns;
   long long total_iters;
@@ -89,6 +98,29 @@ struct BsParams {
   int m_tiles;
   int data_parallel;         // whole tiles per unit, no partial sums
 };
+
+// NVFP4 activation scales, row-major [m][K/16] bytes, re-laid into the order
+// tcgen05.cp .32x128b.warpx4 copies into TMEM: per (token tile mt, stage
+// ks), chunk (MMA i, token half h) is 512 bytes whose byte l*16 + 4c + j is
+// the scale of token h*128 + 32c + l of the tile, K block 16*ks + 4i + j
+// (zero past the tile or the last row).  One thread per 32-bit word.
+__global__ void sfb_relayout_kernel(const uint32_t* __restrict__ sf, int m, int kw, int ntok, int halves,
+                                    int k_stages, uint32_t* __restrict__ out, long long words) {
+  for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < words;
+       w += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(w & 3);
+    const int l = (int)((w >> 2) & 31);
+    long long rest = w >> 7;
+    const int ih = (int)(rest % (4 * halves));
+    rest /= 4 * halves;
+    const int ks = (int)(rest % k_stages);
+    const long long mt = rest / k_stages;
+    const int i = ih / halves, h = ih % halves;
+    const int tok = h * 128 + 32 * c + l;
+    const long long row = mt * ntok + tok;
+    out[w] = (tok < ntok && row < m) ? __ldg(sf + row * kw + ks * 4 + i) : 0u;
+  }
+}
 
 template <int FMT, int NTOK>
 __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, int& nt, int& row0, int& rows,
@@ -129,28 +161,28 @@ __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, i
 template <int FMT, int NTOK>
 __global__ void __launch_bounds__(kBsThreads, 1)
     blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
-                       const __grid_constant__ CUtensorMap tmap_sfb, const BsParams p) {
+                       const BsParams p) {
   using C = BsCfg<FMT, NTOK>;
   constexpr int S = C::kStages;
   constexpr int ACC = C::kAcc;
-  constexpr uint32_t kTx = C::kATx + C::kBTile + C::kSfa + C::kSfbRaw;
+  constexpr int NC = C::kCols;
+  constexpr uint32_t kTx = C::kATx + C::kBTile + C::kSfa + C::kSfb;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + S;
-  uint64_t* sfb_ready = empty + S;
-  uint64_t* acc_full = sfb_ready + S;
+  uint64_t* acc_full = empty + S;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  uint16_t* scratch = reinterpret_cast<uint16_t*>(smem + C::kScrOff);   // 16-byte aligned
 
   auto sA = [&](int s) { return smem + s * C::kStage; };
   auto sB = [&](int s) { return smem + s * C::kStage + C::kATile; };
   auto sSfa = [&](int s) { return smem + s * C::kStage + C::kATile + C::kBTile; };
-  auto sSfbRaw = [&](int s) { return sSfa(s) + C::kSfa; };
-  auto sSfbT = [&](int s) { return sSfbRaw(s) + C::kSfbRaw; };
+  auto sSfb = [&](int s) { return sSfa(s) + C::kSfa; };
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -159,11 +191,10 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&sfb_ready[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], kBsEpiWarps);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -172,7 +203,6 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_w);
     prefetch_tensormap(&tmap_a);
-    if (FMT == kNV) prefetch_tensormap(&tmap_sfb);
   }
   if (warp == 2) {
     tmem_alloc(s_tmem, 512);
@@ -182,7 +212,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  if (FMT == kMX && warp >= 4) {
+  if (FMT == kMX && warp >= 4 && warp < 8) {
     // activations carry no block scale: E8M0 127 (= 1.0) in every byte
     tmem_st_x8(tmem_base + (((warp & 3) * 32) << 16) + C::kSfbConst, 0x7F7F7F7Fu);
     tmem_wait_st();
@@ -216,7 +246,10 @@ __global__ void __launch_bounds__(kBsThreads, 1)
           const int chunks = FMT == kNV ? 4 : 1;
           const uint8_t* src = p.sf_w + ((size_t)nt * p.sf_groups + (size_t)ks * chunks) * 512;
           bulk_g2s(sSfa(s), src, C::kSfa, &full[s], pol_w);
-          if (FMT == kNV) tma_load_2d(sSfbRaw(s), &tmap_sfb, ks * 16, row0, &full[s]);
+          if (FMT == kNV) {
+            const uint8_t* sfb = p.sf_a + ((size_t)(row0 / NTOK) * p.k_stages + ks) * C::kSfb;
+            bulk_g2s(sSfb(s), sfb, C::kSfb, &full[s], policy_evict_last());
+          }
         }
         __syncwarp();
       }
@@ -244,9 +277,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       for (int ks = ks0; ks < ks1; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        bool got = hq_wait_warp(&full[s], ph, p.wait_ns, s_abort);
-        if (got && FMT == kNV) got = hq_wait_warp(&sfb_ready[s], ph, p.wait_ns, s_abort);
-        if (!got) {
+        if (!hq_wait_warp(&full[s], ph, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -264,7 +295,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
               tmem_cp_sf(sfa_t, smem_desc_sf(smem_u32(sSfa(s)) + 512 * i));
 #pragma unroll
               for (int h = 0; h < C::kHalves; ++h)
-                tmem_cp_sf(sfb_t + 4 * h, smem_desc_sf(smem_u32(sSfbT(s)) + 512 * (i * C::kHalves + h)));
+                tmem_cp_sf(sfb_t + 4 * h, smem_desc_sf(smem_u32(sSfb(s)) + 512 * (i * C::kHalves + h)));
               constexpr uint32_t kId = idesc_block_scaled(1, 1, 0, 128, NTOK, 0, 0);
               mma_mxf4nvf4(d_tmem, smem_desc_sw128(a_base + 32 * i), smem_desc_sw128(b_base + 32 * i), kId, sfa_t,
                            sfb_t, (ks > ks0 || i > 0) ? 1u : 0u);
@@ -293,52 +324,18 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       hq_wait(drain, 0, p.wait_ns, nullptr);
     }
     __syncwarp();
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ NVFP4 activation-scale reorder
-    if (FMT == kNV) {
-      uint32_t it = 0;
-      bool ok = true;
-      for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
-        for (int ks = ks0; ks < ks1; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (!hq_wait(&full[s], ph, p.wait_ns, s_abort)) {
-            raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-            ok = false;
-            break;
-          }
-          // raw: [NTOK rows][16 scale bytes]; chunk (MMA i, half h): byte
-          // l*16 + 4c + j = scale of row h*128 + l + 32c, block 4i + j
-          const uint8_t* raw = sSfbRaw(s);
-          uint8_t* dst = sSfbT(s);
-#pragma unroll
-          for (int h = 0; h < C::kHalves; ++h) {
-            uint4 rw[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int row = h * 128 + (int)lane + 32 * c;
-              rw[c] = row < NTOK ? *reinterpret_cast<const uint4*>(raw + row * 16) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const uint32_t w0 = i == 0 ? rw[0].x : i == 1 ? rw[0].y : i == 2 ? rw[0].z : rw[0].w;
-              const uint32_t w1 = i == 0 ? rw[1].x : i == 1 ? rw[1].y : i == 2 ? rw[1].z : rw[1].w;
-              const uint32_t w2 = i == 0 ? rw[2].x : i == 1 ? rw[2].y : i == 2 ? rw[2].z : rw[2].w;
-              const uint32_t w3 = i == 0 ? rw[3].x : i == 1 ? rw[3].y : i == 2 ? rw[3].z : rw[3].w;
-              *reinterpret_cast<uint4*>(dst + (i * C::kHalves + h) * 512 + lane * 16) = make_uint4(w0, w1, w2, w3);
-            }
-          }
-          fence_proxy_async_smem();  // make the reordered scales visible to tcgen05.cp
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sfb_ready[s]);
-        }
-      }
-    }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (8 warps)
+    // warp 4 + 4*hc + q owns weight rows 32q..32q+31 and tokens
+    // hc*NC .. hc*NC+NC-1 of the tile.  It copies its accumulator columns
+    // into registers and hands the accumulator back to the MMA at once, then
+    // scales and stores while the next unit's MMAs run.
     const uint32_t q = warp & 3;
+    const int hc = (int)(warp - 4) >> 2;
     const int r = (int)(q * 32 + lane);
     const uint32_t lane_addr = (q * 32) << 16;
+    const int wslot = hc * 4 + (int)q;
+    uint16_t* scr = scratch + (warp - 4) * (32 * kBsEB);
     const float alpha = FMT == kNV ? p.a_global * __ldg(p.g_w) : 1.f;
     uint32_t uc = 0;
     for (int idx = 0; bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx, ++uc) {
@@ -349,31 +346,42 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         break;
       }
       tc_fence_after();
-      const int n = nt * kBsTileN + r;
-      const bool n_ok = n < p.n;
-      float* part = partial ? p.partials + ((size_t)blockIdx.x * 2 + slot) * NTOK * kBsTileN : nullptr;
-#pragma unroll 1
-      for (int j0 = 0; j0 < NTOK; j0 += 16) {
-        uint32_t v[16];
-        tmem_ld_x16(tmem_base + lane_addr + ab * NTOK + j0, v);
-        tmem_wait_ld();
-        if (partial) {
+      uint32_t v[NC];
+      const uint32_t src = tmem_base + lane_addr + ab * NTOK + hc * NC;
+      if constexpr (NC == 8) {
+        tmem_ld_x8(src, *reinterpret_cast<uint32_t(*)[8]>(v));
+      } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(part + (size_t)(j0 + j) * kBsTileN + r, __uint_as_float(v[j]));
-        } else if (n_ok) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (j0 + j < rows) {
-              const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + j0 + j);
-              p.c[(size_t)(row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(__uint_as_float(v[j]) * sc);
-            }
-          }
-        }
+        for (int j0 = 0; j0 < NC; j0 += 16) tmem_ld_x16(src + j0, *reinterpret_cast<uint32_t(*)[16]>(v + j0));
       }
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
+
+      const int tok0 = hc * NC;                       // first token of this warp's run
+      const int rows_w = rows - tok0;                 // valid tokens in the run (may be <= 0)
+      float* part = partial ? p.partials + (((size_t)blockIdx.x * 2 + slot) * NTOK + tok0) * kBsTileN : nullptr;
+      constexpr int EB = NC < kBsEB ? NC : kBsEB;
+#pragma unroll
+      for (int j0 = 0; j0 < NC; j0 += EB) {
+        float f[EB];
+        if (FMT == kMX && !partial) {
+          // per-token scales: lane j reads token j of the run, then broadcast
+          const int tk = tok0 + j0 + (int)(lane % EB);
+          const float mine = tk < rows ? __ldg(p.a_scale + row0 + tk) : 0.f;
+#pragma unroll
+          for (int j = 0; j < EB; ++j) f[j] = __uint_as_float(v[j0 + j]) * __shfl_sync(0xffffffffu, mine, j);
+        } else {
+#pragma unroll
+          for (int j = 0; j < EB; ++j) f[j] = partial ? __uint_as_float(v[j0 + j]) : __uint_as_float(v[j0 + j]) * alpha;
+        }
+        store_rows_chunk<EB>(p.c, p.n, row0 + tok0, rows_w, nt * kBsTileN + (int)q * 32, r, part, (int)lane, j0, f,
+                             scr);
+      }
       if (partial) {
+        // stream-K fixup: one counter per (tile, epilogue warp); the last
+        // contributing CTA reduces every partial in CTA order
         const long long T = p.total_iters, G = gridDim.x, kst = p.k_stages;
         const long long t0 = (long long)tile * kst;
         const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kst - 1, T, G);
@@ -383,36 +391,39 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         int is_last = 0;
         if (lane == 0) {
           __threadfence();
-          is_last = (atomicAdd(p.counters + tile * 4 + q, 1) == cnt - 1);
+          is_last = (atomicAdd(p.counters + tile * kBsEpiWarps + wslot, 1) == cnt - 1);
           __threadfence();
         }
         is_last = __shfl_sync(0xffffffffu, is_last, 0);
         if (is_last) {
           __threadfence();
-          for (int j0 = 0; j0 < rows; j0 += 16) {
-            float acc[16];
+          const int n = nt * kBsTileN + r;
+          constexpr int RC = NC < 16 ? NC : 16;
+          for (int j0 = 0; j0 < NC && j0 < rows_w; j0 += RC) {
+            float acc[RC];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = 0.f;
+            for (int j = 0; j < RC; ++j) acc[j] = 0.f;
             for (long long ci = first; ci <= last; ++ci) {
               const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
-              const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kBsTileN + r;
-              float v[16];
+              const float* srcp = p.partials + (((size_t)ci * 2 + sl) * NTOK + tok0 + j0) * kBsTileN + r;
+              float w[RC];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + (size_t)j * kBsTileN);
+              for (int j = 0; j < RC; ++j) w[j] = __ldcg(srcp + (size_t)j * kBsTileN);
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc[j] += v[j];
+              for (int j = 0; j < RC; ++j) acc[j] += w[j];
             }
-            if (n_ok) {
+            if (n < p.n) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                if (j0 + j < rows) {
-                  const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + j0 + j);
-                  p.c[(size_t)(row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(acc[j] * sc);
+              for (int j = 0; j < RC; ++j) {
+                if (j0 + j < rows_w) {
+                  const int tk = tok0 + j0 + j;
+                  const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + tk);
+                  p.c[(size_t)(row0 + tk) * p.n + n] = __float2bfloat16_rn(acc[j] * sc);
                 }
               }
             }
           }
-          if (lane == 0) p.counters[tile * 4 + q] = 0;
+          if (lane == 0) p.counters[tile * kBsEpiWarps + wslot] = 0;
         }
       }
     }
@@ -425,8 +436,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
 }
 
 template <int FMT, int NTOK>
-hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& msf, const BsParams& p,
-                      int grid, cudaStream_t stream) {
+hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const BsParams& p, int grid,
+                      cudaStream_t stream) {
   auto kern = blockscaled_kernel<FMT, NTOK>;
   const size_t smem = BsCfg<FMT, NTOK>::kSmem;
   static bool attr_set[64] = {};
@@ -437,7 +448,7 @@ hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const CUtens
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  kern<<<grid, kBsThreads, smem, stream>>>(mw, ma, msf, p);
+  kern<<<grid, kBsThreads, smem, stream>>>(mw, ma, p);
   return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
@@ -486,11 +497,30 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   return cfg;
 }
 
-size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg) {
-  if (cfg.splits == 0) return sizeof(WsHeader);
+// Workspace: header | stream-K counters (8 per tile) and partial tiles (2 per
+// CTA), when K is split | NVFP4 activation scales re-laid for the MMA.
+struct BsWsLayout {
+  size_t counters, partials, sfb, total;
+};
+BsWsLayout bs_ws_layout(const hq_quant_desc& d, int m, const BsConfig& cfg) {
+  BsWsLayout L{};
+  size_t off = sizeof(WsHeader);
   const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
-  return sizeof(WsHeader) + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256 +
-         (size_t)cfg.grid * 2 * cfg.ntok * kBsTileN * sizeof(float);
+  L.counters = off;
+  if (cfg.splits != 0) off += ((kBsEpiWarps * tiles * sizeof(int32_t) + 255) / 256) * 256;
+  L.partials = off;
+  if (cfg.splits != 0) off += (size_t)cfg.grid * 2 * cfg.ntok * kBsTileN * sizeof(float);
+  L.sfb = off;
+  if (d.fmt == HQ_FMT_NVFP4) {
+    const size_t halves = cfg.ntok > 128 ? 2 : 1;
+    off += (size_t)((m + cfg.ntok - 1) / cfg.ntok) * (d.k / 256) * 4 * halves * 512;
+  }
+  L.total = off;
+  return L;
+}
+
+size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg) {
+  return bs_ws_layout(d, m, cfg).total;
 }
 
 hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* packed, const void* a,
@@ -518,13 +548,15 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.total_iters = (long long)tiles * p.k_stages;
   p.m_tiles = (m + cfg.ntok - 1) / cfg.ntok;
   p.data_parallel = cfg.splits == 0 ? 1 : 0;
-  uint8_t* base = static_cast<uint8_t*>(ws) + sizeof(WsHeader);
-  p.counters = reinterpret_cast<int32_t*>(base);
-  p.partials = reinterpret_cast<float*>(base + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256);
+  const BsWsLayout L = bs_ws_layout(d, m, cfg);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  p.counters = reinterpret_cast<int32_t*>(wsb + L.counters);
+  p.partials = reinterpret_cast<float*>(wsb + L.partials);
+  p.sf_a = wsb + L.sfb;
 
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return HQ_ERR_CUDA;
-  CUtensorMap mw{}, ma{}, msf{};
+  CUtensorMap mw{}, ma{};
   cuuint32_t estr[2] = {1, 1};
   // weights: codes [NP][K/2] bytes
   {
@@ -548,21 +580,19 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
   }
-  // NVFP4 activation scales: [M][K/16] bytes, 16 per row per stage
+  // NVFP4 activation scales: re-laid into the MMA's chunk order in the
+  // workspace (a few MB at most), read by the kernel with bulk copies
   if (nv) {
-    cuuint64_t dims[2] = {(cuuint64_t)d.k / 16, (cuuint64_t)m};
-    cuuint64_t strides[1] = {(cuuint64_t)d.k / 16};
-    cuuint32_t box[2] = {16, (cuuint32_t)cfg.ntok};
-    CUresult cr = enc(&msf, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a_sf), dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
-  } else {
-    msf = ma;  // unused
+    const int halves = cfg.ntok > 128 ? 2 : 1;
+    const long long words = (long long)p.m_tiles * p.k_stages * 4 * halves * 128;
+    const int blocks = (int)std::min<long long>((words + 255) / 256, 4LL * 148);
+    sfb_relayout_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint32_t*>(a_sf), m, d.k / 64, cfg.ntok,
+                                                     halves, p.k_stages, reinterpret_cast<uint32_t*>(wsb + L.sfb), words);
+    if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;
   }
 
 #define HQ_BS_CASE(F, NT) \
-  case NT: return bs_launch_t<F, NT>(mw, ma, msf, p, cfg.grid, stream);
+  case NT: return bs_launch_t<F, NT>(mw, ma, p, cfg.grid, stream);
   if (nv) {
     switch (cfg.ntok) {
       HQ_BS_CASE(kNV, 16) HQ_BS_CASE(kNV, 32) HQ_BS_CASE(kNV, 64) HQ_BS_CASE(kNV, 128) HQ_BS_CASE(kNV, 256)

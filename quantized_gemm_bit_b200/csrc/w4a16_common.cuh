@@ -13,6 +13,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include "epilogue.cuh"
 #include "hq_internal.h"
 #include "ptx.cuh"
 
@@ -129,7 +130,7 @@ __device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix,
 template <int NTOK>
 __device__ __forceinline__ void grouped_tables(const W4Params& p, int* s_off, int* s_prefix, int* s_total) {
   const int E = p.num_experts;
-  for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = p.expert_offsets[i];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = p.expert_offsets[i];
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -149,41 +150,13 @@ __device__ __forceinline__ void grouped_tables(const W4Params& p, int* s_off, in
   }
 }
 
-// Writes tokens j0 .. j0+EB-1 of one epilogue warp's 32 weight rows
-// (row n = nt*128 + 32q + lane holds v[j] for token j0+j):
-//   * partial unit: fp32 into this CTA's partial slot (column-major per row);
-//   * whole unit, N % 8 == 0: warp-local transpose through `sc` (32 x EB
-//     bf16) so that each lane writes 16 contiguous bytes of an output row;
-//   * otherwise: one bf16 per (token, row).
+// Writes tokens j0 .. j0+EB-1 of one epilogue warp's 32 weight rows (row
+// n = nt*128 + 32q + lane holds v[j] for token j0+j): fp32 into this CTA's
+// partial slot for a partial unit, else bf16 output (store_rows_chunk).
 template <int EB>
 __device__ __forceinline__ void store_chunk(const W4Params& p, const Unit& x, float* part, int q, int lane, int j0,
                                             const float (&v)[EB], uint16_t* sc) {
-  const int r = q * 32 + lane;
-  const int n = x.nt * kTileN + r;
-  if (part) {
-#pragma unroll
-    for (int j = 0; j < EB; ++j) __stcg(part + (size_t)(j0 + j) * kTileN + r, v[j]);
-  } else if ((p.n % 8) == 0) {
-#pragma unroll
-    for (int j = 0; j < EB; ++j) sc[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
-    __syncwarp();
-    const int seg = lane & 3;
-    const int n0 = x.nt * kTileN + q * 32 + seg * 8;
-#pragma unroll
-    for (int i = 0; i < EB / 8; ++i) {
-      const int jj = (lane >> 2) + 8 * i;
-      if (j0 + jj < x.rows && n0 < p.n) {
-        const uint4 w = *reinterpret_cast<const uint4*>(sc + jj * 32 + seg * 8);
-        *reinterpret_cast<uint4*>(p.c + (size_t)(x.row0 + j0 + jj) * p.n + n0) = w;
-      }
-    }
-    __syncwarp();
-  } else if (n < p.n) {
-#pragma unroll
-    for (int j = 0; j < EB; ++j) {
-      if (j0 + j < x.rows) p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(v[j]);
-    }
-  }
+  store_rows_chunk<EB>(p.c, p.n, x.row0, x.rows, x.nt * kTileN + q * 32, q * 32 + lane, part, lane, j0, v, sc);
 }
 
 // Stream-K fixup after a partial unit's fp32 slot has been written: each

@@ -21,9 +21,11 @@
 //   * each pipeline stage holds two 128-K records; its MMAs write one fresh
 //     fp32 tile D_g (128 x NTOK) per group g into a TMEM ring instead of
 //     accumulating across K;
-//   * warps 8-15 unpack codes cooperatively (warp 8+q: the stage's first
-//     record, 12+q: the second, rows 32q..32q+31), so a stage is ready as
-//     soon as possible and a 3-deep TMEM ring lets them run ahead of the MMA;
+//   * warps 8 and up unpack codes cooperatively (16 warps for 16/32 tokens,
+//     each a quarter of a stage's 32-row slices; 8 warps for 64 tokens), so
+//     a stage is ready as soon as possible, many independent warps hide the
+//     latency of the integer unpacking, and a 3-deep TMEM ring lets them run
+//     ahead of the MMA;
 //   * warps 4-7 ("scale warps") read s for their 32 rows from the stage in
 //     shared memory, then fold s * D_g into fp32 registers as each D_g
 //     lands, and write the output (or the stream-K partial) when a unit
@@ -52,6 +54,12 @@ struct SmallCfg {
   static constexpr int kDStages = NTOK == 16 ? 4 : 2;   // TMEM ring of per-group results
   static constexpr int kACols = kKps * 64;              // TMEM columns per weight stage
   static constexpr int kDCols = kKps * NTOK;            // TMEM columns per result stage
+  // unpacking warps: four per SM sub-partition for 16/32 tokens (each takes
+  // half of one record's rows-quarter), two at 64 tokens, whose scale warps
+  // need more registers than 24 warps leave them
+  static constexpr int kUnpackWarps = NTOK <= 32 ? 16 : 8;
+  static constexpr int kThreads = (8 + kUnpackWarps) * 32;
+  static constexpr int kChunks = 4 * kKps * 4 / kUnpackWarps;   // 32-K chunks per unpacking warp
   static constexpr int kEpiScratch = 4 * 2048;          // warp-local transposes of the output
   static constexpr int kBarBytes = 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
@@ -65,20 +73,21 @@ struct SmallCfg {
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-// Unpack one 128-K block of the packed record into TMEM: thread (warp
-// quarter q, lane) owns weight row r = 32q + lane and writes the 128 exact
-// values bf16(q_k - z) into TMEM lane r, 64 columns from taddr (two weights
-// per 32-bit column, even k in the low half).
-__device__ __forceinline__ void unpack_codes(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
-  uint4 raw[4];
+// Unpack 32-K chunks c0 .. c0+NCH-1 of one 128-K record into TMEM: thread
+// (warp quarter q, lane) owns weight row r = 32q + lane and writes the exact
+// values bf16(q_k - z) into TMEM lane r, 16 columns per chunk from
+// taddr + 16*c (two weights per 32-bit column, even k in the low half).
+template <int NCH>
+__device__ __forceinline__ void unpack_codes(const uint8_t* rec, int c0, int r, int has_zero, uint32_t taddr) {
+  uint4 raw[NCH];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+  for (int c = 0; c < NCH; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + ((c0 + c) * 128 + r) * 16);
   const uint32_t z = has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
   // bf16(128 + z) is exact, and so is (128 + q) - (128 + z) = q - z
   const uint32_t zbits = 0x4300u + z;
   const uint32_t z2 = zbits | (zbits << 16);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < NCH; ++c) {
     const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
     uint32_t out[16];
 #pragma unroll
@@ -91,12 +100,12 @@ __device__ __forceinline__ void unpack_codes(const uint8_t* rec, int r, int has_
         out[w * 4 + j] = bf16x2_sub(x2, z2);
       }
     }
-    tmem_st_x16(taddr + c * 16, out);
+    tmem_st_x16(taddr + (c0 + c) * 16, out);
   }
 }
 
 template <int NTOK>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
     w4a16_small_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
   using C = SmallCfg<NTOK>;
   constexpr int SS = C::kSmemStages;
@@ -134,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 5);
     }
     for (int t = 0; t < AS; ++t) {
-      mbar_init(&aready[t], 8);
+      mbar_init(&aready[t], C::kUnpackWarps);
       mbar_init(&afree[t], 1);
     }
     for (int d = 0; d < DS; ++d) {
@@ -244,9 +253,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 8) {
-    // ------------------------------------------------------------ unpack codes (warps 8-15)
+    // ------------------------------------------------------------ unpack codes (warps 8 and up)
+    // warp 8 + 4u + q unpacks rows 32q..32q+31 of share u of the stage: with
+    // 16 warps, record u/2, chunks 2(u%2), 2(u%2)+1; with 8, record u, all 4
+    constexpr int NCH = C::kChunks;
     const uint32_t q = warp & 3;
-    const int h = (int)(warp - 8) >> 2;               // record of the stage this warp unpacks
+    const int u = (int)(warp - 8) >> 2;
+    const int h = u * NCH / 4;                        // record of the stage this warp unpacks
+    const int c0 = (u * NCH) % 4;                     // first chunk
     const int r = (int)(q * 32 + lane);               // weight row within the tile
     const uint32_t lane_addr = (q * 32) << 16;
     uint32_t it = 0;
@@ -266,7 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        if (h < nrec) unpack_codes(sR + s * kRecs + h * kRecMax, r, p.has_zero, tmem_base + lane_addr + a_col(t) + h * 64);
+        if (h < nrec)
+          unpack_codes<NCH>(sR + s * kRecs + h * kRecMax, c0, r, p.has_zero,
+                            tmem_base + lane_addr + a_col(t) + h * 64);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -278,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q = warp & 3;
     const int r = (int)(q * 32 + lane);
     const uint32_t lane_addr = (q * 32) << 16;
-    constexpr int CH = NTOK >= 32 ? 32 : 16;          // TMEM columns per load batch
+    constexpr int CH = NTOK >= 64 ? 32 : 16;          // TMEM columns per load batch
     uint32_t it = 0;
     bool ok = true;
     Unit x;
@@ -362,7 +378,7 @@ hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cu
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  kern<<<grid, kThreads, smem, stream>>>(map, p);
+  kern<<<grid, SmallCfg<NTOK>::kThreads, smem, stream>>>(map, p);
   return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 

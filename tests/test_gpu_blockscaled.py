@@ -42,7 +42,7 @@ def mx_run(d, blob, aq, asc, m, tuning=None):
     return c
 
 
-@pytest.mark.parametrize("m,n,k", [(16, 256, 512), (5, 200, 384), (70, 384, 1024), (300, 256, 640)])
+@pytest.mark.parametrize("m,n,k", [(16, 256, 512), (5, 200, 384), (70, 384, 1024), (300, 256, 640), (33, 130, 512)])
 def test_mxfp4_full_output(m, n, k):
     d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 200 + m)
     c = mx_run(d, blob, aq, asc, m)
@@ -56,6 +56,17 @@ def test_mxfp4_every_token_tile(tile_m):
     d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 300)
     c = mx_run(d, blob, aq, asc, m, hq.Tuning(tile_m=tile_m))
     check_gemm(c, G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8), k, f"mxfp4 tile_m={tile_m}")
+
+
+@pytest.mark.parametrize("tile_m,splits", [(16, 3), (64, 2), (256, 2)])
+def test_mxfp4_split_k_repeats_bit_for_bit(tile_m, splits):
+    m, n, k = 200, 384, 1024
+    d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 310)
+    t = hq.Tuning(tile_m=tile_m, split_k=splits)
+    c1 = mx_run(d, blob, aq, asc, m, t)
+    c2 = mx_run(d, blob, aq, asc, m, t)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8), k, f"mxfp4 split {tile_m}x{splits}")
 
 
 @pytest.mark.parametrize("m", [16, 256, 4096])
@@ -95,7 +106,8 @@ def nv_run(d, blob, act, m, tuning=None):
     return c
 
 
-@pytest.mark.parametrize("m,n,k", [(16, 256, 512), (7, 200, 768), (130, 384, 1024), (300, 128, 256)])
+@pytest.mark.parametrize("m,n,k", [(16, 256, 512), (7, 200, 768), (130, 384, 1024), (300, 128, 256),
+                                   (33, 130, 512)])
 def test_nvfp4_full_output(m, n, k):
     d, blob, act, w = nv_case(m, n, k, 400 + m)
     c = nv_run(d, blob, act, m)
@@ -109,6 +121,17 @@ def test_nvfp4_every_token_tile(tile_m):
     d, blob, act, w = nv_case(m, n, k, 500)
     c = nv_run(d, blob, act, m, hq.Tuning(tile_m=tile_m))
     check_gemm(c, G.nvfp4_ref(*act, *w), k, f"nvfp4 tile_m={tile_m}")
+
+
+@pytest.mark.parametrize("tile_m,splits", [(16, 3), (128, 2), (256, 2)])
+def test_nvfp4_split_k_repeats_bit_for_bit(tile_m, splits):
+    m, n, k = 300, 256, 1536
+    d, blob, act, w = nv_case(m, n, k, 510)
+    t = hq.Tuning(tile_m=tile_m, split_k=splits)
+    c1 = nv_run(d, blob, act, m, t)
+    c2 = nv_run(d, blob, act, m, t)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.nvfp4_ref(*act, *w), k, f"nvfp4 split {tile_m}x{splits}")
 
 
 @pytest.mark.parametrize("m,n,k", [(8192, 8192, 8192), (16384, 18432, 7168)])
