@@ -177,44 +177,6 @@ def setup_w4a16_sweep(l2_bytes):
     return shapes
 
 
-def build_step_graphs(shapes, gemms, ncopy, stream):
-    """One CUDA graph per rotation offset c: the 14 sweep GEMMs, GEMM mi of a
-    shape reading weight copy (c*7 + mi) mod ncopy, so consecutive GEMMs of a
-    shape never share a copy; each GEMM sits between two timing events
-    recorded as graph nodes."""
-    from quantized_gemm_bit_b200 import hq
-    graphs, gev = [], []
-    side = torch.cuda.Stream()
-    side.wait_stream(stream)
-    for c in range(ncopy):
-        g = torch.cuda.CUDAGraph()
-        evs = {}
-        with torch.cuda.graph(g, stream=side):
-            cap = torch.cuda.current_stream()
-            for (si, mi) in gemms:
-                sh = shapes[si]
-                a = torch.cuda.Event(enable_timing=True, external=True)
-                b = torch.cuda.Event(enable_timing=True, external=True)
-                a.record(cap)
-                blob = sh["blobs"][(c * len(SWEEP_M) + mi) % len(sh["blobs"])]
-                hq.hq_gemm_w4a16(sh["d"], blob, sh["acts"][mi], SWEEP_M[mi], sh["outs"][mi],
-                                 sh["wss"][mi], stream=cap)
-                b.record(cap)
-                evs[(si, mi)] = (a, b)
-        graphs.append(g)
-        gev.append(evs)
-    stream.wait_stream(side)
-    return graphs, gev
-
-
-def launch_times(gev, gemms, ncopy, nlast):
-    """Mean duration (us) of each GEMM over the last replay of each graph."""
-    out = {}
-    for g in gemms:
-        out[g] = statistics.mean(gev[c][g][0].elapsed_time(gev[c][g][1]) for c in range(nlast)) * 1e3
-    return out
-
-
 def run_w4a16_sweep(args, rank, world, peaks):
     from quantized_gemm_bit_b200 import hq
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
@@ -247,33 +209,26 @@ def run_w4a16_sweep(args, rank, world, peaks):
             if st != hq.HQ_OK:
                 raise RuntimeError(f"device status after warm-up: {hq.status_string(st)}")
 
-    # ---- device-resident timed region: one CUDA graph per weight-copy index
-    # (14 GEMMs each), replayed back to back, so host launch cost never
-    # starves the GPU; each GEMM is bracketed by timing events captured in
-    # the graph (they keep the times of each graph's last replay)
+    # ---- device-resident timed region (CUDA graphs, see _time_launches): in
+    # graph c, GEMM mi of a shape reads weight copy (c + mi) mod ncopy, so the
+    # GEMMs of a step never share a copy and a GEMM's back-to-back launches
+    # (c = 0, 1, ...) never repeat one
     ncopy = len(shapes[0]["blobs"])
-    graphs, gev = build_step_graphs(shapes, gemms, ncopy, stream)
-    for i in range(args.warmup):
-        graphs[i % ncopy].replay()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = []
+    for (si, mi) in gemms:
+        def f(c, si=si, mi=mi):
+            sh = shapes[si]
+            blob = sh["blobs"][(c + mi) % len(sh["blobs"])]
+            hq.hq_gemm_w4a16(sh["d"], blob, sh["acts"][mi], SWEEP_M[mi], sh["outs"][mi], sh["wss"][mi])
+        launches.append(f)
     with Clocks(torch.cuda.current_device()) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        t0.record(stream)
-        for i in range(args.steps):
-            graphs[i % ncopy].replay()
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-    ms = max_over_ranks(t0.elapsed_time(t1), world)
-    per_launch_us = launch_times(gev, gemms, ncopy, min(args.steps, ncopy))
+        ms, per = _time_launches(launches, args.steps, args.warmup, world, ncopy=ncopy)
+    per_launch_us = dict(zip(gemms, per))
     for sh in shapes:
         for ws in sh["wss"]:
             st = hq.hq_check_device_status(ws)
             if st != hq.HQ_OK:
                 raise RuntimeError(f"device status after the timed region: {hq.status_string(st)}")
-    del graphs
 
     # ---- end-to-end through the C ABI with host buffers (pinned), copies inside
     for _ in range(max(1, args.warmup // 2)):
@@ -348,7 +303,8 @@ def run_w4a16_sweep(args, rank, world, peaks):
                         "(18432,7168)}, symmetric INT4, group 128",
             "gemms_per_step": len(gemms),
             "l2": f"weights rotate over {len(shapes[0]['blobs'])} copies per shape (>3x L2), no flush",
-            "launch": "one CUDA graph per step (the 14 C-ABI calls captured once per weight copy)",
+            "launch": "CUDA graphs: one per step (the 14 C-ABI calls, captured once per weight-copy rotation); "
+                      "per-launch times from graphs of back-to-back launches of each GEMM",
             "parallelism": f"replicas x{world}",
         },
         "roofline": roof(big, "tensor"),
@@ -370,12 +326,26 @@ def run_w4a16_sweep(args, rank, world, peaks):
 FP8_RATIO, FP4_RATIO = 2.0, 4.0   # nominal dense peaks relative to bf16 (4.5 / 9 vs 2.25 PF)
 
 
+def _capture(fns, side):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for f in fns:
+            f()
+    return g
+
+
 def _time_launches(launches, steps, warmup, world, ncopy=1):
     """Time `launches` (callables f(c) issuing C-ABI calls on the current
-    stream; c = weight-copy index) through CUDA graphs: graph c holds every
-    launch with copy c, each between two timing events captured as graph
-    nodes; step i replays graph i % ncopy.  Returns (total ms over `steps`,
-    per-launch mean microseconds over the last replay of each graph)."""
+    stream; c = weight-copy index) through CUDA graphs, so host launch cost
+    never starves the GPU.
+      * steps: graph c holds every launch with copy c; step i replays graph
+        i % ncopy; the K timed steps sit between two events (barrier and
+        synchronize on both sides);
+      * per launch: one graph of R = max(ncopy, 4) back-to-back launches of
+        it (copies rotating), replayed three times between two events while
+        a fourth replay queued before them keeps the GPU busy; the mean
+        duration includes the launch gaps inside the graph.
+    Returns (total ms over `steps`, per-launch mean microseconds)."""
     stream = torch.cuda.current_stream()
     for i in range(max(1, warmup)):        # host-side first-call setup happens here, outside capture
         for f in launches:
@@ -383,21 +353,7 @@ def _time_launches(launches, steps, warmup, world, ncopy=1):
     torch.cuda.synchronize()
     side = torch.cuda.Stream()
     side.wait_stream(stream)
-    graphs, evs = [], []
-    for c in range(ncopy):
-        g = torch.cuda.CUDAGraph()
-        ev = []
-        with torch.cuda.graph(g, stream=side):
-            cap = torch.cuda.current_stream()
-            for f in launches:
-                a = torch.cuda.Event(enable_timing=True, external=True)
-                b = torch.cuda.Event(enable_timing=True, external=True)
-                a.record(cap)
-                f(c)
-                b.record(cap)
-                ev.append((a, b))
-        graphs.append(g)
-        evs.append(ev)
+    graphs = [_capture([(lambda f=f, c=c: f(c)) for f in launches], side) for c in range(ncopy)]
     stream.wait_stream(side)
     for i in range(warmup):
         graphs[i % ncopy].replay()
@@ -412,10 +368,24 @@ def _time_launches(launches, steps, warmup, world, ncopy=1):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(t0.elapsed_time(t1), world)
-    used = min(steps, ncopy)
-    per = [statistics.mean(evs[c][j][0].elapsed_time(evs[c][j][1]) for c in range(used)) * 1e3
-           for j in range(len(launches))]
     del graphs
+    per = []
+    reps = max(ncopy, 4)
+    for f in launches:
+        side.wait_stream(stream)
+        g = _capture([(lambda f=f, c=c: f(c % ncopy)) for c in range(reps)], side)
+        stream.wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g.replay()                      # keeps the GPU busy while the timed replays are queued
+        a.record(stream)
+        for _ in range(3):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per.append(a.elapsed_time(b) * 1e3 / (3 * reps))
+        del g
     return ms, per
 
 

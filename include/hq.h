@@ -40,6 +40,13 @@
  *     that completes leaves it zero-filled again (apart from the error word,
  *     which hq_check_device_status clears).
  *   - Pointers named *_dev are device pointers; *_host are host pointers.
+ *   - The GEMM kernels are launched as programmatic dependents of the
+ *     previous kernel on the stream: their CTAs may start, set up and fetch
+ *     the first stages of the packed weights while that kernel finishes;
+ *     everything else (activations, scales, offsets, outputs, workspace) is
+ *     touched only after it has completed.  So the kernel launched just
+ *     before a GEMM call must not write that call's packed weights (copies
+ *     and memsets are ordinary stream dependencies and are not affected).
  */
 #ifndef HQ_H_
 #define HQ_H_

@@ -158,6 +158,69 @@ __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, i
   return true;
 }
 
+// Stream-K fixup of one epilogue warp's rows x tokens after its partial slot
+// is written: one counter per (tile, epilogue warp); the last contributing
+// CTA reduces every partial in CTA order (8 tokens at a time, the loads of
+// up to CB contributors in flight together) and writes the scaled output.
+template <int FMT, int NTOK, int CB>
+__device__ __forceinline__ void bs_fixup(const BsParams& p, int tile, int nt, int row0, int rows, int tok0, int wslot,
+                                      int r, int lane, float alpha) {
+  constexpr int NC = BsCfg<FMT, NTOK>::kCols;
+  const int rows_w = rows - tok0;
+  const long long T = p.total_iters, G = gridDim.x, kst = p.k_stages;
+  const long long t0 = (long long)tile * kst;
+  const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kst - 1, T, G);
+  const int cnt = (int)(last - first + 1);
+  __threadfence();
+  __syncwarp();
+  int is_last = 0;
+  if (lane == 0) {
+    __threadfence();
+    is_last = (atomicAdd(p.counters + tile * kBsEpiWarps + wslot, 1) == cnt - 1);
+    __threadfence();
+  }
+  is_last = __shfl_sync(0xffffffffu, is_last, 0);
+  if (!is_last) return;
+  __threadfence();
+  const int n = nt * kBsTileN + r;
+  for (int j0 = 0; j0 < NC && j0 < rows_w; j0 += 8) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    for (long long c0 = first; c0 <= last; c0 += CB) {
+      float w[CB][8];
+#pragma unroll
+      for (int b = 0; b < CB; ++b) {
+        if (c0 + b <= last) {
+          const long long ci = c0 + b;
+          const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
+          const float* srcp = p.partials + (((size_t)ci * 2 + sl) * NTOK + tok0 + j0) * kBsTileN + r;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[b][j] = __ldcg(srcp + (size_t)j * kBsTileN);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < CB; ++b) {
+        if (c0 + b <= last) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j] += w[b][j];
+        }
+      }
+    }
+    if (n < p.n) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j0 + j < rows_w) {
+          const int tk = tok0 + j0 + j;
+          const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + tk);
+          p.c[(size_t)(row0 + tk) * p.n + n] = __float2bfloat16_rn(acc[j] * sc);
+        }
+      }
+    }
+  }
+  if (lane == 0) p.counters[tile * kBsEpiWarps + wslot] = 0;
+}
+
 template <int FMT, int NTOK>
 __global__ void __launch_bounds__(kBsThreads, 1)
     blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
@@ -204,22 +267,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     prefetch_tensormap(&tmap_w);
     prefetch_tensormap(&tmap_a);
   }
-  if (warp == 2) {
-    tmem_alloc(s_tmem, 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *s_tmem;
-  if (FMT == kMX && warp >= 4 && warp < 8) {
-    // activations carry no block scale: E8M0 127 (= 1.0) in every byte
-    tmem_st_x8(tmem_base + (((warp & 3) * 32) << 16) + C::kSfbConst, 0x7F7F7F7Fu);
-    tmem_wait_st();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  __syncthreads();   // barriers visible to every role
 
   int tile, nt, row0, rows, ks0, ks1, partial, slot;
 
@@ -227,25 +276,46 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     // ------------------------------------------------------------ producer (whole warp, one lane issues)
     const bool leader = elect_one();
     const uint64_t pol_w = policy_evict_first();
+    // weights of stage it: codes (K coordinate in elements for the MXFP4
+    // unpacking type, in bytes for NVFP4) and their scale chunks
+    auto load_weights = [&](int s, int ks, int nt_) {
+      tma_load_2d(sA(s), &tmap_w, FMT == kNV ? ks * 128 : ks * C::kKStage, nt_ * kBsTileN, &full[s]);
+      const int chunks = FMT == kNV ? 4 : 1;
+      const uint8_t* src = p.sf_w + ((size_t)nt_ * p.sf_groups + (size_t)ks * chunks) * 512;
+      bulk_g2s(sSfa(s), src, C::kSfa, &full[s], pol_w);
+    };
+    // Phase 1, before the previous kernel on the stream has finished: the
+    // packed weights of the first S stages (no kernel writes them)
+    uint32_t n_pre = 0;
+    for (int idx = 0; n_pre < (uint32_t)S && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
+         ++idx) {
+      for (int ks = ks0; ks < ks1 && n_pre < (uint32_t)S; ++ks, ++n_pre) {
+        if (leader) {
+          mbar_arrive_expect_tx(&full[n_pre], kTx);
+          load_weights((int)n_pre, ks, nt);
+        }
+        __syncwarp();
+      }
+    }
+    pdl_wait();
+    // Phase 2: activations (and their scales) of those stages, then the ring
     uint32_t it = 0;
     bool ok = true;
     for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
       for (int ks = ks0; ks < ks1; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (!hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+        if (it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         if (leader) {
-          mbar_arrive_expect_tx(&full[s], kTx);
-          // weights: K coordinate in elements (MXFP4 unpacking type) or bytes (NVFP4)
-          tma_load_2d(sA(s), &tmap_w, FMT == kNV ? ks * 128 : ks * C::kKStage, nt * kBsTileN, &full[s]);
+          if (it >= n_pre) {
+            mbar_arrive_expect_tx(&full[s], kTx);
+            load_weights(s, ks, nt);
+          }
           tma_load_2d(sB(s), &tmap_a, ks * 128, row0, &full[s]);
-          const int chunks = FMT == kNV ? 4 : 1;
-          const uint8_t* src = p.sf_w + ((size_t)nt * p.sf_groups + (size_t)ks * chunks) * 512;
-          bulk_g2s(sSfa(s), src, C::kSfa, &full[s], pol_w);
           if (FMT == kNV) {
             const uint8_t* sfb = p.sf_a + ((size_t)(row0 / NTOK) * p.k_stages + ks) * C::kSfb;
             bulk_g2s(sSfb(s), sfb, C::kSfb, &full[s], policy_evict_last());
@@ -258,7 +328,29 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       const uint32_t first = it > (uint32_t)S ? it - S : 0;
       for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % S], (j / S) & 1, p.wait_ns, nullptr);
     }
-  } else if (warp == 1) {
+  } else {
+  // The producer needs no TMEM, so it starts loading at once; the other
+  // roles wait here for the allocation (and, for MXFP4, the unit scales).
+  if (warp == 2) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  pdl_wait();   // outputs, partials and counters may be in use by the previous kernel
+  tc_fence_before();
+  named_bar(1, kBsThreads - 32);
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  if (FMT == kMX) {
+    if (warp >= 4 && warp < 8) {
+      // activations carry no block scale: E8M0 127 (= 1.0) in every byte
+      tmem_st_x8(tmem_base + (((warp & 3) * 32) << 16) + C::kSfbConst, 0x7F7F7F7Fu);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    named_bar(2, kBsThreads - 32);
+    tc_fence_after();
+  }
+  if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp, one fixed lane issues)
     const bool leader = elect_one();
     uint32_t it = 0, uc = 0;
@@ -379,60 +471,18 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         store_rows_chunk<EB>(p.c, p.n, row0 + tok0, rows_w, nt * kBsTileN + (int)q * 32, r, part, (int)lane, j0, f,
                              scr);
       }
-      if (partial) {
-        // stream-K fixup: one counter per (tile, epilogue warp); the last
-        // contributing CTA reduces every partial in CTA order
-        const long long T = p.total_iters, G = gridDim.x, kst = p.k_stages;
-        const long long t0 = (long long)tile * kst;
-        const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kst - 1, T, G);
-        const int cnt = (int)(last - first + 1);
-        __threadfence();
-        __syncwarp();
-        int is_last = 0;
-        if (lane == 0) {
-          __threadfence();
-          is_last = (atomicAdd(p.counters + tile * kBsEpiWarps + wslot, 1) == cnt - 1);
-          __threadfence();
-        }
-        is_last = __shfl_sync(0xffffffffu, is_last, 0);
-        if (is_last) {
-          __threadfence();
-          const int n = nt * kBsTileN + r;
-          constexpr int RC = NC < 16 ? NC : 16;
-          for (int j0 = 0; j0 < NC && j0 < rows_w; j0 += RC) {
-            float acc[RC];
-#pragma unroll
-            for (int j = 0; j < RC; ++j) acc[j] = 0.f;
-            for (long long ci = first; ci <= last; ++ci) {
-              const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
-              const float* srcp = p.partials + (((size_t)ci * 2 + sl) * NTOK + tok0 + j0) * kBsTileN + r;
-              float w[RC];
-#pragma unroll
-              for (int j = 0; j < RC; ++j) w[j] = __ldcg(srcp + (size_t)j * kBsTileN);
-#pragma unroll
-              for (int j = 0; j < RC; ++j) acc[j] += w[j];
-            }
-            if (n < p.n) {
-#pragma unroll
-              for (int j = 0; j < RC; ++j) {
-                if (j0 + j < rows_w) {
-                  const int tk = tok0 + j0 + j;
-                  const float sc = FMT == kNV ? alpha : __ldg(p.a_scale + row0 + tk);
-                  p.c[(size_t)(row0 + tk) * p.n + n] = __float2bfloat16_rn(acc[j] * sc);
-                }
-              }
-            }
-          }
-          if (lane == 0) p.counters[tile * kBsEpiWarps + wslot] = 0;
-        }
-      }
+      // the 256-token tile keeps 128 accumulator registers per thread: fewer
+      // contributors in flight there
+      if (partial) bs_fixup<FMT, NTOK, (NTOK > 128 ? 1 : 4)>(p, tile, nt, row0, rows, tok0, wslot, r, (int)lane, alpha);
     }
   }
+
+  }  // non-producer roles
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem_base, 512);
+  if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
 template <int FMT, int NTOK>
@@ -448,8 +498,8 @@ hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const BsPara
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  kern<<<grid, kBsThreads, smem, stream>>>(mw, ma, p);
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(kBsThreads), smem, stream, mw, ma, p) == cudaSuccess ? HQ_OK
+                                                                                                 : HQ_ERR_CUDA;
 }
 
 int bs_tiles(const hq_quant_desc& d, int m, int ntok) {

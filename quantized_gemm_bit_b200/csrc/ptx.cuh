@@ -78,6 +78,41 @@ __device__ __forceinline__ bool hq_wait(uint64_t* bar, uint32_t parity, uint64_t
   }
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait of a whole warp for up to three barriers at once: lane i
+// probes barrier i, so one instruction tests all of them and the warp pays
+// one shared-memory round trip instead of one per barrier.  Returns the
+// same verdict on every lane (false after `limit_ns` or once *abort is set).
+__device__ __forceinline__ bool hq_wait_warp_n(int n, uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1,
+                                               uint64_t* b2, uint32_t p2, uint64_t limit_ns, volatile int* abort) {
+  const uint32_t lane = threadIdx.x & 31;
+  uint64_t* bar = lane == 0 ? b0 : lane == 1 ? b1 : b2;
+  const uint32_t par = lane == 0 ? p0 : lane == 1 ? p1 : p2;
+  const bool mine = (int)lane < n;
+  if (__all_sync(0xffffffffu, !mine || mbar_test_wait(bar, par))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  bool done = !mine;
+  for (uint32_t i = 1;; ++i) {
+    if (!done) done = mbar_try_wait(bar, par);
+    if (__all_sync(0xffffffffu, done)) return true;
+    if ((i & 63) == 0) {
+      const bool stop = (abort != nullptr && *abort) || globaltimer_ns() - t0 > limit_ns;
+      if (__any_sync(0xffffffffu, stop)) return false;
+    }
+  }
+}
+
 // Bounded wait by every lane of a warp; the verdict of lane 0 is returned to
 // all lanes so the warp never diverges on it.
 __device__ __forceinline__ bool hq_wait_warp(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
@@ -279,6 +314,16 @@ __host__ __device__ constexpr uint32_t idesc_block_scaled(uint32_t a_fmt, uint32
   return (b_sf_id << 4) | (a_fmt << 7) | (b_fmt << 10) | ((n >> 3) << 17) | (scale_e8m0 << 23) | ((m >> 4) << 24) |
          (a_sf_id << 29);
 }
+
+// Programmatic dependent launch.  launch_dependents lets the next kernel on
+// the stream (launched with programmatic stream serialization) start its
+// CTAs as this grid's CTAs retire; wait blocks until the previous kernel on
+// the stream has completed and its memory is visible (a no-op when this
+// kernel was not launched as a programmatic dependent).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

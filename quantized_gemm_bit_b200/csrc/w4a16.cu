@@ -165,16 +165,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_a);
-  if (warp == 2) {
-    tmem_alloc(s_tmem, 512);
-    tmem_relinquish();
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  // Everything but the packed weights may be written by the previous kernel
+  // on the stream: grouped mode needs the expert offsets at once
+  if (p.grouped) {
+    pdl_wait();
+    grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
   }
-
-  if (p.grouped) grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *s_tmem;
+  __syncthreads();   // barriers (and the grouped tables) visible to every role
   const int total_grouped = *s_total;
 
   auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * 64 * KPS); };
@@ -184,9 +182,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer (whole warp, elected lane issues)
     const bool leader = elect_one();
     const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_last();
+    Unit x;
+    // Phase 1, before the previous kernel has finished: the packed weights
+    // of the first SS stages (no kernel writes them)
+    uint32_t n_pre = 0;
+    if (!p.grouped) {
+      for (int idx = 0; n_pre < (uint32_t)SS && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+        const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
+        for (int kb = x.kb0; kb < x.kb1 && n_pre < (uint32_t)SS; kb += KPS, ++n_pre) {
+          const int nrec = min(KPS, x.kb1 - kb);
+          if (leader) {
+            uint64_t* fb = full_bar(n_pre);
+            mbar_arrive_expect_tx(fb, (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+            bulk_g2s(sR + n_pre * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), fb,
+                     pol_w);
+          }
+          __syncwarp();
+        }
+      }
+      pdl_wait();
+    }
+    // Phase 2: the activations of those stages, then the steady ring
     uint32_t it = 0;
     bool ok = true;
-    Unit x;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
       const uint8_t* wbase =
           p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
@@ -194,17 +212,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % SS;
         const uint32_t ph = (it / SS) & 1;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+        if (it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         if (leader) {
           uint64_t* fb = full_bar(it);
-          mbar_arrive_expect_tx(fb, (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+          if (it >= n_pre) {
+            mbar_arrive_expect_tx(fb, (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+            // the stage's records are consecutive in the blob: one bulk copy
+            // (long copies stream HBM much faster than record-sized ones)
+            bulk_g2s(sR + s * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), fb, pol_w);
+          }
           for (int r = 0; r < nrec; ++r) {
-            bulk_g2s(sR + s * kRecs + r * kRecMax, wbase + (uint64_t)(kb + r) * p.rec_bytes, (uint32_t)p.rec_bytes,
-                     fb, pol_w);
             uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
             tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, fb);
             tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, fb);
@@ -218,7 +239,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
       for (uint32_t j = first; j < it; ++j) hq_wait(full_bar(j), full_par(j), p.wait_ns, nullptr);
     }
-  } else if (warp == 1) {
+  } else {
+  // The producer needs no TMEM, so it starts loading at once; the other
+  // roles wait here for the allocation.
+  if (warp == 2) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (!p.grouped) pdl_wait();   // outputs, partials and counters may be in use by the previous kernel
+  tc_fence_before();
+  named_bar(1, kThreads - 32);
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
     // one lane, fixed for the whole kernel, issues every MMA and commit: a
     // commit tracks the tcgen05 operations of the thread that issues it
@@ -240,8 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % SS, t = it % TS;
         const uint32_t ph_t = (it / TS) & 1;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp(&aready[t], ph_t, p.wait_ns, s_abort) ||
-            !hq_wait_warp(full_bar(it), full_par(it), p.wait_ns, s_abort)) {
+        if (!hq_wait_warp_n(2, &aready[t], ph_t, full_bar(it), full_par(it), nullptr, 0, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -295,15 +327,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // only ever serve this group, so it observes every phase of the
         // barriers it waits on, one after the other (a parity wait can only
         // tell adjacent phases apart).
-        if (!hq_wait(full_bar(it), full_par(it), p.wait_ns, s_abort) ||
-            !hq_wait(&afree[t], ph_t ^ 1, p.wait_ns, s_abort)) {
-          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        if (!hq_wait_warp_n(2, full_bar(it), full_par(it), &afree[t], ph_t ^ 1, nullptr, 0, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
         for (int rr = 0; rr < nrec; ++rr)
-          dequant_block(sR + s * kRecs + rr * kRecMax, r, p.has_zero, tmem_base + lane_addr + a_col(t) + rr * 64);
+          dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tmem_base + lane_addr + a_col(t) + rr * 64);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -342,10 +373,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  }  // non-producer roles
+
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem_base, 512);
+  if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
 template <int NTOK>
@@ -360,8 +393,7 @@ hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStre
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  kern<<<grid, kThreads, smem, stream>>>(map, p);
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, map, p) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
 int dense_tiles(const hq_quant_desc& d, int m, int ntok) {

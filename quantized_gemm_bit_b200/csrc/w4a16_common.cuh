@@ -162,9 +162,10 @@ __device__ __forceinline__ void store_chunk(const W4Params& p, const Unit& x, fl
 // Stream-K fixup after a partial unit's fp32 slot has been written: each
 // epilogue warp owns 32 rows of the tile and one counter; the last
 // contributing CTA reduces every partial in CTA order, so the result does
-// not depend on arrival order (and nobody waits).
-template <int NTOK>
-__device__ __forceinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, int lane) {
+// not depend on arrival order (and nobody waits).  Not inlined: its
+// registers stay out of the pipelined roles' allocation.
+template <int NTOK, int CB = 4>
+__device__ __noinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, int lane) {
   const int r = q * 32 + lane;
   const int n = x.nt * kTileN + r;
   const bool n_ok = n < p.n;
@@ -183,24 +184,35 @@ __device__ __forceinline__ void sk_fixup(const W4Params& p, const Unit& x, int q
   is_last = __shfl_sync(0xffffffffu, is_last, 0);
   if (!is_last) return;
   __threadfence();
-  // 16 token rows at a time, every contributor's loads in flight together;
-  // the sum runs in contributor order
-  for (int j0 = 0; j0 < x.rows; j0 += 16) {
-    float acc[16];
+  // 8 token rows at a time; the loads of up to CB contributors are in
+  // flight together and the sum runs in contributor order
+  for (int j0 = 0; j0 < x.rows; j0 += 8) {
+    float acc[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.f;
-    for (long long ci = first; ci <= last; ++ci) {
-      const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
-      const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kTileN + r;
-      float v[16];
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    for (long long c0 = first; c0 <= last; c0 += CB) {
+      float v[CB][8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = __ldcg(src + (size_t)j * kTileN);
+      for (int b = 0; b < CB; ++b) {
+        if (c0 + b <= last) {
+          const long long ci = c0 + b;
+          const int sl = sk_start(ci, T, G) >= t0 ? 0 : 1;
+          const float* src = p.partials + (((size_t)ci * 2 + sl) * NTOK + j0) * kTileN + r;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j] += v[j];
+          for (int j = 0; j < 8; ++j) v[b][j] = __ldcg(src + (size_t)j * kTileN);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < CB; ++b) {
+        if (c0 + b <= last) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j] += v[b][j];
+        }
+      }
     }
     if (n_ok) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j)
+      for (int j = 0; j < 8; ++j)
         if (j0 + j < x.rows) p.c[(size_t)(x.row0 + j0 + j) * p.n + n] = __float2bfloat16_rn(acc[j]);
     }
   }

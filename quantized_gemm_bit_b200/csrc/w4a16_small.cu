@@ -60,6 +60,12 @@ struct SmallCfg {
   static constexpr int kUnpackWarps = NTOK <= 32 ? 16 : 8;
   static constexpr int kThreads = (8 + kUnpackWarps) * 32;
   static constexpr int kChunks = 4 * kKps * 4 / kUnpackWarps;   // 32-K chunks per unpacking warp
+  // false: warp 1 issues every MMA.  true: the last unpacking warp to
+  // finish a stage issues that stage's MMAs (stages write separate result
+  // tiles, so MMAs of different stages need no order among themselves);
+  // measured slower on B200 (single-lane issue from a busy warp), kept as an
+  // option for other tile shapes
+  static constexpr bool kSelfIssue = false;
   static constexpr int kEpiScratch = 4 * 2048;          // warp-local transposes of the output
   static constexpr int kBarBytes = 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
@@ -69,7 +75,8 @@ struct SmallCfg {
   static constexpr size_t kSmem = 1024 + kScrOff + kEpiScratch;
   static_assert(kABlock % 1024 == 0 && kRecMax % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
   static_assert(kACols * kAStages + kDCols * kDStages <= 512, "TMEM budget");
-  static_assert(8 * (2 * kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 <= kBarBytes, "barrier area");
+  static_assert(8 * (2 * kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 + 4 * kAStages <= kBarBytes,
+                "barrier area");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -130,6 +137,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort + 1);
+  uint32_t* s_done = reinterpret_cast<uint32_t*>(s_total + 1);   // [AS] unpacked shares per TMEM stage
   int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);  // [kMaxExperts + 1]
   int* s_off = s_prefix + (kMaxExperts + 1);                    // [kMaxExperts + 1]
   uint16_t* epi_scratch = reinterpret_cast<uint16_t*>(smem + C::kScrOff);  // 16-byte aligned
@@ -150,49 +158,69 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
       mbar_init(&dfull[d], 1);
       mbar_init(&dempty[d], 4);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, C::kSelfIssue ? C::kUnpackWarps : 1);
+    for (int t = 0; t < AS; ++t) s_done[t] = 0;
     *s_abort = 0;
     *s_total = 0;
     fence_mbar_init();
   }
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_a);
-  if (warp == 2) {
-    tmem_alloc(s_tmem, 512);
-    tmem_relinquish();
+  // Everything but the packed weights may be written by the previous kernel
+  // on the stream: grouped mode needs the expert offsets at once
+  if (p.grouped) {
+    pdl_wait();
+    grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
   }
-  if (p.grouped) grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *s_tmem;
+  __syncthreads();   // barriers (and the grouped tables) visible to every role
   const int total_grouped = *s_total;
-
-  auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * C::kACols); };
-  auto d_col = [](int d) -> uint32_t { return (uint32_t)(AS * C::kACols + d * C::kDCols); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (whole warp, elected lane issues)
     const bool leader = elect_one();
     const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_last();
+    Unit x;
+    // Phase 1, before the previous kernel has finished: the packed weights
+    // of the first SS stages (no kernel writes them)
+    uint32_t n_pre = 0;
+    if (!p.grouped) {
+      for (int idx = 0; n_pre < (uint32_t)SS && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+        const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
+        for (int kb = x.kb0; kb < x.kb1 && n_pre < (uint32_t)SS; kb += KPS, ++n_pre) {
+          const int nrec = min(KPS, x.kb1 - kb);
+          if (leader) {
+            mbar_arrive_expect_tx(&full[n_pre], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+            bulk_g2s(sR + n_pre * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes),
+                     &full[n_pre], pol_w);
+          }
+          __syncwarp();
+        }
+      }
+      pdl_wait();
+    }
+    // Phase 2: the activations of those stages, then the steady ring
     uint32_t it = 0;
     bool ok = true;
-    Unit x;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
       const uint8_t* wbase =
           p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp(&empty[s], ((it / SS) & 1) ^ 1, p.wait_ns, s_abort)) {
+        if (it >= n_pre && !hq_wait_warp(&empty[s], ((it / SS) & 1) ^ 1, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         if (leader) {
-          mbar_arrive_expect_tx(&full[s], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+          if (it >= n_pre) {
+            mbar_arrive_expect_tx(&full[s], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+            // the stage's records are consecutive in the blob: one bulk copy
+            // (long copies stream HBM much faster than record-sized ones)
+            bulk_g2s(sR + s * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), &full[s],
+                     pol_w);
+          }
           for (int r = 0; r < nrec; ++r) {
-            bulk_g2s(sR + s * kRecs + r * kRecMax, wbase + (uint64_t)(kb + r) * p.rec_bytes, (uint32_t)p.rec_bytes,
-                     &full[s], pol_w);
             uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
             tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, &full[s]);
             tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, &full[s]);
@@ -206,7 +234,41 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
       const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
       for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
     }
-  } else if (warp == 1) {
+  } else {
+  // The producer needs no TMEM, so it starts loading at once; the other
+  // roles wait here for the allocation.
+  if (warp == 2) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (!p.grouped) pdl_wait();   // outputs, partials and counters may be in use by the previous kernel
+  tc_fence_before();
+  named_bar(1, C::kThreads - 32);
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * C::kACols); };
+  auto d_col = [](int d) -> uint32_t { return (uint32_t)(AS * C::kACols + d * C::kDCols); };
+  // MMAs of one stage (called by a single thread): record r of the stage
+  // writes a fresh fp32 tile D(d, r) = W_r^T-slice x A_r, eight K=16 steps;
+  // descriptors advance by constants: 32 B per 16-K step inside a 128-byte
+  // swizzle row, one box (NTOK rows) per 64 K
+  auto issue_stage = [&](int s, int t, int d, int nrec) {
+    const uint64_t b0 = smem_desc_sw128(smem_u32(sA + s * kATile));
+    const uint32_t a0 = tmem_base + a_col(t);
+    const uint32_t d0 = tmem_base + d_col(d);
+    for (int r = 0; r < nrec; ++r) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint64_t bdesc = b0 + (uint64_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
+        mma_bf16_ts(d0 + r * NTOK, a0 + r * 64 + j * 8, bdesc, kIdesc, j > 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(&empty[s]);
+    tc_commit(&afree[t]);
+    tc_commit(&dfull[d]);
+  };
+
+  if (warp == 1 && !C::kSelfIssue) {
     // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
     // one lane, fixed for the whole kernel, issues every MMA and commit: a
     // commit tracks the tcgen05 operations of the thread that issues it
@@ -218,31 +280,14 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, t = it % AS, d = it % DS;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp(&aready[t], (it / AS) & 1, p.wait_ns, s_abort) ||
-            !hq_wait_warp(&full[s], (it / SS) & 1, p.wait_ns, s_abort) ||
-            !hq_wait_warp(&dempty[d], ((it / DS) & 1) ^ 1, p.wait_ns, s_abort)) {
+        if (!hq_wait_warp_n(3, &aready[t], (it / AS) & 1, &full[s], (it / SS) & 1, &dempty[d],
+                            ((it / DS) & 1) ^ 1, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        if (leader) {
-          // descriptors advance by constants: 32 B per 16-K step inside a
-          // 128-byte swizzle row, one box (NTOK rows) per 64 K
-          const uint64_t b0 = smem_desc_sw128(smem_u32(sA + s * kATile));
-          const uint32_t a0 = tmem_base + a_col(t);
-          const uint32_t d0 = tmem_base + d_col(d);
-          for (int r = 0; r < nrec; ++r) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint64_t bdesc = b0 + (uint64_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
-              mma_bf16_ts(d0 + r * NTOK, a0 + r * 64 + j * 8, bdesc, kIdesc, j > 0 ? 1u : 0u);
-            }
-          }
-          tc_commit(&empty[s]);
-          tc_commit(&afree[t]);
-          tc_commit(&dfull[d]);
-        }
+        if (leader) issue_stage(s, t, d, nrec);
         __syncwarp();
       }
     }
@@ -273,21 +318,50 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
         // full[s] cannot move on before this warp's own arrival (through the
         // MMA it enables) and afree[t] before the MMA it enables: every
         // phase of both is observed in order
-        if (!hq_wait(&full[s], (it / SS) & 1, p.wait_ns, s_abort) ||
-            !hq_wait(&afree[t], ((it / AS) & 1) ^ 1, p.wait_ns, s_abort)) {
-          raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        if (!hq_wait_warp_n(2, &full[s], (it / SS) & 1, &afree[t], ((it / AS) & 1) ^ 1, nullptr, 0, p.wait_ns,
+                            s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
         if (h < nrec)
-          unpack_codes<NCH>(sR + s * kRecs + h * kRecMax, c0, r, p.has_zero,
+          unpack_codes<NCH>(sR + s * kRecs + h * p.rec_bytes, c0, r, p.has_zero,
                             tmem_base + lane_addr + a_col(t) + h * 64);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&aready[t]);
+        if constexpr (!C::kSelfIssue) {
+          if (lane == 0) mbar_arrive(&aready[t]);
+        } else {
+          // count this warp's share; the warp completing the stage issues its
+          // MMAs (fence, relaxed atomic, fence: the other warps' TMEM stores
+          // are ordered before the MMAs that read them)
+          uint32_t last = 0;
+          if (lane == 0) {
+            __threadfence_block();
+            last = (atomicAdd(&s_done[t], 1u) + 1) % C::kUnpackWarps == 0;
+            if (last) __threadfence_block();
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            const int d = it % DS;
+            if (!hq_wait_warp(&dempty[d], ((it / DS) & 1) ^ 1, p.wait_ns, s_abort)) {
+              if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (lane == 0) issue_stage(s, t, d, nrec);
+            __syncwarp();
+          }
+        }
       }
+    }
+    if constexpr (C::kSelfIssue) {
+      // no MMA this warp issued may still run when TMEM is released
+      if (lane == 0) tc_commit(drain);
+      __syncwarp();
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ scale warps + epilogue (warps 4-7)
@@ -313,7 +387,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
         float sc[KPS];
 #pragma unroll
         for (int rr = 0; rr < KPS; ++rr)
-          sc[rr] = rr < nrec ? __half2float(reinterpret_cast<const __half*>(sR + s * kRecs + rr * kRecMax +
+          sc[rr] = rr < nrec ? __half2float(reinterpret_cast<const __half*>(sR + s * kRecs + rr * p.rec_bytes +
                                                                             kW4RecCodes)[r])
                              : 0.f;
         __syncwarp();
@@ -356,14 +430,19 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
         for (int j = 0; j < CH; ++j) v[j] = acc[j0 + j];
         store_chunk<CH>(p, x, part, (int)q, (int)lane, j0, v, scr);
       }
-      if (x.partial) sk_fixup<NTOK>(p, x, (int)q, (int)lane);
+      if (x.partial) sk_fixup<NTOK, (C::kThreads > 512 ? 2 : 4)>(p, x, (int)q, (int)lane);
     }
   }
+
+  }  // non-producer roles
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem_base, 512);
+  if (warp == 2) {
+    if constexpr (C::kSelfIssue) hq_wait_warp(drain, 0, p.wait_ns, nullptr);
+    tmem_dealloc(*s_tmem, 512);
+  }
 }
 
 template <int NTOK>
@@ -378,8 +457,9 @@ hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cu
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  kern<<<grid, SmallCfg<NTOK>::kThreads, smem, stream>>>(map, p);
-  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(SmallCfg<NTOK>::kThreads), smem, stream, map, p) == cudaSuccess
+             ? HQ_OK
+             : HQ_ERR_CUDA;
 }
 
 }  // namespace

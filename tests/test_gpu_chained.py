@@ -1,0 +1,92 @@
+"""Back-to-back GEMM calls on one stream, each consuming what the kernel just
+before it wrote (the GEMM kernels start early as programmatic dependents of
+that kernel and must still read its results): a torch kernel rewrites the
+activations, GEMM 1 reads them, GEMM 2 reads GEMM 1's output.  Every result
+is checked against the fp64 oracle, the second GEMM on the first one's
+actual bf16 output."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import check_gemm, workspace
+from oracle import formats as F
+from oracle import gemm as G
+from quantized_gemm_bit_b200 import hq, synth
+from quantized_gemm_bit_b200.build import build
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    build()
+    torch.cuda.init()
+
+
+def _bits(a):
+    return a.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _w4(n, k, seed):
+    q, s, z = synth.w4a16_weights(n, k, 128, True, seed)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 1, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(DEV)
+    return d, blob, (q.numpy(), s.numpy(), z.numpy())
+
+
+@pytest.mark.parametrize("m,variant", [(16, 0), (16, 1), (48, 0), (300, 0)])
+def test_chained_w4a16_calls_read_fresh_inputs(m, variant):
+    k1, n1, n2 = 512, 1024, 384
+    d1, b1, w1 = _w4(n1, k1, 700 + m)
+    d2, b2, w2 = _w4(n2, n1, 710 + m)
+    t = hq.Tuning(variant=variant) if variant else None
+    reps = 6
+    xs = [synth.bf16_normal(m, k1, 720 + m + r).to(DEV) for r in range(reps)]
+    x = torch.empty(m, k1, dtype=torch.bfloat16, device=DEV)
+    y1 = torch.empty(m, n1, dtype=torch.bfloat16, device=DEV)
+    y2 = torch.empty(m, n2, dtype=torch.bfloat16, device=DEV)
+    ws1 = workspace(hq.hq_workspace_size(d1, m, t))
+    ws2 = workspace(hq.hq_workspace_size(d2, m, t))
+    outs = []
+    for r in range(reps):
+        torch.add(xs[r], 0.0, out=x)                       # a kernel writes the activations
+        hq.hq_gemm_w4a16(d1, b1, x, m, y1, ws1, t)         # reads them
+        hq.hq_gemm_w4a16(d2, b2, y1, m, y2, ws2, t)        # reads GEMM 1's output
+        outs.append((y1.clone(), y2.clone()))
+    torch.cuda.synchronize()
+    assert hq.hq_check_device_status(ws1) == hq.HQ_OK
+    assert hq.hq_check_device_status(ws2) == hq.HQ_OK
+    for r, (o1, o2) in enumerate(outs):
+        check_gemm(o1, G.w4a16_ref(_bits(xs[r]), *w1, 128), k1, f"chain m={m} rep={r} gemm1")
+        check_gemm(o2, G.w4a16_ref(_bits(o1), *w2, 128), n1, f"chain m={m} rep={r} gemm2")
+
+
+def test_chained_nvfp4_quantize_then_gemm():
+    """The activation quantizer writes codes and scales, the scale re-layout
+    and the GEMM read them right after."""
+    m, n, k = 64, 256, 1024
+    x = synth.bf16_normal(n, k, 730).float().numpy()
+    wc, wsf, wg = F.nvfp4_quantize(x)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, n, k, 16, 0, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, F.fp4_pack_bytes(wc), wsf, None, float(wg))).to(DEV)
+    c = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, m))
+    codes = torch.empty(m, k // 2, dtype=torch.uint8, device=DEV)
+    sf = torch.empty(m, k // 16, dtype=torch.uint8, device=DEV)
+    g = torch.empty(1, dtype=torch.float32, device=DEV)
+    wsq = workspace(hq.hq_quantize_nvfp4_workspace_size(m, k))
+    for r in range(3):
+        a = synth.bf16_normal(m, k, 740 + r).to(DEV)
+        hq.hq_quantize_nvfp4(a, m, k, codes, sf, g, wsq)
+        # the tensor scale stays on the device: pass it through the host once
+        # per call, as a caller would
+        torch.cuda.synchronize()
+        hq.hq_gemm_nvfp4(d, blob, codes, sf, float(g.item()), m, c, ws)
+        got = c.clone()
+        torch.cuda.synchronize()
+        assert hq.hq_check_device_status(ws) == hq.HQ_OK
+        ref = G.nvfp4_ref(codes.cpu().numpy(), sf.cpu().numpy(), float(g.item()), F.fp4_pack_bytes(wc), wsf,
+                          float(wg))
+        check_gemm(got, ref, k, f"nvfp4 chain rep={r}")
