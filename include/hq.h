@@ -106,12 +106,14 @@ typedef struct {
  *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
  *              splits the whole iteration space evenly when 0)
  *   cta_group: 1 (one SM per MMA)
- *   variant  : W4A16 / grouped MoE: 0 = token tiles of up to 64 feed the
- *              exact integers (q - z) to the tensor core and apply each
- *              group's scale to the fp32 group sums; larger tiles rescale
- *              the weights to bf16, w = bf16((q - z) * s), and accumulate
- *              across K in fp32.  1 = the bf16-rescaled weights for every
- *              tile.  Block-scaled GEMMs: 0.                              */
+ *   variant  : W4A16 / grouped MoE: 0 = the library's choice, currently
+ *              the same as 1.  1 = weights rescaled to bf16 in the kernel,
+ *              w = bf16((q - z) * bf16(s)), fp32 accumulation across K.
+ *              2 = for token tiles of up to 64, the exact integers (q - z)
+ *              go to the tensor core and each 128-K group's scale is
+ *              applied to its fp32 group sum (no rounding of w or s;
+ *              slower on B200 today); larger tiles as 1.
+ *              Block-scaled GEMMs: 0.                                     */
 typedef struct {
   int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;
 } hq_tuning;

@@ -175,7 +175,7 @@ hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const 
     if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
       return HQ_ERR_UNSUPPORTED;
     if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
-        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 1)
+        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
       return HQ_ERR_UNSUPPORTED;
   }
   DeviceInfo dev{};
@@ -204,7 +204,7 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
     if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128)
       return HQ_ERR_UNSUPPORTED;
     if (t->split_k > 1 || (t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->stages != 0 ||
-        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 1)
+        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
       return HQ_ERR_UNSUPPORTED;
   }
   DeviceInfo dev{};

@@ -29,9 +29,9 @@ struct W4Config {
   int stages;   // unused (pipeline depth is fixed per token tile)
   int splits;   // 0: data parallel (whole tiles); else stream-K / split K
   int grid;     // CTAs
-  int variant;  // 0: exact (q - z) weights + per-group fp32 scaling for tiles
-                //    of <= 64 tokens, bf16-rescaled weights above;
-                // 1: bf16-rescaled weights for every tile
+  int variant;  // 0 (library's choice) and 1: bf16-rescaled weights for
+                // every tile; 2: exact (q - z) weights + per-group fp32
+                // scaling for tiles of <= 64 tokens (bf16-rescaled above)
 };
 
 struct DeviceInfo {

@@ -47,15 +47,21 @@ template <int NTOK>
 struct Cfg {
   // records (128-K blocks) per pipeline stage: two for the small token tiles,
   // whose MMAs are cheap, so the per-stage waits and commits are amortized
-  static constexpr int kKps = NTOK <= 64 ? 2 : 1;
+  static constexpr bool kCoop = false;   // see kDqGroups
+  static constexpr int kKps = kCoop && NTOK <= 32 ? 3 : NTOK <= 64 ? 2 : 1;
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
   static constexpr int kRecs = kKps * kRecMax;
-  static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
-  static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;    // 64 * kKps TMEM columns each
+  static constexpr int kSmemStages = kKps == 3 ? (NTOK == 16 ? 5 : 4)
+                                    : NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  static constexpr int kTmemStages = kKps == 3 ? 2 : NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
-  // dequantizing warpgroups: the epilogue warpgroup joins for small tiles
-  static constexpr int kDqGroups = NTOK <= 64 ? 3 : 2;
+  // Dequantizing warpgroups own alternate stages (the epilogue warpgroup
+  // joins for tiles of <= 64 tokens).  kCoop instead lets all twelve warps
+  // share every three-record stage of a 16/32-token tile (warp 4 + 4r + q:
+  // record r, rows 32q..32q+31); measured slower on B200, so off.
+  static constexpr int kDqGroups = kCoop && NTOK <= 32 ? 1 : NTOK <= 64 ? 3 : 2;
+  static constexpr int kDqWarps = kDqGroups == 1 ? 12 : 4;  // arrivals on a TMEM stage's ready barrier
   // full barriers, one per (SMEM stage, dequant group): iteration `it`
   // uses barrier (it % SS, it % NDQ), so every waiter sees each of its
   // barrier's phases in order whatever the ring depth
@@ -75,6 +81,7 @@ struct Cfg {
   static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(64 * kKps * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
   static_assert(kTmemStages % kDqGroups == 0, "every TMEM stage must always return to the same dequant group");
+  static_assert(kDqGroups != 1 || kKps * 4 == 12, "one record-quarter per dequantizing warp");
   static_assert(8 * (kFullBars + kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
 };
 
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < SS; ++s) mbar_init(&empty[s], 1);
     for (int f = 0; f < C::kFullBars; ++f) mbar_init(&full[f], 1);
     for (int t = 0; t < TS; ++t) {
-      mbar_init(&aready[t], 4);
+      mbar_init(&aready[t], C::kDqWarps);
       mbar_init(&afree[t], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -312,8 +319,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (int)(q * 32 + lane);              // weight row within the tile
     const uint32_t lane_addr = (q * 32) << 16;
     const bool epi = warp < 8;
-    const int dq = warp >= 12 ? 1 : warp >= 8 ? 0 : 2;  // dequant group index (2: epilogue warps)
+    // dequant group index (2: epilogue warps); cooperative mode: one group
+    constexpr bool kShare = NDQ == 1;                   // cooperative stages
+    const int dq = kShare ? 0 : warp >= 12 ? 1 : warp >= 8 ? 0 : 2;
     const bool does_dq = dq < NDQ;
+    const int myrec = kShare ? (int)(warp - 4) >> 2 : -1;  // cooperative stages: this warp's record
     uint32_t it = 0, uc = 0;
     bool ok = true;
     Unit x;
@@ -334,7 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         for (int rr = 0; rr < nrec; ++rr)
-          dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tmem_base + lane_addr + a_col(t) + rr * 64);
+          if (!kShare || rr == myrec)
+            dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tmem_base + lane_addr + a_col(t) + rr * 64);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -425,8 +436,9 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   // Whole tiles on persistent CTAs (no partial sums) when they fill the SMs
   // well (a 256-token tile may drop to 128 for that).  Otherwise the K range
   // is shared: large token tiles (big partial sums) split every tile into
-  // the same number of parts; small ones use stream-K over all SMs (every
-  // CTA an equal share of the (tile, k-block) space, >= 4 k-blocks each).
+  // the same number of parts when that fills the SMs; everything else uses
+  // stream-K over all SMs (every CTA an equal share of the (tile, k-block)
+  // space, >= 4 k-blocks each).
   auto dp_eff = [&](int nt) {
     const long long tl = dense_tiles(d, m, nt);
     const long long waves = (tl + dev.num_sms - 1) / dev.num_sms;
@@ -442,7 +454,14 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
     return cfg;
   }
   const bool fixed_tile = t && t->tile_m;
-  if (!fixed_tile && ntok == 256 && dp_eff(256) < 0.85 && dp_eff(128) >= 0.85) ntok = 128;
+  if (!fixed_tile && ntok == 256 && dp_eff(256) < 0.85) {
+    // 128-token tiles either fill the SMs as whole tiles, or (when 256-token
+    // tiles are too few even for an even K split to fill the SMs) share K
+    // by stream-K over every SM: faster than the under-filled split
+    const long long t256 = dense_tiles(d, m, 256);
+    if (dp_eff(128) >= 0.85 || (t256 * 2 <= dev.num_sms && t256 * (dev.num_sms / t256) < 0.85 * dev.num_sms))
+      ntok = 128;
+  }
   cfg.ntok = ntok;
   const long long tiles = dense_tiles(d, m, ntok);
   if (dp_eff(ntok) >= 0.85) {
@@ -450,7 +469,7 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
     return cfg;
   }
-  if (ntok >= 128 && tiles * 2 <= dev.num_sms) {
+  if (ntok >= 128 && tiles * 2 <= dev.num_sms && tiles * (dev.num_sms / tiles) >= 0.85 * dev.num_sms) {
     cfg.splits = (int)(dev.num_sms / tiles);
     cfg.grid = (int)std::min<long long>(tiles * cfg.splits, tiles * kbs);
     return cfg;
@@ -515,7 +534,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
 
-  if (cfg.variant == 0 && cfg.ntok <= 64) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
+  if (cfg.variant == 2 && cfg.ntok <= 64) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
   switch (cfg.ntok) {
     case 16: return launch_t<16>(map, p, cfg.grid, stream);
     case 32: return launch_t<32>(map, p, cfg.grid, stream);

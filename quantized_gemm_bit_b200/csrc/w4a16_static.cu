@@ -75,7 +75,7 @@ extern "C" hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* pa
     if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
       return HQ_ERR_UNSUPPORTED;
     if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
-        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 1)
+        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
       return HQ_ERR_UNSUPPORTED;
   }
   DeviceInfo dev{};

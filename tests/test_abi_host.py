@@ -124,7 +124,7 @@ def test_gemm_argument_errors_need_no_gpu():
     t = hq.Tuning(tile_m=48)
     assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                             None) == hq.HQ_ERR_UNSUPPORTED
-    for bad in (hq.Tuning(variant=2), hq.Tuning(variant=-1), hq.Tuning(stages=3), hq.Tuning(cta_group=2)):
+    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=3), hq.Tuning(cta_group=2)):
         assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
                                 None) == hq.HQ_ERR_UNSUPPORTED
     # grouped: no 256-token tile; block-scaled: no variants

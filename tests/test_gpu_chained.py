@@ -36,7 +36,7 @@ def _w4(n, k, seed):
     return d, blob, (q.numpy(), s.numpy(), z.numpy())
 
 
-@pytest.mark.parametrize("m,variant", [(16, 0), (16, 1), (48, 0), (300, 0)])
+@pytest.mark.parametrize("m,variant", [(16, 0), (16, 2), (48, 0), (48, 2), (300, 0)])
 def test_chained_w4a16_calls_read_fresh_inputs(m, variant):
     k1, n1, n2 = 512, 1024, 384
     d1, b1, w1 = _w4(n1, k1, 700 + m)

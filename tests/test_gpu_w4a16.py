@@ -67,19 +67,19 @@ def test_ragged_shapes_full_output(m, n, k, asym):
     check_gemm(c, ref, k, f"m={m} n={n} k={k}")
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [1, 2])
 @pytest.mark.parametrize("tile_m", [16, 32, 64, 128, 256])
 def test_every_token_tile(tile_m, variant):
-    """Every token tile of both kernels: variant 0 feeds exact (q - z) and
-    scales per group in fp32 for tiles <= 64; variant 1 rescales weights to
-    bf16 for every tile."""
+    """Every token tile of both kernels: variant 1 rescales weights to bf16
+    for every tile; variant 2 feeds exact (q - z) and scales per group in
+    fp32 for tiles <= 64."""
     m, n, k = 70, 384, 1024
     d, blob, a, (q, s, z) = make_case(m, n, k, True, 7)
     c, _ = run(d, blob, a, m, hq.Tuning(tile_m=tile_m, variant=variant))
     check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"tile_m={tile_m} variant={variant}")
 
 
-@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("variant", [1, 2])
 @pytest.mark.parametrize("splits", [2, 3, 7])
 def test_split_k_and_determinism(splits, variant):
     m, n, k = 20, 256, 1792
