@@ -379,18 +379,25 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         const uint32_t b_base = smem_u32(sB(s));
         const uint32_t sf_col = C::kSfBase + s * C::kSfSlot;
         if (leader) {
+          // descriptors: the K step (32 B) and the scale chunks (512 B) only
+          // move the low word's 14-bit start-address field, which cannot
+          // overflow inside shared memory
+          const uint64_t ad = smem_desc_sw128(a_base), bd = smem_desc_sw128(b_base);
+          auto step = [](uint64_t desc, uint32_t bytes) {
+            return (desc & 0xFFFFFFFF00000000ull) | (uint64_t)((uint32_t)desc + (bytes >> 4));
+          };
+          const uint32_t acc0 = ks > ks0 ? 1u : 0u;
           if (FMT == kNV) {
+            const uint64_t fa = smem_desc_sf(smem_u32(sSfa(s))), fb = smem_desc_sf(smem_u32(sSfb(s)));
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const uint32_t sfa_t = tmem_base + sf_col + 4 * i;
               const uint32_t sfb_t = tmem_base + sf_col + 16 + 4 * C::kHalves * i;
-              tmem_cp_sf(sfa_t, smem_desc_sf(smem_u32(sSfa(s)) + 512 * i));
+              tmem_cp_sf(sfa_t, step(fa, 512 * i));
 #pragma unroll
-              for (int h = 0; h < C::kHalves; ++h)
-                tmem_cp_sf(sfb_t + 4 * h, smem_desc_sf(smem_u32(sSfb(s)) + 512 * (i * C::kHalves + h)));
+              for (int h = 0; h < C::kHalves; ++h) tmem_cp_sf(sfb_t + 4 * h, step(fb, 512 * (i * C::kHalves + h)));
               constexpr uint32_t kId = idesc_block_scaled(1, 1, 0, 128, NTOK, 0, 0);
-              mma_mxf4nvf4(d_tmem, smem_desc_sw128(a_base + 32 * i), smem_desc_sw128(b_base + 32 * i), kId, sfa_t,
-                           sfb_t, (ks > ks0 || i > 0) ? 1u : 0u);
+              mma_mxf4nvf4(d_tmem, step(ad, 32 * i), step(bd, 32 * i), kId, sfa_t, sfb_t, i > 0 ? 1u : acc0);
             }
           } else {
             const uint32_t sfa_t = tmem_base + sf_col;
@@ -399,8 +406,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
             for (int i = 0; i < 4; ++i) {
               // byte i of each scale column holds the scale of 32-K block i
               const uint32_t id = idesc_block_scaled(5, 0, 1, 128, NTOK, (uint32_t)i, 0);
-              mma_mxf8f6f4(d_tmem, smem_desc_sw128(a_base + 32 * i), smem_desc_sw128(b_base + 32 * i), id, sfa_t,
-                           tmem_base + C::kSfbConst, (ks > ks0 || i > 0) ? 1u : 0u);
+              mma_mxf8f6f4(d_tmem, step(ad, 32 * i), step(bd, 32 * i), id, sfa_t, tmem_base + C::kSfbConst,
+                           i > 0 ? 1u : acc0);
             }
           }
           tc_commit(&empty[s]);

@@ -85,14 +85,17 @@ struct Cfg {
   static_assert(8 * (kFullBars + kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
 };
 
-// Dequantize one 128-K block of the packed record for TMEM stage t: thread
-// (warp quarter q, lane) owns weight row r = 32q + lane and writes its 128
-// bf16 weights w = (q - z) * s into TMEM lane r, columns t*64 .. t*64+63
-// (two weights per 32-bit column, even k in the low half).
-__device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
-  uint4 raw[4];
+// Dequantize 32-K chunks c0 .. c0+NC-1 of one 128-K packed record: thread
+// (warp quarter q, lane) owns weight row r = 32q + lane and computes its
+// weights w = (q - z) * s as 16 words per chunk (two bf16 per 32-bit word,
+// even k in the low half); store_chunks writes them to TMEM lane r,
+// columns 16*c0 ... of the record's 64.
+template <int NC>
+__device__ __forceinline__ void dequant_chunks(const uint8_t* rec, int c0, int r, int has_zero,
+                                               uint32_t (&out)[NC * 16]) {
+  uint4 raw[NC];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+  for (int c = 0; c < NC; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + ((c0 + c) * 128 + r) * 16);
   const __half sc = reinterpret_cast<const __half*>(rec + kW4RecCodes)[r];
   const uint32_t z = has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
   const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
@@ -101,9 +104,8 @@ __device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has
   const uint32_t zbits = 0x4300u + z;
   const uint32_t z2 = zbits | (zbits << 16);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < NC; ++c) {
     const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-    uint32_t out[16];
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
 #pragma unroll
@@ -111,10 +113,26 @@ __device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has
         // nibbles of k = 2j and 2j+1 sit at bits 4j and 16+4j: OR-ing them
         // into the mantissa of bf16 128.0 gives bf16(128 + q)
         const uint32_t x2 = lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u);
-        out[w * 4 + j] = bf16x2_mul(bf16x2_sub(x2, z2), s2);
+        out[c * 16 + w * 4 + j] = bf16x2_mul(bf16x2_sub(x2, z2), s2);
       }
     }
-    tmem_st_x16(taddr + c * 16, out);
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void store_chunks(const uint32_t (&w)[NC * 16], int c0, uint32_t taddr) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    tmem_st_x16(taddr + (c0 + c) * 16, *reinterpret_cast<const uint32_t(*)[16]>(w + c * 16));
+}
+
+// A whole record, chunk by chunk (dequantize 16 words, store them).
+__device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t w[16];
+    dequant_chunks<1>(rec, c, r, has_zero, w);
+    store_chunks<1>(w, c, taddr);
   }
 }
 
@@ -288,14 +306,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (leader) {
           // descriptors advance by constants: 32 B per 16-K step inside a
-          // 128-byte swizzle row, one box (NTOK rows) per 64 K
+          // 128-byte swizzle row, one box (NTOK rows) per 64 K.  Only the low
+          // word moves (its 14-bit start-address field cannot overflow inside
+          // shared memory), so each MMA costs one 32-bit add.
           const uint64_t b0 = smem_desc_sw128(smem_u32(sA + s * kATile));
+          const uint32_t blo = (uint32_t)b0, bhi = (uint32_t)(b0 >> 32);
           const uint32_t a0 = tmem_base + a_col(t);
-          for (int r = 0; r < nrec; ++r) {
+          const uint32_t acc0 = kb > x.kb0 ? 1u : 0u;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint64_t bdesc = b0 + (uint64_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
-              mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, kIdesc, (kb + r > x.kb0 || j > 0) ? 1u : 0u);
+          for (int r = 0; r < KPS; ++r) {
+            if (r < nrec) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const uint32_t off = (uint32_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
+                const uint64_t bdesc = ((uint64_t)bhi << 32) | (uint64_t)(blo + off);
+                mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, kIdesc, (r > 0 || j > 0) ? 1u : acc0);
+              }
             }
           }
           tc_commit(&empty[s]);
@@ -337,15 +363,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         // only ever serve this group, so it observes every phase of the
         // barriers it waits on, one after the other (a parity wait can only
         // tell adjacent phases apart).
-        if (!hq_wait_warp_n(2, full_bar(it), full_par(it), &afree[t], ph_t ^ 1, nullptr, 0, p.wait_ns, s_abort)) {
+        // kEarly: dequantize the first half-record into registers before the
+        // TMEM stage is known to be free, overlapping that wait with the
+        // arithmetic; off, because the busier dequant warps then take issue
+        // slots from the MMA warp on the same sub-partition (measured slower).
+        constexpr bool kEarly = false;   // measured slower: the MMA warp loses issue slots
+        if (!hq_wait_warp_n(kEarly ? 1 : 2, full_bar(it), full_par(it), &afree[t], ph_t ^ 1, nullptr, 0, p.wait_ns,
+                            s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
-        tc_fence_after();
-        for (int rr = 0; rr < nrec; ++rr)
-          if (!kShare || rr == myrec)
-            dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tmem_base + lane_addr + a_col(t) + rr * 64);
+        const int r0 = kShare ? myrec : 0;
+        const uint32_t tbase = tmem_base + lane_addr + a_col(t);
+        if constexpr (kEarly) {
+          uint32_t wreg[32];
+          if (r0 < nrec) dequant_chunks<2>(sR + s * kRecs + r0 * p.rec_bytes, 0, r, p.has_zero, wreg);
+          if (!hq_wait_warp_n(1, &afree[t], ph_t ^ 1, nullptr, 0, nullptr, 0, p.wait_ns, s_abort)) {
+            if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (r0 < nrec) {
+            store_chunks<2>(wreg, 0, tbase + r0 * 64);
+            dequant_chunks<2>(sR + s * kRecs + r0 * p.rec_bytes, 2, r, p.has_zero, wreg);
+            store_chunks<2>(wreg, 2, tbase + r0 * 64);
+          }
+        } else {
+          tc_fence_after();
+          if (r0 < nrec) dequant_block(sR + s * kRecs + r0 * p.rec_bytes, r, p.has_zero, tbase + r0 * 64);
+        }
+        if (!kShare) {
+          for (int rr = 1; rr < nrec; ++rr)
+            dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -453,18 +505,16 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
     cfg.grid = (int)std::max<long long>(1, std::min<long long>(tiles * t->split_k, tiles * kbs));
     return cfg;
   }
+  // Large tiles keep whole tiles down to 70 % of the SMs busy: their
+  // partial sums are big, and measured, whole tiles beat a shared K range
+  // there (M=256, K=18432, N=7168: 128-token whole tiles on 112 SMs take
+  // 84 us, stream-K over 148 SMs 101 us, a 256-token 2-way split 104 us).
   const bool fixed_tile = t && t->tile_m;
-  if (!fixed_tile && ntok == 256 && dp_eff(256) < 0.85) {
-    // 128-token tiles either fill the SMs as whole tiles, or (when 256-token
-    // tiles are too few even for an even K split to fill the SMs) share K
-    // by stream-K over every SM: faster than the under-filled split
-    const long long t256 = dense_tiles(d, m, 256);
-    if (dp_eff(128) >= 0.85 || (t256 * 2 <= dev.num_sms && t256 * (dev.num_sms / t256) < 0.85 * dev.num_sms))
-      ntok = 128;
-  }
+  const double dp_min = ntok >= 128 ? 0.7 : 0.85;
+  if (!fixed_tile && ntok == 256 && dp_eff(256) < dp_min && dp_eff(128) >= dp_min) ntok = 128;
   cfg.ntok = ntok;
   const long long tiles = dense_tiles(d, m, ntok);
-  if (dp_eff(ntok) >= 0.85) {
+  if (dp_eff(ntok) >= dp_min) {
     cfg.splits = 0;  // data parallel
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
     return cfg;
