@@ -47,15 +47,24 @@ constexpr int kBsEB = 16;          // tokens per transposed output store
 
 enum BsFmt { kMX = 0, kNV = 1 };
 
+// MXFP4 stages of small token tiles carry two 128-K boxes (fewer, longer
+// stages: the per-stage handshakes dominate there); everything else one.
+template <int FMT, int NTOK>
+constexpr int bs_boxes() { return FMT == kMX && NTOK <= 64 ? 2 : 1; }
+
 template <int FMT, int NTOK>
 struct BsCfg {
-  static constexpr int kKStage = FMT == kNV ? 256 : 128;   // K elements per stage: 128 B per row in SMEM
-  static constexpr int kATile = kBsTileN * 128;            // weights in SMEM
+  static constexpr int kBox = bs_boxes<FMT, NTOK>();        // 128-B-row boxes along K per stage
+  static constexpr int kKBox = FMT == kNV ? 256 : 128;     // K elements per box: 128 B per row in SMEM
+  static constexpr int kATileBox = kBsTileN * 128;         // weights in SMEM, one box
+  static constexpr int kATile = kBox * kATileBox;
   // bytes the weight copy moves: NVFP4 loads packed bytes; the MXFP4 load
   // unpacks 4-bit codes into 16-byte slots and counts the packed bytes
-  static constexpr int kATx = FMT == kNV ? kATile : kBsTileN * 64;
-  static constexpr int kBTile = NTOK * 128;                // activations
-  static constexpr int kSfa = FMT == kNV ? 2048 : 512;     // weight scale chunks per stage
+  static constexpr int kATxBox = FMT == kNV ? kATileBox : kBsTileN * 64;
+  static constexpr int kBTileBox = NTOK * 128;             // activations, one box
+  static constexpr int kBTile = kBox * kBTileBox;
+  static constexpr int kSfaBox = FMT == kNV ? 2048 : 512;  // weight scale chunks per box
+  static constexpr int kSfa = kBox * kSfaBox;
   static constexpr int kHalves = NTOK > 128 ? 2 : 1;       // 128-token halves of the token tile
   static constexpr int kSfb = FMT == kNV ? 4 * kHalves * 512 : 0;   // activation scale chunks per stage
   static constexpr int kStageRaw = kATile + kBTile + kSfa + kSfb;
@@ -66,7 +75,7 @@ struct BsCfg {
   static constexpr int kAcc = NTOK <= 128 ? 2 : 1;
   static constexpr int kCols = NTOK / 2;                   // accumulator columns per epilogue warp
   // TMEM columns: accumulators, then per-stage scale slots
-  static constexpr int kSfaCols = FMT == kNV ? 16 : 4;
+  static constexpr int kSfaCols = FMT == kNV ? 16 : 4 * kBox;
   static constexpr int kSfbCols = FMT == kNV ? 16 * kHalves : 0;
   static constexpr int kSfSlot = kSfaCols + kSfbCols;
   static constexpr int kSfBase = kAcc * NTOK;
@@ -78,6 +87,7 @@ struct BsCfg {
   static_assert(kSfbConst + 8 <= 512, "TMEM budget");
   static_assert(8 * (2 * kStages + 5) + 16 <= kBarBytes, "barrier area");
   static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kBTileBox % 1024 == 0 && kATileBox % 1024 == 0, "128-byte swizzle atoms");
 };
 
 struct BsParams {
@@ -94,6 +104,7 @@ struct BsParams {
   long long total_iters;
   int m, n, k;
   int n_tiles, k_stages;
+  int k_boxes;               // 128-B-row boxes along K (K/256 for NVFP4, K/128 for MXFP4)
   int sf_groups;             // 512-byte scale chunks per weight tile (whole K)
   int m_tiles;
   int data_parallel;         // whole tiles per unit, no partial sums
@@ -229,7 +240,12 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   constexpr int S = C::kStages;
   constexpr int ACC = C::kAcc;
   constexpr int NC = C::kCols;
-  constexpr uint32_t kTx = C::kATx + C::kBTile + C::kSfa + C::kSfb;
+  // bytes of a stage with nb boxes
+  auto stage_tx = [](int nb) -> uint32_t {
+    return (uint32_t)(nb * (C::kATxBox + C::kBTileBox + C::kSfaBox) + C::kSfb);
+  };
+  // boxes of stage ks (the last one of an odd box count has one)
+  auto stage_boxes = [&](int ks) -> int { return min(C::kBox, p.k_boxes - ks * C::kBox); };
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -279,10 +295,15 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     // weights of stage it: codes (K coordinate in elements for the MXFP4
     // unpacking type, in bytes for NVFP4) and their scale chunks
     auto load_weights = [&](int s, int ks, int nt_) {
-      tma_load_2d(sA(s), &tmap_w, FMT == kNV ? ks * 128 : ks * C::kKStage, nt_ * kBsTileN, &full[s]);
-      const int chunks = FMT == kNV ? 4 : 1;
-      const uint8_t* src = p.sf_w + ((size_t)nt_ * p.sf_groups + (size_t)ks * chunks) * 512;
-      bulk_g2s(sSfa(s), src, C::kSfa, &full[s], pol_w);
+      const int nb = stage_boxes(ks);
+      for (int b = 0; b < nb; ++b) {
+        const int kbox = ks * C::kBox + b;
+        tma_load_2d(sA(s) + b * C::kATileBox, &tmap_w, FMT == kNV ? kbox * 128 : kbox * C::kKBox, nt_ * kBsTileN,
+                    &full[s]);
+      }
+      const int chunks = FMT == kNV ? 4 : 1;   // 512-byte scale chunks per box
+      const uint8_t* src = p.sf_w + ((size_t)nt_ * p.sf_groups + (size_t)ks * C::kBox * chunks) * 512;
+      bulk_g2s(sSfa(s), src, (uint32_t)(nb * C::kSfaBox), &full[s], pol_w);
     };
     // Phase 1, before the previous kernel on the stream has finished: the
     // packed weights of the first S stages (no kernel writes them)
@@ -291,7 +312,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
          ++idx) {
       for (int ks = ks0; ks < ks1 && n_pre < (uint32_t)S; ++ks, ++n_pre) {
         if (leader) {
-          mbar_arrive_expect_tx(&full[n_pre], kTx);
+          mbar_arrive_expect_tx(&full[n_pre], stage_tx(stage_boxes(ks)));
           load_weights((int)n_pre, ks, nt);
         }
         __syncwarp();
@@ -312,10 +333,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         }
         if (leader) {
           if (it >= n_pre) {
-            mbar_arrive_expect_tx(&full[s], kTx);
+            mbar_arrive_expect_tx(&full[s], stage_tx(stage_boxes(ks)));
             load_weights(s, ks, nt);
           }
-          tma_load_2d(sB(s), &tmap_a, ks * 128, row0, &full[s]);
+          for (int b = 0; b < stage_boxes(ks); ++b)
+            tma_load_2d(sB(s) + b * C::kBTileBox, &tmap_a, (ks * C::kBox + b) * 128, row0, &full[s]);
           if (FMT == kNV) {
             const uint8_t* sfb = p.sf_a + ((size_t)(row0 / NTOK) * p.k_stages + ks) * C::kSfb;
             bulk_g2s(sSfb(s), sfb, C::kSfb, &full[s], policy_evict_last());
@@ -400,14 +422,21 @@ __global__ void __launch_bounds__(kBsThreads, 1)
               mma_mxf4nvf4(d_tmem, step(ad, 32 * i), step(bd, 32 * i), kId, sfa_t, sfb_t, i > 0 ? 1u : acc0);
             }
           } else {
-            const uint32_t sfa_t = tmem_base + sf_col;
-            tmem_cp_sf(sfa_t, smem_desc_sf(smem_u32(sSfa(s))));
+            const uint64_t fa = smem_desc_sf(smem_u32(sSfa(s)));
+            const int nb = stage_boxes(ks);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              // byte i of each scale column holds the scale of 32-K block i
-              const uint32_t id = idesc_block_scaled(5, 0, 1, 128, NTOK, (uint32_t)i, 0);
-              mma_mxf8f6f4(d_tmem, step(ad, 32 * i), step(bd, 32 * i), id, sfa_t, tmem_base + C::kSfbConst,
-                           i > 0 ? 1u : acc0);
+            for (int b = 0; b < C::kBox; ++b) {
+              if (b < nb) {
+                const uint32_t sfa_t = tmem_base + sf_col + 4 * b;
+                tmem_cp_sf(sfa_t, step(fa, 512 * b));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  // byte i of each scale column holds the scale of 32-K block i
+                  const uint32_t id = idesc_block_scaled(5, 0, 1, 128, NTOK, (uint32_t)i, 0);
+                  mma_mxf8f6f4(d_tmem, step(ad, b * C::kATileBox + 32 * i), step(bd, b * C::kBTileBox + 32 * i), id,
+                               sfa_t, tmem_base + C::kSfbConst, (b > 0 || i > 0) ? 1u : acc0);
+                }
+              }
             }
           }
           tc_commit(&empty[s]);
@@ -509,6 +538,13 @@ hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const BsPara
                                                                                                  : HQ_ERR_CUDA;
 }
 
+// 128-B-row boxes along K, and pipeline stages (bs_boxes boxes each).
+long long bs_k_boxes(const hq_quant_desc& d) { return d.k / (d.fmt == HQ_FMT_NVFP4 ? 256 : 128); }
+long long bs_k_stages(const hq_quant_desc& d, int ntok) {
+  const int box = d.fmt == HQ_FMT_MXFP4 && ntok <= 64 ? 2 : 1;   // bs_boxes<FMT, NTOK>()
+  return (bs_k_boxes(d) + box - 1) / box;
+}
+
 int bs_tiles(const hq_quant_desc& d, int m, int ntok) {
   return ((d.n + kBsTileN - 1) / kBsTileN) * ((m + ntok - 1) / ntok);
 }
@@ -519,8 +555,7 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   BsConfig cfg{};
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
-  const int kstage = d.fmt == HQ_FMT_NVFP4 ? 256 : 128;
-  const long long ks = d.k / kstage;
+  const long long ks = bs_k_stages(d, ntok);
   auto dp_eff = [&](int nt) {
     const long long tl = bs_tiles(d, m, nt);
     const long long waves = (tl + dev.num_sms - 1) / dev.num_sms;
@@ -600,7 +635,8 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.n = d.n;
   p.k = d.k;
   p.n_tiles = n_tiles;
-  p.k_stages = d.k / (nv ? 256 : 128);
+  p.k_boxes = (int)bs_k_boxes(d);
+  p.k_stages = (int)bs_k_stages(d, cfg.ntok);
   const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
   p.total_iters = (long long)tiles * p.k_stages;
   p.m_tiles = (m + cfg.ntok - 1) / cfg.ntok;

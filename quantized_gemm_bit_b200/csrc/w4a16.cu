@@ -29,6 +29,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 
 #include "hq_internal.h"
@@ -470,9 +471,13 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) {
     if (grouped) {
-      // average rows per expert decides the token tile
-      const long long avg = (long long)m / std::max(1, d.num_experts);
-      ntok = avg <= 16 ? 16 : avg <= 32 ? 32 : avg <= 64 ? 64 : 128;
+      // A typical expert's rows should fit one token tile: an expert split
+      // over two tiles streams its weights twice, while a larger tile costs
+      // little more at these sizes (HBM bound).  Top-k routing gives about
+      // Poisson(avg) rows per expert, so the tile covers avg + 2 sd.
+      const double avg = (double)m / std::max(1, d.num_experts);
+      const double want = avg + 2.0 * std::sqrt(avg);
+      ntok = want <= 16 ? 16 : want <= 32 ? 32 : want <= 64 ? 64 : 128;
     } else {
       ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
     }
