@@ -344,7 +344,9 @@ def _time_launches(launches, steps, warmup, world, ncopy=1):
       * per launch: one graph of R = max(ncopy, 4) back-to-back launches of
         it (copies rotating), replayed three times between two events while
         a fourth replay queued before them keeps the GPU busy; the mean
-        duration includes the launch gaps inside the graph.
+        duration includes the launch gaps inside the graph.  Each launch is
+        timed alone: the GPU idles for 0.2 s first, so a small GEMM is not
+        measured at the clocks the power cap left after a large one.
     Returns (total ms over `steps`, per-launch mean microseconds)."""
     stream = torch.cuda.current_stream()
     for i in range(max(1, warmup)):        # host-side first-call setup happens here, outside capture
@@ -377,6 +379,7 @@ def _time_launches(launches, steps, warmup, world, ncopy=1):
         stream.wait_stream(side)
         g.replay()
         torch.cuda.synchronize()
+        time.sleep(0.2)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         g.replay()                      # keeps the GPU busy while the timed replays are queued
         a.record(stream)

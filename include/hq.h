@@ -107,12 +107,14 @@ typedef struct {
  *              splits the whole iteration space evenly when 0)
  *   cta_group: 1 (one SM per MMA)
  *   variant  : W4A16 / grouped MoE: 0 = the library's choice, currently
- *              the same as 1.  1 = weights rescaled to bf16 in the kernel,
+ *              2 for 64-token tiles and 1 for every other tile.
+ *              1 = weights rescaled to bf16 in the kernel,
  *              w = bf16((q - z) * bf16(s)), fp32 accumulation across K.
  *              2 = for token tiles of up to 64, the exact integers (q - z)
  *              go to the tensor core and each 128-K group's scale is
  *              applied to its fp32 group sum (no rounding of w or s;
- *              slower on B200 today); larger tiles as 1.
+ *              on B200 faster than 1 at 64-token tiles, slower at 16 and
+ *              32); larger tiles as 1.
  *              Block-scaled GEMMs: 0.                                     */
 typedef struct {
   int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;

@@ -29,7 +29,8 @@ struct W4Config {
   int stages;   // unused (pipeline depth is fixed per token tile)
   int splits;   // 0: data parallel (whole tiles); else stream-K / split K
   int grid;     // CTAs
-  int variant;  // 0 (library's choice) and 1: bf16-rescaled weights for
+  int variant;  // 0: library's choice (exact weights for 64-token tiles,
+                // bf16-rescaled otherwise); 1: bf16-rescaled weights for
                 // every tile; 2: exact (q - z) weights + per-group fp32
                 // scaling for tiles of <= 64 tokens (bf16-rescaled above)
 };

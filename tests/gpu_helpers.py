@@ -1,6 +1,8 @@
 """Shared helpers for the GPU parity tests: tolerance checks written out
 from the stated bars, workspace allocation and tile-covering row samples."""
 
+import os
+
 import numpy as np
 import torch
 
@@ -24,6 +26,10 @@ def check_gemm(c_bf16, ref, k, what=""):
     rms = np.sqrt(np.mean(ref ** 2))
     bound = ELEM_REL * np.abs(ref) + ELEM_ABS * np.sqrt(k) * rms
     worst = np.max(np.abs(err) - bound)
+    log = os.environ.get("HQ_PARITY_LOG")
+    if log:   # one line per check: label, rel Frobenius, worst |err| / element bound
+        with open(log, "a") as f:
+            f.write(f"{what}\t{rel:.3e}\t{np.max(np.abs(err) / np.maximum(bound, 1e-300)):.3e}\n")
     assert rel <= REL_FRO, f"{what}: rel Frobenius {rel:.3e}"
     assert worst <= 0, f"{what}: element bound exceeded by {worst:.3e}"
     return rel
