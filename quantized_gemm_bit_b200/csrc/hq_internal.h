@@ -28,6 +28,7 @@ struct W4Config {
   int ntok;     // token tile (MMA N)
   int stages;   // unused (pipeline depth is fixed per token tile)
   int splits;   // 0: data parallel (whole tiles); else stream-K / split K
+  int dp_tiles; // stream-K plans: tiles run whole before the shared K range
   int grid;     // CTAs
   int variant;  // 0: library's choice (exact weights for 64-token tiles,
                 // bf16-rescaled otherwise); 1: bf16-rescaled weights for
@@ -45,6 +46,9 @@ hq_status device_info(DeviceInfo* out);
 
 // W4A16 (dense or grouped) planning and launch.
 W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t);
+// The same token tile with whole tiles only (no partial sums, no workspace
+// beyond the header).
+W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4Config cfg);
 size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bool grouped);
 hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m,
                     void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream);

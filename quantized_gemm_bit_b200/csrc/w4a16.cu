@@ -537,6 +537,21 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   cfg.ntok = ntok;
   const long long tiles = dense_tiles(d, m, ntok);
   if (dp_eff(ntok) >= dp_min) {
+    const long long waves = tiles / dev.num_sms, rest = tiles % dev.num_sms;
+    if (waves >= 2 && rest != 0 && dp_eff(ntok) < 0.95) {
+      // Whole tiles for all waves but the last full one; that wave and the
+      // ragged rest share their K range stream-K style (every CTA one to two
+      // tiles' worth, each tile split over at most three CTAs), so no SM
+      // idles through a mostly empty last wave.  Measured: M=4096, K=18432,
+      // N=7168 (896 tiles = 6 waves + 8) 831 -> 799 us.  Not with a single
+      // full wave (M=1024, K=18432: 224 tiles, 232 -> 238 us): under the
+      // power cap the SMs of a part-empty last wave run at higher clocks,
+      // and the shared K range pays for partial sums.
+      cfg.splits = 1;
+      cfg.dp_tiles = (int)((waves - 1) * dev.num_sms);
+      cfg.grid = dev.num_sms;
+      return cfg;
+    }
     cfg.splits = 0;  // data parallel
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
     return cfg;
@@ -548,6 +563,13 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   }
   cfg.splits = 1;
   cfg.grid = (int)std::max<long long>(1, std::min<long long>(dev.num_sms, tiles * kbs / 4));
+  return cfg;
+}
+
+W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4Config cfg) {
+  cfg.splits = 0;
+  cfg.dp_tiles = 0;
+  cfg.grid = (int)std::min<long long>(dev.num_sms, dense_tiles(d, m, cfg.ntok));
   return cfg;
 }
 
@@ -585,7 +607,8 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
     p.weights_once = (long long)m <= (long long)cfg.ntok * d.num_experts ? 1 : 0;
   } else {
     const size_t tiles = (size_t)dense_tiles(d, m, cfg.ntok);
-    p.total_iters = (long long)tiles * p.k_blocks;
+    p.dp_tiles = cfg.splits == 0 ? 0 : cfg.dp_tiles;
+    p.total_iters = (long long)(tiles - (size_t)p.dp_tiles) * p.k_blocks;
     p.weights_once = p.m_tiles == 1 ? 1 : 0;
     p.data_parallel = cfg.splits == 0 ? 1 : 0;
     uint8_t* base = static_cast<uint8_t*>(ws) + sizeof(WsHeader);

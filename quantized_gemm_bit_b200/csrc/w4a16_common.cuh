@@ -33,7 +33,8 @@ struct W4Params {
   uint32_t* err;
   uint64_t expert_bytes;
   uint64_t wait_ns;
-  long long total_iters;             // dense: tiles * k_blocks
+  long long total_iters;             // dense stream-K: k-block iterations after the whole tiles
+  int dp_tiles;                      // dense stream-K: tiles run whole first (a multiple of the grid)
   int m;                             // dense: rows of A; grouped: total sorted rows
   int n;                             // output columns
   int n_tiles, k_blocks, m_tiles;
@@ -62,10 +63,7 @@ struct Unit {
 template <int NTOK>
 __device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix, const int* s_off, int total_grouped,
                                          int idx, Unit& x) {
-  if (!p.grouped && p.data_parallel) {
-    // whole tiles, strided over the persistent CTAs
-    const long long tile = (long long)blockIdx.x + (long long)idx * gridDim.x;
-    if (tile >= (long long)p.m_tiles * p.n_tiles) return false;
+  auto whole = [&](long long tile) {
     const int mt = (int)(tile / p.n_tiles);
     x.tile = (int)tile;
     x.nt = (int)(tile - (long long)mt * p.n_tiles);
@@ -76,26 +74,42 @@ __device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix,
     x.kb1 = p.k_blocks;
     x.partial = 0;
     x.slot = 0;
+  };
+  if (!p.grouped && p.data_parallel) {
+    // whole tiles, strided over the persistent CTAs
+    const long long tile = (long long)blockIdx.x + (long long)idx * gridDim.x;
+    if (tile >= (long long)p.m_tiles * p.n_tiles) return false;
+    whole(tile);
     return true;
   }
   if (!p.grouped) {
-    const long long T = p.total_iters, G = gridDim.x, i = blockIdx.x;
+    const long long G = gridDim.x, i = blockIdx.x;
+    // first the whole tiles of the leading waves (none for plain stream-K)
+    const int dp_per = p.dp_tiles / (int)G;
+    if (idx < dp_per) {
+      whole(i + (long long)idx * G);
+      return true;
+    }
+    // then this CTA's share of the k-block iterations of the remaining tiles
+    const int sidx = idx - dp_per;
+    const long long T = p.total_iters;
     const long long beg = sk_start(i, T, G), end = sk_start(i + 1, T, G);
     const long long kb = p.k_blocks;
-    const long long tile = beg / kb + idx;
-    const long long x0 = idx == 0 ? beg : tile * kb;
+    const long long rel = beg / kb + sidx;
+    const long long x0 = sidx == 0 ? beg : rel * kb;
     if (x0 >= end) return false;
-    const long long x1 = min(end, (tile + 1) * kb);
+    const long long x1 = min(end, (rel + 1) * kb);
+    const long long tile = p.dp_tiles + rel;
     const int mt = (int)(tile / p.n_tiles);
     x.tile = (int)tile;
     x.nt = (int)(tile - (long long)mt * p.n_tiles);
     x.expert = 0;
     x.row0 = mt * NTOK;
     x.rows = min(NTOK, p.m - x.row0);
-    x.kb0 = (int)(x0 - tile * kb);
-    x.kb1 = (int)(x1 - tile * kb);
+    x.kb0 = (int)(x0 - rel * kb);
+    x.kb1 = (int)(x1 - rel * kb);
     x.partial = (x.kb0 != 0 || x.kb1 != p.k_blocks) ? 1 : 0;
-    x.slot = idx == 0 ? 0 : 1;
+    x.slot = sidx == 0 ? 0 : 1;
     return true;
   }
   const int u = blockIdx.x + idx * gridDim.x;
@@ -170,7 +184,7 @@ __device__ __noinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, i
   const int n = x.nt * kTileN + r;
   const bool n_ok = n < p.n;
   const long long T = p.total_iters, G = gridDim.x, kbl = p.k_blocks;
-  const long long t0 = (long long)x.tile * kbl;
+  const long long t0 = (long long)(x.tile - p.dp_tiles) * kbl;   // in the stream-K iteration space
   const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kbl - 1, T, G);
   const int cnt = (int)(last - first + 1);
   __threadfence();

@@ -81,7 +81,11 @@ extern "C" hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* pa
   DeviceInfo dev{};
   hq_status st = device_info(&dev);
   if (st != HQ_OK) return st;
-  const W4Config cfg = w4_plan(dev, *d, m, false, t);
+  W4Config cfg = w4_plan(dev, *d, m, false, t);
+  // a whole-tile plan with a stream-K tail falls back to whole tiles when
+  // its partial sums would not fit the scratch array
+  if (cfg.splits != 0 && cfg.dp_tiles > 0 && w4_workspace_bytes(*d, m, cfg, false) > kHqStaticScratchBytes)
+    cfg = w4_whole_tiles(dev, *d, m, cfg);
   const size_t need = w4_workspace_bytes(*d, m, cfg, false);
   if (need > kHqStaticScratchBytes) return HQ_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = static_scratch_address(dev.device);

@@ -106,6 +106,20 @@ def test_stream_k_repeats_bit_for_bit(m):
     check_gemm(c1, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"stream-K m={m}")
 
 
+@pytest.mark.parametrize("m,n,k", [(512, 25600, 256), (700, 14080, 384)])
+def test_whole_waves_then_stream_k_tail(m, n, k):
+    """Default plans whose whole-tile waves would leave the last wave part
+    empty on 148 SMs (400 and 330 tiles of 256 tokens, the second with a
+    ragged last token tile): whole tiles first, then the remaining tiles'
+    K range shared stream-K style.  Full output, repeated bit for bit."""
+    d, blob, a, (q, s, z) = make_case(m, n, k, False, 17 + n)
+    assert hq.hq_workspace_size(d, m) > (1 << 20)     # partial sums: not a whole-tile plan
+    c1, _ = run(d, blob, a, m)
+    c2, _ = run(d, blob, a, m)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"stream-K tail m={m} n={n} k={k}")
+
+
 def test_guard_bands_untouched():
     m, n, k = 33, 200, 512
     d, blob, a, (q, s, z) = make_case(m, n, k, True, 11)
