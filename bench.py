@@ -52,6 +52,28 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# DRAM bytes (read + write) per launch of the sweep GEMMs, from one ncu
+# capture of the bench's first warm-up step (cold caches), recorded in
+# profiles/traffic_w4a16_sweep.md.  Emptied whenever the kernels change, so
+# that `traffic` reads null until the capture is taken again.
+TRAFFIC_BYTES = {
+    (1, 7168, 18432): 69798400,
+    (4, 7168, 18432): 68901376,
+    (16, 7168, 18432): 69559296,
+    (64, 7168, 18432): 70421504,
+    (256, 7168, 18432): 75667200,
+    (1024, 7168, 18432): 165391872,
+    (4096, 7168, 18432): 445985280,
+    (1, 18432, 7168): 69426432,
+    (4, 18432, 7168): 69673216,
+    (16, 18432, 7168): 70456832,
+    (64, 18432, 7168): 73549312,
+    (256, 18432, 7168): 86308864,
+    (1024, 18432, 7168): 201157376,
+    (4096, 18432, 7168): 723845120,
+}
+
+
 def w4a16_bytes(m, k, n):
     """Algorithmic bytes of one W4A16 GEMM: packed codes (K*N/2) + fp16
     scales (2*N*K/128) + bf16 A (2*M*K) + bf16 C (2*M*N), each once."""
@@ -270,15 +292,19 @@ def run_w4a16_sweep(args, rank, world, peaks):
     def roof(entries, bound):
         # the dominant launch class: time-weighted over the given launches
         t = sum(e["us"] for e in entries)
+        keys = [(e["m"], e["k"], e["n"]) for e in entries]
+        traffic = (round(sum(TRAFFIC_BYTES[x] for x in keys) / len(keys))
+                   if all(x in TRAFFIC_BYTES for x in keys) else None)
+        algo = round(sum(w4a16_bytes(*x) for x in keys) / len(keys))
         if bound == "hbm":
             ach = sum(w4a16_bytes(e["m"], e["k"], e["n"]) for e in entries) / (t * 1e-6) / 1e9
             return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm_gbs"], unit="GB/s",
-                        frac=round(ach / peaks["hbm_gbs"], 3), traffic=None,
+                        frac=round(ach / peaks["hbm_gbs"], 3), traffic=traffic, algorithmic_bytes=algo,
                         launches=[f"M={e['m']},K={e['k']},N={e['n']}" for e in entries],
                         peak_source=f"{peaks['source']} (copy bandwidth, burst)")
         ach = sum(w4a16_flops(e["m"], e["k"], e["n"]) for e in entries) / (t * 1e-6) / 1e12
         return dict(bound="tensor", achieved=round(ach, 1), peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                    frac=round(ach / peaks["bf16_tflops"], 3), traffic=None,
+                    frac=round(ach / peaks["bf16_tflops"], 3), traffic=traffic, algorithmic_bytes=algo,
                     launches=[f"M={e['m']},K={e['k']},N={e['n']}" for e in entries],
                     peak_source=f"{peaks['source']} (cuBLAS bf16 8192^3, burst)")
 
