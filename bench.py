@@ -499,12 +499,14 @@ def run_nvfp4(args, rank, world, peaks):
 
 
 def run_moe(args, rank, world, peaks):
-    """Grouped MoE W4A16: 256 experts, top-8, hidden 7168, gate+up N=4096,
-    down K=2048, T in {64, 1024, 8192}: route + permute + two grouped GEMMs."""
+    """MoE layer over the grouped W4A16 GEMMs: 256 experts, top-8, hidden
+    7168, intermediate 2048 (gate+up N=4096, down K=2048), T in
+    {64, 1024, 8192}: route (top-k + softmax weights) + permute/gather +
+    gate_up + SwiGLU + down + weighted combine."""
     from quantized_gemm_bit_b200 import hq, synth
-    E, TOPK, H = 256, 8, 7168
+    E, TOPK, H, I = 256, 8, 7168, 2048
     mats = {}
-    for name, (n, k, seed) in {"gate_up": (4096, H, 3000), "down": (H, 2048, 3010)}.items():
+    for name, (n, k, seed) in {"gate_up": (2 * I, H, 3000), "down": (H, I, 3010)}.items():
         q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=seed, experts=E)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, E)
         mats[name] = (d, torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).cuda(), n, k)
@@ -513,51 +515,66 @@ def run_moe(args, rank, world, peaks):
     for t in (64, 1024, 8192):
         logits = synth.router_logits(t, E, seed=3001).cuda()
         x = synth.bf16_normal(t, H, seed=3002).cuda()
-        xd = synth.bf16_normal(t * TOPK, 2048, seed=3003).cuda()
         ids = torch.empty(t, TOPK, dtype=torch.int32, device="cuda")
+        wts = torch.empty(t, TOPK, dtype=torch.float32, device="cuda")
         src = torch.empty(t * TOPK, dtype=torch.int32, device="cuda")
         off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
         xs = torch.empty(t * TOPK, H, dtype=torch.bfloat16, device="cuda")
         pws = torch.zeros(hq.hq_moe_permute_workspace_size(t, TOPK, E), dtype=torch.uint8, device="cuda")
-        c1 = torch.empty(t * TOPK, 4096, dtype=torch.bfloat16, device="cuda")
+        c1 = torch.empty(t * TOPK, 2 * I, dtype=torch.bfloat16, device="cuda")
+        h = torch.empty(t * TOPK, I, dtype=torch.bfloat16, device="cuda")
         c2 = torch.empty(t * TOPK, H, dtype=torch.bfloat16, device="cuda")
+        out = torch.empty(t, H, dtype=torch.bfloat16, device="cuda")
         d1, w1, _, _ = mats["gate_up"]
         d2, w2, _, _ = mats["down"]
         ws1 = torch.zeros(max(256, hq.hq_workspace_size(d1, t * TOPK)), dtype=torch.uint8, device="cuda")
         ws2 = torch.zeros(max(256, hq.hq_workspace_size(d2, t * TOPK)), dtype=torch.uint8, device="cuda")
+        wsc = torch.zeros(hq.hq_moe_combine_workspace_size(t, TOPK), dtype=torch.uint8, device="cuda")
 
-        def route(cp, t=t, logits=logits, ids=ids, src=src, off=off, x=x, xs=xs, pws=pws):
-            hq.hq_moe_topk(logits, t, E, TOPK, ids)
+        def route(cp, t=t, logits=logits, ids=ids, wts=wts, src=src, off=off, x=x, xs=xs, pws=pws):
+            hq.hq_moe_topk_softmax(logits, t, E, TOPK, ids, wts)
             hq.hq_moe_permute(ids, t, TOPK, E, src, off, pws, a=x, hidden=H, a_sorted=xs)
 
         def g1(cp, t=t, xs=xs, off=off, c1=c1, ws1=ws1):
             hq.hq_grouped_gemm_moe(d1, w1, xs, off, t * TOPK, c1, ws1)
 
-        def g2(cp, t=t, xd=xd, off=off, c2=c2, ws2=ws2):
-            hq.hq_grouped_gemm_moe(d2, w2, xd, off, t * TOPK, c2, ws2)
-        launches += [route, g1, g2]
-        meta.append((t, off))
+        def act(cp, t=t, c1=c1, h=h):
+            hq.hq_moe_swiglu(c1, t * TOPK, I, h)
+
+        def g2(cp, t=t, h=h, off=off, c2=c2, ws2=ws2):
+            hq.hq_grouped_gemm_moe(d2, w2, h, off, t * TOPK, c2, ws2)
+
+        def comb(cp, t=t, c2=c2, src=src, wts=wts, out=out, wsc=wsc):
+            hq.hq_moe_combine(c2, src, wts, t, TOPK, H, out, wsc)
+        launches += [route, g1, act, g2, comb]
+        meta.append((t, off, (ws1, ws2, wsc, pws)))
     ms, per = _time_launches(launches, args.steps, args.warmup, world)
-    tok_total, time_total = 0, 0.0
-    for i, (t, off) in enumerate(meta):
-        r_us, g1_us, g2_us = per[3 * i: 3 * i + 3]
+    for (_, _, wss) in meta:
+        for ws in wss:
+            st = hq.hq_check_device_status(ws)
+            if st != hq.HQ_OK:
+                raise RuntimeError(f"device status after the MoE timing: {hq.status_string(st)}")
+    tok_total = 0
+    for i, (t, off, _) in enumerate(meta):
+        r_us, g1_us, a_us, g2_us, c_us = per[5 * i: 5 * i + 5]
         offs = off.cpu().numpy()
         active = int((offs[1:] > offs[:-1]).sum())
-        wbytes = active * (4096 * 7168 // 2 + 4096 * 56 * 2 + 7168 * 2048 // 2 + 7168 * 16 * 2)
-        fl = 2.0 * t * TOPK * 7168 * 6144
+        wbytes = active * (2 * I * H // 2 + 2 * I * (H // 128) * 2 + H * I // 2 + H * (I // 128) * 2)
+        fl = 2.0 * t * TOPK * H * 3 * I
         gemm_us = g1_us + g2_us
+        layer_us = r_us + g1_us + a_us + g2_us + c_us
         detail.append(dict(tokens=t, active_experts=active, route_permute_us=round(r_us, 2),
-                           gate_up_us=round(g1_us, 2), down_us=round(g2_us, 2),
-                           tok_per_s=round(t / ((gemm_us + r_us) * 1e-6), 1),
+                           gate_up_us=round(g1_us, 2), swiglu_us=round(a_us, 2), down_us=round(g2_us, 2),
+                           combine_us=round(c_us, 2), tok_per_s=round(t / (layer_us * 1e-6), 1),
                            tok_per_s_gemms=round(t / (gemm_us * 1e-6), 1), tflops=round(fl / gemm_us / 1e6, 1),
                            weight_gbs=round(wbytes / gemm_us / 1e3, 1),
                            frac_hbm=round(wbytes / gemm_us / 1e3 / peaks["hbm_gbs"], 3)))
         tok_total += t
-        time_total += gemm_us
-    # value: tokens of all three batches per step over the whole step (routing,
-    # permutation and both grouped GEMMs); the detail gives each batch alone
-    return {"workload": "grouped MoE W4A16: 256 experts, top-8, hidden 7168, gate+up N=4096, down K=2048, "
-                        "T in {64,1024,8192}; one step = route + permute + gate_up + down for each T",
+    # value: tokens of all three batches per step over the whole step (every
+    # launch of the layer); the detail gives each batch alone
+    return {"workload": "MoE layer over grouped W4A16 GEMMs: 256 experts, top-8, hidden 7168, intermediate 2048 "
+                        "(gate+up N=4096, down K=2048), T in {64,1024,8192}; one step = route (top-k + softmax "
+                        "weights) + permute/gather + gate_up + SwiGLU + down + weighted combine for each T",
             "value": round(tok_total * args.steps * world / (ms * 1e-3), 1), "unit": "tok/s",
             "ms_per_step": round(ms / args.steps, 4), "detail": detail}
 

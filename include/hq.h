@@ -222,6 +222,13 @@ hq_status hq_quantize_nvfp4(const void* x_bf16_dev, int32_t rows, int32_t k, voi
 hq_status hq_moe_topk(const float* logits_dev, int32_t t, int32_t e, int32_t k, int32_t* topk_ids_dev,
                       hq_stream_t stream);
 
+/* hq_moe_topk plus the combine weights: the softmax probabilities (over
+ * all e experts, fp32, not renormalised over the k) of the selected
+ * experts, in slot order.
+ *   topk_weights_dev : fp32 [t][k], written */
+hq_status hq_moe_topk_softmax(const float* logits_dev, int32_t t, int32_t e, int32_t k, int32_t* topk_ids_dev,
+                              float* topk_weights_dev, hq_stream_t stream);
+
 /* Workspace bytes hq_moe_permute needs. */
 size_t hq_moe_permute_workspace_size(int32_t t, int32_t k, int32_t e);
 
@@ -247,6 +254,36 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
 hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, const void* a_sorted_dev,
                               const int32_t* expert_offsets_dev, int32_t total_rows, void* c_sorted_dev,
                               const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* Gated activation between the two grouped GEMMs of an MoE layer (the
+ * pages leave the layer around the "Grouped" path open; this is the usual
+ * gated feed-forward): h = silu(g) * u, silu(x) = x / (1 + exp(-x)), fp32
+ * arithmetic, bf16 round to nearest.
+ *   gate_up_dev : bf16 [rows][2*inter]: gate in columns [0, inter), up in
+ *                 [inter, 2*inter) (the gate+up GEMM's output)
+ *   h_dev       : bf16 [rows][inter], written (may not overlap the input)
+ *   inter % 8 == 0; both pointers 16-byte aligned.  Row order is kept, so
+ *   it runs on the expert-sorted rows. */
+hq_status hq_moe_swiglu(const void* gate_up_dev, int32_t rows, int32_t inter, void* h_dev, hq_stream_t stream);
+
+/* Workspace bytes hq_moe_combine needs (the error word and the inverse
+ * of the sorted slot list). */
+size_t hq_moe_combine_workspace_size(int32_t t, int32_t k);
+
+/* Weighted combine after the down GEMM: for every token t,
+ * out[t] = sum_j w[t][j] * y_sorted[p], where sorted_src[p] = t*k + j,
+ * summed in slot order j = 0..k-1 in fp32 (no atomics: the same inputs give
+ * the same bits), bf16 round to nearest.
+ *   y_sorted_dev     : bf16 [t*k][hidden], expert-sorted (the down GEMM's output)
+ *   sorted_src_dev   : int32 [t*k] from hq_moe_permute
+ *   topk_weights_dev : fp32 [t][k] (hq_moe_topk_softmax, or the caller's)
+ *   out_dev          : bf16 [t][hidden], written
+ *   hidden % 8 == 0, k <= 16.  A sorted_src that is not a permutation of
+ *   [0, t*k) sets HQ_ERR_DEVICE_BAD_OFFSETS in the workspace error word;
+ *   nothing is read or written out of bounds. */
+hq_status hq_moe_combine(const void* y_sorted_dev, const int32_t* sorted_src_dev, const float* topk_weights_dev,
+                         int32_t t, int32_t k, int32_t hidden, void* out_dev, void* ws_dev, size_t ws_bytes,
+                         hq_stream_t stream);
 
 /* Synchronizes `stream`, reads the workspace error word, clears it and
  * returns it (HQ_OK when no device-side error was recorded). */

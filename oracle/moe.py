@@ -13,10 +13,18 @@ Readings (the pages are silent):
   * ties go to the lower expert index; slots within a token are ordered by
     descending logit (ties: lower index first);
   * the sorted order is (expert ascending, flattened slot index t*k+j
-    ascending), which is unique and therefore bit-exactly checkable.
+    ascending), which is unique and therefore bit-exactly checkable;
+  * the layer around the two grouped GEMMs is the usual gated MoE feed-
+    forward: the gate+up GEMM's N = 2I columns are the gate (first I) and
+    the up projection (last I), h = silu(gate) * up with
+    silu(x) = x / (1 + exp(-x)); the down GEMM's rows are un-permuted and
+    summed per token with the softmax probabilities of the selected
+    experts as weights (over all E experts, not renormalised over the k).
 """
 
 import numpy as np
+
+from .formats import bf16_bits_to_f64
 
 
 def topk_by_logit(logits, k):
@@ -30,7 +38,7 @@ def topk_by_logit(logits, k):
 
 def softmax_topk_weights(logits, ids):
     """Softmax probabilities (fp64) of the selected experts, not
-    renormalised.  Reported for completeness; no kernel consumes them."""
+    renormalised: the combine weights."""
     l = np.asarray(logits, dtype=np.float64)
     p = np.exp(l - l.max(axis=1, keepdims=True))
     p /= p.sum(axis=1, keepdims=True)
@@ -60,3 +68,29 @@ def gather_rows(a, sorted_src, k):
     """A_sorted[i] = A[sorted_src[i] // k] (a bit copy of the bf16 row)."""
     src_tok = np.asarray(sorted_src, dtype=np.int64) // k
     return np.asarray(a)[src_tok]
+
+
+def silu_mul(gate_up_bf16_bits, inter):
+    """SwiGLU of the gate+up output: bf16 bits [rows, 2*inter] ->
+    fp64 [rows, inter], h = silu(g) * u, g = columns [0, inter),
+    u = columns [inter, 2*inter), silu(x) = x / (1 + exp(-x))."""
+    x = bf16_bits_to_f64(gate_up_bf16_bits)
+    g, u = x[:, :inter], x[:, inter:2 * inter]
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
+
+
+def combine(y_sorted_bf16_bits, sorted_src, weights, k):
+    """Un-permute and weigh the down GEMM's output: bf16 bits
+    [T*k, H] in expert-sorted order -> fp64 [T, H],
+    out[t] = sum_j weights[t, j] * Y[p(t, j)] where sorted_src[p] = t*k + j."""
+    y = bf16_bits_to_f64(y_sorted_bf16_bits)
+    src = np.asarray(sorted_src, dtype=np.int64)
+    w = np.asarray(weights, dtype=np.float64)
+    t = len(src) // k
+    pos = np.empty(len(src), dtype=np.int64)
+    pos[src] = np.arange(len(src))            # position of every flattened slot
+    out = np.zeros((t, y.shape[1]))
+    for j in range(k):
+        out += w[:, j:j + 1] * y[pos[np.arange(t) * k + j]]
+    return out

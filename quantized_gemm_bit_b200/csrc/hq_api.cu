@@ -314,7 +314,47 @@ hq_status hq_moe_topk(const float* logits_dev, int32_t t, int32_t e, int32_t k, 
   DeviceInfo dev{};
   hq_status st = device_info(&dev);
   if (st != HQ_OK) return st;
-  return moe_topk_launch(logits_dev, t, e, k, topk_ids_dev, reinterpret_cast<cudaStream_t>(stream));
+  return moe_topk_launch(logits_dev, t, e, k, topk_ids_dev, nullptr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_moe_topk_softmax(const float* logits_dev, int32_t t, int32_t e, int32_t k, int32_t* topk_ids_dev,
+                              float* topk_weights_dev, hq_stream_t stream) {
+  if (t < 0 || k < 1 || k > 16 || e < k || e > 1024) return HQ_ERR_INVALID_ARG;
+  if (t == 0) return HQ_OK;
+  if (!logits_dev || !topk_ids_dev || !topk_weights_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(logits_dev, 4) || !aligned(topk_ids_dev, 4) || !aligned(topk_weights_dev, 4)) return HQ_ERR_ALIGNMENT;
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  return moe_topk_launch(logits_dev, t, e, k, topk_ids_dev, topk_weights_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_moe_swiglu(const void* gate_up_dev, int32_t rows, int32_t inter, void* h_dev, hq_stream_t stream) {
+  if (rows < 0 || inter < 1 || inter % 8 != 0) return HQ_ERR_INVALID_ARG;
+  if (rows == 0) return HQ_OK;
+  if (!gate_up_dev || !h_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(gate_up_dev, 16) || !aligned(h_dev, 16)) return HQ_ERR_ALIGNMENT;
+  return moe_swiglu_launch(gate_up_dev, rows, inter, h_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t hq_moe_combine_workspace_size(int32_t t, int32_t k) {
+  if (t < 0 || k < 1) return 0;
+  return moe_combine_ws_bytes(t, k);
+}
+
+hq_status hq_moe_combine(const void* y_sorted_dev, const int32_t* sorted_src_dev, const float* topk_weights_dev,
+                         int32_t t, int32_t k, int32_t hidden, void* out_dev, void* ws_dev, size_t ws_bytes,
+                         hq_stream_t stream) {
+  if (t < 0 || k < 1 || k > 16 || hidden < 1 || hidden % 8 != 0) return HQ_ERR_INVALID_ARG;
+  if ((long long)t * k > 0x7fffffffLL) return HQ_ERR_INVALID_ARG;
+  if (t == 0) return HQ_OK;
+  if (!y_sorted_dev || !sorted_src_dev || !topk_weights_dev || !out_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(y_sorted_dev, 16) || !aligned(out_dev, 16) || !aligned(sorted_src_dev, 4) ||
+      !aligned(topk_weights_dev, 4) || !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  if (ws_bytes < moe_combine_ws_bytes(t, k)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return moe_combine_launch(y_sorted_dev, sorted_src_dev, topk_weights_dev, t, k, hidden, out_dev, ws_dev,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t hq_moe_permute_workspace_size(int32_t t, int32_t k, int32_t e) {

@@ -72,7 +72,11 @@ hq_status nvfp4_quant_launch(const void* x, int rows, int k, void* codes, void* 
 
 // MoE helpers.
 size_t moe_permute_ws_bytes(int t, int k, int e);
-hq_status moe_topk_launch(const float* logits, int t, int e, int k, int32_t* ids, cudaStream_t s);
+hq_status moe_topk_launch(const float* logits, int t, int e, int k, int32_t* ids, float* weights, cudaStream_t s);
+hq_status moe_swiglu_launch(const void* x, long long rows, int inter, void* h, cudaStream_t s);
+size_t moe_combine_ws_bytes(int t, int k);
+hq_status moe_combine_launch(const void* y_sorted, const int32_t* sorted_src, const float* weights, int t, int k,
+                             int hidden, void* out, void* ws, cudaStream_t s);
 hq_status moe_permute_launch(const int32_t* ids, int t, int k, int e, int32_t* sorted_src, int32_t* offsets,
                              const void* a, int hidden, void* a_sorted, void* ws, cudaStream_t s);
 

@@ -11,7 +11,14 @@
 //             the flattened slot list ordered by (expert, slot), stable, so
 //             it is unique and matches a plain counting sort bit for bit;
 //   gather  : rows of A copied into expert-sorted order.
-// All integer work; nothing here waits on anything, so nothing can hang.
+// Around the two grouped GEMMs of the layer:
+//   softmax : the selected experts' softmax probabilities (the combine
+//             weights), from the same pass as top-k;
+//   swiglu  : h = silu(gate) * up on the gate+up GEMM's output;
+//   combine : the down GEMM's rows un-permuted and summed per token with
+//             those weights, in slot order (deterministic, no atomics).
+// Nothing here waits on anything, so nothing can hang.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -28,7 +35,8 @@ constexpr int kPermTok = 128;   // tokens per block in the permutation
 
 // One warp per token.  Each lane holds ceil(E/32) logits; k rounds of a
 // warp-wide (value desc, index asc) arg-max pick the experts in order.
-__global__ void topk_kernel(const float* __restrict__ logits, int t, int e, int k, int32_t* __restrict__ ids) {
+__global__ void topk_kernel(const float* __restrict__ logits, int t, int e, int k, int32_t* __restrict__ ids,
+                            float* __restrict__ weights) {
   const int warps = blockDim.x >> 5;
   const int tok = blockIdx.x * warps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -42,6 +50,7 @@ __global__ void topk_kernel(const float* __restrict__ logits, int t, int e, int 
     v[i] = idx < e ? row[idx] : -__int_as_float(0x7f800000);  // -inf
   }
   uint32_t taken = 0;  // bit i: v[i] already selected
+  float vmax = 0.f, vsel = 0.f;
   for (int r = 0; r < k; ++r) {
     float best = 0.f;
     int bidx = 0x7fffffff;
@@ -67,6 +76,21 @@ __global__ void topk_kernel(const float* __restrict__ logits, int t, int e, int 
     }
     if (lane == 0) ids[(size_t)tok * k + r] = bidx;
     if ((bidx & 31) == lane) taken |= 1u << (bidx >> 5);
+    if (r == 0) vmax = best;
+    if (lane == r) vsel = best;            // lane r keeps the logit of slot r
+  }
+  if (weights) {
+    // softmax over all e logits in fp32: each lane sums its own logits in
+    // index order, then a fixed butterfly adds the lanes (deterministic)
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int idx = i * 32 + lane;
+      if (idx < e) sum += expf(v[i] - vmax);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) weights[(size_t)tok * k + lane] = expf(vsel - vmax) / sum;
   }
 }
 
@@ -176,6 +200,92 @@ __global__ void gather_rows_kernel(const int4* __restrict__ a, int hidden_vec, i
   }
 }
 
+// h[r][c] = silu(g) * u with g = x[r][c], u = x[r][inter + c]; 8 columns
+// (16 bytes) per thread and step, fp32 arithmetic, bf16 round to nearest.
+__global__ void swiglu_kernel(const uint4* __restrict__ x, long long rows, int inter_vec, uint4* __restrict__ h) {
+  const long long total = rows * inter_vec;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / inter_vec;
+    const int c = (int)(i - r * inter_vec);
+    const uint4 gv = x[r * 2 * inter_vec + c];
+    const uint4 uv = x[r * 2 * inter_vec + inter_vec + c];
+    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+    const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float g0 = __uint_as_float(gw[q] << 16), g1 = __uint_as_float(gw[q] & 0xFFFF0000u);
+      const float u0 = __uint_as_float(uw[q] << 16), u1 = __uint_as_float(uw[q] & 0xFFFF0000u);
+      const float h0 = g0 / (1.f + expf(-g0)) * u0;
+      const float h1 = g1 / (1.f + expf(-g1)) * u1;
+      o[q] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h0)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(h1)) << 16);
+    }
+    h[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// inv[sorted_src[p]] = p for every sorted position p; a slot index outside
+// [0, rows) is reported instead of written.
+__global__ void inverse_kernel(const int32_t* __restrict__ src, int rows, int32_t* __restrict__ inv,
+                               uint32_t* err) {
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < rows; p += gridDim.x * blockDim.x) {
+    const int sl = src[p];
+    if (sl < 0 || sl >= rows)
+      atomicCAS(err, 0u, (uint32_t)HQ_ERR_DEVICE_BAD_OFFSETS);
+    else
+      inv[sl] = p;
+  }
+}
+
+// out[t] = sum_j w[t][j] * y[inv[t*k + j]] over 8 columns per thread and
+// step, in slot order j = 0..k-1 (fp32 fused multiply-add), bf16 round to
+// nearest.  A slot that no sorted position names (sorted_src was not a
+// permutation) is reported and left out.
+__global__ void combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
+                               const float* __restrict__ w, int t, int k, int hidden_vec, uint4* __restrict__ out,
+                               uint32_t* err) {
+  __shared__ int s_pos[16];
+  __shared__ float s_w[16];
+  for (int tok = blockIdx.x; tok < t; tok += gridDim.x) {
+    __syncthreads();   // the previous token's slots are no longer read
+    if (threadIdx.x < k) {
+      int p = inv[(size_t)tok * k + threadIdx.x];
+      if (p < 0 || p >= t * k) {
+        atomicCAS(err, 0u, (uint32_t)HQ_ERR_DEVICE_BAD_OFFSETS);
+        p = -1;
+      }
+      s_pos[threadIdx.x] = p;
+      s_w[threadIdx.x] = w[(size_t)tok * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < hidden_vec; c += blockDim.x) {
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+      for (int j = 0; j < k; ++j) {
+        const int p = s_pos[j];
+        if (p < 0) continue;
+        const uint4 v = y[(size_t)p * hidden_vec + c];
+        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+        const float wj = s_w[j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] = fmaf(wj, __uint_as_float(vw[q] << 16), acc[2 * q]);
+          acc[2 * q + 1] = fmaf(wj, __uint_as_float(vw[q] & 0xFFFF0000u), acc[2 * q + 1]);
+        }
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o[q] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q])) |
+               ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q + 1])) << 16);
+      out[(size_t)tok * hidden_vec + c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
 __global__ void timeout_probe_kernel(uint32_t* err, uint64_t limit_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -194,9 +304,43 @@ size_t moe_permute_ws_bytes(int t, int k, int e) {
   return sizeof(WsHeader) + ((nb * e * sizeof(int32_t) + 255) / 256) * 256;
 }
 
-hq_status moe_topk_launch(const float* logits, int t, int e, int k, int32_t* ids, cudaStream_t s) {
+hq_status moe_topk_launch(const float* logits, int t, int e, int k, int32_t* ids, float* weights, cudaStream_t s) {
   const int warps = 8;
-  topk_kernel<<<(t + warps - 1) / warps, warps * 32, 0, s>>>(logits, t, e, k, ids);
+  topk_kernel<<<(t + warps - 1) / warps, warps * 32, 0, s>>>(logits, t, e, k, ids, weights);
+  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+hq_status moe_swiglu_launch(const void* x, long long rows, int inter, void* h, cudaStream_t s) {
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  const long long vecs = rows * (inter / 8);
+  const long long want = (vecs + 255) / 256;
+  const int grid = (int)std::max<long long>(1, std::min<long long>(want, (long long)dev.num_sms * 8));
+  swiglu_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), rows, inter / 8, static_cast<uint4*>(h));
+  return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+size_t moe_combine_ws_bytes(int t, int k) {
+  return sizeof(WsHeader) + (((size_t)t * k * sizeof(int32_t) + 255) / 256) * 256;
+}
+
+hq_status moe_combine_launch(const void* y_sorted, const int32_t* sorted_src, const float* weights, int t, int k,
+                             int hidden, void* out, void* ws, cudaStream_t s) {
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  int32_t* inv = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  const int rows = t * k;
+  // every slot starts unnamed (-1): a sorted list that is not a permutation
+  // is reported by the combine instead of read out of bounds
+  if (cudaMemsetAsync(inv, 0xFF, (size_t)rows * sizeof(int32_t), s) != cudaSuccess) return HQ_ERR_CUDA;
+  const int g1 = std::max(1, std::min((rows + 255) / 256, dev.num_sms * 4));
+  inverse_kernel<<<g1, 256, 0, s>>>(sorted_src, rows, inv, err);
+  const int g2 = std::max(1, std::min(t, dev.num_sms * 8));
+  combine_kernel<<<g2, 128, 0, s>>>(static_cast<const uint4*>(y_sorted), inv, weights, t, k, hidden / 8,
+                                    static_cast<uint4*>(out), err);
   return cudaGetLastError() == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 

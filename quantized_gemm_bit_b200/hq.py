@@ -39,8 +39,9 @@ HQ_FMT_NVFP4 = 3
 EXPORTS = (
     "hq_layout_version", "hq_status_string", "hq_quant_desc_init", "hq_packed_size", "hq_pack_weights",
     "hq_workspace_size", "hq_gemm_w4a16", "hq_gemm_mxfp4_a8", "hq_gemm_nvfp4", "hq_quantize_fp8_rows",
-    "hq_quantize_nvfp4_workspace_size", "hq_quantize_nvfp4", "hq_moe_topk",
-    "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_check_device_status",
+    "hq_quantize_nvfp4_workspace_size", "hq_quantize_nvfp4", "hq_moe_topk", "hq_moe_topk_softmax",
+    "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_moe_swiglu",
+    "hq_moe_combine_workspace_size", "hq_moe_combine", "hq_check_device_status",
     "hq_debug_timeout_probe", "hq_gemm_w4a16_static",
 )
 
@@ -89,6 +90,10 @@ def lib():
             "hq_quantize_nvfp4_workspace_size": (sz, [i32, i32]),
             "hq_quantize_nvfp4": (st, [vp, i32, i32, vp, vp, vp, vp, sz, vp]),
             "hq_moe_topk": (st, [vp, i32, i32, i32, vp, vp]),
+            "hq_moe_topk_softmax": (st, [vp, i32, i32, i32, vp, vp, vp]),
+            "hq_moe_swiglu": (st, [vp, i32, i32, vp, vp]),
+            "hq_moe_combine_workspace_size": (sz, [i32, i32]),
+            "hq_moe_combine": (st, [vp, vp, vp, i32, i32, i32, vp, vp, sz, vp]),
             "hq_moe_permute_workspace_size": (sz, [i32, i32, i32]),
             "hq_moe_permute": (st, [vp, i32, i32, i32, vp, vp, vp, i32, vp, vp, sz, vp]),
             "hq_grouped_gemm_moe": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
@@ -213,6 +218,25 @@ def hq_quantize_nvfp4(x, rows, k, codes, sf, g, ws, stream=None):
 
 def hq_moe_topk(logits, t, e, k, topk_ids, stream=None):
     _check(lib().hq_moe_topk(_ptr(logits), int(t), int(e), int(k), _ptr(topk_ids), _stream(stream)), "hq_moe_topk")
+
+
+def hq_moe_topk_softmax(logits, t, e, k, topk_ids, topk_weights, stream=None):
+    _check(lib().hq_moe_topk_softmax(_ptr(logits), int(t), int(e), int(k), _ptr(topk_ids), _ptr(topk_weights),
+                                     _stream(stream)), "hq_moe_topk_softmax")
+
+
+def hq_moe_swiglu(gate_up, rows, inter, h, stream=None):
+    _check(lib().hq_moe_swiglu(_ptr(gate_up), int(rows), int(inter), _ptr(h), _stream(stream)), "hq_moe_swiglu")
+
+
+def hq_moe_combine_workspace_size(t, k):
+    return lib().hq_moe_combine_workspace_size(int(t), int(k))
+
+
+def hq_moe_combine(y_sorted, sorted_src, topk_weights, t, k, hidden, out, ws, stream=None):
+    _check(lib().hq_moe_combine(_ptr(y_sorted), _ptr(sorted_src), _ptr(topk_weights), int(t), int(k), int(hidden),
+                                _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hq_moe_combine")
 
 
 def hq_moe_permute_workspace_size(t, k, e):

@@ -142,6 +142,28 @@ def test_gemm_argument_errors_need_no_gpu():
     assert L_.hq_debug_timeout_probe(256, 10 ** 9, None) == hq.HQ_ERR_INVALID_ARG
 
 
+def test_moe_layer_argument_errors_need_no_gpu():
+    L_ = hq.lib()
+    # routing with weights
+    assert L_.hq_moe_topk_softmax(None, 0, 8, 2, None, None, None) == hq.HQ_OK
+    assert L_.hq_moe_topk_softmax(None, 4, 8, 0, None, None, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_topk_softmax(16, 4, 8, 2, 16, None, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_topk_softmax(16, 4, 8, 2, 16, 18, None) == hq.HQ_ERR_ALIGNMENT
+    # SwiGLU
+    assert L_.hq_moe_swiglu(None, 0, 64, None, None) == hq.HQ_OK
+    assert L_.hq_moe_swiglu(16, 4, 60, 16, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_swiglu(None, 4, 64, 16, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_swiglu(16, 4, 64, 24, None) == hq.HQ_ERR_ALIGNMENT
+    # combine
+    need = hq.hq_moe_combine_workspace_size(10, 8)
+    assert need >= 256 + 4 * 10 * 8
+    assert L_.hq_moe_combine(None, None, None, 0, 8, 64, None, None, 0, None) == hq.HQ_OK
+    assert L_.hq_moe_combine(16, 16, 16, 10, 17, 64, 16, 256, need, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_combine(16, 16, 16, 10, 8, 60, 16, 256, need, None) == hq.HQ_ERR_INVALID_ARG
+    assert L_.hq_moe_combine(16, 16, 16, 10, 8, 64, 24, 256, need, None) == hq.HQ_ERR_ALIGNMENT
+    assert L_.hq_moe_combine(16, 16, 16, 10, 8, 64, 16, 256, need - 1, None) == hq.HQ_ERR_WORKSPACE_TOO_SMALL
+
+
 def test_workspace_size_is_deterministic_and_covers_header():
     d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 7168, 18432, 128, 0, 1)
     a = hq.hq_workspace_size(d, 16)

@@ -2,7 +2,12 @@
 expert-sorted permutation are bit-exact against the oracle; the grouped
 W4A16 GEMM matches the fp64 oracle within the GEMM tolerance, in full on a
 reduced configuration and on sampled rows/columns at the full workload
-(256 experts, top-8, hidden 7168, gate+up N=4096, down K=2048)."""
+(256 experts, top-8, hidden 7168, gate+up N=4096, down K=2048).  The layer
+around the grouped GEMMs: routing weights, SwiGLU and the weighted combine
+against their oracle functions with bounds derived from their fp32
+arithmetic, and the whole layer end to end."""
+
+import os
 
 import numpy as np
 import pytest
@@ -113,9 +118,14 @@ def test_grouped_reduced_config_full_output(tile_m, variant):
     a = synth.bf16_normal(t, k, seed=5002)
     src, off, a_sorted, st = gpu_permute(torch.from_numpy(ids).to(DEV), e, a)
     assert st == hq.HQ_OK
+    # the reference runs on the oracle's own permutation (the GPU's is bit-equal)
+    _, off_ref, src_ref = R.permute(ids, e)
+    a_sorted_ref = R.gather_rows(_bits(a), src_ref, topk)
+    assert np.array_equal(off.cpu().numpy(), off_ref) and np.array_equal(src.cpu().numpy(), src_ref)
+    assert np.array_equal(_bits(a_sorted.cpu()), a_sorted_ref)
     tuning = hq.Tuning(tile_m=tile_m, variant=variant) if (tile_m or variant) else None
     c = _grouped(d, blob, a_sorted, off, t * topk, n, tuning)
-    _, ref = G.grouped_w4a16_ref(_bits(a_sorted.cpu()), off.cpu().numpy(), q.numpy(), s.numpy(), None, 128)
+    _, ref = G.grouped_w4a16_ref(a_sorted_ref, off_ref, q.numpy(), s.numpy(), None, 128)
     check_gemm(c, ref, k, f"grouped tile_m={tile_m} variant={variant}")
 
 
@@ -153,17 +163,24 @@ def test_grouped_full_size_sampled(t, which):
     d, blob, q, s, n, k = _full_weights(which)
     logits = synth.router_logits(t, 256, seed=3001)
     ids = gpu_route(logits, 8)
+    # the oracle's routing and permutation, which the GPU's must equal bit for bit
+    ids_ref = R.topk_by_logit(logits.numpy(), 8)
+    _, off_ref, src_ref = R.permute(ids_ref, 256)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
     if which == "gate_up":
         a = synth.bf16_normal(t, k, seed=3002)
         src, off, a_sorted, st = gpu_permute(ids, 256, a)
         assert st == hq.HQ_OK
+        a_sorted_ref = R.gather_rows(_bits(a), src_ref, 8)
     else:
         src, off, _, st = gpu_permute(ids, 256)
         assert st == hq.HQ_OK
-        a_sorted = synth.bf16_normal(t * 8, k, seed=3003).to(DEV)
+        a_in = synth.bf16_normal(t * 8, k, seed=3003)
+        a_sorted, a_sorted_ref = a_in.to(DEV), _bits(a_in)
+    assert np.array_equal(off.cpu().numpy(), off_ref) and np.array_equal(src.cpu().numpy(), src_ref)
     rows_total = t * 8
     c = _grouped(d, blob, a_sorted, off, rows_total, n)
-    offs = off.cpu().numpy()
+    offs = off_ref
     rng = np.random.default_rng(t)
     rows = []
     for ex in range(256):
@@ -173,7 +190,7 @@ def test_grouped_full_size_sampled(t, which):
     rows = np.array(sorted(set(rows)))
     cols = np.array(sorted({c0 for nt in range(n // 128) for c0 in (nt * 128, nt * 128 + 127,
                                                                      nt * 128 + int(rng.integers(0, 128)))}))
-    a_rows = _bits(a_sorted[torch.from_numpy(rows).to(DEV)].cpu())
+    a_rows = a_sorted_ref[rows]
     expert_of = np.searchsorted(offs, rows, side="right") - 1
     ref = np.zeros((len(rows), len(cols)))
     for ex in np.unique(expert_of):
@@ -182,3 +199,152 @@ def test_grouped_full_size_sampled(t, which):
         ref[sel] = F.bf16_bits_to_f64(a_rows[sel]) @ w.T
     got = c[torch.from_numpy(rows).to(DEV)][:, torch.from_numpy(cols).to(DEV)]
     check_gemm(got, ref, k, f"moe {which} t={t}")
+
+
+# ---------------------------------------------------------------- the MoE layer around the grouped GEMMs
+
+@pytest.mark.parametrize("t", [1, 64, 1024])
+def test_topk_softmax_ids_and_weights(t):
+    """Ids bit-exact (and equal to hq_moe_topk's); weights = the oracle's
+    softmax probabilities within fp32 rounding: E exps, a 256-term sum and
+    a division, each a few fp32 ulps, so |w - ref| <= 1e-5 * ref."""
+    logits = synth.router_logits(t, 256, seed=3300 + t)
+    ids = torch.empty(t, 8, dtype=torch.int32, device=DEV)
+    w = torch.empty(t, 8, dtype=torch.float32, device=DEV)
+    hq.hq_moe_topk_softmax(logits.to(DEV), t, 256, 8, ids, w)
+    ids_ref = R.topk_by_logit(logits.numpy(), 8)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    assert np.array_equal(gpu_route(logits, 8).cpu().numpy(), ids_ref)
+    w_ref = R.softmax_topk_weights(logits.numpy(), ids_ref)
+    assert np.all(np.abs(w.cpu().numpy() - w_ref) <= 1e-5 * w_ref)
+
+
+def _bf16_bits(x):
+    return F.f32_to_bf16_bits_rne(np.asarray(x, dtype=np.float32))
+
+
+@pytest.mark.parametrize("rows,inter", [(1, 8), (37, 24), (512, 2048)])
+def test_swiglu_elementwise(rows, inter):
+    """h = silu(g) * u in fp32, rounded to bf16: |h - ref| <= 2^-8 |ref|
+    plus the smallest bf16 subnormal (fp32 arithmetic adds ~1e-6 relative
+    to the half-ulp of the bf16 rounding)."""
+    rng = np.random.default_rng(rows + inter)
+    x = rng.normal(0.0, 3.0, (rows, 2 * inter))
+    x[0, :4] = [0.0, -100.0, 100.0, -0.5]                 # zero, both tails
+    bits = _bf16_bits(x)
+    gu = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(DEV)
+    h = torch.empty(rows, inter, dtype=torch.bfloat16, device=DEV)
+    hq.hq_moe_swiglu(gu, rows, inter, h)
+    got = h.float().double().cpu().numpy()
+    ref = R.silu_mul(bits, inter)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -133)
+
+
+def _combine_case(t, k, e, hidden, seed):
+    logits = synth.router_logits(t, e, seed=seed)
+    ids = R.topk_by_logit(logits.numpy(), k)
+    _, _, src = R.permute(ids, e)
+    w = R.softmax_topk_weights(logits.numpy(), ids).astype(np.float32)
+    y = _bf16_bits(np.random.default_rng(seed).normal(size=(t * k, hidden)))
+    return src, w, y
+
+
+def _gpu_combine(y, src, w, t, k, hidden):
+    out = torch.empty(t, hidden, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_moe_combine_workspace_size(t, k))
+    yd = torch.from_numpy(y.view(np.int16)).view(torch.bfloat16).to(DEV)
+    hq.hq_moe_combine(yd, torch.from_numpy(src).to(DEV), torch.from_numpy(w).to(DEV), t, k, hidden, out, ws)
+    return out, hq.hq_check_device_status(ws)
+
+
+@pytest.mark.parametrize("t,hidden", [(1, 8), (50, 264), (1024, 7168)])
+def test_combine_against_oracle(t, hidden):
+    """fp32 fused multiply-adds in slot order then one bf16 rounding:
+    |out - ref| <= 2^-8 |ref| + 2^-20 sum_j |w_j y_j|."""
+    k, e = 8, 256
+    src, w, y = _combine_case(t, k, e, hidden, 3400 + t)
+    out, st = _gpu_combine(y, src, w, t, k, hidden)
+    assert st == hq.HQ_OK
+    got = out.float().double().cpu().numpy()
+    ref = R.combine(y, src, w, k)
+    mag = R.combine(y & np.uint16(0x7FFF), src, np.abs(w), k)    # sum_j |w_j y_j|
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * mag)
+    out2, _ = _gpu_combine(y, src, w, t, k, hidden)
+    assert torch.equal(out, out2)                                   # no atomics: same bits
+
+
+@pytest.mark.parametrize("bad", ["duplicate", "out_of_range"])
+def test_combine_reports_a_sorted_list_that_is_not_a_permutation(bad):
+    t, k, e, hidden = 20, 4, 16, 64
+    src, w, y = _combine_case(t, k, e, hidden, 3500)
+    src = src.copy()
+    if bad == "duplicate":
+        src[3] = src[5]
+    else:
+        src[7] = t * k + 3
+    _, st = _gpu_combine(y, src, w, t, k, hidden)
+    assert st == hq.HQ_ERR_DEVICE_BAD_OFFSETS
+
+
+def _layer_oracle(x_bits, logits, q1, s1, q2, s2, k, e, inter):
+    """The layer from oracle pieces only, rounding to bf16 wherever the GPU
+    path stores bf16 (after each GEMM and after SwiGLU)."""
+    ids = R.topk_by_logit(logits, k)
+    w = R.softmax_topk_weights(logits, ids)
+    _, off, src = R.permute(ids, e)
+    xs = R.gather_rows(x_bits, src, k)
+    _, c1 = G.grouped_w4a16_ref(xs, off, q1, s1, None, 128)
+    h = R.silu_mul(_bf16_bits(c1), inter)
+    _, c2 = G.grouped_w4a16_ref(_bf16_bits(h), off, q2, s2, None, 128)
+    return R.combine(_bf16_bits(c2), src, w, k), ids, off, src
+
+
+@pytest.mark.parametrize("variant", [0, 2])
+def test_moe_layer_end_to_end(variant):
+    """Route (top-k + weights) -> permute + gather -> gate+up grouped GEMM ->
+    SwiGLU -> down grouped GEMM -> weighted combine, all through the C ABI
+    on one stream, against the oracle's layer (32 experts, top-4, T=64,
+    hidden 1024, intermediate 256).  Routing and permutation bit-exact.  The
+    layer output carries the errors of two GEMMs in a row (the first one's
+    reaches the second through SwiGLU), so its bar is the sum of the two
+    GEMM bars: rel-Frobenius <= 1e-2 and, per element,
+    |err| <= 2e-2 |ref| + 4e-3 sqrt(K) rms(ref) with the down GEMM's K."""
+    t, e, k, hid, inter = 64, 32, 4, 1024, 256
+    q1, s1, _ = synth.w4a16_weights(2 * inter, hid, 128, False, seed=3600, experts=e)
+    q2, s2, _ = synth.w4a16_weights(hid, inter, 128, False, seed=3601, experts=e)
+    d1 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 2 * inter, hid, 128, 0, e)
+    d2 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, hid, inter, 128, 0, e)
+    b1 = torch.from_numpy(hq.hq_pack_weights(d1, q1, s1, None)).to(DEV)
+    b2 = torch.from_numpy(hq.hq_pack_weights(d2, q2, s2, None)).to(DEV)
+    logits = synth.router_logits(t, e, seed=3602)
+    x = synth.bf16_normal(t, hid, seed=3603)
+    tun = hq.Tuning(variant=variant) if variant else None
+    # GPU layer
+    ids = torch.empty(t, k, dtype=torch.int32, device=DEV)
+    wts = torch.empty(t, k, dtype=torch.float32, device=DEV)
+    hq.hq_moe_topk_softmax(logits.to(DEV), t, e, k, ids, wts)
+    src, off, xs, st = gpu_permute(ids, e, x)
+    assert st == hq.HQ_OK
+    c1 = _grouped(d1, b1, xs, off, t * k, 2 * inter, tun)
+    h = torch.empty(t * k, inter, dtype=torch.bfloat16, device=DEV)
+    hq.hq_moe_swiglu(c1, t * k, inter, h)
+    c2 = _grouped(d2, b2, h, off, t * k, hid, tun)
+    out = torch.empty(t, hid, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_moe_combine_workspace_size(t, k))
+    hq.hq_moe_combine(c2, src, wts, t, k, hid, out, ws)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    # oracle layer
+    ref, ids_ref, off_ref, src_ref = _layer_oracle(_bits(x), logits.numpy(), q1.numpy(), s1.numpy(), q2.numpy(),
+                                                   s2.numpy(), k, e, inter)
+    assert np.array_equal(ids.cpu().numpy(), ids_ref)
+    assert np.array_equal(off.cpu().numpy(), off_ref) and np.array_equal(src.cpu().numpy(), src_ref)
+    got = out.float().double().cpu().numpy()
+    err = got - ref
+    rel = np.linalg.norm(err) / np.linalg.norm(ref)
+    bound = 2e-2 * np.abs(ref) + 4e-3 * np.sqrt(inter) * np.sqrt(np.mean(ref ** 2))
+    log = os.environ.get("HQ_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(f"moe layer variant={variant} (two-GEMM bar)\t{rel:.3e}\t{np.max(np.abs(err) / bound):.3e}\n")
+    assert rel <= 1e-2, f"moe layer: rel Frobenius {rel:.3e}"
+    assert np.all(np.abs(err) <= bound), f"moe layer: element bound exceeded by {np.max(np.abs(err) - bound):.3e}"

@@ -129,3 +129,82 @@ def test_synth_distributions():
     codes, e8 = synth.mxfp4_weights(64, 1024, seed=2)
     assert set(np.unique(e8.numpy()).tolist()) == set(range(119, 126))
     assert list(itertools.islice(range(3), 1)) == [0]
+
+
+# ---------------------------------------------------------------- MoE layer: SwiGLU and combine
+
+def _bf16(x):
+    return F.f32_to_bf16_bits_rne(np.asarray(x, dtype=np.float32))
+
+
+def test_silu_mul_against_logistic_function_and_identities():
+    """silu(g) * u against scipy's logistic function (a routine the oracle
+    does not call), the identity silu(x) - silu(-x) = x, silu(0) = 0, the
+    tails silu(x) -> x and silu(-x) -> -0, and the column split (gate first)."""
+    from scipy.special import expit
+    rng = np.random.default_rng(5)
+    g = rng.normal(0, 4, (6, 8))
+    u = rng.normal(0, 1, (6, 8))
+    x = np.concatenate([_bf16(g), _bf16(u)], axis=1)
+    gb, ub = F.bf16_bits_to_f64(x[:, :8]), F.bf16_bits_to_f64(x[:, 8:])
+    h = R.silu_mul(x, 8)
+    assert np.allclose(h, gb * expit(gb) * ub, rtol=1e-14, atol=0)
+    ones = np.concatenate([x[:, :8], _bf16(np.ones((6, 8)))], axis=1)
+    neg = np.concatenate([_bf16(-gb), _bf16(np.ones((6, 8)))], axis=1)
+    assert np.allclose(R.silu_mul(ones, 8) - R.silu_mul(neg, 8), gb, rtol=0, atol=1e-12)
+    edge = np.concatenate([_bf16([[0.0, 200.0, -200.0, 1.0]]), _bf16([[3.0, 1.0, 1.0, 0.0]])], axis=1)
+    he = R.silu_mul(edge, 4)[0]
+    assert he[0] == 0.0 and he[1] == 200.0 and -1e-80 < he[2] <= 0.0 and he[3] == 0.0
+    # the gate is the first half: swapping the halves changes the result
+    swapped = np.concatenate([x[:, 8:], x[:, :8]], axis=1)
+    assert not np.allclose(R.silu_mul(swapped, 8), h)
+
+
+def _combine_brute(y_bits, src, w, k):
+    y = F.bf16_bits_to_f64(y_bits)
+    t = len(src) // k
+    out = [[0.0] * y.shape[1] for _ in range(t)]
+    for p, slot in enumerate(src):
+        tok, j = divmod(int(slot), k)
+        for c in range(y.shape[1]):
+            out[tok][c] += float(w[tok][j]) * y[p][c]
+    return np.array(out)
+
+
+def test_combine_brute_force_one_hot_and_linearity():
+    rng = np.random.default_rng(6)
+    t, e, k, h = 7, 9, 3, 5
+    ids = R.topk_by_logit(rng.normal(size=(t, e)).astype(np.float32), k)
+    _, _, src = R.permute(ids, e)
+    y = _bf16(rng.normal(size=(t * k, h)))
+    w = rng.random((t, k)).astype(np.float32)
+    out = R.combine(y, src, w, k)
+    assert np.allclose(out, _combine_brute(y, src, w, k), rtol=1e-15, atol=1e-15)
+    # one-hot weights pick slot j of each token, un-permuted
+    for j in range(k):
+        oh = np.zeros((t, k), dtype=np.float32)
+        oh[:, j] = 1.0
+        pos = {int(s): p for p, s in enumerate(src)}
+        want = F.bf16_bits_to_f64(y[[pos[tok * k + j] for tok in range(t)]])
+        assert np.array_equal(R.combine(y, src, oh, k), want)
+    w2 = rng.random((t, k)).astype(np.float32)
+    wsum = w.astype(np.float64) + w2.astype(np.float64)
+    assert np.allclose(R.combine(y, src, wsum, k), out + R.combine(y, src, w2, k), rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_topk_weights_properties():
+    """Over all experts the probabilities sum to 1; ratios are exp of logit
+    differences; the selected ones are the k largest, in slot order."""
+    rng = np.random.default_rng(7)
+    logits = rng.normal(size=(5, 16)).astype(np.float32)
+    all_ids = np.tile(np.arange(16), (5, 1))
+    assert np.allclose(R.softmax_topk_weights(logits, all_ids).sum(axis=1), 1.0, rtol=1e-14)
+    ids = R.topk_by_logit(logits, 4)
+    w = R.softmax_topk_weights(logits, ids)
+    l64 = logits.astype(np.float64)
+    for tkn in range(5):
+        for a, b in itertools.combinations(range(4), 2):
+            ratio = np.exp(l64[tkn, ids[tkn, a]] - l64[tkn, ids[tkn, b]])
+            assert np.isclose(w[tkn, a] / w[tkn, b], ratio, rtol=1e-12)
+        assert np.all(np.diff(w[tkn]) <= 0)
+    assert np.all(w.sum(axis=1) < 1.0)       # not renormalised over the k selected

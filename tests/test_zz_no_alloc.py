@@ -13,6 +13,7 @@ import pytest
 import torch
 
 from gpu_helpers import check_gemm, workspace
+from oracle import gemm as G
 from quantized_gemm_bit_b200 import hq, synth
 from quantized_gemm_bit_b200.build import build
 
@@ -43,16 +44,18 @@ def test_static_scratch_matches_workspace_entry_point(m, n, k, asym):
     a = synth.bf16_normal(m, k, seed=9001 + m).to(DEV)
     d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, int(asym), 1)
     blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(DEV)
-    ref = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
+    via_ws = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
     ws = workspace(hq.hq_workspace_size(d, m))
-    hq.hq_gemm_w4a16(d, blob, a, m, ref, ws)
+    hq.hq_gemm_w4a16(d, blob, a, m, via_ws, ws)
     assert hq.hq_check_device_status(ws) == hq.HQ_OK
-    ref64 = ref.double().cpu().numpy()
+    ref = G.w4a16_ref(a.cpu().view(torch.int16).numpy().view(np.uint16), q.numpy(), s.numpy(),
+                      None if z is None else z.numpy(), 128)
     for call in range(2):
         c = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device=DEV)
         assert _call_static(d, blob, a, m, c) == hq.HQ_OK
         torch.cuda.synchronize()
-        check_gemm(c, ref64, k, f"static scratch call {call}")
+        check_gemm(c, ref, k, f"static scratch call {call}")
+        assert torch.equal(c, via_ws)      # same launch plan, same bits as the workspace entry point
 
 
 def test_static_scratch_rejects_plans_beyond_its_size():
