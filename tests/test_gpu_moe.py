@@ -129,6 +129,26 @@ def test_grouped_reduced_config_full_output(tile_m, variant):
     check_gemm(c, ref, k, f"grouped tile_m={tile_m} variant={variant}")
 
 
+def test_grouped_maximum_expert_count():
+    """1024 experts (the device tile table's limit), 600 tokens top-2: most
+    experts hold one or two rows, many none; full output."""
+    e, n, k, t, topk = 1024, 128, 128, 600, 2
+    q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=5200, experts=e)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, e)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(DEV)
+    logits = synth.router_logits(t, e, seed=5201)
+    ids = R.topk_by_logit(logits.numpy(), topk)
+    a = synth.bf16_normal(t, k, seed=5202)
+    src, off, a_sorted, st = gpu_permute(torch.from_numpy(ids).to(DEV), e, a)
+    assert st == hq.HQ_OK
+    _, off_ref, src_ref = R.permute(ids, e)
+    assert np.array_equal(off.cpu().numpy(), off_ref) and np.array_equal(src.cpu().numpy(), src_ref)
+    a_sorted_ref = R.gather_rows(_bits(a), src_ref, topk)
+    c = _grouped(d, blob, a_sorted, off, t * topk, n)
+    _, ref = G.grouped_w4a16_ref(a_sorted_ref, off_ref, q.numpy(), s.numpy(), None, 128)
+    check_gemm(c, ref, k, "grouped 1024 experts")
+
+
 def test_grouped_bad_offsets_are_reported():
     e, n, k = 4, 128, 256
     q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=5100, experts=e)

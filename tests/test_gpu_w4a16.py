@@ -67,6 +67,32 @@ def test_ragged_shapes_full_output(m, n, k, asym):
     check_gemm(c, ref, k, f"m={m} n={n} k={k}")
 
 
+@pytest.mark.parametrize("m,n,k,variant", [(1, 1, 128, 1), (3, 7, 128, 2), (16, 8, 256, 1), (64, 9, 128, 2),
+                                           (300, 1, 128, 1), (33, 136, 128, 0)])
+def test_narrow_and_single_block_shapes(m, n, k, variant):
+    """Degenerate shapes: N below one 32-row slice (the scalar store path
+    when N % 8 != 0), a single 128-K block, single-row outputs."""
+    d, blob, a, (q, s, z) = make_case(m, n, k, True, 300 + m + n)
+    c, _ = run(d, blob, a, m, hq.Tuning(variant=variant) if variant else None)
+    check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"narrow m={m} n={n} k={k}")
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+def test_zero_weights_give_exact_zeros(variant):
+    """Every code equal to its zero point: w = (q - z) s = 0 exactly, so the
+    output is exactly zero (both kernels, and the stream-K partial sums)."""
+    m, n, k = 16, 384, 1024
+    q = torch.full((n, k // 8), 0x55555555, dtype=torch.int32)          # every nibble 5
+    s = torch.full((n, k // 128), 0.01, dtype=torch.float16)
+    z = torch.full((n, k // 128), 5, dtype=torch.uint8)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 1, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(DEV)
+    a = synth.bf16_normal(m, k, 333)
+    c, _ = run(d, blob, a, m, hq.Tuning(variant=variant))
+    assert torch.count_nonzero(c) == 0
+    assert np.all(G.w4a16_ref(_bits(a), q.numpy(), s.numpy(), z.numpy(), 128) == 0.0)
+
+
 @pytest.mark.parametrize("variant", [1, 2])
 @pytest.mark.parametrize("tile_m", [16, 32, 64, 128, 256])
 def test_every_token_tile(tile_m, variant):
