@@ -48,21 +48,18 @@ template <int NTOK>
 struct Cfg {
   // records (128-K blocks) per pipeline stage: two for the small token tiles,
   // whose MMAs are cheap, so the per-stage waits and commits are amortized
-  static constexpr bool kCoop = false;   // see kDqGroups
-  static constexpr int kKps = kCoop && NTOK <= 32 ? 3 : NTOK <= 64 ? 2 : 1;
+  static constexpr int kKps = NTOK <= 64 ? 2 : 1;
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
   static constexpr int kRecs = kKps * kRecMax;
-  static constexpr int kSmemStages = kKps == 3 ? (NTOK == 16 ? 5 : 4)
-                                    : NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
-  static constexpr int kTmemStages = kKps == 3 ? 2 : NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
+  static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
   // Dequantizing warpgroups own alternate stages (the epilogue warpgroup
-  // joins for tiles of <= 64 tokens).  kCoop instead lets all twelve warps
-  // share every three-record stage of a 16/32-token tile (warp 4 + 4r + q:
-  // record r, rows 32q..32q+31); measured slower on B200, so off.
-  static constexpr int kDqGroups = kCoop && NTOK <= 32 ? 1 : NTOK <= 64 ? 3 : 2;
-  static constexpr int kDqWarps = kDqGroups == 1 ? 12 : 4;  // arrivals on a TMEM stage's ready barrier
+  // joins for tiles of <= 64 tokens).  Measured slower on B200 and dropped:
+  // all twelve warps sharing every three-record stage of a 16/32-token tile.
+  static constexpr int kDqGroups = NTOK <= 64 ? 3 : 2;
+  static constexpr int kDqWarps = 4;  // arrivals on a TMEM stage's ready barrier
   // full barriers, one per (SMEM stage, dequant group): iteration `it`
   // uses barrier (it % SS, it % NDQ), so every waiter sees each of its
   // barrier's phases in order whatever the ring depth
@@ -82,7 +79,6 @@ struct Cfg {
   static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(64 * kKps * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
   static_assert(kTmemStages % kDqGroups == 0, "every TMEM stage must always return to the same dequant group");
-  static_assert(kDqGroups != 1 || kKps * 4 == 12, "one record-quarter per dequantizing warp");
   static_assert(8 * (kFullBars + kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
 };
 
@@ -117,30 +113,10 @@ __device__ __forceinline__ void dequant_chunk(const uint4& raw, RowQ qp, uint32_
   }
 }
 
-// Dequantize 32-K chunks c0 .. c0+NC-1 of one record: thread (warp quarter
-// q, lane) owns weight row r = 32q + lane; store_chunks writes them to TMEM
-// lane r, columns 16*c0 ... of the record's 64.
-template <int NC>
-__device__ __forceinline__ void dequant_chunks(const uint8_t* rec, int c0, int r, int has_zero,
-                                               uint32_t (&out)[NC * 16]) {
-  uint4 raw[NC];
-#pragma unroll
-  for (int c = 0; c < NC; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + ((c0 + c) * 128 + r) * 16);
-  const RowQ qp = row_qparams(rec, r, has_zero);
-#pragma unroll
-  for (int c = 0; c < NC; ++c) dequant_chunk(raw[c], qp, out + c * 16);
-}
-
-template <int NC>
-__device__ __forceinline__ void store_chunks(const uint32_t (&w)[NC * 16], int c0, uint32_t taddr) {
-#pragma unroll
-  for (int c = 0; c < NC; ++c)
-    tmem_st_x16(taddr + (c0 + c) * 16, *reinterpret_cast<const uint32_t(*)[16]>(w + c * 16));
-}
-
-// A whole record: its 64 code bytes per row and the row's scale and zero
-// point are read from shared memory first (one round trip), then each chunk
-// is dequantized and stored to TMEM.
+// A whole 128-K record for weight row r (thread lane of warp quarter q owns
+// row r = 32q + lane, TMEM lane r, columns taddr .. taddr + 63): its 64 code
+// bytes and the row's scale and zero point are read from shared memory
+// first (one round trip), then each 32-K chunk is dequantized and stored.
 __device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
   uint4 raw[4];
 #pragma unroll
@@ -363,11 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (int)(q * 32 + lane);              // weight row within the tile
     const uint32_t lane_addr = (q * 32) << 16;
     const bool epi = warp < 8;
-    // dequant group index (2: epilogue warps); cooperative mode: one group
-    constexpr bool kShare = NDQ == 1;                   // cooperative stages
-    const int dq = kShare ? 0 : warp >= 12 ? 1 : warp >= 8 ? 0 : 2;
+    // dequant group index (2: the epilogue warps)
+    const int dq = warp >= 12 ? 1 : warp >= 8 ? 0 : 2;
     const bool does_dq = dq < NDQ;
-    const int myrec = kShare ? (int)(warp - 4) >> 2 : -1;  // cooperative stages: this warp's record
     uint32_t it = 0, uc = 0;
     bool ok = true;
     Unit x;
@@ -381,41 +355,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // only ever serve this group, so it observes every phase of the
         // barriers it waits on, one after the other (a parity wait can only
         // tell adjacent phases apart).
-        // kEarly: dequantize the first half-record into registers before the
-        // TMEM stage is known to be free, overlapping that wait with the
-        // arithmetic; off, because the busier dequant warps then take issue
-        // slots from the MMA warp on the same sub-partition (measured slower).
-        constexpr bool kEarly = false;   // measured slower: the MMA warp loses issue slots
-        if (!hq_wait_warp_n(kEarly ? 1 : 2, full_bar(it), full_par(it), &afree[t], ph_t ^ 1, nullptr, 0, p.wait_ns,
-                            s_abort)) {
+        // (Dequantizing the first half-record into registers before the TMEM
+        // stage is known to be free measured slower: the busier dequant warps
+        // take issue slots from the MMA warp on the same sub-partition.)
+        if (!hq_wait_warp_n(2, full_bar(it), full_par(it), &afree[t], ph_t ^ 1, nullptr, 0, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
-        const int r0 = kShare ? myrec : 0;
         const uint32_t tbase = tmem_base + lane_addr + a_col(t);
-        if constexpr (kEarly) {
-          uint32_t wreg[32];
-          if (r0 < nrec) dequant_chunks<2>(sR + s * kRecs + r0 * p.rec_bytes, 0, r, p.has_zero, wreg);
-          if (!hq_wait_warp_n(1, &afree[t], ph_t ^ 1, nullptr, 0, nullptr, 0, p.wait_ns, s_abort)) {
-            if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (r0 < nrec) {
-            store_chunks<2>(wreg, 0, tbase + r0 * 64);
-            dequant_chunks<2>(sR + s * kRecs + r0 * p.rec_bytes, 2, r, p.has_zero, wreg);
-            store_chunks<2>(wreg, 2, tbase + r0 * 64);
-          }
-        } else {
-          tc_fence_after();
-          if (r0 < nrec) dequant_block(sR + s * kRecs + r0 * p.rec_bytes, r, p.has_zero, tbase + r0 * 64);
-        }
-        if (!kShare) {
-          for (int rr = 1; rr < nrec; ++rr)
-            dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
-        }
+        tc_fence_after();
+        for (int rr = 0; rr < nrec; ++rr)
+          dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();

@@ -60,12 +60,9 @@ struct SmallCfg {
   static constexpr int kUnpackWarps = NTOK <= 32 ? 16 : 8;
   static constexpr int kThreads = (8 + kUnpackWarps) * 32;
   static constexpr int kChunks = 4 * kKps * 4 / kUnpackWarps;   // 32-K chunks per unpacking warp
-  // false: warp 1 issues every MMA.  true: the last unpacking warp to
-  // finish a stage issues that stage's MMAs (stages write separate result
-  // tiles, so MMAs of different stages need no order among themselves);
-  // measured slower on B200 (single-lane issue from a busy warp), kept as an
-  // option for other tile shapes
-  static constexpr bool kSelfIssue = false;
+  // Warp 1 issues every MMA.  (Letting the last unpacking warp to finish a
+  // stage issue that stage's MMAs measured slower on B200: single-lane issue
+  // from a busy warp.)
   static constexpr int kEpiScratch = 4 * 2048;          // warp-local transposes of the output
   static constexpr int kBarBytes = 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
@@ -75,7 +72,7 @@ struct SmallCfg {
   static constexpr size_t kSmem = 1024 + kScrOff + kEpiScratch;
   static_assert(kABlock % 1024 == 0 && kRecMax % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
   static_assert(kACols * kAStages + kDCols * kDStages <= 512, "TMEM budget");
-  static_assert(8 * (2 * kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 + 4 * kAStages <= kBarBytes,
+  static_assert(8 * (2 * kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 <= kBarBytes,
                 "barrier area");
   static_assert(kSmem <= 232448, "shared memory budget");
 };
@@ -137,7 +134,6 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort + 1);
-  uint32_t* s_done = reinterpret_cast<uint32_t*>(s_total + 1);   // [AS] unpacked shares per TMEM stage
   int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);  // [kMaxExperts + 1]
   int* s_off = s_prefix + (kMaxExperts + 1);                    // [kMaxExperts + 1]
   uint16_t* epi_scratch = reinterpret_cast<uint16_t*>(smem + C::kScrOff);  // 16-byte aligned
@@ -158,8 +154,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
       mbar_init(&dfull[d], 1);
       mbar_init(&dempty[d], 4);
     }
-    mbar_init(drain, C::kSelfIssue ? C::kUnpackWarps : 1);
-    for (int t = 0; t < AS; ++t) s_done[t] = 0;
+    mbar_init(drain, 1);
     *s_abort = 0;
     *s_total = 0;
     fence_mbar_init();
@@ -268,7 +263,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
     tc_commit(&dfull[d]);
   };
 
-  if (warp == 1 && !C::kSelfIssue) {
+  if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
     // one lane, fixed for the whole kernel, issues every MMA and commit: a
     // commit tracks the tcgen05 operations of the thread that issues it
@@ -331,37 +326,8 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if constexpr (!C::kSelfIssue) {
-          if (lane == 0) mbar_arrive(&aready[t]);
-        } else {
-          // count this warp's share; the warp completing the stage issues its
-          // MMAs (fence, relaxed atomic, fence: the other warps' TMEM stores
-          // are ordered before the MMAs that read them)
-          uint32_t last = 0;
-          if (lane == 0) {
-            __threadfence_block();
-            last = (atomicAdd(&s_done[t], 1u) + 1) % C::kUnpackWarps == 0;
-            if (last) __threadfence_block();
-          }
-          last = __shfl_sync(0xffffffffu, last, 0);
-          if (last) {
-            const int d = it % DS;
-            if (!hq_wait_warp(&dempty[d], ((it / DS) & 1) ^ 1, p.wait_ns, s_abort)) {
-              if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (lane == 0) issue_stage(s, t, d, nrec);
-            __syncwarp();
-          }
-        }
+        if (lane == 0) mbar_arrive(&aready[t]);
       }
-    }
-    if constexpr (C::kSelfIssue) {
-      // no MMA this warp issued may still run when TMEM is released
-      if (lane == 0) tc_commit(drain);
-      __syncwarp();
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ scale warps + epilogue (warps 4-7)
@@ -439,10 +405,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) {
-    if constexpr (C::kSelfIssue) hq_wait_warp(drain, 0, p.wait_ns, nullptr);
-    tmem_dealloc(*s_tmem, 512);
-  }
+  if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
 template <int NTOK>
