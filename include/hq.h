@@ -99,7 +99,6 @@ typedef struct {
 /* Execution choices (the Tuning Config of [P-fa2] paragraph 3).  Pass NULL
  * to let the library's heuristic choose; a zero field also means "choose".
  *   tile_m   : token tile (the MMA N extent): 16, 32, 64, 128 or 256
- *              (hq_grouped_gemm_moe: 16, 32, 64 or 128)
  *   tile_n   : weight rows per tile: 128 (the only value)
  *   tile_k   : K per pipeline stage: 128 (fixed by the packed layout)
  *   stages   : 0 (the pipeline depth is fixed per token tile)

@@ -16,8 +16,8 @@ namespace hq {
 // output element (row0 + j0 + j, n_warp + lane).
 //   part != nullptr : fp32 into a partial tile slot laid out [token][128]
 //                     (column r_tile = the row of the weight tile);
-//   n_total % 8 == 0: bf16 through the transpose buffer `sc` (32 x EB
-//                     uint16, 16-byte aligned), 16-byte stores;
+//   n_total % 8 == 0 and sc != nullptr: bf16 through the transpose buffer
+//                     `sc` (32 x EB uint16, 16-byte aligned), 16-byte stores;
 //   otherwise       : one bf16 per (token, column).
 // Rows at or past `rows` (tokens beyond the tile's valid rows) and columns
 // at or past n_total are not written.  `sc` is reused after the call (the
@@ -30,7 +30,7 @@ __device__ __forceinline__ void store_rows_chunk(__nv_bfloat16* c, int n_total, 
   if (part) {
 #pragma unroll
     for (int j = 0; j < EB; ++j) __stcg(part + (size_t)(j0 + j) * 128 + r_tile, v[j]);
-  } else if ((n_total % 8) == 0) {
+  } else if ((n_total % 8) == 0 && sc != nullptr) {
 #pragma unroll
     for (int j = 0; j < EB; ++j) sc[j * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
     __syncwarp();

@@ -199,9 +199,7 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
       !aligned(expert_offsets_dev, 4) || !aligned(ws_dev, 256))
     return HQ_ERR_ALIGNMENT;
   if (t) {
-    // grouped token tiles: 16..128 (the 256-token tile keeps no room for
-    // the per-expert tables)
-    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128)
+    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
       return HQ_ERR_UNSUPPORTED;
     if (t->split_k > 1 || (t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->stages != 0 ||
         (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)

@@ -65,8 +65,9 @@ struct Cfg {
   // barrier's phases in order whatever the ring depth
   static constexpr int kFullBars = kSmemStages * kDqGroups;
   static constexpr int kFullPeriod = kSmemStages / cgcd(kSmemStages, kDqGroups) * kDqGroups;  // lcm
-  // warp-local transpose buffer for 16-byte output stores (aliases the
-  // expert tables at 256 tokens, a dense-only tile)
+  // warp-local transpose buffer for 16-byte output stores; at 256 tokens
+  // it aliases the expert tables, so grouped 256-token tiles store their
+  // outputs element by element instead
   static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
   static constexpr int kBarBytes = 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* part = x.partial ? p.partials + ((size_t)blockIdx.x * 2 + x.slot) * NTOK * kTileN : nullptr;
       // batched TMEM loads (EB columns), then fp32 partials or bf16 stores
       constexpr int EB = NTOK >= 32 ? 32 : 16;
-      uint16_t* sc = epi_scratch + q * 1024;
+      uint16_t* sc = (C::kEpiScratch == 0 && p.grouped) ? nullptr : epi_scratch + q * 1024;
 #pragma unroll 1
       for (int j0 = 0; j0 < NTOK; j0 += EB) {
         uint32_t v0[16], v1[16];
@@ -445,6 +446,8 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
       // Poisson(avg) rows per expert, so the tile covers avg + 2 sd.
       const double avg = (double)m / std::max(1, d.num_experts);
       const double want = avg + 2.0 * std::sqrt(avg);
+      // (256-token tiles, on request only: measured slower for every T tried,
+      // e.g. T=8192 top-8 over 256 experts, down: 2.3 ms at 128, 2.9 at 256)
       ntok = want <= 16 ? 16 : want <= 32 ? 32 : want <= 64 ? 64 : 128;
     } else {
       ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;

@@ -127,11 +127,11 @@ def test_gemm_argument_errors_need_no_gpu():
     for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=3), hq.Tuning(cta_group=2)):
         assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
                                 None) == hq.HQ_ERR_UNSUPPORTED
-    # grouped: no 256-token tile; block-scaled: no variants
+    # grouped: no K split, no 512-token tile; block-scaled: no variants
     dg = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 256, 256, 128, 0, 8)
-    t = hq.Tuning(tile_m=256)
-    assert L_.hq_grouped_gemm_moe(ctypes.byref(dg), 16, 16, 16, 40, 32, ctypes.byref(t), 256, 1 << 20,
-                                  None) == hq.HQ_ERR_UNSUPPORTED
+    for bad in (hq.Tuning(tile_m=512), hq.Tuning(split_k=2)):
+        assert L_.hq_grouped_gemm_moe(ctypes.byref(dg), 16, 16, 16, 40, 32, ctypes.byref(bad), 256, 1 << 20,
+                                      None) == hq.HQ_ERR_UNSUPPORTED
     dm = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 256, 256, 32, 0, 1)
     t = hq.Tuning(variant=1)
     assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dm), 4096, 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,

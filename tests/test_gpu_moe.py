@@ -106,7 +106,8 @@ def _grouped(desc, blob, a_sorted, off, rows, n, tuning=None):
     return c
 
 
-@pytest.mark.parametrize("tile_m,variant", [(0, 0), (16, 0), (32, 0), (64, 0), (128, 0), (16, 2), (32, 2), (64, 2)])
+@pytest.mark.parametrize("tile_m,variant", [(0, 0), (16, 0), (32, 0), (64, 0), (128, 0), (256, 0), (16, 2), (32, 2),
+                                            (64, 2)])
 def test_grouped_reduced_config_full_output(tile_m, variant):
     e, n, k, t, topk = 8, 256, 512, 40, 2
     q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=5000, experts=e)
