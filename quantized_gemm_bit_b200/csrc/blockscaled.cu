@@ -555,26 +555,40 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   BsConfig cfg{};
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
-  const long long ks = bs_k_stages(d, ntok);
   auto dp_eff = [&](int nt) {
     const long long tl = bs_tiles(d, m, nt);
     const long long waves = (tl + dev.num_sms - 1) / dev.num_sms;
     return (double)tl / (double)(waves * dev.num_sms);
   };
   if (t && t->split_k > 0) {
+    const long long ks = bs_k_stages(d, ntok);
     cfg.ntok = ntok;
     cfg.splits = t->split_k;
     cfg.grid = (int)std::max<long long>(1, std::min<long long>((long long)bs_tiles(d, m, ntok) * t->split_k,
                                                                 (long long)bs_tiles(d, m, ntok) * ks));
     return cfg;
   }
-  // same policy as the W4A16 kernel: whole tiles when they fill the SMs,
-  // an even K split for large token tiles, stream-K otherwise
+  // Whole tiles when they fill the SMs well, a large token tile dropping
+  // to a smaller one for that (one step when that fills >= 85 % of the
+  // SMs; down to 64 tokens for >= 70 %, below which a smaller tile would
+  // re-read the weights from HBM at sizes that are bound by it).  Measured,
+  // whole tiles beat a shared K range here, whose fp32 partial tiles are
+  // large: MXFP4 K=N=7168, M=256: 128-token whole tiles on 112 SMs 23.1 us,
+  // 256-token stream-K 36.8 us; M=128: 64-token whole tiles 16.0 us against
+  // 22.7.  Then an even K split for large tiles, stream-K otherwise.
   const bool fixed_tile = t && t->tile_m;
-  if (!fixed_tile && ntok == 256 && dp_eff(256) < 0.85 && dp_eff(128) >= 0.85) ntok = 128;
+  if (!fixed_tile && ntok >= 64) {
+    int pick = 0;
+    for (int nt = ntok; nt >= ntok / 2 && nt >= 64 && !pick; nt /= 2)
+      if (dp_eff(nt) >= 0.85) pick = nt;
+    for (int nt = ntok; nt >= 64 && !pick; nt /= 2)
+      if (dp_eff(nt) >= 0.7) pick = nt;
+    if (pick) ntok = pick;
+  }
   cfg.ntok = ntok;
+  const long long ks = bs_k_stages(d, ntok);
   const long long tiles = bs_tiles(d, m, ntok);
-  if (dp_eff(ntok) >= 0.85) {
+  if (dp_eff(ntok) >= (ntok >= 64 ? 0.7 : 0.85)) {
     cfg.splits = 0;
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
     return cfg;
