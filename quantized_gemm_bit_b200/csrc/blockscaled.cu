@@ -568,32 +568,32 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
                                                                 (long long)bs_tiles(d, m, ntok) * ks));
     return cfg;
   }
-  // Whole tiles when they fill the SMs well, a large token tile dropping
-  // to a smaller one for that (one step when that fills >= 85 % of the
-  // SMs; down to 64 tokens for >= 70 %, below which a smaller tile would
-  // re-read the weights from HBM at sizes that are bound by it).  Measured,
-  // whole tiles beat a shared K range here, whose fp32 partial tiles are
-  // large: MXFP4 K=N=7168, M=256: 128-token whole tiles on 112 SMs 23.1 us,
-  // 256-token stream-K 36.8 us; M=128: 64-token whole tiles 16.0 us against
-  // 22.7.  Then an even K split for large tiles, stream-K otherwise.
+  // Whole tiles when they fill the SMs well, a token tile dropping to a
+  // smaller one for that (one step when that fills >= 85 % of the SMs; down
+  // to 32 tokens for >= 70 %); else an even K split when whole tiles fill
+  // under half the SMs; else stream-K.  Measured on B200 (K=N=7168), the
+  // fp32 partial tiles of a shared K range cost more than idle SMs here:
+  // MXFP4 M=256: 128-token whole tiles on 112 SMs 23.1 us, 256-token
+  // stream-K 36.8 us; M=64: 32-token whole tiles 14.5 us, stream-K 17.5;
+  // M=16: two K halves per tile on 112 SMs 11.7 us, stream-K 12.8.
   const bool fixed_tile = t && t->tile_m;
-  if (!fixed_tile && ntok >= 64) {
-    int pick = 0;
+  int pick = 0;
+  if (!fixed_tile) {
     for (int nt = ntok; nt >= ntok / 2 && nt >= 64 && !pick; nt /= 2)
       if (dp_eff(nt) >= 0.85) pick = nt;
-    for (int nt = ntok; nt >= 64 && !pick; nt /= 2)
+    for (int nt = ntok; nt >= 32 && !pick; nt /= 2)
       if (dp_eff(nt) >= 0.7) pick = nt;
     if (pick) ntok = pick;
   }
   cfg.ntok = ntok;
   const long long ks = bs_k_stages(d, ntok);
   const long long tiles = bs_tiles(d, m, ntok);
-  if (dp_eff(ntok) >= (ntok >= 64 ? 0.7 : 0.85)) {
+  if (pick || dp_eff(ntok) >= 0.85) {
     cfg.splits = 0;
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
     return cfg;
   }
-  if (ntok >= 128 && tiles * 2 <= dev.num_sms) {
+  if (tiles * 2 <= dev.num_sms && tiles * (dev.num_sms / tiles) >= 0.7 * dev.num_sms) {
     cfg.splits = (int)(dev.num_sms / tiles);
     cfg.grid = (int)std::min<long long>(tiles * cfg.splits, tiles * ks);
     return cfg;
