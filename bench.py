@@ -57,20 +57,20 @@ def load_peaks():
 # profiles/traffic_w4a16_sweep.md.  Emptied whenever the kernels change, so
 # that `traffic` reads null until the capture is taken again.
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 69798400,
-    (4, 7168, 18432): 68901376,
-    (16, 7168, 18432): 69559296,
-    (64, 7168, 18432): 70421504,
-    (256, 7168, 18432): 75667200,
-    (1024, 7168, 18432): 165391872,
-    (4096, 7168, 18432): 445985280,
-    (1, 18432, 7168): 69426432,
-    (4, 18432, 7168): 69673216,
-    (16, 18432, 7168): 70456832,
-    (64, 18432, 7168): 73549312,
-    (256, 18432, 7168): 86308864,
-    (1024, 18432, 7168): 201157376,
-    (4096, 18432, 7168): 723845120,
+    (1, 7168, 18432): 69719808,
+    (4, 7168, 18432): 68965120,
+    (16, 7168, 18432): 69436160,
+    (64, 7168, 18432): 70581760,
+    (256, 7168, 18432): 75671552,
+    (1024, 7168, 18432): 170001152,
+    (4096, 7168, 18432): 465380096,
+    (1, 18432, 7168): 69458176,
+    (4, 18432, 7168): 69744384,
+    (16, 18432, 7168): 70380288,
+    (64, 18432, 7168): 73538816,
+    (256, 18432, 7168): 85825024,
+    (1024, 18432, 7168): 196450304,
+    (4096, 18432, 7168): 715486464,
 }
 
 

@@ -7,8 +7,6 @@ around the grouped GEMMs: routing weights, SwiGLU and the weighted combine
 against their oracle functions with bounds derived from their fp32
 arithmetic, and the whole layer end to end."""
 
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -359,13 +357,4 @@ def test_moe_layer_end_to_end(variant):
                                                    s2.numpy(), k, e, inter)
     assert np.array_equal(ids.cpu().numpy(), ids_ref)
     assert np.array_equal(off.cpu().numpy(), off_ref) and np.array_equal(src.cpu().numpy(), src_ref)
-    got = out.float().double().cpu().numpy()
-    err = got - ref
-    rel = np.linalg.norm(err) / np.linalg.norm(ref)
-    bound = 2e-2 * np.abs(ref) + 4e-3 * np.sqrt(inter) * np.sqrt(np.mean(ref ** 2))
-    log = os.environ.get("HQ_PARITY_LOG")
-    if log:
-        with open(log, "a") as f:
-            f.write(f"moe layer variant={variant} (two-GEMM bar)\t{rel:.3e}\t{np.max(np.abs(err) / bound):.3e}\n")
-    assert rel <= 1e-2, f"moe layer: rel Frobenius {rel:.3e}"
-    assert np.all(np.abs(err) <= bound), f"moe layer: element bound exceeded by {np.max(np.abs(err) - bound):.3e}"
+    check_gemm(out, ref, inter, f"moe layer variant={variant} (two-GEMM bar)", gemms=2)
