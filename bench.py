@@ -96,7 +96,11 @@ class Clocks:
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        # the raw samples go to $HQ_CLOCKS_DIR (default: the system temp
+        # directory); the line printed carries their summary
+        import tempfile
+        out_dir = os.environ.get("HQ_CLOCKS_DIR", tempfile.gettempdir())
+        self.path = os.path.join(out_dir, f"hq_clocks_rank{device_index}.csv")
 
     def __enter__(self):
         try:
