@@ -1,0 +1,190 @@
+"""Offline autotuning of the launch plan for one GEMM shape, through the C ABI.
+
+The pages separate the quantization description from the execution choices
+(token tile, K split, MMA variant) and leave the choice to heuristics, with
+tuning on the roadmap ("Humming: open-source kernel library for quantized
+inference", summary paragraph 3 and key points).  This sweeps those choices
+for one shape on the GPU at hand:
+
+    python -m quantized_gemm_bit_b200.autotune --kind w4a16 --m 16 --k 7168 --n 18432
+    python -m quantized_gemm_bit_b200.autotune --kind mxfp4 --m 256 --k 7168 --n 7168
+    python -m quantized_gemm_bit_b200.autotune --kind moe --m 1024 --k 7168 --n 4096
+
+Every candidate `hq_tuning` (and the library's own choice, `None`) runs as a
+CUDA graph of back-to-back launches over weight copies rotating across more
+than 3x L2, timed with CUDA events; candidates the library refuses are
+skipped, and a candidate whose run records a device-side error is an error.
+The result is a table sorted by time plus the best tuning and its speed-up
+over the library's choice: one entry of a per-shape heuristic table.
+"""
+
+import argparse
+import json
+
+import torch
+
+from . import hq, synth
+
+TILES = (16, 32, 64, 128, 256)
+
+
+def candidates(kind, m):
+    """Tunings worth trying at m rows: token tiles up to twice the rows
+    (at least 16), K splits 0 (the library's choice) to 3, and for the
+    W4A16 kernels both weight variants."""
+    cap = max(16, 2 * m)
+    tiles = [t for t in TILES if t <= cap] or [16]
+    variants = (1, 2) if kind in ("w4a16", "moe") else (0,)
+    splits = (0,) if kind == "moe" else (0, 1, 2, 3)
+    out = [None]
+    for t in tiles:
+        for s in splits:
+            for v in variants:
+                if v == 2 and t > 64:
+                    continue
+                out.append(hq.Tuning(tile_m=t, split_k=s, variant=v))
+    return out
+
+
+def _describe(t):
+    return "library" if t is None else f"tile_m={t.tile_m} split_k={t.split_k} variant={t.variant}"
+
+
+def _time(fn, ncopy, reps=3):
+    """Mean microseconds per call of fn(copy) in a CUDA graph of max(ncopy, 4)
+    back-to-back calls, replayed `reps` times after one warm replay."""
+    r = max(ncopy, 4)
+    for i in range(2):
+        fn(i % ncopy)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for i in range(r):
+            fn(i % ncopy)
+    torch.cuda.current_stream().wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * r)
+
+
+def _copies(blob):
+    l2 = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 126 << 20)
+    n = max(2, -(-3 * l2 // blob.numel()) + 1)
+    return [blob] + [blob.clone() for _ in range(n - 1)]
+
+
+def _setup(kind, m, n, k, experts, topk, dev):
+    """Seeded synthetic inputs of the shape and a call(tuning, copy, c, ws)."""
+    if kind == "w4a16":
+        q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=1000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, 1)
+        blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev))
+        a = synth.bf16_normal(m, k, seed=1001).to(dev)
+        rows = m
+
+        def call(t, i, c, ws):
+            hq.hq_gemm_w4a16(d, blobs[i], a, m, c, ws, t)
+    elif kind == "mxfp4":
+        codes, e8 = synth.mxfp4_weights(n, k, seed=2000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, n, k, 32, 0, 1)
+        blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(dev))
+        aq, asc = synth.fp8_activations(m, k, seed=2001)
+        aq, asc = aq.to(dev), asc.to(dev)
+        rows = m
+
+        def call(t, i, c, ws):
+            hq.hq_gemm_mxfp4_a8(d, blobs[i], aq, asc, m, c, ws, t)
+    elif kind == "nvfp4":
+        def quant(r, seed):
+            x = synth.bf16_normal(r, k, seed).to(dev)
+            codes = torch.empty(r, k // 2, dtype=torch.uint8, device=dev)
+            sf = torch.empty(r, k // 16, dtype=torch.uint8, device=dev)
+            g = torch.empty(1, dtype=torch.float32, device=dev)
+            wsq = torch.zeros(hq.hq_quantize_nvfp4_workspace_size(r, k), dtype=torch.uint8, device=dev)
+            hq.hq_quantize_nvfp4(x, r, k, codes, sf, g, wsq)
+            return codes, sf, float(g.item())
+        wc, wsf, wg = quant(n, 4000)
+        ac, asf, ag = quant(m, 4100)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, n, k, 16, 0, 1)
+        blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, wc.cpu(), wsf.cpu(), None, wg)).to(dev))
+        rows = m
+
+        def call(t, i, c, ws):
+            hq.hq_gemm_nvfp4(d, blobs[i], ac, asf, ag, m, c, ws, t)
+    elif kind == "moe":
+        # m = tokens routed top-k over `experts`; the grouped GEMM runs on the
+        # m * topk expert-sorted rows
+        q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=3000, experts=experts)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, experts)
+        blobs = [torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev)]
+        logits = synth.router_logits(m, experts, seed=3001).to(dev)
+        ids = torch.empty(m, topk, dtype=torch.int32, device=dev)
+        src = torch.empty(m * topk, dtype=torch.int32, device=dev)
+        off = torch.empty(experts + 1, dtype=torch.int32, device=dev)
+        pws = torch.zeros(hq.hq_moe_permute_workspace_size(m, topk, experts), dtype=torch.uint8, device=dev)
+        hq.hq_moe_topk(logits, m, experts, topk, ids)
+        hq.hq_moe_permute(ids, m, topk, experts, src, off, pws)
+        rows = m * topk
+        a = synth.bf16_normal(rows, k, seed=3002).to(dev)
+
+        def call(t, i, c, ws):
+            hq.hq_grouped_gemm_moe(d, blobs[i], a, off, rows, c, ws, t)
+    else:
+        raise ValueError(kind)
+    return d, rows, len(blobs), call
+
+
+def autotune(kind, m, n, k, experts=256, topk=8, tunings=None, dev="cuda"):
+    """Times every candidate tuning; returns (rows sorted by time, best row,
+    the library's row).  A row is {"tuning": ..., "us": ..., "desc": ...}."""
+    d, rows, ncopy, call = _setup(kind, m, n, k, experts, topk, dev)
+    c = torch.empty(rows, n, dtype=torch.bfloat16, device=dev)
+    results = []
+    for t in (candidates(kind, m) if tunings is None else tunings):
+        try:
+            ws = torch.zeros(max(256, hq.hq_workspace_size(d, rows, t)), dtype=torch.uint8, device=dev)
+            us = _time(lambda i: call(t, i, c, ws), ncopy)
+        except hq.HQError:
+            continue                      # refused by the library: not a valid plan here
+        st = hq.hq_check_device_status(ws)
+        if st != hq.HQ_OK:
+            raise RuntimeError(f"{_describe(t)}: device status {hq.status_string(st)}")
+        results.append({"tuning": t, "us": us, "desc": _describe(t)})
+    results.sort(key=lambda r: r["us"])
+    library = next(r for r in results if r["tuning"] is None)
+    return results, results[0], library
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "mxfp4", "nvfp4", "moe"])
+    ap.add_argument("--m", type=int, default=16, help="rows (tokens for --kind moe)")
+    ap.add_argument("--k", type=int, default=7168)
+    ap.add_argument("--n", type=int, default=18432)
+    ap.add_argument("--experts", type=int, default=256)
+    ap.add_argument("--topk", type=int, default=8)
+    a = ap.parse_args(argv)
+    from .build import build
+    build()
+    results, best, library = autotune(a.kind, a.m, a.n, a.k, a.experts, a.topk)
+    for r in results:
+        print(f"{r['us']:10.2f} us  {r['desc']}")
+    t = best["tuning"]
+    print(json.dumps({"kind": a.kind, "m": a.m, "n": a.n, "k": a.k,
+                      "best": None if t is None else {"tile_m": t.tile_m, "split_k": t.split_k, "variant": t.variant},
+                      "best_us": round(best["us"], 2), "library_us": round(library["us"], 2),
+                      "speedup_over_library": round(library["us"] / best["us"], 3)}))
+
+
+if __name__ == "__main__":
+    main()

@@ -174,3 +174,12 @@ def test_workspace_size_is_deterministic_and_covers_header():
 def test_status_strings():
     for s in range(10):
         assert hq.status_string(s)
+
+
+def test_autotune_candidates_need_no_gpu():
+    from quantized_gemm_bit_b200 import autotune
+    c = autotune.candidates("w4a16", 16)
+    assert c[0] is None and all(t.tile_m in (16, 32) for t in c[1:])
+    assert not any(t.variant == 2 and t.tile_m > 64 for t in autotune.candidates("w4a16", 4096)[1:])
+    assert all(t.variant == 0 for t in autotune.candidates("nvfp4", 256)[1:])
+    assert all(t.split_k == 0 for t in autotune.candidates("moe", 64)[1:])
