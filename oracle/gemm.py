@@ -179,6 +179,25 @@ def nvfp4_ref_exact(a_packed, a_sf, a_g, w_packed, w_sf, w_g):
 # ---------------------------------------------------------------------------
 
 
+def _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols):
+    """Rows of C_sorted: row i uses the weights of the expert e whose range
+    [offsets[e], offsets[e+1]) holds i; dequant(e) gives W_hat_e (fp64,
+    ncols rows)."""
+    off = np.asarray(expert_offsets, dtype=np.int64)
+    e_count = off.shape[0] - 1
+    assert e_count >= 1
+    total = int(off[-1])
+    rows = np.arange(total) if row_subset is None else np.asarray(row_subset, dtype=np.int64)
+    expert_of = np.searchsorted(off, rows, side="right") - 1
+    out = np.zeros((len(rows), ncols))
+    for e in np.unique(expert_of):
+        sel = np.nonzero(expert_of == e)[0]
+        w = dequant(int(e))
+        a = F.bf16_bits_to_f64(np.asarray(a_sorted_bf16)[rows[sel]])
+        out[sel] = a @ w.T
+    return rows, out
+
+
 def grouped_w4a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, group,
                       row_subset=None, cols=None):
     """C_sorted[i, :] = A_sorted_hat[i, :] @ W_hat_e.T for the expert e whose
@@ -189,19 +208,33 @@ def grouped_w4a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, gr
     in the given order); cols restricts the output columns.
     Returns (rows, C) with C fp64 [len(rows), len(cols) or N].
     """
-    off = np.asarray(expert_offsets, dtype=np.int64)
-    e_count = off.shape[0] - 1
-    total = int(off[-1])
-    rows = np.arange(total) if row_subset is None else np.asarray(row_subset, dtype=np.int64)
-    n = np.asarray(qweights).shape[1]
-    ncols = n if cols is None else len(cols)
-    out = np.zeros((len(rows), ncols))
-    expert_of = np.searchsorted(off, rows, side="right") - 1
-    for e in np.unique(expert_of):
-        sel = np.nonzero(expert_of == e)[0]
+    def dequant(e):
         z = None if zeros is None else zeros[e]
-        w = w4a16_dequant(qweights[e], scales[e], z, group, rows=cols)
-        a = F.bf16_bits_to_f64(np.asarray(a_sorted_bf16)[rows[sel]])
-        out[sel] = a @ w.T
-    assert e_count >= 1
-    return rows, out
+        return w4a16_dequant(qweights[e], scales[e], z, group, rows=cols)
+    ncols = np.asarray(qweights).shape[1] if cols is None else len(cols)
+    return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 weights x bf16 activations (the W4A16 kernels with MXFP4 weights)
+# ---------------------------------------------------------------------------
+
+
+def mxfp4_a16_ref(a_bf16, w_packed, w_e8m0, rows=None, cols=None):
+    """C = A_hat @ W_hat.T in fp64 with A_hat the bf16 activations widened
+    exactly and W_hat[n, k] = e2m1(c[n, k]) * 2**(e[n, k // 32] - 127), the
+    MXFP4 weight of the OCP MX definition (the pages list MXFP4 among the
+    weight types and bf16 among the activation types, "Humming: open-source
+    kernel library for quantized inference", summary, second paragraph)."""
+    a = F.bf16_bits_to_f64(a_bf16 if rows is None else np.asarray(a_bf16)[rows])
+    w = mxfp4_dequant(w_packed, w_e8m0, rows=cols)
+    return a @ w.T
+
+
+def grouped_mxfp4_a16_ref(a_sorted_bf16, expert_offsets, w_packed, w_e8m0, row_subset=None, cols=None):
+    """Grouped form of mxfp4_a16_ref over expert-sorted rows: w_packed uint8
+    [E, N, K/2], w_e8m0 uint8 [E, N, K/32].  Returns (rows, C)."""
+    def dequant(e):
+        return mxfp4_dequant(w_packed[e], w_e8m0[e], rows=cols)
+    ncols = np.asarray(w_packed).shape[1] if cols is None else len(cols)
+    return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)

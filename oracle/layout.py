@@ -19,6 +19,9 @@ INT4 W4A16, layout version 1 (group size 128):
     zero   : uint8 at byte 8192 + 256 + r (only with zero points).
   Rows n >= N (tile padding) hold code 0, scale 0 and zero 0.
   Experts (MoE) are stored one after another, each NT*KB*REC bytes.
+
+MXFP4 / NVFP4 for the block-scaled kernels, and MXFP4 for the W4A16
+kernels (bf16 activations), follow further down, each with its formulas.
 """
 
 import numpy as np
@@ -150,3 +153,85 @@ def fp4_pack(codes_packed, scales, block, global_scale=None):
     if global_scale is not None:
         out[-16:-12] = np.frombuffer(np.float32(global_scale).tobytes(), dtype=np.uint8)
     return out
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 weights for bf16 activations (W4A16 kernels), layout version 1
+#   Records as for INT4: one per (tile nt of 128 rows, block kb of 128 K), in
+#   (nt, kb) order, experts one after another; record size 8192 + 512 bytes.
+#   codes : the 32-bit little-endian word at byte (c*128 + r)*16 + 4*w of the
+#           record holds the 8 codes kk = 32c + 8w + 2j + h (j < 4, h < 2),
+#           where r = n - 128*nt and kk = k - 128*kb.  Bit b of code
+#           (b = 0 mantissa, 1 and 2 exponent, 3 sign) sits at word bit
+#           MXA16_BITS[j][h][b].
+#   scales: the E8M0 byte of row n, 32-K block 4*kb + c at byte 8192 + 4*r + c.
+#   Rows n >= N (tile padding) hold code 0 and scale byte 0.
+# ---------------------------------------------------------------------------
+
+MXA16_REC = 8192 + 512
+
+# [pair j][half h] -> word bit of (mantissa, exponent bit 0, exponent bit 1, sign)
+MXA16_BITS = (
+    ((6, 7, 8, 15), (22, 23, 24, 31)),
+    ((10, 11, 12, 19), (26, 27, 28, 3)),
+    ((16, 17, 18, 25), (0, 1, 2, 9)),
+    ((4, 5, 14, 13), (20, 21, 30, 29)),
+)
+
+
+def mxa16_packed_bytes(n, k, num_experts=1):
+    return num_experts * (-(-n // 128)) * (k // 128) * MXA16_REC
+
+
+def mxa16_code_word_and_bits(n, k, kdim):
+    """Elementwise formula: (byte offset of the 32-bit word in the expert
+    blob, [4] word bits of code bits 0..3) for code (n, k)."""
+    n = np.asarray(n, dtype=np.int64)
+    k = np.asarray(k, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    kb, kk = k // 128, k % 128
+    c, w, j, h = kk // 32, (kk % 32) // 8, (kk % 8) // 2, kk % 2
+    word = (nt * (kdim // 128) + kb) * MXA16_REC + (c * 128 + r) * 16 + 4 * w
+    table = np.asarray(MXA16_BITS, dtype=np.int64)        # [4, 2, 4]
+    return word, table[j, h]
+
+
+def mxa16_scale_byte(n, blk, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    blk = np.asarray(blk, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    kb, c = blk // 4, blk % 4
+    return (nt * (kdim // 128) + kb) * MXA16_REC + 8192 + 4 * r + c
+
+
+def mxa16_pack(codes_packed, scales):
+    """Canonical (uint8 [N, K/2] even k low nibble, uint8 E8M0 [N, K/32])
+    -> packed blob of one expert, by placing every code bit and every scale
+    byte where the formulas above say."""
+    codes = F.fp4_unpack_bytes(np.asarray(codes_packed, dtype=np.uint8)).astype(np.uint32)
+    n, k = codes.shape
+    out = np.zeros(mxa16_packed_bytes(n, k), dtype=np.uint8)
+    words = np.zeros(out.size // 4, dtype=np.uint32)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    word, bits = mxa16_code_word_and_bits(nn.ravel(), kk.ravel(), k)
+    c = codes.ravel()
+    for b in range(4):
+        np.bitwise_or.at(words, word // 4, ((c >> b) & 1) << bits[:, b].astype(np.uint32))
+    out[:] = words.view(np.uint8)                          # little endian words
+    ns, bs = np.meshgrid(np.arange(n), np.arange(k // 32), indexing="ij")
+    out[mxa16_scale_byte(ns.ravel(), bs.ravel(), k)] = np.asarray(scales, dtype=np.uint8).ravel()
+    return out
+
+
+def mxa16_unpack(blob, n, k):
+    """Inverse of mxa16_pack: blob -> (codes uint8 [N, K], scales uint8 [N, K/32])."""
+    words = np.asarray(blob, dtype=np.uint8).view(np.uint32)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    word, bits = mxa16_code_word_and_bits(nn.ravel(), kk.ravel(), k)
+    wv = words[word // 4]
+    codes = np.zeros(n * k, dtype=np.uint32)
+    for b in range(4):
+        codes |= ((wv >> bits[:, b].astype(np.uint32)) & 1) << b
+    ns, bs = np.meshgrid(np.arange(n), np.arange(k // 32), indexing="ij")
+    scales = np.asarray(blob, dtype=np.uint8)[mxa16_scale_byte(ns.ravel(), bs.ravel(), k)]
+    return codes.reshape(n, k).astype(np.uint8), scales.reshape(n, k // 32)

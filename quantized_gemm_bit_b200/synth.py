@@ -12,8 +12,9 @@ Recipes (one per workload; seed = workload index * 1000 + shape index):
     0.002 + 0.01*|N(0,1)| per (row, group of 128 along K); zero points
     uniform in [0, 15] (asymmetric) or none (symmetric, zero point 8);
     activations bf16 N(0,1).
-  * W4A8-MXFP4: FP4 codes uniform over the 16 codes, two per byte (even k
-    low nibble); one E8M0 scale per 32 K with exponent uniform in [-8, -2];
+  * W4A8-MXFP4 (and MXFP4 weights with bf16 activations): FP4 codes
+    uniform over the 16 codes, two per byte (even k low nibble); one E8M0
+    scale per 32 K with exponent uniform in [-8, -2];
     activations bf16 N(0,1) widened to fp32, per-token scale amax/448 (fp32),
     E4M3 codes by torch's cast of x/scale (clamped to +-448).
   * NVFP4: bf16 N(0,1) draws for both operands; the two-level quantization
@@ -52,13 +53,15 @@ def w4a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
     return qweight, scales, zeros
 
 
-def mxfp4_weights(n, k, seed=0):
-    """MXFP4 weights: codes uint8 [N, K/2] (two uniform FP4 codes per byte),
-    E8M0 scales uint8 [N, K/32] with exponent uniform in [-8, -2]."""
+def mxfp4_weights(n, k, seed=0, experts=None):
+    """MXFP4 weights: codes uint8 [.., N, K/2] (two uniform FP4 codes per
+    byte), E8M0 scales uint8 [.., N, K/32] with exponent uniform in [-8, -2].
+    With `experts` set, a leading expert dimension is added."""
     assert k % 32 == 0
     g = _gen(seed)
-    codes = torch.randint(0, 256, (n, k // 2), generator=g, dtype=torch.uint8)
-    e8m0 = (127 + torch.randint(-8, -1, (n, k // 32), generator=g, dtype=torch.int32)).to(torch.uint8)
+    lead = () if experts is None else (experts,)
+    codes = torch.randint(0, 256, lead + (n, k // 2), generator=g, dtype=torch.uint8)
+    e8m0 = (127 + torch.randint(-8, -1, lead + (n, k // 32), generator=g, dtype=torch.int32)).to(torch.uint8)
     return codes, e8m0
 
 
