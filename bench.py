@@ -465,6 +465,43 @@ def run_mxfp4(args, rank, world, peaks):
             "detail": out}
 
 
+def run_mxfp4_a16(args, rank, world, peaks):
+    """MXFP4 weights x bf16 activations on the W4A16 kernels: M in
+    {16, 64, 256, 4096}, K=7168, N=18432."""
+    from quantized_gemm_bit_b200 import hq, synth
+    k, n = 7168, 18432
+    codes, e8 = synth.mxfp4_weights(n, k, seed=6000)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, n, k, 32, 0, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).cuda()
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    ms_list = (16, 64, 256, 4096)
+    ncopy_w = max(2, int(np.ceil(3 * l2 / blob.numel())) + 1)
+    blobs = [blob] + [blob.clone() for _ in range(ncopy_w - 1)]
+    launches = []
+    for j, m in enumerate(ms_list):
+        a = synth.bf16_normal(m, k, seed=6001 + m).cuda()
+        c = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(max(256, hq.hq_workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+
+        def f(cp, j=j, m=m, a=a, c=c, ws=ws):
+            hq.hq_gemm_w4a16(d, blobs[(cp * len(ms_list) + j) % len(blobs)], a, m, c, ws)
+        launches.append(f)
+    ncopy = len(blobs) // np.gcd(len(blobs), len(ms_list))
+    ms, per = _time_launches(launches, args.steps, args.warmup, world, ncopy=int(ncopy))
+    out = []
+    for m, us in zip(ms_list, per):
+        fl = 2.0 * m * n * k
+        by = n * k // 2 + n * k // 32 + 2 * m * k + 2 * m * n
+        out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1), gbs=round(by / us / 1e3, 1),
+                        frac_hbm=round(by / us / 1e3 / peaks["hbm_gbs"], 3),
+                        frac_bf16_peak=round(fl / us / 1e6 / peaks["bf16_tflops"], 3)))
+    flops = sum(2.0 * m * n * k for m in ms_list)
+    return {"workload": "MXFP4 weights x bf16 activations (W4A16 kernels), M in {16,64,256,4096}, K=7168, N=18432",
+            "value": round(flops * args.steps * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms / args.steps, 4), "dtype": "bf16 x e2m1 (fp32 accumulate)", "detail": out}
+
+
 def run_nvfp4(args, rank, world, peaks):
     """NVFP4 W4A4: 8192^3 and M=16384, K=7168, N=18432 (inputs quantized from
     bf16 N(0,1) draws on the GPU by the library's own quantizer)."""
@@ -653,7 +690,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "nvfp4", "moe"])
+    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "nvfp4", "moe"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -676,7 +713,7 @@ def main():
     if args.workload == "w4a16_sweep":
         line = run_w4a16_sweep(args, rank, world, peaks)
     else:
-        fn = {"mxfp4": run_mxfp4, "nvfp4": run_nvfp4, "moe": run_moe}[args.workload]
+        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "nvfp4": run_nvfp4, "moe": run_moe}[args.workload]
         line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "data": "synthetic (seeded)"}
         line.update(fn(args, rank, world, peaks))

@@ -81,7 +81,9 @@ typedef enum {
 typedef enum {
   HQ_FMT_INT4 = 1,  /* unsigned INT4 codes, fp16 scale + optional uint4 zero point per group of 128 K */
   HQ_FMT_MXFP4 = 2, /* e2m1 codes, E8M0 scale per 32 K                                             */
-  HQ_FMT_NVFP4 = 3  /* e2m1 codes, E4M3 scale per 16 K, fp32 tensor scale                          */
+  HQ_FMT_NVFP4 = 3, /* e2m1 codes, E4M3 scale per 16 K, fp32 tensor scale                          */
+  HQ_FMT_MXFP4_A16 = 4 /* e2m1 codes, E8M0 scale per 32 K, for bf16 activations: the W4A16 entry
+                          points dequantize it in registers like INT4                               */
 } hq_format;
 
 /* Quantization description ([P-fa2] paragraph 2) plus the Layer Config
@@ -91,7 +93,7 @@ typedef struct {
   int32_t fmt;            /* hq_format                                                 */
   int32_t n;              /* output features (weight rows), per expert                 */
   int32_t k;              /* input features (reduction length)                         */
-  int32_t group_size;     /* INT4: 128; MXFP4: 32; NVFP4: 16                           */
+  int32_t group_size;     /* INT4: 128; MXFP4, MXFP4_A16: 32; NVFP4: 16                */
   int32_t has_zero_point; /* INT4: 1 = uint4 zero point per group, 0 = symmetric (8)   */
   int32_t num_experts;    /* 1 = dense layer; >1 = MoE weights stored expert after expert */
 } hq_quant_desc;
@@ -130,7 +132,8 @@ const char* hq_status_string(hq_status s);
  *   INT4 : k % 128 == 0, group_size == 128, n >= 1
  *   MXFP4: k % 128 == 0, group_size == 32, has_zero_point == 0
  *   NVFP4: k % 256 == 0, group_size == 16, has_zero_point == 0
- *   num_experts >= 1 (MoE only for INT4). */
+ *   MXFP4_A16: k % 128 == 0, group_size == 32, has_zero_point == 0
+ *   num_experts 1..1024 for INT4 and MXFP4_A16 (MoE), 1 otherwise. */
 hq_status hq_quant_desc_init(hq_quant_desc* d, int32_t fmt, int32_t n, int32_t k, int32_t group_size,
                              int32_t has_zero_point, int32_t num_experts);
 
@@ -148,6 +151,9 @@ size_t hq_packed_size(const hq_quant_desc* d);
  *          scales_host = uint8 E8M0 [N][K/32]
  *   NVFP4: codes_host  = uint8 [N][K/2]; scales_host = uint8 E4M3 [N][K/16];
  *          global_scale = the fp32 tensor scale of the weights.
+ *   MXFP4_A16: codes_host = uint8 [E][N][K/2] (even k in the low nibble),
+ *          scales_host = uint8 E8M0 [E][N][K/32], every byte <= 252 (a
+ *          larger scale would overflow bf16 weights, 255 is NaN).
  * The output layout (layout version 1) is spelled out in the header comment
  * of the packer source, hq_pack.cpp.
  * Errors: HQ_ERR_INVALID_ARG (NULL pointers, zeros given for a symmetric
@@ -156,14 +162,21 @@ size_t hq_packed_size(const hq_quant_desc* d);
 hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
                           const void* zeros_host, float global_scale, void* out_host, size_t out_bytes);
 
-/* Workspace bytes that hq_gemm_w4a16 (fmt INT4, num_experts 1),
+/* Workspace bytes that hq_gemm_w4a16 (fmt INT4 or MXFP4_A16, num_experts 1),
  * hq_gemm_mxfp4_a8, hq_gemm_nvfp4 or hq_grouped_gemm_moe need for M rows
  * (total sorted rows for MoE) and the given tuning (NULL = heuristic). */
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
 
 /* Dense W4A16 GEMM ([P-fa] table row "W4A16 dense"): C = A * W_hat^T with
  * W_hat[n,k] = (q[n,k] - z[n,k/128]) * s[n,k/128] dequantized in-kernel.
- *   d            : INT4 descriptor with num_experts == 1
+ *   d            : INT4 or MXFP4_A16 descriptor with num_experts == 1.
+ *                  MXFP4_A16 (MXFP4 weights with bf16 activations; [P-fa2]
+ *                  paragraph 2 lists MXFP4 weights and bf16 activations):
+ *                  W_hat[n,k] = e2m1(c[n,k]) * 2^(e[n,k/32] - 127), each
+ *                  weight converted to bf16 exactly (every scale byte <= 252
+ *                  keeps it finite) and accumulated in fp32; tuning variant
+ *                  2 is refused with HQ_ERR_UNSUPPORTED (one scale per 32 K
+ *                  leaves nothing to factor out of a 128-K group).
  *   packed_w_dev : blob from hq_pack_weights (hq_packed_size bytes)
  *   a_dev        : bf16 [m][d->k]
  *   m            : rows of A (m == 0 returns HQ_OK without launching)
@@ -245,7 +258,9 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
  * "MoE W4A16"): for every expert e, rows [off[e], off[e+1]) of A_sorted
  * times W_hat_e^T.  The tile scheduler reads expert_offsets on the device
  * (no host synchronization).
- *   d              : INT4 descriptor, num_experts = e (per-expert n, k)
+ *   d              : INT4 or MXFP4_A16 descriptor, num_experts = e
+ *                    (per-expert n, k); MXFP4_A16 weights as for
+ *                    hq_gemm_w4a16
  *   packed_w_dev   : blob of all experts from hq_pack_weights
  *   a_sorted_dev   : bf16 [total_rows][k]
  *   expert_offsets_dev : int32 [e+1], monotone, offsets[e] == total_rows

@@ -72,12 +72,41 @@ hq_status check_desc(const hq_quant_desc* d) {
       if (d->group_size != 16 || d->k % 256 != 0 || d->has_zero_point || d->num_experts != 1)
         return HQ_ERR_UNSUPPORTED;
       return HQ_OK;
+    case HQ_FMT_MXFP4_A16:
+      if (d->group_size != 32 || d->k % 128 != 0 || d->has_zero_point || d->num_experts > 1024)
+        return HQ_ERR_UNSUPPORTED;
+      return HQ_OK;
     default:
       return HQ_ERR_INVALID_ARG;
   }
 }
 
+// Formats the W4A16 kernels read (dequantized in registers, bf16 MMA).
+bool w4_format(const hq_quant_desc* d) { return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_MXFP4_A16; }
+
+// Tuning checks shared by the W4A16 entry points (dense: split_k free;
+// grouped: at most one CTA per tile).
+hq_status check_w4_tuning(const hq_quant_desc* d, const hq_tuning* t, bool grouped) {
+  if (!t) return HQ_OK;
+  if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
+    return HQ_ERR_UNSUPPORTED;
+  if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
+      (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
+    return HQ_ERR_UNSUPPORTED;
+  if (grouped && t->split_k > 1) return HQ_ERR_UNSUPPORTED;
+  // exact (q - z) weights need one scale per 128-K group
+  if (d->fmt == HQ_FMT_MXFP4_A16 && t->variant == 2) return HQ_ERR_UNSUPPORTED;
+  return HQ_OK;
+}
+
 }  // namespace
+
+hq_status check_w4_call(const hq_quant_desc* d, const hq_tuning* t, bool grouped) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (!w4_format(d) || (grouped ? d->num_experts < 2 : d->num_experts != 1)) return HQ_ERR_INVALID_ARG;
+  return check_w4_tuning(d, t, grouped);
+}
 
 // Packed size per format (the layouts are written out in hq_pack.cpp).
 size_t packed_size_impl(const hq_quant_desc& d);
@@ -152,7 +181,7 @@ size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t) 
     // still an upper bound the caller can allocate
     dev.num_sms = 148;
   }
-  if (d->fmt != HQ_FMT_INT4) {
+  if (!w4_format(d)) {
     BsConfig cfg = bs_plan(dev, *d, m < 1 ? 1 : m, t);
     return bs_workspace_bytes(*d, m < 1 ? 1 : m, cfg);
   }
@@ -165,19 +194,14 @@ hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const 
                         void* c_dev, const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
-  if (d->fmt != HQ_FMT_INT4 || d->num_experts != 1) return HQ_ERR_INVALID_ARG;
+  if (!w4_format(d) || d->num_experts != 1) return HQ_ERR_INVALID_ARG;
   if (m < 0) return HQ_ERR_INVALID_ARG;
   if (m == 0) return HQ_OK;
   if (!packed_w_dev || !a_dev || !c_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
   if (!aligned(packed_w_dev, 16) || !aligned(a_dev, 16) || !aligned(c_dev, 16) || !aligned(ws_dev, 256))
     return HQ_ERR_ALIGNMENT;
-  if (t) {
-    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
-      return HQ_ERR_UNSUPPORTED;
-    if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
-        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
-      return HQ_ERR_UNSUPPORTED;
-  }
+  st = check_w4_tuning(d, t, false);
+  if (st != HQ_OK) return st;
   DeviceInfo dev{};
   st = device_info(&dev);
   if (st != HQ_OK) return st;
@@ -191,20 +215,15 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
                               const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
-  if (d->fmt != HQ_FMT_INT4 || d->num_experts < 2) return HQ_ERR_INVALID_ARG;
+  if (!w4_format(d) || d->num_experts < 2) return HQ_ERR_INVALID_ARG;
   if (total_rows < 0) return HQ_ERR_INVALID_ARG;
   if (total_rows == 0) return HQ_OK;
   if (!packed_w_dev || !a_sorted_dev || !expert_offsets_dev || !c_sorted_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
   if (!aligned(packed_w_dev, 16) || !aligned(a_sorted_dev, 16) || !aligned(c_sorted_dev, 16) ||
       !aligned(expert_offsets_dev, 4) || !aligned(ws_dev, 256))
     return HQ_ERR_ALIGNMENT;
-  if (t) {
-    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
-      return HQ_ERR_UNSUPPORTED;
-    if (t->split_k > 1 || (t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->stages != 0 ||
-        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
-      return HQ_ERR_UNSUPPORTED;
-  }
+  st = check_w4_tuning(d, t, true);
+  if (st != HQ_OK) return st;
   DeviceInfo dev{};
   st = device_info(&dev);
   if (st != HQ_OK) return st;

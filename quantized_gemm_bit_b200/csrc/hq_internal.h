@@ -20,6 +20,9 @@ constexpr int kTileN = 128;      // weight rows per tile (MMA M)
 constexpr int kBlockK = 128;     // K per packed record / pipeline stage
 constexpr int kW4RecCodes = 8192;
 inline int w4_record_bytes(bool has_zero) { return kW4RecCodes + 256 + (has_zero ? 128 : 0); }
+// MXFP4 weights for the W4A16 kernels: 8192 code bytes, then one E8M0 byte
+// per (row, 32-K block) of the record
+constexpr int kMxA16RecBytes = kW4RecCodes + 512;
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -43,6 +46,10 @@ struct DeviceInfo {
   size_t max_smem_optin;
 };
 hq_status device_info(DeviceInfo* out);
+
+// Descriptor, format and tuning checks of a W4A16-family call (INT4 or
+// MXFP4_A16 weights; grouped: num_experts >= 2, else exactly 1).
+hq_status check_w4_call(const hq_quant_desc* d, const hq_tuning* t, bool grouped);
 
 // W4A16 (dense or grouped) planning and launch.
 W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t);

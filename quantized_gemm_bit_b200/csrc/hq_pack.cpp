@@ -32,6 +32,21 @@
 //           in (nt, g) order; byte l*16 + 4*c + j = scale of row
 //           nt*128 + l + 32*c for the 16-K block 4*g + j
 //   tail  : 16 bytes; the fp32 tensor scale in the first 4.
+//
+// MXFP4 for bf16 activations (MXFP4_A16: the W4A16 kernels dequantize it).
+// Records as for INT4 (one per (tile nt, 128-K block kb), experts one after
+// another), 8192 + 512 bytes each:
+//   [0, 8192)      codes: the 32-bit word at byte (c*128 + r)*16 + 4*w holds
+//                  the 8 codes kk = 32c + 8w + 2j + h (pair j < 4, half
+//                  h < 2); bit b of a code (0 mantissa, 1-2 exponent, 3
+//                  sign) sits at word bit kMxBits[j][h][b].
+//   [8192, 8704)   E8M0 scale of row r, 32-K block c at 8192 + 4r + c.
+// The bit positions are chosen so that pair j's two codes land, after the
+// kernel rotates the word right by 0, 4 or 10 bits (j = 0, 1, 2) or merges
+// two rotations (j = 3), on the bits a bf16x2 word gives its sign (15), the
+// low two exponent bits (8..7) and the top mantissa bit (6): one mask per
+// pair then leaves two bf16 values e2m1 * 2^-126, and one multiply by a
+// power of two applies 2^126 times the block scale.
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -116,6 +131,56 @@ hq_status pack_int4(const hq_quant_desc& d, const int32_t* codes, const uint16_t
   return HQ_OK;
 }
 
+// [pair j][half h][code bit b] -> bit of the 32-bit word
+constexpr int kMxBits[4][2][4] = {
+    {{6, 7, 8, 15}, {22, 23, 24, 31}},
+    {{10, 11, 12, 19}, {26, 27, 28, 3}},
+    {{16, 17, 18, 25}, {0, 1, 2, 9}},
+    {{4, 5, 14, 13}, {20, 21, 30, 29}},
+};
+
+hq_status pack_mx_a16(const hq_quant_desc& d, const uint8_t* codes, const uint8_t* scales, uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int nt_count = (n + kTileN - 1) / kTileN;
+  const int kb_count = k / kBlockK;
+  const size_t rec = (size_t)kMxA16RecBytes;
+  const size_t expert_bytes = (size_t)nt_count * kb_count * rec;
+  const size_t row_bytes = (size_t)k / 2, row_scales = (size_t)k / 32;
+  // scales above 2^125 would make bf16 weights overflow (255 is NaN)
+  const size_t total_scales = (size_t)d.num_experts * n * row_scales;
+  for (size_t i = 0; i < total_scales; ++i)
+    if (scales[i] > 252) return HQ_ERR_INVALID_ARG;
+  const size_t jobs = (size_t)d.num_experts * nt_count;
+  parallel_for(jobs, [&](size_t job) {
+    const size_t e = job / nt_count;
+    const int nt = (int)(job % nt_count);
+    uint8_t* ebase = out + e * expert_bytes;
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint8_t* r0 = ebase + ((size_t)nt * kb_count + kb) * rec;
+      std::memset(r0, 0, rec);
+      for (int r = 0; r < kTileN; ++r) {
+        const int row = nt * kTileN + r;
+        if (row >= n) break;
+        const uint8_t* src = codes + (e * n + row) * row_bytes + (size_t)kb * 64;
+        for (int c = 0; c < 4; ++c) {
+          for (int w = 0; w < 4; ++w) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j)
+              for (int h = 0; h < 2; ++h) {
+                const int kk = 32 * c + 8 * w + 2 * j + h;
+                const uint32_t code = (src[kk / 2] >> (4 * (kk % 2))) & 0xF;
+                for (int b = 0; b < 4; ++b) word |= ((code >> b) & 1u) << kMxBits[j][h][b];
+              }
+            std::memcpy(r0 + ((size_t)c * 128 + r) * 16 + 4 * w, &word, 4);
+          }
+          r0[kW4RecCodes + 4 * r + c] = scales[(e * n + row) * row_scales + (size_t)kb * 4 + c];
+        }
+      }
+    }
+  });
+  return HQ_OK;
+}
+
 // Block-scaled formats: copy codes row by row, then lay out scale blocks.
 hq_status pack_fp4(const hq_quant_desc& d, const uint8_t* codes, const uint8_t* scales, float g, uint8_t* out) {
   const int n = d.n, k = d.k;
@@ -159,6 +224,8 @@ size_t packed_size_impl(const hq_quant_desc& d) {
       return nt * kTileN * (size_t)d.k / 2 + nt * (d.k / 128) * 512;
     case HQ_FMT_NVFP4:
       return nt * kTileN * (size_t)d.k / 2 + nt * (d.k / 64) * 512 + 16;
+    case HQ_FMT_MXFP4_A16:
+      return (size_t)d.num_experts * nt * (d.k / kBlockK) * kMxA16RecBytes;
     default:
       return 0;
   }
@@ -174,6 +241,9 @@ hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scale
     case HQ_FMT_NVFP4:
       return pack_fp4(d, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales), g,
                       static_cast<uint8_t*>(out));
+    case HQ_FMT_MXFP4_A16:
+      return pack_mx_a16(d, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales),
+                         static_cast<uint8_t*>(out));
     default:
       return HQ_ERR_INVALID_ARG;
   }

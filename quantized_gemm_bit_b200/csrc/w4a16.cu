@@ -44,14 +44,17 @@ namespace {
 
 constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 
-template <int NTOK>
+// MX: MXFP4 weight records (8704 bytes; the tighter barrier area keeps the
+// 256-token tile inside the shared-memory limit)
+template <int NTOK, bool MX = false>
 struct Cfg {
   // records (128-K blocks) per pipeline stage: two for the small token tiles,
   // whose MMAs are cheap, so the per-stage waits and commits are amortized
   static constexpr int kKps = NTOK <= 64 ? 2 : 1;
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
-  static constexpr int kRecs = kKps * kRecMax;
+  static constexpr int kRecStride = MX ? kMxA16RecBytes : kRecMax;
+  static constexpr int kRecs = kKps * kRecStride;
   static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
   static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
@@ -69,13 +72,13 @@ struct Cfg {
   // it aliases the expert tables, so grouped 256-token tiles store their
   // outputs element by element instead
   static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
-  static constexpr int kBarBytes = 512;
+  static constexpr int kBarBytes = MX ? 384 : 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
   static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
   static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
   static constexpr size_t kScrOff = (kTabOff + 2 * (kMaxExperts + 1) * sizeof(int) + 127) / 128 * 128;
   static constexpr size_t kSmem = 1024 + kScrOff + kEpiScratch;
-  static_assert(kABlock % 1024 == 0 && kRecMax % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
+  static_assert(kABlock % 1024 == 0 && kRecStride % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
   static_assert(kEpiScratch != 0 || 2 * (kMaxExperts + 1) * sizeof(int) >= 4 * 2048, "aliased scratch size");
   static_assert(kSmem <= 232448, "shared memory budget");
   static_assert(64 * kKps * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
@@ -131,10 +134,72 @@ __device__ __forceinline__ void dequant_block(const uint8_t* rec, int r, int has
   }
 }
 
-template <int NTOK>
+// ---- MXFP4 weights (e2m1 codes, E8M0 scale per 32 K)
+//
+// One 32-bit word of a chunk holds 4 pairs of codes (k even, k odd) with
+// their bits placed by the packer so that, after a rotation (pairs 0-2) or
+// two (pair 3), one mask leaves a bf16x2 word whose halves carry the sign at
+// bit 15, the code's two exponent bits at 8..7 and its mantissa bit at 6:
+// the bf16 value e2m1(c) * 2^-126 (the code 0.5 lands as the subnormal
+// 2^-127, which bf16 arithmetic keeps).
+__device__ __forceinline__ uint32_t rotr32(uint32_t x, int n) { return __funnelshift_r(x, x, n); }
+
+__device__ __forceinline__ void mx_pairs(uint32_t w, uint32_t* o) {
+  constexpr uint32_t kMask = 0x81C081C0u;
+  o[0] = w & kMask;
+  o[1] = rotr32(w, 4) & kMask;
+  o[2] = rotr32(w, 10) & kMask;
+  o[3] = (rotr32(w, 30) & 0x80C080C0u) | (rotr32(w, 6) & 0x01000100u);
+}
+
+// One 32-K chunk of row r -> 16 bf16x2 words w = e2m1(c) * 2^(e - 127),
+// exact (scale bytes <= 252).  ONE_MUL: the scale is below 2^1, so a single
+// multiply by bf16 2^(e - 1) suffices; otherwise the codes are first brought
+// to their e2m1 values (times 2^126, exact) and then scaled by 2^(e - 127)
+// (2^-127 is the bf16 subnormal 0x0040).
+template <bool ONE_MUL>
+__device__ __forceinline__ void mx_dequant_chunk(const uint4& raw, uint32_t e, uint32_t* out) {
+  const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+  const uint32_t sbits = ONE_MUL ? (e + 126u) << 7 : (e ? e << 7 : 0x40u);
+  const uint32_t s2 = sbits | (sbits << 16);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t o[4];
+    mx_pairs(wv[w], o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      out[w * 4 + j] = ONE_MUL ? bf16x2_mul(o[j], s2) : bf16x2_mul(bf16x2_mul(o[j], 0x7E807E80u), s2);
+  }
+}
+
+template <bool ONE_MUL>
+__device__ __forceinline__ void mx_dequant_chunks(const uint4* raw, uint32_t e4, uint32_t taddr) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t w[16];
+    mx_dequant_chunk<ONE_MUL>(raw[c], (e4 >> (8 * c)) & 0xFFu, w);
+    tmem_st_x16(taddr + c * 16, w);
+  }
+}
+
+// A whole 128-K MXFP4 record for weight row r into TMEM (as dequant_block).
+// The single-multiply path runs when every scale byte of the warp's 32 rows
+// is below 128 (a warp-uniform choice; both paths give the same bits).
+__device__ __forceinline__ void mx_dequant_block(const uint8_t* rec, int r, uint32_t taddr) {
+  uint4 raw[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+  const uint32_t e4 = *reinterpret_cast<const uint32_t*>(rec + kW4RecCodes + 4 * r);
+  if (__all_sync(0xffffffffu, (e4 & 0x80808080u) == 0u))
+    mx_dequant_chunks<true>(raw, e4, taddr);
+  else
+    mx_dequant_chunks<false>(raw, e4, taddr);
+}
+
+template <int NTOK, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
-  using C = Cfg<NTOK>;
+  using C = Cfg<NTOK, MX>;
   constexpr int SS = C::kSmemStages;
   constexpr int TS = C::kTmemStages;
   constexpr int ACC = C::kAccBufs;
@@ -366,8 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t tbase = tmem_base + lane_addr + a_col(t);
         tc_fence_after();
-        for (int rr = 0; rr < nrec; ++rr)
-          dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
+        for (int rr = 0; rr < nrec; ++rr) {
+          if constexpr (MX)
+            mx_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, tbase + rr * 64);
+          else
+            dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -414,10 +483,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
-template <int NTOK>
+template <int NTOK, bool MX = false>
 hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_kernel<NTOK>;
-  const size_t smem = Cfg<NTOK>::kSmem;
+  auto kern = w4a16_kernel<NTOK, MX>;
+  const size_t smem = Cfg<NTOK, MX>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -545,8 +614,9 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.c = static_cast<__nv_bfloat16*>(c);
   p.expert_offsets = expert_offsets;
   p.err = static_cast<uint32_t*>(ws);
+  const bool mx = d.fmt == HQ_FMT_MXFP4_A16;
   p.has_zero = d.has_zero_point ? 1 : 0;
-  p.rec_bytes = w4_record_bytes(p.has_zero);
+  p.rec_bytes = mx ? kMxA16RecBytes : w4_record_bytes(p.has_zero);
   p.n_tiles = (d.n + kTileN - 1) / kTileN;
   p.k_blocks = d.k / kBlockK;
   p.expert_bytes = (uint64_t)p.n_tiles * p.k_blocks * p.rec_bytes;
@@ -587,8 +657,19 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   // the library's choice for 64-token tiles, where it measured faster
   // (dense M=64: 26.3 vs 28.4 us at K=7168, N=18432; grouped 64-token tiles
   // up to 13 % faster); the bf16-rescaled kernel everywhere else.
-  const bool exact = cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
+  // (MXFP4 weights: always the rescaled kernel, one scale per 32 K.)
+  const bool exact = !mx && cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
   if (exact) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
+  if (mx) {
+    switch (cfg.ntok) {
+      case 16: return launch_t<16, true>(map, p, cfg.grid, stream);
+      case 32: return launch_t<32, true>(map, p, cfg.grid, stream);
+      case 64: return launch_t<64, true>(map, p, cfg.grid, stream);
+      case 128: return launch_t<128, true>(map, p, cfg.grid, stream);
+      case 256: return launch_t<256, true>(map, p, cfg.grid, stream);
+      default: return HQ_ERR_UNSUPPORTED;
+    }
+  }
   switch (cfg.ntok) {
     case 16: return launch_t<16>(map, p, cfg.grid, stream);
     case 32: return launch_t<32>(map, p, cfg.grid, stream);

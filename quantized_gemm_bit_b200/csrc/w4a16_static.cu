@@ -1,4 +1,5 @@
-// Dense W4A16 GEMM entry point that allocates nothing.
+// Dense W4A16 GEMM entry point that allocates nothing (INT4 or MXFP4_A16
+// weights, as hq_gemm_w4a16).
 //
 // Some callers cannot allocate device memory at the point where they run a
 // layer: an inference engine that plans every buffer up front and then
@@ -63,23 +64,15 @@ extern "C" hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* pa
                                           int32_t m, void* c_dev, const hq_tuning* t, hq_stream_t stream) {
   if (!d) return HQ_ERR_INVALID_ARG;
   if (d->layout_version != HQ_LAYOUT_VERSION) return HQ_ERR_LAYOUT_VERSION;
-  if (d->fmt != HQ_FMT_INT4 || d->num_experts != 1 || d->group_size != 128 || d->n < 1 || d->k < 1 ||
-      d->k % 128 != 0 || (d->has_zero_point != 0 && d->has_zero_point != 1))
-    return HQ_ERR_INVALID_ARG;
   if (m < 0) return HQ_ERR_INVALID_ARG;
+  hq_status st = check_w4_call(d, t, false);
+  if (st != HQ_OK) return st;
   if (m == 0) return HQ_OK;
   if (!packed_w_dev || !a_dev || !c_dev) return HQ_ERR_INVALID_ARG;
   auto aligned16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!aligned16(packed_w_dev) || !aligned16(a_dev) || !aligned16(c_dev)) return HQ_ERR_ALIGNMENT;
-  if (t) {
-    if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
-      return HQ_ERR_UNSUPPORTED;
-    if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
-        (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
-      return HQ_ERR_UNSUPPORTED;
-  }
   DeviceInfo dev{};
-  hq_status st = device_info(&dev);
+  st = device_info(&dev);
   if (st != HQ_OK) return st;
   W4Config cfg = w4_plan(dev, *d, m, false, t);
   // a whole-tile plan with a stream-K tail falls back to whole tiles when

@@ -34,6 +34,7 @@ HQ_ERR_NO_DEVICE = 9
 HQ_FMT_INT4 = 1
 HQ_FMT_MXFP4 = 2
 HQ_FMT_NVFP4 = 3
+HQ_FMT_MXFP4_A16 = 4
 
 # Every symbol include/hq.h declares.
 EXPORTS = (

@@ -41,6 +41,10 @@ def test_desc_validation():
                        ((hq.HQ_FMT_INT4, 0, 1024, 128, 0, 1), hq.HQ_ERR_INVALID_ARG),
                        ((hq.HQ_FMT_MXFP4, 128, 128, 32, 1, 1), hq.HQ_ERR_UNSUPPORTED),
                        ((hq.HQ_FMT_NVFP4, 128, 128, 16, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_MXFP4_A16, 128, 128, 16, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_MXFP4_A16, 128, 96, 32, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_MXFP4_A16, 128, 128, 32, 1, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_MXFP4_A16, 128, 128, 32, 0, 1025), hq.HQ_ERR_UNSUPPORTED),
                        ((7, 128, 128, 16, 0, 1), hq.HQ_ERR_INVALID_ARG)]:
         with pytest.raises(hq.HQError) as e:
             hq.hq_quant_desc_init(*args)
@@ -77,6 +81,37 @@ def test_fp4_pack_matches_oracle_layout(fmt, block, n):
     blob = hq.hq_pack_weights(d, codes, scales, None, g)
     ref = L.fp4_pack(codes, scales, block, g if fmt == hq.HQ_FMT_NVFP4 else None)
     assert np.array_equal(blob, ref)
+
+
+@pytest.mark.parametrize("n,k,experts", [(128, 128, 1), (300, 384, 1), (136, 256, 3)])
+def test_mxfp4_a16_pack_matches_oracle_layout(n, k, experts):
+    codes, e8 = synth.mxfp4_weights(n, k, seed=n + k, experts=experts if experts > 1 else None)
+    if experts == 1:
+        # the whole scale range the packer accepts
+        e8 = torch.from_numpy(np.random.default_rng(n).integers(0, 253, size=(n, k // 32), dtype=np.uint8))
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, n, k, 32, 0, experts)
+    blob = hq.hq_pack_weights(d, codes, e8)
+    assert blob.size == L.mxa16_packed_bytes(n, k, experts)
+    cn, en = codes.numpy(), e8.numpy()
+    if experts == 1:
+        ref = L.mxa16_pack(cn, en)
+    else:
+        ref = np.concatenate([L.mxa16_pack(cn[e], en[e]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+def test_mxfp4_a16_pack_rejects_scales_that_overflow_bf16():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 128, 128, 32, 0, 1)
+    codes, e8 = synth.mxfp4_weights(128, 128, seed=5)
+    for bad in (253, 255):
+        eb = e8.clone()
+        eb[3, 1] = bad
+        with pytest.raises(hq.HQError) as e:
+            hq.hq_pack_weights(d, codes, eb)
+        assert e.value.status == hq.HQ_ERR_INVALID_ARG
+    with pytest.raises(hq.HQError) as e:                 # no zero points for this format
+        hq.hq_pack_weights(d, codes, e8, torch.zeros(128, 4, dtype=torch.uint8))
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
 
 
 def test_fp4_scale_layout_is_a_bijection():
@@ -132,6 +167,19 @@ def test_gemm_argument_errors_need_no_gpu():
     for bad in (hq.Tuning(tile_m=512), hq.Tuning(split_k=2)):
         assert L_.hq_grouped_gemm_moe(ctypes.byref(dg), 16, 16, 16, 40, 32, ctypes.byref(bad), 256, 1 << 20,
                                       None) == hq.HQ_ERR_UNSUPPORTED
+    # MXFP4 weights with bf16 activations: no exact-integer variant; the
+    # block-scaled entry points do not take them
+    dx = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 1)
+    t = hq.Tuning(variant=2)
+    assert L_.hq_gemm_w4a16(ctypes.byref(dx), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
+                            None) == hq.HQ_ERR_UNSUPPORTED
+    assert L_.hq_gemm_w4a16_static(ctypes.byref(dx), 16, 16, 4, 32, ctypes.byref(t), None) == hq.HQ_ERR_UNSUPPORTED
+    assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dx), 4096, 16, 16, 4, 32, None, 256, 1 << 20,
+                               None) == hq.HQ_ERR_INVALID_ARG
+    dxg = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 8)
+    assert L_.hq_grouped_gemm_moe(ctypes.byref(dxg), 16, 16, 16, 40, 32, ctypes.byref(t), 256, 1 << 20,
+                                  None) == hq.HQ_ERR_UNSUPPORTED
+    assert L_.hq_gemm_w4a16(ctypes.byref(dxg), 16, 16, 4, 32, None, 256, 1 << 20, None) == hq.HQ_ERR_INVALID_ARG
     dm = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 256, 256, 32, 0, 1)
     t = hq.Tuning(variant=1)
     assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dm), 4096, 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
@@ -182,4 +230,5 @@ def test_autotune_candidates_need_no_gpu():
     assert c[0] is None and all(t.tile_m in (16, 32) for t in c[1:])
     assert not any(t.variant == 2 and t.tile_m > 64 for t in autotune.candidates("w4a16", 4096)[1:])
     assert all(t.variant == 0 for t in autotune.candidates("nvfp4", 256)[1:])
+    assert all(t.variant == 1 for t in autotune.candidates("mxfp4_a16", 16)[1:])
     assert all(t.split_k == 0 for t in autotune.candidates("moe", 64)[1:])
