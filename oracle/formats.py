@@ -5,6 +5,9 @@ Formats (the pages only name them; meanings from the public standards):
   * INT4 (unsigned code 0..15) with group scale / zero point:
     "Humming: open-source kernel library for quantized inference", summary,
     second paragraph (weight, scale and zero point described separately).
+  * INT3 (unsigned code 0..7, GPTQ INT3 weights: the Vietnamese edition
+    of the Humming news, section "meaning for domestic deployers"), with
+    the same group scale / zero point.
   * e2m1 (FP4): OCP MX v1.0, section 5.3.3 "FP4 (E2M1)": 1 sign bit,
     2 exponent bits with bias 1, 1 mantissa bit, no inf/NaN, max 6.0.
   * E8M0 scale: OCP MX v1.0, section 5.4 "E8M0": value 2**(e-127), 0xFF NaN.
@@ -259,3 +262,30 @@ def fp4_pack_bytes(codes):
     """codes [R, K] -> uint8 [R, K/2]; even k in the low nibble."""
     c = np.asarray(codes, dtype=np.uint8)
     return ((c[:, 0::2] & 0xF) | ((c[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+
+
+def int3_unpack_stream(qweight):
+    """int32 [N, 3K/32] -> uint8 codes [N, K] (0..7).
+
+    Canonical INT3 container (the pages name GPTQ INT3 weights and give no
+    packing; the plainest reading): each row's K codes form one little-endian
+    bit stream, code k in stream bits [3k, 3k+3), stream bit b being bit
+    b % 32 of word b // 32 (so 32 codes fill 3 words and some codes straddle
+    two words)."""
+    w = np.asarray(qweight).astype(np.int64) & 0xFFFFFFFF
+    n, nw = w.shape
+    k = nw * 32 // 3
+    bits = ((w[:, :, None] >> np.arange(32, dtype=np.int64)[None, None, :]) & 1).reshape(n, nw * 32)
+    b3 = bits[:, : 3 * k].reshape(n, k, 3)
+    return (b3[:, :, 0] | (b3[:, :, 1] << 1) | (b3[:, :, 2] << 2)).astype(np.uint8)
+
+
+def int3_pack_stream(codes):
+    """uint8 codes [N, K] (0..7), K % 32 == 0 -> int32 [N, 3K/32] (inverse
+    of int3_unpack_stream)."""
+    c = np.asarray(codes).astype(np.int64)
+    n, k = c.shape
+    assert k % 32 == 0
+    bits = np.stack([(c >> i) & 1 for i in range(3)], axis=2).reshape(n, 3 * k)
+    words = (bits.reshape(n, 3 * k // 32, 32) << np.arange(32, dtype=np.int64)).sum(axis=2)
+    return words.astype(np.uint32).view(np.int32)

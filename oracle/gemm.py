@@ -56,6 +56,35 @@ def w4a16_ref(a_bf16, qweight, scales, zeros, group, rows=None, cols=None):
     return a @ w.T
 
 
+def w3a16_dequant(qweight, scales, zeros, group, rows=None):
+    """INT3 weights: W_hat[n, k] = (q[n, k] - z[n, k // G]) * s[n, k // G]
+    (fp64), the same definition as INT4 with 3-bit codes.
+
+    qweight: int32 [N, 3K/32] (each row one little-endian bit stream of
+             3-bit codes, see formats.int3_unpack_stream)
+    scales : float16 [N, K/G]
+    zeros  : uint8 [N, K/G] holding 0..7, or None for the symmetric form
+             (zero point 4, the middle of the code range as 8 is for INT4)
+    """
+    if rows is not None:
+        qweight = np.asarray(qweight)[rows]
+        scales = np.asarray(scales)[rows]
+        zeros = None if zeros is None else np.asarray(zeros)[rows]
+    q = F.int3_unpack_stream(qweight).astype(np.float64)
+    n, k = q.shape
+    g = np.arange(k) // group
+    s = np.asarray(scales, dtype=np.float16).astype(np.float64)[:, g]
+    z = 4.0 if zeros is None else np.asarray(zeros).astype(np.float64)[:, g]
+    return (q - z) * s
+
+
+def w3a16_ref(a_bf16, qweight, scales, zeros, group, rows=None, cols=None):
+    """C = A_hat @ W_hat.T in fp64 for INT3 weights (bf16 bit patterns in)."""
+    a = F.bf16_bits_to_f64(a_bf16 if rows is None else np.asarray(a_bf16)[rows])
+    w = w3a16_dequant(qweight, scales, zeros, group, rows=cols)
+    return a @ w.T
+
+
 def w4a16_ref_integer_domain(a_bf16, qweight, scales, zeros, group):
     """The same product evaluated as sum_g s_g * sum_{k in g} a_k (q_k - z_g):
     the group sums use integer weights (q - z), the scale enters once per
@@ -237,4 +266,14 @@ def grouped_mxfp4_a16_ref(a_sorted_bf16, expert_offsets, w_packed, w_e8m0, row_s
     def dequant(e):
         return mxfp4_dequant(w_packed[e], w_e8m0[e], rows=cols)
     ncols = np.asarray(w_packed).shape[1] if cols is None else len(cols)
+    return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)
+
+
+def grouped_w3a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, group, row_subset=None, cols=None):
+    """Grouped form of w3a16_ref: qweights int32 [E, N, 3K/32], scales
+    float16 [E, N, K/G], zeros uint8 [E, N, K/G] or None.  Returns (rows, C)."""
+    def dequant(e):
+        z = None if zeros is None else zeros[e]
+        return w3a16_dequant(qweights[e], scales[e], z, group, rows=cols)
+    ncols = np.asarray(qweights).shape[1] if cols is None else len(cols)
     return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)

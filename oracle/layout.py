@@ -235,3 +235,102 @@ def mxa16_unpack(blob, n, k):
     ns, bs = np.meshgrid(np.arange(n), np.arange(k // 32), indexing="ij")
     scales = np.asarray(blob, dtype=np.uint8)[mxa16_scale_byte(ns.ravel(), bs.ravel(), k)]
     return codes.reshape(n, k).astype(np.uint8), scales.reshape(n, k // 32)
+
+
+# ---------------------------------------------------------------------------
+# INT3 W3A16 (group 128), layout version 1
+#   Records as for INT4: one per (tile nt of 128 rows, block kb of 128 K), in
+#   (nt, kb) order, experts one after another; record size
+#   6144 + 256 (+ 128 with zero points) bytes.
+#   codes : row r's 12 code words; word q (q = 3c + p: 32-K chunk c, part
+#           p < 3) is the 32-bit little-endian word at byte
+#           (q // 4 * 128 + r) * 16 + 4 * (q % 4).  Code kk = k - 128*kb of
+#           chunk c = kk // 32, pair i = (kk % 32) // 2, half h = kk % 2:
+#             i < 15: word 3c + i // 5, code bit b at bit 3*(i % 5) + b + 16*h;
+#             i = 15: code bit b in word 3c + b, at bit 15 + 16*h.
+#   scale : fp16 bits at byte 6144 + 2*r;  zero: uint8 at 6144 + 256 + r.
+#   Rows n >= N (tile padding) hold code 0, scale 0 and zero 0.
+# ---------------------------------------------------------------------------
+
+
+def w3a16_record_bytes(has_zero):
+    return 6144 + 256 + (128 if has_zero else 0)
+
+
+def w3a16_packed_bytes(n, k, has_zero, num_experts=1):
+    return num_experts * (-(-n // 128)) * (k // 128) * w3a16_record_bytes(has_zero)
+
+
+def w3a16_code_bits(n, k, kdim, has_zero):
+    """Elementwise formula: ([.., 3] byte offsets of the words holding code
+    bits 0..2 of code (n, k) in the expert blob, [.., 3] bit positions)."""
+    n = np.asarray(n, dtype=np.int64)
+    k = np.asarray(k, dtype=np.int64)
+    rec = w3a16_record_bytes(has_zero)
+    nt, r = n // 128, n % 128
+    kb, kk = k // 128, k % 128
+    c, i, h = kk // 32, (kk % 32) // 2, kk % 2
+    b = np.arange(3, dtype=np.int64)
+    last = (i == 15)[..., None]
+    q = np.where(last, 3 * c[..., None] + b, (3 * c + np.minimum(i, 14) // 5)[..., None] + 0 * b)
+    bit = np.where(last, 15 + 16 * h[..., None] + 0 * b, (3 * (np.minimum(i, 14) % 5) + 16 * h)[..., None] + b)
+    base = ((nt * (kdim // 128) + kb) * rec)[..., None]
+    word = base + (q // 4 * 128 + r[..., None]) * 16 + 4 * (q % 4)
+    return word, bit
+
+
+def w3a16_scale_byte(n, kb, kdim, has_zero):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    return (nt * (kdim // 128) + kb) * w3a16_record_bytes(has_zero) + 6144 + 2 * r
+
+
+def w3a16_zero_byte(n, kb, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    return (nt * (kdim // 128) + kb) * w3a16_record_bytes(True) + 6144 + 256 + r
+
+
+def w3a16_pack(qweight, scales, zeros, group=128):
+    """Canonical (int32 [N, 3K/32] bit streams, fp16 [N, K/128], uint8
+    [N, K/128] | None) -> packed blob of one expert, every code bit, scale
+    and zero point placed where the formulas above say."""
+    assert group == 128
+    codes = F.int3_unpack_stream(qweight).astype(np.uint32)
+    n, k = codes.shape
+    has_zero = zeros is not None
+    out = np.zeros(w3a16_packed_bytes(n, k, has_zero), dtype=np.uint8)
+    words = np.zeros(out.size // 4, dtype=np.uint32)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    word, bit = w3a16_code_bits(nn.ravel(), kk.ravel(), k, has_zero)
+    c = codes.ravel()
+    for b in range(3):
+        np.bitwise_or.at(words, word[:, b] // 4, ((c >> b) & 1) << bit[:, b].astype(np.uint32))
+    out[:] = words.view(np.uint8)
+    sb = np.asarray(scales, dtype=np.float16).view(np.uint16)
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    off = w3a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    out[off] = (sb.ravel() & 0xFF).astype(np.uint8)
+    out[off + 1] = (sb.ravel() >> 8).astype(np.uint8)
+    if has_zero:
+        out[w3a16_zero_byte(ng.ravel(), gg.ravel(), k)] = np.asarray(zeros, dtype=np.uint8).ravel()
+    return out
+
+
+def w3a16_unpack(blob, n, k, has_zero):
+    """Inverse of w3a16_pack: blob -> (codes uint8 [N, K], scales fp16
+    [N, K/128], zeros uint8 [N, K/128] | None)."""
+    blob = np.asarray(blob, dtype=np.uint8)
+    words = blob.view(np.uint32)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    word, bit = w3a16_code_bits(nn.ravel(), kk.ravel(), k, has_zero)
+    codes = np.zeros(n * k, dtype=np.uint32)
+    for b in range(3):
+        codes |= ((words[word[:, b] // 4] >> bit[:, b].astype(np.uint32)) & 1) << b
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    off = w3a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    sbits = blob[off].astype(np.uint16) | (blob[off + 1].astype(np.uint16) << 8)
+    zeros = blob[w3a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // 128) if has_zero else None
+    return codes.reshape(n, k).astype(np.uint8), sbits.reshape(n, k // 128).view(np.float16), zeros

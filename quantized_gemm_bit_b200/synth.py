@@ -12,6 +12,9 @@ Recipes (one per workload; seed = workload index * 1000 + shape index):
     0.002 + 0.01*|N(0,1)| per (row, group of 128 along K); zero points
     uniform in [0, 15] (asymmetric) or none (symmetric, zero point 8);
     activations bf16 N(0,1).
+  * W3A16 (INT3): as W4A16 with 3 K/32 int32 words per row (every bit
+    uniform = uniform 3-bit codes in a little-endian bit stream) and zero
+    points uniform in [0, 7] (symmetric: zero point 4).
   * W4A8-MXFP4 (and MXFP4 weights with bf16 activations): FP4 codes
     uniform over the 16 codes, two per byte (even k low nibble); one E8M0
     scale per 32 K with exponent uniform in [-8, -2];
@@ -50,6 +53,22 @@ def w4a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
     zeros = None
     if asym:
         zeros = torch.randint(0, 16, lead + (n, k // group), generator=g, dtype=torch.uint8)
+    return qweight, scales, zeros
+
+
+def w3a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
+    """Canonical INT3 weights: qweight int32 [.., N, 3K/32] with every bit
+    uniform (= uniform 3-bit codes in each row's little-endian bit stream),
+    fp16 scales as for W4A16, zero points uniform in [0, 7] (asymmetric) or
+    none (symmetric, zero point 4)."""
+    assert k % group == 0 and k % 32 == 0
+    g = _gen(seed)
+    lead = () if experts is None else (experts,)
+    qweight = torch.randint(-(2 ** 31), 2 ** 31, lead + (n, 3 * k // 32), generator=g, dtype=torch.int32)
+    scales = (0.002 + 0.01 * torch.randn(lead + (n, k // group), generator=g).abs()).to(torch.float16)
+    zeros = None
+    if asym:
+        zeros = torch.randint(0, 8, lead + (n, k // group), generator=g, dtype=torch.uint8)
     return qweight, scales, zeros
 
 
