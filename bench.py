@@ -465,14 +465,25 @@ def run_mxfp4(args, rank, world, peaks):
             "detail": out}
 
 
-def run_mxfp4_a16(args, rank, world, peaks):
-    """MXFP4 weights x bf16 activations on the W4A16 kernels: M in
-    {16, 64, 256, 4096}, K=7168, N=18432."""
+def _run_w16_format(args, world, peaks, fmt):
+    """Another weight format on the W4A16 kernels (bf16 activations):
+    M in {16, 64, 256, 4096}, K=7168, N=18432.  fmt "mxfp4_a16": e2m1 codes
+    with an E8M0 scale per 32 K; "w3a16": INT3 codes with an fp16 scale per
+    128 K (symmetric)."""
     from quantized_gemm_bit_b200 import hq, synth
     k, n = 7168, 18432
-    codes, e8 = synth.mxfp4_weights(n, k, seed=6000)
-    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, n, k, 32, 0, 1)
-    blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).cuda()
+    if fmt == "mxfp4_a16":
+        codes, e8 = synth.mxfp4_weights(n, k, seed=6000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, n, k, 32, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).cuda()
+        wbytes = n * k // 2 + n * k // 32
+        name, dt = "MXFP4 weights x bf16 activations", "bf16 x e2m1 (fp32 accumulate)"
+    else:
+        q, sc, _ = synth.w3a16_weights(n, k, 128, False, seed=7000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, sc)).cuda()
+        wbytes = 3 * n * k // 8 + 2 * n * (k // GROUP)
+        name, dt = "INT3 weights (group 128) x bf16 activations", "bf16 x int3 (fp32 accumulate)"
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
     ms_list = (16, 64, 256, 4096)
@@ -492,14 +503,22 @@ def run_mxfp4_a16(args, rank, world, peaks):
     out = []
     for m, us in zip(ms_list, per):
         fl = 2.0 * m * n * k
-        by = n * k // 2 + n * k // 32 + 2 * m * k + 2 * m * n
+        by = wbytes + 2 * m * k + 2 * m * n
         out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1), gbs=round(by / us / 1e3, 1),
                         frac_hbm=round(by / us / 1e3 / peaks["hbm_gbs"], 3),
                         frac_bf16_peak=round(fl / us / 1e6 / peaks["bf16_tflops"], 3)))
     flops = sum(2.0 * m * n * k for m in ms_list)
-    return {"workload": "MXFP4 weights x bf16 activations (W4A16 kernels), M in {16,64,256,4096}, K=7168, N=18432",
+    return {"workload": f"{name} (W4A16 kernels), M in {{16,64,256,4096}}, K=7168, N=18432",
             "value": round(flops * args.steps * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(ms / args.steps, 4), "dtype": "bf16 x e2m1 (fp32 accumulate)", "detail": out}
+            "ms_per_step": round(ms / args.steps, 4), "dtype": dt, "detail": out}
+
+
+def run_mxfp4_a16(args, rank, world, peaks):
+    return _run_w16_format(args, world, peaks, "mxfp4_a16")
+
+
+def run_w3a16(args, rank, world, peaks):
+    return _run_w16_format(args, world, peaks, "w3a16")
 
 
 def run_nvfp4(args, rank, world, peaks):
@@ -690,7 +709,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "nvfp4", "moe"])
+    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "w3a16", "nvfp4", "moe"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -713,7 +732,8 @@ def main():
     if args.workload == "w4a16_sweep":
         line = run_w4a16_sweep(args, rank, world, peaks)
     else:
-        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "nvfp4": run_nvfp4, "moe": run_moe}[args.workload]
+        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "w3a16": run_w3a16, "nvfp4": run_nvfp4,
+              "moe": run_moe}[args.workload]
         line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "data": "synthetic (seeded)"}
         line.update(fn(args, rank, world, peaks))

@@ -20,6 +20,9 @@
  *           paragraph 5 (the "Grouped" MoE path).
  *   [P-pt]  "Ant Group e vLLM lancam a biblioteca open source Humming"
  *           (aube.news), quantization paragraph (dense and MoE layers).
+ *   [P-vi]  the Vietnamese edition of the same news (news.cocoloop.cn, vi),
+ *           section on what it means for domestic deployers (GPTQ INT3
+ *           weights served through the library).
  * Element formats follow the public standards the pages name: OCP MX v1.0
  * (e2m1, E8M0, 32-element blocks), OCP FP8 (E4M3), NVIDIA NVFP4 (e2m1 with
  * an E4M3 scale per 16 elements and an fp32 tensor scale).
@@ -82,8 +85,10 @@ typedef enum {
   HQ_FMT_INT4 = 1,  /* unsigned INT4 codes, fp16 scale + optional uint4 zero point per group of 128 K */
   HQ_FMT_MXFP4 = 2, /* e2m1 codes, E8M0 scale per 32 K                                             */
   HQ_FMT_NVFP4 = 3, /* e2m1 codes, E4M3 scale per 16 K, fp32 tensor scale                          */
-  HQ_FMT_MXFP4_A16 = 4 /* e2m1 codes, E8M0 scale per 32 K, for bf16 activations: the W4A16 entry
-                          points dequantize it in registers like INT4                               */
+  HQ_FMT_MXFP4_A16 = 4, /* e2m1 codes, E8M0 scale per 32 K, for bf16 activations: the W4A16 entry
+                           points dequantize it in registers like INT4                              */
+  HQ_FMT_INT3 = 5       /* unsigned INT3 codes, fp16 scale + optional uint3 zero point per group of
+                           128 K, for bf16 activations (the W4A16 entry points)                     */
 } hq_format;
 
 /* Quantization description ([P-fa2] paragraph 2) plus the Layer Config
@@ -93,8 +98,8 @@ typedef struct {
   int32_t fmt;            /* hq_format                                                 */
   int32_t n;              /* output features (weight rows), per expert                 */
   int32_t k;              /* input features (reduction length)                         */
-  int32_t group_size;     /* INT4: 128; MXFP4, MXFP4_A16: 32; NVFP4: 16                */
-  int32_t has_zero_point; /* INT4: 1 = uint4 zero point per group, 0 = symmetric (8)   */
+  int32_t group_size;     /* INT4, INT3: 128; MXFP4, MXFP4_A16: 32; NVFP4: 16          */
+  int32_t has_zero_point; /* INT4 / INT3: 1 = zero point per group, 0 = symmetric (8 / 4) */
   int32_t num_experts;    /* 1 = dense layer; >1 = MoE weights stored expert after expert */
 } hq_quant_desc;
 
@@ -133,7 +138,8 @@ const char* hq_status_string(hq_status s);
  *   MXFP4: k % 128 == 0, group_size == 32, has_zero_point == 0
  *   NVFP4: k % 256 == 0, group_size == 16, has_zero_point == 0
  *   MXFP4_A16: k % 128 == 0, group_size == 32, has_zero_point == 0
- *   num_experts 1..1024 for INT4 and MXFP4_A16 (MoE), 1 otherwise. */
+ *   INT3 : k % 128 == 0, group_size == 128
+ *   num_experts 1..1024 for INT4, INT3 and MXFP4_A16 (MoE), 1 otherwise. */
 hq_status hq_quant_desc_init(hq_quant_desc* d, int32_t fmt, int32_t n, int32_t k, int32_t group_size,
                              int32_t has_zero_point, int32_t num_experts);
 
@@ -151,6 +157,11 @@ size_t hq_packed_size(const hq_quant_desc* d);
  *          scales_host = uint8 E8M0 [N][K/32]
  *   NVFP4: codes_host  = uint8 [N][K/2]; scales_host = uint8 E4M3 [N][K/16];
  *          global_scale = the fp32 tensor scale of the weights.
+ *   INT3 : codes_host  = int32 [E][N][3K/32]: each row's codes as one
+ *          little-endian bit stream, code k in stream bits 3k..3k+2 (stream
+ *          bit b = bit b%32 of word b/32), the container of GPTQ INT3
+ *          scales_host = fp16 bits [E][N][K/128]
+ *          zeros_host  = uint8 [E][N][K/128] (0..7), NULL when symmetric
  *   MXFP4_A16: codes_host = uint8 [E][N][K/2] (even k in the low nibble),
  *          scales_host = uint8 E8M0 [E][N][K/32], every byte <= 252 (a
  *          larger scale would overflow bf16 weights, 255 is NaN).
@@ -162,14 +173,18 @@ size_t hq_packed_size(const hq_quant_desc* d);
 hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
                           const void* zeros_host, float global_scale, void* out_host, size_t out_bytes);
 
-/* Workspace bytes that hq_gemm_w4a16 (fmt INT4 or MXFP4_A16, num_experts 1),
+/* Workspace bytes that hq_gemm_w4a16 (fmt INT4, INT3 or MXFP4_A16, num_experts 1),
  * hq_gemm_mxfp4_a8, hq_gemm_nvfp4 or hq_grouped_gemm_moe need for M rows
  * (total sorted rows for MoE) and the given tuning (NULL = heuristic). */
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
 
 /* Dense W4A16 GEMM ([P-fa] table row "W4A16 dense"): C = A * W_hat^T with
  * W_hat[n,k] = (q[n,k] - z[n,k/128]) * s[n,k/128] dequantized in-kernel.
- *   d            : INT4 or MXFP4_A16 descriptor with num_experts == 1.
+ *   d            : INT4, INT3 or MXFP4_A16 descriptor, num_experts == 1.
+ *                  INT3 (GPTQ INT3 weights, [P-vi] "meaning for domestic
+ *                  deployers"): W_hat = (q - z) * s with 3-bit codes and
+ *                  the symmetric zero point 4, computed as for INT4 (tuning
+ *                  variant 1 for every tile; variant 2 is refused).
  *                  MXFP4_A16 (MXFP4 weights with bf16 activations; [P-fa2]
  *                  paragraph 2 lists MXFP4 weights and bf16 activations):
  *                  W_hat[n,k] = e2m1(c[n,k]) * 2^(e[n,k/32] - 127), each
@@ -258,8 +273,8 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
  * "MoE W4A16"): for every expert e, rows [off[e], off[e+1]) of A_sorted
  * times W_hat_e^T.  The tile scheduler reads expert_offsets on the device
  * (no host synchronization).
- *   d              : INT4 or MXFP4_A16 descriptor, num_experts = e
- *                    (per-expert n, k); MXFP4_A16 weights as for
+ *   d              : INT4, INT3 or MXFP4_A16 descriptor, num_experts = e
+ *                    (per-expert n, k); INT3 and MXFP4_A16 weights as for
  *                    hq_gemm_w4a16
  *   packed_w_dev   : blob of all experts from hq_pack_weights
  *   a_sorted_dev   : bf16 [total_rows][k]

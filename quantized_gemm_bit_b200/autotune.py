@@ -9,6 +9,7 @@ for one shape on the GPU at hand:
     python -m quantized_gemm_bit_b200.autotune --kind w4a16 --m 16 --k 7168 --n 18432
     python -m quantized_gemm_bit_b200.autotune --kind mxfp4 --m 256 --k 7168 --n 7168
     python -m quantized_gemm_bit_b200.autotune --kind mxfp4_a16 --m 16 --k 7168 --n 18432
+    python -m quantized_gemm_bit_b200.autotune --kind w3a16 --m 16 --k 7168 --n 18432
     python -m quantized_gemm_bit_b200.autotune --kind moe --m 1024 --k 7168 --n 4096
 
 Every candidate `hq_tuning` (and the library's own choice, `None`) runs as a
@@ -32,11 +33,11 @@ TILES = (16, 32, 64, 128, 256)
 def candidates(kind, m):
     """Tunings worth trying at m rows: token tiles up to twice the rows
     (at least 16), K splits 0 (the library's choice) to 3, and for the
-    W4A16 kernels with INT4 weights both weight variants (MXFP4 weights
-    have only the rescaled one)."""
+    W4A16 kernels with INT4 weights both weight variants (MXFP4 and INT3
+    weights have only the rescaled one)."""
     cap = max(16, 2 * m)
     tiles = [t for t in TILES if t <= cap] or [16]
-    variants = (1, 2) if kind in ("w4a16", "moe") else (1,) if kind == "mxfp4_a16" else (0,)
+    variants = (1, 2) if kind in ("w4a16", "moe") else (1,) if kind in ("mxfp4_a16", "w3a16") else (0,)
     splits = (0,) if kind == "moe" else (0, 1, 2, 3)
     out = [None]
     for t in tiles:
@@ -92,6 +93,15 @@ def _setup(kind, m, n, k, experts, topk, dev):
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, 1)
         blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev))
         a = synth.bf16_normal(m, k, seed=1001).to(dev)
+        rows = m
+
+        def call(t, i, c, ws):
+            hq.hq_gemm_w4a16(d, blobs[i], a, m, c, ws, t)
+    elif kind == "w3a16":
+        q, s, _ = synth.w3a16_weights(n, k, 128, False, seed=7000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
+        blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev))
+        a = synth.bf16_normal(m, k, seed=7001).to(dev)
         rows = m
 
         def call(t, i, c, ws):
@@ -178,7 +188,7 @@ def autotune(kind, m, n, k, experts=256, topk=8, tunings=None, dev="cuda"):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "mxfp4_a16", "mxfp4", "nvfp4", "moe"])
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "mxfp4_a16", "mxfp4", "nvfp4", "moe"])
     ap.add_argument("--m", type=int, default=16, help="rows (tokens for --kind moe)")
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)

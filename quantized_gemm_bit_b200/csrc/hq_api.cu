@@ -76,13 +76,20 @@ hq_status check_desc(const hq_quant_desc* d) {
       if (d->group_size != 32 || d->k % 128 != 0 || d->has_zero_point || d->num_experts > 1024)
         return HQ_ERR_UNSUPPORTED;
       return HQ_OK;
+    case HQ_FMT_INT3:
+      if (d->group_size != 128 || d->k % 128 != 0) return HQ_ERR_UNSUPPORTED;
+      if (d->has_zero_point != 0 && d->has_zero_point != 1) return HQ_ERR_INVALID_ARG;
+      if (d->num_experts > 1024) return HQ_ERR_UNSUPPORTED;
+      return HQ_OK;
     default:
       return HQ_ERR_INVALID_ARG;
   }
 }
 
 // Formats the W4A16 kernels read (dequantized in registers, bf16 MMA).
-bool w4_format(const hq_quant_desc* d) { return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_MXFP4_A16; }
+bool w4_format(const hq_quant_desc* d) {
+  return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_MXFP4_A16;
+}
 
 // Tuning checks shared by the W4A16 entry points (dense: split_k free;
 // grouped: at most one CTA per tile).
@@ -94,8 +101,9 @@ hq_status check_w4_tuning(const hq_quant_desc* d, const hq_tuning* t, bool group
       (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
     return HQ_ERR_UNSUPPORTED;
   if (grouped && t->split_k > 1) return HQ_ERR_UNSUPPORTED;
-  // exact (q - z) weights need one scale per 128-K group
-  if (d->fmt == HQ_FMT_MXFP4_A16 && t->variant == 2) return HQ_ERR_UNSUPPORTED;
+  // the exact-weight kernel reads INT4 records only (and MXFP4's scale per
+  // 32 K leaves no 128-K group scale to factor out)
+  if (d->fmt != HQ_FMT_INT4 && t->variant == 2) return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
 
@@ -164,7 +172,7 @@ hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const 
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
   if (!codes_host || !scales_host || !out_host) return HQ_ERR_INVALID_ARG;
-  if (d->fmt == HQ_FMT_INT4) {
+  if (d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3) {
     if ((d->has_zero_point != 0) != (zeros_host != nullptr)) return HQ_ERR_INVALID_ARG;
   } else if (zeros_host) {
     return HQ_ERR_INVALID_ARG;

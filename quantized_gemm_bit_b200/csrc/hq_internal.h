@@ -23,6 +23,10 @@ inline int w4_record_bytes(bool has_zero) { return kW4RecCodes + 256 + (has_zero
 // MXFP4 weights for the W4A16 kernels: 8192 code bytes, then one E8M0 byte
 // per (row, 32-K block) of the record
 constexpr int kMxA16RecBytes = kW4RecCodes + 512;
+// INT3 weights: 6144 code bytes, then fp16 scales (256) and zero points
+// (128, with zero points) as in the INT4 record
+constexpr int kW3RecCodes = 6144;
+inline int w3_record_bytes(bool has_zero) { return kW3RecCodes + 256 + (has_zero ? 128 : 0); }
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 

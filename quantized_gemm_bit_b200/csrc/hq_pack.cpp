@@ -41,12 +41,26 @@
 //                  h < 2); bit b of a code (0 mantissa, 1-2 exponent, 3
 //                  sign) sits at word bit kMxBits[j][h][b].
 //   [8192, 8704)   E8M0 scale of row r, 32-K block c at 8192 + 4r + c.
+// (The INT3 layout follows below.)
 // The bit positions are chosen so that pair j's two codes land, after the
 // kernel rotates the word right by 0, 4 or 10 bits (j = 0, 1, 2) or merges
 // two rotations (j = 3), on the bits a bf16x2 word gives its sign (15), the
 // low two exponent bits (8..7) and the top mantissa bit (6): one mask per
 // pair then leaves two bf16 values e2m1 * 2^-126, and one multiply by a
 // power of two applies 2^126 times the block scale.
+//
+// INT3 (group 128).  Records as for INT4, 6144 + 256 (+128) bytes:
+//   [0, 6144)      codes: row r's 12 words; word q = 3c + p (32-K chunk c,
+//                  part p < 3) at byte (q/4*128 + r)*16 + 4*(q%4), so a
+//                  thread reads its row's record in three 16-byte loads.
+//                  Pair i < 15 of chunk c (codes 32c + 2i, 32c + 2i + 1)
+//                  sits in word 3c + i/5 at bits 3*(i%5) (even k) and
+//                  16 + 3*(i%5) (odd k); pair 15 keeps code bit p at bit 15
+//                  (even k) and bit 31 (odd k) of word 3c + p.  As for INT4,
+//                  one shift and one LOP3 with 0x00070007 / 0x43004300 give
+//                  the bf16 pair (128 + q, 128 + q').
+//   [6144, 6400)   fp16 scale of row r at 6144 + 2r
+//   [6400, 6528)   uint3 zero point of row r at 6400 + r (asymmetric only)
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -125,6 +139,62 @@ hq_status pack_int4(const hq_quant_desc& d, const int32_t* codes, const uint16_t
         const uint16_t s = scales[(e * n + row) * kg + kb];
         std::memcpy(r0 + kW4RecCodes + 2 * r, &s, 2);
         if (hz) r0[kW4RecCodes + 256 + r] = zeros[(e * n + row) * kg + kb];
+      }
+    }
+  });
+  return HQ_OK;
+}
+
+hq_status pack_int3(const hq_quant_desc& d, const int32_t* codes, const uint16_t* scales, const uint8_t* zeros,
+                    uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int nt_count = (n + kTileN - 1) / kTileN;
+  const int kb_count = k / kBlockK;
+  const bool hz = zeros != nullptr;
+  const size_t rec = (size_t)w3_record_bytes(hz);
+  const size_t expert_bytes = (size_t)nt_count * kb_count * rec;
+  const size_t kw = (size_t)k * 3 / 32;  // canonical words per row
+  const size_t kg = (size_t)k / 128;
+  if (hz) {
+    const size_t total = (size_t)d.num_experts * n * kg;
+    for (size_t i = 0; i < total; ++i)
+      if (zeros[i] > 7) return HQ_ERR_INVALID_ARG;
+  }
+  const size_t jobs = (size_t)d.num_experts * nt_count;
+  parallel_for(jobs, [&](size_t job) {
+    const size_t e = job / nt_count;
+    const int nt = (int)(job % nt_count);
+    uint8_t* ebase = out + e * expert_bytes;
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint8_t* r0 = ebase + ((size_t)nt * kb_count + kb) * rec;
+      std::memset(r0, 0, rec);
+      for (int r = 0; r < kTileN; ++r) {
+        const int row = nt * kTileN + r;
+        if (row >= n) break;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(codes + (e * n + row) * kw);
+        // code k of the row: stream bits 3k .. 3k+2
+        auto code = [&](int kk) {
+          uint32_t v = 0;
+          for (int b = 0; b < 3; ++b) {
+            const size_t bit = (size_t)3 * ((size_t)kb * 128 + kk) + b;
+            v |= ((src[bit / 32] >> (bit % 32)) & 1u) << b;
+          }
+          return v;
+        };
+        uint32_t words[12] = {};
+        for (int kk = 0; kk < 128; ++kk) {
+          const int c = kk / 32, i = (kk % 32) / 2, h = kk % 2;
+          const uint32_t v = code(kk);
+          if (i < 15) {
+            words[3 * c + i / 5] |= v << (3 * (i % 5) + 16 * h);
+          } else {
+            for (int b = 0; b < 3; ++b) words[3 * c + b] |= ((v >> b) & 1u) << (15 + 16 * h);
+          }
+        }
+        for (int q = 0; q < 12; ++q) std::memcpy(r0 + ((size_t)(q / 4) * 128 + r) * 16 + 4 * (q % 4), &words[q], 4);
+        const uint16_t s = scales[(e * n + row) * kg + kb];
+        std::memcpy(r0 + kW3RecCodes + 2 * r, &s, 2);
+        if (hz) r0[kW3RecCodes + 256 + r] = zeros[(e * n + row) * kg + kb];
       }
     }
   });
@@ -226,6 +296,8 @@ size_t packed_size_impl(const hq_quant_desc& d) {
       return nt * kTileN * (size_t)d.k / 2 + nt * (d.k / 64) * 512 + 16;
     case HQ_FMT_MXFP4_A16:
       return (size_t)d.num_experts * nt * (d.k / kBlockK) * kMxA16RecBytes;
+    case HQ_FMT_INT3:
+      return (size_t)d.num_experts * nt * (d.k / kBlockK) * w3_record_bytes(d.has_zero_point != 0);
     default:
       return 0;
   }
@@ -244,6 +316,9 @@ hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scale
     case HQ_FMT_MXFP4_A16:
       return pack_mx_a16(d, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales),
                          static_cast<uint8_t*>(out));
+    case HQ_FMT_INT3:
+      return pack_int3(d, static_cast<const int32_t*>(codes), static_cast<const uint16_t*>(scales),
+                       static_cast<const uint8_t*>(zeros), static_cast<uint8_t*>(out));
     default:
       return HQ_ERR_INVALID_ARG;
   }

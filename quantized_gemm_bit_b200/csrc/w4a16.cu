@@ -1,5 +1,6 @@
 // Dense and grouped (MoE) W4A16 GEMM for sm_100a with the INT4 dequantization
-// fused into the kernel.
+// fused into the kernel (also run with INT3 or MXFP4 weights: the same
+// kernel with another record decode).
 //
 // Method: the weights are stored as 4-bit codes with a per-group fp16 scale
 // and an optional uint4 zero point, described separately ("Humming:
@@ -44,16 +45,19 @@ namespace {
 
 constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 
-// MX: MXFP4 weight records (8704 bytes; the tighter barrier area keeps the
-// 256-token tile inside the shared-memory limit)
-template <int NTOK, bool MX = false>
+// Weight formats of the kernel: INT4 records, MXFP4 records (8704 bytes; a
+// tighter barrier area keeps the 256-token tile inside the shared-memory
+// limit) and INT3 records (at most 6528 bytes).
+constexpr int kFmtInt4 = 0, kFmtMx = 1, kFmtInt3 = 2;
+
+template <int NTOK, int FMT = kFmtInt4>
 struct Cfg {
   // records (128-K blocks) per pipeline stage: two for the small token tiles,
   // whose MMAs are cheap, so the per-stage waits and commits are amortized
   static constexpr int kKps = NTOK <= 64 ? 2 : 1;
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
-  static constexpr int kRecStride = MX ? kMxA16RecBytes : kRecMax;
+  static constexpr int kRecStride = FMT == kFmtMx ? kMxA16RecBytes : FMT == kFmtInt3 ? kW3RecCodes + 384 : kRecMax;
   static constexpr int kRecs = kKps * kRecStride;
   static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
   static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
@@ -72,7 +76,7 @@ struct Cfg {
   // it aliases the expert tables, so grouped 256-token tiles store their
   // outputs element by element instead
   static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
-  static constexpr int kBarBytes = MX ? 384 : 512;
+  static constexpr int kBarBytes = FMT == kFmtMx ? 384 : 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
   static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
   static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
@@ -196,10 +200,51 @@ __device__ __forceinline__ void mx_dequant_block(const uint8_t* rec, int r, uint
     mx_dequant_chunks<false>(raw, e4, taddr);
 }
 
-template <int NTOK, bool MX>
+// ---- INT3 weights (3-bit codes, fp16 scale and uint3 zero point per 128 K)
+__device__ __forceinline__ RowQ row_qparams3(const uint8_t* rec, int r, int has_zero) {
+  const __half sc = reinterpret_cast<const __half*>(rec + kW3RecCodes)[r];
+  const uint32_t z = has_zero ? rec[kW3RecCodes + 256 + r] : 4u;
+  const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
+  const uint32_t zbits = 0x4300u + z;
+  return RowQ{sbits | (sbits << 16), zbits | (zbits << 16)};
+}
+
+// A whole 128-K INT3 record for weight row r (as dequant_block): the row's
+// 12 code words come in three 16-byte loads.  In each 32-K chunk (words
+// 3c .. 3c+2) pairs 0-14 sit at bits 3j / 16 + 3j of their word, so one
+// shift and one LOP3 give bf16 (128 + q, 128 + q'); pair 15 gathers code
+// bit p from bits 15 / 31 of word p.  Then w = ((128 + q) - (128 + z)) * s
+// as for INT4.
+__device__ __forceinline__ void w3_dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
+  uint4 raw[3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) raw[i] = *reinterpret_cast<const uint4*>(rec + (i * 128 + r) * 16);
+  const uint32_t wv[12] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y,
+                           raw[1].z, raw[1].w, raw[2].x, raw[2].y, raw[2].z, raw[2].w};
+  const RowQ qp = row_qparams3(rec, r, has_zero);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t out[16];
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        const uint32_t x2 = lop3_and_or(wv[3 * c + p] >> (3 * j), 0x00070007u, 0x43004300u);
+        out[5 * p + j] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+      }
+    }
+    uint32_t x2 = lop3_and_or(wv[3 * c] >> 15, 0x00010001u, 0x43004300u);
+    x2 = lop3_and_or(wv[3 * c + 1] >> 14, 0x00020002u, x2);
+    x2 = lop3_and_or(wv[3 * c + 2] >> 13, 0x00040004u, x2);
+    out[15] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+    tmem_st_x16(taddr + c * 16, out);
+  }
+}
+
+template <int NTOK, int FMT>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
-  using C = Cfg<NTOK, MX>;
+  using C = Cfg<NTOK, FMT>;
   constexpr int SS = C::kSmemStages;
   constexpr int TS = C::kTmemStages;
   constexpr int ACC = C::kAccBufs;
@@ -432,8 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tbase = tmem_base + lane_addr + a_col(t);
         tc_fence_after();
         for (int rr = 0; rr < nrec; ++rr) {
-          if constexpr (MX)
+          if constexpr (FMT == kFmtMx)
             mx_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, tbase + rr * 64);
+          else if constexpr (FMT == kFmtInt3)
+            w3_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
           else
             dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
         }
@@ -483,10 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
-template <int NTOK, bool MX = false>
+template <int NTOK, int FMT = kFmtInt4>
 hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_kernel<NTOK, MX>;
-  const size_t smem = Cfg<NTOK, MX>::kSmem;
+  auto kern = w4a16_kernel<NTOK, FMT>;
+  const size_t smem = Cfg<NTOK, FMT>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -615,8 +662,9 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.expert_offsets = expert_offsets;
   p.err = static_cast<uint32_t*>(ws);
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16;
+  const bool int3 = d.fmt == HQ_FMT_INT3;
   p.has_zero = d.has_zero_point ? 1 : 0;
-  p.rec_bytes = mx ? kMxA16RecBytes : w4_record_bytes(p.has_zero);
+  p.rec_bytes = mx ? kMxA16RecBytes : int3 ? w3_record_bytes(p.has_zero) : w4_record_bytes(p.has_zero);
   p.n_tiles = (d.n + kTileN - 1) / kTileN;
   p.k_blocks = d.k / kBlockK;
   p.expert_bytes = (uint64_t)p.n_tiles * p.k_blocks * p.rec_bytes;
@@ -657,16 +705,26 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   // the library's choice for 64-token tiles, where it measured faster
   // (dense M=64: 26.3 vs 28.4 us at K=7168, N=18432; grouped 64-token tiles
   // up to 13 % faster); the bf16-rescaled kernel everywhere else.
-  // (MXFP4 weights: always the rescaled kernel, one scale per 32 K.)
-  const bool exact = !mx && cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
+  // (MXFP4 and INT3 weights: always the rescaled kernel.)
+  const bool exact = !mx && !int3 && cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
   if (exact) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
   if (mx) {
     switch (cfg.ntok) {
-      case 16: return launch_t<16, true>(map, p, cfg.grid, stream);
-      case 32: return launch_t<32, true>(map, p, cfg.grid, stream);
-      case 64: return launch_t<64, true>(map, p, cfg.grid, stream);
-      case 128: return launch_t<128, true>(map, p, cfg.grid, stream);
-      case 256: return launch_t<256, true>(map, p, cfg.grid, stream);
+      case 16: return launch_t<16, kFmtMx>(map, p, cfg.grid, stream);
+      case 32: return launch_t<32, kFmtMx>(map, p, cfg.grid, stream);
+      case 64: return launch_t<64, kFmtMx>(map, p, cfg.grid, stream);
+      case 128: return launch_t<128, kFmtMx>(map, p, cfg.grid, stream);
+      case 256: return launch_t<256, kFmtMx>(map, p, cfg.grid, stream);
+      default: return HQ_ERR_UNSUPPORTED;
+    }
+  }
+  if (int3) {
+    switch (cfg.ntok) {
+      case 16: return launch_t<16, kFmtInt3>(map, p, cfg.grid, stream);
+      case 32: return launch_t<32, kFmtInt3>(map, p, cfg.grid, stream);
+      case 64: return launch_t<64, kFmtInt3>(map, p, cfg.grid, stream);
+      case 128: return launch_t<128, kFmtInt3>(map, p, cfg.grid, stream);
+      case 256: return launch_t<256, kFmtInt3>(map, p, cfg.grid, stream);
       default: return HQ_ERR_UNSUPPORTED;
     }
   }

@@ -45,6 +45,9 @@ def test_desc_validation():
                        ((hq.HQ_FMT_MXFP4_A16, 128, 96, 32, 0, 1), hq.HQ_ERR_UNSUPPORTED),
                        ((hq.HQ_FMT_MXFP4_A16, 128, 128, 32, 1, 1), hq.HQ_ERR_UNSUPPORTED),
                        ((hq.HQ_FMT_MXFP4_A16, 128, 128, 32, 0, 1025), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT3, 128, 128, 64, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT3, 128, 160, 128, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT3, 128, 128, 128, 2, 1), hq.HQ_ERR_INVALID_ARG),
                        ((7, 128, 128, 16, 0, 1), hq.HQ_ERR_INVALID_ARG)]:
         with pytest.raises(hq.HQError) as e:
             hq.hq_quant_desc_init(*args)
@@ -81,6 +84,34 @@ def test_fp4_pack_matches_oracle_layout(fmt, block, n):
     blob = hq.hq_pack_weights(d, codes, scales, None, g)
     ref = L.fp4_pack(codes, scales, block, g if fmt == hq.HQ_FMT_NVFP4 else None)
     assert np.array_equal(blob, ref)
+
+
+@pytest.mark.parametrize("n,k,asym,experts", [(256, 384, False, 1), (200, 256, True, 1), (136, 256, True, 3)])
+def test_int3_pack_matches_oracle_layout(n, k, asym, experts):
+    q, s, z = synth.w3a16_weights(n, k, 128, asym, seed=n + 3, experts=experts if experts > 1 else None)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, int(asym), experts)
+    blob = hq.hq_pack_weights(d, q, s, z)
+    assert blob.size == L.w3a16_packed_bytes(n, k, asym, experts)
+    qn, sn = q.numpy(), s.numpy()
+    zn = None if z is None else z.numpy()
+    if experts == 1:
+        ref = L.w3a16_pack(qn, sn, zn)
+    else:
+        ref = np.concatenate([L.w3a16_pack(qn[e], sn[e], None if zn is None else zn[e]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+def test_int3_pack_rejects_bad_zero_points():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 128, 128, 128, 1, 1)
+    q, s, z = synth.w3a16_weights(128, 128, 128, True, seed=4)
+    zb = z.clone()
+    zb[5, 0] = 8
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_pack_weights(d, q, s, zb)
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
+    with pytest.raises(hq.HQError) as e:                 # zeros missing for an asymmetric descriptor
+        hq.hq_pack_weights(d, q, s, None)
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("n,k,experts", [(128, 128, 1), (300, 384, 1), (136, 256, 3)])
@@ -176,6 +207,9 @@ def test_gemm_argument_errors_need_no_gpu():
     assert L_.hq_gemm_w4a16_static(ctypes.byref(dx), 16, 16, 4, 32, ctypes.byref(t), None) == hq.HQ_ERR_UNSUPPORTED
     assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dx), 4096, 16, 16, 4, 32, None, 256, 1 << 20,
                                None) == hq.HQ_ERR_INVALID_ARG
+    d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 256, 256, 128, 1, 1)
+    assert L_.hq_gemm_w4a16(ctypes.byref(d3), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
+                            None) == hq.HQ_ERR_UNSUPPORTED
     dxg = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 8)
     assert L_.hq_grouped_gemm_moe(ctypes.byref(dxg), 16, 16, 16, 40, 32, ctypes.byref(t), 256, 1 << 20,
                                   None) == hq.HQ_ERR_UNSUPPORTED
@@ -231,4 +265,5 @@ def test_autotune_candidates_need_no_gpu():
     assert not any(t.variant == 2 and t.tile_m > 64 for t in autotune.candidates("w4a16", 4096)[1:])
     assert all(t.variant == 0 for t in autotune.candidates("nvfp4", 256)[1:])
     assert all(t.variant == 1 for t in autotune.candidates("mxfp4_a16", 16)[1:])
+    assert all(t.variant == 1 for t in autotune.candidates("w3a16", 64)[1:])
     assert all(t.split_k == 0 for t in autotune.candidates("moe", 64)[1:])
