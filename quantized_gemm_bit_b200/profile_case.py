@@ -2,6 +2,7 @@
 
     python -m quantized_gemm_bit_b200.profile_case --kind w4a16 --m 16 --k 7168 --n 18432 --iters 3
     python -m quantized_gemm_bit_b200.profile_case --kind nvfp4 --m 8192 --k 8192 --n 8192 --iters 2
+    python -m quantized_gemm_bit_b200.profile_case --kind w3a16 --m 16 --k 7168 --n 18432 --iters 3
 
 Inputs are the seeded synthetic workload tensors; the device status is
 checked at the end (non-zero exit on any error).  Used to capture ncu
@@ -19,7 +20,7 @@ from .build import build
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "moe", "mxfp4", "nvfp4"])
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "mxfp4_a16", "moe", "mxfp4", "nvfp4"])
     ap.add_argument("--m", type=int, default=16)
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)
@@ -65,10 +66,20 @@ def main(argv=None):
         ws = torch.zeros(max(256, hq.hq_workspace_size(d, a.m, tuning)), dtype=torch.uint8, device=dev)
         for _ in range(a.iters):
             run(c, ws)
-    elif a.kind == "w4a16":
-        q, s, z = synth.w4a16_weights(a.n, a.k, 128, a.asym, seed=1000)
-        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, int(a.asym), 1)
-        blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+    elif a.kind in ("w4a16", "w3a16", "mxfp4_a16"):
+        # the W4A16 kernels with INT4, INT3 or MXFP4 weights
+        if a.kind == "w4a16":
+            q, s, z = synth.w4a16_weights(a.n, a.k, 128, a.asym, seed=1000)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, int(a.asym), 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+        elif a.kind == "w3a16":
+            q, s, z = synth.w3a16_weights(a.n, a.k, 128, a.asym, seed=7000)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, a.n, a.k, 128, int(a.asym), 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+        else:
+            codes, e8 = synth.mxfp4_weights(a.n, a.k, seed=6000)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, a.n, a.k, 32, 0, 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(dev)
         x = synth.bf16_normal(a.m, a.k, seed=1001).to(dev)
         c = torch.empty(a.m, a.n, dtype=torch.bfloat16, device=dev)
         ws = torch.zeros(max(256, hq.hq_workspace_size(d, a.m, tuning)), dtype=torch.uint8, device=dev)
