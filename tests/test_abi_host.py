@@ -145,6 +145,27 @@ def test_mxfp4_a16_pack_rejects_scales_that_overflow_bf16():
     assert e.value.status == hq.HQ_ERR_INVALID_ARG
 
 
+def test_mxfp4_a16_pack_accepts_the_largest_finite_scale():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 128, 128, 32, 0, 1)
+    codes, e8 = synth.mxfp4_weights(128, 128, seed=6)
+    e8[:] = 252
+    blob = hq.hq_pack_weights(d, codes, e8)
+    assert np.array_equal(blob, L.mxa16_pack(codes.numpy(), e8.numpy()))
+
+
+def test_w4a16_family_formats_share_one_launch_plan():
+    """INT3 and MXFP4 weights run the INT4 kernels' plan: the same workspace
+    for the same shape, token count and tuning (no device needed; the size
+    is computed for a 148-SM part)."""
+    for m, t in ((1, None), (16, None), (300, None), (4096, None), (40, hq.Tuning(split_k=3)),
+                 (200, hq.Tuning(tile_m=128))):
+        d4 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
+        d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 18432, 7168, 128, 1, 1)
+        dx = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 18432, 7168, 32, 0, 1)
+        w = hq.hq_workspace_size(d4, m, t)
+        assert w >= 256 and hq.hq_workspace_size(d3, m, t) == w == hq.hq_workspace_size(dx, m, t)
+
+
 def test_fp4_scale_layout_is_a_bijection():
     n, k, block = 256, 512, 16
     nn, bb = np.meshgrid(np.arange(n), np.arange(k // block), indexing="ij")
