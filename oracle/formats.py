@@ -8,6 +8,9 @@ Formats (the pages only name them; meanings from the public standards):
   * INT3 (unsigned code 0..7, GPTQ INT3 weights: the Vietnamese edition
     of the Humming news, section "meaning for domestic deployers"), with
     the same group scale / zero point.
+  * INT2 (unsigned code 0..3; INT1..INT8 weights are listed on the same
+    page, section "one library, many formats"), with the same group scale
+    / zero point.
   * e2m1 (FP4): OCP MX v1.0, section 5.3.3 "FP4 (E2M1)": 1 sign bit,
     2 exponent bits with bias 1, 1 mantissa bit, no inf/NaN, max 6.0.
   * E8M0 scale: OCP MX v1.0, section 5.4 "E8M0": value 2**(e-127), 0xFF NaN.
@@ -289,3 +292,28 @@ def int3_pack_stream(codes):
     bits = np.stack([(c >> i) & 1 for i in range(3)], axis=2).reshape(n, 3 * k)
     words = (bits.reshape(n, 3 * k // 32, 32) << np.arange(32, dtype=np.int64)).sum(axis=2)
     return words.astype(np.uint32).view(np.int32)
+
+
+def int2_unpack_words(qweight):
+    """int32 [N, K/16] words -> uint8 codes [N, K] (0..3).
+
+    Canonical INT2 container (the pages list INT1..INT8 weights without a
+    packing; the INT4 reading with 2-bit fields): element k of a row lives
+    in bits [2*(k%16), 2*(k%16)+2) of word k//16 (low bits first)."""
+    w = np.asarray(qweight).astype(np.int64) & 0xFFFFFFFF
+    n, kw = w.shape
+    shifts = 2 * np.arange(16, dtype=np.int64)
+    return ((w[:, :, None] >> shifts[None, None, :]) & 3).reshape(n, kw * 16).astype(np.uint8)
+
+
+def int2_pack_words(codes):
+    """uint8 codes [N, K] (0..3), K % 16 == 0 -> int32 [N, K/16] (inverse of
+    int2_unpack_words)."""
+    c = np.asarray(codes).astype(np.int64)
+    n, k = c.shape
+    assert k % 16 == 0
+    c = c.reshape(n, k // 16, 16)
+    w = np.zeros((n, k // 16), dtype=np.int64)
+    for e in range(16):
+        w |= (c[:, :, e] & 3) << (2 * e)
+    return w.astype(np.uint32).view(np.int32)

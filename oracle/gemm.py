@@ -85,6 +85,29 @@ def w3a16_ref(a_bf16, qweight, scales, zeros, group, rows=None, cols=None):
     return a @ w.T
 
 
+def w2a16_dequant(qweight, scales, zeros, group, rows=None):
+    """INT2 weights: W_hat[n, k] = (q[n, k] - z[n, k // G]) * s[n, k // G]
+    (fp64) with 2-bit codes (formats.int2_unpack_words); symmetric zero
+    point 2, the middle of the code range."""
+    if rows is not None:
+        qweight = np.asarray(qweight)[rows]
+        scales = np.asarray(scales)[rows]
+        zeros = None if zeros is None else np.asarray(zeros)[rows]
+    q = F.int2_unpack_words(qweight).astype(np.float64)
+    n, k = q.shape
+    g = np.arange(k) // group
+    s = np.asarray(scales, dtype=np.float16).astype(np.float64)[:, g]
+    z = 2.0 if zeros is None else np.asarray(zeros).astype(np.float64)[:, g]
+    return (q - z) * s
+
+
+def w2a16_ref(a_bf16, qweight, scales, zeros, group, rows=None, cols=None):
+    """C = A_hat @ W_hat.T in fp64 for INT2 weights (bf16 bit patterns in)."""
+    a = F.bf16_bits_to_f64(a_bf16 if rows is None else np.asarray(a_bf16)[rows])
+    w = w2a16_dequant(qweight, scales, zeros, group, rows=cols)
+    return a @ w.T
+
+
 def w4a16_ref_integer_domain(a_bf16, qweight, scales, zeros, group):
     """The same product evaluated as sum_g s_g * sum_{k in g} a_k (q_k - z_g):
     the group sums use integer weights (q - z), the scale enters once per
@@ -275,5 +298,15 @@ def grouped_w3a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, gr
     def dequant(e):
         z = None if zeros is None else zeros[e]
         return w3a16_dequant(qweights[e], scales[e], z, group, rows=cols)
+    ncols = np.asarray(qweights).shape[1] if cols is None else len(cols)
+    return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)
+
+
+def grouped_w2a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, group, row_subset=None, cols=None):
+    """Grouped form of w2a16_ref: qweights int32 [E, N, K/16], scales
+    float16 [E, N, K/G], zeros uint8 [E, N, K/G] or None.  Returns (rows, C)."""
+    def dequant(e):
+        z = None if zeros is None else zeros[e]
+        return w2a16_dequant(qweights[e], scales[e], z, group, rows=cols)
     ncols = np.asarray(qweights).shape[1] if cols is None else len(cols)
     return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)

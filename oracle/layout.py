@@ -334,3 +334,91 @@ def w3a16_unpack(blob, n, k, has_zero):
     sbits = blob[off].astype(np.uint16) | (blob[off + 1].astype(np.uint16) << 8)
     zeros = blob[w3a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // 128) if has_zero else None
     return codes.reshape(n, k).astype(np.uint8), sbits.reshape(n, k // 128).view(np.float16), zeros
+
+
+# ---------------------------------------------------------------------------
+# INT2 W2A16 (group 128), layout version 1
+#   Records as for INT4: one per (tile nt of 128 rows, block kb of 128 K), in
+#   (nt, kb) order, experts one after another; record size
+#   4096 + 256 (+ 128 with zero points) bytes.
+#   codes : row r's 8 code words; word q (q = 2c + p: 32-K chunk c, part
+#           p < 2) is the 32-bit little-endian word at byte
+#           (q // 4 * 128 + r) * 16 + 4 * (q % 4).  Code kk = k - 128*kb of
+#           chunk c = kk // 32, pair i = (kk % 32) // 2, half h = kk % 2
+#           sits in word 2c + i // 8 at bits 2*(i % 8) + 16*h .. +1.
+#   scale : fp16 bits at byte 4096 + 2*r;  zero: uint8 at 4096 + 256 + r.
+#   Rows n >= N (tile padding) hold code 0, scale 0 and zero 0.
+# ---------------------------------------------------------------------------
+
+
+def w2a16_record_bytes(has_zero):
+    return 4096 + 256 + (128 if has_zero else 0)
+
+
+def w2a16_packed_bytes(n, k, has_zero, num_experts=1):
+    return num_experts * (-(-n // 128)) * (k // 128) * w2a16_record_bytes(has_zero)
+
+
+def w2a16_code_word_and_bit(n, k, kdim, has_zero):
+    """Elementwise formula: (byte offset of the word holding code (n, k) in
+    the expert blob, bit position of its low bit)."""
+    n = np.asarray(n, dtype=np.int64)
+    k = np.asarray(k, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    kb, kk = k // 128, k % 128
+    c, i, h = kk // 32, (kk % 32) // 2, kk % 2
+    q = 2 * c + i // 8
+    word = (nt * (kdim // 128) + kb) * w2a16_record_bytes(has_zero) + (q // 4 * 128 + r) * 16 + 4 * (q % 4)
+    return word, 2 * (i % 8) + 16 * h
+
+
+def w2a16_scale_byte(n, kb, kdim, has_zero):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    return (nt * (kdim // 128) + kb) * w2a16_record_bytes(has_zero) + 4096 + 2 * r
+
+
+def w2a16_zero_byte(n, kb, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    return (nt * (kdim // 128) + kb) * w2a16_record_bytes(True) + 4096 + 256 + r
+
+
+def w2a16_pack(qweight, scales, zeros, group=128):
+    """Canonical (int32 [N, K/16], fp16 [N, K/128], uint8 [N, K/128] | None)
+    -> packed blob of one expert, placed by the formulas above."""
+    assert group == 128
+    codes = F.int2_unpack_words(qweight).astype(np.uint32)
+    n, k = codes.shape
+    has_zero = zeros is not None
+    out = np.zeros(w2a16_packed_bytes(n, k, has_zero), dtype=np.uint8)
+    words = np.zeros(out.size // 4, dtype=np.uint32)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    word, bit = w2a16_code_word_and_bit(nn.ravel(), kk.ravel(), k, has_zero)
+    np.bitwise_or.at(words, word // 4, codes.ravel() << bit.astype(np.uint32))
+    out[:] = words.view(np.uint8)
+    sb = np.asarray(scales, dtype=np.float16).view(np.uint16)
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    off = w2a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    out[off] = (sb.ravel() & 0xFF).astype(np.uint8)
+    out[off + 1] = (sb.ravel() >> 8).astype(np.uint8)
+    if has_zero:
+        out[w2a16_zero_byte(ng.ravel(), gg.ravel(), k)] = np.asarray(zeros, dtype=np.uint8).ravel()
+    return out
+
+
+def w2a16_unpack(blob, n, k, has_zero):
+    """Inverse of w2a16_pack -> (codes uint8 [N, K], scales fp16 [N, K/128],
+    zeros uint8 [N, K/128] | None)."""
+    blob = np.asarray(blob, dtype=np.uint8)
+    words = blob.view(np.uint32)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    word, bit = w2a16_code_word_and_bit(nn.ravel(), kk.ravel(), k, has_zero)
+    codes = (words[word // 4] >> bit.astype(np.uint32)) & 3
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    off = w2a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    sbits = blob[off].astype(np.uint16) | (blob[off + 1].astype(np.uint16) << 8)
+    zeros = blob[w2a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // 128) if has_zero else None
+    return codes.reshape(n, k).astype(np.uint8), sbits.reshape(n, k // 128).view(np.float16), zeros

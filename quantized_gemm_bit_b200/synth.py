@@ -15,6 +15,8 @@ Recipes (one per workload; seed = workload index * 1000 + shape index):
   * W3A16 (INT3): as W4A16 with 3 K/32 int32 words per row (every bit
     uniform = uniform 3-bit codes in a little-endian bit stream) and zero
     points uniform in [0, 7] (symmetric: zero point 4).
+  * W2A16 (INT2): as W4A16 with K/16 int32 words per row (16 uniform
+    2-bit codes each) and zero points uniform in [0, 3] (symmetric: 2).
   * W4A8-MXFP4 (and MXFP4 weights with bf16 activations): FP4 codes
     uniform over the 16 codes, two per byte (even k low nibble); one E8M0
     scale per 32 K with exponent uniform in [-8, -2];
@@ -53,6 +55,22 @@ def w4a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
     zeros = None
     if asym:
         zeros = torch.randint(0, 16, lead + (n, k // group), generator=g, dtype=torch.uint8)
+    return qweight, scales, zeros
+
+
+def w2a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
+    """Canonical INT2 weights: qweight int32 [.., N, K/16] with every bit
+    uniform (= 16 uniform 2-bit codes per word along K, low bits first), fp16
+    scales as for W4A16, zero points uniform in [0, 3] (asymmetric) or none
+    (symmetric, zero point 2)."""
+    assert k % group == 0 and k % 16 == 0
+    g = _gen(seed)
+    lead = () if experts is None else (experts,)
+    qweight = torch.randint(-(2 ** 31), 2 ** 31, lead + (n, k // 16), generator=g, dtype=torch.int32)
+    scales = (0.002 + 0.01 * torch.randn(lead + (n, k // group), generator=g).abs()).to(torch.float16)
+    zeros = None
+    if asym:
+        zeros = torch.randint(0, 4, lead + (n, k // group), generator=g, dtype=torch.uint8)
     return qweight, scales, zeros
 
 
