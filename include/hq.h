@@ -87,7 +87,9 @@ typedef enum {
   HQ_FMT_NVFP4 = 3, /* e2m1 codes, E4M3 scale per 16 K, fp32 tensor scale                          */
   HQ_FMT_MXFP4_A16 = 4, /* e2m1 codes, E8M0 scale per 32 K, for bf16 activations: the W4A16 entry
                            points dequantize it in registers like INT4                              */
-  HQ_FMT_INT3 = 5       /* unsigned INT3 codes, fp16 scale + optional uint3 zero point per group of
+  HQ_FMT_INT3 = 5,      /* unsigned INT3 codes, fp16 scale + optional uint3 zero point per group of
+                           128 K, for bf16 activations (the W4A16 entry points)                     */
+  HQ_FMT_INT2 = 6       /* unsigned INT2 codes, fp16 scale + optional uint2 zero point per group of
                            128 K, for bf16 activations (the W4A16 entry points)                     */
 } hq_format;
 
@@ -98,8 +100,9 @@ typedef struct {
   int32_t fmt;            /* hq_format                                                 */
   int32_t n;              /* output features (weight rows), per expert                 */
   int32_t k;              /* input features (reduction length)                         */
-  int32_t group_size;     /* INT4, INT3: 128; MXFP4, MXFP4_A16: 32; NVFP4: 16          */
-  int32_t has_zero_point; /* INT4 / INT3: 1 = zero point per group, 0 = symmetric (8 / 4) */
+  int32_t group_size;     /* INT4, INT3, INT2: 128; MXFP4, MXFP4_A16: 32; NVFP4: 16    */
+  int32_t has_zero_point; /* INT4 / INT3 / INT2: 1 = zero point per group, 0 = symmetric
+                             (zero point 8 / 4 / 2)                                    */
   int32_t num_experts;    /* 1 = dense layer; >1 = MoE weights stored expert after expert */
 } hq_quant_desc;
 
@@ -138,8 +141,8 @@ const char* hq_status_string(hq_status s);
  *   MXFP4: k % 128 == 0, group_size == 32, has_zero_point == 0
  *   NVFP4: k % 256 == 0, group_size == 16, has_zero_point == 0
  *   MXFP4_A16: k % 128 == 0, group_size == 32, has_zero_point == 0
- *   INT3 : k % 128 == 0, group_size == 128
- *   num_experts 1..1024 for INT4, INT3 and MXFP4_A16 (MoE), 1 otherwise. */
+ *   INT3, INT2: k % 128 == 0, group_size == 128
+ *   num_experts 1..1024 for INT4, INT3, INT2 and MXFP4_A16 (MoE), 1 otherwise. */
 hq_status hq_quant_desc_init(hq_quant_desc* d, int32_t fmt, int32_t n, int32_t k, int32_t group_size,
                              int32_t has_zero_point, int32_t num_experts);
 
@@ -162,29 +165,36 @@ size_t hq_packed_size(const hq_quant_desc* d);
  *          bit b = bit b%32 of word b/32), the container of GPTQ INT3
  *          scales_host = fp16 bits [E][N][K/128]
  *          zeros_host  = uint8 [E][N][K/128] (0..7), NULL when symmetric
+ *   INT2 : codes_host  = int32 [E][N][K/16], element k in bits 2*(k%16)..+1
+ *          scales_host = fp16 bits [E][N][K/128]
+ *          zeros_host  = uint8 [E][N][K/128] (0..3), NULL when symmetric
  *   MXFP4_A16: codes_host = uint8 [E][N][K/2] (even k in the low nibble),
  *          scales_host = uint8 E8M0 [E][N][K/32], every byte <= 252 (a
  *          larger scale would overflow bf16 weights, 255 is NaN).
  * The output layout (layout version 1) is spelled out in the header comment
  * of the packer source, hq_pack.cpp.
  * Errors: HQ_ERR_INVALID_ARG (NULL pointers, zeros given for a symmetric
- * descriptor or missing for an asymmetric one, a zero point > 15),
+ * descriptor or missing for an asymmetric one, a zero point above the
+ * code range (15 / 7 / 3 for INT4 / INT3 / INT2), an MXFP4_A16 scale byte
+ * > 252),
  * HQ_ERR_WORKSPACE_TOO_SMALL (out_bytes < hq_packed_size). */
 hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
                           const void* zeros_host, float global_scale, void* out_host, size_t out_bytes);
 
-/* Workspace bytes that hq_gemm_w4a16 (fmt INT4, INT3 or MXFP4_A16, num_experts 1),
+/* Workspace bytes that hq_gemm_w4a16 (fmt INT4, INT3, INT2 or MXFP4_A16, num_experts 1),
  * hq_gemm_mxfp4_a8, hq_gemm_nvfp4 or hq_grouped_gemm_moe need for M rows
  * (total sorted rows for MoE) and the given tuning (NULL = heuristic). */
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
 
 /* Dense W4A16 GEMM ([P-fa] table row "W4A16 dense"): C = A * W_hat^T with
  * W_hat[n,k] = (q[n,k] - z[n,k/128]) * s[n,k/128] dequantized in-kernel.
- *   d            : INT4, INT3 or MXFP4_A16 descriptor, num_experts == 1.
+ *   d            : INT4, INT3, INT2 or MXFP4_A16 descriptor, num_experts == 1.
  *                  INT3 (GPTQ INT3 weights, [P-vi] "meaning for domestic
  *                  deployers"): W_hat = (q - z) * s with 3-bit codes and
  *                  the symmetric zero point 4, computed as for INT4 (tuning
- *                  variant 1 for every tile; variant 2 is refused).
+ *                  variant 1 for every tile; variant 2 is refused).  INT2
+ *                  ([P-fa] format list INT1..INT8) likewise, with 2-bit codes
+ *                  and the symmetric zero point 2.
  *                  MXFP4_A16 (MXFP4 weights with bf16 activations; [P-fa2]
  *                  paragraph 2 lists MXFP4 weights and bf16 activations):
  *                  W_hat[n,k] = e2m1(c[n,k]) * 2^(e[n,k/32] - 127), each
@@ -273,8 +283,8 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
  * "MoE W4A16"): for every expert e, rows [off[e], off[e+1]) of A_sorted
  * times W_hat_e^T.  The tile scheduler reads expert_offsets on the device
  * (no host synchronization).
- *   d              : INT4, INT3 or MXFP4_A16 descriptor, num_experts = e
- *                    (per-expert n, k); INT3 and MXFP4_A16 weights as for
+ *   d              : INT4, INT3, INT2 or MXFP4_A16 descriptor, num_experts =
+ *                    e (per-expert n, k); INT3, INT2 and MXFP4_A16 weights as for
  *                    hq_gemm_w4a16
  *   packed_w_dev   : blob of all experts from hq_pack_weights
  *   a_sorted_dev   : bf16 [total_rows][k]

@@ -77,6 +77,7 @@ hq_status check_desc(const hq_quant_desc* d) {
         return HQ_ERR_UNSUPPORTED;
       return HQ_OK;
     case HQ_FMT_INT3:
+    case HQ_FMT_INT2:
       if (d->group_size != 128 || d->k % 128 != 0) return HQ_ERR_UNSUPPORTED;
       if (d->has_zero_point != 0 && d->has_zero_point != 1) return HQ_ERR_INVALID_ARG;
       if (d->num_experts > 1024) return HQ_ERR_UNSUPPORTED;
@@ -88,7 +89,7 @@ hq_status check_desc(const hq_quant_desc* d) {
 
 // Formats the W4A16 kernels read (dequantized in registers, bf16 MMA).
 bool w4_format(const hq_quant_desc* d) {
-  return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_MXFP4_A16;
+  return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_INT2 || d->fmt == HQ_FMT_MXFP4_A16;
 }
 
 // Tuning checks shared by the W4A16 entry points (dense: split_k free;
@@ -172,7 +173,7 @@ hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const 
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
   if (!codes_host || !scales_host || !out_host) return HQ_ERR_INVALID_ARG;
-  if (d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3) {
+  if (d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_INT2) {
     if ((d->has_zero_point != 0) != (zeros_host != nullptr)) return HQ_ERR_INVALID_ARG;
   } else if (zeros_host) {
     return HQ_ERR_INVALID_ARG;

@@ -27,6 +27,9 @@ constexpr int kMxA16RecBytes = kW4RecCodes + 512;
 // (128, with zero points) as in the INT4 record
 constexpr int kW3RecCodes = 6144;
 inline int w3_record_bytes(bool has_zero) { return kW3RecCodes + 256 + (has_zero ? 128 : 0); }
+// INT2 weights: 4096 code bytes, then scales and zero points as for INT4
+constexpr int kW2RecCodes = 4096;
+inline int w2_record_bytes(bool has_zero) { return kW2RecCodes + 256 + (has_zero ? 128 : 0); }
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 

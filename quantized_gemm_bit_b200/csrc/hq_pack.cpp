@@ -61,6 +61,16 @@
 //                  the bf16 pair (128 + q, 128 + q').
 //   [6144, 6400)   fp16 scale of row r at 6144 + 2r
 //   [6400, 6528)   uint3 zero point of row r at 6400 + r (asymmetric only)
+//
+// INT2 (group 128).  Records as for INT4, 4096 + 256 (+128) bytes:
+//   [0, 4096)      codes: row r's 8 words; word q = 2c + p (32-K chunk c,
+//                  part p < 2) at byte (q/4*128 + r)*16 + 4*(q%4).  Pair i
+//                  of chunk c (codes 32c + 2i, 32c + 2i + 1) sits in word
+//                  2c + i/8 at bits 2*(i%8) (even k) and 16 + 2*(i%8) (odd
+//                  k): one shift and one LOP3 with 0x00030003 / 0x43004300
+//                  give the bf16 pair (128 + q, 128 + q').
+//   [4096, 4352)   fp16 scale of row r at 4096 + 2r
+//   [4352, 4480)   uint2 zero point of row r at 4352 + r (asymmetric only)
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -201,6 +211,49 @@ hq_status pack_int3(const hq_quant_desc& d, const int32_t* codes, const uint16_t
   return HQ_OK;
 }
 
+hq_status pack_int2(const hq_quant_desc& d, const int32_t* codes, const uint16_t* scales, const uint8_t* zeros,
+                    uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int nt_count = (n + kTileN - 1) / kTileN;
+  const int kb_count = k / kBlockK;
+  const bool hz = zeros != nullptr;
+  const size_t rec = (size_t)w2_record_bytes(hz);
+  const size_t expert_bytes = (size_t)nt_count * kb_count * rec;
+  const size_t kw = (size_t)k / 16;  // canonical words per row
+  const size_t kg = (size_t)k / 128;
+  if (hz) {
+    const size_t total = (size_t)d.num_experts * n * kg;
+    for (size_t i = 0; i < total; ++i)
+      if (zeros[i] > 3) return HQ_ERR_INVALID_ARG;
+  }
+  const size_t jobs = (size_t)d.num_experts * nt_count;
+  parallel_for(jobs, [&](size_t job) {
+    const size_t e = job / nt_count;
+    const int nt = (int)(job % nt_count);
+    uint8_t* ebase = out + e * expert_bytes;
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint8_t* r0 = ebase + ((size_t)nt * kb_count + kb) * rec;
+      std::memset(r0, 0, rec);
+      for (int r = 0; r < kTileN; ++r) {
+        const int row = nt * kTileN + r;
+        if (row >= n) break;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(codes + (e * n + row) * kw) + (size_t)kb * 8;
+        uint32_t words[8] = {};
+        for (int kk = 0; kk < 128; ++kk) {
+          const uint32_t v = (src[kk / 16] >> (2 * (kk % 16))) & 3u;
+          const int c = kk / 32, i = (kk % 32) / 2, h = kk % 2;
+          words[2 * c + i / 8] |= v << (2 * (i % 8) + 16 * h);
+        }
+        for (int q = 0; q < 8; ++q) std::memcpy(r0 + ((size_t)(q / 4) * 128 + r) * 16 + 4 * (q % 4), &words[q], 4);
+        const uint16_t s = scales[(e * n + row) * kg + kb];
+        std::memcpy(r0 + kW2RecCodes + 2 * r, &s, 2);
+        if (hz) r0[kW2RecCodes + 256 + r] = zeros[(e * n + row) * kg + kb];
+      }
+    }
+  });
+  return HQ_OK;
+}
+
 // [pair j][half h][code bit b] -> bit of the 32-bit word
 constexpr int kMxBits[4][2][4] = {
     {{6, 7, 8, 15}, {22, 23, 24, 31}},
@@ -298,6 +351,8 @@ size_t packed_size_impl(const hq_quant_desc& d) {
       return (size_t)d.num_experts * nt * (d.k / kBlockK) * kMxA16RecBytes;
     case HQ_FMT_INT3:
       return (size_t)d.num_experts * nt * (d.k / kBlockK) * w3_record_bytes(d.has_zero_point != 0);
+    case HQ_FMT_INT2:
+      return (size_t)d.num_experts * nt * (d.k / kBlockK) * w2_record_bytes(d.has_zero_point != 0);
     default:
       return 0;
   }
@@ -318,6 +373,9 @@ hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scale
                          static_cast<uint8_t*>(out));
     case HQ_FMT_INT3:
       return pack_int3(d, static_cast<const int32_t*>(codes), static_cast<const uint16_t*>(scales),
+                       static_cast<const uint8_t*>(zeros), static_cast<uint8_t*>(out));
+    case HQ_FMT_INT2:
+      return pack_int2(d, static_cast<const int32_t*>(codes), static_cast<const uint16_t*>(scales),
                        static_cast<const uint8_t*>(zeros), static_cast<uint8_t*>(out));
     default:
       return HQ_ERR_INVALID_ARG;

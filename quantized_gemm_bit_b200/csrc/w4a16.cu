@@ -1,6 +1,6 @@
 // Dense and grouped (MoE) W4A16 GEMM for sm_100a with the INT4 dequantization
-// fused into the kernel (also run with INT3 or MXFP4 weights: the same
-// kernel with another record decode).
+// fused into the kernel (also run with INT3, INT2 or MXFP4 weights: the
+// same kernel with another record decode).
 //
 // Method: the weights are stored as 4-bit codes with a per-group fp16 scale
 // and an optional uint4 zero point, described separately ("Humming:
@@ -47,8 +47,8 @@ constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 
 // Weight formats of the kernel: INT4 records, MXFP4 records (8704 bytes; a
 // tighter barrier area keeps the 256-token tile inside the shared-memory
-// limit) and INT3 records (at most 6528 bytes).
-constexpr int kFmtInt4 = 0, kFmtMx = 1, kFmtInt3 = 2;
+// limit), INT3 records (at most 6528 bytes) and INT2 records (at most 4480).
+constexpr int kFmtInt4 = 0, kFmtMx = 1, kFmtInt3 = 2, kFmtInt2 = 3;
 
 template <int NTOK, int FMT = kFmtInt4>
 struct Cfg {
@@ -57,7 +57,10 @@ struct Cfg {
   static constexpr int kKps = NTOK <= 64 ? 2 : 1;
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
-  static constexpr int kRecStride = FMT == kFmtMx ? kMxA16RecBytes : FMT == kFmtInt3 ? kW3RecCodes + 384 : kRecMax;
+  static constexpr int kRecStride = FMT == kFmtMx     ? kMxA16RecBytes
+                                    : FMT == kFmtInt3 ? kW3RecCodes + 384
+                                    : FMT == kFmtInt2 ? kW2RecCodes + 384
+                                                      : kRecMax;
   static constexpr int kRecs = kKps * kRecStride;
   static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
   static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
@@ -237,6 +240,40 @@ __device__ __forceinline__ void w3_dequant_block(const uint8_t* rec, int r, int 
     x2 = lop3_and_or(wv[3 * c + 1] >> 14, 0x00020002u, x2);
     x2 = lop3_and_or(wv[3 * c + 2] >> 13, 0x00040004u, x2);
     out[15] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+    tmem_st_x16(taddr + c * 16, out);
+  }
+}
+
+// ---- INT2 weights (2-bit codes, fp16 scale and uint2 zero point per 128 K)
+__device__ __forceinline__ RowQ row_qparams2(const uint8_t* rec, int r, int has_zero) {
+  const __half sc = reinterpret_cast<const __half*>(rec + kW2RecCodes)[r];
+  const uint32_t z = has_zero ? rec[kW2RecCodes + 256 + r] : 2u;
+  const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
+  const uint32_t zbits = 0x4300u + z;
+  return RowQ{sbits | (sbits << 16), zbits | (zbits << 16)};
+}
+
+// A whole 128-K INT2 record for weight row r (as dequant_block): the row's
+// 8 code words come in two 16-byte loads; pair i of 32-K chunk c sits at
+// bits 2j / 16 + 2j (j = i % 8) of word 2c + i / 8, so one shift and one
+// LOP3 give bf16 (128 + q, 128 + q'), then w = ((128 + q) - (128 + z)) * s.
+__device__ __forceinline__ void w2_dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
+  uint4 raw[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) raw[i] = *reinterpret_cast<const uint4*>(rec + (i * 128 + r) * 16);
+  const uint32_t wv[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y, raw[1].z, raw[1].w};
+  const RowQ qp = row_qparams2(rec, r, has_zero);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t out[16];
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t x2 = lop3_and_or(wv[2 * c + p] >> (2 * j), 0x00030003u, 0x43004300u);
+        out[8 * p + j] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+      }
+    }
     tmem_st_x16(taddr + c * 16, out);
   }
 }
@@ -481,6 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, tbase + rr * 64);
           else if constexpr (FMT == kFmtInt3)
             w3_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
+          else if constexpr (FMT == kFmtInt2)
+            w2_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
           else
             dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
         }
@@ -663,8 +702,12 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.err = static_cast<uint32_t*>(ws);
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16;
   const bool int3 = d.fmt == HQ_FMT_INT3;
+  const bool int2 = d.fmt == HQ_FMT_INT2;
   p.has_zero = d.has_zero_point ? 1 : 0;
-  p.rec_bytes = mx ? kMxA16RecBytes : int3 ? w3_record_bytes(p.has_zero) : w4_record_bytes(p.has_zero);
+  p.rec_bytes = mx     ? kMxA16RecBytes
+                : int3 ? w3_record_bytes(p.has_zero)
+                : int2 ? w2_record_bytes(p.has_zero)
+                       : w4_record_bytes(p.has_zero);
   p.n_tiles = (d.n + kTileN - 1) / kTileN;
   p.k_blocks = d.k / kBlockK;
   p.expert_bytes = (uint64_t)p.n_tiles * p.k_blocks * p.rec_bytes;
@@ -705,8 +748,8 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   // the library's choice for 64-token tiles, where it measured faster
   // (dense M=64: 26.3 vs 28.4 us at K=7168, N=18432; grouped 64-token tiles
   // up to 13 % faster); the bf16-rescaled kernel everywhere else.
-  // (MXFP4 and INT3 weights: always the rescaled kernel.)
-  const bool exact = !mx && !int3 && cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
+  // (MXFP4, INT3 and INT2 weights: always the rescaled kernel.)
+  const bool exact = d.fmt == HQ_FMT_INT4 && cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
   if (exact) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
   if (mx) {
     switch (cfg.ntok) {
@@ -725,6 +768,16 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
       case 64: return launch_t<64, kFmtInt3>(map, p, cfg.grid, stream);
       case 128: return launch_t<128, kFmtInt3>(map, p, cfg.grid, stream);
       case 256: return launch_t<256, kFmtInt3>(map, p, cfg.grid, stream);
+      default: return HQ_ERR_UNSUPPORTED;
+    }
+  }
+  if (int2) {
+    switch (cfg.ntok) {
+      case 16: return launch_t<16, kFmtInt2>(map, p, cfg.grid, stream);
+      case 32: return launch_t<32, kFmtInt2>(map, p, cfg.grid, stream);
+      case 64: return launch_t<64, kFmtInt2>(map, p, cfg.grid, stream);
+      case 128: return launch_t<128, kFmtInt2>(map, p, cfg.grid, stream);
+      case 256: return launch_t<256, kFmtInt2>(map, p, cfg.grid, stream);
       default: return HQ_ERR_UNSUPPORTED;
     }
   }

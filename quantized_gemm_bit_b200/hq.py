@@ -36,6 +36,7 @@ HQ_FMT_MXFP4 = 2
 HQ_FMT_NVFP4 = 3
 HQ_FMT_MXFP4_A16 = 4
 HQ_FMT_INT3 = 5
+HQ_FMT_INT2 = 6
 
 # Every symbol include/hq.h declares.
 EXPORTS = (

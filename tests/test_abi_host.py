@@ -48,6 +48,8 @@ def test_desc_validation():
                        ((hq.HQ_FMT_INT3, 128, 128, 64, 0, 1), hq.HQ_ERR_UNSUPPORTED),
                        ((hq.HQ_FMT_INT3, 128, 160, 128, 0, 1), hq.HQ_ERR_UNSUPPORTED),
                        ((hq.HQ_FMT_INT3, 128, 128, 128, 2, 1), hq.HQ_ERR_INVALID_ARG),
+                       ((hq.HQ_FMT_INT2, 128, 128, 32, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT2, 128, 128, 128, 0, 1025), hq.HQ_ERR_UNSUPPORTED),
                        ((7, 128, 128, 16, 0, 1), hq.HQ_ERR_INVALID_ARG)]:
         with pytest.raises(hq.HQError) as e:
             hq.hq_quant_desc_init(*args)
@@ -99,6 +101,31 @@ def test_int3_pack_matches_oracle_layout(n, k, asym, experts):
     else:
         ref = np.concatenate([L.w3a16_pack(qn[e], sn[e], None if zn is None else zn[e]) for e in range(experts)])
     assert np.array_equal(blob, ref)
+
+
+@pytest.mark.parametrize("n,k,asym,experts", [(256, 384, False, 1), (200, 256, True, 1), (136, 256, True, 3)])
+def test_int2_pack_matches_oracle_layout(n, k, asym, experts):
+    q, s, z = synth.w2a16_weights(n, k, 128, asym, seed=n + 2, experts=experts if experts > 1 else None)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, n, k, 128, int(asym), experts)
+    blob = hq.hq_pack_weights(d, q, s, z)
+    assert blob.size == L.w2a16_packed_bytes(n, k, asym, experts)
+    qn, sn = q.numpy(), s.numpy()
+    zn = None if z is None else z.numpy()
+    if experts == 1:
+        ref = L.w2a16_pack(qn, sn, zn)
+    else:
+        ref = np.concatenate([L.w2a16_pack(qn[e], sn[e], None if zn is None else zn[e]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+def test_int2_pack_rejects_bad_zero_points():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, 128, 128, 128, 1, 1)
+    q, s, z = synth.w2a16_weights(128, 128, 128, True, seed=4)
+    zb = z.clone()
+    zb[9, 0] = 4
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_pack_weights(d, q, s, zb)
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
 
 
 def test_int3_pack_rejects_bad_zero_points():
@@ -162,8 +189,10 @@ def test_w4a16_family_formats_share_one_launch_plan():
         d4 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
         d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 18432, 7168, 128, 1, 1)
         dx = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 18432, 7168, 32, 0, 1)
+        d2 = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, 18432, 7168, 128, 0, 1)
         w = hq.hq_workspace_size(d4, m, t)
         assert w >= 256 and hq.hq_workspace_size(d3, m, t) == w == hq.hq_workspace_size(dx, m, t)
+        assert hq.hq_workspace_size(d2, m, t) == w
 
 
 def test_fp4_scale_layout_is_a_bijection():
@@ -228,9 +257,10 @@ def test_gemm_argument_errors_need_no_gpu():
     assert L_.hq_gemm_w4a16_static(ctypes.byref(dx), 16, 16, 4, 32, ctypes.byref(t), None) == hq.HQ_ERR_UNSUPPORTED
     assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dx), 4096, 16, 16, 4, 32, None, 256, 1 << 20,
                                None) == hq.HQ_ERR_INVALID_ARG
-    d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 256, 256, 128, 1, 1)
-    assert L_.hq_gemm_w4a16(ctypes.byref(d3), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
-                            None) == hq.HQ_ERR_UNSUPPORTED
+    for fmt in (hq.HQ_FMT_INT3, hq.HQ_FMT_INT2):
+        d3 = hq.hq_quant_desc_init(fmt, 256, 256, 128, 1, 1)
+        assert L_.hq_gemm_w4a16(ctypes.byref(d3), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
+                                None) == hq.HQ_ERR_UNSUPPORTED
     dxg = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 8)
     assert L_.hq_grouped_gemm_moe(ctypes.byref(dxg), 16, 16, 16, 40, 32, ctypes.byref(t), 256, 1 << 20,
                                   None) == hq.HQ_ERR_UNSUPPORTED
