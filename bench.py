@@ -468,8 +468,8 @@ def run_mxfp4(args, rank, world, peaks):
 def _run_w16_format(args, world, peaks, fmt):
     """Another weight format on the W4A16 kernels (bf16 activations):
     M in {16, 64, 256, 4096}, K=7168, N=18432.  fmt "mxfp4_a16": e2m1 codes
-    with an E8M0 scale per 32 K; "w3a16": INT3 codes with an fp16 scale per
-    128 K (symmetric)."""
+    with an E8M0 scale per 32 K; "w3a16" / "w2a16": INT3 / INT2 codes with
+    an fp16 scale per 128 K (symmetric)."""
     from quantized_gemm_bit_b200 import hq, synth
     k, n = 7168, 18432
     if fmt == "mxfp4_a16":
@@ -478,12 +478,18 @@ def _run_w16_format(args, world, peaks, fmt):
         blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).cuda()
         wbytes = n * k // 2 + n * k // 32
         name, dt = "MXFP4 weights x bf16 activations", "bf16 x e2m1 (fp32 accumulate)"
-    else:
+    elif fmt == "w3a16":
         q, sc, _ = synth.w3a16_weights(n, k, 128, False, seed=7000)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
         blob = torch.from_numpy(hq.hq_pack_weights(d, q, sc)).cuda()
         wbytes = 3 * n * k // 8 + 2 * n * (k // GROUP)
         name, dt = "INT3 weights (group 128) x bf16 activations", "bf16 x int3 (fp32 accumulate)"
+    else:
+        q, sc, _ = synth.w2a16_weights(n, k, 128, False, seed=7500)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, n, k, 128, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, sc)).cuda()
+        wbytes = n * k // 4 + 2 * n * (k // GROUP)
+        name, dt = "INT2 weights (group 128) x bf16 activations", "bf16 x int2 (fp32 accumulate)"
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
     ms_list = (16, 64, 256, 4096)
@@ -519,6 +525,10 @@ def run_mxfp4_a16(args, rank, world, peaks):
 
 def run_w3a16(args, rank, world, peaks):
     return _run_w16_format(args, world, peaks, "w3a16")
+
+
+def run_w2a16(args, rank, world, peaks):
+    return _run_w16_format(args, world, peaks, "w2a16")
 
 
 def run_nvfp4(args, rank, world, peaks):
@@ -709,7 +719,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "w3a16", "nvfp4", "moe"])
+    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "w3a16", "w2a16", "nvfp4", "moe"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -732,7 +742,7 @@ def main():
     if args.workload == "w4a16_sweep":
         line = run_w4a16_sweep(args, rank, world, peaks)
     else:
-        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "w3a16": run_w3a16, "nvfp4": run_nvfp4,
+        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "w3a16": run_w3a16, "w2a16": run_w2a16, "nvfp4": run_nvfp4,
               "moe": run_moe}[args.workload]
         line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "data": "synthetic (seeded)"}

@@ -33,11 +33,11 @@ TILES = (16, 32, 64, 128, 256)
 def candidates(kind, m):
     """Tunings worth trying at m rows: token tiles up to twice the rows
     (at least 16), K splits 0 (the library's choice) to 3, and for the
-    W4A16 kernels with INT4 weights both weight variants (MXFP4 and INT3
-    weights have only the rescaled one)."""
+    W4A16 kernels with INT4 weights both weight variants (MXFP4, INT3 and
+    INT2 weights have only the rescaled one)."""
     cap = max(16, 2 * m)
     tiles = [t for t in TILES if t <= cap] or [16]
-    variants = (1, 2) if kind in ("w4a16", "moe") else (1,) if kind in ("mxfp4_a16", "w3a16") else (0,)
+    variants = (1, 2) if kind in ("w4a16", "moe") else (1,) if kind in ("mxfp4_a16", "w3a16", "w2a16") else (0,)
     splits = (0,) if kind == "moe" else (0, 1, 2, 3)
     out = [None]
     for t in tiles:
@@ -97,9 +97,13 @@ def _setup(kind, m, n, k, experts, topk, dev):
 
         def call(t, i, c, ws):
             hq.hq_gemm_w4a16(d, blobs[i], a, m, c, ws, t)
-    elif kind == "w3a16":
-        q, s, _ = synth.w3a16_weights(n, k, 128, False, seed=7000)
-        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
+    elif kind in ("w3a16", "w2a16"):
+        if kind == "w3a16":
+            q, s, _ = synth.w3a16_weights(n, k, 128, False, seed=7000)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
+        else:
+            q, s, _ = synth.w2a16_weights(n, k, 128, False, seed=7500)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, n, k, 128, 0, 1)
         blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev))
         a = synth.bf16_normal(m, k, seed=7001).to(dev)
         rows = m
@@ -188,7 +192,7 @@ def autotune(kind, m, n, k, experts=256, topk=8, tunings=None, dev="cuda"):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "mxfp4_a16", "mxfp4", "nvfp4", "moe"])
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "w2a16", "mxfp4_a16", "mxfp4", "nvfp4", "moe"])
     ap.add_argument("--m", type=int, default=16, help="rows (tokens for --kind moe)")
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)

@@ -20,7 +20,7 @@ from .build import build
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "mxfp4_a16", "moe", "mxfp4", "nvfp4"])
+    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "w2a16", "mxfp4_a16", "moe", "mxfp4", "nvfp4"])
     ap.add_argument("--m", type=int, default=16)
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)
@@ -66,8 +66,8 @@ def main(argv=None):
         ws = torch.zeros(max(256, hq.hq_workspace_size(d, a.m, tuning)), dtype=torch.uint8, device=dev)
         for _ in range(a.iters):
             run(c, ws)
-    elif a.kind in ("w4a16", "w3a16", "mxfp4_a16"):
-        # the W4A16 kernels with INT4, INT3 or MXFP4 weights
+    elif a.kind in ("w4a16", "w3a16", "w2a16", "mxfp4_a16"):
+        # the W4A16 kernels with INT4, INT3, INT2 or MXFP4 weights
         if a.kind == "w4a16":
             q, s, z = synth.w4a16_weights(a.n, a.k, 128, a.asym, seed=1000)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, int(a.asym), 1)
@@ -75,6 +75,10 @@ def main(argv=None):
         elif a.kind == "w3a16":
             q, s, z = synth.w3a16_weights(a.n, a.k, 128, a.asym, seed=7000)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, a.n, a.k, 128, int(a.asym), 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+        elif a.kind == "w2a16":
+            q, s, z = synth.w2a16_weights(a.n, a.k, 128, a.asym, seed=7500)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, a.n, a.k, 128, int(a.asym), 1)
             blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
         else:
             codes, e8 = synth.mxfp4_weights(a.n, a.k, seed=6000)

@@ -317,4 +317,5 @@ def test_autotune_candidates_need_no_gpu():
     assert all(t.variant == 0 for t in autotune.candidates("nvfp4", 256)[1:])
     assert all(t.variant == 1 for t in autotune.candidates("mxfp4_a16", 16)[1:])
     assert all(t.variant == 1 for t in autotune.candidates("w3a16", 64)[1:])
+    assert all(t.variant == 1 for t in autotune.candidates("w2a16", 16)[1:])
     assert all(t.split_k == 0 for t in autotune.candidates("moe", 64)[1:])
