@@ -317,3 +317,36 @@ def int2_pack_words(codes):
     for e in range(16):
         w |= (c[:, :, e] & 3) << (2 * e)
     return w.astype(np.uint32).view(np.int32)
+
+
+def int8_unpack_words(qweight):
+    """int32 [N, K/4] words -> uint8 codes [N, K] (0..255).
+
+    Canonical INT8 container (the pages list INT1..INT8 weights without a
+    packing; the INT4 reading with 8-bit fields): element k of a row lives in
+    bits [8*(k%4), 8*(k%4)+8) of word k//4 (low byte first)."""
+    w = np.asarray(qweight).astype(np.int64) & 0xFFFFFFFF
+    n, kw = w.shape
+    shifts = 8 * np.arange(4, dtype=np.int64)
+    return ((w[:, :, None] >> shifts[None, None, :]) & 0xFF).reshape(n, kw * 4).astype(np.uint8)
+
+
+def int8_pack_words(codes):
+    """uint8 codes [N, K], K % 4 == 0 -> int32 [N, K/4] (inverse of
+    int8_unpack_words)."""
+    c = np.asarray(codes).astype(np.int64)
+    n, k = c.shape
+    assert k % 4 == 0
+    c = c.reshape(n, k // 4, 4)
+    w = np.zeros((n, k // 4), dtype=np.int64)
+    for e in range(4):
+        w |= (c[:, :, e] & 0xFF) << (8 * e)
+    return w.astype(np.uint32).view(np.int32)
+
+
+def int4_twos_complement(codes):
+    """4-bit code (0..15) -> its two's-complement integer (-8..7): the MXINT4
+    element (an integer element with a shared E8M0 scale per 32 K, the MX
+    integer format read at 4 bits)."""
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    return np.where(c >= 8, c - 16, c)

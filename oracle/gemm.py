@@ -108,6 +108,30 @@ def w2a16_ref(a_bf16, qweight, scales, zeros, group, rows=None, cols=None):
     return a @ w.T
 
 
+def w8a16_dequant(qweight, scales, zeros, group, rows=None):
+    """INT8 weights: W_hat[n, k] = (q[n, k] - z[n, k // G]) * s[n, k // G]
+    (fp64), the INT4 definition with 8-bit codes (formats.int8_unpack_words);
+    zeros uint8 [N, K/G] holding 0..255, or None for the symmetric form
+    (zero point 128, the middle of the code range as 8 is for INT4)."""
+    if rows is not None:
+        qweight = np.asarray(qweight)[rows]
+        scales = np.asarray(scales)[rows]
+        zeros = None if zeros is None else np.asarray(zeros)[rows]
+    q = F.int8_unpack_words(qweight).astype(np.float64)
+    n, k = q.shape
+    g = np.arange(k) // group
+    s = np.asarray(scales, dtype=np.float16).astype(np.float64)[:, g]
+    z = 128.0 if zeros is None else np.asarray(zeros).astype(np.float64)[:, g]
+    return (q - z) * s
+
+
+def w8a16_ref(a_bf16, qweight, scales, zeros, group, rows=None, cols=None):
+    """C = A_hat @ W_hat.T in fp64 for INT8 weights (bf16 bit patterns in)."""
+    a = F.bf16_bits_to_f64(a_bf16 if rows is None else np.asarray(a_bf16)[rows])
+    w = w8a16_dequant(qweight, scales, zeros, group, rows=cols)
+    return a @ w.T
+
+
 def w4a16_ref_integer_domain(a_bf16, qweight, scales, zeros, group):
     """The same product evaluated as sum_g s_g * sum_{k in g} a_k (q_k - z_g):
     the group sums use integer weights (q - z), the scale enters once per
@@ -309,4 +333,51 @@ def grouped_w2a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, gr
         z = None if zeros is None else zeros[e]
         return w2a16_dequant(qweights[e], scales[e], z, group, rows=cols)
     ncols = np.asarray(qweights).shape[1] if cols is None else len(cols)
+    return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)
+
+
+def grouped_w8a16_ref(a_sorted_bf16, expert_offsets, qweights, scales, zeros, group, row_subset=None, cols=None):
+    """Grouped form of w8a16_ref: qweights int32 [E, N, K/4], scales
+    float16 [E, N, K/G], zeros uint8 [E, N, K/G] or None.  Returns (rows, C)."""
+    def dequant(e):
+        z = None if zeros is None else zeros[e]
+        return w8a16_dequant(qweights[e], scales[e], z, group, rows=cols)
+    ncols = np.asarray(qweights).shape[1] if cols is None else len(cols)
+    return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)
+
+
+# ---------------------------------------------------------------------------
+# MXINT4 weights x bf16 activations
+# ---------------------------------------------------------------------------
+
+
+def mxint4_dequant(w_packed, w_e8m0, rows=None):
+    """W_hat[n, k] = c[n, k] * 2**(e[n, k // 32] - 127) (fp64, exact): c the
+    two's-complement integer of the 4-bit code (formats.int4_twos_complement),
+    e the E8M0 scale byte of its 32-K block.  w_packed uint8 [N, K/2] (even
+    k in the low nibble), w_e8m0 uint8 [N, K/32]."""
+    if rows is not None:
+        w_packed = np.asarray(w_packed)[rows]
+        w_e8m0 = np.asarray(w_e8m0)[rows]
+    c = F.int4_twos_complement(F.fp4_unpack_bytes(w_packed)).astype(np.float64)
+    n, k = c.shape
+    e = np.asarray(w_e8m0).astype(np.int64)[:, np.arange(k) // MX_BLOCK]
+    return c * np.ldexp(1.0, e - 127)
+
+
+def mxint4_a16_ref(a_bf16, w_packed, w_e8m0, rows=None, cols=None):
+    """C = A_hat @ W_hat.T in fp64 for MXINT4 weights (the pages list MXINT4
+    among the weight types; Humming news page, section "one library, many
+    formats") and bf16 activations."""
+    a = F.bf16_bits_to_f64(a_bf16 if rows is None else np.asarray(a_bf16)[rows])
+    w = mxint4_dequant(w_packed, w_e8m0, rows=cols)
+    return a @ w.T
+
+
+def grouped_mxint4_a16_ref(a_sorted_bf16, expert_offsets, w_packed, w_e8m0, row_subset=None, cols=None):
+    """Grouped form of mxint4_a16_ref: w_packed uint8 [E, N, K/2], w_e8m0
+    uint8 [E, N, K/32].  Returns (rows, C)."""
+    def dequant(e):
+        return mxint4_dequant(w_packed[e], w_e8m0[e], rows=cols)
+    ncols = np.asarray(w_packed).shape[1] if cols is None else len(cols)
     return _grouped(a_sorted_bf16, expert_offsets, dequant, row_subset, ncols)

@@ -422,3 +422,160 @@ def w2a16_unpack(blob, n, k, has_zero):
     sbits = blob[off].astype(np.uint16) | (blob[off + 1].astype(np.uint16) << 8)
     zeros = blob[w2a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // 128) if has_zero else None
     return codes.reshape(n, k).astype(np.uint8), sbits.reshape(n, k // 128).view(np.float16), zeros
+
+
+# ---------------------------------------------------------------------------
+# Gated gate+up row order (for the GEMM with the SwiGLU epilogue), any of the
+# W4A16-family layouts above.  The canonical weights have N = 2I rows, gate
+# rows [0, I) and up rows [I, 2I).  Packed row p (tile j = p // 128, row
+# r = p % 128 of it, quarter q = r // 32, lane l = r % 32) holds canonical
+# row
+#     64 j + 16 q + l            for l < 16   (gate), and
+#     I + 64 j + 16 q + l - 16   for l >= 16  (up, the same feature),
+# so a 128-row tile covers features [64 j, 64 j + 64) of both projections.
+# The blob is the format's packed layout of the rows in this order.
+# ---------------------------------------------------------------------------
+
+
+def gated_source_rows(n):
+    """[n] int64: canonical row of every packed row p (n % 128 == 0)."""
+    assert n % 128 == 0
+    p = np.arange(n, dtype=np.int64)
+    j, r = p // 128, p % 128
+    q, lane = r // 32, r % 32
+    return np.where(lane < 16, 64 * j + 16 * q + lane, n // 2 + 64 * j + 16 * q + lane - 16)
+
+
+# ---------------------------------------------------------------------------
+# INT8 W8A16 (group 128), layout version 1
+#   Records as for INT4: one per (tile nt of 128 rows, block kb of 128 K), in
+#   (nt, kb) order, experts one after another; record size
+#   16384 + 256 (+ 128 with zero points) bytes.
+#   codes : code kk = k - 128*kb of row r at byte (kk // 16 * 128 + r) * 16
+#           + kk % 16 (row r's 16-K chunk c is 16 contiguous bytes, the
+#           chunks of 128 rows are 2 KB apart: conflict-free 16-byte reads);
+#   scale : fp16 bits at byte 16384 + 2*r;  zero: uint8 at 16384 + 256 + r.
+#   Rows n >= N (tile padding) hold code 0, scale 0 and zero 0.
+# ---------------------------------------------------------------------------
+
+
+def w8a16_record_bytes(has_zero):
+    return 16384 + 256 + (128 if has_zero else 0)
+
+
+def w8a16_packed_bytes(n, k, has_zero, num_experts=1):
+    return num_experts * (-(-n // 128)) * (k // 128) * w8a16_record_bytes(has_zero)
+
+
+def w8a16_code_byte(n, k, kdim, has_zero):
+    """Elementwise formula: byte offset of code (n, k) in the expert blob."""
+    n = np.asarray(n, dtype=np.int64)
+    k = np.asarray(k, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    kb, kk = k // 128, k % 128
+    return (nt * (kdim // 128) + kb) * w8a16_record_bytes(has_zero) + (kk // 16 * 128 + r) * 16 + kk % 16
+
+
+def w8a16_scale_byte(n, kb, kdim, has_zero):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    return (nt * (kdim // 128) + kb) * w8a16_record_bytes(has_zero) + 16384 + 2 * r
+
+
+def w8a16_zero_byte(n, kb, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    kb = np.asarray(kb, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    return (nt * (kdim // 128) + kb) * w8a16_record_bytes(True) + 16384 + 256 + r
+
+
+def w8a16_pack(qweight, scales, zeros, group=128):
+    """Canonical (int32 [N, K/4], fp16 [N, K/128], uint8 [N, K/128] | None)
+    -> packed blob of one expert, placed by the formulas above."""
+    assert group == 128
+    codes = F.int8_unpack_words(qweight)
+    n, k = codes.shape
+    has_zero = zeros is not None
+    out = np.zeros(w8a16_packed_bytes(n, k, has_zero), dtype=np.uint8)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    out[w8a16_code_byte(nn.ravel(), kk.ravel(), k, has_zero)] = codes.ravel()
+    sb = np.asarray(scales, dtype=np.float16).view(np.uint16)
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    off = w8a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    out[off] = (sb.ravel() & 0xFF).astype(np.uint8)
+    out[off + 1] = (sb.ravel() >> 8).astype(np.uint8)
+    if has_zero:
+        out[w8a16_zero_byte(ng.ravel(), gg.ravel(), k)] = np.asarray(zeros, dtype=np.uint8).ravel()
+    return out
+
+
+def w8a16_unpack(blob, n, k, has_zero):
+    """Inverse of w8a16_pack -> (codes uint8 [N, K], scales fp16 [N, K/128],
+    zeros uint8 [N, K/128] | None)."""
+    blob = np.asarray(blob, dtype=np.uint8)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    codes = blob[w8a16_code_byte(nn.ravel(), kk.ravel(), k, has_zero)]
+    ng, gg = np.meshgrid(np.arange(n), np.arange(k // 128), indexing="ij")
+    off = w8a16_scale_byte(ng.ravel(), gg.ravel(), k, has_zero)
+    sbits = blob[off].astype(np.uint16) | (blob[off + 1].astype(np.uint16) << 8)
+    zeros = blob[w8a16_zero_byte(ng.ravel(), gg.ravel(), k)].reshape(n, k // 128) if has_zero else None
+    return codes.reshape(n, k), sbits.reshape(n, k // 128).view(np.float16), zeros
+
+
+# ---------------------------------------------------------------------------
+# MXINT4 for bf16 activations, layout version 1
+#   Records as for MXFP4_A16: one per (tile nt, block kb), experts one after
+#   another, 8192 + 512 bytes each.
+#   codes : the 4-bit code (two's complement) of (n, k) where the INT4
+#           layout puts its code (w4a16_code_byte_and_nibble);
+#   scale : E8M0 byte of row r, 32-K block c of the record at 8192 + 4r + c.
+# ---------------------------------------------------------------------------
+
+MXI4_REC = 8192 + 512
+
+
+def mxi4_packed_bytes(n, k, num_experts=1):
+    return num_experts * (-(-n // 128)) * (k // 128) * MXI4_REC
+
+
+def mxi4_code_byte_and_nibble(n, k, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    k = np.asarray(k, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    kb, kk = k // 128, k % 128
+    c, w, e = kk // 32, (kk % 32) // 8, kk % 8
+    p = (e % 2) * 4 + e // 2
+    return (nt * (kdim // 128) + kb) * MXI4_REC + (c * 128 + r) * 16 + w * 4 + p // 2, p % 2
+
+
+def mxi4_scale_byte(n, blk, kdim):
+    n = np.asarray(n, dtype=np.int64)
+    blk = np.asarray(blk, dtype=np.int64)
+    nt, r = n // 128, n % 128
+    kb, c = blk // 4, blk % 4
+    return (nt * (kdim // 128) + kb) * MXI4_REC + 8192 + 4 * r + c
+
+
+def mxi4_pack(codes_packed, scales):
+    """Canonical (uint8 [N, K/2] even k low nibble, uint8 E8M0 [N, K/32])
+    -> packed blob of one expert, placed by the formulas above."""
+    codes = F.fp4_unpack_bytes(np.asarray(codes_packed, dtype=np.uint8))
+    n, k = codes.shape
+    out = np.zeros(mxi4_packed_bytes(n, k), dtype=np.uint8)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    byte, nib = mxi4_code_byte_and_nibble(nn.ravel(), kk.ravel(), k)
+    np.bitwise_or.at(out, byte, (codes.ravel() << (4 * nib)).astype(np.uint8))
+    ns, bs = np.meshgrid(np.arange(n), np.arange(k // 32), indexing="ij")
+    out[mxi4_scale_byte(ns.ravel(), bs.ravel(), k)] = np.asarray(scales, dtype=np.uint8).ravel()
+    return out
+
+
+def mxi4_unpack(blob, n, k):
+    """Inverse of mxi4_pack: blob -> (codes uint8 [N, K], scales uint8 [N, K/32])."""
+    blob = np.asarray(blob, dtype=np.uint8)
+    nn, kk = np.meshgrid(np.arange(n), np.arange(k), indexing="ij")
+    byte, nib = mxi4_code_byte_and_nibble(nn.ravel(), kk.ravel(), k)
+    codes = (blob[byte] >> (4 * nib)) & 0xF
+    ns, bs = np.meshgrid(np.arange(n), np.arange(k // 32), indexing="ij")
+    return codes.reshape(n, k).astype(np.uint8), blob[mxi4_scale_byte(ns.ravel(), bs.ravel(), k)].reshape(n, k // 32)

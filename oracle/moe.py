@@ -80,6 +80,16 @@ def silu_mul(gate_up_bf16_bits, inter):
         return g / (1.0 + np.exp(-g)) * u
 
 
+def silu_mul_f64(gate_up, inter):
+    """SwiGLU on unrounded gate+up values: fp64 [rows, 2*inter] -> fp64
+    [rows, inter], h = silu(g) * u as in silu_mul (the form the GEMM with
+    the fused SwiGLU epilogue computes: no bf16 rounding of g and u)."""
+    x = np.asarray(gate_up, dtype=np.float64)
+    g, u = x[:, :inter], x[:, inter:2 * inter]
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
+
+
 def combine(y_sorted_bf16_bits, sorted_src, weights, k):
     """Un-permute and weigh the down GEMM's output: bf16 bits
     [T*k, H] in expert-sorted order -> fp64 [T, H],

@@ -177,3 +177,44 @@ def test_nvfp4_quantizer_properties():
     i, j = 5, 37
     d = np.float32(F.e4m3_decode(sb[i, j // 16]) * g)
     assert c[i, j] == F.e2m1_quantize_rne(np.array([x[i, j] / d], dtype=np.float32))[0]
+
+
+def test_nvfp4_quantizer_against_torch_fp32_steps():
+    """Pins of the two-level NVFP4 quantizer that do not reuse its code:
+    the tensor scale is torch's fp32 amax / fp32(2688); every block scale
+    is torch's float8_e4m3fn cast (round to nearest even) of the fp32
+    quotient amax_block / (6 g) with 6 g an fp32 product, saturated at 448;
+    every code is the nearest point of the e2m1 grid {0, .5, 1, 1.5, 2, 3,
+    4, 6} to the fp32 quotient x / fp32(E4M3(sb) g), ties to the even
+    code, found by brute force over the grid.  Blocks span many binades, so
+    a rounding step done in the wrong precision or order moves some block
+    scale by one E4M3 step and fails here."""
+    import torch
+    rng = np.random.default_rng(11)
+    rows, k = 64, 1024
+    x = rng.standard_normal((rows, k)).astype(np.float32)
+    x *= np.exp2(rng.integers(-12, 6, size=(rows, k // 16, 1))).repeat(16, axis=2).reshape(rows, k).astype(np.float32)
+    x[3, 32:48] = 0.0                                   # an all-zero block
+    c, sb, g = F.nvfp4_quantize(x)
+    xt = torch.from_numpy(x)
+    g_t = xt.abs().max() / torch.tensor(2688.0, dtype=torch.float32)
+    assert g_t.dtype == torch.float32 and np.float32(g) == np.float32(g_t.item())
+    bmax = xt.abs().reshape(rows, k // 16, 16).amax(dim=2)
+    ratio = bmax / (torch.tensor(6.0, dtype=torch.float32) * g_t)
+    sb_t = ratio.clamp(max=448.0).to(torch.float8_e4m3fn)
+    assert np.array_equal(sb, sb_t.view(torch.uint8).numpy())
+    # codes: brute force over the grid on torch's fp32 quotient
+    d = (sb_t.to(torch.float32) * g_t).reshape(rows, k // 16, 1)
+    safe = torch.where(d > 0, d, torch.ones_like(d))
+    r = (xt.reshape(rows, k // 16, 16) / safe).reshape(rows, k).double().numpy()
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    dist = np.abs(np.abs(r)[..., None] - grid)
+    best = dist.min(axis=-1, keepdims=True)
+    cand = dist == best
+    # ties: the even code of the two candidates
+    mag = np.where(cand[..., ::2].any(axis=-1), np.argmax(cand & (np.arange(8) % 2 == 0), axis=-1),
+                   np.argmax(cand, axis=-1))
+    expect = np.where((r < 0) & (mag > 0), mag | 8, mag)
+    zero_blk = (d.reshape(rows, k // 16) == 0).numpy().repeat(16, axis=1)
+    expect = np.where(zero_blk, 0, expect)
+    assert np.array_equal(c, expect.astype(np.uint8))

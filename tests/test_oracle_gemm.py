@@ -86,9 +86,9 @@ def test_w4a16_row_and_column_subsets():
 
 def test_mxfp4_matches_exact_integer_evaluation():
     codes, e8 = synth.mxfp4_weights(64, 256, seed=21)
-    aq, asc = synth.fp8_activations(7, 256, seed=22)
-    c1 = G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes.numpy(), e8.numpy())
-    c2 = G.mxfp4_a8_ref_exact(aq.numpy(), asc.numpy(), codes.numpy(), e8.numpy())
+    aq, asc = F.fp8_per_token_quantize(synth.bf16_normal(7, 256, seed=22).float().numpy())
+    c1 = G.mxfp4_a8_ref(aq, asc, codes.numpy(), e8.numpy())
+    c2 = G.mxfp4_a8_ref_exact(aq, asc, codes.numpy(), e8.numpy())
     assert np.max(np.abs(c1 - c2)) <= 1e-12 * np.max(np.abs(c1))
 
 
@@ -98,10 +98,10 @@ def test_mxfp4_unit_scales_is_plain_matmul_of_decoded_values():
     e2m1 table."""
     codes, _ = synth.mxfp4_weights(32, 128, seed=23)
     e8 = np.full((32, 4), 127, dtype=np.uint8)
-    aq, _ = synth.fp8_activations(4, 128, seed=24)
+    aq, _ = F.fp8_per_token_quantize(synth.bf16_normal(4, 128, seed=24).float().numpy())
     one = np.ones(4, dtype=np.float32)
-    got = G.mxfp4_a8_ref(aq.numpy(), one, codes.numpy(), e8)
-    a_t = aq.view(torch.float8_e4m3fn).to(torch.float64)
+    got = G.mxfp4_a8_ref(aq, one, codes.numpy(), e8)
+    a_t = torch.from_numpy(aq).view(torch.float8_e4m3fn).to(torch.float64)
     table = torch.tensor([0, .5, 1, 1.5, 2, 3, 4, 6, -0.0, -.5, -1, -1.5, -2, -3, -4, -6],
                          dtype=torch.float64)
     lo = codes.to(torch.int64) & 0xF

@@ -109,15 +109,6 @@ def test_gather_rows():
     assert np.array_equal(out, a[[2, 0, 3, 1]])
 
 
-def test_synth_fp8_matches_oracle_quantizer():
-    """The generator's library cast and the oracle's own quantizer agree."""
-    q, s = synth.fp8_activations(16, 512, seed=2000)
-    x = synth.bf16_normal(16, 512, 2000).float().numpy()
-    q2, s2 = F.fp8_per_token_quantize(x)
-    assert np.array_equal(s.numpy(), s2)
-    assert np.array_equal(F.e4m3_decode(q.numpy()), F.e4m3_decode(q2))
-
-
 def test_synth_distributions():
     q, s, z = synth.w4a16_weights(256, 1024, 128, True, seed=0)
     codes = F.int4_unpack_words(q.numpy())
@@ -208,3 +199,36 @@ def test_softmax_topk_weights_properties():
             assert np.isclose(w[tkn, a] / w[tkn, b], ratio, rtol=1e-12)
         assert np.all(np.diff(w[tkn]) <= 0)
     assert np.all(w.sum(axis=1) < 1.0)       # not renormalised over the k selected
+
+
+def test_silu_mul_f64_matches_the_bf16_form_and_the_logistic_function():
+    """The unrounded SwiGLU (for the fused epilogue) is the same function:
+    on bf16-representable inputs it equals silu_mul exactly, and on any
+    inputs g * expit(g) * u (scipy)."""
+    from scipy.special import expit
+    rng = np.random.default_rng(8)
+    g = rng.normal(0, 3, (5, 16))
+    u = rng.normal(0, 1, (5, 16))
+    x = np.concatenate([_bf16(g), _bf16(u)], axis=1)
+    assert np.array_equal(R.silu_mul_f64(F.bf16_bits_to_f64(x), 16), R.silu_mul(x, 16))
+    h = R.silu_mul_f64(np.concatenate([g, u], axis=1), 16)
+    assert np.allclose(h, g * expit(g) * u, rtol=1e-14, atol=0)
+
+
+def test_gated_row_order_hand_example_and_bijection():
+    """Packed row p of the gated order: gate rows in lanes 0-15 of every
+    32-row quarter, the up rows of the same features in lanes 16-31."""
+    src = L.gated_source_rows(256)            # I = 128
+    assert src[0] == 0 and src[15] == 15      # tile 0, quarter 0: gate 0..15
+    assert src[16] == 128 and src[31] == 143  # ... then up 0..15
+    assert src[32] == 16 and src[48] == 144   # quarter 1: features 16..31
+    assert src[127] == 128 + 63               # tile 0 ends with up feature 63
+    assert src[128] == 64 and src[144] == 192  # tile 1: features 64..127
+    assert np.array_equal(np.sort(src), np.arange(256))
+    big = L.gated_source_rows(4096)
+    assert np.array_equal(np.sort(big), np.arange(4096))
+    # every tile covers 64 gate features and the same 64 up features
+    for j in range(4096 // 128):
+        t = big[128 * j:128 * (j + 1)]
+        assert np.array_equal(np.sort(t[t < 2048]), np.arange(64 * j, 64 * j + 64))
+        assert np.array_equal(np.sort(t[t >= 2048]) - 2048, np.arange(64 * j, 64 * j + 64))
