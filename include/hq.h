@@ -6,23 +6,23 @@
  * in a low-bit format and are dequantized inside the GEMM kernel.  The
  * method (the Humming quantized-inference kernel library) is described on
  * news pages only:
- *   [P-fa]  Humming news page (news.cocoloop.cn, fr), section "Une seule
- *           bibliotheque pour une longue liste de formats": WnA16 / W8A8 /
- *           W4A8 / W4A4; INT1..INT8, FP4..FP8, MXFP4, MXINT4, NVFP4; table
- *           rows "W4A16 dense, petits lots", "W4A8-MXFP4, H200",
- *           "MoE W4A16, B300, grands lots".
- *   [P-fa2] "Humming: open-source kernel library for quantized inference"
- *           (news.ditty.ir), summary paragraph 2 (one standard description
- *           in which weight, scale, zero point and the other parameters are
- *           described separately), paragraph 3 (Layer / Compute / Tuning
- *           configs: shapes+dtype+arch / GEMM type / tile, stages, MMA),
- *           paragraph 4 (MXFP4 weights converted inside the kernel),
- *           paragraph 5 (the "Grouped" MoE path).
- *   [P-pt]  "Ant Group e vLLM lancam a biblioteca open source Humming"
- *           (aube.news), quantization paragraph (dense and MoE layers).
- *   [P-vi]  the Vietnamese edition of the same news (news.cocoloop.cn, vi),
- *           section on what it means for domestic deployers (GPTQ INT3
- *           weights served through the library).
+ *   [fr]  the French edition of the Ant/vLLM Humming kernels news
+ *         (news.cocoloop.cn), section "one library, many formats": WnA16 /
+ *         W8A8 / W4A8 / W4A4; INT1..INT8, FP4..FP8, MXFP4, MXINT4, NVFP4;
+ *         comparison-table rows "W4A16 dense, small batch", "W4A8-MXFP4,
+ *         H200", "MoE W4A16, B300, large batch".
+ *   [fa]  "Humming: open-source kernel library for quantized inference"
+ *         (news.ditty.ir), summary paragraph 2 (one standard description in
+ *         which weight, scale, zero point and the other parameters are
+ *         described separately), paragraph 3 (Layer / Compute / Tuning
+ *         configs: shapes+dtype+arch / GEMM type / tile, stages, MMA),
+ *         paragraph 4 (MXFP4 weights converted inside the kernel),
+ *         paragraph 5 (the "Grouped" MoE path).
+ *   [pt]  "Ant Group e vLLM lancam a biblioteca open source Humming"
+ *         (aube.news), quantization explainer (dense and MoE layers).
+ *   [vi]  the Vietnamese edition of the same news (news.cocoloop.cn),
+ *         section "meaning for domestic deployers" (GPTQ INT3 weights
+ *         served through the library) and "one library, many formats".
  * Element formats follow the public standards the pages name: OCP MX v1.0
  * (e2m1, E8M0, 32-element blocks), OCP FP8 (E4M3), NVIDIA NVFP4 (e2m1 with
  * an E4M3 scale per 16 elements and an fp32 tensor scale).
@@ -49,7 +49,8 @@
  *     everything else (activations, scales, offsets, outputs, workspace) is
  *     touched only after it has completed.  So the kernel launched just
  *     before a GEMM call must not write that call's packed weights (copies
- *     and memsets are ordinary stream dependencies and are not affected).
+ *     and memsets are ordinary stream dependencies and are not affected),
+ *     unless the call's tuning sets HQ_TUNE_NO_EARLY_WEIGHTS.
  */
 #ifndef HQ_H_
 #define HQ_H_
@@ -89,12 +90,16 @@ typedef enum {
                            points dequantize it in registers like INT4                              */
   HQ_FMT_INT3 = 5,      /* unsigned INT3 codes, fp16 scale + optional uint3 zero point per group of
                            128 K, for bf16 activations (the W4A16 entry points)                     */
-  HQ_FMT_INT2 = 6       /* unsigned INT2 codes, fp16 scale + optional uint2 zero point per group of
+  HQ_FMT_INT2 = 6,      /* unsigned INT2 codes, fp16 scale + optional uint2 zero point per group of
                            128 K, for bf16 activations (the W4A16 entry points)                     */
+  HQ_FMT_INT8 = 7,      /* unsigned INT8 codes, fp16 scale + optional uint8 zero point per group of
+                           128 K, for bf16 activations (the W4A16 entry points)                     */
+  HQ_FMT_MXINT4 = 8     /* two's-complement 4-bit integer codes, E8M0 scale per 32 K, for bf16
+                           activations (the W4A16 entry points)                                     */
 } hq_format;
 
-/* Quantization description ([P-fa2] paragraph 2) plus the Layer Config
- * shape fields ([P-fa2] paragraph 3).  Fill it with hq_quant_desc_init. */
+/* Quantization description ([fa] paragraph 2) plus the Layer Config
+ * shape fields ([fa] paragraph 3).  Fill it with hq_quant_desc_init. */
 typedef struct {
   int32_t layout_version; /* HQ_LAYOUT_VERSION                                         */
   int32_t fmt;            /* hq_format                                                 */
@@ -106,7 +111,7 @@ typedef struct {
   int32_t num_experts;    /* 1 = dense layer; >1 = MoE weights stored expert after expert */
 } hq_quant_desc;
 
-/* Execution choices (the Tuning Config of [P-fa2] paragraph 3).  Pass NULL
+/* Execution choices (the Tuning Config of [fa] paragraph 3).  Pass NULL
  * to let the library's heuristic choose; a zero field also means "choose".
  *   tile_m   : token tile (the MMA N extent): 16, 32, 64, 128 or 256
  *   tile_n   : weight rows per tile: 128 (the only value)
@@ -116,18 +121,28 @@ typedef struct {
  *              splits the whole iteration space evenly when 0)
  *   cta_group: 1 (one SM per MMA)
  *   variant  : W4A16 / grouped MoE: 0 = the library's choice, currently
- *              2 for 64-token tiles and 1 for every other tile.
- *              1 = weights rescaled to bf16 in the kernel,
- *              w = bf16((q - z) * bf16(s)), fp32 accumulation across K.
+ *              2 for token tiles of up to 64 and 1 for larger tiles
+ *              (MXFP4_A16 weights: always 1).
+ *              1 = weights rescaled to bf16 in the kernel: each weight is
+ *              the correctly rounded bf16 of (q - z) * s (one rounding),
+ *              fp32 accumulation across K.
  *              2 = for token tiles of up to 64, the exact integers (q - z)
  *              go to the tensor core and each 128-K group's scale is
- *              applied to its fp32 group sum (no rounding of w or s;
- *              on B200 faster than 1 at 64-token tiles, slower at 16 and
- *              32); larger tiles as 1.
+ *              applied to its fp32 group sum (no rounding of w or s);
+ *              larger tiles as 1.  INT4, INT3 and INT2 weights.
  *              Block-scaled GEMMs: 0.                                     */
 typedef struct {
   int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;
+  int32_t flags; /* HQ_TUNE_* bits below, 0 = none                         */
 } hq_tuning;
+
+/* hq_tuning.flags: the GEMM kernels do not fetch packed weights before the
+ * previous kernel on the stream has completed (see the launch-overlap rule
+ * in the header comment above).  For callers whose kernel just before a
+ * GEMM call writes that call's packed weights (an in-place repack or a
+ * weight update); costs the overlap of the weight prefetch with that
+ * kernel's tail. */
+#define HQ_TUNE_NO_EARLY_WEIGHTS 1
 
 /* Library and layout version. */
 int hq_layout_version(void);
@@ -149,7 +164,7 @@ hq_status hq_quant_desc_init(hq_quant_desc* d, int32_t fmt, int32_t n, int32_t k
 /* Size in bytes of the packed weight blob for *d (0 if *d is invalid). */
 size_t hq_packed_size(const hq_quant_desc* d);
 
-/* Offline weight packer ([P-fa2] paragraph 2: weight, scale and zero point
+/* Offline weight packer ([fa] paragraph 2: weight, scale and zero point
  * described separately -> one device layout).  Host memory in, host memory
  * out; the caller copies the result to the device.  Canonical inputs,
  * experts back to back:
@@ -186,16 +201,15 @@ hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const 
  * (total sorted rows for MoE) and the given tuning (NULL = heuristic). */
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
 
-/* Dense W4A16 GEMM ([P-fa] table row "W4A16 dense"): C = A * W_hat^T with
+/* Dense W4A16 GEMM ([fr] table row "W4A16 dense"): C = A * W_hat^T with
  * W_hat[n,k] = (q[n,k] - z[n,k/128]) * s[n,k/128] dequantized in-kernel.
  *   d            : INT4, INT3, INT2 or MXFP4_A16 descriptor, num_experts == 1.
- *                  INT3 (GPTQ INT3 weights, [P-vi] "meaning for domestic
+ *                  INT3 (GPTQ INT3 weights, [vi] "meaning for domestic
  *                  deployers"): W_hat = (q - z) * s with 3-bit codes and
- *                  the symmetric zero point 4, computed as for INT4 (tuning
- *                  variant 1 for every tile; variant 2 is refused).  INT2
- *                  ([P-fa] format list INT1..INT8) likewise, with 2-bit codes
+ *                  the symmetric zero point 4, computed as for INT4.  INT2
+ *                  ([fr] format list INT1..INT8) likewise, with 2-bit codes
  *                  and the symmetric zero point 2.
- *                  MXFP4_A16 (MXFP4 weights with bf16 activations; [P-fa2]
+ *                  MXFP4_A16 (MXFP4 weights with bf16 activations; [fa]
  *                  paragraph 2 lists MXFP4 weights and bf16 activations):
  *                  W_hat[n,k] = e2m1(c[n,k]) * 2^(e[n,k/32] - 127), each
  *                  weight converted to bf16 exactly (every scale byte <= 252
@@ -210,14 +224,14 @@ size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
 hq_status hq_gemm_w4a16(const hq_quant_desc* d, const void* packed_w_dev, const void* a_dev, int32_t m,
                         void* c_dev, const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
 
-/* W4A8-MXFP4 GEMM ([P-fa] table row "W4A8-MXFP4"; [P-fa2] paragraph 4):
+/* W4A8-MXFP4 GEMM ([fr] table row "W4A8-MXFP4"; [fa] paragraph 4):
  * C[m,n] = s_m * sum_k E4M3(a[m,k]) * e2m1(w[n,k]) * 2^(e[n,k/32]-127).
  *   a_e4m3_dev : uint8 [m][k] E4M3 codes;  a_scale_dev : fp32 [m] */
 hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, const void* a_e4m3_dev,
                            const float* a_scale_dev, int32_t m, void* c_dev, const hq_tuning* t, void* ws_dev,
                            size_t ws_bytes, hq_stream_t stream);
 
-/* NVFP4 W4A4 GEMM ([P-fa] format list, W4A4 combination):
+/* NVFP4 W4A4 GEMM ([fr] format list, W4A4 combination):
  * C = (g_a * g_w) * sum_k e2m1(a)*sf_a * e2m1(w)*sf_w.
  *   a_fp4_dev : uint8 [m][k/2] (even k low nibble); a_sf_dev : uint8 E4M3
  *   [m][k/16]; a_global : fp32 tensor scale of A.  g_w is in the blob.
@@ -229,7 +243,7 @@ hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const 
                         const void* a_sf_dev, float a_global, int32_t m, void* c_dev, const hq_tuning* t,
                         void* ws_dev, size_t ws_bytes, hq_stream_t stream);
 
-/* Activation quantization for the W4A8 GEMM ([P-fa] W4A8 combination):
+/* Activation quantization for the W4A8 GEMM ([fr] W4A8 combination):
  * per row r, s_r = amax_r / 448 (1 for an all-zero row) and
  * q[r][k] = RNE_E4M3(x[r][k] / s_r), saturating, every step in fp32 (OCP FP8
  * rounding); zero results are written as +0.
@@ -241,7 +255,7 @@ hq_status hq_quantize_fp8_rows(const void* x_bf16_dev, int32_t rows, int32_t k, 
 /* Workspace bytes hq_quantize_nvfp4 needs. */
 size_t hq_quantize_nvfp4_workspace_size(int32_t rows, int32_t k);
 
-/* Activation quantization for the W4A4 GEMM ([P-fa] NVFP4 type, W4A4):
+/* Activation quantization for the W4A4 GEMM ([fr] NVFP4 type, W4A4):
  * g = amax / (448*6) over the whole tensor (1 if all zero);
  * per 16 contiguous K: sb = RNE_E4M3(amax_block / (6 g)), d = E4M3(sb) * g,
  * c = RNE_e2m1(x / d) saturating (0 when d == 0); fp32 throughout.
@@ -251,7 +265,7 @@ size_t hq_quantize_nvfp4_workspace_size(int32_t rows, int32_t k);
 hq_status hq_quantize_nvfp4(const void* x_bf16_dev, int32_t rows, int32_t k, void* codes_dev, void* sf_dev,
                             float* global_dev, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
 
-/* MoE routing ([P-fa2] paragraph 5, "Grouped" path): top-k experts per
+/* MoE routing ([fa] paragraph 5, "Grouped" path): top-k experts per
  * token by router logit (equal to top-k by softmax probability), ties to
  * the lower expert index, slots in descending logit order.
  *   logits_dev : fp32 [t][e];  topk_ids_dev : int32 [t][k], written
@@ -279,7 +293,7 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
                          int32_t* expert_offsets_dev, const void* a_dev, int32_t hidden, void* a_sorted_dev,
                          void* ws_dev, size_t ws_bytes, hq_stream_t stream);
 
-/* Grouped MoE W4A16 GEMM, one launch for all experts ([P-fa] table row
+/* Grouped MoE W4A16 GEMM, one launch for all experts ([fr] table row
  * "MoE W4A16"): for every expert e, rows [off[e], off[e+1]) of A_sorted
  * times W_hat_e^T.  The tile scheduler reads expert_offsets on the device
  * (no host synchronization).
@@ -293,6 +307,31 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
 hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, const void* a_sorted_dev,
                               const int32_t* expert_offsets_dev, int32_t total_rows, void* c_sorted_dev,
                               const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
+
+/* Offline packer for the gate+up weights of a gated feed-forward, for
+ * hq_grouped_gemm_moe_swiglu: the same canonical inputs as hq_pack_weights
+ * (d->n = 2I rows: gate rows [0, I), up rows [I, 2I), per expert), packed
+ * in the gated row order: in every 32-row quarter q of 128-row tile j, rows
+ * 0-15 are the gate rows 64j + 16q + l and rows 16-31 the up rows
+ * I + 64j + 16q + l (l < 16), so that one tile's accumulators hold matching
+ * gate and up values.  Same blob size as hq_pack_weights.
+ *   d : INT4, INT3, INT2 or MXFP4_A16 descriptor with d->n % 128 == 0.
+ * Errors as hq_pack_weights; HQ_ERR_UNSUPPORTED for other formats or n. */
+hq_status hq_pack_weights_gated(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
+                                const void* zeros_host, void* out_host, size_t out_bytes);
+
+/* Grouped gate+up GEMM with the gated activation fused into its epilogue
+ * (the layer around the "Grouped" path; [fa] paragraph 5): for every expert
+ * e, rows [off[e], off[e+1]) of A_sorted times the expert's gate and up
+ * weights, then h = silu(gate) * up, silu(x) = x / (1 + exp(-x)), from the
+ * fp32 accumulators (no bf16 rounding of gate and up), one bf16 rounding.
+ *   d              : as for hq_grouped_gemm_moe, d->n = 2I, d->n % 128 == 0
+ *   packed_w_dev   : blob from hq_pack_weights_gated
+ *   h_sorted_dev   : bf16 [total_rows][d->n / 2], written
+ *   other arguments, tuning, workspace and errors as hq_grouped_gemm_moe. */
+hq_status hq_grouped_gemm_moe_swiglu(const hq_quant_desc* d, const void* packed_w_dev, const void* a_sorted_dev,
+                                     const int32_t* expert_offsets_dev, int32_t total_rows, void* h_sorted_dev,
+                                     const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream);
 
 /* Gated activation between the two grouped GEMMs of an MoE layer (the
  * pages leave the layer around the "Grouped" path open; this is the usual
@@ -342,17 +381,27 @@ hq_status hq_debug_timeout_probe(void* ws_dev, uint64_t limit_ns, hq_stream_t st
  * workspace (split-K tile counters and fp32 partial sums) lives here in one
  * fixed 16 MiB array inside the library, present on every device that loads
  * it until the process exits.
- *   Same arguments and result as hq_gemm_w4a16, without ws_dev / ws_bytes.
+ *   Same arguments and result as hq_gemm_w4a16 (INT4, INT3, INT2 or
+ *   MXFP4_A16 weights), without ws_dev / ws_bytes.
  *   A launch plan needing more than 16 MiB of scratch is refused with
  *   HQ_ERR_WORKSPACE_TOO_SMALL before anything runs (a smaller tile_m in
- *   `t` needs less).  Each call clears the part of the array that must start
- *   at zero on its own stream.  All calls share the array: calls that may
- *   overlap on the GPU (unordered streams) race; calls ordered on one stream
- *   are safe.  The first call on a device looks up the array's device
- *   address (cudaGetSymbolAddress), so make it before any stream capture.
- *   Device-side errors of this entry point are not reported separately. */
+ *   `t` needs less); a plan of whole tiles with a split-K tail whose partial
+ *   sums would not fit runs as whole tiles instead.  Each call that splits K
+ *   clears the array's tile counters on its own stream before the kernel.
+ *   All calls share the array: calls that may overlap on the GPU (unordered
+ *   streams) race; calls ordered on one stream are safe.  The first call in
+ *   each CUDA context looks up the array's device address
+ *   (cudaGetSymbolAddress), so make it before any stream capture.
+ *   A device-side error of any call (a bounded wait that ran out, after
+ *   which the output may be partly written) is kept in the array until
+ *   hq_static_check_device_status reads it. */
 hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* packed_w_dev, const void* a_dev, int32_t m,
                                void* c_dev, const hq_tuning* t, hq_stream_t stream);
+
+/* Synchronizes `stream`, then reads, clears and returns the first
+ * device-side error recorded by hq_gemm_w4a16_static calls on the current
+ * device since the last such read (HQ_OK when none).  Allocates nothing. */
+hq_status hq_static_check_device_status(hq_stream_t stream);
 
 #ifdef __cplusplus
 }

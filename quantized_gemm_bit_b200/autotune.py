@@ -33,11 +33,11 @@ TILES = (16, 32, 64, 128, 256)
 def candidates(kind, m):
     """Tunings worth trying at m rows: token tiles up to twice the rows
     (at least 16), K splits 0 (the library's choice) to 3, and for the
-    W4A16 kernels with INT4 weights both weight variants (MXFP4, INT3 and
-    INT2 weights have only the rescaled one)."""
+    W4A16 kernels with INT4, INT3 or INT2 weights both weight variants
+    (MXFP4 weights have only the rescaled one)."""
     cap = max(16, 2 * m)
     tiles = [t for t in TILES if t <= cap] or [16]
-    variants = (1, 2) if kind in ("w4a16", "moe") else (1,) if kind in ("mxfp4_a16", "w3a16", "w2a16") else (0,)
+    variants = (1, 2) if kind in ("w4a16", "moe", "w3a16", "w2a16") else (1,) if kind == "mxfp4_a16" else (0,)
     splits = (0,) if kind == "moe" else (0, 1, 2, 3)
     out = [None]
     for t in tiles:
@@ -123,8 +123,11 @@ def _setup(kind, m, n, k, experts, topk, dev):
         codes, e8 = synth.mxfp4_weights(n, k, seed=2000)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, n, k, 32, 0, 1)
         blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(dev))
-        aq, asc = synth.fp8_activations(m, k, seed=2001)
-        aq, asc = aq.to(dev), asc.to(dev)
+        # E4M3 activations from the library's own per-token quantizer
+        x = synth.bf16_normal(m, k, seed=2001).to(dev)
+        aq = torch.empty(m, k, dtype=torch.uint8, device=dev)
+        asc = torch.empty(m, dtype=torch.float32, device=dev)
+        hq.hq_quantize_fp8_rows(x, m, k, aq, asc)
         rows = m
 
         def call(t, i, c, ws):

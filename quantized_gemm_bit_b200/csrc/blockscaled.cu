@@ -108,6 +108,7 @@ struct BsParams {
   int sf_groups;             // 512-byte scale chunks per weight tile (whole K)
   int m_tiles;
   int data_parallel;         // whole tiles per unit, no partial sums
+  int early_weights;         // fetch the first stages' weights before griddepcontrol.wait
 };
 
 // NVFP4 activation scales, row-major [m][K/16] bytes, re-laid into the order
@@ -308,7 +309,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     // Phase 1, before the previous kernel on the stream has finished: the
     // packed weights of the first S stages (no kernel writes them)
     uint32_t n_pre = 0;
-    for (int idx = 0; n_pre < (uint32_t)S && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
+    for (int idx = 0; p.early_weights && n_pre < (uint32_t)S &&
+                      bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
          ++idx) {
       for (int ks = ks0; ks < ks1 && n_pre < (uint32_t)S; ++ks, ++n_pre) {
         if (leader) {
@@ -553,6 +555,7 @@ int bs_tiles(const hq_quant_desc& d, int m, int ntok) {
 
 BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t) {
   BsConfig cfg{};
+  cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
   auto dp_eff = [&](int nt) {
@@ -655,6 +658,7 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.total_iters = (long long)tiles * p.k_stages;
   p.m_tiles = (m + cfg.ntok - 1) / cfg.ntok;
   p.data_parallel = cfg.splits == 0 ? 1 : 0;
+  p.early_weights = cfg.early_weights;
   const BsWsLayout L = bs_ws_layout(d, m, cfg);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.counters = reinterpret_cast<int32_t*>(wsb + L.counters);

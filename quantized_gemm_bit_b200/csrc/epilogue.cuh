@@ -53,4 +53,57 @@ __device__ __forceinline__ void store_rows_chunk(__nv_bfloat16* c, int n_total, 
   }
 }
 
+// SwiGLU epilogue of a gate+up GEMM whose weights were packed in the gated
+// row order: in every 32-row quarter of a 128-row weight tile, lanes 0-15
+// hold 16 gate features and lanes 16-31 the up features of the same 16
+// indices.  Lane l holds v[j] for tokens j0 .. j0+EB-1 of its row; lanes l
+// and l ^ 16 swap values, so each has gate g and up u of feature
+// h_col0 + (l & 15); lane l < 16 computes tokens j0 .. j0+EB/2-1, lane
+// l >= 16 the rest: h = silu(g) * u, silu(x) = x / (1 + exp(-x)), fp32, one
+// bf16 rounding.  Stores as store_rows_chunk (16-byte rows of 8 features
+// through the transpose buffer `sc`, 16 x EB uint16; element by element
+// when sc is null or h_cols % 8 != 0).  Rows at or past `rows` are not
+// written.
+template <int EB>
+__device__ __forceinline__ void store_swiglu_chunk(__nv_bfloat16* h, int h_cols, int row0, int rows, int h_col0,
+                                                   int lane, int j0, const float (&v)[EB], uint16_t* sc) {
+  static_assert(EB % 8 == 0, "token runs of 8");
+  const bool up_lane = lane >= 16;
+  const int f = h_col0 + (lane & 15);
+  uint16_t hv[EB / 2];
+#pragma unroll
+  for (int j = 0; j < EB / 2; ++j) {
+    // the gate lane sends its value of token j + EB/2 and receives the up
+    // value of token j; the up lane sends token j and receives the gate
+    // value of token j + EB/2
+    const float mine = up_lane ? v[j + EB / 2] : v[j];
+    const float recv = __shfl_xor_sync(0xffffffffu, up_lane ? v[j] : v[j + EB / 2], 16);
+    const float g = up_lane ? recv : mine;
+    const float u = up_lane ? mine : recv;
+    hv[j] = __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.f + expf(-g)) * u));
+  }
+  const int jbase = up_lane ? EB / 2 : 0;
+  if (sc != nullptr && (h_cols % 8) == 0) {
+#pragma unroll
+    for (int j = 0; j < EB / 2; ++j) sc[(jbase + j) * 16 + (lane & 15)] = hv[j];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < EB / 16; ++i) {
+      const int jj = (lane >> 1) + 16 * i;   // token of this lane's 16-byte piece
+      const int half = lane & 1;             // features 0-7 or 8-15 of the warp's 16
+      const int col = h_col0 + half * 8;
+      if (j0 + jj < rows && col < h_cols) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sc + jj * 16 + half * 8);
+        *reinterpret_cast<uint4*>(h + (size_t)(row0 + j0 + jj) * h_cols + col) = w;
+      }
+    }
+    __syncwarp();
+  } else if (f < h_cols) {
+#pragma unroll
+    for (int j = 0; j < EB / 2; ++j) {
+      if (j0 + jbase + j < rows) h[(size_t)(row0 + j0 + jbase + j) * h_cols + f] = __ushort_as_bfloat16(hv[j]);
+    }
+  }
+}
+
 }  // namespace hq

@@ -76,8 +76,13 @@ hq_status check_desc(const hq_quant_desc* d) {
       if (d->group_size != 32 || d->k % 128 != 0 || d->has_zero_point || d->num_experts > 1024)
         return HQ_ERR_UNSUPPORTED;
       return HQ_OK;
+    case HQ_FMT_MXINT4:
+      if (d->group_size != 32 || d->k % 128 != 0 || d->has_zero_point || d->num_experts > 1024)
+        return HQ_ERR_UNSUPPORTED;
+      return HQ_OK;
     case HQ_FMT_INT3:
     case HQ_FMT_INT2:
+    case HQ_FMT_INT8:
       if (d->group_size != 128 || d->k % 128 != 0) return HQ_ERR_UNSUPPORTED;
       if (d->has_zero_point != 0 && d->has_zero_point != 1) return HQ_ERR_INVALID_ARG;
       if (d->num_experts > 1024) return HQ_ERR_UNSUPPORTED;
@@ -89,7 +94,8 @@ hq_status check_desc(const hq_quant_desc* d) {
 
 // Formats the W4A16 kernels read (dequantized in registers, bf16 MMA).
 bool w4_format(const hq_quant_desc* d) {
-  return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_INT2 || d->fmt == HQ_FMT_MXFP4_A16;
+  return d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_INT2 || d->fmt == HQ_FMT_INT8 ||
+         d->fmt == HQ_FMT_MXFP4_A16 || d->fmt == HQ_FMT_MXINT4;
 }
 
 // Tuning checks shared by the W4A16 entry points (dense: split_k free;
@@ -99,12 +105,13 @@ hq_status check_w4_tuning(const hq_quant_desc* d, const hq_tuning* t, bool group
   if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
     return HQ_ERR_UNSUPPORTED;
   if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
-      (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2)
+      (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2 ||
+      (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
     return HQ_ERR_UNSUPPORTED;
   if (grouped && t->split_k > 1) return HQ_ERR_UNSUPPORTED;
-  // the exact-weight kernel reads INT4 records only (and MXFP4's scale per
-  // 32 K leaves no 128-K group scale to factor out)
-  if (d->fmt != HQ_FMT_INT4 && t->variant == 2) return HQ_ERR_UNSUPPORTED;
+  // the exact-weight kernel factors a 128-K group scale out of the sum:
+  // the MX formats' scale per 32 K leaves none
+  if ((d->fmt == HQ_FMT_MXFP4_A16 || d->fmt == HQ_FMT_MXINT4) && t->variant == 2) return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
 
@@ -121,6 +128,8 @@ hq_status check_w4_call(const hq_quant_desc* d, const hq_tuning* t, bool grouped
 size_t packed_size_impl(const hq_quant_desc& d);
 hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scales, const void* zeros, float g,
                     void* out);
+hq_status pack_gated_impl(const hq_quant_desc& d, const void* codes, const void* scales, const void* zeros,
+                          void* out);
 
 }  // namespace hq
 
@@ -173,13 +182,26 @@ hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const 
   hq_status st = check_desc(d);
   if (st != HQ_OK) return st;
   if (!codes_host || !scales_host || !out_host) return HQ_ERR_INVALID_ARG;
-  if (d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_INT2) {
+  if (d->fmt == HQ_FMT_INT4 || d->fmt == HQ_FMT_INT3 || d->fmt == HQ_FMT_INT2 || d->fmt == HQ_FMT_INT8) {
     if ((d->has_zero_point != 0) != (zeros_host != nullptr)) return HQ_ERR_INVALID_ARG;
   } else if (zeros_host) {
     return HQ_ERR_INVALID_ARG;
   }
   if (out_bytes < packed_size_impl(*d)) return HQ_ERR_WORKSPACE_TOO_SMALL;
   return pack_impl(*d, codes_host, scales_host, zeros_host, global_scale, out_host);
+}
+
+hq_status hq_pack_weights_gated(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
+                                const void* zeros_host, void* out_host, size_t out_bytes) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (!w4_format(d) || d->n % 128 != 0) return HQ_ERR_UNSUPPORTED;
+  if (!codes_host || !scales_host || !out_host) return HQ_ERR_INVALID_ARG;
+  if ((d->fmt == HQ_FMT_MXFP4_A16 || d->fmt == HQ_FMT_MXINT4) ? zeros_host != nullptr
+                                                               : (d->has_zero_point != 0) != (zeros_host != nullptr))
+    return HQ_ERR_INVALID_ARG;
+  if (out_bytes < packed_size_impl(*d)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return pack_gated_impl(*d, codes_host, scales_host, zeros_host, out_host);
 }
 
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t) {
@@ -242,13 +264,37 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
+hq_status hq_grouped_gemm_moe_swiglu(const hq_quant_desc* d, const void* packed_w_dev, const void* a_sorted_dev,
+                                     const int32_t* expert_offsets_dev, int32_t total_rows, void* h_sorted_dev,
+                                     const hq_tuning* t, void* ws_dev, size_t ws_bytes, hq_stream_t stream) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (!w4_format(d) || d->num_experts < 2) return HQ_ERR_INVALID_ARG;
+  if (d->n % 128 != 0) return HQ_ERR_UNSUPPORTED;
+  if (total_rows < 0) return HQ_ERR_INVALID_ARG;
+  if (total_rows == 0) return HQ_OK;
+  if (!packed_w_dev || !a_sorted_dev || !expert_offsets_dev || !h_sorted_dev || !ws_dev) return HQ_ERR_INVALID_ARG;
+  if (!aligned(packed_w_dev, 16) || !aligned(a_sorted_dev, 16) || !aligned(h_sorted_dev, 16) ||
+      !aligned(expert_offsets_dev, 4) || !aligned(ws_dev, 256))
+    return HQ_ERR_ALIGNMENT;
+  st = check_w4_tuning(d, t, true);
+  if (st != HQ_OK) return st;
+  DeviceInfo dev{};
+  st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  W4Config cfg = w4_plan(dev, *d, total_rows, true, t);
+  if (ws_bytes < w4_workspace_bytes(*d, total_rows, cfg, true)) return HQ_ERR_WORKSPACE_TOO_SMALL;
+  return w4_launch(*d, cfg, packed_w_dev, a_sorted_dev, total_rows, h_sorted_dev, expert_offsets_dev, ws_dev,
+                   reinterpret_cast<cudaStream_t>(stream), 1);
+}
+
 namespace {
 hq_status check_bs_tuning(const hq_tuning* t) {
   if (!t) return HQ_OK;
   if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
     return HQ_ERR_UNSUPPORTED;
   if ((t->tile_n && t->tile_n != 128) || t->tile_k || t->split_k < 0 || t->stages != 0 ||
-      (t->cta_group && t->cta_group != 1) || t->variant != 0)
+      (t->cta_group && t->cta_group != 1) || t->variant != 0 || (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
     return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }

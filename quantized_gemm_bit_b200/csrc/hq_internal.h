@@ -30,6 +30,12 @@ inline int w3_record_bytes(bool has_zero) { return kW3RecCodes + 256 + (has_zero
 // INT2 weights: 4096 code bytes, then scales and zero points as for INT4
 constexpr int kW2RecCodes = 4096;
 inline int w2_record_bytes(bool has_zero) { return kW2RecCodes + 256 + (has_zero ? 128 : 0); }
+// INT8 weights: 16384 code bytes, then scales and zero points as for INT4
+constexpr int kW8RecCodes = 16384;
+inline int w8_record_bytes(bool has_zero) { return kW8RecCodes + 256 + (has_zero ? 128 : 0); }
+// MXINT4 weights: 8192 code bytes (the INT4 nibble layout), then one E8M0
+// byte per (row, 32-K block) as for MXFP4_A16
+constexpr int kMxi4RecBytes = kW4RecCodes + 512;
 
 constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -40,8 +46,9 @@ struct W4Config {
   int splits;   // 0: data parallel (whole tiles); else stream-K / split K
   int dp_tiles; // stream-K plans: tiles run whole before the shared K range
   int grid;     // CTAs
-  int variant;  // 0: library's choice (exact weights for 64-token tiles,
-                // bf16-rescaled otherwise); 1: bf16-rescaled weights for
+  int early_weights;  // fetch packed weights before the previous kernel completes
+  int variant;  // 0: library's choice (exact weights for tiles of <= 64
+                // tokens, bf16-rescaled above); 1: bf16-rescaled weights for
                 // every tile; 2: exact (q - z) weights + per-group fp32
                 // scaling for tiles of <= 64 tokens (bf16-rescaled above)
 };
@@ -54,8 +61,8 @@ struct DeviceInfo {
 };
 hq_status device_info(DeviceInfo* out);
 
-// Descriptor, format and tuning checks of a W4A16-family call (INT4 or
-// MXFP4_A16 weights; grouped: num_experts >= 2, else exactly 1).
+// Descriptor, format and tuning checks of a W4A16-family call (INT4, INT3,
+// INT2 or MXFP4_A16 weights; grouped: num_experts >= 2, else exactly 1).
 hq_status check_w4_call(const hq_quant_desc* d, const hq_tuning* t, bool grouped);
 
 // W4A16 (dense or grouped) planning and launch.
@@ -64,14 +71,17 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
 // beyond the header).
 W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4Config cfg);
 size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bool grouped);
+// swiglu: grouped only, weights packed in the gated gate+up row order; c
+// receives h = silu(gate) * up, [m][d.n / 2].
 hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m,
-                    void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream);
+                    void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream, int swiglu = 0);
 
 // Block-scaled 4-bit GEMMs (MXFP4 weights x E4M3 activations; NVFP4 x NVFP4).
 struct BsConfig {
   int ntok;
   int splits;   // 0: whole tiles per CTA (no partial sums)
   int grid;
+  int early_weights;  // fetch packed weights before the previous kernel completes
 };
 BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t);
 size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg);

@@ -304,6 +304,82 @@ hq_status pack_mx_a16(const hq_quant_desc& d, const uint8_t* codes, const uint8_
   return HQ_OK;
 }
 
+// INT8 (group 128): row r's 16-K chunk c of a record is its 16 code bytes
+// at (c*128 + r)*16, in K order; scales and zero points as for INT4.
+hq_status pack_int8(const hq_quant_desc& d, const int32_t* codes, const uint16_t* scales, const uint8_t* zeros,
+                    uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int nt_count = (n + kTileN - 1) / kTileN;
+  const int kb_count = k / kBlockK;
+  const bool hz = zeros != nullptr;
+  const size_t rec = (size_t)w8_record_bytes(hz);
+  const size_t expert_bytes = (size_t)nt_count * kb_count * rec;
+  const size_t row_bytes = (size_t)k;   // canonical: four codes per int32, low byte first
+  const size_t kg = (size_t)k / 128;
+  const size_t jobs = (size_t)d.num_experts * nt_count;
+  parallel_for(jobs, [&](size_t job) {
+    const size_t e = job / nt_count;
+    const int nt = (int)(job % nt_count);
+    uint8_t* ebase = out + e * expert_bytes;
+    const uint8_t* cb = reinterpret_cast<const uint8_t*>(codes);
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint8_t* r0 = ebase + ((size_t)nt * kb_count + kb) * rec;
+      std::memset(r0, 0, rec);
+      for (int r = 0; r < kTileN; ++r) {
+        const int row = nt * kTileN + r;
+        if (row >= n) break;
+        // little-endian words: code k is byte k of the row
+        const uint8_t* src = cb + (e * n + row) * row_bytes + (size_t)kb * 128;
+        for (int c = 0; c < 8; ++c) std::memcpy(r0 + ((size_t)c * 128 + r) * 16, src + 16 * c, 16);
+        const uint16_t s = scales[(e * n + row) * kg + kb];
+        std::memcpy(r0 + kW8RecCodes + 2 * r, &s, 2);
+        if (hz) r0[kW8RecCodes + 256 + r] = zeros[(e * n + row) * kg + kb];
+      }
+    }
+  });
+  return HQ_OK;
+}
+
+// MXINT4 (E8M0 scale per 32 K): the INT4 nibble layout of the codes, the
+// MXFP4_A16 placement of the scales.
+hq_status pack_mxi4(const hq_quant_desc& d, const uint8_t* codes, const uint8_t* scales, uint8_t* out) {
+  const int n = d.n, k = d.k;
+  const int nt_count = (n + kTileN - 1) / kTileN;
+  const int kb_count = k / kBlockK;
+  const size_t rec = (size_t)kMxi4RecBytes;
+  const size_t expert_bytes = (size_t)nt_count * kb_count * rec;
+  const size_t row_bytes = (size_t)k / 2, row_scales = (size_t)k / 32;
+  // scales above 2^124 would make bf16 weights of magnitude 8 overflow
+  const size_t total_scales = (size_t)d.num_experts * n * row_scales;
+  for (size_t i = 0; i < total_scales; ++i)
+    if (scales[i] > 251) return HQ_ERR_INVALID_ARG;
+  const size_t jobs = (size_t)d.num_experts * nt_count;
+  parallel_for(jobs, [&](size_t job) {
+    const size_t e = job / nt_count;
+    const int nt = (int)(job % nt_count);
+    uint8_t* ebase = out + e * expert_bytes;
+    for (int kb = 0; kb < kb_count; ++kb) {
+      uint8_t* r0 = ebase + ((size_t)nt * kb_count + kb) * rec;
+      std::memset(r0, 0, rec);
+      for (int r = 0; r < kTileN; ++r) {
+        const int row = nt * kTileN + r;
+        if (row >= n) break;
+        const uint8_t* src = codes + (e * n + row) * row_bytes + (size_t)kb * 64;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(r0 + ((size_t)c * 128 + r) * 16);
+          for (int w = 0; w < 4; ++w) {
+            uint32_t word;   // eight codes, even k in the low nibble of each byte: the canonical INT4 word
+            std::memcpy(&word, src + 16 * c + 4 * w, 4);
+            dst[w] = permute_word(word);
+          }
+          r0[kW4RecCodes + 4 * r + c] = scales[(e * n + row) * row_scales + (size_t)kb * 4 + c];
+        }
+      }
+    }
+  });
+  return HQ_OK;
+}
+
 // Block-scaled formats: copy codes row by row, then lay out scale blocks.
 hq_status pack_fp4(const hq_quant_desc& d, const uint8_t* codes, const uint8_t* scales, float g, uint8_t* out) {
   const int n = d.n, k = d.k;
@@ -353,6 +429,10 @@ size_t packed_size_impl(const hq_quant_desc& d) {
       return (size_t)d.num_experts * nt * (d.k / kBlockK) * w3_record_bytes(d.has_zero_point != 0);
     case HQ_FMT_INT2:
       return (size_t)d.num_experts * nt * (d.k / kBlockK) * w2_record_bytes(d.has_zero_point != 0);
+    case HQ_FMT_INT8:
+      return (size_t)d.num_experts * nt * (d.k / kBlockK) * w8_record_bytes(d.has_zero_point != 0);
+    case HQ_FMT_MXINT4:
+      return (size_t)d.num_experts * nt * (d.k / kBlockK) * kMxi4RecBytes;
     default:
       return 0;
   }
@@ -377,9 +457,62 @@ hq_status pack_impl(const hq_quant_desc& d, const void* codes, const void* scale
     case HQ_FMT_INT2:
       return pack_int2(d, static_cast<const int32_t*>(codes), static_cast<const uint16_t*>(scales),
                        static_cast<const uint8_t*>(zeros), static_cast<uint8_t*>(out));
+    case HQ_FMT_INT8:
+      return pack_int8(d, static_cast<const int32_t*>(codes), static_cast<const uint16_t*>(scales),
+                       static_cast<const uint8_t*>(zeros), static_cast<uint8_t*>(out));
+    case HQ_FMT_MXINT4:
+      return pack_mxi4(d, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(scales),
+                       static_cast<uint8_t*>(out));
     default:
       return HQ_ERR_INVALID_ARG;
   }
+}
+
+// Canonical bytes per weight row of the W4A16-family formats: codes, scales
+// and zero points (0 for formats without them).
+struct RowBytes {
+  size_t codes, scales, zeros;
+};
+static bool w16_row_bytes(const hq_quant_desc& d, RowBytes* rb) {
+  const size_t k = (size_t)d.k;
+  switch (d.fmt) {
+    case HQ_FMT_INT4: *rb = {k / 2, 2 * (k / 128), k / 128}; return true;
+    case HQ_FMT_INT3: *rb = {3 * k / 8, 2 * (k / 128), k / 128}; return true;
+    case HQ_FMT_INT2: *rb = {k / 4, 2 * (k / 128), k / 128}; return true;
+    case HQ_FMT_MXFP4_A16: *rb = {k / 2, k / 32, 0}; return true;
+    case HQ_FMT_INT8: *rb = {k, 2 * (k / 128), k / 128}; return true;
+    case HQ_FMT_MXINT4: *rb = {k / 2, k / 32, 0}; return true;
+    default: return false;
+  }
+}
+
+// Canonical row of packed row p in the gated gate+up order (n = 2I rows,
+// gate rows [0, I), up rows [I, 2I)): in every 32-row quarter q of tile j,
+// rows 0-15 are gate rows 64j + 16q + l and rows 16-31 the up rows of the
+// same indices, I + 64j + 16q + (l - 16).
+static int gated_source_row(int p, int n) {
+  const int j = p / 128, r = p % 128, q = r / 32, l = r % 32;
+  return l < 16 ? 64 * j + 16 * q + l : n / 2 + 64 * j + 16 * q + (l - 16);
+}
+
+hq_status pack_gated_impl(const hq_quant_desc& d, const void* codes, const void* scales, const void* zeros,
+                          void* out) {
+  RowBytes rb{};
+  if (!w16_row_bytes(d, &rb) || d.n % 128 != 0) return HQ_ERR_UNSUPPORTED;
+  const size_t rows = (size_t)d.num_experts * d.n;
+  std::vector<uint8_t> c2(rows * rb.codes), s2(rows * rb.scales), z2(zeros ? rows * rb.zeros : 0);
+  const uint8_t* c = static_cast<const uint8_t*>(codes);
+  const uint8_t* sc = static_cast<const uint8_t*>(scales);
+  const uint8_t* z = static_cast<const uint8_t*>(zeros);
+  for (size_t e = 0; e < (size_t)d.num_experts; ++e) {
+    for (int p = 0; p < d.n; ++p) {
+      const size_t dst = e * d.n + p, src = e * d.n + gated_source_row(p, d.n);
+      std::memcpy(&c2[dst * rb.codes], c + src * rb.codes, rb.codes);
+      std::memcpy(&s2[dst * rb.scales], sc + src * rb.scales, rb.scales);
+      if (z) std::memcpy(&z2[dst * rb.zeros], z + src * rb.zeros, rb.zeros);
+    }
+  }
+  return pack_impl(d, c2.data(), s2.data(), z ? z2.data() : nullptr, 0.f, out);
 }
 
 }  // namespace hq

@@ -45,11 +45,6 @@ namespace {
 
 constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 
-// Weight formats of the kernel: INT4 records, MXFP4 records (8704 bytes; a
-// tighter barrier area keeps the 256-token tile inside the shared-memory
-// limit), INT3 records (at most 6528 bytes) and INT2 records (at most 4480).
-constexpr int kFmtInt4 = 0, kFmtMx = 1, kFmtInt3 = 2, kFmtInt2 = 3;
-
 template <int NTOK, int FMT = kFmtInt4>
 struct Cfg {
   // records (128-K blocks) per pipeline stage: two for the small token tiles,
@@ -57,12 +52,20 @@ struct Cfg {
   static constexpr int kKps = NTOK <= 64 ? 2 : 1;
   static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
-  static constexpr int kRecStride = FMT == kFmtMx     ? kMxA16RecBytes
-                                    : FMT == kFmtInt3 ? kW3RecCodes + 384
-                                    : FMT == kFmtInt2 ? kW2RecCodes + 384
-                                                      : kRecMax;
+  static constexpr int kRecStride = (FMT == kFmtMx || FMT == kFmtMxi4) ? kMxA16RecBytes
+                                    : FMT == kFmtInt3                  ? kW3RecCodes + 384
+                                    : FMT == kFmtInt2                  ? kW2RecCodes + 384
+                                    : FMT == kFmtInt8                  ? kW8RecCodes + 384
+                                                                       : kRecMax;
   static constexpr int kRecs = kKps * kRecStride;
-  static constexpr int kSmemStages = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  static constexpr int kBarBytes = (FMT == kFmtMx || FMT == kFmtMxi4) ? 384 : 512;
+  static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
+  // as many SMEM stages as fit, up to a preferred depth per token tile
+  static constexpr int kSmemPref = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  static constexpr int kSmemFit =
+      (int)((232448 - 1024 - kBarBytes - 2 * (kMaxExperts + 1) * sizeof(int) - 128 - kEpiScratch) /
+            (kATile + kRecs));
+  static constexpr int kSmemStages = kSmemPref < kSmemFit ? kSmemPref : kSmemFit;
   static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;
   // Dequantizing warpgroups own alternate stages (the epilogue warpgroup
@@ -75,11 +78,9 @@ struct Cfg {
   // barrier's phases in order whatever the ring depth
   static constexpr int kFullBars = kSmemStages * kDqGroups;
   static constexpr int kFullPeriod = kSmemStages / cgcd(kSmemStages, kDqGroups) * kDqGroups;  // lcm
-  // warp-local transpose buffer for 16-byte output stores; at 256 tokens
-  // it aliases the expert tables, so grouped 256-token tiles store their
-  // outputs element by element instead
-  static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
-  static constexpr int kBarBytes = FMT == kFmtMx ? 384 : 512;
+  // (kEpiScratch: the warp-local transpose buffer for 16-byte output
+  // stores; at 256 tokens it aliases the expert tables, so grouped 256-token
+  // tiles store their outputs element by element instead)
   // byte offsets from the 1024-aligned base of dynamic shared memory
   static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
   static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
@@ -88,38 +89,55 @@ struct Cfg {
   static_assert(kABlock % 1024 == 0 && kRecStride % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
   static_assert(kEpiScratch != 0 || 2 * (kMaxExperts + 1) * sizeof(int) >= 4 * 2048, "aliased scratch size");
   static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kSmemStages >= 2, "pipeline depth");
   static_assert(64 * kKps * kTmemStages + kAccBufs * NTOK <= 512, "TMEM budget");
   static_assert(kTmemStages % kDqGroups == 0, "every TMEM stage must always return to the same dequant group");
   static_assert(8 * (kFullBars + kSmemStages + 2 * kTmemStages + 5) + 16 <= kBarBytes, "barrier area");
 };
 
 // Weight row r of one 128-K packed record: its scale and zero point as
-// bf16x2 pairs (s2 = bf16(s) twice, z2 = bf16(128 + z) twice; 128 + z is
-// exact in bf16).
+// bf16x2 pairs.  The fp16 scale s is split exactly into s_hi = bf16(s) and
+// s_lo = s - s_hi (at most three significant bits, so bf16 holds it), and
+// z2 = bf16(128 + z) twice (exact).
 struct RowQ {
-  uint32_t s2, z2;
+  uint32_t shi2, slo2, z2;
 };
-__device__ __forceinline__ RowQ row_qparams(const uint8_t* rec, int r, int has_zero) {
-  const __half sc = reinterpret_cast<const __half*>(rec + kW4RecCodes)[r];
-  const uint32_t z = has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
-  const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
+template <int CODE_BYTES, uint32_t ZSYM>
+__device__ __forceinline__ RowQ row_qparams_t(const uint8_t* rec, int r, int has_zero) {
+  const float s = __half2float(reinterpret_cast<const __half*>(rec + CODE_BYTES)[r]);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(s);
+  const uint32_t hbits = (uint32_t)__bfloat16_as_ushort(hi);
+  // s - s_hi is exact in fp32 and a bf16 number: no rounding here
+  const uint32_t lbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(s - __bfloat162float(hi)));
+  const uint32_t z = has_zero ? rec[CODE_BYTES + 256 + r] : ZSYM;
   const uint32_t zbits = 0x4300u + z;
-  return RowQ{sbits | (sbits << 16), zbits | (zbits << 16)};
+  return RowQ{hbits | (hbits << 16), lbits | (lbits << 16), zbits | (zbits << 16)};
+}
+__device__ __forceinline__ RowQ row_qparams(const uint8_t* rec, int r, int has_zero) {
+  return row_qparams_t<kW4RecCodes, 8u>(rec, r, has_zero);
+}
+
+// bf16x2 pair of bf16(128 + q) -> the weights (q - z) * s, each rounded to
+// bf16 once: d = q - z is exact, d * s_lo is exact (at most 4 + 3
+// significant bits), and the fused multiply-add rounds d * s_hi + d * s_lo
+// = d * s a single time.
+__device__ __forceinline__ uint32_t rescale(uint32_t x2, const RowQ& qp) {
+  const uint32_t d = bf16x2_sub(x2, qp.z2);
+  return bf16x2_fma(d, qp.shi2, bf16x2_mul(d, qp.slo2));
 }
 
 // One 32-K chunk of row r (16 bytes of codes) -> its weights w = (q - z) * s
 // as 16 words, two bf16 per 32-bit word (even k in the low half).
-__device__ __forceinline__ void dequant_chunk(const uint4& raw, RowQ qp, uint32_t* out) {
+__device__ __forceinline__ void dequant_chunk(const uint4& raw, const RowQ& qp, uint32_t* out) {
   const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       // nibbles of k = 2j and 2j+1 sit at bits 4j and 16+4j: OR-ing them
-      // into the mantissa of bf16 128.0 gives bf16(128 + q); then
-      // (128 + q) - (128 + z) = q - z exactly, and one rounding in the product
+      // into the mantissa of bf16 128.0 gives bf16(128 + q)
       const uint32_t x2 = lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u);
-      out[w * 4 + j] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+      out[w * 4 + j] = rescale(x2, qp);
     }
   }
 }
@@ -204,27 +222,18 @@ __device__ __forceinline__ void mx_dequant_block(const uint8_t* rec, int r, uint
 }
 
 // ---- INT3 weights (3-bit codes, fp16 scale and uint3 zero point per 128 K)
-__device__ __forceinline__ RowQ row_qparams3(const uint8_t* rec, int r, int has_zero) {
-  const __half sc = reinterpret_cast<const __half*>(rec + kW3RecCodes)[r];
-  const uint32_t z = has_zero ? rec[kW3RecCodes + 256 + r] : 4u;
-  const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
-  const uint32_t zbits = 0x4300u + z;
-  return RowQ{sbits | (sbits << 16), zbits | (zbits << 16)};
-}
-
 // A whole 128-K INT3 record for weight row r (as dequant_block): the row's
 // 12 code words come in three 16-byte loads.  In each 32-K chunk (words
 // 3c .. 3c+2) pairs 0-14 sit at bits 3j / 16 + 3j of their word, so one
 // shift and one LOP3 give bf16 (128 + q, 128 + q'); pair 15 gathers code
-// bit p from bits 15 / 31 of word p.  Then w = ((128 + q) - (128 + z)) * s
-// as for INT4.
+// bit p from bits 15 / 31 of word p.  Then w = (q - z) * s as for INT4.
 __device__ __forceinline__ void w3_dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
   uint4 raw[3];
 #pragma unroll
   for (int i = 0; i < 3; ++i) raw[i] = *reinterpret_cast<const uint4*>(rec + (i * 128 + r) * 16);
   const uint32_t wv[12] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y,
                            raw[1].z, raw[1].w, raw[2].x, raw[2].y, raw[2].z, raw[2].w};
-  const RowQ qp = row_qparams3(rec, r, has_zero);
+  const RowQ qp = row_qparams_t<kW3RecCodes, 4u>(rec, r, has_zero);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint32_t out[16];
@@ -233,36 +242,28 @@ __device__ __forceinline__ void w3_dequant_block(const uint8_t* rec, int r, int 
 #pragma unroll
       for (int j = 0; j < 5; ++j) {
         const uint32_t x2 = lop3_and_or(wv[3 * c + p] >> (3 * j), 0x00070007u, 0x43004300u);
-        out[5 * p + j] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+        out[5 * p + j] = rescale(x2, qp);
       }
     }
     uint32_t x2 = lop3_and_or(wv[3 * c] >> 15, 0x00010001u, 0x43004300u);
     x2 = lop3_and_or(wv[3 * c + 1] >> 14, 0x00020002u, x2);
     x2 = lop3_and_or(wv[3 * c + 2] >> 13, 0x00040004u, x2);
-    out[15] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+    out[15] = rescale(x2, qp);
     tmem_st_x16(taddr + c * 16, out);
   }
 }
 
 // ---- INT2 weights (2-bit codes, fp16 scale and uint2 zero point per 128 K)
-__device__ __forceinline__ RowQ row_qparams2(const uint8_t* rec, int r, int has_zero) {
-  const __half sc = reinterpret_cast<const __half*>(rec + kW2RecCodes)[r];
-  const uint32_t z = has_zero ? rec[kW2RecCodes + 256 + r] : 2u;
-  const uint32_t sbits = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__half2float(sc)));
-  const uint32_t zbits = 0x4300u + z;
-  return RowQ{sbits | (sbits << 16), zbits | (zbits << 16)};
-}
-
 // A whole 128-K INT2 record for weight row r (as dequant_block): the row's
 // 8 code words come in two 16-byte loads; pair i of 32-K chunk c sits at
 // bits 2j / 16 + 2j (j = i % 8) of word 2c + i / 8, so one shift and one
-// LOP3 give bf16 (128 + q, 128 + q'), then w = ((128 + q) - (128 + z)) * s.
+// LOP3 give bf16 (128 + q, 128 + q'), then w = (q - z) * s as for INT4.
 __device__ __forceinline__ void w2_dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
   uint4 raw[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) raw[i] = *reinterpret_cast<const uint4*>(rec + (i * 128 + r) * 16);
   const uint32_t wv[8] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w, raw[1].x, raw[1].y, raw[1].z, raw[1].w};
-  const RowQ qp = row_qparams2(rec, r, has_zero);
+  const RowQ qp = row_qparams_t<kW2RecCodes, 2u>(rec, r, has_zero);
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     uint32_t out[16];
@@ -271,7 +272,61 @@ __device__ __forceinline__ void w2_dequant_block(const uint8_t* rec, int r, int 
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const uint32_t x2 = lop3_and_or(wv[2 * c + p] >> (2 * j), 0x00030003u, 0x43004300u);
-        out[8 * p + j] = bf16x2_mul(bf16x2_sub(x2, qp.z2), qp.s2);
+        out[8 * p + j] = rescale(x2, qp);
+      }
+    }
+    tmem_st_x16(taddr + c * 16, out);
+  }
+}
+
+// ---- INT8 weights (8-bit codes, fp16 scale and uint8 zero point per 128 K)
+// A whole 128-K INT8 record for weight row r (as dequant_block): eight
+// 16-byte chunks of 16 codes; each code becomes q - z exactly in fp32, the
+// product with the fp16 scale is exact in fp32 (8 + 11 significant bits),
+// and the one rounding is the conversion to bf16.
+__device__ __forceinline__ void w8_dequant_block(const uint8_t* rec, int r, int has_zero, uint32_t taddr) {
+  const float s = __half2float(reinterpret_cast<const __half*>(rec + kW8RecCodes)[r]);
+  const float zf = 8388608.f + (float)(has_zero ? rec[kW8RecCodes + 256 + r] : 128u);
+#pragma unroll
+  for (int c2 = 0; c2 < 4; ++c2) {
+    uint32_t out[16];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(rec + ((2 * c2 + h) * 128 + r) * 16);
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        out[8 * h + 2 * w] = pack_bf16x2(u8_minus_zero(wv[w], 0, zf) * s, u8_minus_zero(wv[w], 1, zf) * s);
+        out[8 * h + 2 * w + 1] = pack_bf16x2(u8_minus_zero(wv[w], 2, zf) * s, u8_minus_zero(wv[w], 3, zf) * s);
+      }
+    }
+    tmem_st_x16(taddr + c2 * 16, out);
+  }
+}
+
+// ---- MXINT4 weights (two's-complement 4-bit codes, E8M0 scale per 32 K)
+// The INT4 nibble placement: flipping bit 3 of a code (the LOP3 XOR) maps
+// the integer c in -8..7 to c + 8, so the bf16 pair is (136 + c, 136 + c');
+// subtracting 136 and multiplying by 2^(e - 127) are exact (scale bytes
+// <= 251 keep every weight finite; 2^-127 is the bf16 subnormal 0x0040).
+__device__ __forceinline__ void mxi4_dequant_block(const uint8_t* rec, int r, uint32_t taddr) {
+  uint4 raw[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+  const uint32_t e4 = *reinterpret_cast<const uint32_t*>(rec + kW4RecCodes + 4 * r);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t e = (e4 >> (8 * c)) & 0xFFu;
+    const uint32_t sbits = e ? e << 7 : 0x40u;
+    const uint32_t s2 = sbits | (sbits << 16);
+    const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+    uint32_t out[16];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t x2 = lop3_and_xor(wv[w] >> (4 * j), 0x000F000Fu, 0x43084308u);
+        out[w * 4 + j] = bf16x2_mul(bf16x2_sub(x2, 0x43084308u), s2);
       }
     }
     tmem_st_x16(taddr + c * 16, out);
@@ -354,7 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // of the first SS stages (no kernel writes them)
     uint32_t n_pre = 0;
     if (!p.grouped) {
-      for (int idx = 0; n_pre < (uint32_t)SS && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      for (int idx = 0; p.early_weights && n_pre < (uint32_t)SS &&
+                        get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
+           ++idx) {
         const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
         for (int kb = x.kb0; kb < x.kb1 && n_pre < (uint32_t)SS; kb += KPS, ++n_pre) {
           const int nrec = min(KPS, x.kb1 - kb);
@@ -516,6 +573,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int rr = 0; rr < nrec; ++rr) {
           if constexpr (FMT == kFmtMx)
             mx_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, tbase + rr * 64);
+          else if constexpr (FMT == kFmtMxi4)
+            mxi4_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, tbase + rr * 64);
+          else if constexpr (FMT == kFmtInt8)
+            w8_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
           else if constexpr (FMT == kFmtInt3)
             w3_dequant_block(sR + s * kRecs + rr * p.rec_bytes, r, p.has_zero, tbase + rr * 64);
           else if constexpr (FMT == kFmtInt2)
@@ -611,6 +672,7 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   cfg.stages = 0;
   cfg.splits = 1;
   cfg.variant = t ? t->variant : 0;
+  cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
   if (grouped) {
     cfg.ntok = ntok;
     cfg.grid = dev.num_sms;
@@ -693,7 +755,7 @@ size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bo
 }
 
 hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m,
-                    void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream) {
+                    void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream, int swiglu) {
   const bool grouped = expert_offsets != nullptr;
   W4Params p{};
   p.packed = static_cast<const uint8_t*>(packed);
@@ -701,12 +763,16 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.expert_offsets = expert_offsets;
   p.err = static_cast<uint32_t*>(ws);
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16;
+  const bool mxi4 = d.fmt == HQ_FMT_MXINT4;
   const bool int3 = d.fmt == HQ_FMT_INT3;
   const bool int2 = d.fmt == HQ_FMT_INT2;
+  const bool int8 = d.fmt == HQ_FMT_INT8;
   p.has_zero = d.has_zero_point ? 1 : 0;
   p.rec_bytes = mx     ? kMxA16RecBytes
+                : mxi4 ? kMxi4RecBytes
                 : int3 ? w3_record_bytes(p.has_zero)
                 : int2 ? w2_record_bytes(p.has_zero)
+                : int8 ? w8_record_bytes(p.has_zero)
                        : w4_record_bytes(p.has_zero);
   p.n_tiles = (d.n + kTileN - 1) / kTileN;
   p.k_blocks = d.k / kBlockK;
@@ -717,6 +783,8 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.num_experts = grouped ? d.num_experts : 1;
   p.grouped = grouped ? 1 : 0;
   p.wait_ns = kDefaultWaitNs;
+  p.early_weights = cfg.early_weights;
+  p.swiglu = swiglu;
   if (grouped) {
     // an expert's weight tile is re-read by each of its token tiles
     p.weights_once = (long long)m <= (long long)cfg.ntok * d.num_experts ? 1 : 0;
@@ -744,13 +812,29 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
 
-  // The exact-weight kernel: on request for tiles of up to 64 tokens, and as
-  // the library's choice for 64-token tiles, where it measured faster
-  // (dense M=64: 26.3 vs 28.4 us at K=7168, N=18432; grouped 64-token tiles
-  // up to 13 % faster); the bf16-rescaled kernel everywhere else.
-  // (MXFP4, INT3 and INT2 weights: always the rescaled kernel.)
-  const bool exact = d.fmt == HQ_FMT_INT4 && cfg.ntok <= 64 && (cfg.variant == 2 || (cfg.variant == 0 && cfg.ntok == 64));
-  if (exact) return small_launch(cfg.ntok, map, p, cfg.grid, stream);
+  // The exact-weight kernel for tiles of up to 64 tokens (INT4, INT3, INT2
+  // and INT8 weights): the library's choice there, and on request; the
+  // bf16-rescaled kernel for larger tiles, for the MX formats (exact in
+  // bf16 already) and on request (variant 1).
+  const int kfmt = int3 ? kFmtInt3 : int2 ? kFmtInt2 : int8 ? kFmtInt8 : kFmtInt4;
+  const bool exact = !mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1;
+  if (exact) return small_launch(cfg.ntok, kfmt, map, p, cfg.grid, stream);
+  auto by_tile = [&](auto f16, auto f32, auto f64, auto f128, auto f256) -> hq_status {
+    switch (cfg.ntok) {
+      case 16: return f16(map, p, cfg.grid, stream);
+      case 32: return f32(map, p, cfg.grid, stream);
+      case 64: return f64(map, p, cfg.grid, stream);
+      case 128: return f128(map, p, cfg.grid, stream);
+      case 256: return f256(map, p, cfg.grid, stream);
+      default: return HQ_ERR_UNSUPPORTED;
+    }
+  };
+  if (mxi4)
+    return by_tile(launch_t<16, kFmtMxi4>, launch_t<32, kFmtMxi4>, launch_t<64, kFmtMxi4>, launch_t<128, kFmtMxi4>,
+                   launch_t<256, kFmtMxi4>);
+  if (int8)
+    return by_tile(launch_t<16, kFmtInt8>, launch_t<32, kFmtInt8>, launch_t<64, kFmtInt8>, launch_t<128, kFmtInt8>,
+                   launch_t<256, kFmtInt8>);
   if (mx) {
     switch (cfg.ntok) {
       case 16: return launch_t<16, kFmtMx>(map, p, cfg.grid, stream);

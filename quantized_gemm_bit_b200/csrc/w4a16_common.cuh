@@ -24,6 +24,22 @@ constexpr int kThreads = 512;
 constexpr int kRecMax = 8576;        // packed record with zero points
 constexpr int kMaxExperts = 1024;
 
+// Weight formats of the W4A16 kernels: INT4 records, MXFP4 records (8704
+// bytes), INT3 records (at most 6528 bytes), INT2 records (at most 4480),
+// INT8 records (at most 16768) and MXINT4 records (8704).
+constexpr int kFmtInt4 = 0, kFmtMx = 1, kFmtInt3 = 2, kFmtInt2 = 3, kFmtInt8 = 4, kFmtMxi4 = 5;
+
+// INT8 codes to exact fp32: __byte_perm places code byte j of `w` under the
+// exponent of 2^23 (0x4B000000), giving 2^23 + q exactly; subtracting
+// zf = 2^23 + z leaves q - z exactly.
+__device__ __forceinline__ float u8_minus_zero(uint32_t w, int j, float zf) {
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)j)) - zf;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 struct W4Params {
   const uint8_t* packed;             // expert 0, record (0, 0)
   __nv_bfloat16* c;
@@ -44,6 +60,8 @@ struct W4Params {
   int grouped;
   int weights_once;                  // each weight tile is read by one CTA
   int data_parallel;                 // dense: whole tiles per unit, no partials
+  int early_weights;                 // dense: fetch the first stages' weights before griddepcontrol.wait
+  int swiglu;                        // grouped: gated gate+up weights, write h = silu(gate) * up [rows][n/2]
 };
 
 // One unit of work: a K range of one (expert, token tile, weight tile).
@@ -166,11 +184,16 @@ __device__ __forceinline__ void grouped_tables(const W4Params& p, int* s_off, in
 
 // Writes tokens j0 .. j0+EB-1 of one epilogue warp's 32 weight rows (row
 // n = nt*128 + 32q + lane holds v[j] for token j0+j): fp32 into this CTA's
-// partial slot for a partial unit, else bf16 output (store_rows_chunk).
+// partial slot for a partial unit, else bf16 output (store_rows_chunk); for
+// gated gate+up weights the SwiGLU of the warp's 16 gate/up row pairs, 16
+// features of h from feature nt*64 + 16q (store_swiglu_chunk).
 template <int EB>
 __device__ __forceinline__ void store_chunk(const W4Params& p, const Unit& x, float* part, int q, int lane, int j0,
                                             const float (&v)[EB], uint16_t* sc) {
-  store_rows_chunk<EB>(p.c, p.n, x.row0, x.rows, x.nt * kTileN + q * 32, q * 32 + lane, part, lane, j0, v, sc);
+  if (p.swiglu)
+    store_swiglu_chunk<EB>(p.c, p.n >> 1, x.row0, x.rows, x.nt * (kTileN / 2) + q * 16, lane, j0, v, sc);
+  else
+    store_rows_chunk<EB>(p.c, p.n, x.row0, x.rows, x.nt * kTileN + q * 32, q * 32 + lane, part, lane, j0, v, sc);
 }
 
 // Stream-K fixup after a partial unit's fp32 slot has been written: each
@@ -233,8 +256,9 @@ __device__ __noinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, i
   if (lane == 0) p.counters[x.tile * 4 + q] = 0;  // leave the workspace zeroed
 }
 
-// Host side: launch the small-token-tile kernel (16, 32 or 64 tokens).
-hq_status small_launch(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream);
+// Host side: launch the exact-weight kernel (16, 32 or 64 tokens; INT4,
+// INT3 or INT2 records).
+hq_status small_launch(int ntok, int fmt, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream);
 
 }  // namespace w4
 }  // namespace hq

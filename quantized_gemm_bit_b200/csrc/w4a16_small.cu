@@ -43,79 +43,157 @@ namespace w4 {
 
 namespace {
 
-template <int NTOK>
+constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
+
+template <int NTOK, int FMT>
 struct SmallCfg {
   static constexpr int kKps = 2;                        // records (groups) per stage
   static constexpr int kABlock = NTOK * 256;            // one record's activations: two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
-  static constexpr int kRecs = kKps * kRecMax;
-  static constexpr int kSmemStages = NTOK == 16 ? 8 : NTOK == 32 ? 6 : 4;
+  static constexpr int kCodeBytes = FMT == kFmtInt3   ? kW3RecCodes
+                                    : FMT == kFmtInt2 ? kW2RecCodes
+                                    : FMT == kFmtInt8 ? kW8RecCodes
+                                                      : kW4RecCodes;
+  static constexpr int kRecStride = kCodeBytes + 384;  // codes, fp16 scales, zero points
+  static constexpr int kRecs = kKps * kRecStride;
+  static constexpr uint32_t kZSym = FMT == kFmtInt3 ? 4u : FMT == kFmtInt2 ? 2u : FMT == kFmtInt8 ? 128u : 8u;
+  // Unpacking warps form kNdq groups of kGroupWarps; group g owns the
+  // stages it with it % kNdq == g, and its warps split each of its stages
+  // (4 row quarters x kGroupWarps / 4 parts of the stage's 32-K chunks).
+  // Groups owning whole stages keep several stages in flight with few
+  // synchronizations each (measured on B200 against every warp sharing
+  // every stage).
+  static constexpr int kNdq = NTOK == 64 ? 2 : 3;
+  static constexpr int kGroupWarps = 4;
+  static constexpr int kUnpackWarps = kNdq * kGroupWarps;
+  static constexpr int kChunks = 4 * kKps * 4 / kGroupWarps;   // 32-K chunks per unpacking warp and stage
+  static constexpr int kEpiScratch = 4 * 2048;          // warp-local transposes of the output
+  static constexpr int kBarBytes = 512;
+  // as many SMEM stages as fit, up to a preferred depth per token tile
+  static constexpr int kSmemPref = NTOK == 16 ? 8 : NTOK == 32 ? 6 : 4;
+  static constexpr int kSmemFit =
+      (int)((232448 - 1024 - kBarBytes - 2 * (kMaxExperts + 1) * sizeof(int) - 128 - kEpiScratch) /
+            (kATile + kRecs));
+  static constexpr int kSmemStages = kSmemPref < kSmemFit ? kSmemPref : kSmemFit;
   static constexpr int kAStages = NTOK == 64 ? 2 : 3;   // TMEM ring of unpacked weights
   static constexpr int kDStages = NTOK == 16 ? 4 : 2;   // TMEM ring of per-group results
   static constexpr int kACols = kKps * 64;              // TMEM columns per weight stage
   static constexpr int kDCols = kKps * NTOK;            // TMEM columns per result stage
-  // unpacking warps: four per SM sub-partition for 16/32 tokens (each takes
-  // half of one record's rows-quarter), two at 64 tokens, whose scale warps
-  // need more registers than 24 warps leave them
-  static constexpr int kUnpackWarps = NTOK <= 32 ? 16 : 8;
   static constexpr int kThreads = (8 + kUnpackWarps) * 32;
-  static constexpr int kChunks = 4 * kKps * 4 / kUnpackWarps;   // 32-K chunks per unpacking warp
+  // full barriers, one per (SMEM stage, unpacking group): iteration `it`
+  // uses barrier (it % SS, it % NDQ), so every waiter sees each phase of
+  // its barriers in order whatever the ring depth
+  static constexpr int kFullBars = kSmemStages * kNdq;
+  static constexpr int kFullPeriod = kSmemStages / cgcd(kSmemStages, kNdq) * kNdq;  // lcm
   // Warp 1 issues every MMA.  (Letting the last unpacking warp to finish a
   // stage issue that stage's MMAs measured slower on B200: single-lane issue
   // from a busy warp.)
-  static constexpr int kEpiScratch = 4 * 2048;          // warp-local transposes of the output
-  static constexpr int kBarBytes = 512;
   // byte offsets from the 1024-aligned base of dynamic shared memory
   static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
   static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
   static constexpr size_t kScrOff = (kTabOff + 2 * (kMaxExperts + 1) * sizeof(int) + 127) / 128 * 128;
   static constexpr size_t kSmem = 1024 + kScrOff + kEpiScratch;
-  static_assert(kABlock % 1024 == 0 && kRecMax % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
+  static_assert(kABlock % 1024 == 0 && kRecStride % 16 == 0 && kBarOff % 16 == 0, "stage alignment");
   static_assert(kACols * kAStages + kDCols * kDStages <= 512, "TMEM budget");
-  static_assert(8 * (2 * kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 <= kBarBytes,
+  static_assert(kAStages % kNdq == 0, "every TMEM weight stage must always return to the same group");
+  static_assert(kGroupWarps % 4 == 0 && kChunks * kGroupWarps == 16 * kKps, "chunk split");
+  static_assert(8 * (kFullBars + kSmemStages + 2 * kAStages + 2 * kDStages + 1) + 16 <= kBarBytes,
                 "barrier area");
   static_assert(kSmem <= 232448, "shared memory budget");
+  static_assert(kSmemStages >= 2, "pipeline depth");
 };
 
-// Unpack 32-K chunks c0 .. c0+NCH-1 of one 128-K record into TMEM: thread
-// (warp quarter q, lane) owns weight row r = 32q + lane and writes the exact
-// values bf16(q_k - z) into TMEM lane r, 16 columns per chunk from
-// taddr + 16*c (two weights per 32-bit column, even k in the low half).
-template <int NCH>
-__device__ __forceinline__ void unpack_codes(const uint8_t* rec, int c0, int r, int has_zero, uint32_t taddr) {
-  uint4 raw[NCH];
-#pragma unroll
-  for (int c = 0; c < NCH; ++c) raw[c] = *reinterpret_cast<const uint4*>(rec + ((c0 + c) * 128 + r) * 16);
-  const uint32_t z = has_zero ? rec[kW4RecCodes + 256 + r] : 8u;
-  // bf16(128 + z) is exact, and so is (128 + q) - (128 + z) = q - z
+// One 32-K chunk c of weight row r of a record, exact: the bf16 values
+// (q - z) (bf16 holds every such integer, up to 255 in magnitude) as 16
+// words of two weights (even k in the low half).  Codes of up to 4 bits:
+// OR-ing a code into the mantissa of bf16 128.0 gives bf16(128 + q), and
+// (128 + q) - (128 + z) is q - z exactly.  INT8 codes: 2^23 + q in fp32,
+// minus 2^23 + z, is q - z exactly, and so is its conversion to bf16.
+template <int FMT>
+__device__ __forceinline__ void unpack_chunk(const uint8_t* rec, int c, int r, uint32_t z, uint32_t (&out)[16]) {
   const uint32_t zbits = 0x4300u + z;
   const uint32_t z2 = zbits | (zbits << 16);
+  if constexpr (FMT == kFmtInt8) {
+    // 16-K chunks 2c and 2c + 1 of the row, 16 code bytes each
+    const float zf = 8388608.f + (float)z;
 #pragma unroll
-  for (int c = 0; c < NCH; ++c) {
-    const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-    uint32_t out[16];
+    for (int h = 0; h < 2; ++h) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(rec + ((2 * c + h) * 128 + r) * 16);
+      const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        out[8 * h + 2 * w] = pack_bf16x2(u8_minus_zero(wv[w], 0, zf), u8_minus_zero(wv[w], 1, zf));
+        out[8 * h + 2 * w + 1] = pack_bf16x2(u8_minus_zero(wv[w], 2, zf), u8_minus_zero(wv[w], 3, zf));
+      }
+    }
+  } else if constexpr (FMT == kFmtInt3) {
+    // words 3c .. 3c+2 of the row: pairs 0-14 at bits 3j / 16 + 3j of word
+    // 3c + i/5, pair 15 from bit p at 15 / 31 of word 3c + p
+    uint32_t wv[3];
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+      const int q = 3 * c + p;
+      wv[p] = *reinterpret_cast<const uint32_t*>(rec + ((q >> 2) * 128 + r) * 16 + 4 * (q & 3));
+    }
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+#pragma unroll
+      for (int j = 0; j < 5; ++j)
+        out[5 * p + j] = bf16x2_sub(lop3_and_or(wv[p] >> (3 * j), 0x00070007u, 0x43004300u), z2);
+    }
+    uint32_t x2 = lop3_and_or(wv[0] >> 15, 0x00010001u, 0x43004300u);
+    x2 = lop3_and_or(wv[1] >> 14, 0x00020002u, x2);
+    x2 = lop3_and_or(wv[2] >> 13, 0x00040004u, x2);
+    out[15] = bf16x2_sub(x2, z2);
+  } else if constexpr (FMT == kFmtInt2) {
+    // words 2c, 2c+1 of the row: pair i at bits 2j / 16 + 2j of word 2c + i/8
+    const uint2 wv = *reinterpret_cast<const uint2*>(rec + ((c >> 1) * 128 + r) * 16 + 8 * (c & 1));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      out[j] = bf16x2_sub(lop3_and_or(wv.x >> (2 * j), 0x00030003u, 0x43004300u), z2);
+      out[8 + j] = bf16x2_sub(lop3_and_or(wv.y >> (2 * j), 0x00030003u, 0x43004300u), z2);
+    }
+  } else {
+    // 16 bytes: the nibbles of k = 2j and 2j+1 of each word at bits 4j and 16+4j
+    const uint4 raw = *reinterpret_cast<const uint4*>(rec + (c * 128 + r) * 16);
+    const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // the nibbles of k = 2j and 2j+1 sit at bits 4j and 16+4j: OR-ing
-        // them into the mantissa of bf16 128.0 gives bf16(128 + q)
-        const uint32_t x2 = lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u);
-        out[w * 4 + j] = bf16x2_sub(x2, z2);
-      }
+      for (int j = 0; j < 4; ++j) out[w * 4 + j] = bf16x2_sub(lop3_and_or(wv[w] >> (4 * j), 0x000F000Fu, 0x43004300u), z2);
     }
-    tmem_st_x16(taddr + (c0 + c) * 16, out);
   }
 }
 
-template <int NTOK>
-__global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
+// Unpack the chunks [c0, c0 + NCH) of a stage (chunk i = record i / 4,
+// 32-K chunk i % 4 of it) for weight row r into TMEM lane r: each chunk
+// fills 16 columns from taddr + 16 * i.  Records at or past `nrec` (the
+// ragged end of a unit) are skipped.
+template <int FMT, int NCH, int CODE_BYTES, uint32_t ZSYM>
+__device__ __forceinline__ void unpack_stage(const uint8_t* recs, int rec_bytes, int nrec, int c0, int r, int has_zero,
+                                             uint32_t taddr) {
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    const int ci = c0 + i;
+    const int rr = ci >> 2;
+    if (rr >= nrec) break;
+    const uint8_t* rec = recs + rr * rec_bytes;
+    const uint32_t z = has_zero ? rec[CODE_BYTES + 256 + r] : ZSYM;
+    uint32_t out[16];
+    unpack_chunk<FMT>(rec, ci & 3, r, z, out);
+    tmem_st_x16(taddr + ci * 16, out);
+  }
+}
+
+template <int NTOK, int FMT>
+__global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
     w4a16_small_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
-  using C = SmallCfg<NTOK>;
+  using C = SmallCfg<NTOK, FMT>;
   constexpr int SS = C::kSmemStages;
   constexpr int AS = C::kAStages;
   constexpr int DS = C::kDStages;
   constexpr int KPS = C::kKps;
+  constexpr int NDQ = C::kNdq;
   constexpr int kATile = C::kATile;
   constexpr int kRecs = C::kRecs;
   constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
@@ -125,8 +203,8 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
   uint8_t* sA = smem;                               // SS * kATile (activations, 128-byte swizzle)
   uint8_t* sR = smem + SS * kATile;                 // SS * kRecs (packed weight records)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* empty = full + SS;      // MMA commit + the four scale warps
-  uint64_t* aready = empty + SS;    // eight unpacking warps
+  uint64_t* empty = full + C::kFullBars;  // MMA commit + the four scale warps
+  uint64_t* aready = empty + SS;    // the owning group's unpacking warps
   uint64_t* afree = aready + AS;    // MMA commit
   uint64_t* dfull = afree + AS;     // MMA commit
   uint64_t* dempty = dfull + DS;    // four scale warps
@@ -137,17 +215,17 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
   int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);  // [kMaxExperts + 1]
   int* s_off = s_prefix + (kMaxExperts + 1);                    // [kMaxExperts + 1]
   uint16_t* epi_scratch = reinterpret_cast<uint16_t*>(smem + C::kScrOff);  // 16-byte aligned
+  auto full_bar = [&](uint32_t i) { return &full[(i % SS) * NDQ + (i % NDQ)]; };
+  auto full_par = [](uint32_t i) { return (i / C::kFullPeriod) & 1; };
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SS; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 5);
-    }
+    for (int f = 0; f < C::kFullBars; ++f) mbar_init(&full[f], 1);
+    for (int s = 0; s < SS; ++s) mbar_init(&empty[s], 5);
     for (int t = 0; t < AS; ++t) {
-      mbar_init(&aready[t], C::kUnpackWarps);
+      mbar_init(&aready[t], C::kGroupWarps);
       mbar_init(&afree[t], 1);
     }
     for (int d = 0; d < DS; ++d) {
@@ -179,14 +257,17 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
     // of the first SS stages (no kernel writes them)
     uint32_t n_pre = 0;
     if (!p.grouped) {
-      for (int idx = 0; n_pre < (uint32_t)SS && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
+      for (int idx = 0; p.early_weights && n_pre < (uint32_t)SS &&
+                        get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
+           ++idx) {
         const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
         for (int kb = x.kb0; kb < x.kb1 && n_pre < (uint32_t)SS; kb += KPS, ++n_pre) {
           const int nrec = min(KPS, x.kb1 - kb);
           if (leader) {
-            mbar_arrive_expect_tx(&full[n_pre], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
-            bulk_g2s(sR + n_pre * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes),
-                     &full[n_pre], pol_w);
+            uint64_t* fb = full_bar(n_pre);
+            mbar_arrive_expect_tx(fb, (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+            bulk_g2s(sR + n_pre * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), fb,
+                     pol_w);
           }
           __syncwarp();
         }
@@ -208,17 +289,17 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
           break;
         }
         if (leader) {
+          uint64_t* fb = full_bar(it);
           if (it >= n_pre) {
-            mbar_arrive_expect_tx(&full[s], (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
+            mbar_arrive_expect_tx(fb, (uint32_t)nrec * ((uint32_t)p.rec_bytes + C::kABlock));
             // the stage's records are consecutive in the blob: one bulk copy
             // (long copies stream HBM much faster than record-sized ones)
-            bulk_g2s(sR + s * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), &full[s],
-                     pol_w);
+            bulk_g2s(sR + s * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), fb, pol_w);
           }
           for (int r = 0; r < nrec; ++r) {
             uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
-            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, &full[s]);
-            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, &full[s]);
+            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, fb);
+            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, fb);
           }
         }
         __syncwarp();
@@ -227,7 +308,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
     if (!ok && lane == 0) {
       // let every copy already issued land before the CTA exits
       const uint32_t first = it > (uint32_t)SS ? it - SS : 0;
-      for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % SS], (j / SS) & 1, p.wait_ns, nullptr);
+      for (uint32_t j = first; j < it; ++j) hq_wait(full_bar(j), full_par(j), p.wait_ns, nullptr);
     }
   } else {
   // The producer needs no TMEM, so it starts loading at once; the other
@@ -275,7 +356,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, t = it % AS, d = it % DS;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp_n(3, &aready[t], (it / AS) & 1, &full[s], (it / SS) & 1, &dempty[d],
+        if (!hq_wait_warp_n(3, &aready[t], (it / AS) & 1, full_bar(it), full_par(it), &dempty[d],
                             ((it / DS) & 1) ^ 1, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
@@ -294,13 +375,15 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
     __syncwarp();
   } else if (warp >= 8) {
     // ------------------------------------------------------------ unpack codes (warps 8 and up)
-    // warp 8 + 4u + q unpacks rows 32q..32q+31 of share u of the stage: with
-    // 16 warps, record u/2, chunks 2(u%2), 2(u%2)+1; with 8, record u, all 4
+    // warp 8 + kGroupWarps * g + 4u + q belongs to group g and unpacks rows
+    // 32q .. 32q+31 of the chunks [u * NCH, (u + 1) * NCH) of every stage
+    // the group owns
     constexpr int NCH = C::kChunks;
+    const int wi = (int)warp - 8;
+    const int g = wi / C::kGroupWarps;
+    const int u = (wi % C::kGroupWarps) >> 2;
     const uint32_t q = warp & 3;
-    const int u = (int)(warp - 8) >> 2;
-    const int h = u * NCH / 4;                        // record of the stage this warp unpacks
-    const int c0 = (u * NCH) % 4;                     // first chunk
+    const int c0 = u * NCH;
     const int r = (int)(q * 32 + lane);               // weight row within the tile
     const uint32_t lane_addr = (q * 32) << 16;
     uint32_t it = 0;
@@ -308,21 +391,22 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
     Unit x;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
+        if ((int)(it % NDQ) != g) continue;
         const int s = it % SS, t = it % AS;
         const int nrec = min(KPS, x.kb1 - kb);
-        // full[s] cannot move on before this warp's own arrival (through the
-        // MMA it enables) and afree[t] before the MMA it enables: every
-        // phase of both is observed in order
-        if (!hq_wait_warp_n(2, &full[s], (it / SS) & 1, &afree[t], ((it / AS) & 1) ^ 1, nullptr, 0, p.wait_ns,
+        // The full barrier of (stage, group) and TMEM stage t (AS % NDQ == 0)
+        // only ever serve this group, and neither can move on before this
+        // group's own arrival (through the MMA it enables): every phase of
+        // both is observed in order
+        if (!hq_wait_warp_n(2, full_bar(it), full_par(it), &afree[t], ((it / AS) & 1) ^ 1, nullptr, 0, p.wait_ns,
                             s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        if (h < nrec)
-          unpack_codes<NCH>(sR + s * kRecs + h * p.rec_bytes, c0, r, p.has_zero,
-                            tmem_base + lane_addr + a_col(t) + h * 64);
+        unpack_stage<FMT, NCH, C::kCodeBytes, C::kZSym>(sR + s * kRecs, p.rec_bytes, nrec, c0, r, p.has_zero,
+                                                         tmem_base + lane_addr + a_col(t));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -345,7 +429,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, d = it % DS;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait(&full[s], (it / SS) & 1, p.wait_ns, s_abort)) {
+        if (!hq_wait(full_bar(it), full_par(it), p.wait_ns, s_abort)) {
           raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -354,7 +438,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < KPS; ++rr)
           sc[rr] = rr < nrec ? __half2float(reinterpret_cast<const __half*>(sR + s * kRecs + rr * p.rec_bytes +
-                                                                            kW4RecCodes)[r])
+                                                                            C::kCodeBytes)[r])
                              : 0.f;
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -408,10 +492,11 @@ __global__ void __launch_bounds__(SmallCfg<NTOK>::kThreads, 1)
   if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
-template <int NTOK>
+template <int NTOK, int FMT>
 hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_small_kernel<NTOK>;
-  const size_t smem = SmallCfg<NTOK>::kSmem;
+  auto kern = w4a16_small_kernel<NTOK, FMT>;
+  using C = SmallCfg<NTOK, FMT>;
+  const size_t smem = C::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -420,18 +505,27 @@ hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cu
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  return launch_pdl(kern, dim3(grid), dim3(SmallCfg<NTOK>::kThreads), smem, stream, map, p) == cudaSuccess
-             ? HQ_OK
-             : HQ_ERR_CUDA;
+  return launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, stream, map, p) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+template <int FMT>
+hq_status small_launch_f(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+  switch (ntok) {
+    case 16: return launch_small_t<16, FMT>(map, p, grid, stream);
+    case 32: return launch_small_t<32, FMT>(map, p, grid, stream);
+    case 64: return launch_small_t<64, FMT>(map, p, grid, stream);
+    default: return HQ_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace
 
-hq_status small_launch(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  switch (ntok) {
-    case 16: return launch_small_t<16>(map, p, grid, stream);
-    case 32: return launch_small_t<32>(map, p, grid, stream);
-    case 64: return launch_small_t<64>(map, p, grid, stream);
+hq_status small_launch(int ntok, int fmt, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+  switch (fmt) {
+    case kFmtInt4: return small_launch_f<kFmtInt4>(ntok, map, p, grid, stream);
+    case kFmtInt3: return small_launch_f<kFmtInt3>(ntok, map, p, grid, stream);
+    case kFmtInt2: return small_launch_f<kFmtInt2>(ntok, map, p, grid, stream);
+    case kFmtInt8: return small_launch_f<kFmtInt8>(ntok, map, p, grid, stream);
     default: return HQ_ERR_UNSUPPORTED;
   }
 }

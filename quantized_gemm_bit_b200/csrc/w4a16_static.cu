@@ -1,5 +1,5 @@
-// Dense W4A16 GEMM entry point that allocates nothing (INT4 or MXFP4_A16
-// weights, as hq_gemm_w4a16).
+// Dense W4A16 GEMM entry point that allocates nothing (INT4, INT3, INT2 or
+// MXFP4_A16 weights, as hq_gemm_w4a16).
 //
 // Some callers cannot allocate device memory at the point where they run a
 // layer: an inference engine that plans every buffer up front and then
@@ -18,15 +18,17 @@
 //   * every call uses the same array, so calls that overlap on the GPU
 //     (different streams, no ordering) race on it; calls ordered on one
 //     stream do not;
-//   * each call clears the part that must start at zero (error word and
-//     tile counters) on its stream before the kernel.
+//   * each call whose plan splits K clears the tile counters (which must
+//     start at zero) on its stream before the kernel;
+//   * its first word records the first device-side error of any call
+//     (a bounded wait that ran out) until hq_static_check_device_status
+//     reads and clears it.
 // Host code cannot use the array's name as a device address: the first call
-// on each device looks the address up with cudaGetSymbolAddress (with that
-// device current) and caches it, so the first call on a device should come
-// before any stream capture.
+// in each CUDA context looks the address up with cudaGetSymbolAddress (with
+// that context current) and caches it per context, so the first call in a
+// context should come before any stream capture.
 #include <cuda_runtime.h>
 
-#include <algorithm>
 #include <mutex>
 
 #include "hq_internal.h"
@@ -39,19 +41,61 @@ constexpr size_t kHqStaticScratchBytes = 16u << 20;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kHqStaticScratchBytes];
 
-// Device address of g_static_scratch on the current device (looked up once
-// per device), or nullptr when the lookup fails.
-void* static_scratch_address(int device) {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (0 when none is current or the driver
+// cannot say).  A context destroyed and created again (cudaDeviceReset)
+// gets a new id, and its module, with this array, may load elsewhere.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = []() -> CtxGetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  static CtxGetIdFn get_id = []() -> CtxGetIdFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<CtxGetIdFn>(p);
+  }();
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_static_scratch in the current context, looked up once
+// per context (keyed by its unique id), or nullptr when the lookup fails.
+void* static_scratch_address() {
   static std::mutex mu;
-  static void* addr[64] = {};
-  if (device < 0 || device >= 64) return nullptr;
+  constexpr int kSlots = 64;
+  static unsigned long long ids[kSlots] = {};
+  static void* addrs[kSlots] = {};
+  static int next = 0;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[device] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
-    addr[device] = ptr;
+  unsigned long long id = current_context_id();
+  if (id != 0) {
+    for (int i = 0; i < kSlots; ++i)
+      if (ids[i] == id) return addrs[i];
   }
-  return addr[device];
+  void* ptr = nullptr;
+  // makes the device's primary context current if no context was
+  if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+  if (id == 0) id = current_context_id();
+  if (id != 0) {
+    ids[next] = id;
+    addrs[next] = ptr;
+    next = (next + 1) % kSlots;
+  }
+  return ptr;
 }
 
 }  // namespace
@@ -81,12 +125,32 @@ extern "C" hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* pa
     cfg = w4_whole_tiles(dev, *d, m, cfg);
   const size_t need = w4_workspace_bytes(*d, m, cfg, false);
   if (need > kHqStaticScratchBytes) return HQ_ERR_WORKSPACE_TOO_SMALL;
-  void* scratch = static_scratch_address(dev.device);
+  void* scratch = static_scratch_address();
   if (!scratch) return HQ_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // error word and tile counters start at zero (the partial sums need not)
-  const size_t tiles = (size_t)((d->n + kTileN - 1) / kTileN) * (size_t)((m + cfg.ntok - 1) / cfg.ntok);
-  const size_t zero_bytes = std::min(need, sizeof(WsHeader) + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256);
-  if (cudaMemsetAsync(scratch, 0, zero_bytes, s) != cudaSuccess) return HQ_ERR_CUDA;
+  // the tile counters start at zero (the partial sums need not, and the
+  // error word keeps the first error until it is read)
+  if (cfg.splits != 0) {
+    const size_t tiles = (size_t)((d->n + kTileN - 1) / kTileN) * (size_t)((m + cfg.ntok - 1) / cfg.ntok);
+    const size_t counter_bytes = ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256;
+    if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + sizeof(WsHeader), 0, counter_bytes, s) != cudaSuccess)
+      return HQ_ERR_CUDA;
+  }
   return w4_launch(*d, cfg, packed_w_dev, a_dev, m, c_dev, nullptr, scratch, s);
+}
+
+extern "C" hq_status hq_static_check_device_status(hq_stream_t stream) {
+  DeviceInfo dev{};
+  hq_status st = device_info(&dev);
+  if (st != HQ_OK) return st;
+  void* scratch = static_scratch_address();
+  if (!scratch) return HQ_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HQ_ERR_CUDA;
+  uint32_t err = 0;
+  if (cudaMemcpy(&err, scratch, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess) return HQ_ERR_CUDA;
+  if (err != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpy(scratch, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HQ_ERR_CUDA;
+  }
+  return static_cast<hq_status>(err);
 }

@@ -37,6 +37,8 @@ HQ_FMT_NVFP4 = 3
 HQ_FMT_MXFP4_A16 = 4
 HQ_FMT_INT3 = 5
 HQ_FMT_INT2 = 6
+HQ_FMT_INT8 = 7
+HQ_FMT_MXINT4 = 8
 
 # Every symbol include/hq.h declares.
 EXPORTS = (
@@ -45,7 +47,8 @@ EXPORTS = (
     "hq_quantize_nvfp4_workspace_size", "hq_quantize_nvfp4", "hq_moe_topk", "hq_moe_topk_softmax",
     "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_moe_swiglu",
     "hq_moe_combine_workspace_size", "hq_moe_combine", "hq_check_device_status",
-    "hq_debug_timeout_probe", "hq_gemm_w4a16_static",
+    "hq_debug_timeout_probe", "hq_gemm_w4a16_static", "hq_static_check_device_status",
+    "hq_pack_weights_gated", "hq_grouped_gemm_moe_swiglu",
 )
 
 
@@ -56,7 +59,10 @@ class QuantDesc(ctypes.Structure):
 
 class Tuning(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in
-                ("tile_m", "tile_n", "tile_k", "stages", "split_k", "cta_group", "variant")]
+                ("tile_m", "tile_n", "tile_k", "stages", "split_k", "cta_group", "variant", "flags")]
+
+
+HQ_TUNE_NO_EARLY_WEIGHTS = 1
 
 
 class HQError(RuntimeError):
@@ -103,6 +109,9 @@ def lib():
             "hq_check_device_status": (st, [vp, vp]),
             "hq_debug_timeout_probe": (st, [vp, ctypes.c_uint64, vp]),
             "hq_gemm_w4a16_static": (st, [dp, vp, vp, i32, vp, tp, vp]),
+            "hq_static_check_device_status": (st, [vp]),
+            "hq_pack_weights_gated": (st, [dp, vp, vp, vp, vp, sz]),
+            "hq_grouped_gemm_moe_swiglu": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -184,6 +193,18 @@ def hq_pack_weights(desc, codes, scales, zeros=None, global_scale=0.0):
     return out
 
 
+def hq_pack_weights_gated(desc, codes, scales, zeros=None):
+    """Host packer of gate+up weights in the gated row order (for
+    hq_grouped_gemm_moe_swiglu): returns the blob as a numpy uint8 array."""
+    codes, scales, zeros = _host(codes), _host(scales), _host(zeros)
+    if scales.dtype == np.float16:
+        scales = scales.view(np.uint16)
+    out = np.empty(hq_packed_size(desc), dtype=np.uint8)
+    _check(lib().hq_pack_weights_gated(ctypes.byref(desc), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(out),
+                                       out.nbytes), "hq_pack_weights_gated")
+    return out
+
+
 def hq_workspace_size(desc, m, tuning=None):
     return lib().hq_workspace_size(ctypes.byref(desc), int(m), _tuning(tuning))
 
@@ -260,6 +281,14 @@ def hq_grouped_gemm_moe(desc, packed_w, a_sorted, expert_offsets, total_rows, c_
                                      ws.numel() * ws.element_size(), _stream(stream)), "hq_grouped_gemm_moe")
 
 
+def hq_grouped_gemm_moe_swiglu(desc, packed_w, a_sorted, expert_offsets, total_rows, h_sorted, ws, tuning=None,
+                               stream=None):
+    _check(lib().hq_grouped_gemm_moe_swiglu(ctypes.byref(desc), _ptr(packed_w), _ptr(a_sorted),
+                                            _ptr(expert_offsets), int(total_rows), _ptr(h_sorted), _tuning(tuning),
+                                            _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hq_grouped_gemm_moe_swiglu")
+
+
 def hq_check_device_status(ws, stream=None):
     """Returns the device-side status recorded in the workspace (and clears it)."""
     return lib().hq_check_device_status(_ptr(ws), _stream(stream))
@@ -275,3 +304,9 @@ def hq_gemm_w4a16_static(desc, packed_w, a, m, c, tuning=None, stream=None):
     include/hq.h for its size and sharing rules)."""
     _check(lib().hq_gemm_w4a16_static(ctypes.byref(desc), _ptr(packed_w), _ptr(a), int(m), _ptr(c),
                                       _tuning(tuning), _stream(stream)), "hq_gemm_w4a16_static")
+
+
+def hq_static_check_device_status(stream=None):
+    """First device-side error of the allocation-free calls since the last
+    read (HQ_OK when none); synchronizes the stream."""
+    return int(lib().hq_static_check_device_status(_stream(stream)))

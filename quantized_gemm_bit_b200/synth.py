@@ -2,9 +2,8 @@
 
 This module only draws random numbers (torch CPU generator, fixed seeds) and
 puts them in the canonical containers the library and the oracle both read.
-It holds none of the method's arithmetic: no dequantization, no GEMM, no
-routing.  The one quantization step it performs (FP8 activations for the
-W4A8-MXFP4 workload) uses torch's own float8_e4m3fn cast, a library routine.
+It holds none of the method's arithmetic: no quantization, no
+dequantization, no GEMM, no routing.
 
 Recipes (one per workload; seed = workload index * 1000 + shape index):
   * W4A16: qweight int32 [N, K/8] with every bit uniform (= eight uniform
@@ -17,11 +16,17 @@ Recipes (one per workload; seed = workload index * 1000 + shape index):
     points uniform in [0, 7] (symmetric: zero point 4).
   * W2A16 (INT2): as W4A16 with K/16 int32 words per row (16 uniform
     2-bit codes each) and zero points uniform in [0, 3] (symmetric: 2).
+  * W8A16 (INT8): as W4A16 with K/4 int32 words per row (4 uniform 8-bit
+    codes each) and zero points uniform in [0, 255] (symmetric: 128).
+  * MXINT4 weights: 4-bit codes uniform over the 16 codes (two's
+    complement -8..7), two per byte (even k low nibble); one E8M0 scale per
+    32 K with exponent uniform in [-8, -2], as for MXFP4.
   * W4A8-MXFP4 (and MXFP4 weights with bf16 activations): FP4 codes
     uniform over the 16 codes, two per byte (even k low nibble); one E8M0
     scale per 32 K with exponent uniform in [-8, -2];
-    activations bf16 N(0,1) widened to fp32, per-token scale amax/448 (fp32),
-    E4M3 codes by torch's cast of x/scale (clamped to +-448).
+    activations bf16 N(0,1) draws; their per-token FP8 quantization
+    (scale amax/448) is the method's arithmetic and is not done here (the
+    GPU path runs the library's quantizer, the tests the oracle's).
   * NVFP4: bf16 N(0,1) draws for both operands; the two-level quantization
     that turns them into codes is the method's arithmetic and is not done
     here.
@@ -90,6 +95,29 @@ def w3a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
     return qweight, scales, zeros
 
 
+def w8a16_weights(n, k, group=128, asym=False, seed=0, experts=None):
+    """Canonical INT8 weights: qweight int32 [.., N, K/4] with every bit
+    uniform (= 4 uniform 8-bit codes per word along K, low byte first), fp16
+    scales as for W4A16, zero points uniform in [0, 255] (asymmetric) or none
+    (symmetric, zero point 128)."""
+    assert k % group == 0 and k % 4 == 0
+    g = _gen(seed)
+    lead = () if experts is None else (experts,)
+    qweight = torch.randint(-(2 ** 31), 2 ** 31, lead + (n, k // 4), generator=g, dtype=torch.int32)
+    scales = (0.002 + 0.01 * torch.randn(lead + (n, k // group), generator=g).abs()).to(torch.float16)
+    zeros = None
+    if asym:
+        zeros = torch.randint(0, 256, lead + (n, k // group), generator=g, dtype=torch.uint8)
+    return qweight, scales, zeros
+
+
+def mxint4_weights(n, k, seed=0, experts=None):
+    """MXINT4 weights: codes uint8 [.., N, K/2] (two uniform 4-bit codes per
+    byte, even k low nibble), E8M0 scales uint8 [.., N, K/32] with exponent
+    uniform in [-8, -2] (the MXFP4 recipe's draws)."""
+    return mxfp4_weights(n, k, seed=seed, experts=experts)
+
+
 def mxfp4_weights(n, k, seed=0, experts=None):
     """MXFP4 weights: codes uint8 [.., N, K/2] (two uniform FP4 codes per
     byte), E8M0 scales uint8 [.., N, K/32] with exponent uniform in [-8, -2].
@@ -100,17 +128,6 @@ def mxfp4_weights(n, k, seed=0, experts=None):
     codes = torch.randint(0, 256, lead + (n, k // 2), generator=g, dtype=torch.uint8)
     e8m0 = (127 + torch.randint(-8, -1, lead + (n, k // 32), generator=g, dtype=torch.int32)).to(torch.uint8)
     return codes, e8m0
-
-
-def fp8_activations(m, k, seed=0):
-    """E4M3 activations with a per-token fp32 scale amax/448 (library cast).
-    Returns (codes uint8 [M, K], scale float32 [M])."""
-    x = bf16_normal(m, k, seed).to(torch.float32)
-    amax = x.abs().amax(dim=1)
-    s = amax / 448.0
-    s = torch.where(amax > 0, s, torch.ones_like(s))
-    q = (x / s[:, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
-    return q.view(torch.uint8), s.to(torch.float32)
 
 
 def router_logits(t, e, seed=0):

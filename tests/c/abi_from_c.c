@@ -67,12 +67,14 @@ int main(void) {
   CHECK(hq_quant_desc_init(&d, HQ_FMT_INT4, n, 100, 128, 0, 1) == HQ_ERR_UNSUPPORTED);
   CHECK(hq_quant_desc_init(&d, 42, n, k, 128, 0, 1) == HQ_ERR_INVALID_ARG);
   CHECK(hq_quant_desc_init(NULL, HQ_FMT_INT4, n, k, 128, 0, 1) == HQ_ERR_INVALID_ARG);
-  CHECK(hq_quant_desc_init(&d, HQ_FMT_INT3, n, k, 128, 1, 1) == HQ_OK);
+  /* exact-integer weights need a 128-K group scale: MXFP4 (one per 32 K) has none */
+  CHECK(hq_quant_desc_init(&d, HQ_FMT_MXFP4_A16, n, k, 32, 0, 1) == HQ_OK);
   hq_tuning t;
   memset(&t, 0, sizeof t);
-  t.variant = 2; /* exact-integer weights: INT4 only */
+  t.variant = 2;
   CHECK(hq_gemm_w4a16(&d, (void*)16, (void*)16, 4, (void*)32, &t, (void*)256, 1 << 20, NULL) ==
         HQ_ERR_UNSUPPORTED);
+  CHECK(hq_quant_desc_init(&d, HQ_FMT_INT3, n, k, 128, 1, 1) == HQ_OK);
   CHECK(hq_gemm_w4a16(&d, NULL, NULL, 0, NULL, NULL, NULL, 0, NULL) == HQ_OK); /* m == 0 */
   CHECK(hq_gemm_w4a16(&d, (void*)16, (void*)18, 4, (void*)32, NULL, (void*)256, 1 << 20, NULL) ==
         HQ_ERR_ALIGNMENT);

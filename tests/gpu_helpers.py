@@ -53,3 +53,34 @@ def tile_rows(m, tile, rng, per_tile=2):
         rows.update({t0, t1})
         rows.update(rng.integers(t0, t1 + 1, size=per_tile).tolist())
     return np.array(sorted(rows))
+
+
+def check_swiglu(h_bf16, gate_up_ref, inter, k, what=""):
+    """Output of the gate+up GEMM with the fused SwiGLU epilogue against the
+    oracle's fp64 gate and up values (one GEMM's output, so the GEMM's
+    relative Frobenius bar), and per element the GEMM element bound carried
+    through h = silu(g) * u to first order,
+        |err_h| <= |silu'(g) u| B + |silu(g)| B + 2^-8 |h|,
+    B = 1e-2 |ref| + 2e-3 sqrt(K) rms(ref) taken for g and u, plus the
+    bf16 rounding of h."""
+    h = h_bf16.float().double().cpu().numpy() if isinstance(h_bf16, torch.Tensor) else np.asarray(h_bf16)
+    gu = np.asarray(gate_up_ref, dtype=np.float64)
+    g, u = gu[:, :inter], gu[:, inter:2 * inter]
+    sig = 1.0 / (1.0 + np.exp(-g))
+    ref = g * sig * u
+    dsilu = sig * (1.0 + g * (1.0 - sig))
+    rms = np.sqrt(np.mean(gu ** 2))
+    bg = ELEM_REL * np.abs(g) + ELEM_ABS * np.sqrt(k) * rms
+    bu = ELEM_REL * np.abs(u) + ELEM_ABS * np.sqrt(k) * rms
+    bound = np.abs(dsilu * u) * bg + np.abs(g * sig) * bu + 2.0 ** -8 * np.abs(ref)
+    assert h.shape == ref.shape and np.all(np.isfinite(h)), what
+    err = h - ref
+    rel = np.linalg.norm(err) / np.linalg.norm(ref)
+    log = os.environ.get("HQ_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(f"{what}\t{rel:.3e}\t{np.max(np.abs(err) / np.maximum(bound, 1e-300)):.3e}\n")
+    assert rel <= REL_FRO, f"{what}: rel Frobenius {rel:.3e}"
+    worst = np.max(np.abs(err) - bound)
+    assert worst <= 0, f"{what}: element bound exceeded by {worst:.3e}"
+    return rel

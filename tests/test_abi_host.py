@@ -50,7 +50,8 @@ def test_desc_validation():
                        ((hq.HQ_FMT_INT3, 128, 128, 128, 2, 1), hq.HQ_ERR_INVALID_ARG),
                        ((hq.HQ_FMT_INT2, 128, 128, 32, 0, 1), hq.HQ_ERR_UNSUPPORTED),
                        ((hq.HQ_FMT_INT2, 128, 128, 128, 0, 1025), hq.HQ_ERR_UNSUPPORTED),
-                       ((7, 128, 128, 16, 0, 1), hq.HQ_ERR_INVALID_ARG)]:
+                       ((hq.HQ_FMT_INT8, 128, 128, 128, 2, 1), hq.HQ_ERR_INVALID_ARG),
+                       ((9, 128, 128, 16, 0, 1), hq.HQ_ERR_INVALID_ARG)]:
         with pytest.raises(hq.HQError) as e:
             hq.hq_quant_desc_init(*args)
         assert e.value.status == code
@@ -240,7 +241,8 @@ def test_gemm_argument_errors_need_no_gpu():
     t = hq.Tuning(tile_m=48)
     assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                             None) == hq.HQ_ERR_UNSUPPORTED
-    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=3), hq.Tuning(cta_group=2)):
+    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=3), hq.Tuning(cta_group=2),
+                hq.Tuning(flags=2)):
         assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
                                 None) == hq.HQ_ERR_UNSUPPORTED
     # grouped: no K split, no 512-token tile; block-scaled: no variants
@@ -248,8 +250,8 @@ def test_gemm_argument_errors_need_no_gpu():
     for bad in (hq.Tuning(tile_m=512), hq.Tuning(split_k=2)):
         assert L_.hq_grouped_gemm_moe(ctypes.byref(dg), 16, 16, 16, 40, 32, ctypes.byref(bad), 256, 1 << 20,
                                       None) == hq.HQ_ERR_UNSUPPORTED
-    # MXFP4 weights with bf16 activations: no exact-integer variant; the
-    # block-scaled entry points do not take them
+    # MXFP4 weights with bf16 activations: no exact-integer variant (INT3 and
+    # INT2 weights have one); the block-scaled entry points do not take them
     dx = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 1)
     t = hq.Tuning(variant=2)
     assert L_.hq_gemm_w4a16(ctypes.byref(dx), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
@@ -257,10 +259,6 @@ def test_gemm_argument_errors_need_no_gpu():
     assert L_.hq_gemm_w4a16_static(ctypes.byref(dx), 16, 16, 4, 32, ctypes.byref(t), None) == hq.HQ_ERR_UNSUPPORTED
     assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dx), 4096, 16, 16, 4, 32, None, 256, 1 << 20,
                                None) == hq.HQ_ERR_INVALID_ARG
-    for fmt in (hq.HQ_FMT_INT3, hq.HQ_FMT_INT2):
-        d3 = hq.hq_quant_desc_init(fmt, 256, 256, 128, 1, 1)
-        assert L_.hq_gemm_w4a16(ctypes.byref(d3), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
-                                None) == hq.HQ_ERR_UNSUPPORTED
     dxg = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 8)
     assert L_.hq_grouped_gemm_moe(ctypes.byref(dxg), 16, 16, 16, 40, 32, ctypes.byref(t), 256, 1 << 20,
                                   None) == hq.HQ_ERR_UNSUPPORTED
@@ -316,6 +314,102 @@ def test_autotune_candidates_need_no_gpu():
     assert not any(t.variant == 2 and t.tile_m > 64 for t in autotune.candidates("w4a16", 4096)[1:])
     assert all(t.variant == 0 for t in autotune.candidates("nvfp4", 256)[1:])
     assert all(t.variant == 1 for t in autotune.candidates("mxfp4_a16", 16)[1:])
-    assert all(t.variant == 1 for t in autotune.candidates("w3a16", 64)[1:])
-    assert all(t.variant == 1 for t in autotune.candidates("w2a16", 16)[1:])
+    assert {t.variant for t in autotune.candidates("w3a16", 64)[1:]} == {1, 2}
+    assert {t.variant for t in autotune.candidates("w2a16", 16)[1:]} == {1, 2}
     assert all(t.split_k == 0 for t in autotune.candidates("moe", 64)[1:])
+
+
+@pytest.mark.parametrize("fmt", [hq.HQ_FMT_INT4, hq.HQ_FMT_INT3, hq.HQ_FMT_INT2, hq.HQ_FMT_MXFP4_A16])
+@pytest.mark.parametrize("experts", [1, 3])
+def test_gated_pack_matches_oracle_row_order(fmt, experts):
+    """hq_pack_weights_gated equals the format's oracle layout of the rows
+    taken in the gated gate+up order, bit for bit."""
+    n, k = 256, 256
+    ex = experts if experts > 1 else None
+    perm = L.gated_source_rows(n)
+    if fmt == hq.HQ_FMT_MXFP4_A16:
+        codes, e8 = synth.mxfp4_weights(n, k, seed=31, experts=ex)
+        d = hq.hq_quant_desc_init(fmt, n, k, 32, 0, experts)
+        blob = hq.hq_pack_weights_gated(d, codes, e8)
+        cn, en = codes.numpy().reshape(experts, n, -1), e8.numpy().reshape(experts, n, -1)
+        ref = np.concatenate([L.mxa16_pack(cn[e][perm], en[e][perm]) for e in range(experts)])
+    else:
+        make, pack = {hq.HQ_FMT_INT4: (synth.w4a16_weights, L.w4a16_pack),
+                      hq.HQ_FMT_INT3: (synth.w3a16_weights, L.w3a16_pack),
+                      hq.HQ_FMT_INT2: (synth.w2a16_weights, L.w2a16_pack)}[fmt]
+        q, s, z = make(n, k, 128, True, seed=32, experts=ex)
+        d = hq.hq_quant_desc_init(fmt, n, k, 128, 1, experts)
+        blob = hq.hq_pack_weights_gated(d, q, s, z)
+        qn, sn, zn = (x.numpy().reshape(experts, n, -1) for x in (q, s, z))
+        ref = np.concatenate([pack(qn[e][perm], sn[e][perm], zn[e][perm]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+def test_gated_pack_and_fused_swiglu_argument_errors():
+    L_ = hq.lib()
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 192, 256, 128, 0, 4)       # n % 128 != 0
+    assert L_.hq_pack_weights_gated(ctypes.byref(d), 16, 16, None, 16, 1 << 30) == hq.HQ_ERR_UNSUPPORTED
+    assert L_.hq_grouped_gemm_moe_swiglu(ctypes.byref(d), 16, 16, 16, 40, 16, None, 256, 1 << 20,
+                                         None) == hq.HQ_ERR_UNSUPPORTED
+    dn = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, 256, 256, 16, 0, 1)
+    assert L_.hq_pack_weights_gated(ctypes.byref(dn), 16, 16, None, 16, 1 << 30) == hq.HQ_ERR_UNSUPPORTED
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 256, 256, 128, 0, 4)
+    assert L_.hq_grouped_gemm_moe_swiglu(ctypes.byref(d), 16, 16, 16, 0, 16, None, 256, 1 << 20, None) == hq.HQ_OK
+    assert L_.hq_grouped_gemm_moe_swiglu(ctypes.byref(d), 16, 16, 16, 40, 24, None, 256, 1 << 20,
+                                         None) == hq.HQ_ERR_ALIGNMENT
+    d1 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 256, 256, 128, 0, 1)     # dense: not grouped
+    assert L_.hq_grouped_gemm_moe_swiglu(ctypes.byref(d1), 16, 16, 16, 40, 16, None, 256, 1 << 20,
+                                         None) == hq.HQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("n,k,asym,experts", [(256, 384, False, 1), (200, 256, True, 1), (136, 256, True, 3)])
+def test_int8_pack_matches_oracle_layout(n, k, asym, experts):
+    q, s, z = synth.w8a16_weights(n, k, 128, asym, seed=n + 8, experts=experts if experts > 1 else None)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT8, n, k, 128, int(asym), experts)
+    blob = hq.hq_pack_weights(d, q, s, z)
+    assert blob.size == L.w8a16_packed_bytes(n, k, asym, experts)
+    qn, sn = q.numpy(), s.numpy()
+    zn = None if z is None else z.numpy()
+    if experts == 1:
+        ref = L.w8a16_pack(qn, sn, zn)
+    else:
+        ref = np.concatenate([L.w8a16_pack(qn[e], sn[e], None if zn is None else zn[e]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+@pytest.mark.parametrize("n,k,experts", [(128, 128, 1), (300, 384, 1), (136, 256, 3)])
+def test_mxint4_pack_matches_oracle_layout(n, k, experts):
+    codes, e8 = synth.mxint4_weights(n, k, seed=n + k + 4, experts=experts if experts > 1 else None)
+    if experts == 1:
+        # the whole scale range the packer accepts
+        e8 = torch.from_numpy(np.random.default_rng(n).integers(0, 252, size=(n, k // 32), dtype=np.uint8))
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXINT4, n, k, 32, 0, experts)
+    blob = hq.hq_pack_weights(d, codes, e8)
+    assert blob.size == L.mxi4_packed_bytes(n, k, experts)
+    cn, en = codes.numpy(), e8.numpy()
+    if experts == 1:
+        ref = L.mxi4_pack(cn, en)
+    else:
+        ref = np.concatenate([L.mxi4_pack(cn[e], en[e]) for e in range(experts)])
+    assert np.array_equal(blob, ref)
+
+
+def test_mxint4_pack_rejects_scales_that_overflow_bf16_and_descriptor_rules():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXINT4, 128, 128, 32, 0, 1)
+    codes, e8 = synth.mxint4_weights(128, 128, seed=9)
+    e8 = e8.clone()
+    e8[3, 1] = 252
+    with pytest.raises(hq.HQError) as e:
+        hq.hq_pack_weights(d, codes, e8)
+    assert e.value.status == hq.HQ_ERR_INVALID_ARG
+    for args, code in (((hq.HQ_FMT_MXINT4, 128, 128, 16, 0, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_MXINT4, 128, 128, 32, 1, 1), hq.HQ_ERR_UNSUPPORTED),
+                       ((hq.HQ_FMT_INT8, 128, 100, 128, 0, 1), hq.HQ_ERR_UNSUPPORTED)):
+        with pytest.raises(hq.HQError) as e:
+            hq.hq_quant_desc_init(*args)
+        assert e.value.status == code
+    # MXINT4 has no exact-integer variant (one scale per 32 K)
+    L_ = hq.lib()
+    t = hq.Tuning(variant=2)
+    assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
+                            None) == hq.HQ_ERR_UNSUPPORTED

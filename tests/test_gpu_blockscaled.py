@@ -28,7 +28,9 @@ def _setup():
 
 def mx_case(m, n, k, seed):
     codes, e8 = synth.mxfp4_weights(n, k, seed=seed)
-    aq, asc = synth.fp8_activations(m, k, seed=seed + 1)
+    # E4M3 activations from the oracle's per-token quantizer (amax / 448)
+    aq, asc = (torch.from_numpy(v) for v in F.fp8_per_token_quantize(
+        synth.bf16_normal(m, k, seed=seed + 1).float().numpy()))
     d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, n, k, 32, 0, 1)
     blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(DEV)
     return d, blob, aq, asc, codes.numpy(), e8.numpy()

@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import check_gemm, workspace
+from gpu_helpers import check_gemm, check_swiglu, workspace
 from oracle import formats as F
 from oracle import gemm as G
 from oracle import moe as R
@@ -305,29 +305,99 @@ def test_combine_reports_a_sorted_list_that_is_not_a_permutation(bad):
     assert st == hq.HQ_ERR_DEVICE_BAD_OFFSETS
 
 
-def _layer_oracle(x_bits, logits, q1, s1, q2, s2, k, e, inter):
+def _layer_oracle(x_bits, logits, q1, s1, q2, s2, k, e, inter, fused=False):
     """The layer from oracle pieces only, rounding to bf16 wherever the GPU
-    path stores bf16 (after each GEMM and after SwiGLU)."""
+    path stores bf16 (after each GEMM and after SwiGLU; with the SwiGLU fused
+    into the gate+up GEMM, gate and up are not rounded)."""
     ids = R.topk_by_logit(logits, k)
     w = R.softmax_topk_weights(logits, ids)
     _, off, src = R.permute(ids, e)
     xs = R.gather_rows(x_bits, src, k)
     _, c1 = G.grouped_w4a16_ref(xs, off, q1, s1, None, 128)
-    h = R.silu_mul(_bf16_bits(c1), inter)
+    h = R.silu_mul_f64(c1, inter) if fused else R.silu_mul(_bf16_bits(c1), inter)
     _, c2 = G.grouped_w4a16_ref(_bf16_bits(h), off, q2, s2, None, 128)
     return R.combine(_bf16_bits(c2), src, w, k), ids, off, src
 
 
-@pytest.mark.parametrize("variant", [0, 2])
-def test_moe_layer_end_to_end(variant):
+@pytest.mark.parametrize("tile_m,variant,fmt", [(0, 0, hq.HQ_FMT_INT4), (16, 0, hq.HQ_FMT_INT4),
+                                                (64, 0, hq.HQ_FMT_INT4), (128, 0, hq.HQ_FMT_INT4),
+                                                (256, 0, hq.HQ_FMT_INT4), (32, 1, hq.HQ_FMT_INT4),
+                                                (0, 0, hq.HQ_FMT_INT3), (0, 0, hq.HQ_FMT_MXFP4_A16)])
+def test_grouped_swiglu_fused_reduced_config(tile_m, variant, fmt):
+    """Gate+up grouped GEMM with the SwiGLU epilogue (weights packed in the
+    gated row order) against the oracle's fp64 gate and up values: 8
+    experts, 40 tokens top-2, one expert never chosen, I = 192 (three
+    128-row gated tiles), every token tile and both weight variants."""
+    e, inter, k, t, topk = 8, 192, 512, 40, 2
+    n = 2 * inter
+    if fmt == hq.HQ_FMT_MXFP4_A16:
+        codes, e8 = synth.mxfp4_weights(n, k, seed=5400, experts=e)
+        d = hq.hq_quant_desc_init(fmt, n, k, 32, 0, e)
+        blob = torch.from_numpy(hq.hq_pack_weights_gated(d, codes, e8)).to(DEV)
+        ref_fn = lambda xs, off: G.grouped_mxfp4_a16_ref(xs, off, codes.numpy(), e8.numpy())[1]
+    else:
+        make, ref = ((synth.w4a16_weights, G.grouped_w4a16_ref) if fmt == hq.HQ_FMT_INT4
+                     else (synth.w3a16_weights, G.grouped_w3a16_ref))
+        q, s, z = make(n, k, 128, True, seed=5400, experts=e)
+        d = hq.hq_quant_desc_init(fmt, n, k, 128, 1, e)
+        blob = torch.from_numpy(hq.hq_pack_weights_gated(d, q, s, z)).to(DEV)
+        ref_fn = lambda xs, off: ref(xs, off, q.numpy(), s.numpy(), z.numpy(), 128)[1]
+    logits = synth.router_logits(t, e, seed=5401)
+    logits[:, 3] = -100.0
+    ids = R.topk_by_logit(logits.numpy(), topk)
+    _, off, src = R.permute(ids, e)
+    a = synth.bf16_normal(t, k, seed=5402)
+    a_sorted = R.gather_rows(_bits(a), src, topk)
+    rows = t * topk
+    tuning = hq.Tuning(tile_m=tile_m, variant=variant) if (tile_m or variant) else None
+    h = torch.full((rows, inter), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, rows, tuning))
+    a_dev = torch.from_numpy(a_sorted.view(np.int16)).view(torch.bfloat16).to(DEV)
+    hq.hq_grouped_gemm_moe_swiglu(d, blob, a_dev, torch.from_numpy(off.astype(np.int32)).to(DEV), rows, h, ws, tuning)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    check_swiglu(h, ref_fn(a_sorted, off), inter, k, f"swiglu fused fmt={fmt} tile_m={tile_m} variant={variant}")
+
+
+@pytest.mark.parametrize("t", [64, 8192])
+def test_grouped_swiglu_fused_full_size_sampled(t):
+    """The layer's gate+up GEMM with the fused SwiGLU at the full workload
+    (256 experts, top-8, hidden 7168, I = 2048), in the bench's launch
+    configuration; sampled rows (at least two per non-empty expert), every
+    output feature."""
+    e, topk, hid, inter = 256, 8, 7168, 2048
+    n = 2 * inter
+    q, s, _ = synth.w4a16_weights(n, hid, 128, False, seed=5500, experts=e)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, hid, 128, 0, e)
+    blob = torch.from_numpy(hq.hq_pack_weights_gated(d, q, s, None)).to(DEV)
+    logits = synth.router_logits(t, e, seed=5501 + t)
+    ids = R.topk_by_logit(logits.numpy(), topk)
+    _, off, src = R.permute(ids, e)
+    x = synth.bf16_normal(t, hid, seed=5502 + t)
+    a_sorted = R.gather_rows(_bits(x), src, topk)
+    rows = t * topk
+    h = torch.empty(rows, inter, dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, rows))
+    a_dev = torch.from_numpy(a_sorted.view(np.int16)).view(torch.bfloat16).to(DEV)
+    hq.hq_grouped_gemm_moe_swiglu(d, blob, a_dev, torch.from_numpy(off.astype(np.int32)).to(DEV), rows, h, ws)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    rng = np.random.default_rng(5503)
+    sample = []
+    for ex in range(e):
+        lo, hi = int(off[ex]), int(off[ex + 1])
+        if hi > lo:
+            sample += sorted(set(rng.integers(lo, hi, size=2).tolist()))
+    sample = np.array(sorted(set(sample)))
+    _, ref = G.grouped_w4a16_ref(a_sorted, off, q.numpy(), s.numpy(), None, 128, row_subset=sample)
+    check_swiglu(h.cpu()[sample], ref, inter, hid, f"swiglu fused full size T={t}")
+
+
+@pytest.mark.parametrize("variant,fused", [(0, False), (2, False), (0, True), (2, True)])
+def test_moe_layer_end_to_end(variant, fused):
     """Route (top-k + weights) -> permute + gather -> gate+up grouped GEMM ->
     SwiGLU -> down grouped GEMM -> weighted combine, all through the C ABI
     on one stream, against the oracle's layer (32 experts, top-4, T=64,
-    hidden 1024, intermediate 256).  Routing and permutation bit-exact.  The
-    layer output carries the errors of two GEMMs in a row (the first one's
-    reaches the second through SwiGLU), so its bar is the sum of the two
-    GEMM bars: rel-Frobenius <= 1e-2 and, per element,
-    |err| <= 2e-2 |ref| + 4e-3 sqrt(K) rms(ref) with the down GEMM's K."""
+    hidden 1024, intermediate 256).  Routing and permutation bit-exact; the
+    layer output at the GEMM tolerance, with the down GEMM's K."""
     t, e, k, hid, inter = 64, 32, 4, 1024, 256
     q1, s1, _ = synth.w4a16_weights(2 * inter, hid, 128, False, seed=3600, experts=e)
     q2, s2, _ = synth.w4a16_weights(hid, inter, 128, False, seed=3601, experts=e)
@@ -344,9 +414,16 @@ def test_moe_layer_end_to_end(variant):
     hq.hq_moe_topk_softmax(logits.to(DEV), t, e, k, ids, wts)
     src, off, xs, st = gpu_permute(ids, e, x)
     assert st == hq.HQ_OK
-    c1 = _grouped(d1, b1, xs, off, t * k, 2 * inter, tun)
     h = torch.empty(t * k, inter, dtype=torch.bfloat16, device=DEV)
-    hq.hq_moe_swiglu(c1, t * k, inter, h)
+    if fused:
+        # gate+up weights in the gated row order, SwiGLU in the GEMM's epilogue
+        b1g = torch.from_numpy(hq.hq_pack_weights_gated(d1, q1, s1, None)).to(DEV)
+        ws1 = workspace(hq.hq_workspace_size(d1, t * k, tun))
+        hq.hq_grouped_gemm_moe_swiglu(d1, b1g, xs, off, t * k, h, ws1, tun)
+        assert hq.hq_check_device_status(ws1) == hq.HQ_OK
+    else:
+        c1 = _grouped(d1, b1, xs, off, t * k, 2 * inter, tun)
+        hq.hq_moe_swiglu(c1, t * k, inter, h)
     c2 = _grouped(d2, b2, h, off, t * k, hid, tun)
     out = torch.empty(t, hid, dtype=torch.bfloat16, device=DEV)
     ws = workspace(hq.hq_moe_combine_workspace_size(t, k))
@@ -354,7 +431,7 @@ def test_moe_layer_end_to_end(variant):
     assert hq.hq_check_device_status(ws) == hq.HQ_OK
     # oracle layer
     ref, ids_ref, off_ref, src_ref = _layer_oracle(_bits(x), logits.numpy(), q1.numpy(), s1.numpy(), q2.numpy(),
-                                                   s2.numpy(), k, e, inter)
+                                                   s2.numpy(), k, e, inter, fused)
     assert np.array_equal(ids.cpu().numpy(), ids_ref)
     assert np.array_equal(off.cpu().numpy(), off_ref) and np.array_equal(src.cpu().numpy(), src_ref)
-    check_gemm(out, ref, inter, f"moe layer variant={variant} (two-GEMM bar)", gemms=2)
+    check_gemm(out, ref, inter, f"moe layer variant={variant} fused={fused}")

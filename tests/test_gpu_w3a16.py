@@ -63,6 +63,19 @@ def test_dense_full_output(m, n, k, asym, tile_m, split_k):
     check_gemm(c, ref, k, f"w3a16 m={m} n={n} k={k} asym={asym} tile={tile_m} split={split_k}")
 
 
+@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("tile_m", [16, 32, 64])
+def test_small_tiles_both_variants(tile_m, variant):
+    """Tiles of up to 64 tokens: variant 1 (weights correctly rounded to
+    bf16, the rescaling kernel) and 2 (exact (q - z), per-group fp32 scale,
+    the library's default there), with zero points and a ragged tail."""
+    m, n, k = 2 * tile_m - 3, 384, 1408
+    d, blob, w = make(n, k, True, 9650 + tile_m + variant)
+    a = synth.bf16_normal(m, k, 9651 + tile_m)
+    c = run(d, blob, a, m, hq.Tuning(tile_m=tile_m, variant=variant))
+    check_gemm(c, G.w3a16_ref(_bits(a), *w, 128), k, f"w3a16 tile={tile_m} variant={variant}")
+
+
 @pytest.mark.parametrize("m,n,k", [(16, 18432, 7168), (4096, 7168, 7168)])
 def test_full_size_sampled(m, n, k):
     d, blob, w = make(n, k, False, 9300 + m)
