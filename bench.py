@@ -1,15 +1,20 @@
 """Benchmark of the fused-dequant low-bit GEMM path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload w4a16_sweep|moe|mxfp4|nvfp4]
+                    [--workload w4a16_sweep|moe|mxfp4|nvfp4|tiny|mxfp4_a16|w3a16|w2a16|w8a16|mxint4_a16]
+                    [--sweep-only]
 
 Default workload (one "step"): the dense W4A16 M-sweep, M in {1, 4, 16, 64,
 256, 1024, 4096} for (K, N) = (7168, 18432) and (18432, 7168), symmetric
 INT4, group 128, fp16 scales, bf16 activations: 14 GEMMs through the C ABI.
-`value` is the sweep's aggregate TFLOP/s (total FLOPs / total time).
+`value` is the sweep's aggregate TFLOP/s (total FLOPs / total time).  The
+same line then carries the rest of the metric, each timed the same way with
+its own roofline: the W4A8-MXFP4 GEMMs (`mxfp4_a8`), the NVFP4 W4A4 GEMMs
+(`nvfp4`), the MoE layer (`moe`, tok/s) and the tiny dense case (`tiny`,
+microseconds); --sweep-only leaves them out.
 
-Other workloads (--workload): the grouped MoE layer GEMMs (tok/s), the
-W4A8-MXFP4 GEMMs and the NVFP4 W4A4 GEMMs, each printed as its own line.
+Other workloads (--workload) print their own line: each of those, and the
+other weight formats on the W4A16 kernels.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronize, timed with CUDA events on the launching stream; weight
@@ -54,24 +59,27 @@ def load_peaks():
 
 # DRAM bytes (read + write) per launch of the sweep GEMMs, from one ncu
 # capture of the bench's first warm-up step (cold caches), recorded in
-# profiles/traffic_w4a16_sweep.md.  Emptied whenever the kernels change, so
-# that `traffic` reads null until the capture is taken again.
-TRAFFIC_BYTES = {
-    (1, 7168, 18432): 69719808,
-    (4, 7168, 18432): 68965120,
-    (16, 7168, 18432): 69436160,
-    (64, 7168, 18432): 70581760,
-    (256, 7168, 18432): 75671552,
-    (1024, 7168, 18432): 170001152,
-    (4096, 7168, 18432): 465380096,
-    (1, 18432, 7168): 69458176,
-    (4, 18432, 7168): 69744384,
-    (16, 18432, 7168): 70380288,
-    (64, 18432, 7168): 73538816,
-    (256, 18432, 7168): 85825024,
-    (1024, 18432, 7168): 196450304,
-    (4096, 18432, 7168): 715486464,
-}
+# profiles/traffic_w4a16_sweep.md with the commit it ran on.  The capture
+# holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
+# csrc/ and include/): once they change, `traffic` reads null until the
+# capture is taken again.
+TRAFFIC_COMMIT = None
+TRAFFIC_SOURCES = None
+TRAFFIC_BYTES = {}
+
+
+def kernel_sources_fingerprint():
+    """sha256 (first 16 hex digits) of the library's sources, in name order."""
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "quantized_gemm_bit_b200", "csrc", "*")))
+    files.append(os.path.join(ROOT, "include", "hq.h"))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def w4a16_bytes(m, k, n):
@@ -300,20 +308,23 @@ def run_w4a16_sweep(args, rank, world, peaks):
         # the dominant launch class: time-weighted over the given launches
         t = sum(e["us"] for e in entries)
         keys = [(e["m"], e["k"], e["n"]) for e in entries]
+        fresh = TRAFFIC_SOURCES is not None and TRAFFIC_SOURCES == kernel_sources_fingerprint()
         traffic = (round(sum(TRAFFIC_BYTES[x] for x in keys) / len(keys))
-                   if all(x in TRAFFIC_BYTES for x in keys) else None)
+                   if fresh and all(x in TRAFFIC_BYTES for x in keys) else None)
+        tinfo = dict(traffic_commit=TRAFFIC_COMMIT, traffic_sources=TRAFFIC_SOURCES,
+                     sources=kernel_sources_fingerprint())
         algo = round(sum(w4a16_bytes(*x) for x in keys) / len(keys))
         if bound == "hbm":
             ach = sum(w4a16_bytes(e["m"], e["k"], e["n"]) for e in entries) / (t * 1e-6) / 1e9
             return dict(bound="hbm", achieved=round(ach, 1), peak=peaks["hbm_gbs"], unit="GB/s",
                         frac=round(ach / peaks["hbm_gbs"], 3), traffic=traffic, algorithmic_bytes=algo,
                         launches=[f"M={e['m']},K={e['k']},N={e['n']}" for e in entries],
-                        peak_source=f"{peaks['source']} (copy bandwidth, burst)")
+                        peak_source=_peak_src(peaks, "hbm"), **tinfo)
         ach = sum(w4a16_flops(e["m"], e["k"], e["n"]) for e in entries) / (t * 1e-6) / 1e12
         return dict(bound="tensor", achieved=round(ach, 1), peak=peaks["bf16_tflops"], unit="TFLOP/s",
                     frac=round(ach / peaks["bf16_tflops"], 3), traffic=traffic, algorithmic_bytes=algo,
                     launches=[f"M={e['m']},K={e['k']},N={e['n']}" for e in entries],
-                    peak_source=f"{peaks['source']} (cuBLAS bf16 8192^3, burst)")
+                    peak_source=_peak_src(peaks, "bf16"), **tinfo)
 
     big = [e for e in sweep if e["m"] == 4096]
     small = [e for e in sweep if e["m"] <= 16]
@@ -357,6 +368,22 @@ def run_w4a16_sweep(args, rank, world, peaks):
 # ---------------------------------------------------------------- other workloads
 
 FP8_RATIO, FP4_RATIO = 2.0, 4.0   # nominal dense peaks relative to bf16 (4.5 / 9 vs 2.25 PF)
+
+
+def _peak_src(peaks, kind):
+    """Where a roofline denominator comes from."""
+    src = peaks["source"]
+    return {"hbm": f"{src} copy bandwidth (burst)",
+            "bf16": f"{src} cuBLAS bf16 8192^3 (burst)",
+            "fp8": f"{src} cuBLAS bf16 (burst) x nominal fp8/bf16 ratio 2 (4.5 / 2.25 PFLOP/s)",
+            "fp4": f"{src} cuBLAS bf16 (burst) x nominal fp4/bf16 ratio 4 (9 / 2.25 PFLOP/s)"}[kind]
+
+
+def _bound(flops, nbytes, tensor_peak_tflops, peaks):
+    """Which roofline a launch sits under (its arithmetic intensity against
+    the ridge point) and its fraction of that roofline."""
+    ridge = tensor_peak_tflops * 1e3 / peaks["hbm_gbs"]     # flop per byte
+    return {"bound": "hbm" if flops / nbytes < ridge else "tensor"}
 
 
 def _capture(fns, side):
@@ -457,12 +484,18 @@ def run_mxfp4(args, rank, world, peaks):
         fl = 2.0 * m * n * k
         by = n * k // 2 + n * k // 32 + m * k + 4 * m + 2 * m * n
         out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1), gbs=round(by / us / 1e3, 1),
-                        frac_fp8_peak=round(fl / us / 1e6 / peak, 3), frac_hbm=round(by / us / 1e3 / peaks["hbm_gbs"], 3)))
+                        frac_fp8_peak=round(fl / us / 1e6 / peak, 3), frac_hbm=round(by / us / 1e3 / peaks["hbm_gbs"], 3),
+                        **_bound(fl, by, peak, peaks)))
     flops = sum(2.0 * m * n * k for m in rows)
+    big = out[-1]
     return {"workload": "W4A8-MXFP4 GEMM, M in {16,256,4096}, K=N=7168", "value": round(flops * args.steps * world
             / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms / args.steps, 4),
-            "peak_fp8_tflops": round(peak, 1), "peak_source": "measured bf16 x nominal fp8/bf16 ratio 2",
-            "detail": out}
+            "peak_fp8_tflops": round(peak, 1), "peak_source": _peak_src(peaks, "fp8"),
+            "roofline": dict(bound="tensor", launch="M=4096", achieved=big["tflops"], peak=round(peak, 1),
+                             unit="TFLOP/s", frac=big["frac_fp8_peak"], peak_source=_peak_src(peaks, "fp8")),
+            "roofline_small_m": dict(bound="hbm", launch="M=16", achieved=out[0]["gbs"], peak=peaks["hbm_gbs"],
+                                     unit="GB/s", frac=out[0]["frac_hbm"], peak_source=_peak_src(peaks, "hbm")),
+            "gpu_launches": len(rows) * args.steps, "detail": out}
 
 
 def _run_w16_format(args, world, peaks, fmt):
@@ -484,6 +517,18 @@ def _run_w16_format(args, world, peaks, fmt):
         blob = torch.from_numpy(hq.hq_pack_weights(d, q, sc)).cuda()
         wbytes = 3 * n * k // 8 + 2 * n * (k // GROUP)
         name, dt = "INT3 weights (group 128) x bf16 activations", "bf16 x int3 (fp32 accumulate)"
+    elif fmt == "w8a16":
+        q, sc, _ = synth.w8a16_weights(n, k, 128, False, seed=7800)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT8, n, k, 128, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, q, sc)).cuda()
+        wbytes = n * k + 2 * n * (k // GROUP)
+        name, dt = "INT8 weights (group 128) x bf16 activations", "bf16 x int8 (fp32 accumulate)"
+    elif fmt == "mxint4_a16":
+        codes, e8 = synth.mxint4_weights(n, k, seed=7900)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_MXINT4, n, k, 32, 0, 1)
+        blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).cuda()
+        wbytes = n * k // 2 + n * k // 32
+        name, dt = "MXINT4 weights x bf16 activations", "bf16 x int4 e8m0-scaled (fp32 accumulate)"
     else:
         q, sc, _ = synth.w2a16_weights(n, k, 128, False, seed=7500)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, n, k, 128, 0, 1)
@@ -531,6 +576,14 @@ def run_w2a16(args, rank, world, peaks):
     return _run_w16_format(args, world, peaks, "w2a16")
 
 
+def run_w8a16(args, rank, world, peaks):
+    return _run_w16_format(args, world, peaks, "w8a16")
+
+
+def run_mxint4_a16(args, rank, world, peaks):
+    return _run_w16_format(args, world, peaks, "mxint4_a16")
+
+
 def run_nvfp4(args, rank, world, peaks):
     """NVFP4 W4A4: 8192^3 and M=16384, K=7168, N=18432 (inputs quantized from
     bf16 N(0,1) draws on the GPU by the library's own quantizer)."""
@@ -562,27 +615,37 @@ def run_nvfp4(args, rank, world, peaks):
     out = []
     for (m, n, k), us in zip(shapes, per):
         fl = 2.0 * m * n * k
-        out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1),
-                        frac_fp4_peak=round(fl / us / 1e6 / peak, 3)))
+        # codes + E4M3 block scales of both operands, the weights' tensor scale, bf16 C
+        by = (m + n) * k // 2 + (m + n) * k // 16 + 16 + 2 * m * n
+        out.append(dict(m=m, k=k, n=n, us=round(us, 2), tflops=round(fl / us / 1e6, 1), gbs=round(by / us / 1e3, 1),
+                        frac_fp4_peak=round(fl / us / 1e6 / peak, 3), **_bound(fl, by, peak, peaks)))
     flops = sum(2.0 * m * n * k for m, n, k in shapes)
+    t_all = sum(e["us"] for e in out)
+    ach = flops / (t_all * 1e-6) / 1e12
     return {"workload": "NVFP4 W4A4 GEMM, 8192^3 and M=16384 K=7168 N=18432", "value": round(
             flops * args.steps * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "ms_per_step": round(ms / args.steps, 4), "peak_fp4_tflops": round(peak, 1),
-            "peak_source": "measured bf16 x nominal fp4/bf16 ratio 4", "detail": out}
+            "peak_source": _peak_src(peaks, "fp4"),
+            "roofline": dict(bound="tensor", launch="both shapes (time-weighted)", achieved=round(ach, 1),
+                             peak=round(peak, 1), unit="TFLOP/s", frac=round(ach / peak, 3),
+                             peak_source=_peak_src(peaks, "fp4")),
+            "gpu_launches": 2 * len(shapes) * args.steps, "detail": out}
 
 
 def run_moe(args, rank, world, peaks):
     """MoE layer over the grouped W4A16 GEMMs: 256 experts, top-8, hidden
     7168, intermediate 2048 (gate+up N=4096, down K=2048), T in
     {64, 1024, 8192}: route (top-k + softmax weights) + permute/gather +
-    gate_up + SwiGLU + down + weighted combine."""
+    gate_up with SwiGLU in its epilogue + down + weighted combine."""
     from quantized_gemm_bit_b200 import hq, synth
     E, TOPK, H, I = 256, 8, 7168, 2048
     mats = {}
     for name, (n, k, seed) in {"gate_up": (2 * I, H, 3000), "down": (H, I, 3010)}.items():
         q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=seed, experts=E)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, E)
-        mats[name] = (d, torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).cuda(), n, k)
+        # gate+up in the gated row order: SwiGLU runs in that GEMM's epilogue
+        pack = hq.hq_pack_weights_gated if name == "gate_up" else hq.hq_pack_weights
+        mats[name] = (d, torch.from_numpy(pack(d, q, s, None)).cuda(), n, k)
         del q, s
     detail, launches, meta = [], [], []
     for t in (64, 1024, 8192):
@@ -594,7 +657,6 @@ def run_moe(args, rank, world, peaks):
         off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
         xs = torch.empty(t * TOPK, H, dtype=torch.bfloat16, device="cuda")
         pws = torch.zeros(hq.hq_moe_permute_workspace_size(t, TOPK, E), dtype=torch.uint8, device="cuda")
-        c1 = torch.empty(t * TOPK, 2 * I, dtype=torch.bfloat16, device="cuda")
         h = torch.empty(t * TOPK, I, dtype=torch.bfloat16, device="cuda")
         c2 = torch.empty(t * TOPK, H, dtype=torch.bfloat16, device="cuda")
         out = torch.empty(t, H, dtype=torch.bfloat16, device="cuda")
@@ -608,18 +670,15 @@ def run_moe(args, rank, world, peaks):
             hq.hq_moe_topk_softmax(logits, t, E, TOPK, ids, wts)
             hq.hq_moe_permute(ids, t, TOPK, E, src, off, pws, a=x, hidden=H, a_sorted=xs)
 
-        def g1(cp, t=t, xs=xs, off=off, c1=c1, ws1=ws1):
-            hq.hq_grouped_gemm_moe(d1, w1, xs, off, t * TOPK, c1, ws1)
-
-        def act(cp, t=t, c1=c1, h=h):
-            hq.hq_moe_swiglu(c1, t * TOPK, I, h)
+        def g1(cp, t=t, xs=xs, off=off, h=h, ws1=ws1):
+            hq.hq_grouped_gemm_moe_swiglu(d1, w1, xs, off, t * TOPK, h, ws1)
 
         def g2(cp, t=t, h=h, off=off, c2=c2, ws2=ws2):
             hq.hq_grouped_gemm_moe(d2, w2, h, off, t * TOPK, c2, ws2)
 
         def comb(cp, t=t, c2=c2, src=src, wts=wts, out=out, wsc=wsc):
             hq.hq_moe_combine(c2, src, wts, t, TOPK, H, out, wsc)
-        launches += [route, g1, act, g2, comb]
+        launches += [route, g1, g2, comb]
         meta.append((t, off, (ws1, ws2, wsc, pws)))
     ms, per = _time_launches(launches, args.steps, args.warmup, world)
     for (_, _, wss) in meta:
@@ -629,15 +688,15 @@ def run_moe(args, rank, world, peaks):
                 raise RuntimeError(f"device status after the MoE timing: {hq.status_string(st)}")
     tok_total = 0
     for i, (t, off, _) in enumerate(meta):
-        r_us, g1_us, a_us, g2_us, c_us = per[5 * i: 5 * i + 5]
+        r_us, g1_us, g2_us, c_us = per[4 * i: 4 * i + 4]
         offs = off.cpu().numpy()
         active = int((offs[1:] > offs[:-1]).sum())
         wbytes = active * (2 * I * H // 2 + 2 * I * (H // 128) * 2 + H * I // 2 + H * (I // 128) * 2)
         fl = 2.0 * t * TOPK * H * 3 * I
         gemm_us = g1_us + g2_us
-        layer_us = r_us + g1_us + a_us + g2_us + c_us
+        layer_us = r_us + g1_us + g2_us + c_us
         detail.append(dict(tokens=t, active_experts=active, route_permute_us=round(r_us, 2),
-                           gate_up_us=round(g1_us, 2), swiglu_us=round(a_us, 2), down_us=round(g2_us, 2),
+                           gate_up_swiglu_us=round(g1_us, 2), down_us=round(g2_us, 2),
                            combine_us=round(c_us, 2), tok_per_s=round(t / (layer_us * 1e-6), 1),
                            tok_per_s_gemms=round(t / (gemm_us * 1e-6), 1), tflops=round(fl / gemm_us / 1e6, 1),
                            weight_gbs=round(wbytes / gemm_us / 1e3, 1),
@@ -645,11 +704,48 @@ def run_moe(args, rank, world, peaks):
         tok_total += t
     # value: tokens of all three batches per step over the whole step (every
     # launch of the layer); the detail gives each batch alone
+    small = [x for x in detail if x["tokens"] <= 1024]
+    gb_small = sum(x["weight_gbs"] * (x["gate_up_swiglu_us"] + x["down_us"]) for x in small) / sum(
+        x["gate_up_swiglu_us"] + x["down_us"] for x in small)
+    big = [x for x in detail if x["tokens"] == 8192][0]
     return {"workload": "MoE layer over grouped W4A16 GEMMs: 256 experts, top-8, hidden 7168, intermediate 2048 "
                         "(gate+up N=4096, down K=2048), T in {64,1024,8192}; one step = route (top-k + softmax "
-                        "weights) + permute/gather + gate_up + SwiGLU + down + weighted combine for each T",
+                        "weights) + permute/gather + gate_up with fused SwiGLU + down + weighted combine for each T",
             "value": round(tok_total * args.steps * world / (ms * 1e-3), 1), "unit": "tok/s",
-            "ms_per_step": round(ms / args.steps, 4), "detail": detail}
+            "ms_per_step": round(ms / args.steps, 4),
+            "roofline": dict(bound="tensor", launch="T=8192 gate_up + down", achieved=big["tflops"],
+                             peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                             frac=round(big["tflops"] / peaks["bf16_tflops"], 3), peak_source=_peak_src(peaks, "bf16")),
+            "roofline_small_t": dict(bound="hbm", launch="T=64 and T=1024 gate_up + down (active-expert weights)",
+                                     achieved=round(gb_small, 1), peak=peaks["hbm_gbs"], unit="GB/s",
+                                     frac=round(gb_small / peaks["hbm_gbs"], 3), peak_source=_peak_src(peaks, "hbm")),
+            "gpu_launches": 9 * len(detail) * args.steps, "detail": detail}
+
+
+def run_tiny(args, rank, world, peaks):
+    """Dense W4A16 tiny: M=16, K=N=1024, asymmetric INT4 (zero points),
+    group 128: a latency-bound launch, reported in microseconds."""
+    from quantized_gemm_bit_b200 import hq, synth
+    m, n, k = 16, 1024, 1024
+    q, s, z = synth.w4a16_weights(n, k, GROUP, True, seed=0)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, GROUP, 1, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).cuda()
+    a = synth.bf16_normal(m, k, seed=1).cuda()
+    c = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(256, hq.hq_workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+
+    def f(cp):
+        hq.hq_gemm_w4a16(d, blob, a, m, c, ws)
+    ms, per = _time_launches([f], args.steps, args.warmup, world)
+    st = hq.hq_check_device_status(ws)
+    if st != hq.HQ_OK:
+        raise RuntimeError(f"device status after the tiny timing: {hq.status_string(st)}")
+    by = k * n // 2 + 2 * n * (k // GROUP) + n * (k // GROUP) + 2 * m * k + 2 * m * n
+    us = per[0]
+    return {"workload": "dense W4A16 tiny: M=16, K=N=1024, asymmetric INT4 group 128 (weights stay in L2)",
+            "value": round(us, 2), "unit": "us per launch", "higher_is_better": False,
+            "ms_per_step": round(ms / args.steps, 4), "gbs": round(by / us / 1e3, 1),
+            "algorithmic_bytes": by, "gpu_launches": args.steps}
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -719,9 +815,13 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="w4a16_sweep", choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "w3a16", "w2a16", "nvfp4", "moe"])
+    ap.add_argument("--workload", default="w4a16_sweep",
+                    choices=["w4a16_sweep", "mxfp4", "mxfp4_a16", "w3a16", "w2a16", "w8a16", "mxint4_a16", "nvfp4", "moe",
+                             "tiny"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-only", action="store_true",
+                    help="default workload: time the W4A16 sweep alone, without the FP4, MoE and tiny lines")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -741,9 +841,16 @@ def main():
     peaks = load_peaks()
     if args.workload == "w4a16_sweep":
         line = run_w4a16_sweep(args, rank, world, peaks)
+        if not args.sweep_only:
+            # the rest of the metric, each with its own roofline: the
+            # block-scaled GEMMs, the MoE layer and the tiny dense case
+            for key, fn in (("mxfp4_a8", run_mxfp4), ("nvfp4", run_nvfp4), ("moe", run_moe), ("tiny", run_tiny)):
+                torch.cuda.empty_cache()
+                line[key] = fn(args, rank, world, peaks)
     else:
-        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "w3a16": run_w3a16, "w2a16": run_w2a16, "nvfp4": run_nvfp4,
-              "moe": run_moe}[args.workload]
+        fn = {"mxfp4": run_mxfp4, "mxfp4_a16": run_mxfp4_a16, "w3a16": run_w3a16, "w2a16": run_w2a16,
+              "w8a16": run_w8a16, "mxint4_a16": run_mxint4_a16, "nvfp4": run_nvfp4, "moe": run_moe,
+              "tiny": run_tiny}[args.workload]
         line = {"metric": METRIC, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "data": "synthetic (seeded)"}
         line.update(fn(args, rank, world, peaks))
