@@ -116,7 +116,10 @@ typedef struct {
  *   tile_m   : token tile (the MMA N extent): 16, 32, 64, 128 or 256
  *   tile_n   : weight rows per tile: 128 (the only value)
  *   tile_k   : K per pipeline stage: 128 (fixed by the packed layout)
- *   stages   : 0 (the pipeline depth is fixed per token tile)
+ *   stages   : pipeline stages the producer keeps in flight (each a slot
+ *              of the kernel's shared-memory ring: one or two 128-K
+ *              records, or one or two block-scaled boxes); 0 = the whole
+ *              ring; larger than the ring = the whole ring
  *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
  *              splits the whole iteration space evenly when 0)
  *   cta_group: 1 (one SM per MMA)
@@ -143,6 +146,42 @@ typedef struct {
  * weight update); costs the overlap of the weight prefetch with that
  * kernel's tail. */
 #define HQ_TUNE_NO_EARLY_WEIGHTS 1
+
+/* A per-shape tuning table (the offline autotuner writes one): a call that
+ * passes no tuning (t == NULL) runs with the tuning of the first entry
+ * whose fmt, n, k and num_experts equal its descriptor's and whose
+ * [m_min, m_max] holds its m (total sorted rows for MoE), and with the
+ * library's rules otherwise.  The pages name heuristics that are not
+ * globally optimal and an autotuner on the roadmap ([vi] "stated
+ * limitations"; [fa] key points). */
+typedef struct {
+  int32_t fmt, n, k, num_experts;
+  int32_t m_min, m_max;
+  hq_tuning tuning;
+} hq_tuning_entry;
+
+/* Replaces the process-wide table with a copy of entries[0 .. count)
+ * (count 0 clears it).  Every entry's tuning is checked as the matching
+ * entry point would check it; on an error the table is left as it was.
+ * Safe to call from any thread; calls running concurrently see the old or
+ * the new table. */
+hq_status hq_tuning_table_set(const hq_tuning_entry* entries, int32_t count);
+
+/* The launch plan a call would run (tuning t, else the table, else the
+ * rules), without a GPU if none is current (148 SMs assumed, as for
+ * hq_workspace_size). */
+typedef struct {
+  int32_t kernel;      /* 1: W4A16 weights rescaled to bf16, 2: W4A16 exact weights, 3: block-scaled */
+  int32_t tile_m;      /* token tile                                                                 */
+  int32_t grid;        /* CTAs                                                                       */
+  int32_t split;       /* 0: whole tiles; >0: tiles share their K range (stream-K or a K split)      */
+  int32_t whole_tiles; /* dense W4A16 split plans: tiles run whole before the shared tail            */
+  int32_t stages;      /* pipeline stages in flight                                                  */
+  int32_t ring_stages; /* the kernel's shared-memory ring depth                                      */
+  int32_t from_table;  /* 1 when the tuning came from the table                                      */
+  size_t workspace_bytes;
+} hq_plan;
+hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t, hq_plan* out);
 
 /* Library and layout version. */
 int hq_layout_version(void);

@@ -17,11 +17,17 @@ CUDA graph of back-to-back launches over weight copies rotating across more
 than 3x L2, timed with CUDA events; candidates the library refuses are
 skipped, and a candidate whose run records a device-side error is an error.
 The result is a table sorted by time plus the best tuning and its speed-up
-over the library's choice: one entry of a per-shape heuristic table.
+over the library's choice: one entry of a per-shape heuristic table.  With
+--table PATH the entry is merged into a JSON table file, which load_table()
+installs in the library (hq_tuning_table_set): calls of that shape that pass
+no tuning then run the table's plan.
+
+    python -m quantized_gemm_bit_b200.autotune --kind w4a16 --m 16 --table tuning.json --m-range 1,16
 """
 
 import argparse
 import json
+import os
 
 import torch
 
@@ -30,14 +36,19 @@ from . import hq, synth
 TILES = (16, 32, 64, 128, 256)
 
 
+STAGES = (0, 2, 4)
+
+
 def candidates(kind, m):
     """Tunings worth trying at m rows: token tiles up to twice the rows
-    (at least 16), K splits 0 (the library's choice) to 3, and for the
-    W4A16 kernels with INT4, INT3 or INT2 weights both weight variants
-    (MXFP4 weights have only the rescaled one)."""
+    (at least 16), K splits 0 (the library's choice) to 3, pipeline stages
+    in flight (0 = the kernel's whole ring, 2, 4), and for the W4A16 kernels
+    with INT4, INT3, INT2 or INT8 weights both weight variants (the MX
+    formats have only the rescaled one)."""
     cap = max(16, 2 * m)
     tiles = [t for t in TILES if t <= cap] or [16]
-    variants = (1, 2) if kind in ("w4a16", "moe", "w3a16", "w2a16") else (1,) if kind == "mxfp4_a16" else (0,)
+    variants = ((1, 2) if kind in ("w4a16", "moe", "w3a16", "w2a16", "w8a16")
+                else (1,) if kind in ("mxfp4_a16", "mxint4_a16") else (0,))
     splits = (0,) if kind == "moe" else (0, 1, 2, 3)
     out = [None]
     for t in tiles:
@@ -45,12 +56,46 @@ def candidates(kind, m):
             for v in variants:
                 if v == 2 and t > 64:
                     continue
-                out.append(hq.Tuning(tile_m=t, split_k=s, variant=v))
+                for st in STAGES:
+                    out.append(hq.Tuning(tile_m=t, split_k=s, variant=v, stages=st))
     return out
 
 
 def _describe(t):
-    return "library" if t is None else f"tile_m={t.tile_m} split_k={t.split_k} variant={t.variant}"
+    return ("library" if t is None
+            else f"tile_m={t.tile_m} split_k={t.split_k} variant={t.variant} stages={t.stages}")
+
+
+def _tuning_dict(t):
+    return {f: int(getattr(t, f)) for f, _ in hq.Tuning._fields_}
+
+
+def table_entry(d, m_min, m_max, t):
+    """One entry of the per-shape table (a dict, as the JSON file holds it)."""
+    return {"fmt": int(d.fmt), "n": int(d.n), "k": int(d.k), "num_experts": int(d.num_experts),
+            "m_min": int(m_min), "m_max": int(m_max), "tuning": _tuning_dict(t)}
+
+
+def merge_table(path, entry):
+    """Add `entry` to the JSON table at `path`, replacing an entry of the
+    same shape and m range."""
+    table = {"entries": []}
+    if os.path.exists(path):
+        with open(path) as f:
+            table = json.load(f)
+    key = lambda e: (e["fmt"], e["n"], e["k"], e["num_experts"], e["m_min"], e["m_max"])
+    table["entries"] = [e for e in table["entries"] if key(e) != key(entry)] + [entry]
+    with open(path, "w") as f:
+        json.dump(table, f, indent=1)
+    return table
+
+
+def load_table(path):
+    """Install the JSON table at `path` in the library (hq_tuning_table_set)."""
+    with open(path) as f:
+        table = json.load(f)
+    hq.hq_tuning_table_set(table["entries"])
+    return table
 
 
 def _time(fn, ncopy, reps=3):
@@ -97,10 +142,13 @@ def _setup(kind, m, n, k, experts, topk, dev):
 
         def call(t, i, c, ws):
             hq.hq_gemm_w4a16(d, blobs[i], a, m, c, ws, t)
-    elif kind in ("w3a16", "w2a16"):
+    elif kind in ("w3a16", "w2a16", "w8a16"):
         if kind == "w3a16":
             q, s, _ = synth.w3a16_weights(n, k, 128, False, seed=7000)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
+        elif kind == "w8a16":
+            q, s, _ = synth.w8a16_weights(n, k, 128, False, seed=7800)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT8, n, k, 128, 0, 1)
         else:
             q, s, _ = synth.w2a16_weights(n, k, 128, False, seed=7500)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, n, k, 128, 0, 1)
@@ -110,9 +158,10 @@ def _setup(kind, m, n, k, experts, topk, dev):
 
         def call(t, i, c, ws):
             hq.hq_gemm_w4a16(d, blobs[i], a, m, c, ws, t)
-    elif kind == "mxfp4_a16":
-        codes, e8 = synth.mxfp4_weights(n, k, seed=6000)
-        d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, n, k, 32, 0, 1)
+    elif kind in ("mxfp4_a16", "mxint4_a16"):
+        mxi = kind == "mxint4_a16"
+        codes, e8 = (synth.mxint4_weights if mxi else synth.mxfp4_weights)(n, k, seed=6000)
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_MXINT4 if mxi else hq.HQ_FMT_MXFP4_A16, n, k, 32, 0, 1)
         blobs = _copies(torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(dev))
         a = synth.bf16_normal(m, k, seed=6001).to(dev)
         rows = m
@@ -190,28 +239,34 @@ def autotune(kind, m, n, k, experts=256, topk=8, tunings=None, dev="cuda"):
         results.append({"tuning": t, "us": us, "desc": _describe(t)})
     results.sort(key=lambda r: r["us"])
     library = next(r for r in results if r["tuning"] is None)
-    return results, results[0], library
+    return results, results[0], library, d, rows
 
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "w2a16", "mxfp4_a16", "mxfp4", "nvfp4", "moe"])
+    ap.add_argument("--kind", default="w4a16",
+                    choices=["w4a16", "w3a16", "w2a16", "w8a16", "mxfp4_a16", "mxint4_a16", "mxfp4", "nvfp4", "moe"])
     ap.add_argument("--m", type=int, default=16, help="rows (tokens for --kind moe)")
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)
     ap.add_argument("--experts", type=int, default=256)
     ap.add_argument("--topk", type=int, default=8)
+    ap.add_argument("--table", default=None, help="merge the best tuning into this JSON table file")
+    ap.add_argument("--m-range", default=None, help="lo,hi: the rows the table entry applies to (default m,m)")
     a = ap.parse_args(argv)
     from .build import build
     build()
-    results, best, library = autotune(a.kind, a.m, a.n, a.k, a.experts, a.topk)
+    results, best, library, d, rows = autotune(a.kind, a.m, a.n, a.k, a.experts, a.topk)
     for r in results:
         print(f"{r['us']:10.2f} us  {r['desc']}")
     t = best["tuning"]
     print(json.dumps({"kind": a.kind, "m": a.m, "n": a.n, "k": a.k,
-                      "best": None if t is None else {"tile_m": t.tile_m, "split_k": t.split_k, "variant": t.variant},
+                      "best": None if t is None else _tuning_dict(t),
                       "best_us": round(best["us"], 2), "library_us": round(library["us"], 2),
                       "speedup_over_library": round(library["us"] / best["us"], 3)}))
+    if a.table and t is not None:
+        lo, hi = (rows, rows) if a.m_range is None else (int(x) for x in a.m_range.split(","))
+        merge_table(a.table, table_entry(d, lo, hi, t))
 
 
 if __name__ == "__main__":

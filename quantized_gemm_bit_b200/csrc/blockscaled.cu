@@ -109,6 +109,7 @@ struct BsParams {
   int m_tiles;
   int data_parallel;         // whole tiles per unit, no partial sums
   int early_weights;         // fetch the first stages' weights before griddepcontrol.wait
+  int stage_limit;           // pipeline stages in flight (0 or >= the ring depth: the whole ring)
 };
 
 // NVFP4 activation scales, row-major [m][K/16] bytes, re-laid into the order
@@ -309,10 +310,11 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     // Phase 1, before the previous kernel on the stream has finished: the
     // packed weights of the first S stages (no kernel writes them)
     uint32_t n_pre = 0;
-    for (int idx = 0; p.early_weights && n_pre < (uint32_t)S &&
+    const uint32_t depth = (p.stage_limit > 0 && p.stage_limit < S) ? (uint32_t)p.stage_limit : (uint32_t)S;
+    for (int idx = 0; p.early_weights && n_pre < depth &&
                       bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
          ++idx) {
-      for (int ks = ks0; ks < ks1 && n_pre < (uint32_t)S; ++ks, ++n_pre) {
+      for (int ks = ks0; ks < ks1 && n_pre < depth; ++ks, ++n_pre) {
         if (leader) {
           mbar_arrive_expect_tx(&full[n_pre], stage_tx(stage_boxes(ks)));
           load_weights((int)n_pre, ks, nt);
@@ -328,7 +330,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       for (int ks = ks0; ks < ks1; ++ks, ++it) {
         const int s = it % S;
         const uint32_t ph = (it / S) & 1;
-        if (it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+        if ((it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) ||
+            !throttle_stages<S>(empty, it, p.stage_limit, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -555,7 +558,11 @@ int bs_tiles(const hq_quant_desc& d, int m, int ntok) {
 
 BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t) {
   BsConfig cfg{};
+  // no tuning from the caller: the caller's per-shape table first, then the rules below
+  hq_tuning from_table;
+  if (!t) t = tuning_from_table(d, m, &from_table);
   cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
+  cfg.stages = t ? t->stages : 0;
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
   auto dp_eff = [&](int nt) {
@@ -628,6 +635,17 @@ BsWsLayout bs_ws_layout(const hq_quant_desc& d, int m, const BsConfig& cfg) {
   return L;
 }
 
+int bs_ring_depth(const hq_quant_desc& d, const BsConfig& cfg) {
+  const bool nv = d.fmt == HQ_FMT_NVFP4;
+  switch (cfg.ntok) {
+    case 16: return nv ? BsCfg<kNV, 16>::kStages : BsCfg<kMX, 16>::kStages;
+    case 32: return nv ? BsCfg<kNV, 32>::kStages : BsCfg<kMX, 32>::kStages;
+    case 64: return nv ? BsCfg<kNV, 64>::kStages : BsCfg<kMX, 64>::kStages;
+    case 128: return nv ? BsCfg<kNV, 128>::kStages : BsCfg<kMX, 128>::kStages;
+    default: return nv ? BsCfg<kNV, 256>::kStages : BsCfg<kMX, 256>::kStages;
+  }
+}
+
 size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg) {
   return bs_ws_layout(d, m, cfg).total;
 }
@@ -659,6 +677,7 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.m_tiles = (m + cfg.ntok - 1) / cfg.ntok;
   p.data_parallel = cfg.splits == 0 ? 1 : 0;
   p.early_weights = cfg.early_weights;
+  p.stage_limit = cfg.stages;
   const BsWsLayout L = bs_ws_layout(d, m, cfg);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.counters = reinterpret_cast<int32_t*>(wsb + L.counters);

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "hq_internal.h"
 
@@ -104,7 +105,7 @@ hq_status check_w4_tuning(const hq_quant_desc* d, const hq_tuning* t, bool group
   if (!t) return HQ_OK;
   if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
     return HQ_ERR_UNSUPPORTED;
-  if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages != 0 ||
+  if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages < 0 ||
       (t->cta_group && t->cta_group != 1) || t->variant < 0 || t->variant > 2 ||
       (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
     return HQ_ERR_UNSUPPORTED;
@@ -116,6 +117,24 @@ hq_status check_w4_tuning(const hq_quant_desc* d, const hq_tuning* t, bool group
 }
 
 }  // namespace
+
+// ---- the caller's per-shape tuning table
+namespace {
+std::mutex g_table_mu;
+std::vector<hq_tuning_entry> g_table;
+}  // namespace
+
+const hq_tuning* tuning_from_table(const hq_quant_desc& d, int m, hq_tuning* tmp) {
+  std::lock_guard<std::mutex> lock(g_table_mu);
+  for (const hq_tuning_entry& e : g_table) {
+    if (e.fmt == d.fmt && e.n == d.n && e.k == d.k && e.num_experts == d.num_experts && m >= e.m_min &&
+        m <= e.m_max) {
+      *tmp = e.tuning;
+      return tmp;
+    }
+  }
+  return nullptr;
+}
 
 hq_status check_w4_call(const hq_quant_desc* d, const hq_tuning* t, bool grouped) {
   hq_status st = check_desc(d);
@@ -293,7 +312,7 @@ hq_status check_bs_tuning(const hq_tuning* t) {
   if (!t) return HQ_OK;
   if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
     return HQ_ERR_UNSUPPORTED;
-  if ((t->tile_n && t->tile_n != 128) || t->tile_k || t->split_k < 0 || t->stages != 0 ||
+  if ((t->tile_n && t->tile_n != 128) || t->tile_k || t->split_k < 0 || t->stages < 0 ||
       (t->cta_group && t->cta_group != 1) || t->variant != 0 || (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
     return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
@@ -450,6 +469,67 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
   if (st != HQ_OK) return st;
   return moe_permute_launch(topk_ids_dev, t, k, e, sorted_src_dev, expert_offsets_dev, a_dev, hidden, a_sorted_dev,
                             ws_dev, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hq_status hq_tuning_table_set(const hq_tuning_entry* entries, int32_t count) {
+  if (count < 0 || (count > 0 && !entries)) return HQ_ERR_INVALID_ARG;
+  std::vector<hq_tuning_entry> next(entries, entries + count);
+  // every entry must be a tuning the matching entry point accepts
+  for (const hq_tuning_entry& e : next) {
+    if (e.m_min < 0 || e.m_max < e.m_min) return HQ_ERR_INVALID_ARG;
+    hq_quant_desc d{};
+    hq_status st = hq_quant_desc_init(&d, e.fmt, e.n, e.k, e.fmt == HQ_FMT_INT4 || e.fmt == HQ_FMT_INT3 ||
+                                                               e.fmt == HQ_FMT_INT2 || e.fmt == HQ_FMT_INT8
+                                                           ? 128
+                                                           : e.fmt == HQ_FMT_NVFP4 ? 16 : 32,
+                                      0, e.num_experts);
+    if (st != HQ_OK) return st;
+    st = w4_format(&d) ? check_w4_tuning(&d, &e.tuning, d.num_experts > 1) : check_bs_tuning(&e.tuning);
+    if (st != HQ_OK) return st;
+  }
+  std::lock_guard<std::mutex> lock(g_table_mu);
+  g_table.swap(next);
+  return HQ_OK;
+}
+
+hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t, hq_plan* out) {
+  hq_status st = check_desc(d);
+  if (st != HQ_OK) return st;
+  if (!out || m < 1) return HQ_ERR_INVALID_ARG;
+  const bool w16 = w4_format(d);
+  st = w16 ? check_w4_tuning(d, t, d->num_experts > 1) : check_bs_tuning(t);
+  if (st != HQ_OK) return st;
+  DeviceInfo dev{};
+  if (device_info(&dev) != HQ_OK) dev.num_sms = 148;   // as hq_workspace_size
+  hq_tuning tmp;
+  hq_plan p{};
+  p.from_table = (!t && tuning_from_table(*d, m, &tmp)) ? 1 : 0;
+  if (w16) {
+    const bool grouped = d->num_experts > 1;
+    const W4Config cfg = w4_plan(dev, *d, m, grouped, t);
+    const int depth = w4_ring_depth(*d, cfg);
+    const bool mx = d->fmt == HQ_FMT_MXFP4_A16 || d->fmt == HQ_FMT_MXINT4;
+    p.tile_m = cfg.ntok;
+    p.grid = cfg.grid;
+    p.split = grouped ? 0 : cfg.splits == 0 ? 0 : cfg.splits;
+    p.whole_tiles = grouped ? 0 : cfg.dp_tiles;
+    p.kernel = (!mx && cfg.ntok <= 64 && cfg.variant != 1) ? 2 : 1;
+    p.ring_stages = depth;
+    p.stages = (cfg.stages > 0 && cfg.stages < depth) ? cfg.stages : depth;
+    p.workspace_bytes = w4_workspace_bytes(*d, m, cfg, grouped);
+  } else {
+    const BsConfig cfg = bs_plan(dev, *d, m, t);
+    const int depth = bs_ring_depth(*d, cfg);
+    p.tile_m = cfg.ntok;
+    p.grid = cfg.grid;
+    p.split = cfg.splits;
+    p.kernel = 3;
+    p.ring_stages = depth;
+    p.stages = (cfg.stages > 0 && cfg.stages < depth) ? cfg.stages : depth;
+    p.workspace_bytes = bs_workspace_bytes(*d, m, cfg);
+  }
+  *out = p;
+  return HQ_OK;
 }
 
 hq_status hq_check_device_status(void* ws_dev, hq_stream_t stream) {

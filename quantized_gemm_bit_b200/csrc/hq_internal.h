@@ -42,7 +42,7 @@ constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per wait
 // Resolved launch configuration of the W4A16 kernel family.
 struct W4Config {
   int ntok;     // token tile (MMA N)
-  int stages;   // unused (pipeline depth is fixed per token tile)
+  int stages;   // pipeline stages the producer keeps in flight, 0 = the kernel's ring depth
   int splits;   // 0: data parallel (whole tiles); else stream-K / split K
   int dp_tiles; // stream-K plans: tiles run whole before the shared K range
   int grid;     // CTAs
@@ -60,6 +60,11 @@ struct DeviceInfo {
   size_t max_smem_optin;
 };
 hq_status device_info(DeviceInfo* out);
+
+// The caller's tuning table (hq_tuning_table_set): the tuning of the first
+// entry matching (fmt, n, k, num_experts) with m in [m_min, m_max], copied
+// into *tmp, or nullptr.
+const hq_tuning* tuning_from_table(const hq_quant_desc& d, int m, hq_tuning* tmp);
 
 // Descriptor, format and tuning checks of a W4A16-family call (INT4, INT3,
 // INT2 or MXFP4_A16 weights; grouped: num_experts >= 2, else exactly 1).
@@ -81,12 +86,17 @@ struct BsConfig {
   int ntok;
   int splits;   // 0: whole tiles per CTA (no partial sums)
   int grid;
+  int stages;   // pipeline stages the producer keeps in flight, 0 = the kernel's ring depth
   int early_weights;  // fetch packed weights before the previous kernel completes
 };
 BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t);
 size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg);
 hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* packed, const void* a, const void* a_sf,
                     const float* a_scale, float a_global, int m, void* c, void* ws, cudaStream_t stream);
+
+// Ring depth (SMEM pipeline stages) of the kernel a plan launches.
+int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg);
+int bs_ring_depth(const hq_quant_desc& d, const BsConfig& cfg);
 
 // Activation quantizers.
 size_t nvfp4_quant_ws_bytes(int rows, int k);

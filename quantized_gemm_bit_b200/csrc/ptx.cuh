@@ -120,6 +120,19 @@ __device__ __forceinline__ bool hq_wait_warp(uint64_t* bar, uint32_t parity, uin
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// Producer: before issuing iteration `it`, wait until iteration
+// it - limit has been consumed, so that at most `limit` stages are in
+// flight (limit < SS).  Its slot is next refilled at it - limit + SS > it,
+// so the slot's empty barrier cannot have moved past that phase: the parity
+// wait is exact.  Returns false when the bounded wait gave up.
+template <int SS>
+__device__ __forceinline__ bool throttle_stages(uint64_t* empty, uint32_t it, int limit, uint64_t wait_ns,
+                                                volatile int* abort) {
+  if (limit <= 0 || limit >= SS || it < (uint32_t)limit) return true;
+  const uint32_t j = it - (uint32_t)limit;
+  return hq_wait_warp(&empty[j % SS], (j / SS) & 1, wait_ns, abort);
+}
+
 // ---------------------------------------------------------------- copies
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes).
 __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar,

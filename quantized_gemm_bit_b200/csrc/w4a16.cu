@@ -409,11 +409,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // of the first SS stages (no kernel writes them)
     uint32_t n_pre = 0;
     if (!p.grouped) {
-      for (int idx = 0; p.early_weights && n_pre < (uint32_t)SS &&
-                        get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
+      const uint32_t depth = (p.stage_limit > 0 && p.stage_limit < SS) ? (uint32_t)p.stage_limit : (uint32_t)SS;
+      for (int idx = 0; p.early_weights && n_pre < depth && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
            ++idx) {
         const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
-        for (int kb = x.kb0; kb < x.kb1 && n_pre < (uint32_t)SS; kb += KPS, ++n_pre) {
+        for (int kb = x.kb0; kb < x.kb1 && n_pre < depth; kb += KPS, ++n_pre) {
           const int nrec = min(KPS, x.kb1 - kb);
           if (leader) {
             uint64_t* fb = full_bar(n_pre);
@@ -436,7 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % SS;
         const uint32_t ph = (it / SS) & 1;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) {
+        if ((it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) ||
+            !throttle_stages<SS>(empty, it, p.stage_limit, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -653,6 +654,9 @@ int dense_tiles(const hq_quant_desc& d, int m, int ntok) {
 
 W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t) {
   W4Config cfg{};
+  // no tuning from the caller: the caller's per-shape table first, then the rules below
+  hq_tuning from_table;
+  if (!t) t = tuning_from_table(d, m, &from_table);
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) {
     if (grouped) {
@@ -669,7 +673,7 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
       ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
     }
   }
-  cfg.stages = 0;
+  cfg.stages = t ? t->stages : 0;
   cfg.splits = 1;
   cfg.variant = t ? t->variant : 0;
   cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
@@ -737,6 +741,33 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   return cfg;
 }
 
+namespace {
+template <int FMT>
+int rescaled_depth(int ntok) {
+  switch (ntok) {
+    case 16: return Cfg<16, FMT>::kSmemStages;
+    case 32: return Cfg<32, FMT>::kSmemStages;
+    case 64: return Cfg<64, FMT>::kSmemStages;
+    case 128: return Cfg<128, FMT>::kSmemStages;
+    default: return Cfg<256, FMT>::kSmemStages;
+  }
+}
+}  // namespace
+
+int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg) {
+  const bool mx = d.fmt == HQ_FMT_MXFP4_A16, mxi4 = d.fmt == HQ_FMT_MXINT4;
+  const int kfmt = d.fmt == HQ_FMT_INT3 ? kFmtInt3 : d.fmt == HQ_FMT_INT2 ? kFmtInt2 : d.fmt == HQ_FMT_INT8 ? kFmtInt8 : kFmtInt4;
+  if (!mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1) return small_ring_depth(cfg.ntok, kfmt);
+  if (mx) return rescaled_depth<kFmtMx>(cfg.ntok);
+  if (mxi4) return rescaled_depth<kFmtMxi4>(cfg.ntok);
+  switch (kfmt) {
+    case kFmtInt3: return rescaled_depth<kFmtInt3>(cfg.ntok);
+    case kFmtInt2: return rescaled_depth<kFmtInt2>(cfg.ntok);
+    case kFmtInt8: return rescaled_depth<kFmtInt8>(cfg.ntok);
+    default: return rescaled_depth<kFmtInt4>(cfg.ntok);
+  }
+}
+
 W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4Config cfg) {
   cfg.splits = 0;
   cfg.dp_tiles = 0;
@@ -785,6 +816,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.wait_ns = kDefaultWaitNs;
   p.early_weights = cfg.early_weights;
   p.swiglu = swiglu;
+  p.stage_limit = cfg.stages;
   if (grouped) {
     // an expert's weight tile is re-read by each of its token tiles
     p.weights_once = (long long)m <= (long long)cfg.ntok * d.num_experts ? 1 : 0;

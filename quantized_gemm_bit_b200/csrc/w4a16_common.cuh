@@ -62,7 +62,10 @@ struct W4Params {
   int data_parallel;                 // dense: whole tiles per unit, no partials
   int early_weights;                 // dense: fetch the first stages' weights before griddepcontrol.wait
   int swiglu;                        // grouped: gated gate+up weights, write h = silu(gate) * up [rows][n/2]
+  int stage_limit;                   // pipeline stages in flight (0 or >= the ring depth: the whole ring)
 };
+
+
 
 // One unit of work: a K range of one (expert, token tile, weight tile).
 struct Unit {
@@ -256,8 +259,9 @@ __device__ __noinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, i
   if (lane == 0) p.counters[x.tile * 4 + q] = 0;  // leave the workspace zeroed
 }
 
-// Host side: launch the exact-weight kernel (16, 32 or 64 tokens; INT4,
-// INT3 or INT2 records).
+// Host side: the exact-weight kernel's ring depth, and its launch (16, 32 or
+// 64 tokens; INT4, INT3, INT2 or INT8 records).
+int small_ring_depth(int ntok, int fmt);
 hq_status small_launch(int ntok, int fmt, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream);
 
 }  // namespace w4

@@ -257,11 +257,11 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
     // of the first SS stages (no kernel writes them)
     uint32_t n_pre = 0;
     if (!p.grouped) {
-      for (int idx = 0; p.early_weights && n_pre < (uint32_t)SS &&
-                        get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
+      const uint32_t depth = (p.stage_limit > 0 && p.stage_limit < SS) ? (uint32_t)p.stage_limit : (uint32_t)SS;
+      for (int idx = 0; p.early_weights && n_pre < depth && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
            ++idx) {
         const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
-        for (int kb = x.kb0; kb < x.kb1 && n_pre < (uint32_t)SS; kb += KPS, ++n_pre) {
+        for (int kb = x.kb0; kb < x.kb1 && n_pre < depth; kb += KPS, ++n_pre) {
           const int nrec = min(KPS, x.kb1 - kb);
           if (leader) {
             uint64_t* fb = full_bar(n_pre);
@@ -283,7 +283,8 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (it >= n_pre && !hq_wait_warp(&empty[s], ((it / SS) & 1) ^ 1, p.wait_ns, s_abort)) {
+        if ((it >= n_pre && !hq_wait_warp(&empty[s], ((it / SS) & 1) ^ 1, p.wait_ns, s_abort)) ||
+            !throttle_stages<SS>(empty, it, p.stage_limit, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -519,6 +520,23 @@ hq_status small_launch_f(int ntok, const CUtensorMap& map, const W4Params& p, in
 }
 
 }  // namespace
+
+namespace {
+template <int FMT>
+int small_depth_f(int ntok) {
+  return ntok == 16 ? SmallCfg<16, FMT>::kSmemStages : ntok == 32 ? SmallCfg<32, FMT>::kSmemStages
+                                                                  : SmallCfg<64, FMT>::kSmemStages;
+}
+}  // namespace
+
+int small_ring_depth(int ntok, int fmt) {
+  switch (fmt) {
+    case kFmtInt3: return small_depth_f<kFmtInt3>(ntok);
+    case kFmtInt2: return small_depth_f<kFmtInt2>(ntok);
+    case kFmtInt8: return small_depth_f<kFmtInt8>(ntok);
+    default: return small_depth_f<kFmtInt4>(ntok);
+  }
+}
 
 hq_status small_launch(int ntok, int fmt, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
   switch (fmt) {

@@ -48,7 +48,7 @@ EXPORTS = (
     "hq_moe_permute_workspace_size", "hq_moe_permute", "hq_grouped_gemm_moe", "hq_moe_swiglu",
     "hq_moe_combine_workspace_size", "hq_moe_combine", "hq_check_device_status",
     "hq_debug_timeout_probe", "hq_gemm_w4a16_static", "hq_static_check_device_status",
-    "hq_pack_weights_gated", "hq_grouped_gemm_moe_swiglu",
+    "hq_pack_weights_gated", "hq_grouped_gemm_moe_swiglu", "hq_tuning_table_set", "hq_plan_describe",
 )
 
 
@@ -63,6 +63,17 @@ class Tuning(ctypes.Structure):
 
 
 HQ_TUNE_NO_EARLY_WEIGHTS = 1
+
+
+class TuningEntry(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in ("fmt", "n", "k", "num_experts", "m_min", "m_max")] + \
+               [("tuning", Tuning)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int32) for f in
+                ("kernel", "tile_m", "grid", "split", "whole_tiles", "stages", "ring_stages", "from_table")] + \
+               [("workspace_bytes", ctypes.c_size_t)]
 
 
 class HQError(RuntimeError):
@@ -112,6 +123,8 @@ def lib():
             "hq_static_check_device_status": (st, [vp]),
             "hq_pack_weights_gated": (st, [dp, vp, vp, vp, vp, sz]),
             "hq_grouped_gemm_moe_swiglu": (st, [dp, vp, vp, vp, i32, vp, tp, vp, sz, vp]),
+            "hq_tuning_table_set": (st, [ctypes.POINTER(TuningEntry), i32]),
+            "hq_plan_describe": (st, [dp, i32, tp, ctypes.POINTER(Plan)]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -310,3 +323,24 @@ def hq_static_check_device_status(stream=None):
     """First device-side error of the allocation-free calls since the last
     read (HQ_OK when none); synchronizes the stream."""
     return int(lib().hq_static_check_device_status(_stream(stream)))
+
+
+def hq_tuning_table_set(entries):
+    """Install a per-shape tuning table: a list of TuningEntry (or dicts with
+    fmt, n, k, num_experts, m_min, m_max and tuning fields)."""
+    ents = []
+    for e in entries:
+        if isinstance(e, dict):
+            t = Tuning(**{f: int(e.get("tuning", {}).get(f, 0)) for f, _ in Tuning._fields_})
+            e = TuningEntry(int(e["fmt"]), int(e["n"]), int(e["k"]), int(e.get("num_experts", 1)),
+                            int(e["m_min"]), int(e["m_max"]), t)
+        ents.append(e)
+    arr = (TuningEntry * max(1, len(ents)))(*ents)
+    _check(lib().hq_tuning_table_set(arr, len(ents)), "hq_tuning_table_set")
+
+
+def hq_plan_describe(desc, m, tuning=None):
+    """The launch plan a call with these arguments would run (a Plan)."""
+    out = Plan()
+    _check(lib().hq_plan_describe(ctypes.byref(desc), int(m), _tuning(tuning), ctypes.byref(out)), "hq_plan_describe")
+    return out

@@ -241,7 +241,7 @@ def test_gemm_argument_errors_need_no_gpu():
     t = hq.Tuning(tile_m=48)
     assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                             None) == hq.HQ_ERR_UNSUPPORTED
-    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=3), hq.Tuning(cta_group=2),
+    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=-1), hq.Tuning(cta_group=2),
                 hq.Tuning(flags=2)):
         assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
                                 None) == hq.HQ_ERR_UNSUPPORTED
@@ -315,6 +315,7 @@ def test_autotune_candidates_need_no_gpu():
     assert all(t.variant == 0 for t in autotune.candidates("nvfp4", 256)[1:])
     assert all(t.variant == 1 for t in autotune.candidates("mxfp4_a16", 16)[1:])
     assert {t.variant for t in autotune.candidates("w3a16", 64)[1:]} == {1, 2}
+    assert {t.stages for t in autotune.candidates("w4a16", 16)[1:]} == set(autotune.STAGES)
     assert {t.variant for t in autotune.candidates("w2a16", 16)[1:]} == {1, 2}
     assert all(t.split_k == 0 for t in autotune.candidates("moe", 64)[1:])
 
@@ -413,3 +414,53 @@ def test_mxint4_pack_rejects_scales_that_overflow_bf16_and_descriptor_rules():
     t = hq.Tuning(variant=2)
     assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                             None) == hq.HQ_ERR_UNSUPPORTED
+
+
+def test_tuning_table_entry_changes_the_plan():
+    """A table entry replaces the library's rules for calls without a tuning
+    of its shape and m range; an explicit tuning still wins; clearing the
+    table restores the rules.  The workspace size follows the plan."""
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
+    base16 = hq.hq_plan_describe(d, 16)
+    assert (base16.tile_m, base16.kernel, base16.from_table) == (16, 2, 0)
+    assert base16.stages == base16.ring_stages >= 2
+    base64 = hq.hq_plan_describe(d, 64)
+    entry = {"fmt": hq.HQ_FMT_INT4, "n": 18432, "k": 7168, "num_experts": 1, "m_min": 1, "m_max": 32,
+             "tuning": {"tile_m": 32, "variant": 1, "stages": 3, "split_k": 2}}
+    try:
+        hq.hq_tuning_table_set([entry])
+        p = hq.hq_plan_describe(d, 16)
+        assert (p.tile_m, p.kernel, p.stages, p.from_table) == (32, 1, 3, 1)
+        assert p.split == 2 and p.grid == 2 * 144
+        assert hq.hq_workspace_size(d, 16) == p.workspace_bytes != base16.workspace_bytes
+        p64 = hq.hq_plan_describe(d, 64)                    # outside the entry's m range
+        assert (p64.tile_m, p64.kernel, p64.from_table) == (base64.tile_m, base64.kernel, 0)
+        pe = hq.hq_plan_describe(d, 16, hq.Tuning(tile_m=16))   # an explicit tuning wins
+        assert (pe.tile_m, pe.from_table) == (16, 0)
+        d2 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 1, 1)   # zero points: same shape key
+        assert hq.hq_plan_describe(d2, 16).from_table == 1
+        d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 18432, 7168, 128, 0, 1)   # another format: not matched
+        assert hq.hq_plan_describe(d3, 16).from_table == 0
+        # a bad entry is refused and leaves the table as it was
+        bad = dict(entry, tuning={"tile_m": 48})
+        with pytest.raises(hq.HQError) as e:
+            hq.hq_tuning_table_set([bad])
+        assert e.value.status == hq.HQ_ERR_UNSUPPORTED
+        assert hq.hq_plan_describe(d, 16).from_table == 1
+        # block-scaled entries go to that planner
+        dm = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 7168, 7168, 32, 0, 1)
+        hq.hq_tuning_table_set([entry, {"fmt": hq.HQ_FMT_MXFP4, "n": 7168, "k": 7168, "m_min": 200, "m_max": 300,
+                                        "tuning": {"tile_m": 256, "stages": 2}}])
+        pm = hq.hq_plan_describe(dm, 256)
+        assert (pm.kernel, pm.tile_m, pm.stages, pm.from_table) == (3, 256, 2, 1)
+    finally:
+        hq.hq_tuning_table_set([])
+    assert hq.hq_plan_describe(d, 16).from_table == 0
+
+
+def test_stages_above_the_ring_mean_the_whole_ring():
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 4096, 4096, 128, 0, 1)
+    p = hq.hq_plan_describe(d, 256, hq.Tuning(stages=99))
+    assert p.stages == p.ring_stages
+    p = hq.hq_plan_describe(d, 256, hq.Tuning(stages=2))
+    assert p.stages == 2 < p.ring_stages or p.ring_stages == 2
