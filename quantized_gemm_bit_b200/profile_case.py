@@ -20,7 +20,9 @@ from .build import build
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kind", default="w4a16", choices=["w4a16", "w3a16", "w2a16", "mxfp4_a16", "moe", "mxfp4", "nvfp4"])
+    ap.add_argument("--kind", default="w4a16",
+                    choices=["w4a16", "w3a16", "w2a16", "w8a16", "mxfp4_a16", "mxint4_a16", "moe", "moe_swiglu",
+                             "mxfp4", "nvfp4"])
     ap.add_argument("--m", type=int, default=16)
     ap.add_argument("--k", type=int, default=7168)
     ap.add_argument("--n", type=int, default=18432)
@@ -31,11 +33,12 @@ def main(argv=None):
     ap.add_argument("--tile-m", type=int, default=0)
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--variant", type=int, default=0)
+    ap.add_argument("--stages", type=int, default=0)
     a = ap.parse_args(argv)
     build()
     dev = "cuda"
-    tuning = (hq.Tuning(tile_m=a.tile_m, split_k=a.split_k, variant=a.variant)
-              if (a.tile_m or a.split_k or a.variant) else None)
+    tuning = (hq.Tuning(tile_m=a.tile_m, split_k=a.split_k, variant=a.variant, stages=a.stages)
+              if (a.tile_m or a.split_k or a.variant or a.stages) else None)
     if a.kind in ("mxfp4", "nvfp4"):
         ws = None
         if a.kind == "mxfp4":
@@ -66,8 +69,8 @@ def main(argv=None):
         ws = torch.zeros(max(256, hq.hq_workspace_size(d, a.m, tuning)), dtype=torch.uint8, device=dev)
         for _ in range(a.iters):
             run(c, ws)
-    elif a.kind in ("w4a16", "w3a16", "w2a16", "mxfp4_a16"):
-        # the W4A16 kernels with INT4, INT3, INT2 or MXFP4 weights
+    elif a.kind in ("w4a16", "w3a16", "w2a16", "w8a16", "mxfp4_a16", "mxint4_a16"):
+        # the W4A16 kernels with INT4, INT3, INT2, INT8, MXFP4 or MXINT4 weights
         if a.kind == "w4a16":
             q, s, z = synth.w4a16_weights(a.n, a.k, 128, a.asym, seed=1000)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, int(a.asym), 1)
@@ -80,6 +83,14 @@ def main(argv=None):
             q, s, z = synth.w2a16_weights(a.n, a.k, 128, a.asym, seed=7500)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, a.n, a.k, 128, int(a.asym), 1)
             blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+        elif a.kind == "w8a16":
+            q, s, z = synth.w8a16_weights(a.n, a.k, 128, a.asym, seed=7800)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_INT8, a.n, a.k, 128, int(a.asym), 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, z)).to(dev)
+        elif a.kind == "mxint4_a16":
+            codes, e8 = synth.mxint4_weights(a.n, a.k, seed=7900)
+            d = hq.hq_quant_desc_init(hq.HQ_FMT_MXINT4, a.n, a.k, 32, 0, 1)
+            blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(dev)
         else:
             codes, e8 = synth.mxfp4_weights(a.n, a.k, seed=6000)
             d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, a.n, a.k, 32, 0, 1)
@@ -93,20 +104,24 @@ def main(argv=None):
         t, e, k_top = a.m, a.experts, a.topk
         q, s, _ = synth.w4a16_weights(a.n, a.k, 128, False, seed=3000, experts=e)
         d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, a.n, a.k, 128, 0, e)
-        blob = torch.from_numpy(hq.hq_pack_weights(d, q, s, None)).to(dev)
+        gated = a.kind == "moe_swiglu"       # gate+up weights in the gated order, SwiGLU in the epilogue
+        blob = torch.from_numpy((hq.hq_pack_weights_gated if gated else hq.hq_pack_weights)(d, q, s, None)).to(dev)
         logits = synth.router_logits(t, e, seed=3001).to(dev)
         x = synth.bf16_normal(t, a.k, seed=3002).to(dev)
         ids = torch.empty(t, k_top, dtype=torch.int32, device=dev)
         src = torch.empty(t * k_top, dtype=torch.int32, device=dev)
         off = torch.empty(e + 1, dtype=torch.int32, device=dev)
         xs = torch.empty(t * k_top, a.k, dtype=torch.bfloat16, device=dev)
-        c = torch.empty(t * k_top, a.n, dtype=torch.bfloat16, device=dev)
+        c = torch.empty(t * k_top, a.n // 2 if gated else a.n, dtype=torch.bfloat16, device=dev)
         pws = torch.zeros(hq.hq_moe_permute_workspace_size(t, k_top, e), dtype=torch.uint8, device=dev)
         ws = torch.zeros(max(256, hq.hq_workspace_size(d, t * k_top, tuning)), dtype=torch.uint8, device=dev)
         for _ in range(a.iters):
             hq.hq_moe_topk(logits, t, e, k_top, ids)
             hq.hq_moe_permute(ids, t, k_top, e, src, off, pws, a=x, hidden=a.k, a_sorted=xs)
-            hq.hq_grouped_gemm_moe(d, blob, xs, off, t * k_top, c, ws, tuning)
+            if gated:
+                hq.hq_grouped_gemm_moe_swiglu(d, blob, xs, off, t * k_top, c, ws, tuning)
+            else:
+                hq.hq_grouped_gemm_moe(d, blob, xs, off, t * k_top, c, ws, tuning)
         st = hq.hq_check_device_status(pws)
         if st != hq.HQ_OK:
             print("device status", hq.status_string(st))
