@@ -387,8 +387,13 @@ def test_grouped_swiglu_fused_full_size_sampled(t):
         if hi > lo:
             sample += sorted(set(rng.integers(lo, hi, size=2).tolist()))
     sample = np.array(sorted(set(sample)))
-    _, ref = G.grouped_w4a16_ref(a_sorted, off, q.numpy(), s.numpy(), None, 128, row_subset=sample)
-    check_swiglu(h.cpu()[sample], ref, inter, hid, f"swiglu fused full size T={t}")
+    # output features: first, last and one random of every 64-feature tile;
+    # the oracle computes their gate rows f and up rows I + f only
+    feats = np.array(sorted({f for j in range(inter // 64)
+                             for f in (64 * j, 64 * j + 63, 64 * j + int(rng.integers(0, 64)))}))
+    _, ref = G.grouped_w4a16_ref(a_sorted, off, q.numpy(), s.numpy(), None, 128, row_subset=sample,
+                                 cols=np.concatenate([feats, inter + feats]))
+    check_swiglu(h.cpu()[sample][:, feats], ref, len(feats), hid, f"swiglu fused full size T={t}")
 
 
 @pytest.mark.parametrize("variant,fused", [(0, False), (2, False), (0, True), (2, True)])
