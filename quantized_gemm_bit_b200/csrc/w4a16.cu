@@ -344,7 +344,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kATile = C::kATile;
   constexpr int KPS = C::kKps;
   constexpr int kRecs = C::kRecs;
-  constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -494,6 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc_col(ab);
+      // the MMAs cover the unit's valid tokens, rounded up to 16 (a ragged
+      // tile of an expert or of the last token rows costs no more tensor
+      // work than it needs); accumulator columns past them are never stored
+      const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)min(NTOK, (x.rows + 15) & ~15));
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, t = it % TS;
         const uint32_t ph_t = (it / TS) & 1;
@@ -520,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int j = 0; j < 8; ++j) {
                 const uint32_t off = (uint32_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
                 const uint64_t bdesc = ((uint64_t)bhi << 32) | (uint64_t)(blo + off);
-                mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, kIdesc, (r > 0 || j > 0) ? 1u : acc0);
+                mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, idesc, (r > 0 || j > 0) ? 1u : acc0);
               }
             }
           }
