@@ -62,9 +62,11 @@ struct Cfg {
   static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
   // as many SMEM stages as fit, up to a preferred depth per token tile
   static constexpr int kSmemPref = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  // (exact: the budget less the base alignment and the scratch is a
+  // multiple of 128, so rounding the tables' end up to 128 stays inside it
+  // whenever the unrounded end does)
   static constexpr int kSmemFit =
-      (int)((232448 - 1024 - kBarBytes - 2 * (kMaxExperts + 1) * sizeof(int) - 128 - kEpiScratch) /
-            (kATile + kRecs));
+      (int)((232448 - 1024 - kEpiScratch - kBarBytes - 2 * (kMaxExperts + 1) * sizeof(int)) / (kATile + kRecs));
   static constexpr int kSmemStages = kSmemPref < kSmemFit ? kSmemPref : kSmemFit;
   static constexpr int kTmemStages = NTOK <= 64 ? 3 : 4;   // 64 * kKps TMEM columns each
   static constexpr int kAccBufs = NTOK <= 128 ? 2 : 1;

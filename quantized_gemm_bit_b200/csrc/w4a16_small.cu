@@ -71,9 +71,11 @@ struct SmallCfg {
   static constexpr int kBarBytes = 512;
   // as many SMEM stages as fit, up to a preferred depth per token tile
   static constexpr int kSmemPref = NTOK == 16 ? 8 : NTOK == 32 ? 6 : 4;
+  // (exact: the budget less the base alignment and the scratch is a
+  // multiple of 128, so rounding the tables' end up to 128 stays inside it
+  // whenever the unrounded end does)
   static constexpr int kSmemFit =
-      (int)((232448 - 1024 - kBarBytes - 2 * (kMaxExperts + 1) * sizeof(int) - 128 - kEpiScratch) /
-            (kATile + kRecs));
+      (int)((232448 - 1024 - kEpiScratch - kBarBytes - 2 * (kMaxExperts + 1) * sizeof(int)) / (kATile + kRecs));
   static constexpr int kSmemStages = kSmemPref < kSmemFit ? kSmemPref : kSmemFit;
   static constexpr int kAStages = NTOK == 64 ? 2 : 3;   // TMEM ring of unpacked weights
   static constexpr int kDStages = NTOK == 16 ? 4 : 2;   // TMEM ring of per-group results
