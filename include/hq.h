@@ -122,7 +122,14 @@ typedef struct {
  *              ring; larger than the ring = the whole ring
  *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
  *              splits the whole iteration space evenly when 0)
- *   cta_group: 1 (one SM per MMA)
+ *   cta_group: block-scaled GEMMs: 0 = the library's choice (CTA pairs
+ *              for 256-token whole tiles when N is a multiple of 256
+ *              and the pairs fill the SMs), 1 = one CTA per 128-row
+ *              weight tile, 2 = CTA pairs: clusters of two CTAs run
+ *              256-row weight tiles with cta_group::2 MMAs (each CTA
+ *              stages its 128 weight rows and half of the token tile);
+ *              needs N % 256 == 0, tile_m 0, 128 or 256, split_k 0.
+ *              W4A16: 0 or 1.
  *   variant  : W4A16 / grouped MoE: 0 = the library's choice, currently
  *              2 for token tiles of up to 64 and 1 for larger tiles
  *              (MXFP4_A16 weights: always 1).
@@ -179,6 +186,7 @@ typedef struct {
   int32_t stages;      /* pipeline stages in flight                                                  */
   int32_t ring_stages; /* the kernel's shared-memory ring depth                                      */
   int32_t from_table;  /* 1 when the tuning came from the table                                      */
+  int32_t cta_group;   /* 2: block-scaled CTA pairs (cta_group::2 MMAs), else 1                     */
   size_t workspace_bytes;
 } hq_plan;
 hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t, hq_plan* out);

@@ -42,9 +42,10 @@ STAGES = (0, 2, 4)
 def candidates(kind, m):
     """Tunings worth trying at m rows: token tiles up to twice the rows
     (at least 16), K splits 0 (the library's choice) to 3, pipeline stages
-    in flight (0 = the kernel's whole ring, 2, 4), and for the W4A16 kernels
+    in flight (0 = the kernel's whole ring, 2, 4), for the W4A16 kernels
     with INT4, INT3, INT2 or INT8 weights both weight variants (the MX
-    formats have only the rescaled one)."""
+    formats have only the rescaled one), and for the block-scaled GEMMs
+    with 128/256-token tiles one CTA per weight tile or CTA pairs."""
     cap = max(16, 2 * m)
     tiles = [t for t in TILES if t <= cap] or [16]
     variants = ((1, 2) if kind in ("w4a16", "moe", "w3a16", "w2a16", "w8a16")
@@ -58,12 +59,20 @@ def candidates(kind, m):
                     continue
                 for st in STAGES:
                     out.append(hq.Tuning(tile_m=t, split_k=s, variant=v, stages=st))
+    # block-scaled 128/256-token whole tiles: one CTA per weight tile, or
+    # CTA pairs (the library's choice at 256 picks either)
+    if kind in ("mxfp4", "nvfp4"):
+        for t in (x for x in tiles if x >= 128):
+            for g in (1, 2):
+                for st in STAGES:
+                    out.append(hq.Tuning(tile_m=t, cta_group=g, stages=st))
     return out
 
 
 def _describe(t):
     return ("library" if t is None
-            else f"tile_m={t.tile_m} split_k={t.split_k} variant={t.variant} stages={t.stages}")
+            else f"tile_m={t.tile_m} split_k={t.split_k} variant={t.variant} stages={t.stages}"
+                 + (f" cta_group={t.cta_group}" if t.cta_group else ""))
 
 
 def _tuning_dict(t):

@@ -52,8 +52,12 @@ enum BsFmt { kMX = 0, kNV = 1 };
 template <int FMT, int NTOK>
 constexpr int bs_boxes() { return FMT == kMX && NTOK <= 64 ? 2 : 1; }
 
-template <int FMT, int NTOK>
+// CG = 2: a CTA pair (cluster of two) runs one 256-row weight tile with
+// cta_group::2 MMAs; each CTA stages its own 128 weight rows and half of the
+// token tile, and the scales of the whole token tile.
+template <int FMT, int NTOK, int CG = 1>
 struct BsCfg {
+  static_assert(CG == 1 || (CG == 2 && NTOK >= 128), "CTA pairs run 128- or 256-token tiles");
   static constexpr int kBox = bs_boxes<FMT, NTOK>();        // 128-B-row boxes along K per stage
   static constexpr int kKBox = FMT == kNV ? 256 : 128;     // K elements per box: 128 B per row in SMEM
   static constexpr int kATileBox = kBsTileN * 128;         // weights in SMEM, one box
@@ -61,7 +65,7 @@ struct BsCfg {
   // bytes the weight copy moves: NVFP4 loads packed bytes; the MXFP4 load
   // unpacks 4-bit codes into 16-byte slots and counts the packed bytes
   static constexpr int kATxBox = FMT == kNV ? kATileBox : kBsTileN * 64;
-  static constexpr int kBTileBox = NTOK * 128;             // activations, one box
+  static constexpr int kBTileBox = NTOK / CG * 128;        // this CTA's activations, one box
   static constexpr int kBTile = kBox * kBTileBox;
   static constexpr int kSfaBox = FMT == kNV ? 2048 : 512;  // weight scale chunks per box
   static constexpr int kSfa = kBox * kSfaBox;
@@ -110,6 +114,7 @@ struct BsParams {
   int data_parallel;         // whole tiles per unit, no partial sums
   int early_weights;         // fetch the first stages' weights before griddepcontrol.wait
   int stage_limit;           // pipeline stages in flight (0 or >= the ring depth: the whole ring)
+  int n_pairs;               // CTA pairs: 256-row weight tiles (n_tiles / 2)
 };
 
 // NVFP4 activation scales, row-major [m][K/16] bytes, re-laid into the order
@@ -135,9 +140,26 @@ __global__ void sfb_relayout_kernel(const uint32_t* __restrict__ sf, int m, int 
   }
 }
 
-template <int FMT, int NTOK>
+template <int FMT, int NTOK, int CG = 1>
 __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, int& nt, int& row0, int& rows,
                                         int& ks0, int& ks1, int& partial, int& slot) {
+  if constexpr (CG == 2) {
+    // whole (token tile, 256-row weight tile) units over the clusters; CTA
+    // rank r of the pair owns 128-row weight tile 2 * pair + r
+    const long long ncl = gridDim.x / 2, cl = blockIdx.x / 2;
+    const long long t = cl + (long long)idx * ncl;
+    if (t >= (long long)p.m_tiles * p.n_pairs) return false;
+    const int mt = (int)(t / p.n_pairs);
+    tile = (int)t;
+    nt = 2 * (int)(t - (long long)mt * p.n_pairs) + (int)(blockIdx.x & 1);
+    row0 = mt * NTOK;
+    rows = min(NTOK, p.m - row0);
+    ks0 = 0;
+    ks1 = p.k_stages;
+    partial = 0;
+    slot = 0;
+    return true;
+  }
   if (p.data_parallel) {
     const long long t = (long long)blockIdx.x + (long long)idx * gridDim.x;
     if (t >= (long long)p.m_tiles * p.n_tiles) return false;
@@ -234,15 +256,16 @@ __device__ __forceinline__ void bs_fixup(const BsParams& p, int tile, int nt, in
   if (lane == 0) p.counters[tile * kBsEpiWarps + wslot] = 0;
 }
 
-template <int FMT, int NTOK>
+template <int FMT, int NTOK, int CG>
 __global__ void __launch_bounds__(kBsThreads, 1)
     blockscaled_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_a,
+                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                        const BsParams p) {
-  using C = BsCfg<FMT, NTOK>;
+  using C = BsCfg<FMT, NTOK, CG>;
   constexpr int S = C::kStages;
   constexpr int ACC = C::kAcc;
   constexpr int NC = C::kCols;
-  // bytes of a stage with nb boxes
+  // bytes of a stage with nb boxes (this CTA's share)
   auto stage_tx = [](int nb) -> uint32_t {
     return (uint32_t)(nb * (C::kATxBox + C::kBTileBox + C::kSfaBox) + C::kSfb);
   };
@@ -267,6 +290,9 @@ __global__ void __launch_bounds__(kBsThreads, 1)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
+  // CTA pairs: rank 0 issues the pair's MMAs; every stage's copies of both
+  // CTAs complete on rank 0's full barrier
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -275,7 +301,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kBsEpiWarps);
+      mbar_init(&acc_empty[b], kBsEpiWarps * CG);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -284,9 +310,28 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmap_w);
     prefetch_tensormap(&tmap_a);
+    if (CG == 2) {
+      prefetch_tensormap(&tmap_sfa);
+      if (FMT == kNV) prefetch_tensormap(&tmap_sfb);
+    }
   }
   if (threadIdx.x == 0) pdl_launch_dependents();
-  __syncthreads();   // barriers visible to every role
+  if constexpr (CG == 2) {
+    // MXFP4 activations carry no block scale: 32 rows x 16 bytes of E8M0 127
+    // (= 1.0) that rank 0 copies into both CTAs' TMEM before its first MMA
+    if (FMT == kMX && threadIdx.x < 128) reinterpret_cast<uint32_t*>(scratch)[threadIdx.x] = 0x7F7F7F7Fu;
+    // the pair's TMEM is allocated by both CTAs together; the barriers and
+    // the allocation are visible to both CTAs after the cluster barrier
+    if (warp == 2) {
+      tmem_alloc_pair(s_tmem, 512);
+      tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+  } else {
+    __syncthreads();   // barriers visible to every role
+  }
 
   int tile, nt, row0, rows, ks0, ks1, partial, slot;
 
@@ -294,29 +339,43 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     // ------------------------------------------------------------ producer (whole warp, one lane issues)
     const bool leader = elect_one();
     const uint64_t pol_w = policy_evict_first();
+    // rank 0's full barrier of stage s, as a cluster address (pairs)
+    auto full_cl = [&](int s) -> uint32_t { return CG == 2 ? mapa_u32(&full[s], 0) : 0u; };
     // weights of stage it: codes (K coordinate in elements for the MXFP4
     // unpacking type, in bytes for NVFP4) and their scale chunks
     auto load_weights = [&](int s, int ks, int nt_) {
       const int nb = stage_boxes(ks);
-      for (int b = 0; b < nb; ++b) {
-        const int kbox = ks * C::kBox + b;
-        tma_load_2d(sA(s) + b * C::kATileBox, &tmap_w, FMT == kNV ? kbox * 128 : kbox * C::kKBox, nt_ * kBsTileN,
-                    &full[s]);
-      }
       const int chunks = FMT == kNV ? 4 : 1;   // 512-byte scale chunks per box
-      const uint8_t* src = p.sf_w + ((size_t)nt_ * p.sf_groups + (size_t)ks * C::kBox * chunks) * 512;
-      bulk_g2s(sSfa(s), src, (uint32_t)(nb * C::kSfaBox), &full[s], pol_w);
+      if constexpr (CG == 2) {
+        const uint32_t fb = full_cl(s);
+        for (int b = 0; b < nb; ++b) {
+          const int kbox = ks * C::kBox + b;
+          tma_load_2d_pair(sA(s) + b * C::kATileBox, &tmap_w, FMT == kNV ? kbox * 128 : kbox * C::kKBox,
+                           nt_ * kBsTileN, fb);
+        }
+        // scale chunks as rows of 128 words
+        tma_load_2d_pair(sSfa(s), &tmap_sfa, 0, nt_ * p.sf_groups + ks * C::kBox * chunks, fb);
+      } else {
+        for (int b = 0; b < nb; ++b) {
+          const int kbox = ks * C::kBox + b;
+          tma_load_2d(sA(s) + b * C::kATileBox, &tmap_w, FMT == kNV ? kbox * 128 : kbox * C::kKBox, nt_ * kBsTileN,
+                      &full[s]);
+        }
+        const uint8_t* src = p.sf_w + ((size_t)nt_ * p.sf_groups + (size_t)ks * C::kBox * chunks) * 512;
+        bulk_g2s(sSfa(s), src, (uint32_t)(nb * C::kSfaBox), &full[s], pol_w);
+      }
     };
     // Phase 1, before the previous kernel on the stream has finished: the
     // packed weights of the first S stages (no kernel writes them)
     uint32_t n_pre = 0;
-    const uint32_t depth = (p.stage_limit > 0 && p.stage_limit < S) ? (uint32_t)p.stage_limit : (uint32_t)S;
-    for (int idx = 0; p.early_weights && n_pre < depth &&
-                      bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
+    const uint32_t lim = (p.stage_limit > 0 && p.stage_limit < S) ? (uint32_t)p.stage_limit : (uint32_t)S;
+    for (int idx = 0; p.early_weights && n_pre < lim &&
+                      bs_unit<FMT, NTOK, CG>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
          ++idx) {
-      for (int ks = ks0; ks < ks1 && n_pre < depth; ++ks, ++n_pre) {
+      for (int ks = ks0; ks < ks1 && n_pre < lim; ++ks, ++n_pre) {
         if (leader) {
-          mbar_arrive_expect_tx(&full[n_pre], stage_tx(stage_boxes(ks)));
+          // rank 0 expects the bytes of both CTAs of a pair
+          if (rank == 0) mbar_arrive_expect_tx(&full[n_pre], CG * stage_tx(stage_boxes(ks)));
           load_weights((int)n_pre, ks, nt);
         }
         __syncwarp();
@@ -326,39 +385,55 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     // Phase 2: activations (and their scales) of those stages, then the ring
     uint32_t it = 0;
     bool ok = true;
-    for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
+    for (int idx = 0; ok && bs_unit<FMT, NTOK, CG>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx) {
       for (int ks = ks0; ks < ks1; ++ks, ++it) {
         const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        if ((it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) ||
-            !throttle_stages<S>(empty, it, p.stage_limit, p.wait_ns, s_abort)) {
+        if (!wait_stage_free<S>(empty, it, lim, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
         }
         if (leader) {
           if (it >= n_pre) {
-            mbar_arrive_expect_tx(&full[s], stage_tx(stage_boxes(ks)));
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], CG * stage_tx(stage_boxes(ks)));
             load_weights(s, ks, nt);
           }
-          for (int b = 0; b < stage_boxes(ks); ++b)
-            tma_load_2d(sB(s) + b * C::kBTileBox, &tmap_a, (ks * C::kBox + b) * 128, row0, &full[s]);
-          if (FMT == kNV) {
-            const uint8_t* sfb = p.sf_a + ((size_t)(row0 / NTOK) * p.k_stages + ks) * C::kSfb;
-            bulk_g2s(sSfb(s), sfb, C::kSfb, &full[s], policy_evict_last());
+          if constexpr (CG == 2) {
+            const uint32_t fb = full_cl(s);
+            // this CTA's half of the token tile
+            for (int b = 0; b < stage_boxes(ks); ++b)
+              tma_load_2d_pair(sB(s) + b * C::kBTileBox, &tmap_a, (ks * C::kBox + b) * 128,
+                               row0 + (int)rank * (NTOK / 2), fb);
+            if (FMT == kNV)
+              tma_load_2d_pair(sSfb(s), &tmap_sfb, 0, ((row0 / NTOK) * p.k_stages + ks) * (C::kSfb / 512), fb);
+          } else {
+            for (int b = 0; b < stage_boxes(ks); ++b)
+              tma_load_2d(sB(s) + b * C::kBTileBox, &tmap_a, (ks * C::kBox + b) * 128, row0, &full[s]);
+            if (FMT == kNV) {
+              const uint8_t* sfb = p.sf_a + ((size_t)(row0 / NTOK) * p.k_stages + ks) * C::kSfb;
+              bulk_g2s(sSfb(s), sfb, C::kSfb, &full[s], policy_evict_last());
+            }
           }
         }
         __syncwarp();
       }
     }
     if (!ok && lane == 0) {
-      const uint32_t first = it > (uint32_t)S ? it - S : 0;
-      for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % S], (j / S) & 1, p.wait_ns, nullptr);
+      if constexpr (CG == 2) {
+        // this CTA's copies complete on rank 0's barriers: give the last
+        // ones issued time to land before the CTA can exit
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 50000) {
+        }
+      } else {
+        const uint32_t first = it > (uint32_t)S ? it - S : 0;
+        for (uint32_t j = first; j < it; ++j) hq_wait(&full[j % S], (j / S) & 1, p.wait_ns, nullptr);
+      }
     }
   } else {
   // The producer needs no TMEM, so it starts loading at once; the other
   // roles wait here for the allocation (and, for MXFP4, the unit scales).
-  if (warp == 2) {
+  if (CG == 1 && warp == 2) {
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
   }
@@ -367,7 +442,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   named_bar(1, kBsThreads - 32);
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  if (FMT == kMX) {
+  if (CG == 1 && FMT == kMX) {
     if (warp >= 4 && warp < 8) {
       // activations carry no block scale: E8M0 127 (= 1.0) in every byte
       tmem_st_x8(tmem_base + (((warp & 3) * 32) << 16) + C::kSfbConst, 0x7F7F7F7Fu);
@@ -379,14 +454,25 @@ __global__ void __launch_bounds__(kBsThreads, 1)
   }
   if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (whole warp, one fixed lane issues)
+    // (pairs: rank 0 only, for both CTAs)
     const bool leader = elect_one();
     uint32_t it = 0, uc = 0;
-    bool ok = true;
-    for (int idx = 0; ok && bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
+    bool ok = rank == 0;
+    if (CG == 2 && FMT == kMX && ok) {
+      // the unit scales: 8 columns, as the one-CTA kernel stores them
+      if (leader) {
+        tmem_cp_sf_pair(tmem_base + C::kSfbConst, smem_desc_sf(smem_u32(scratch)));
+        tmem_cp_sf_pair(tmem_base + C::kSfbConst + 4, smem_desc_sf(smem_u32(scratch)));
+      }
+      __syncwarp();
+    }
+    for (int idx = 0; ok && bs_unit<FMT, NTOK, CG>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot);
          ++idx, ++uc) {
       const int ab = uc % ACC;
       const uint32_t aph = (uc / ACC) & 1;
-      if (!hq_wait_warp(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
+      // (pairs: the epilogue warps of both CTAs arrive)
+      if (!(CG == 2 ? hq_wait_warp_cl(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)
+                    : hq_wait_warp(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort))) {
         if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
         ok = false;
         break;
@@ -420,11 +506,20 @@ __global__ void __launch_bounds__(kBsThreads, 1)
             for (int i = 0; i < 4; ++i) {
               const uint32_t sfa_t = tmem_base + sf_col + 4 * i;
               const uint32_t sfb_t = tmem_base + sf_col + 16 + 4 * C::kHalves * i;
-              tmem_cp_sf(sfa_t, step(fa, 512 * i));
+              constexpr uint32_t kId = idesc_block_scaled(1, 1, 0, 128 * CG, NTOK, 0, 0);
+              if constexpr (CG == 2) {
+                tmem_cp_sf_pair(sfa_t, step(fa, 512 * i));
 #pragma unroll
-              for (int h = 0; h < C::kHalves; ++h) tmem_cp_sf(sfb_t + 4 * h, step(fb, 512 * (i * C::kHalves + h)));
-              constexpr uint32_t kId = idesc_block_scaled(1, 1, 0, 128, NTOK, 0, 0);
-              mma_mxf4nvf4(d_tmem, step(ad, 32 * i), step(bd, 32 * i), kId, sfa_t, sfb_t, i > 0 ? 1u : acc0);
+                for (int h = 0; h < C::kHalves; ++h)
+                  tmem_cp_sf_pair(sfb_t + 4 * h, step(fb, 512 * (i * C::kHalves + h)));
+                mma_mxf4nvf4_pair(d_tmem, step(ad, 32 * i), step(bd, 32 * i), kId, sfa_t, sfb_t, i > 0 ? 1u : acc0);
+              } else {
+                tmem_cp_sf(sfa_t, step(fa, 512 * i));
+#pragma unroll
+                for (int h = 0; h < C::kHalves; ++h)
+                  tmem_cp_sf(sfb_t + 4 * h, step(fb, 512 * (i * C::kHalves + h)));
+                mma_mxf4nvf4(d_tmem, step(ad, 32 * i), step(bd, 32 * i), kId, sfa_t, sfb_t, i > 0 ? 1u : acc0);
+              }
             }
           } else {
             const uint64_t fa = smem_desc_sf(smem_u32(sSfa(s)));
@@ -433,27 +528,46 @@ __global__ void __launch_bounds__(kBsThreads, 1)
             for (int b = 0; b < C::kBox; ++b) {
               if (b < nb) {
                 const uint32_t sfa_t = tmem_base + sf_col + 4 * b;
-                tmem_cp_sf(sfa_t, step(fa, 512 * b));
+                if constexpr (CG == 2)
+                  tmem_cp_sf_pair(sfa_t, step(fa, 512 * b));
+                else
+                  tmem_cp_sf(sfa_t, step(fa, 512 * b));
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   // byte i of each scale column holds the scale of 32-K block i
-                  const uint32_t id = idesc_block_scaled(5, 0, 1, 128, NTOK, (uint32_t)i, 0);
-                  mma_mxf8f6f4(d_tmem, step(ad, b * C::kATileBox + 32 * i), step(bd, b * C::kBTileBox + 32 * i), id,
-                               sfa_t, tmem_base + C::kSfbConst, (b > 0 || i > 0) ? 1u : acc0);
+                  const uint32_t id = idesc_block_scaled(5, 0, 1, 128 * CG, NTOK, (uint32_t)i, 0);
+                  const uint64_t a_d = step(ad, b * C::kATileBox + 32 * i), b_d = step(bd, b * C::kBTileBox + 32 * i);
+                  const uint32_t acc = (b > 0 || i > 0) ? 1u : acc0;
+                  if constexpr (CG == 2)
+                    mma_mxf8f6f4_pair(d_tmem, a_d, b_d, id, sfa_t, tmem_base + C::kSfbConst, acc);
+                  else
+                    mma_mxf8f6f4(d_tmem, a_d, b_d, id, sfa_t, tmem_base + C::kSfbConst, acc);
                 }
               }
             }
           }
-          tc_commit(&empty[s]);
+          // the stage's slot in both CTAs of a pair is free once these MMAs are done
+          if constexpr (CG == 2)
+            tc_commit_pair(&empty[s]);
+          else
+            tc_commit(&empty[s]);
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (leader) tc_commit(&acc_full[ab]);
+      if (leader) {
+        if constexpr (CG == 2)
+          tc_commit_pair(&acc_full[ab]);
+        else
+          tc_commit(&acc_full[ab]);
+      }
       __syncwarp();
     }
-    if (leader) {
-      tc_commit(drain);
+    if (leader && (CG == 1 || rank == 0)) {
+      if constexpr (CG == 2)
+        tc_commit_pair_local(drain);
+      else
+        tc_commit(drain);
       hq_wait(drain, 0, p.wait_ns, nullptr);
     }
     __syncwarp();
@@ -471,7 +585,7 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     uint16_t* scr = scratch + (warp - 4) * (32 * kBsEB);
     const float alpha = FMT == kNV ? p.a_global * __ldg(p.g_w) : 1.f;
     uint32_t uc = 0;
-    for (int idx = 0; bs_unit<FMT, NTOK>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx, ++uc) {
+    for (int idx = 0; bs_unit<FMT, NTOK, CG>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx, ++uc) {
       const int ab = uc % ACC;
       const uint32_t aph = (uc / ACC) & 1;
       if (!hq_wait(&acc_full[ab], aph, p.wait_ns, s_abort)) {
@@ -490,7 +604,13 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (lane == 0) {
+        // (pairs: the accumulator's owner is rank 0's MMA issuer)
+        if constexpr (CG == 2)
+          mbar_arrive_cluster(mapa_u32(&acc_empty[ab], 0));
+        else
+          mbar_arrive(&acc_empty[ab]);
+      }
 
       const int tok0 = hc * NC;                       // first token of this warp's run
       const int rows_w = rows - tok0;                 // valid tokens in the run (may be <= 0)
@@ -514,7 +634,8 @@ __global__ void __launch_bounds__(kBsThreads, 1)
       }
       // the 256-token tile keeps 128 accumulator registers per thread: fewer
       // contributors in flight there
-      if (partial) bs_fixup<FMT, NTOK, (NTOK > 128 ? 1 : 4)>(p, tile, nt, row0, rows, tok0, wslot, r, (int)lane, alpha);
+      if (CG == 1 && partial)
+        bs_fixup<FMT, NTOK, (NTOK > 128 ? 1 : 4)>(p, tile, nt, row0, rows, tok0, wslot, r, (int)lane, alpha);
     }
   }
 
@@ -522,25 +643,73 @@ __global__ void __launch_bounds__(kBsThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair's CTAs leave together: rank 0's MMAs read the other CTA's shared
+  // memory and write its TMEM until rank 0 has drained them
+  if constexpr (CG == 2) cluster_sync();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(*s_tmem, 512);
+  if (warp == 2) {
+    if constexpr (CG == 2)
+      tmem_dealloc_pair(*s_tmem, 512);
+    else
+      tmem_dealloc(*s_tmem, 512);
+  }
 }
 
-template <int FMT, int NTOK>
-hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const BsParams& p, int grid,
-                      cudaStream_t stream) {
-  auto kern = blockscaled_kernel<FMT, NTOK>;
-  const size_t smem = BsCfg<FMT, NTOK>::kSmem;
+template <int FMT, int NTOK, int CG>
+bool bs_smem_attr() {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return HQ_ERR_CUDA;
-    attr_set[dev] = true;
+  if (dev < 64 && attr_set[dev]) return true;
+  if (cudaFuncSetAttribute(blockscaled_kernel<FMT, NTOK, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)BsCfg<FMT, NTOK, CG>::kSmem) != cudaSuccess)
+    return false;
+  if (dev < 64) attr_set[dev] = true;
+  return true;
+}
+
+template <int FMT, int NTOK, int CG>
+hq_status bs_launch_t(const CUtensorMap& mw, const CUtensorMap& ma, const CUtensorMap& msfa, const CUtensorMap& msfb,
+                      const BsParams& p, int grid, cudaStream_t stream) {
+  auto kern = blockscaled_kernel<FMT, NTOK, CG>;
+  const size_t smem = BsCfg<FMT, NTOK, CG>::kSmem;
+  if (!bs_smem_attr<FMT, NTOK, CG>()) return HQ_ERR_CUDA;
+  const cudaError_t e = CG == 2 ? launch_pdl_pairs(kern, dim3(grid), dim3(kBsThreads), smem, stream, mw, ma, msfa, msfb, p)
+                                : launch_pdl(kern, dim3(grid), dim3(kBsThreads), smem, stream, mw, ma, msfa, msfb, p);
+  return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+// Clusters of two of the CTA-pair kernel that are resident at once (0 when
+// the query fails), per device.
+template <int FMT, int NTOK>
+int bs_pair_slots_t() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  if (!bs_smem_attr<FMT, NTOK, 2>()) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kBsThreads);
+  cfg.dynamicSmemBytes = BsCfg<FMT, NTOK, 2>::kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, blockscaled_kernel<FMT, NTOK, 2>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
   }
-  return launch_pdl(kern, dim3(grid), dim3(kBsThreads), smem, stream, mw, ma, p) == cudaSuccess ? HQ_OK
-                                                                                                 : HQ_ERR_CUDA;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+int bs_pair_slots(bool nv, int ntok) {
+  if (nv) return ntok == 128 ? bs_pair_slots_t<kNV, 128>() : bs_pair_slots_t<kNV, 256>();
+  return ntok == 128 ? bs_pair_slots_t<kMX, 128>() : bs_pair_slots_t<kMX, 256>();
 }
 
 // 128-B-row boxes along K, and pipeline stages (bs_boxes boxes each).
@@ -563,6 +732,18 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   if (!t) t = tuning_from_table(d, m, &from_table);
   cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
   cfg.stages = t ? t->stages : 0;
+  cfg.cta_group = 1;
+  if (t && t->cta_group == 2) {
+    // CTA pairs: whole 256-row weight tiles of 128 or 256 tokens, one per
+    // resident cluster at a time
+    cfg.cta_group = 2;
+    cfg.ntok = t->tile_m ? t->tile_m : (m <= 128 ? 128 : 256);
+    cfg.splits = 0;
+    const long long pair_tiles = (long long)(d.n / 256) * ((m + cfg.ntok - 1) / cfg.ntok);
+    const long long slots = bs_pair_slots(d.fmt == HQ_FMT_NVFP4, cfg.ntok);
+    cfg.grid = (int)(2 * std::max<long long>(1, std::min<long long>(slots > 0 ? slots : dev.num_sms / 2, pair_tiles)));
+    return cfg;
+  }
   int ntok = (t && t->tile_m) ? t->tile_m : 0;
   if (!ntok) ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
   auto dp_eff = [&](int nt) {
@@ -601,6 +782,21 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   if (pick || dp_eff(ntok) >= 0.85) {
     cfg.splits = 0;
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
+    // 256-token whole tiles run on CTA pairs when the pairs' waves are as
+    // full (the caller may ask for one CTA per tile with cta_group 1).
+    // Measured on B200: NVFP4 8192^3 247 -> 207 us, M=16384 K=7168
+    // N=18432 1008 -> 923 us; MXFP4 M=4096 K=N=7168 162 -> 150 us.
+    if (ntok == 256 && d.n % 256 == 0 && !(t && t->cta_group == 1)) {
+      const long long pair_tiles = (long long)(d.n / 256) * ((m + 255) / 256);
+      const long long slots = bs_pair_slots(d.fmt == HQ_FMT_NVFP4, 256);
+      if (slots > 0) {
+        const long long waves = (pair_tiles + slots - 1) / slots;
+        if ((double)pair_tiles / (double)(waves * slots) >= 0.85) {
+          cfg.cta_group = 2;
+          cfg.grid = (int)(2 * std::min<long long>(slots, pair_tiles));
+        }
+      }
+    }
     return cfg;
   }
   if (tiles * 2 <= dev.num_sms && tiles * (dev.num_sms / tiles) >= 0.7 * dev.num_sms) {
@@ -637,6 +833,9 @@ BsWsLayout bs_ws_layout(const hq_quant_desc& d, int m, const BsConfig& cfg) {
 
 int bs_ring_depth(const hq_quant_desc& d, const BsConfig& cfg) {
   const bool nv = d.fmt == HQ_FMT_NVFP4;
+  if (cfg.cta_group == 2)
+    return cfg.ntok == 128 ? (nv ? BsCfg<kNV, 128, 2>::kStages : BsCfg<kMX, 128, 2>::kStages)
+                           : (nv ? BsCfg<kNV, 256, 2>::kStages : BsCfg<kMX, 256, 2>::kStages);
   switch (cfg.ntok) {
     case 16: return nv ? BsCfg<kNV, 16>::kStages : BsCfg<kMX, 16>::kStages;
     case 32: return nv ? BsCfg<kNV, 32>::kStages : BsCfg<kMX, 32>::kStages;
@@ -678,6 +877,7 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.data_parallel = cfg.splits == 0 ? 1 : 0;
   p.early_weights = cfg.early_weights;
   p.stage_limit = cfg.stages;
+  p.n_pairs = n_tiles / 2;
   const BsWsLayout L = bs_ws_layout(d, m, cfg);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.counters = reinterpret_cast<int32_t*>(wsb + L.counters);
@@ -704,7 +904,7 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
     const cuuint64_t row_bytes = nv ? (cuuint64_t)d.k / 2 : (cuuint64_t)d.k;
     cuuint64_t dims[2] = {row_bytes, (cuuint64_t)m};
     cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {128, (cuuint32_t)cfg.ntok};
+    cuuint32_t box[2] = {128, (cuuint32_t)(cfg.ntok / cfg.cta_group)};
     CUresult cr = enc(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a), dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -721,8 +921,40 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
     if (cudaGetLastError() != cudaSuccess) return HQ_ERR_CUDA;
   }
 
+  // CTA pairs: the scale chunks come by tensor copy (their completion is
+  // counted on the other CTA's barrier), as rows of 128 32-bit words
+  CUtensorMap msfa{}, msfb{};
+  if (cfg.cta_group == 2) {
+    {
+      cuuint64_t dims[2] = {128, (cuuint64_t)n_tiles * p.sf_groups};
+      cuuint64_t strides[1] = {512};
+      cuuint32_t box[2] = {128, (cuuint32_t)(nv ? 4 : 1)};
+      CUresult cr = enc(&msfa, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(p.sf_w), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
+    }
+    if (nv) {
+      const int chunks = 4 * (cfg.ntok > 128 ? 2 : 1);   // 512-byte chunks per (token tile, stage)
+      cuuint64_t dims[2] = {128, (cuuint64_t)p.m_tiles * p.k_stages * chunks};
+      cuuint64_t strides[1] = {512};
+      cuuint32_t box[2] = {128, (cuuint32_t)chunks};
+      CUresult cr = enc(&msfb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, wsb + L.sfb, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
+    }
+    if (cfg.ntok == 128)
+      return nv ? bs_launch_t<kNV, 128, 2>(mw, ma, msfa, msfb, p, cfg.grid, stream)
+                : bs_launch_t<kMX, 128, 2>(mw, ma, msfa, msfb, p, cfg.grid, stream);
+    if (cfg.ntok == 256)
+      return nv ? bs_launch_t<kNV, 256, 2>(mw, ma, msfa, msfb, p, cfg.grid, stream)
+                : bs_launch_t<kMX, 256, 2>(mw, ma, msfa, msfb, p, cfg.grid, stream);
+    return HQ_ERR_UNSUPPORTED;
+  }
+
 #define HQ_BS_CASE(F, NT) \
-  case NT: return bs_launch_t<F, NT>(mw, ma, p, cfg.grid, stream);
+  case NT: return bs_launch_t<F, NT, 1>(mw, ma, msfa, msfb, p, cfg.grid, stream);
   if (nv) {
     switch (cfg.ntok) {
       HQ_BS_CASE(kNV, 16) HQ_BS_CASE(kNV, 32) HQ_BS_CASE(kNV, 64) HQ_BS_CASE(kNV, 128) HQ_BS_CASE(kNV, 256)

@@ -308,12 +308,15 @@ hq_status hq_grouped_gemm_moe_swiglu(const hq_quant_desc* d, const void* packed_
 }
 
 namespace {
-hq_status check_bs_tuning(const hq_tuning* t) {
+hq_status check_bs_tuning(const hq_quant_desc* d, const hq_tuning* t) {
   if (!t) return HQ_OK;
   if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
     return HQ_ERR_UNSUPPORTED;
-  if ((t->tile_n && t->tile_n != 128) || t->tile_k || t->split_k < 0 || t->stages < 0 ||
-      (t->cta_group && t->cta_group != 1) || t->variant != 0 || (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
+  if ((t->tile_n && t->tile_n != 128) || t->tile_k || t->split_k < 0 || t->stages < 0 || t->cta_group < 0 ||
+      t->cta_group > 2 || t->variant != 0 || (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
+    return HQ_ERR_UNSUPPORTED;
+  // CTA pairs: 256-row weight tiles, 128- or 256-token tiles, whole tiles
+  if (t->cta_group == 2 && (d->n % 256 != 0 || (t->tile_m && t->tile_m < 128) || t->split_k != 0))
     return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
@@ -331,7 +334,7 @@ hq_status hq_gemm_mxfp4_a8(const hq_quant_desc* d, const void* packed_w_dev, con
   if (!aligned(packed_w_dev, 256) || !aligned(a_e4m3_dev, 16) || !aligned(a_scale_dev, 4) || !aligned(c_dev, 16) ||
       !aligned(ws_dev, 256))
     return HQ_ERR_ALIGNMENT;
-  st = check_bs_tuning(t);
+  st = check_bs_tuning(d, t);
   if (st != HQ_OK) return st;
   DeviceInfo dev{};
   st = device_info(&dev);
@@ -353,7 +356,7 @@ hq_status hq_gemm_nvfp4(const hq_quant_desc* d, const void* packed_w_dev, const 
   if (!aligned(packed_w_dev, 256) || !aligned(a_fp4_dev, 16) || !aligned(a_sf_dev, 16) || !aligned(c_dev, 16) ||
       !aligned(ws_dev, 256))
     return HQ_ERR_ALIGNMENT;
-  st = check_bs_tuning(t);
+  st = check_bs_tuning(d, t);
   if (st != HQ_OK) return st;
   DeviceInfo dev{};
   st = device_info(&dev);
@@ -484,7 +487,7 @@ hq_status hq_tuning_table_set(const hq_tuning_entry* entries, int32_t count) {
                                                            : e.fmt == HQ_FMT_NVFP4 ? 16 : 32,
                                       0, e.num_experts);
     if (st != HQ_OK) return st;
-    st = w4_format(&d) ? check_w4_tuning(&d, &e.tuning, d.num_experts > 1) : check_bs_tuning(&e.tuning);
+    st = w4_format(&d) ? check_w4_tuning(&d, &e.tuning, d.num_experts > 1) : check_bs_tuning(&d, &e.tuning);
     if (st != HQ_OK) return st;
   }
   std::lock_guard<std::mutex> lock(g_table_mu);
@@ -497,7 +500,7 @@ hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t
   if (st != HQ_OK) return st;
   if (!out || m < 1) return HQ_ERR_INVALID_ARG;
   const bool w16 = w4_format(d);
-  st = w16 ? check_w4_tuning(d, t, d->num_experts > 1) : check_bs_tuning(t);
+  st = w16 ? check_w4_tuning(d, t, d->num_experts > 1) : check_bs_tuning(d, t);
   if (st != HQ_OK) return st;
   DeviceInfo dev{};
   if (device_info(&dev) != HQ_OK) dev.num_sms = 148;   // as hq_workspace_size
@@ -514,6 +517,7 @@ hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t
     p.split = grouped ? 0 : cfg.splits == 0 ? 0 : cfg.splits;
     p.whole_tiles = grouped ? 0 : cfg.dp_tiles;
     p.kernel = (!mx && cfg.ntok <= 64 && cfg.variant != 1) ? 2 : 1;
+    p.cta_group = 1;
     p.ring_stages = depth;
     p.stages = (cfg.stages > 0 && cfg.stages < depth) ? cfg.stages : depth;
     p.workspace_bytes = w4_workspace_bytes(*d, m, cfg, grouped);
@@ -524,6 +528,7 @@ hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t
     p.grid = cfg.grid;
     p.split = cfg.splits;
     p.kernel = 3;
+    p.cta_group = cfg.cta_group;
     p.ring_stages = depth;
     p.stages = (cfg.stages > 0 && cfg.stages < depth) ? cfg.stages : depth;
     p.workspace_bytes = bs_workspace_bytes(*d, m, cfg);

@@ -120,16 +120,71 @@ __device__ __forceinline__ bool hq_wait_warp(uint64_t* bar, uint32_t parity, uin
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// Producer: before issuing iteration `it`, wait until iteration
-// it - limit has been consumed, so that at most `limit` stages are in
-// flight (limit < SS).  Its slot is next refilled at it - limit + SS > it,
-// so the slot's empty barrier cannot have moved past that phase: the parity
-// wait is exact.  Returns false when the bounded wait gave up.
-template <int SS>
-__device__ __forceinline__ bool throttle_stages(uint64_t* empty, uint32_t it, int limit, uint64_t wait_ns,
+// ---------------------------------------------------------------- CTA pairs
+// Clusters of two CTAs whose tensor-core work is issued as one (cta_group::2):
+// rank 0 issues every MMA of the pair.
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the object at p's offset in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_u32(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier of any CTA of the cluster (release, cluster scope).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// Every thread of both CTAs: all memory operations before it are visible
+// to the whole cluster after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Bounded wait (as hq_wait) that acquires at cluster scope: for barriers
+// the other CTA of the pair arrives on.
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool hq_wait_cl(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
+  if (mbar_try_wait_cl(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+__device__ __forceinline__ bool hq_wait_warp_cl(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                                 volatile int* abort) {
-  if (limit <= 0 || limit >= SS || it < (uint32_t)limit) return true;
-  const uint32_t j = it - (uint32_t)limit;
+  const bool ok = hq_wait_cl(bar, parity, limit_ns, abort);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Producer: before issuing iteration `it` of a ring of SS stages, wait
+// until iteration it - lim has been consumed, so that at most lim stages are
+// in flight (lim in 1..SS; lim = SS is the plain ring, waiting for the
+// slot's previous use).  The slot of it - lim is next refilled at
+// it - lim + SS >= it, by this call's caller at the earliest, so its empty
+// barrier cannot have moved past that phase: the parity wait is exact.
+// Returns false when the bounded wait gave up.
+template <int SS>
+__device__ __forceinline__ bool wait_stage_free(uint64_t* empty, uint32_t it, uint32_t lim, uint64_t wait_ns,
+                                                volatile int* abort) {
+  if (it < lim) return true;
+  const uint32_t j = it - lim;
   return hq_wait_warp(&empty[j % SS], (j / SS) & 1, wait_ns, abort);
 }
 
@@ -326,6 +381,71 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, u
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
           d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// The same operations issued for a CTA pair (cta_group::2, rank 0 issues):
+// every shared-memory and TMEM address names the same offset in both CTAs.
+// The MMA's M is 256: rows 0-127 come from (and accumulate in) rank 0,
+// rows 128-255 in rank 1; B's N columns are split in halves the same way,
+// each CTA holding its half; each CTA's TMEM holds its rows' scale factors
+// and the scale factors of all N columns.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Arrive once on the mbarrier at bar's offset in both CTAs of the pair
+// when every tcgen05 operation this thread issued so far is done.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+// As tc_commit_pair, on this CTA's barrier only.
+__device__ __forceinline__ void tc_commit_pair_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void mma_mxf8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// 2-D tiled tensor copy global -> this CTA's shared memory whose completion
+// is counted on an mbarrier of either CTA of the pair (bar_cluster, a
+// shared::cluster address); no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
       : "memory");
 }
 

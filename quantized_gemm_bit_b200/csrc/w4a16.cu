@@ -335,7 +335,7 @@ __device__ __forceinline__ void mxi4_dequant_block(const uint8_t* rec, int r, ui
   }
 }
 
-template <int NTOK, int FMT>
+template <int NTOK, int FMT, bool SW>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
   using C = Cfg<NTOK, FMT>;
@@ -409,12 +409,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Phase 1, before the previous kernel has finished: the packed weights
     // of the first SS stages (no kernel writes them)
     uint32_t n_pre = 0;
+    // stages in flight: the whole ring unless the caller asked for fewer
+    const uint32_t lim = (p.stage_limit > 0 && p.stage_limit < SS) ? (uint32_t)p.stage_limit : (uint32_t)SS;
     if (!p.grouped) {
-      const uint32_t depth = (p.stage_limit > 0 && p.stage_limit < SS) ? (uint32_t)p.stage_limit : (uint32_t)SS;
-      for (int idx = 0; p.early_weights && n_pre < depth && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
+      for (int idx = 0; p.early_weights && n_pre < lim && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
            ++idx) {
         const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
-        for (int kb = x.kb0; kb < x.kb1 && n_pre < depth; kb += KPS, ++n_pre) {
+        for (int kb = x.kb0; kb < x.kb1 && n_pre < lim; kb += KPS, ++n_pre) {
           const int nrec = min(KPS, x.kb1 - kb);
           if (leader) {
             uint64_t* fb = full_bar(n_pre);
@@ -435,10 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.packed + (uint64_t)x.expert * p.expert_bytes + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS;
-        const uint32_t ph = (it / SS) & 1;
         const int nrec = min(KPS, x.kb1 - kb);
-        if ((it >= n_pre && !hq_wait_warp(&empty[s], ph ^ 1, p.wait_ns, s_abort)) ||
-            !throttle_stages<SS>(empty, it, p.stage_limit, p.wait_ns, s_abort)) {
+        if (!wait_stage_free<SS>(empty, it, lim, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -619,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[EB];
 #pragma unroll
         for (int j = 0; j < EB; ++j) v[j] = __uint_as_float(j < 16 ? v0[j] : v1[j - 16]);
-        store_chunk<EB>(p, x, part, (int)q, (int)lane, j0, v, sc);
+        store_chunk<EB, SW>(p, x, part, (int)q, (int)lane, j0, v, sc);
       }
       tc_fence_before();
       __syncwarp();
@@ -636,9 +635,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
-template <int NTOK, int FMT = kFmtInt4>
+template <int NTOK, int FMT, bool SW>
 hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_kernel<NTOK, FMT>;
+  auto kern = w4a16_kernel<NTOK, FMT, SW>;
   const size_t smem = Cfg<NTOK, FMT>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -649,6 +648,25 @@ hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStre
     attr_set[dev] = true;
   }
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, map, p) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+// One format's launch for a token tile, with or without the SwiGLU epilogue.
+template <int FMT, bool SW>
+hq_status launch_tiles(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+  switch (ntok) {
+    case 16: return launch_t<16, FMT, SW>(map, p, grid, stream);
+    case 32: return launch_t<32, FMT, SW>(map, p, grid, stream);
+    case 64: return launch_t<64, FMT, SW>(map, p, grid, stream);
+    case 128: return launch_t<128, FMT, SW>(map, p, grid, stream);
+    case 256: return launch_t<256, FMT, SW>(map, p, grid, stream);
+    default: return HQ_ERR_UNSUPPORTED;
+  }
+}
+template <int FMT>
+hq_status launch_fmt(int ntok, bool swiglu, const CUtensorMap& map, const W4Params& p, int grid,
+                     cudaStream_t stream) {
+  return swiglu ? launch_tiles<FMT, true>(ntok, map, p, grid, stream)
+                : launch_tiles<FMT, false>(ntok, map, p, grid, stream);
 }
 
 int dense_tiles(const hq_quant_desc& d, int m, int ntok) {
@@ -820,7 +838,6 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.grouped = grouped ? 1 : 0;
   p.wait_ns = kDefaultWaitNs;
   p.early_weights = cfg.early_weights;
-  p.swiglu = swiglu;
   p.stage_limit = cfg.stages;
   if (grouped) {
     // an expert's weight tile is re-read by each of its token tiles
@@ -855,61 +872,14 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   // bf16 already) and on request (variant 1).
   const int kfmt = int3 ? kFmtInt3 : int2 ? kFmtInt2 : int8 ? kFmtInt8 : kFmtInt4;
   const bool exact = !mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1;
-  if (exact) return small_launch(cfg.ntok, kfmt, map, p, cfg.grid, stream);
-  auto by_tile = [&](auto f16, auto f32, auto f64, auto f128, auto f256) -> hq_status {
-    switch (cfg.ntok) {
-      case 16: return f16(map, p, cfg.grid, stream);
-      case 32: return f32(map, p, cfg.grid, stream);
-      case 64: return f64(map, p, cfg.grid, stream);
-      case 128: return f128(map, p, cfg.grid, stream);
-      case 256: return f256(map, p, cfg.grid, stream);
-      default: return HQ_ERR_UNSUPPORTED;
-    }
-  };
-  if (mxi4)
-    return by_tile(launch_t<16, kFmtMxi4>, launch_t<32, kFmtMxi4>, launch_t<64, kFmtMxi4>, launch_t<128, kFmtMxi4>,
-                   launch_t<256, kFmtMxi4>);
-  if (int8)
-    return by_tile(launch_t<16, kFmtInt8>, launch_t<32, kFmtInt8>, launch_t<64, kFmtInt8>, launch_t<128, kFmtInt8>,
-                   launch_t<256, kFmtInt8>);
-  if (mx) {
-    switch (cfg.ntok) {
-      case 16: return launch_t<16, kFmtMx>(map, p, cfg.grid, stream);
-      case 32: return launch_t<32, kFmtMx>(map, p, cfg.grid, stream);
-      case 64: return launch_t<64, kFmtMx>(map, p, cfg.grid, stream);
-      case 128: return launch_t<128, kFmtMx>(map, p, cfg.grid, stream);
-      case 256: return launch_t<256, kFmtMx>(map, p, cfg.grid, stream);
-      default: return HQ_ERR_UNSUPPORTED;
-    }
-  }
-  if (int3) {
-    switch (cfg.ntok) {
-      case 16: return launch_t<16, kFmtInt3>(map, p, cfg.grid, stream);
-      case 32: return launch_t<32, kFmtInt3>(map, p, cfg.grid, stream);
-      case 64: return launch_t<64, kFmtInt3>(map, p, cfg.grid, stream);
-      case 128: return launch_t<128, kFmtInt3>(map, p, cfg.grid, stream);
-      case 256: return launch_t<256, kFmtInt3>(map, p, cfg.grid, stream);
-      default: return HQ_ERR_UNSUPPORTED;
-    }
-  }
-  if (int2) {
-    switch (cfg.ntok) {
-      case 16: return launch_t<16, kFmtInt2>(map, p, cfg.grid, stream);
-      case 32: return launch_t<32, kFmtInt2>(map, p, cfg.grid, stream);
-      case 64: return launch_t<64, kFmtInt2>(map, p, cfg.grid, stream);
-      case 128: return launch_t<128, kFmtInt2>(map, p, cfg.grid, stream);
-      case 256: return launch_t<256, kFmtInt2>(map, p, cfg.grid, stream);
-      default: return HQ_ERR_UNSUPPORTED;
-    }
-  }
-  switch (cfg.ntok) {
-    case 16: return launch_t<16>(map, p, cfg.grid, stream);
-    case 32: return launch_t<32>(map, p, cfg.grid, stream);
-    case 64: return launch_t<64>(map, p, cfg.grid, stream);
-    case 128: return launch_t<128>(map, p, cfg.grid, stream);
-    case 256: return launch_t<256>(map, p, cfg.grid, stream);
-    default: return HQ_ERR_UNSUPPORTED;
-  }
+  if (exact) return small_launch(cfg.ntok, kfmt, swiglu != 0, map, p, cfg.grid, stream);
+  const bool sw = swiglu != 0;
+  if (mx) return launch_fmt<kFmtMx>(cfg.ntok, sw, map, p, cfg.grid, stream);
+  if (mxi4) return launch_fmt<kFmtMxi4>(cfg.ntok, sw, map, p, cfg.grid, stream);
+  if (int8) return launch_fmt<kFmtInt8>(cfg.ntok, sw, map, p, cfg.grid, stream);
+  if (int3) return launch_fmt<kFmtInt3>(cfg.ntok, sw, map, p, cfg.grid, stream);
+  if (int2) return launch_fmt<kFmtInt2>(cfg.ntok, sw, map, p, cfg.grid, stream);
+  return launch_fmt<kFmtInt4>(cfg.ntok, sw, map, p, cfg.grid, stream);
 }
 
 }  // namespace hq

@@ -61,7 +61,6 @@ struct W4Params {
   int weights_once;                  // each weight tile is read by one CTA
   int data_parallel;                 // dense: whole tiles per unit, no partials
   int early_weights;                 // dense: fetch the first stages' weights before griddepcontrol.wait
-  int swiglu;                        // grouped: gated gate+up weights, write h = silu(gate) * up [rows][n/2]
   int stage_limit;                   // pipeline stages in flight (0 or >= the ring depth: the whole ring)
 };
 
@@ -187,13 +186,16 @@ __device__ __forceinline__ void grouped_tables(const W4Params& p, int* s_off, in
 
 // Writes tokens j0 .. j0+EB-1 of one epilogue warp's 32 weight rows (row
 // n = nt*128 + 32q + lane holds v[j] for token j0+j): fp32 into this CTA's
-// partial slot for a partial unit, else bf16 output (store_rows_chunk); for
-// gated gate+up weights the SwiGLU of the warp's 16 gate/up row pairs, 16
-// features of h from feature nt*64 + 16q (store_swiglu_chunk).
-template <int EB>
+// partial slot for a partial unit, else bf16 output (store_rows_chunk); with
+// SW (grouped gate+up weights in the gated row order, written as
+// h = silu(gate) * up [rows][n/2]) the SwiGLU of the warp's 16 gate/up row
+// pairs, 16 features of h from feature nt*64 + 16q (store_swiglu_chunk).
+// SW is a kernel template parameter: the SwiGLU code would otherwise weigh
+// on every other kernel's epilogue (measured ~4 % at M=4096 on B200).
+template <int EB, bool SW>
 __device__ __forceinline__ void store_chunk(const W4Params& p, const Unit& x, float* part, int q, int lane, int j0,
                                             const float (&v)[EB], uint16_t* sc) {
-  if (p.swiglu)
+  if constexpr (SW)
     store_swiglu_chunk<EB>(p.c, p.n >> 1, x.row0, x.rows, x.nt * (kTileN / 2) + q * 16, lane, j0, v, sc);
   else
     store_rows_chunk<EB>(p.c, p.n, x.row0, x.rows, x.nt * kTileN + q * 32, q * 32 + lane, part, lane, j0, v, sc);
@@ -262,7 +264,8 @@ __device__ __noinline__ void sk_fixup(const W4Params& p, const Unit& x, int q, i
 // Host side: the exact-weight kernel's ring depth, and its launch (16, 32 or
 // 64 tokens; INT4, INT3, INT2 or INT8 records).
 int small_ring_depth(int ntok, int fmt);
-hq_status small_launch(int ntok, int fmt, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream);
+hq_status small_launch(int ntok, int fmt, bool swiglu, const CUtensorMap& map, const W4Params& p, int grid,
+                       cudaStream_t stream);
 
 }  // namespace w4
 }  // namespace hq

@@ -21,11 +21,11 @@
 //   * each pipeline stage holds two 128-K records; its MMAs write one fresh
 //     fp32 tile D_g (128 x NTOK) per group g into a TMEM ring instead of
 //     accumulating across K;
-//   * warps 8 and up unpack codes cooperatively (16 warps for 16/32 tokens,
-//     each a quarter of a stage's 32-row slices; 8 warps for 64 tokens), so
-//     a stage is ready as soon as possible, many independent warps hide the
-//     latency of the integer unpacking, and a 3-deep TMEM ring lets them run
-//     ahead of the MMA;
+//   * warps 8 and up unpack codes in groups of four warps (one per 32-row
+//     quarter; three groups for 16/32 tokens, two for 64), each group
+//     owning every stage it == g (mod groups) and one TMEM weight slot, so
+//     several stages are unpacked at once and the groups run ahead of the
+//     MMA;
 //   * warps 4-7 ("scale warps") read s for their 32 rows from the stage in
 //     shared memory, then fold s * D_g into fp32 registers as each D_g
 //     lands, and write the output (or the stream-K partial) when a unit
@@ -187,7 +187,7 @@ __device__ __forceinline__ void unpack_stage(const uint8_t* recs, int rec_bytes,
   }
 }
 
-template <int NTOK, int FMT>
+template <int NTOK, int FMT, bool SW>
 __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
     w4a16_small_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
   using C = SmallCfg<NTOK, FMT>;
@@ -258,12 +258,13 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
     // Phase 1, before the previous kernel has finished: the packed weights
     // of the first SS stages (no kernel writes them)
     uint32_t n_pre = 0;
+    // stages in flight: the whole ring unless the caller asked for fewer
+    const uint32_t lim = (p.stage_limit > 0 && p.stage_limit < SS) ? (uint32_t)p.stage_limit : (uint32_t)SS;
     if (!p.grouped) {
-      const uint32_t depth = (p.stage_limit > 0 && p.stage_limit < SS) ? (uint32_t)p.stage_limit : (uint32_t)SS;
-      for (int idx = 0; p.early_weights && n_pre < depth && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
+      for (int idx = 0; p.early_weights && n_pre < lim && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x);
            ++idx) {
         const uint8_t* wbase = p.packed + (uint64_t)x.nt * p.k_blocks * p.rec_bytes;
-        for (int kb = x.kb0; kb < x.kb1 && n_pre < depth; kb += KPS, ++n_pre) {
+        for (int kb = x.kb0; kb < x.kb1 && n_pre < lim; kb += KPS, ++n_pre) {
           const int nrec = min(KPS, x.kb1 - kb);
           if (leader) {
             uint64_t* fb = full_bar(n_pre);
@@ -285,8 +286,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS;
         const int nrec = min(KPS, x.kb1 - kb);
-        if ((it >= n_pre && !hq_wait_warp(&empty[s], ((it / SS) & 1) ^ 1, p.wait_ns, s_abort)) ||
-            !throttle_stages<SS>(empty, it, p.stage_limit, p.wait_ns, s_abort)) {
+        if (!wait_stage_free<SS>(empty, it, lim, p.wait_ns, s_abort)) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
         float v[CH];
 #pragma unroll
         for (int j = 0; j < CH; ++j) v[j] = acc[j0 + j];
-        store_chunk<CH>(p, x, part, (int)q, (int)lane, j0, v, scr);
+        store_chunk<CH, SW>(p, x, part, (int)q, (int)lane, j0, v, scr);
       }
       if (x.partial) sk_fixup<NTOK, (C::kThreads > 512 ? 2 : 4)>(p, x, (int)q, (int)lane);
     }
@@ -495,9 +495,9 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
   if (warp == 2) tmem_dealloc(*s_tmem, 512);
 }
 
-template <int NTOK, int FMT>
+template <int NTOK, int FMT, bool SW>
 hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_small_kernel<NTOK, FMT>;
+  auto kern = w4a16_small_kernel<NTOK, FMT, SW>;
   using C = SmallCfg<NTOK, FMT>;
   const size_t smem = C::kSmem;
   static bool attr_set[64] = {};
@@ -511,14 +511,21 @@ hq_status launch_small_t(const CUtensorMap& map, const W4Params& p, int grid, cu
   return launch_pdl(kern, dim3(grid), dim3(C::kThreads), smem, stream, map, p) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
 }
 
-template <int FMT>
+template <int FMT, bool SW>
 hq_status small_launch_f(int ntok, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
   switch (ntok) {
-    case 16: return launch_small_t<16, FMT>(map, p, grid, stream);
-    case 32: return launch_small_t<32, FMT>(map, p, grid, stream);
-    case 64: return launch_small_t<64, FMT>(map, p, grid, stream);
+    case 16: return launch_small_t<16, FMT, SW>(map, p, grid, stream);
+    case 32: return launch_small_t<32, FMT, SW>(map, p, grid, stream);
+    case 64: return launch_small_t<64, FMT, SW>(map, p, grid, stream);
     default: return HQ_ERR_UNSUPPORTED;
   }
+}
+
+template <int FMT>
+hq_status small_launch_sw(int ntok, bool swiglu, const CUtensorMap& map, const W4Params& p, int grid,
+                          cudaStream_t stream) {
+  return swiglu ? small_launch_f<FMT, true>(ntok, map, p, grid, stream)
+                : small_launch_f<FMT, false>(ntok, map, p, grid, stream);
 }
 
 }  // namespace
@@ -540,12 +547,13 @@ int small_ring_depth(int ntok, int fmt) {
   }
 }
 
-hq_status small_launch(int ntok, int fmt, const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+hq_status small_launch(int ntok, int fmt, bool swiglu, const CUtensorMap& map, const W4Params& p, int grid,
+                       cudaStream_t stream) {
   switch (fmt) {
-    case kFmtInt4: return small_launch_f<kFmtInt4>(ntok, map, p, grid, stream);
-    case kFmtInt3: return small_launch_f<kFmtInt3>(ntok, map, p, grid, stream);
-    case kFmtInt2: return small_launch_f<kFmtInt2>(ntok, map, p, grid, stream);
-    case kFmtInt8: return small_launch_f<kFmtInt8>(ntok, map, p, grid, stream);
+    case kFmtInt4: return small_launch_sw<kFmtInt4>(ntok, swiglu, map, p, grid, stream);
+    case kFmtInt3: return small_launch_sw<kFmtInt3>(ntok, swiglu, map, p, grid, stream);
+    case kFmtInt2: return small_launch_sw<kFmtInt2>(ntok, swiglu, map, p, grid, stream);
+    case kFmtInt8: return small_launch_sw<kFmtInt8>(ntok, swiglu, map, p, grid, stream);
     default: return HQ_ERR_UNSUPPORTED;
   }
 }

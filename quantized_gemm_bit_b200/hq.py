@@ -72,7 +72,8 @@ class TuningEntry(ctypes.Structure):
 
 class Plan(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int32) for f in
-                ("kernel", "tile_m", "grid", "split", "whole_tiles", "stages", "ring_stages", "from_table")] + \
+                ("kernel", "tile_m", "grid", "split", "whole_tiles", "stages", "ring_stages", "from_table",
+                 "cta_group")] + \
                [("workspace_bytes", ctypes.c_size_t)]
 
 

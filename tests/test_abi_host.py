@@ -267,6 +267,17 @@ def test_gemm_argument_errors_need_no_gpu():
     t = hq.Tuning(variant=1)
     assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dm), 4096, 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                                None) == hq.HQ_ERR_UNSUPPORTED
+    # CTA pairs (cta_group 2): 256-row weight tiles (N a multiple of 256),
+    # 128- or 256-token tiles, whole tiles (no K split); no third group
+    dm2 = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 384, 256, 32, 0, 1)
+    dn2 = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, 256, 256, 16, 0, 1)
+    for dd, bad in ((dm2, hq.Tuning(cta_group=2)), (dm, hq.Tuning(cta_group=2, tile_m=64)),
+                    (dm, hq.Tuning(cta_group=2, split_k=2)), (dm, hq.Tuning(cta_group=3))):
+        assert L_.hq_gemm_mxfp4_a8(ctypes.byref(dd), 4096, 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
+                                   None) == hq.HQ_ERR_UNSUPPORTED
+    bad = hq.Tuning(cta_group=2, tile_m=32)
+    assert L_.hq_gemm_nvfp4(ctypes.byref(dn2), 4096, 16, 16, ctypes.c_float(1.0), 4, 32, ctypes.byref(bad), 256,
+                            1 << 20, None) == hq.HQ_ERR_UNSUPPORTED
     # routing arguments
     assert L_.hq_moe_topk(None, 4, 8, 0, None, None) == hq.HQ_ERR_INVALID_ARG
     assert L_.hq_moe_topk(None, 4, 4, 8, None, None) == hq.HQ_ERR_INVALID_ARG

@@ -148,3 +148,78 @@ def test_nvfp4_full_size(m, n, k):
     ref = G.nvfp4_ref(*act, *w, rows=rows, cols=cols)
     got = c[torch.from_numpy(rows).to(DEV)][:, torch.from_numpy(cols).to(DEV)]
     check_gemm(got, ref, k, f"nvfp4 full m={m} n={n} k={k}")
+
+
+# ---------------------------------------------------------------- CTA pairs (cta_group::2)
+
+@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("m,n,k", [(300, 512, 1024), (129, 768, 640)])
+def test_mxfp4_cta_pairs(m, n, k, tile_m):
+    """256-row weight tiles on CTA pairs (cta_group::2 MMAs, each CTA
+    staging its 128 weight rows and half of the token tile): every output
+    against the oracle, a ragged last token tile, and the same call twice
+    gives the same bits."""
+    d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 600 + m)
+    t = hq.Tuning(tile_m=tile_m, cta_group=2)
+    c1 = mx_run(d, blob, aq, asc, m, t)
+    c2 = mx_run(d, blob, aq, asc, m, t)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8), k, f"mxfp4 pairs {tile_m} m={m} n={n}")
+
+
+@pytest.mark.parametrize("tile_m", [128, 256])
+@pytest.mark.parametrize("m,n,k", [(300, 512, 1024), (129, 768, 1536)])
+def test_nvfp4_cta_pairs(m, n, k, tile_m):
+    d, blob, act, w = nv_case(m, n, k, 700 + m)
+    t = hq.Tuning(tile_m=tile_m, cta_group=2)
+    c1 = nv_run(d, blob, act, m, t)
+    c2 = nv_run(d, blob, act, m, t)
+    assert torch.equal(c1, c2)
+    check_gemm(c1, G.nvfp4_ref(*act, *w), k, f"nvfp4 pairs {tile_m} m={m} n={n}")
+
+
+def test_cta_pairs_more_tiles_than_clusters():
+    """More (token tile, 256-row weight tile) units than resident clusters:
+    every cluster runs several units, accumulators alternating."""
+    m, n, k = 1100, 4096, 512
+    d, blob, act, w = nv_case(m, n, k, 720)
+    c = nv_run(d, blob, act, m, hq.Tuning(tile_m=128, cta_group=2))
+    rows = tile_rows(m, 128, np.random.default_rng(5))
+    ref = G.nvfp4_ref(*act, *w, rows=rows)
+    check_gemm(c[torch.from_numpy(rows).to(DEV)], ref, k, "nvfp4 pairs, many units")
+
+
+@pytest.mark.parametrize("m,n,k", [(8192, 8192, 8192)])
+def test_nvfp4_one_cta_per_tile_full_size(m, n, k):
+    """The library runs this size on CTA pairs; one CTA per 128-row weight
+    tile (cta_group 1) must give the same results."""
+    d, blob, act, w = nv_case(m, n, k, 4000)
+    plan = hq.hq_plan_describe(d, m, hq.Tuning(cta_group=1))
+    assert plan.tile_m == 256 and plan.split == 0 and plan.cta_group == 1
+    c = nv_run(d, blob, act, m, hq.Tuning(cta_group=1))
+    rng = np.random.default_rng(m + 1)
+    rows = tile_rows(m, 256, rng, per_tile=1)
+    cols = np.array(sorted({c0 for nt in range(n // 128)
+                            for c0 in (nt * 128, nt * 128 + 127, nt * 128 + int(rng.integers(0, 128)))}))
+    ref = G.nvfp4_ref(*act, *w, rows=rows, cols=cols)
+    got = c[torch.from_numpy(rows).to(DEV)][:, torch.from_numpy(cols).to(DEV)]
+    check_gemm(got, ref, k, f"nvfp4 one CTA per tile, full m={m} n={n} k={k}")
+
+
+def test_mxfp4_one_cta_per_tile_full_size():
+    m = 4096
+    n = k = 7168
+    d, blob, aq, asc, codes, e8 = mx_case(m, n, k, 2000 + m)
+    c = mx_run(d, blob, aq, asc, m, hq.Tuning(cta_group=1))
+    rows = tile_rows(m, 128, np.random.default_rng(m + 1))
+    ref = G.mxfp4_a8_ref(aq.numpy(), asc.numpy(), codes, e8, rows=rows)
+    check_gemm(c[torch.from_numpy(rows).to(DEV)], ref, k, f"mxfp4 one CTA per tile, full m={m}")
+
+
+def test_large_tiles_default_to_cta_pairs():
+    """The plan the full-size workloads run: 256-token whole tiles on CTA
+    pairs (grid = two CTAs per resident cluster)."""
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, 8192, 8192, 16, 0, 1)
+    plan = hq.hq_plan_describe(d, 8192)
+    assert (plan.tile_m, plan.split, plan.cta_group, plan.grid % 2) == (256, 0, 2, 0)
+    assert hq.hq_plan_describe(d, 8192, hq.Tuning(cta_group=1)).cta_group == 1
