@@ -123,8 +123,8 @@ typedef struct {
  *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
  *              splits the whole iteration space evenly when 0)
  *   cta_group: block-scaled GEMMs: 0 = the library's choice (CTA pairs
- *              for 256-token whole tiles when N is a multiple of 256
- *              and the pairs fill the SMs), 1 = one CTA per 128-row
+ *              for 128/256-token whole tiles when N is a multiple of
+ *              256 and the pairs fill the SMs), 1 = one CTA per 128-row
  *              weight tile, 2 = CTA pairs: clusters of two CTAs run
  *              256-row weight tiles with cta_group::2 MMAs (each CTA
  *              stages its 128 weight rows and half of the token tile);

@@ -782,16 +782,18 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   if (pick || dp_eff(ntok) >= 0.85) {
     cfg.splits = 0;
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
-    // 256-token whole tiles run on CTA pairs when the pairs' waves are as
-    // full (the caller may ask for one CTA per tile with cta_group 1).
-    // Measured on B200: NVFP4 8192^3 247 -> 207 us, M=16384 K=7168
-    // N=18432 1008 -> 923 us; MXFP4 M=4096 K=N=7168 162 -> 150 us.
-    if (ntok == 256 && d.n % 256 == 0 && !(t && t->cta_group == 1)) {
-      const long long pair_tiles = (long long)(d.n / 256) * ((m + 255) / 256);
-      const long long slots = bs_pair_slots(d.fmt == HQ_FMT_NVFP4, 256);
+    // 128/256-token whole tiles run on CTA pairs when the pairs' waves are
+    // as full (the caller may ask for one CTA per tile with cta_group 1).
+    // Measured on B200, one CTA per tile -> pairs: NVFP4 8192^3 244 -> 204
+    // us, M=16384 K=7168 N=18432 990 -> 898 us, M=256 K=N=8192 20.7 ->
+    // 17.9 us; MXFP4 K=N=7168 M=4096 159 -> 147 us, M=2048 128 -> 109 us,
+    // M=256 23.2 -> 21.5 us.
+    if (ntok >= 128 && d.n % 256 == 0 && !(t && t->cta_group == 1)) {
+      const long long pair_tiles = (long long)(d.n / 256) * ((m + ntok - 1) / ntok);
+      const long long slots = bs_pair_slots(d.fmt == HQ_FMT_NVFP4, ntok);
       if (slots > 0) {
         const long long waves = (pair_tiles + slots - 1) / slots;
-        if ((double)pair_tiles / (double)(waves * slots) >= 0.85) {
+        if ((double)pair_tiles / (double)(waves * slots) >= dp_eff(ntok) - 0.02) {
           cfg.cta_group = 2;
           cfg.grid = (int)(2 * std::min<long long>(slots, pair_tiles));
         }
