@@ -34,11 +34,13 @@ def main(argv=None):
     ap.add_argument("--split-k", type=int, default=0)
     ap.add_argument("--variant", type=int, default=0)
     ap.add_argument("--stages", type=int, default=0)
+    ap.add_argument("--cta-group", type=int, default=0, help="block-scaled: 1 = one CTA per tile, 2 = CTA pairs")
     a = ap.parse_args(argv)
     build()
     dev = "cuda"
-    tuning = (hq.Tuning(tile_m=a.tile_m, split_k=a.split_k, variant=a.variant, stages=a.stages)
-              if (a.tile_m or a.split_k or a.variant or a.stages) else None)
+    tuning = (hq.Tuning(tile_m=a.tile_m, split_k=a.split_k, variant=a.variant, stages=a.stages,
+                        cta_group=a.cta_group)
+              if (a.tile_m or a.split_k or a.variant or a.stages or a.cta_group) else None)
     if a.kind in ("mxfp4", "nvfp4"):
         ws = None
         if a.kind == "mxfp4":
