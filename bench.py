@@ -63,23 +63,23 @@ def load_peaks():
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
 # capture is taken again.
-TRAFFIC_COMMIT = "dcb06b2"
-TRAFFIC_SOURCES = "0ae0b77bd91ff581"
+TRAFFIC_COMMIT = "ca770ba"
+TRAFFIC_SOURCES = "a8780046785d559f"
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 71160064,
-    (4, 7168, 18432): 69321728,
-    (16, 7168, 18432): 69740288,
-    (64, 7168, 18432): 70749696,
-    (256, 7168, 18432): 76625152,
-    (1024, 7168, 18432): 180431104,
-    (4096, 7168, 18432): 499533056,
-    (1, 18432, 7168): 70045184,
-    (4, 18432, 7168): 70405376,
-    (16, 18432, 7168): 71154432,
-    (64, 18432, 7168): 73819392,
-    (256, 18432, 7168): 88400128,
-    (1024, 18432, 7168): 200986624,
-    (4096, 18432, 7168): 726529536,
+    (1, 7168, 18432): 70243840,
+    (4, 7168, 18432): 69139712,
+    (16, 7168, 18432): 69765376,
+    (64, 7168, 18432): 70627328,
+    (256, 7168, 18432): 75611648,
+    (1024, 7168, 18432): 166250496,
+    (4096, 7168, 18432): 452718336,
+    (1, 18432, 7168): 69945856,
+    (4, 18432, 7168): 70013952,
+    (16, 18432, 7168): 70983680,
+    (64, 18432, 7168): 73936640,
+    (256, 18432, 7168): 86089984,
+    (1024, 18432, 7168): 201865728,
+    (4096, 18432, 7168): 724283136,
 }
 
 
