@@ -115,7 +115,20 @@ struct BsParams {
   int early_weights;         // fetch the first stages' weights before griddepcontrol.wait
   int stage_limit;           // pipeline stages in flight (0 or >= the ring depth: the whole ring)
   int n_pairs;               // CTA pairs: 256-row weight tiles (n_tiles / 2)
+  int raster;                // whole-tile order: groups of this many weight tiles (pairs) over all token tiles
 };
+
+// Whole-tile order: unit t -> (token tile, weight tile) in groups of `width`
+// weight tiles, each group walking every token tile before the next group
+// starts, so that the CTAs of one wave share few weight tiles (width =
+// n_w is plain token-tile-major order).
+__device__ __forceinline__ void raster_tile(long long t, int n_w, int m_tiles, int width, int& mt, int& wt) {
+  const long long per_group = (long long)width * m_tiles;
+  const long long g = t / per_group, r = t - g * per_group;
+  const int w = min(width, n_w - (int)g * width);   // the last group may be narrower
+  mt = (int)(r / w);
+  wt = (int)g * width + (int)(r - (long long)mt * w);
+}
 
 // NVFP4 activation scales, row-major [m][K/16] bytes, re-laid into the order
 // tcgen05.cp .32x128b.warpx4 copies into TMEM: per (token tile mt, stage
@@ -149,9 +162,10 @@ __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, i
     const long long ncl = gridDim.x / 2, cl = blockIdx.x / 2;
     const long long t = cl + (long long)idx * ncl;
     if (t >= (long long)p.m_tiles * p.n_pairs) return false;
-    const int mt = (int)(t / p.n_pairs);
+    int mt, pnt;
+    raster_tile(t, p.n_pairs, p.m_tiles, p.raster, mt, pnt);
     tile = (int)t;
-    nt = 2 * (int)(t - (long long)mt * p.n_pairs) + (int)(blockIdx.x & 1);
+    nt = 2 * pnt + (int)(blockIdx.x & 1);
     row0 = mt * NTOK;
     rows = min(NTOK, p.m - row0);
     ks0 = 0;
@@ -163,9 +177,9 @@ __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, i
   if (p.data_parallel) {
     const long long t = (long long)blockIdx.x + (long long)idx * gridDim.x;
     if (t >= (long long)p.m_tiles * p.n_tiles) return false;
-    const int mt = (int)(t / p.n_tiles);
+    int mt;
+    raster_tile(t, p.n_tiles, p.m_tiles, p.raster, mt, nt);
     tile = (int)t;
-    nt = (int)(t - (long long)mt * p.n_tiles);
     row0 = mt * NTOK;
     rows = min(NTOK, p.m - row0);
     ks0 = 0;
@@ -880,6 +894,15 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
   p.early_weights = cfg.early_weights;
   p.stage_limit = cfg.stages;
   p.n_pairs = n_tiles / 2;
+  // Whole-tile order: token-tile-major, except on CTA pairs when the packed
+  // weights outgrow L2's comfortable share (> 48 MB, about 3/8 of it): then
+  // groups of 16 pair tiles, so that a wave's clusters share 15 MB of weights
+  // instead of streaming the whole matrix past the outputs' stores.
+  // Measured on B200: NVFP4 M=16384 K=7168 N=18432 (66 MB) 900 -> 817 us;
+  // at NVFP4 8192^3 (34 MB) and MXFP4 K=N=7168 groups of 4-16 were 0-5 %
+  // slower than token-tile-major.
+  p.raster = n_tiles;
+  if (cfg.cta_group == 2) p.raster = codes_bytes > (size_t)48 << 20 ? std::min(16, p.n_pairs) : p.n_pairs;
   const BsWsLayout L = bs_ws_layout(d, m, cfg);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.counters = reinterpret_cast<int32_t*>(wsb + L.counters);
