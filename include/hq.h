@@ -129,7 +129,10 @@ typedef struct {
  *              256-row weight tiles with cta_group::2 MMAs (each CTA
  *              stages its 128 weight rows and half of the token tile);
  *              needs N % 256 == 0, tile_m 0, 128 or 256, split_k 0.
- *              W4A16: 0 or 1.
+ *              W4A16 (dense): 0 or 1 = one CTA per tile; 2 = CTA pairs
+ *              for 256-token whole tiles (each CTA dequantizes its
+ *              128 rows; N % 256 == 0, tile_m 0 or 256, split_k 0;
+ *              measured slower than one CTA per tile, kept on request).
  *   variant  : W4A16 / grouped MoE: 0 = the library's choice, currently
  *              2 for token tiles of up to 64 and 1 for larger tiles
  *              (MXFP4_A16 weights: always 1).

@@ -47,6 +47,7 @@ struct W4Config {
   int dp_tiles; // stream-K plans: tiles run whole before the shared K range
   int grid;     // CTAs
   int early_weights;  // fetch packed weights before the previous kernel completes
+  int cta_group;      // 2: dense 256-token whole tiles on CTA pairs (cta_group::2 MMAs)
   int variant;  // 0: library's choice (exact weights for tiles of <= 64
                 // tokens, bf16-rescaled above); 1: bf16-rescaled weights for
                 // every tile; 2: exact (q - z) weights + per-group fp32

@@ -45,12 +45,16 @@ namespace {
 
 constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
 
-template <int NTOK, int FMT = kFmtInt4>
+// CG = 2: a CTA pair (cluster of two) runs one 256-row weight tile with
+// cta_group::2 MMAs; each CTA dequantizes its own 128 weight rows into its
+// TMEM and stages half of the token tile.
+template <int NTOK, int FMT = kFmtInt4, int CG = 1>
 struct Cfg {
+  static_assert(CG == 1 || NTOK == 256, "CTA pairs run 256-token tiles");
   // records (128-K blocks) per pipeline stage: two for the small token tiles,
   // whose MMAs are cheap, so the per-stage waits and commits are amortized
   static constexpr int kKps = NTOK <= 64 ? 2 : 1;
-  static constexpr int kABlock = NTOK * 256;                // one record's activations: two 64-K boxes
+  static constexpr int kABlock = NTOK / CG * 256;           // one record's activations (this CTA's): two 64-K boxes
   static constexpr int kATile = kKps * kABlock;
   static constexpr int kRecStride = (FMT == kFmtMx || FMT == kFmtMxi4) ? kMxA16RecBytes
                                     : FMT == kFmtInt3                  ? kW3RecCodes + 384
@@ -61,7 +65,7 @@ struct Cfg {
   static constexpr int kBarBytes = (FMT == kFmtMx || FMT == kFmtMxi4) ? 384 : 512;
   static constexpr int kEpiScratch = NTOK == 256 ? 0 : 4 * 2048;
   // as many SMEM stages as fit, up to a preferred depth per token tile
-  static constexpr int kSmemPref = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : 3;
+  static constexpr int kSmemPref = NTOK == 16 ? 6 : NTOK == 32 ? 6 : NTOK == 64 ? 3 : NTOK == 128 ? 5 : CG == 2 ? 8 : 3;
   // (exact: the budget less the base alignment and the scratch is a
   // multiple of 128, so rounding the tables' end up to 128 stays inside it
   // whenever the unrounded end does)
@@ -335,10 +339,10 @@ __device__ __forceinline__ void mxi4_dequant_block(const uint8_t* rec, int r, ui
   }
 }
 
-template <int NTOK, int FMT, bool SW>
+template <int NTOK, int FMT, bool SW, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmap_a, const W4Params p) {
-  using C = Cfg<NTOK, FMT>;
+  using C = Cfg<NTOK, FMT, CG>;
   constexpr int SS = C::kSmemStages;
   constexpr int TS = C::kTmemStages;
   constexpr int ACC = C::kAccBufs;
@@ -370,17 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
+  // CTA pairs: rank 0 issues the pair's MMAs; the dequantizing and epilogue
+  // warps of both CTAs report to rank 0's barriers
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SS; ++s) mbar_init(&empty[s], 1);
     for (int f = 0; f < C::kFullBars; ++f) mbar_init(&full[f], 1);
     for (int t = 0; t < TS; ++t) {
-      mbar_init(&aready[t], C::kDqWarps);
+      mbar_init(&aready[t], C::kDqWarps * CG);
       mbar_init(&afree[t], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], 4 * CG);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -395,7 +402,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
     grouped_tables<NTOK>(p, s_off, s_prefix, s_total);
   }
-  __syncthreads();   // barriers (and the grouped tables) visible to every role
+  if constexpr (CG == 2) {
+    // the pair's TMEM is allocated by both CTAs together; barriers and the
+    // allocation are visible to both CTAs after the cluster barrier
+    if (warp == 2) {
+      tmem_alloc_pair(s_tmem, 512);
+      tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+  } else {
+    __syncthreads();   // barriers (and the grouped tables) visible to every role
+  }
   const int total_grouped = *s_total;
 
   auto a_col = [](int t) -> uint32_t { return (uint32_t)(t * 64 * KPS); };
@@ -450,10 +469,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (long copies stream HBM much faster than record-sized ones)
             bulk_g2s(sR + s * kRecs, wbase + (uint64_t)kb * p.rec_bytes, (uint32_t)(nrec * p.rec_bytes), fb, pol_w);
           }
+          // (pairs: this CTA's half of the token tile)
+          const int arow = x.row0 + (int)rank * (NTOK / CG);
           for (int r = 0; r < nrec; ++r) {
             uint8_t* a_dst = sA + s * kATile + r * C::kABlock;
-            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, x.row0, fb);
-            tma_load_2d(a_dst + NTOK * 128, &tmap_a, (kb + r) * kBlockK + 64, x.row0, fb);
+            tma_load_2d(a_dst, &tmap_a, (kb + r) * kBlockK, arow, fb);
+            tma_load_2d(a_dst + NTOK / CG * 128, &tmap_a, (kb + r) * kBlockK + 64, arow, fb);
           }
         }
         __syncwarp();
@@ -467,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
   // The producer needs no TMEM, so it starts loading at once; the other
   // roles wait here for the allocation.
-  if (warp == 2) {
+  if (CG == 1 && warp == 2) {
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
   }
@@ -480,14 +501,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (whole warp, elected lane issues)
     // one lane, fixed for the whole kernel, issues every MMA and commit: a
     // commit tracks the tcgen05 operations of the thread that issues it
+    // (pairs: rank 0 only, for both CTAs)
     const bool leader = elect_one();
     uint32_t it = 0, uc = 0;
-    bool ok = true;
+    bool ok = rank == 0;
     Unit x;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
       const int ab = uc % ACC;
       const uint32_t aph = (uc / ACC) & 1;
-      if (!hq_wait_warp(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)) {
+      // (pairs: the epilogue warps of both CTAs arrive)
+      if (!(CG == 2 ? hq_wait_warp_cl(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort)
+                    : hq_wait_warp(&acc_empty[ab], aph ^ 1, p.wait_ns, s_abort))) {
         if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
         ok = false;
         break;
@@ -496,13 +520,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t d_tmem = tmem_base + acc_col(ab);
       // the MMAs cover the unit's valid tokens, rounded up to 16 (a ragged
       // tile of an expert or of the last token rows costs no more tensor
-      // work than it needs); accumulator columns past them are never stored
-      const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)min(NTOK, (x.rows + 15) & ~15));
+      // work than it needs); accumulator columns past them are never stored.
+      // A pair's MMA takes each CTA's half of the tile at a fixed place, so
+      // it always covers the whole tile.
+      const uint32_t idesc = CG == 2 ? idesc_bf16_f32(256, (uint32_t)NTOK)
+                                     : idesc_bf16_f32(128, (uint32_t)min(NTOK, (x.rows + 15) & ~15));
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         const int s = it % SS, t = it % TS;
         const uint32_t ph_t = (it / TS) & 1;
         const int nrec = min(KPS, x.kb1 - kb);
-        if (!hq_wait_warp_n(2, &aready[t], ph_t, full_bar(it), full_par(it), nullptr, 0, p.wait_ns, s_abort)) {
+        // weights of both CTAs in TMEM (their dequantizing warps waited for
+        // their own stage, records and activations alike), this CTA's stage
+        const bool ready = CG == 2 ? (hq_wait_warp_cl(&aready[t], ph_t, p.wait_ns, s_abort) &&
+                                      hq_wait_warp(full_bar(it), full_par(it), p.wait_ns, s_abort))
+                                   : hq_wait_warp_n(2, &aready[t], ph_t, full_bar(it), full_par(it), nullptr, 0,
+                                                    p.wait_ns, s_abort);
+        if (!ready) {
           if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
           ok = false;
           break;
@@ -522,24 +555,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (r < nrec) {
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const uint32_t off = (uint32_t)((r * C::kABlock + (j >> 2) * (NTOK * 128) + (j & 3) * 32) >> 4);
+                const uint32_t off = (uint32_t)((r * C::kABlock + (j >> 2) * (NTOK / CG * 128) + (j & 3) * 32) >> 4);
                 const uint64_t bdesc = ((uint64_t)bhi << 32) | (uint64_t)(blo + off);
-                mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, idesc, (r > 0 || j > 0) ? 1u : acc0);
+                if constexpr (CG == 2)
+                  mma_bf16_ts_pair(d_tmem, a0 + r * 64 + j * 8, bdesc, idesc, (r > 0 || j > 0) ? 1u : acc0);
+                else
+                  mma_bf16_ts(d_tmem, a0 + r * 64 + j * 8, bdesc, idesc, (r > 0 || j > 0) ? 1u : acc0);
               }
             }
           }
-          tc_commit(&empty[s]);
-          tc_commit(&afree[t]);
+          // (pairs: both CTAs' stage slots and weight slots)
+          if constexpr (CG == 2) {
+            tc_commit_pair(&empty[s]);
+            tc_commit_pair(&afree[t]);
+          } else {
+            tc_commit(&empty[s]);
+            tc_commit(&afree[t]);
+          }
         }
         __syncwarp();
       }
       if (!ok) break;
-      if (leader) tc_commit(&acc_full[ab]);
+      if (leader) {
+        if constexpr (CG == 2)
+          tc_commit_pair(&acc_full[ab]);
+        else
+          tc_commit(&acc_full[ab]);
+      }
       __syncwarp();
     }
     // make sure no MMA is still running when TMEM is released
-    if (leader) {
-      tc_commit(drain);
+    if (leader && rank == 0) {
+      if constexpr (CG == 2)
+        tc_commit_pair_local(drain);
+      else
+        tc_commit(drain);
       hq_wait(drain, 0, p.wait_ns, nullptr);
     }
     __syncwarp();
@@ -592,7 +642,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&aready[t]);
+        if (lane == 0) {
+          // (pairs: the MMA issuer is rank 0's)
+          if constexpr (CG == 2)
+            mbar_arrive_cluster(mapa_u32(&aready[t], 0));
+          else
+            mbar_arrive(&aready[t]);
+        }
       }
       if (!ok || !epi) continue;
 
@@ -622,7 +678,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      if (lane == 0) {
+        if constexpr (CG == 2)
+          mbar_arrive_cluster(mapa_u32(&acc_empty[ab], 0));
+        else
+          mbar_arrive(&acc_empty[ab]);
+      }
       if (x.partial) sk_fixup<NTOK>(p, x, (int)q, (int)lane);
     }
   }
@@ -631,23 +692,68 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair's CTAs leave together: rank 0's MMAs read the other CTA's shared
+  // memory and TMEM until rank 0 has drained them
+  if constexpr (CG == 2) cluster_sync();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(*s_tmem, 512);
+  if (warp == 2) {
+    if constexpr (CG == 2)
+      tmem_dealloc_pair(*s_tmem, 512);
+    else
+      tmem_dealloc(*s_tmem, 512);
+  }
 }
 
-template <int NTOK, int FMT, bool SW>
-hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_kernel<NTOK, FMT, SW>;
-  const size_t smem = Cfg<NTOK, FMT>::kSmem;
+template <int NTOK, int FMT, bool SW, int CG>
+bool smem_attr() {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return HQ_ERR_CUDA;
-    attr_set[dev] = true;
+  if (dev < 64 && attr_set[dev]) return true;
+  if (cudaFuncSetAttribute(w4a16_kernel<NTOK, FMT, SW, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Cfg<NTOK, FMT, CG>::kSmem) != cudaSuccess)
+    return false;
+  if (dev < 64) attr_set[dev] = true;
+  return true;
+}
+
+template <int NTOK, int FMT, bool SW, int CG = 1>
+hq_status launch_t(const CUtensorMap& map, const W4Params& p, int grid, cudaStream_t stream) {
+  auto kern = w4a16_kernel<NTOK, FMT, SW, CG>;
+  const size_t smem = Cfg<NTOK, FMT, CG>::kSmem;
+  if (!smem_attr<NTOK, FMT, SW, CG>()) return HQ_ERR_CUDA;
+  const cudaError_t e = CG == 2 ? launch_pdl_pairs(kern, dim3(grid), dim3(kThreads), smem, stream, map, p)
+                                : launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, map, p);
+  return e == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+}
+
+// Clusters of two of the CTA-pair kernel resident at once (0 when the query
+// fails), per device.
+template <int FMT>
+int pair_slots_t() {
+  static int cached[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  if (!smem_attr<256, FMT, false, 2>()) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Cfg<256, FMT, 2>::kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, w4a16_kernel<256, FMT, false, 2>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
   }
-  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, map, p) == cudaSuccess ? HQ_OK : HQ_ERR_CUDA;
+  if (dev < 64) cached[dev] = n;
+  return n;
 }
 
 // One format's launch for a token tile, with or without the SwiGLU epilogue.
@@ -663,10 +769,26 @@ hq_status launch_tiles(int ntok, const CUtensorMap& map, const W4Params& p, int 
   }
 }
 template <int FMT>
-hq_status launch_fmt(int ntok, bool swiglu, const CUtensorMap& map, const W4Params& p, int grid,
+hq_status launch_fmt(int ntok, bool swiglu, bool pairs, const CUtensorMap& map, const W4Params& p, int grid,
                      cudaStream_t stream) {
+  if (pairs) return ntok == 256 && !swiglu ? launch_t<256, FMT, false, 2>(map, p, grid, stream) : HQ_ERR_UNSUPPORTED;
   return swiglu ? launch_tiles<FMT, true>(ntok, map, p, grid, stream)
                 : launch_tiles<FMT, false>(ntok, map, p, grid, stream);
+}
+
+int pair_slots(int kfmt) {
+  switch (kfmt) {
+    case kFmtMx: return pair_slots_t<kFmtMx>();
+    case kFmtMxi4: return pair_slots_t<kFmtMxi4>();
+    case kFmtInt3: return pair_slots_t<kFmtInt3>();
+    case kFmtInt2: return pair_slots_t<kFmtInt2>();
+    case kFmtInt8: return pair_slots_t<kFmtInt8>();
+    default: return pair_slots_t<kFmtInt4>();
+  }
+}
+int kernel_fmt(const hq_quant_desc& d) {
+  return d.fmt == HQ_FMT_MXFP4_A16 ? kFmtMx : d.fmt == HQ_FMT_MXINT4 ? kFmtMxi4 : d.fmt == HQ_FMT_INT3 ? kFmtInt3
+         : d.fmt == HQ_FMT_INT2 ? kFmtInt2 : d.fmt == HQ_FMT_INT8 ? kFmtInt8 : kFmtInt4;
 }
 
 int dense_tiles(const hq_quant_desc& d, int m, int ntok) {
@@ -698,11 +820,23 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   }
   cfg.stages = t ? t->stages : 0;
   cfg.splits = 1;
+  cfg.cta_group = 1;
   cfg.variant = t ? t->variant : 0;
   cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
   if (grouped) {
     cfg.ntok = ntok;
     cfg.grid = dev.num_sms;
+    return cfg;
+  }
+  if (t && t->cta_group == 2) {
+    // CTA pairs on request: 256-token whole tiles, one per resident cluster
+    // at a time
+    cfg.ntok = 256;
+    cfg.splits = 0;
+    cfg.cta_group = 2;
+    const long long pair_tiles = (long long)dense_tiles(d, m, 256) / 2;
+    const long long slots = pair_slots(kernel_fmt(d));
+    cfg.grid = (int)(2 * std::max<long long>(1, std::min<long long>(slots > 0 ? slots : dev.num_sms / 2, pair_tiles)));
     return cfg;
   }
   // Whole tiles on persistent CTAs (no partial sums) when they fill the SMs
@@ -752,6 +886,11 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
     }
     cfg.splits = 0;  // data parallel
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
+    // (CTA pairs for these tiles run only on request, cta_group 2: measured
+    // slower on B200 than one CTA per tile despite 5 pipeline stages instead
+    // of 3, e.g. M=4096 K=7168 N=18432 815 -> 881 us, M=1024 208 -> 223 us;
+    // each record waits for both CTAs' dequantization and one SM issues
+    // both SMs' MMAs)
     return cfg;
   }
   if (ntok >= 128 && tiles * 2 <= dev.num_sms && tiles * (dev.num_sms / tiles) >= 0.85 * dev.num_sms) {
@@ -766,7 +905,8 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
 
 namespace {
 template <int FMT>
-int rescaled_depth(int ntok) {
+int rescaled_depth(int ntok, int cta_group) {
+  if (cta_group == 2) return Cfg<256, FMT, 2>::kSmemStages;
   switch (ntok) {
     case 16: return Cfg<16, FMT>::kSmemStages;
     case 32: return Cfg<32, FMT>::kSmemStages;
@@ -781,19 +921,20 @@ int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg) {
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16, mxi4 = d.fmt == HQ_FMT_MXINT4;
   const int kfmt = d.fmt == HQ_FMT_INT3 ? kFmtInt3 : d.fmt == HQ_FMT_INT2 ? kFmtInt2 : d.fmt == HQ_FMT_INT8 ? kFmtInt8 : kFmtInt4;
   if (!mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1) return small_ring_depth(cfg.ntok, kfmt);
-  if (mx) return rescaled_depth<kFmtMx>(cfg.ntok);
-  if (mxi4) return rescaled_depth<kFmtMxi4>(cfg.ntok);
+  if (mx) return rescaled_depth<kFmtMx>(cfg.ntok, cfg.cta_group);
+  if (mxi4) return rescaled_depth<kFmtMxi4>(cfg.ntok, cfg.cta_group);
   switch (kfmt) {
-    case kFmtInt3: return rescaled_depth<kFmtInt3>(cfg.ntok);
-    case kFmtInt2: return rescaled_depth<kFmtInt2>(cfg.ntok);
-    case kFmtInt8: return rescaled_depth<kFmtInt8>(cfg.ntok);
-    default: return rescaled_depth<kFmtInt4>(cfg.ntok);
+    case kFmtInt3: return rescaled_depth<kFmtInt3>(cfg.ntok, cfg.cta_group);
+    case kFmtInt2: return rescaled_depth<kFmtInt2>(cfg.ntok, cfg.cta_group);
+    case kFmtInt8: return rescaled_depth<kFmtInt8>(cfg.ntok, cfg.cta_group);
+    default: return rescaled_depth<kFmtInt4>(cfg.ntok, cfg.cta_group);
   }
 }
 
 W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4Config cfg) {
   cfg.splits = 0;
   cfg.dp_tiles = 0;
+  cfg.cta_group = 1;
   cfg.grid = (int)std::min<long long>(dev.num_sms, dense_tiles(d, m, cfg.ntok));
   return cfg;
 }
@@ -839,6 +980,8 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   p.wait_ns = kDefaultWaitNs;
   p.early_weights = cfg.early_weights;
   p.stage_limit = cfg.stages;
+  p.cta_pairs = cfg.cta_group == 2 ? 1 : 0;
+  p.n_pairs = p.n_tiles / 2;
   if (grouped) {
     // an expert's weight tile is re-read by each of its token tiles
     p.weights_once = (long long)m <= (long long)cfg.ntok * d.num_experts ? 1 : 0;
@@ -859,7 +1002,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   if (!enc) return HQ_ERR_CUDA;
   cuuint64_t dims[2] = {(cuuint64_t)d.k, (cuuint64_t)m};
   cuuint64_t strides[1] = {(cuuint64_t)d.k * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)cfg.ntok};
+  cuuint32_t box[2] = {64, (cuuint32_t)(cfg.cta_group == 2 ? cfg.ntok / 2 : cfg.ntok)};   // pairs: half a tile
   cuuint32_t estr[2] = {1, 1};
   CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -874,12 +1017,13 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
   const bool exact = !mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1;
   if (exact) return small_launch(cfg.ntok, kfmt, swiglu != 0, map, p, cfg.grid, stream);
   const bool sw = swiglu != 0;
-  if (mx) return launch_fmt<kFmtMx>(cfg.ntok, sw, map, p, cfg.grid, stream);
-  if (mxi4) return launch_fmt<kFmtMxi4>(cfg.ntok, sw, map, p, cfg.grid, stream);
-  if (int8) return launch_fmt<kFmtInt8>(cfg.ntok, sw, map, p, cfg.grid, stream);
-  if (int3) return launch_fmt<kFmtInt3>(cfg.ntok, sw, map, p, cfg.grid, stream);
-  if (int2) return launch_fmt<kFmtInt2>(cfg.ntok, sw, map, p, cfg.grid, stream);
-  return launch_fmt<kFmtInt4>(cfg.ntok, sw, map, p, cfg.grid, stream);
+  const bool pr = cfg.cta_group == 2;
+  if (mx) return launch_fmt<kFmtMx>(cfg.ntok, sw, pr, map, p, cfg.grid, stream);
+  if (mxi4) return launch_fmt<kFmtMxi4>(cfg.ntok, sw, pr, map, p, cfg.grid, stream);
+  if (int8) return launch_fmt<kFmtInt8>(cfg.ntok, sw, pr, map, p, cfg.grid, stream);
+  if (int3) return launch_fmt<kFmtInt3>(cfg.ntok, sw, pr, map, p, cfg.grid, stream);
+  if (int2) return launch_fmt<kFmtInt2>(cfg.ntok, sw, pr, map, p, cfg.grid, stream);
+  return launch_fmt<kFmtInt4>(cfg.ntok, sw, pr, map, p, cfg.grid, stream);
 }
 
 }  // namespace hq

@@ -61,6 +61,8 @@ struct W4Params {
   int weights_once;                  // each weight tile is read by one CTA
   int data_parallel;                 // dense: whole tiles per unit, no partials
   int early_weights;                 // dense: fetch the first stages' weights before griddepcontrol.wait
+  int cta_pairs;                     // dense, whole tiles on CTA pairs (clusters of two, 256-row weight tiles)
+  int n_pairs;                       // CTA pairs: n_tiles / 2
   int stage_limit;                   // pipeline stages in flight (0 or >= the ring depth: the whole ring)
 };
 
@@ -95,6 +97,24 @@ __device__ __forceinline__ bool get_unit(const W4Params& p, const int* s_prefix,
     x.partial = 0;
     x.slot = 0;
   };
+  if (p.cta_pairs) {
+    // whole (token tile, 256-row weight tile) units over the clusters; CTA
+    // rank r of the pair owns 128-row weight tile 2 * pair + r
+    const long long ncl = gridDim.x / 2, cl = blockIdx.x / 2;
+    const long long t = cl + (long long)idx * ncl;
+    if (t >= (long long)p.m_tiles * p.n_pairs) return false;
+    const int mt = (int)(t / p.n_pairs);
+    x.tile = (int)t;
+    x.nt = 2 * (int)(t - (long long)mt * p.n_pairs) + (int)(blockIdx.x & 1);
+    x.expert = 0;
+    x.row0 = mt * NTOK;
+    x.rows = min(NTOK, p.m - x.row0);
+    x.kb0 = 0;
+    x.kb1 = p.k_blocks;
+    x.partial = 0;
+    x.slot = 0;
+    return true;
+  }
   if (!p.grouped && p.data_parallel) {
     // whole tiles, strided over the persistent CTAs
     const long long tile = (long long)blockIdx.x + (long long)idx * gridDim.x;

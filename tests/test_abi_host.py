@@ -241,15 +241,20 @@ def test_gemm_argument_errors_need_no_gpu():
     t = hq.Tuning(tile_m=48)
     assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                             None) == hq.HQ_ERR_UNSUPPORTED
-    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=-1), hq.Tuning(cta_group=2),
-                hq.Tuning(flags=2)):
+    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=-1), hq.Tuning(cta_group=3),
+                hq.Tuning(cta_group=2, tile_m=128), hq.Tuning(cta_group=2, split_k=2), hq.Tuning(flags=2)):
         assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
                                 None) == hq.HQ_ERR_UNSUPPORTED
     # grouped: no K split, no 512-token tile; block-scaled: no variants
     dg = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 256, 256, 128, 0, 8)
-    for bad in (hq.Tuning(tile_m=512), hq.Tuning(split_k=2)):
+    for bad in (hq.Tuning(tile_m=512), hq.Tuning(split_k=2), hq.Tuning(cta_group=2)):
         assert L_.hq_grouped_gemm_moe(ctypes.byref(dg), 16, 16, 16, 40, 32, ctypes.byref(bad), 256, 1 << 20,
                                       None) == hq.HQ_ERR_UNSUPPORTED
+    # CTA pairs need 256-row weight tiles: N a multiple of 256
+    d384 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 384, 256, 128, 0, 1)
+    t2 = hq.Tuning(cta_group=2)
+    assert L_.hq_gemm_w4a16(ctypes.byref(d384), 16, 16, 4, 32, ctypes.byref(t2), 256, 1 << 20,
+                            None) == hq.HQ_ERR_UNSUPPORTED
     # MXFP4 weights with bf16 activations: no exact-integer variant (INT3 and
     # INT2 weights have one); the block-scaled entry points do not take them
     dx = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 256, 256, 32, 0, 1)
