@@ -63,23 +63,23 @@ def load_peaks():
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
 # capture is taken again.
-TRAFFIC_COMMIT = "ca770ba"
-TRAFFIC_SOURCES = "a8780046785d559f"
+TRAFFIC_COMMIT = "5d5f59e"
+TRAFFIC_SOURCES = "03d4e1894ae72e31"
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 70243840,
-    (4, 7168, 18432): 69139712,
-    (16, 7168, 18432): 69765376,
-    (64, 7168, 18432): 70627328,
-    (256, 7168, 18432): 75611648,
-    (1024, 7168, 18432): 166250496,
-    (4096, 7168, 18432): 452718336,
-    (1, 18432, 7168): 69945856,
-    (4, 18432, 7168): 70013952,
-    (16, 18432, 7168): 70983680,
-    (64, 18432, 7168): 73936640,
-    (256, 18432, 7168): 86089984,
-    (1024, 18432, 7168): 201865728,
-    (4096, 18432, 7168): 724283136,
+    (1, 7168, 18432): 70747648,
+    (4, 7168, 18432): 69487104,
+    (16, 7168, 18432): 69657600,
+    (64, 7168, 18432): 70790400,
+    (256, 7168, 18432): 75858432,
+    (1024, 7168, 18432): 169720320,
+    (4096, 7168, 18432): 484772352,
+    (1, 18432, 7168): 69968896,
+    (4, 18432, 7168): 70297856,
+    (16, 18432, 7168): 71056896,
+    (64, 18432, 7168): 73740032,
+    (256, 18432, 7168): 86312448,
+    (1024, 18432, 7168): 197902848,
+    (4096, 18432, 7168): 715587584,
 }
 
 
