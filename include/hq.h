@@ -39,9 +39,13 @@
  *     are not monotone) are written to the workspace error word and read
  *     back by hq_check_device_status.
  *   - Device pointers must be 16-byte aligned; workspaces 256-byte aligned.
- *   - A workspace must be zero-filled once after allocation; every call
- *     that completes leaves it zero-filled again (apart from the error word,
- *     which hq_check_device_status clears).
+ *   - A workspace must be zero-filled once after allocation.  Every
+ *     workspace starts with the same two parts: a 256-byte header (the
+ *     error word, which hq_check_device_status clears) and a 256 KiB region
+ *     of stream-K tile counters; scratch that needs no initial value
+ *     follows.  Counters must start at zero, and every call that completes
+ *     leaves the ones it used at zero again, so one workspace may serve any
+ *     sequence of calls (of any entry points and plans) ordered on a stream.
  *   - Pointers named *_dev are device pointers; *_host are host pointers.
  *   - The GEMM kernels are launched as programmatic dependents of the
  *     previous kernel on the stream: their CTAs may start, set up and fetch
@@ -120,8 +124,12 @@ typedef struct {
  *              of the kernel's shared-memory ring: one or two 128-K
  *              records, or one or two block-scaled boxes); 0 = the whole
  *              ring; larger than the ring = the whole ring
- *   split_k  : dense W4A16 only: CTAs sharing each tile's K range (stream-K
- *              splits the whole iteration space evenly when 0)
+ *   split_k  : dense GEMMs: CTAs sharing each tile's K range (stream-K
+ *              splits the whole iteration space evenly when 0).  A split
+ *              plan needs a counter per output tile and epilogue warp in
+ *              the workspace's counter region (up to 16384 output tiles
+ *              for W4A16, 8192 for the block-scaled GEMMs); one with more
+ *              tiles runs as whole tiles.
  *   cta_group: block-scaled GEMMs: 0 = the library's choice (CTA pairs
  *              for 128/256-token whole tiles when N is a multiple of
  *              256 and the pairs fill the SMs), 1 = one CTA per 128-row
@@ -431,14 +439,17 @@ hq_status hq_debug_timeout_probe(void* ws_dev, uint64_t limit_ns, hq_stream_t st
  * workspace (split-K tile counters and fp32 partial sums) lives here in one
  * fixed 16 MiB array inside the library, present on every device that loads
  * it until the process exits.
- *   Same arguments and result as hq_gemm_w4a16 (INT4, INT3, INT2 or
- *   MXFP4_A16 weights), without ws_dev / ws_bytes.
+ *   Same arguments and result as hq_gemm_w4a16 (INT4, INT3, INT2, INT8,
+ *   MXFP4_A16 or MXINT4 weights), without ws_dev / ws_bytes.
  *   A launch plan needing more than 16 MiB of scratch is refused with
  *   HQ_ERR_WORKSPACE_TOO_SMALL before anything runs (a smaller tile_m in
  *   `t` needs less); a plan of whole tiles with a split-K tail whose partial
- *   sums would not fit runs as whole tiles instead.  Each call that splits K
- *   clears the array's tile counters on its own stream before the kernel.
- *   All calls share the array: calls that may overlap on the GPU (unordered
+ *   sums would not fit runs as whole tiles instead.  The array is laid out
+ *   as a workspace: its tile counters start at zero and every call that
+ *   completes leaves them at zero; after a call that recorded a device-side
+ *   error, hq_static_check_device_status (which reports it) zeroes them and
+ *   the error word again, so check the status after an error before the
+ *   next call.  All calls share the array: calls that may overlap on the GPU (unordered
  *   streams) race; calls ordered on one stream are safe.  The first call in
  *   each CUDA context looks up the array's device address
  *   (cudaGetSymbolAddress), so make it before any stream capture.
@@ -448,9 +459,11 @@ hq_status hq_debug_timeout_probe(void* ws_dev, uint64_t limit_ns, hq_stream_t st
 hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* packed_w_dev, const void* a_dev, int32_t m,
                                void* c_dev, const hq_tuning* t, hq_stream_t stream);
 
-/* Synchronizes `stream`, then reads, clears and returns the first
- * device-side error recorded by hq_gemm_w4a16_static calls on the current
- * device since the last such read (HQ_OK when none).  Allocates nothing. */
+/* Synchronizes `stream`, then reads and returns the first device-side error
+ * recorded by hq_gemm_w4a16_static calls on the current device since the
+ * last such read (HQ_OK when none).  When there was one it zeroes the
+ * array's error word and tile counters (and synchronizes the device).
+ * Allocates nothing. */
 hq_status hq_static_check_device_status(hq_stream_t stream);
 
 #ifdef __cplusplus

@@ -739,7 +739,8 @@ int bs_tiles(const hq_quant_desc& d, int m, int ntok) {
 
 }  // namespace
 
-BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t) {
+namespace {
+BsConfig bs_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t) {
   BsConfig cfg{};
   // no tuning from the caller: the caller's per-shape table first, then the rules below
   hq_tuning from_table;
@@ -824,18 +825,31 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
   cfg.grid = (int)std::max<long long>(1, std::min<long long>(dev.num_sms, tiles * ks / 4));
   return cfg;
 }
+}  // namespace
 
-// Workspace: header | stream-K counters (8 per tile) and partial tiles (2 per
-// CTA), when K is split | NVFP4 activation scales re-laid for the MMA.
+BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_tuning* t) {
+  BsConfig cfg = bs_plan_rules(dev, d, m, t);
+  // eight tile counters per output tile, in the workspace's fixed counter region
+  if (cfg.splits != 0 && (size_t)bs_tiles(d, m, cfg.ntok) * kBsEpiWarps * sizeof(int32_t) > kWsCounterBytes) {
+    cfg.splits = 0;
+    cfg.cta_group = 1;
+    cfg.grid = (int)std::min<long long>(dev.num_sms, (long long)bs_tiles(d, m, cfg.ntok));
+  }
+  return cfg;
+}
+
+// Workspace: header | the fixed stream-K counter region (8 counters per
+// tile, when K is split) | partial tiles (2 per CTA, when K is split) |
+// NVFP4 activation scales re-laid for the MMA.  Scratch always starts past
+// the counter region, so no call's data lies where another call's counters
+// do.
 struct BsWsLayout {
   size_t counters, partials, sfb, total;
 };
 BsWsLayout bs_ws_layout(const hq_quant_desc& d, int m, const BsConfig& cfg) {
   BsWsLayout L{};
-  size_t off = sizeof(WsHeader);
-  const size_t tiles = (size_t)bs_tiles(d, m, cfg.ntok);
-  L.counters = off;
-  if (cfg.splits != 0) off += ((kBsEpiWarps * tiles * sizeof(int32_t) + 255) / 256) * 256;
+  L.counters = sizeof(WsHeader);
+  size_t off = kWsScratchOff;
   L.partials = off;
   if (cfg.splits != 0) off += (size_t)cfg.grid * 2 * cfg.ntok * kBsTileN * sizeof(float);
   L.sfb = off;
@@ -843,7 +857,7 @@ BsWsLayout bs_ws_layout(const hq_quant_desc& d, int m, const BsConfig& cfg) {
     const size_t halves = cfg.ntok > 128 ? 2 : 1;
     off += (size_t)((m + cfg.ntok - 1) / cfg.ntok) * (d.k / 256) * 4 * halves * 512;
   }
-  L.total = off;
+  L.total = (cfg.splits != 0 || d.fmt == HQ_FMT_NVFP4) ? off : sizeof(WsHeader);
   return L;
 }
 

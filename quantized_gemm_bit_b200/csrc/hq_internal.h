@@ -15,6 +15,16 @@ struct WsHeader {
   uint32_t reserved[63];
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+// Workspace layout of every entry point: the header, a fixed region of
+// stream-K tile counters (used by GEMM plans that split K), then scratch
+// (fp32 partial sums, re-laid activation scales, histograms, block maxima,
+// inverse permutations).  The counters sit at the same offsets whatever the
+// call, and each call that completes sets the ones it used back to zero,
+// while no call keeps data below kWsScratchOff: one workspace serves any
+// sequence of calls in turn, and the scratch needs no initial value.  A
+// split plan whose counters would not fit runs as whole tiles.
+constexpr size_t kWsCounterBytes = 256u << 10;
+constexpr size_t kWsScratchOff = sizeof(WsHeader) + kWsCounterBytes;
 
 constexpr int kTileN = 128;      // weight rows per tile (MMA M)
 constexpr int kBlockK = 128;     // K per packed record / pipeline stage

@@ -301,7 +301,7 @@ __global__ void timeout_probe_kernel(uint32_t* err, uint64_t limit_ns) {
 size_t moe_permute_ws_bytes(int t, int k, int e) {
   (void)k;
   const size_t nb = (size_t)(t + kPermTok - 1) / kPermTok;
-  return sizeof(WsHeader) + ((nb * e * sizeof(int32_t) + 255) / 256) * 256;
+  return kWsScratchOff + ((nb * e * sizeof(int32_t) + 255) / 256) * 256;
 }
 
 hq_status moe_topk_launch(const float* logits, int t, int e, int k, int32_t* ids, float* weights, cudaStream_t s) {
@@ -322,7 +322,7 @@ hq_status moe_swiglu_launch(const void* x, long long rows, int inter, void* h, c
 }
 
 size_t moe_combine_ws_bytes(int t, int k) {
-  return sizeof(WsHeader) + (((size_t)t * k * sizeof(int32_t) + 255) / 256) * 256;
+  return kWsScratchOff + (((size_t)t * k * sizeof(int32_t) + 255) / 256) * 256;
 }
 
 hq_status moe_combine_launch(const void* y_sorted, const int32_t* sorted_src, const float* weights, int t, int k,
@@ -331,7 +331,7 @@ hq_status moe_combine_launch(const void* y_sorted, const int32_t* sorted_src, co
   hq_status st = device_info(&dev);
   if (st != HQ_OK) return st;
   uint32_t* err = static_cast<uint32_t*>(ws);
-  int32_t* inv = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  int32_t* inv = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kWsScratchOff);
   const int rows = t * k;
   // every slot starts unnamed (-1): a sorted list that is not a permutation
   // is reported by the combine instead of read out of bounds
@@ -347,7 +347,7 @@ hq_status moe_combine_launch(const void* y_sorted, const int32_t* sorted_src, co
 hq_status moe_permute_launch(const int32_t* ids, int t, int k, int e, int32_t* sorted_src, int32_t* offsets,
                              const void* a, int hidden, void* a_sorted, void* ws, cudaStream_t s) {
   uint32_t* err = static_cast<uint32_t*>(ws);
-  int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  int32_t* counts = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + kWsScratchOff);
   const int nb = (t + kPermTok - 1) / kPermTok;
   if (nb > 0) {
     perm_count_kernel<<<nb, 256, e * sizeof(int32_t), s>>>(ids, t, k, e, counts, err);

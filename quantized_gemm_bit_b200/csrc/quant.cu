@@ -161,7 +161,7 @@ size_t nvfp4_quant_ws_bytes(int rows, int k) {
   (void)k;
   DeviceInfo dev{};
   int sms = device_info(&dev) == HQ_OK ? dev.num_sms : 148;
-  return sizeof(WsHeader) + (size_t)sms * 4 * sizeof(float);
+  return kWsScratchOff + (size_t)sms * 4 * sizeof(float);
 }
 
 hq_status fp8_rows_launch(const void* x, int rows, int k, void* q, float* scale, cudaStream_t s) {
@@ -174,7 +174,7 @@ hq_status nvfp4_quant_launch(const void* x, int rows, int k, void* codes, void* 
   DeviceInfo dev{};
   device_info(&dev);
   const int grid = dev.num_sms * 4;
-  float* block_max = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + sizeof(WsHeader));
+  float* block_max = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kWsScratchOff);
   const size_t n = (size_t)rows * k;
   amax_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), n / 8, block_max);
   nvfp4_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), n / 16, block_max, grid, static_cast<uint2*>(codes),

@@ -797,7 +797,8 @@ int dense_tiles(const hq_quant_desc& d, int m, int ntok) {
 
 }  // namespace
 
-W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t) {
+namespace {
+W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t) {
   W4Config cfg{};
   // no tuning from the caller: the caller's per-shape table first, then the rules below
   hq_tuning from_table;
@@ -870,6 +871,27 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   const long long tiles = dense_tiles(d, m, ntok);
   if (dp_eff(ntok) >= dp_min) {
     const long long waves = tiles / dev.num_sms, rest = tiles % dev.num_sms;
+    // CTA pairs: 256-token whole tiles of 256-row weight tiles, one pair
+    // tile per resident cluster at a time
+    // (used for 256-token tiles whose single-CTA ring is shallow, below)
+    auto use_pairs = [&](long long tiles_) {
+      const long long pair_tiles = tiles_ / 2;
+      const long long slots = pair_slots(kernel_fmt(d));
+      if (slots <= 0) return false;
+      cfg.cta_group = 2;
+      cfg.splits = 0;
+      cfg.dp_tiles = 0;
+      cfg.grid = (int)(2 * std::min<long long>(slots, pair_tiles));
+      return true;
+    };
+    // CTA pairs (half the activation tile per CTA, a deeper ring) only where
+    // one CTA's ring holds fewer than 3 stages: INT8 records (16.8 KB) leave
+    // room for 2 at 256 tokens, pairs hold 4 (M=4096 K=7168 N=18432
+    // 1175 -> 1075 us, M=1024 308 -> 272 us on B200).  With 3 stages one CTA
+    // per tile wins (INT4 M=4096 815 us against 881 on pairs): each record
+    // waits for both CTAs' dequantization and one SM issues both SMs' MMAs.
+    if (ntok == 256 && d.n % 256 == 0 && w4_ring_depth(d, cfg) < 3 && !(t && t->cta_group == 1) && use_pairs(tiles))
+      return cfg;
     if (waves >= 2 && rest != 0 && dp_eff(ntok) < 0.95) {
       // Whole tiles for all waves but the last full one; that wave and the
       // ragged rest share their K range stream-K style (every CTA one to two
@@ -886,11 +908,6 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
     }
     cfg.splits = 0;  // data parallel
     cfg.grid = (int)std::min<long long>(dev.num_sms, tiles);
-    // (CTA pairs for these tiles run only on request, cta_group 2: measured
-    // slower on B200 than one CTA per tile despite 5 pipeline stages instead
-    // of 3, e.g. M=4096 K=7168 N=18432 815 -> 881 us, M=1024 208 -> 223 us;
-    // each record waits for both CTAs' dequantization and one SM issues
-    // both SMs' MMAs)
     return cfg;
   }
   if (ntok >= 128 && tiles * 2 <= dev.num_sms && tiles * (dev.num_sms / tiles) >= 0.85 * dev.num_sms) {
@@ -900,6 +917,15 @@ W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grou
   }
   cfg.splits = 1;
   cfg.grid = (int)std::max<long long>(1, std::min<long long>(dev.num_sms, tiles * kbs / 4));
+  return cfg;
+}
+}  // namespace
+
+W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t) {
+  W4Config cfg = w4_plan_rules(dev, d, m, grouped, t);
+  // four tile counters per output tile, in the workspace's fixed counter region
+  if (!grouped && cfg.splits != 0 && (size_t)dense_tiles(d, m, cfg.ntok) * 4 * sizeof(int32_t) > kWsCounterBytes)
+    cfg = w4_whole_tiles(dev, d, m, cfg);
   return cfg;
 }
 
@@ -943,8 +969,7 @@ size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bo
   size_t bytes = sizeof(WsHeader);
   if (grouped) return bytes;
   if (cfg.splits == 0) return bytes;  // data parallel: no partial sums
-  const size_t tiles = (size_t)dense_tiles(d, m, cfg.ntok);
-  bytes += ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256;                   // counters, 4 per tile
+  bytes += kWsCounterBytes;                                                     // counters, 4 per tile (fixed region)
   bytes += (size_t)cfg.grid * 2 * cfg.ntok * kTileN * sizeof(float);            // partial tiles, 2 per CTA
   return bytes;
 }
@@ -993,7 +1018,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
     p.data_parallel = cfg.splits == 0 ? 1 : 0;
     uint8_t* base = static_cast<uint8_t*>(ws) + sizeof(WsHeader);
     p.counters = reinterpret_cast<int32_t*>(base);
-    p.partials = reinterpret_cast<float*>(base + ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256);
+    p.partials = reinterpret_cast<float*>(base + kWsCounterBytes);
   }
 
   // Activations: bf16 [rows][K], boxes of 64 K x NTOK rows, 128-byte swizzle.

@@ -18,11 +18,13 @@
 //   * every call uses the same array, so calls that overlap on the GPU
 //     (different streams, no ordering) race on it; calls ordered on one
 //     stream do not;
-//   * each call whose plan splits K clears the tile counters (which must
-//     start at zero) on its stream before the kernel;
+//   * it is laid out as a workspace (error word, the fixed tile-counter
+//     region, then partial sums); the tile counters start at zero, as the
+//     array does, and every call that completes leaves them at zero again;
 //   * its first word records the first device-side error of any call
 //     (a bounded wait that ran out) until hq_static_check_device_status
-//     reads and clears it.
+//     reads it; that call then zeroes the error word and the counters,
+//     which a call that gave up may have left behind.
 // Host code cannot use the array's name as a device address: the first call
 // in each CUDA context looks the address up with cudaGetSymbolAddress (with
 // that context current) and caches it per context, so the first call in a
@@ -128,14 +130,11 @@ extern "C" hq_status hq_gemm_w4a16_static(const hq_quant_desc* d, const void* pa
   void* scratch = static_scratch_address();
   if (!scratch) return HQ_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the tile counters start at zero (the partial sums need not, and the
-  // error word keeps the first error until it is read)
-  if (cfg.splits != 0) {
-    const size_t tiles = (size_t)((d->n + kTileN - 1) / kTileN) * (size_t)((m + cfg.ntok - 1) / cfg.ntok);
-    const size_t counter_bytes = ((4 * tiles * sizeof(int32_t) + 255) / 256) * 256;
-    if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + sizeof(WsHeader), 0, counter_bytes, s) != cudaSuccess)
-      return HQ_ERR_CUDA;
-  }
+  // The tile counters are zero here, as in a workspace: the array starts
+  // zero-filled, every call that completes leaves them at zero, and
+  // hq_static_check_device_status clears them after a call that did not
+  // (nothing runs between the previous kernel on the stream and this one,
+  // so the launch overlap of consecutive calls holds)
   return w4_launch(*d, cfg, packed_w_dev, a_dev, m, c_dev, nullptr, scratch, s);
 }
 
@@ -149,8 +148,10 @@ extern "C" hq_status hq_static_check_device_status(hq_stream_t stream) {
   uint32_t err = 0;
   if (cudaMemcpy(&err, scratch, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess) return HQ_ERR_CUDA;
   if (err != 0) {
-    const uint32_t zero = 0;
-    if (cudaMemcpy(scratch, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return HQ_ERR_CUDA;
+    // a call that ran out of a bounded wait may have left tile counters
+    // behind: zero them and the error word for the next call
+    if (cudaMemset(scratch, 0, kWsScratchOff) != cudaSuccess) return HQ_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return HQ_ERR_CUDA;
   }
   return static_cast<hq_status>(err);
 }

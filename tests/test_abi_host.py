@@ -432,6 +432,30 @@ def test_mxint4_pack_rejects_scales_that_overflow_bf16_and_descriptor_rules():
                             None) == hq.HQ_ERR_UNSUPPORTED
 
 
+def test_split_plans_fit_the_workspace_counter_region():
+    """Stream-K tile counters live in a fixed 256 KiB region after the
+    256-byte header (4 per tile for W4A16, 8 for the block-scaled GEMMs):
+    a split request on more tiles than that holds runs as whole tiles, and
+    every scratch area starts past the region."""
+    header, region = 256, 256 << 10
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
+    t = hq.Tuning(tile_m=16, split_k=2)
+    p = hq.hq_plan_describe(d, 16, t)
+    assert p.split == 2 and p.workspace_bytes == header + region + p.grid * 2 * 16 * 128 * 4
+    assert hq.hq_plan_describe(d, 16 * 113, t).split == 2          # 16272 tiles
+    big = hq.hq_plan_describe(d, 16 * 114, t)                      # 16416 tiles
+    assert (big.split, big.workspace_bytes) == (0, header)
+    dm = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 18432, 7168, 32, 0, 1)
+    assert hq.hq_plan_describe(dm, 16 * 56, t).split == 2          # 8064 tiles
+    assert hq.hq_plan_describe(dm, 16 * 57, t).split == 0          # 8208 tiles
+    dn = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, 8192, 8192, 16, 0, 1)
+    pn = hq.hq_plan_describe(dn, 8192)
+    assert pn.split == 0 and pn.workspace_bytes > header + region  # re-laid scales past the region
+    assert hq.hq_moe_combine_workspace_size(10, 8) >= header + region + 4 * 10 * 8
+    assert hq.hq_moe_permute_workspace_size(64, 8, 256) > header + region
+    assert hq.hq_quantize_nvfp4_workspace_size(64, 1024) > header + region
+
+
 def test_tuning_table_entry_changes_the_plan():
     """A table entry replaces the library's rules for calls without a tuning
     of its shape and m range; an explicit tuning still wins; clearing the

@@ -223,3 +223,38 @@ def test_large_tiles_default_to_cta_pairs():
     plan = hq.hq_plan_describe(d, 8192)
     assert (plan.tile_m, plan.split, plan.cta_group, plan.grid % 2) == (256, 0, 2, 0)
     assert hq.hq_plan_describe(d, 8192, hq.Tuning(cta_group=1)).cta_group == 1
+
+
+def test_workspace_shared_across_entry_points_and_plans():
+    """One workspace serves, in turn, NVFP4 calls (whose re-laid activation
+    scales stay behind as scratch, split or not) and MXFP4 split-K calls of
+    different plans: the tile counters sit in the fixed region after the
+    256-byte header, which every completed call leaves at zero, and no
+    call keeps data there."""
+    n, k = 512, 2048
+    codes, e8 = synth.mxfp4_weights(n, k, seed=740)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, n, k, 32, 0, 1)
+    blob = torch.from_numpy(hq.hq_pack_weights(d, codes, e8)).to(DEV)
+    dn, nblob, nact, nw = nv_case(300, 256, 1536, 745)
+    ws = workspace(1 << 24)
+    counter_region = ws[:256 + (256 << 10)]
+    for step, (m, t) in enumerate([(None, None), (16, hq.Tuning(tile_m=16, split_k=3)),
+                                   (None, hq.Tuning(tile_m=16, split_k=3)), (200, hq.Tuning(tile_m=16, split_k=3)),
+                                   (16, hq.Tuning(tile_m=64, split_k=2))]):
+        if m is None:
+            ap, asf, ag = nact
+            c = torch.empty(300, dn.n, dtype=torch.bfloat16, device=DEV)
+            assert hq.hq_workspace_size(dn, 300, t) <= ws.numel()
+            hq.hq_gemm_nvfp4(dn, nblob, torch.from_numpy(ap).to(DEV), torch.from_numpy(asf).to(DEV), float(ag), 300,
+                             c, ws, t)
+            assert hq.hq_check_device_status(ws) == hq.HQ_OK
+            check_gemm(c, G.nvfp4_ref(*nact, *nw), 1536, f"nvfp4 shared workspace step {step}")
+        else:
+            aq, asc = F.fp8_per_token_quantize(synth.bf16_normal(m, k, 741 + m).float().numpy())
+            c = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
+            assert hq.hq_workspace_size(d, m, t) <= ws.numel()
+            hq.hq_gemm_mxfp4_a8(d, blob, torch.from_numpy(aq).to(DEV), torch.from_numpy(asc).to(DEV), m, c, ws, t)
+            assert hq.hq_check_device_status(ws) == hq.HQ_OK
+            check_gemm(c, G.mxfp4_a8_ref(aq, asc, codes.numpy(), e8.numpy()), k, f"mxfp4 shared workspace step {step}")
+        assert torch.count_nonzero(counter_region) == 0
+    assert torch.count_nonzero(ws) > 0      # scratch stays behind, past the counters

@@ -189,3 +189,23 @@ def test_m_sweep_full_size_sampled_rows(m, k, n):
     rows = tile_rows(m, 128, np.random.default_rng(m))
     ref = F.bf16_bits_to_f64(_bits(a)[rows]) @ w.T
     check_gemm(c[torch.from_numpy(rows).to(DEV)], ref, k, f"sweep m={m} k={k} n={n}")
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+def test_workspace_reused_across_split_plans(variant):
+    """One workspace serves split-K calls of different plans in turn (few
+    tiles, then many, then few again): the tile counters sit in a fixed
+    region after the 256-byte header, every call that completes leaves them
+    at zero, and the partial sums lie past that region."""
+    n, k = 1024, 2048
+    d, blob, _, (q, s, z) = make_case(8, n, k, True, 1500)
+    ws = workspace(1 << 22)
+    for m in (16, 100, 16, 100):
+        t = hq.Tuning(tile_m=16, split_k=3, variant=variant)
+        assert hq.hq_workspace_size(d, m, t) <= ws.numel()
+        a = synth.bf16_normal(m, k, 1501 + m)
+        c = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
+        hq.hq_gemm_w4a16(d, blob, a.to(DEV), m, c, ws, t)
+        assert hq.hq_check_device_status(ws) == hq.HQ_OK
+        check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, f"reused workspace m={m} variant={variant}")
+        assert torch.count_nonzero(ws[:256 + (256 << 10)]) == 0

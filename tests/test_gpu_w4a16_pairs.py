@@ -116,3 +116,18 @@ def test_pairs_refused_where_they_do_not_apply():
     for bad in (hq.Tuning(cta_group=2, tile_m=128), hq.Tuning(cta_group=2, split_k=2)):
         with pytest.raises(hq.HQError):
             hq.hq_gemm_w4a16(d2, blob2, a, 256, c2, ws, bad)
+
+
+def test_int8_large_tiles_default_to_pairs():
+    """INT8 records leave room for only two 256-token stages on one CTA; the
+    library runs such whole tiles on CTA pairs (four stages), and the result
+    is the oracle's."""
+    m, n, k = 1024, 4608, 1024            # 18 x 4 256-row x 256-token tiles: whole tiles
+    d, blob, ref = case("int8", n, k, True, 930)
+    plan = hq.hq_plan_describe(d, m)
+    assert (plan.cta_group, plan.tile_m, plan.split) == (2, 256, 0)
+    assert plan.ring_stages > hq.hq_plan_describe(d, m, hq.Tuning(cta_group=1)).ring_stages
+    a = synth.bf16_normal(m, k, 931)
+    c = run(d, blob, a, m)
+    rows = tile_rows(m, 256, np.random.default_rng(9))
+    check_gemm(c[torch.from_numpy(rows).to(DEV)], ref(_bits(a), rows=rows), k, "w4a16 int8 default pairs")
