@@ -207,29 +207,34 @@ __device__ __forceinline__ bool bs_unit(const BsParams& p, int idx, int& tile, i
   return true;
 }
 
-// Stream-K fixup of one epilogue warp's rows x tokens after its partial slot
-// is written: one counter per (tile, epilogue warp); the last contributing
-// CTA reduces every partial in CTA order (8 tokens at a time, the loads of
-// up to CB contributors in flight together) and writes the scaled output.
+// Stream-K partial sums, as in the W4A16 kernels: one counter per (tile,
+// epilogue warp).  Every contributor of a split tile writes its partial
+// slot; all but the last signal and go on; the last (the owner of the
+// tile's final k-stages, the first unit of its range) reduces the tile
+// after its own last unit, once the others -- all of lower CTA index --
+// have signalled: every partial in CTA order (8 tokens at a time, the
+// loads of up to CB contributors in flight together), then the scaled
+// output.
+__device__ __noinline__ void bs_signal(const BsParams& p, int tile, int wslot, int lane) {
+  __threadfence();  // this lane's partial stores, visible before the signal
+  __syncwarp();
+  if (lane == 0) atomicAdd(p.counters + tile * kBsEpiWarps + wslot, 1);
+}
+
 template <int FMT, int NTOK, int CB>
-__device__ __forceinline__ void bs_fixup(const BsParams& p, int tile, int nt, int row0, int rows, int tok0, int wslot,
-                                      int r, int lane, float alpha) {
+__device__ __noinline__ void bs_reduce(const BsParams& p, int tile, int nt, int row0, int rows, int tok0, int wslot,
+                                       int r, int lane, float alpha) {
   constexpr int NC = BsCfg<FMT, NTOK>::kCols;
   const int rows_w = rows - tok0;
   const long long T = p.total_iters, G = gridDim.x, kst = p.k_stages;
   const long long t0 = (long long)tile * kst;
   const long long first = sk_owner(t0, T, G), last = sk_owner(t0 + kst - 1, T, G);
-  const int cnt = (int)(last - first + 1);
-  __threadfence();
-  __syncwarp();
-  int is_last = 0;
+  int* ctr = p.counters + tile * kBsEpiWarps + wslot;
   if (lane == 0) {
-    __threadfence();
-    is_last = (atomicAdd(p.counters + tile * kBsEpiWarps + wslot, 1) == cnt - 1);
-    __threadfence();
+    if (!hq_wait_count(ctr, (int)(last - first), p.wait_ns)) atomicCAS(p.err, 0u, (uint32_t)HQ_ERR_DEVICE_TIMEOUT);
+    *ctr = 0;  // every other contributor has signalled: leave the counter at zero
   }
-  is_last = __shfl_sync(0xffffffffu, is_last, 0);
-  if (!is_last) return;
+  __syncwarp();
   __threadfence();
   const int n = nt * kBsTileN + r;
   for (int j0 = 0; j0 < NC && j0 < rows_w; j0 += 8) {
@@ -267,7 +272,6 @@ __device__ __forceinline__ void bs_fixup(const BsParams& p, int tile, int nt, in
       }
     }
   }
-  if (lane == 0) p.counters[tile * kBsEpiWarps + wslot] = 0;
 }
 
 template <int FMT, int NTOK, int CG>
@@ -599,11 +603,14 @@ __global__ void __launch_bounds__(kBsThreads, 1)
     uint16_t* scr = scratch + (warp - 4) * (32 * kBsEB);
     const float alpha = FMT == kNV ? p.a_global * __ldg(p.g_w) : 1.f;
     uint32_t uc = 0;
+    bool ok = true;
+    int pend_tile = -1, pend_nt = 0, pend_row0 = 0, pend_rows = 0;   // the split tile this CTA reduces last
     for (int idx = 0; bs_unit<FMT, NTOK, CG>(p, idx, tile, nt, row0, rows, ks0, ks1, partial, slot); ++idx, ++uc) {
       const int ab = uc % ACC;
       const uint32_t aph = (uc / ACC) & 1;
       if (!hq_wait(&acc_full[ab], aph, p.wait_ns, s_abort)) {
         raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
         break;
       }
       tc_fence_after();
@@ -646,11 +653,22 @@ __global__ void __launch_bounds__(kBsThreads, 1)
         store_rows_chunk<EB>(p.c, p.n, row0 + tok0, rows_w, nt * kBsTileN + (int)q * 32, r, part, (int)lane, j0, f,
                              scr);
       }
-      // the 256-token tile keeps 128 accumulator registers per thread: fewer
-      // contributors in flight there
-      if (CG == 1 && partial)
-        bs_fixup<FMT, NTOK, (NTOK > 128 ? 1 : 4)>(p, tile, nt, row0, rows, tok0, wslot, r, (int)lane, alpha);
+      if (CG == 1 && partial) {
+        if (ks1 == p.k_stages) {
+          pend_tile = tile;
+          pend_nt = nt;
+          pend_row0 = row0;
+          pend_rows = rows;
+        } else {
+          bs_signal(p, tile, wslot, (int)lane);
+        }
+      }
     }
+    // (the 256-token tile keeps 128 accumulator registers per thread: fewer
+    // contributors in flight there)
+    if (CG == 1 && ok && pend_tile >= 0)
+      bs_reduce<FMT, NTOK, (NTOK > 128 ? 1 : 4)>(p, pend_tile, pend_nt, pend_row0, pend_rows, hc * NC, wslot, r,
+                                                 (int)lane, alpha);
   }
 
   }  // non-producer roles

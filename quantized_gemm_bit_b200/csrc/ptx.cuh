@@ -1,7 +1,8 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers with bounded waits, bulk
 // and tensor (TMA) copies, tcgen05 (TMEM alloc / MMA / ld / st / commit).
-// Every wait in this library goes through hq_wait(), which gives up after a
-// wall-clock limit and reports a timeout instead of spinning forever.
+// Every wait in this library (on an mbarrier through hq_wait(), on a global
+// counter through hq_wait_count()) gives up after a wall-clock limit and
+// reports a timeout instead of spinning forever.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -75,6 +76,22 @@ __device__ __forceinline__ bool hq_wait(uint64_t* bar, uint32_t parity, uint64_t
       if (abort != nullptr && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+  }
+}
+
+// Bounded wait of one thread until a global counter, written by other CTAs
+// with release semantics (a fence before their atomic), reaches `target`.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool hq_wait_count(const int* ctr, int target, uint64_t limit_ns) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 

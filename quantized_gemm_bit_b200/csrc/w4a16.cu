@@ -604,7 +604,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool does_dq = dq < NDQ;
     uint32_t it = 0, uc = 0;
     bool ok = true;
-    Unit x;
+    Unit x, pend;          // pend: the split tile this CTA reduces after its last unit
+    bool has_pend = false;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx, ++uc) {
       for (int kb = x.kb0; kb < x.kb1; kb += KPS, ++it) {
         if (!does_dq || (int)(it % NDQ) != dq) continue;
@@ -684,8 +685,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(&acc_empty[ab]);
       }
-      if (x.partial) sk_fixup<NTOK>(p, x, (int)q, (int)lane);
+      if (sk_is_reducer(p, x)) {
+        pend = x;
+        has_pend = true;
+      } else if (x.partial) {
+        sk_signal(p, x, (int)q, (int)lane);
+      }
     }
+    if (ok && has_pend) sk_reduce<NTOK>(p, pend, (int)q, (int)lane);
   }
 
   }  // non-producer roles

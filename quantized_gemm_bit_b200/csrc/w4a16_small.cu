@@ -89,7 +89,13 @@ struct SmallCfg {
   static constexpr int kFullPeriod = kSmemStages / cgcd(kSmemStages, kNdq) * kNdq;  // lcm
   // Warp 1 issues every MMA.  (Letting the last unpacking warp to finish a
   // stage issue that stage's MMAs measured slower on B200: single-lane issue
-  // from a busy warp.)
+  // from a busy warp; so did one issuing warp per unpacking group, whose
+  // unpacking then ran slower.  A clock trace of one CTA at M=16 shows each
+  // stage costs the issuer ~1260 SM cycles: ~450 for one probe of its three
+  // (already complete) mbarriers, ~480 to issue the 16 MMAs, the rest its
+  // loop.  Several issuers would also need a result ring of at least as
+  // many stages as groups, or a parity wait could mistake a phase two
+  // behind for the one it waits for.)
   // byte offsets from the 1024-aligned base of dynamic shared memory
   static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
   static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
@@ -424,7 +430,8 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
     constexpr int CH = NTOK >= 64 ? 32 : 16;          // TMEM columns per load batch
     uint32_t it = 0;
     bool ok = true;
-    Unit x;
+    Unit x, pend;          // pend: the split tile this CTA reduces after its last unit
+    bool has_pend = false;
     for (int idx = 0; ok && get_unit<NTOK>(p, s_prefix, s_off, total_grouped, idx, x); ++idx) {
       float acc[NTOK];
 #pragma unroll
@@ -483,8 +490,14 @@ __global__ void __launch_bounds__(SmallCfg<NTOK, FMT>::kThreads, 1)
         for (int j = 0; j < CH; ++j) v[j] = acc[j0 + j];
         store_chunk<CH, SW>(p, x, part, (int)q, (int)lane, j0, v, scr);
       }
-      if (x.partial) sk_fixup<NTOK, (C::kThreads > 512 ? 2 : 4)>(p, x, (int)q, (int)lane);
+      if (sk_is_reducer(p, x)) {
+        pend = x;
+        has_pend = true;
+      } else if (x.partial) {
+        sk_signal(p, x, (int)q, (int)lane);
+      }
     }
+    if (ok && has_pend) sk_reduce<NTOK, (C::kThreads > 512 ? 2 : 4)>(p, pend, (int)q, (int)lane);
   }
 
   }  // non-producer roles
