@@ -47,10 +47,13 @@ constexpr int kBsEB = 16;          // tokens per transposed output store
 
 enum BsFmt { kMX = 0, kNV = 1 };
 
-// MXFP4 stages of small token tiles carry two 128-K boxes (fewer, longer
-// stages: the per-stage handshakes dominate there); everything else one.
+// MXFP4 stages of small token tiles carry several 128-K boxes (fewer,
+// longer stages: the per-stage handshakes dominate there): three at 32
+// tokens (measured on B200, M=64 K=N=7168 on 32-token tiles: 15.2 -> 14.1
+// us against two), two at 16 and 64 (three gains nothing at 16); everything
+// else one.
 template <int FMT, int NTOK>
-constexpr int bs_boxes() { return FMT == kMX && NTOK <= 64 ? 2 : 1; }
+constexpr int bs_boxes() { return FMT == kMX && NTOK == 32 ? 3 : FMT == kMX && NTOK <= 64 ? 2 : 1; }
 
 // CG = 2: a CTA pair (cluster of two) runs one 256-row weight tile with
 // cta_group::2 MMAs; each CTA stages its own 128 weight rows and half of the
@@ -747,7 +750,7 @@ int bs_pair_slots(bool nv, int ntok) {
 // 128-B-row boxes along K, and pipeline stages (bs_boxes boxes each).
 long long bs_k_boxes(const hq_quant_desc& d) { return d.k / (d.fmt == HQ_FMT_NVFP4 ? 256 : 128); }
 long long bs_k_stages(const hq_quant_desc& d, int ntok) {
-  const int box = d.fmt == HQ_FMT_MXFP4 && ntok <= 64 ? 2 : 1;   // bs_boxes<FMT, NTOK>()
+  const int box = d.fmt != HQ_FMT_MXFP4 ? 1 : ntok == 32 ? 3 : ntok <= 64 ? 2 : 1;   // bs_boxes<FMT, NTOK>()
   return (bs_k_boxes(d) + box - 1) / box;
 }
 
