@@ -86,7 +86,8 @@ struct Cfg {
   static constexpr int kFullPeriod = kSmemStages / cgcd(kSmemStages, kDqGroups) * kDqGroups;  // lcm
   // (kEpiScratch: the warp-local transpose buffer for 16-byte output
   // stores; at 256 tokens it aliases the expert tables, so grouped 256-token
-  // tiles store their outputs element by element instead)
+  // tiles use 1 KB per warp after the tables, 16 tokens at a time, when the
+  // tables take at most half of their area)
   // byte offsets from the 1024-aligned base of dynamic shared memory
   static constexpr size_t kBarOff = (size_t)kSmemStages * (kATile + kRecs);
   static constexpr size_t kTabOff = kBarOff + kBarBytes;                          // s_prefix, s_off
@@ -365,10 +366,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort + 1);
-  int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);  // [kMaxExperts + 1]
-  int* s_off = s_prefix + (kMaxExperts + 1);                    // [kMaxExperts + 1]
+  // expert tables packed at the start of their area: [E + 1] each
+  int* s_prefix = reinterpret_cast<int*>(smem + C::kTabOff);
+  int* s_off = s_prefix + (p.grouped ? p.num_experts + 1 : kMaxExperts + 1);
   // 16-byte aligned: read back with 16-byte loads
   uint16_t* epi_scratch = reinterpret_cast<uint16_t*>(smem + (C::kEpiScratch ? C::kScrOff : C::kTabOff));
+  // 256-token grouped tiles: 16-token transposes in the second half of the
+  // table area, free when the tables take at most 4 KB (<= 511 experts)
+  uint16_t* grouped_scratch =
+      (C::kEpiScratch == 0 && p.grouped && 2 * (p.num_experts + 1) * (int)sizeof(int) <= 4096)
+          ? reinterpret_cast<uint16_t*>(smem + C::kTabOff + 4096)
+          : nullptr;
   auto full_bar = [&](uint32_t i) { return &full[(i % SS) * NDQ + (i % NDQ)]; };
   auto full_par = [](uint32_t i) { return (i / C::kFullPeriod) & 1; };
 
@@ -665,17 +673,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* part = x.partial ? p.partials + ((size_t)blockIdx.x * 2 + x.slot) * NTOK * kTileN : nullptr;
       // batched TMEM loads (EB columns), then fp32 partials or bf16 stores
       constexpr int EB = NTOK >= 32 ? 32 : 16;
-      uint16_t* sc = (C::kEpiScratch == 0 && p.grouped) ? nullptr : epi_scratch + q * 1024;
+      if (C::kEpiScratch == 0 && p.grouped) {
+        // 256-token grouped tiles: 16 tokens per batch through the 1 KB
+        // transposes after the expert tables (element by element when the
+        // tables leave no room)
+        uint16_t* sc = grouped_scratch ? grouped_scratch + q * 512 : nullptr;
 #pragma unroll 1
-      for (int j0 = 0; j0 < NTOK; j0 += EB) {
-        uint32_t v0[16], v1[16];
-        tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0, v0);
-        if (EB == 32) tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0 + 16, v1);
-        tmem_wait_ld();
-        float v[EB];
+        for (int j0 = 0; j0 < NTOK; j0 += 16) {
+          uint32_t v0[16];
+          tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0, v0);
+          tmem_wait_ld();
+          float v[16];
 #pragma unroll
-        for (int j = 0; j < EB; ++j) v[j] = __uint_as_float(j < 16 ? v0[j] : v1[j - 16]);
-        store_chunk<EB, SW>(p, x, part, (int)q, (int)lane, j0, v, sc);
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(v0[j]);
+          store_chunk<16, SW>(p, x, part, (int)q, (int)lane, j0, v, sc);
+        }
+      } else {
+        uint16_t* sc = epi_scratch + q * 1024;
+#pragma unroll 1
+        for (int j0 = 0; j0 < NTOK; j0 += EB) {
+          uint32_t v0[16], v1[16];
+          tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0, v0);
+          if (EB == 32) tmem_ld_x16(tmem_base + lane_addr + acc_col(ab) + j0 + 16, v1);
+          tmem_wait_ld();
+          float v[EB];
+#pragma unroll
+          for (int j = 0; j < EB; ++j) v[j] = __uint_as_float(j < 16 ? v0[j] : v1[j - 16]);
+          store_chunk<EB, SW>(p, x, part, (int)q, (int)lane, j0, v, sc);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -819,9 +844,14 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
       // Poisson(avg) rows per expert, so the tile covers avg + 2 sd.
       const double avg = (double)m / std::max(1, d.num_experts);
       const double want = avg + 2.0 * std::sqrt(avg);
-      // (256-token tiles, on request only: measured slower for every T tried,
-      // e.g. T=8192 top-8 over 256 experts, down: 2.3 ms at 128, 2.9 at 256)
-      ntok = want <= 16 ? 16 : want <= 32 ? 32 : want <= 64 ? 64 : 128;
+      // 256-token tiles for long K ranges only, and only where their output
+      // transposes fit beside the expert tables (at most 511 experts).
+      // Measured on B200, T=8192 top-8 over 256 experts: gate+up (K=7168)
+      // with the fused SwiGLU 4571 us at 128 tokens, 4157 at 256; down
+      // (K=2048, 16 k-blocks per unit, whose single 256-token accumulator
+      // leaves the epilogue unoverlapped) 2337 at 128, 2399 at 256.
+      ntok = want <= 16 ? 16 : want <= 32 ? 32 : want <= 64 ? 64
+           : (want > 192 && d.k >= 4096 && d.num_experts <= 511) ? 256 : 128;
     } else {
       ntok = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
     }
