@@ -63,23 +63,23 @@ def load_peaks():
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
 # capture is taken again.
-TRAFFIC_COMMIT = "5d5f59e"
-TRAFFIC_SOURCES = "03d4e1894ae72e31"
+TRAFFIC_COMMIT = "fb566ad"
+TRAFFIC_SOURCES = "dde022aa6bbfebf3"
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 70747648,
-    (4, 7168, 18432): 69487104,
-    (16, 7168, 18432): 69657600,
-    (64, 7168, 18432): 70790400,
-    (256, 7168, 18432): 75858432,
-    (1024, 7168, 18432): 169720320,
-    (4096, 7168, 18432): 484772352,
-    (1, 18432, 7168): 69968896,
-    (4, 18432, 7168): 70297856,
-    (16, 18432, 7168): 71056896,
-    (64, 18432, 7168): 73740032,
-    (256, 18432, 7168): 86312448,
-    (1024, 18432, 7168): 197902848,
-    (4096, 18432, 7168): 715587584,
+    (1, 7168, 18432): 70462720,
+    (4, 7168, 18432): 69294592,
+    (16, 7168, 18432): 69672704,
+    (64, 7168, 18432): 71269120,
+    (256, 7168, 18432): 75859968,
+    (1024, 7168, 18432): 150655488,
+    (4096, 7168, 18432): 343374080,
+    (1, 18432, 7168): 69810432,
+    (4, 18432, 7168): 70138624,
+    (16, 18432, 7168): 70899200,
+    (64, 18432, 7168): 74140928,
+    (256, 18432, 7168): 86837248,
+    (1024, 18432, 7168): 197917440,
+    (4096, 18432, 7168): 711796992,
 }
 
 
