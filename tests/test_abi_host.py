@@ -456,6 +456,22 @@ def test_split_plans_fit_the_workspace_counter_region():
     assert hq.hq_quantize_nvfp4_workspace_size(64, 1024) > header + region
 
 
+def test_grouped_token_tile_rule():
+    """Grouped GEMMs: the token tile covers a typical expert's rows (avg +
+    2 sd of Poisson(avg) rows per expert); above 128 it is 256 only for K of
+    at least 4096 and at most 511 experts (the 256-token tile's output
+    transposes sit beside the expert tables), else 128."""
+    def tile(n, k, e, rows):
+        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, e)
+        return hq.hq_plan_describe(d, rows).tile_m
+    assert tile(4096, 7168, 256, 64 * 8) == 16          # T=64, top-8 of 256: 2 rows per expert
+    assert tile(4096, 7168, 256, 1024 * 8) == 64        # 32 rows per expert
+    assert tile(4096, 7168, 256, 8192 * 8) == 256       # 256 rows per expert, long K
+    assert tile(7168, 2048, 256, 8192 * 8) == 128       # short K
+    assert tile(4096, 7168, 600, 600 * 256) == 128      # tables too large for the transposes
+    assert tile(4096, 7168, 256, 256 * 150) == 128      # 150 + 2 sd <= 192
+
+
 def test_tuning_table_entry_changes_the_plan():
     """A table entry replaces the library's rules for calls without a tuning
     of its shape and m range; an explicit tuning still wins; clearing the
