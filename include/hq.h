@@ -254,19 +254,22 @@ size_t hq_packed_size(const hq_quant_desc* d);
 hq_status hq_pack_weights(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
                           const void* zeros_host, float global_scale, void* out_host, size_t out_bytes);
 
-/* Workspace bytes that hq_gemm_w4a16 (fmt INT4, INT3, INT2 or MXFP4_A16, num_experts 1),
+/* Workspace bytes that hq_gemm_w4a16 (a W4A16-family fmt: INT4, INT3, INT2, INT8,
+ * MXFP4_A16 or MXINT4; num_experts 1),
  * hq_gemm_mxfp4_a8, hq_gemm_nvfp4 or hq_grouped_gemm_moe need for M rows
  * (total sorted rows for MoE) and the given tuning (NULL = heuristic). */
 size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
 
 /* Dense W4A16 GEMM ([fr] table row "W4A16 dense"): C = A * W_hat^T with
  * W_hat[n,k] = (q[n,k] - z[n,k/128]) * s[n,k/128] dequantized in-kernel.
- *   d            : INT4, INT3, INT2 or MXFP4_A16 descriptor, num_experts == 1.
+ *   d            : INT4, INT3, INT2, INT8, MXFP4_A16 or MXINT4 descriptor,
+ *                  num_experts == 1.
  *                  INT3 (GPTQ INT3 weights, [vi] "meaning for domestic
  *                  deployers"): W_hat = (q - z) * s with 3-bit codes and
  *                  the symmetric zero point 4, computed as for INT4.  INT2
  *                  ([fr] format list INT1..INT8) likewise, with 2-bit codes
- *                  and the symmetric zero point 2.
+ *                  and the symmetric zero point 2; INT8 likewise, with
+ *                  8-bit codes and the symmetric zero point 128.
  *                  MXFP4_A16 (MXFP4 weights with bf16 activations; [fa]
  *                  paragraph 2 lists MXFP4 weights and bf16 activations):
  *                  W_hat[n,k] = e2m1(c[n,k]) * 2^(e[n,k/32] - 127), each
@@ -274,6 +277,9 @@ size_t hq_workspace_size(const hq_quant_desc* d, int32_t m, const hq_tuning* t);
  *                  keeps it finite) and accumulated in fp32; tuning variant
  *                  2 is refused with HQ_ERR_UNSUPPORTED (one scale per 32 K
  *                  leaves nothing to factor out of a 128-K group).
+ *                  MXINT4 (MXINT8's element rule at 4 bits): W_hat[n,k] =
+ *                  c[n,k] * 2^(e[n,k/32] - 127) with c a two's-complement
+ *                  4-bit integer, as for MXFP4_A16 (variant 2 refused too).
  *   packed_w_dev : blob from hq_pack_weights (hq_packed_size bytes)
  *   a_dev        : bf16 [m][d->k]
  *   m            : rows of A (m == 0 returns HQ_OK without launching)
@@ -355,9 +361,9 @@ hq_status hq_moe_permute(const int32_t* topk_ids_dev, int32_t t, int32_t k, int3
  * "MoE W4A16"): for every expert e, rows [off[e], off[e+1]) of A_sorted
  * times W_hat_e^T.  The tile scheduler reads expert_offsets on the device
  * (no host synchronization).
- *   d              : INT4, INT3, INT2 or MXFP4_A16 descriptor, num_experts =
- *                    e (per-expert n, k); INT3, INT2 and MXFP4_A16 weights as for
- *                    hq_gemm_w4a16
+ *   d              : INT4, INT3, INT2, INT8, MXFP4_A16 or MXINT4 descriptor,
+ *                    num_experts = e (per-expert n, k); the other formats'
+ *                    weights as for hq_gemm_w4a16
  *   packed_w_dev   : blob of all experts from hq_pack_weights
  *   a_sorted_dev   : bf16 [total_rows][k]
  *   expert_offsets_dev : int32 [e+1], monotone, offsets[e] == total_rows
@@ -373,7 +379,8 @@ hq_status hq_grouped_gemm_moe(const hq_quant_desc* d, const void* packed_w_dev, 
  * 0-15 are the gate rows 64j + 16q + l and rows 16-31 the up rows
  * I + 64j + 16q + l (l < 16), so that one tile's accumulators hold matching
  * gate and up values.  Same blob size as hq_pack_weights.
- *   d : INT4, INT3, INT2 or MXFP4_A16 descriptor with d->n % 128 == 0.
+ *   d : INT4, INT3, INT2, INT8, MXFP4_A16 or MXINT4 descriptor with
+ *       d->n % 128 == 0.
  * Errors as hq_pack_weights; HQ_ERR_UNSUPPORTED for other formats or n. */
 hq_status hq_pack_weights_gated(const hq_quant_desc* d, const void* codes_host, const void* scales_host,
                                 const void* zeros_host, void* out_host, size_t out_bytes);

@@ -78,7 +78,8 @@ hq_status device_info(DeviceInfo* out);
 const hq_tuning* tuning_from_table(const hq_quant_desc& d, int m, hq_tuning* tmp);
 
 // Descriptor, format and tuning checks of a W4A16-family call (INT4, INT3,
-// INT2 or MXFP4_A16 weights; grouped: num_experts >= 2, else exactly 1).
+// INT2, INT8, MXFP4_A16 or MXINT4 weights; grouped: num_experts >= 2, else
+// exactly 1).
 hq_status check_w4_call(const hq_quant_desc* d, const hq_tuning* t, bool grouped);
 
 // W4A16 (dense or grouped) planning and launch.

@@ -1,6 +1,6 @@
 // Dense and grouped (MoE) W4A16 GEMM for sm_100a with the INT4 dequantization
-// fused into the kernel (also run with INT3, INT2 or MXFP4 weights: the
-// same kernel with another record decode).
+// fused into the kernel (also run with INT3, INT2, INT8, MXFP4 or MXINT4
+// weights: the same kernel with another record decode).
 //
 // Method: the weights are stored as 4-bit codes with a per-group fp16 scale
 // and an optional uint4 zero point, described separately ("Humming:

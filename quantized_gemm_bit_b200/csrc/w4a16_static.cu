@@ -1,5 +1,5 @@
-// Dense W4A16 GEMM entry point that allocates nothing (INT4, INT3, INT2 or
-// MXFP4_A16 weights, as hq_gemm_w4a16).
+// Dense W4A16 GEMM entry point that allocates nothing (INT4, INT3, INT2,
+// INT8, MXFP4_A16 or MXINT4 weights, as hq_gemm_w4a16).
 //
 // Some callers cannot allocate device memory at the point where they run a
 // layer: an inference engine that plans every buffer up front and then
