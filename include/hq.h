@@ -151,6 +151,11 @@ typedef struct {
  *              go to the tensor core and each 128-K group's scale is
  *              applied to its fp32 group sum (no rounding of w or s);
  *              larger tiles as 1.  INT4, INT3 and INT2 weights.
+ *              3 = dense INT4 GEMMs of 1 to 16 tokens: the register-path
+ *              kernel (codes dequantized straight into mma.sync register
+ *              fragments, exact (q - z) with each group's scale applied to
+ *              its fp32 sum, as 2); split_k = CTAs per weight tile (0: the
+ *              library's split).  Other calls run the library's choice.
  *              Block-scaled GEMMs: 0.                                     */
 typedef struct {
   int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;
@@ -189,7 +194,8 @@ hq_status hq_tuning_table_set(const hq_tuning_entry* entries, int32_t count);
  * rules), without a GPU if none is current (148 SMs assumed, as for
  * hq_workspace_size). */
 typedef struct {
-  int32_t kernel;      /* 1: W4A16 weights rescaled to bf16, 2: W4A16 exact weights, 3: block-scaled */
+  int32_t kernel;      /* 1: W4A16 weights rescaled to bf16, 2: W4A16 exact weights, 3: block-scaled,
+                          4: W4A16 register path (exact weights in mma.sync fragments)              */
   int32_t tile_m;      /* token tile                                                                 */
   int32_t grid;        /* CTAs                                                                       */
   int32_t split;       /* 0: whole tiles; >0: tiles share their K range (stream-K or a K split)      */

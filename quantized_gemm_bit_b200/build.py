@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libhq.so")
-SOURCES = ["hq_api.cu", "w4a16.cu", "w4a16_small.cu", "w4a16_static.cu", "blockscaled.cu", "quant.cu", "moe.cu", "hq_pack.cpp"]
+SOURCES = ["hq_api.cu", "w4a16.cu", "w4a16_small.cu", "w4a16_reg.cu", "w4a16_static.cu", "blockscaled.cu", "quant.cu", "moe.cu", "hq_pack.cpp"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

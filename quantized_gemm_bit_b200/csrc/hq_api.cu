@@ -106,7 +106,7 @@ hq_status check_w4_tuning(const hq_quant_desc* d, const hq_tuning* t, bool group
   if (t->tile_m && t->tile_m != 16 && t->tile_m != 32 && t->tile_m != 64 && t->tile_m != 128 && t->tile_m != 256)
     return HQ_ERR_UNSUPPORTED;
   if ((t->tile_n && t->tile_n != 128) || (t->tile_k && t->tile_k != 128) || t->split_k < 0 || t->stages < 0 ||
-      t->cta_group < 0 || t->cta_group > 2 || t->variant < 0 || t->variant > 2 ||
+      t->cta_group < 0 || t->cta_group > 2 || t->variant < 0 || t->variant > 3 ||
       (t->flags & ~HQ_TUNE_NO_EARLY_WEIGHTS) != 0)
     return HQ_ERR_UNSUPPORTED;
   if (grouped && t->split_k > 1) return HQ_ERR_UNSUPPORTED;
@@ -517,9 +517,10 @@ hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t
     const bool mx = d->fmt == HQ_FMT_MXFP4_A16 || d->fmt == HQ_FMT_MXINT4;
     p.tile_m = cfg.ntok;
     p.grid = cfg.grid;
-    p.split = grouped ? 0 : cfg.splits == 0 ? 0 : cfg.splits;
+    const bool reg = !grouped && cfg.variant == 3;
+    p.split = grouped ? 0 : cfg.splits == 0 || (reg && cfg.splits == 1) ? 0 : cfg.splits;
     p.whole_tiles = grouped ? 0 : cfg.dp_tiles;
-    p.kernel = (!mx && cfg.ntok <= 64 && cfg.variant != 1) ? 2 : 1;
+    p.kernel = reg ? 4 : (!mx && cfg.ntok <= 64 && cfg.variant != 1) ? 2 : 1;
     p.cta_group = cfg.cta_group;
     p.ring_stages = depth;
     p.stages = (cfg.stages > 0 && cfg.stages < depth) ? cfg.stages : depth;

@@ -61,7 +61,10 @@ struct W4Config {
   int variant;  // 0: library's choice (exact weights for tiles of <= 64
                 // tokens, bf16-rescaled above); 1: bf16-rescaled weights for
                 // every tile; 2: exact (q - z) weights + per-group fp32
-                // scaling for tiles of <= 64 tokens (bf16-rescaled above)
+                // scaling for tiles of <= 64 tokens (bf16-rescaled above);
+                // 3: dense INT4 at 1..16 tokens on the register-path kernel
+                // (exact (q - z) weights in mma.sync fragments, splits = K
+                // slices per weight tile, grid = tiles * splits)
 };
 
 struct DeviceInfo {
@@ -106,6 +109,16 @@ BsConfig bs_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, const hq_
 size_t bs_workspace_bytes(const hq_quant_desc& d, int m, const BsConfig& cfg);
 hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* packed, const void* a, const void* a_sf,
                     const float* a_scale, float a_global, int m, void* c, void* ws, cudaStream_t stream);
+
+// Register-path W4A16 kernel (INT4 weights, dense, 1..16 tokens; tuning
+// variant 3): the K slices per weight tile that fill the SMs in one wave of
+// kRegCtasPerSm CTAs per SM, its workspace and its launch.
+constexpr int kRegCtasPerSm = 4;
+constexpr int kRegRing = 3;          // activation ring depth (stages of 2 records)
+int reg_splits(int num_sms, const hq_quant_desc& d);
+size_t reg_workspace_bytes(const W4Config& cfg);
+hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m, void* c,
+                     void* ws, cudaStream_t stream);
 
 // Ring depth (SMEM pipeline stages) of the kernel a plan launches.
 int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg);

@@ -861,6 +861,34 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
   cfg.cta_group = 1;
   cfg.variant = t ? t->variant : 0;
   cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
+  // The register-path kernel: dense INT4 at 1..16 tokens, on request
+  // (variant 3); a request that does not apply (more tokens, another
+  // format, MoE) gets the library's choice.  The library's choice takes it
+  // for 1..8 tokens (one 8-token MMA tile), and for 9..16 tokens where the
+  // exact-weight kernel would share K ranges between CTAs (its whole-tile
+  // plan does not fill the SMs).  Measured on B200 (per launch, back to
+  // back): M <= 8, K=7168 N=18432 22.4-22.7 us against 24.5-24.9 for the
+  // exact-weight kernel, K=18432 N=7168 23.7-24.0 against 30.2-30.9;
+  // M=16 27.6 against 25.2 (whole tiles) and 29.1 against 32.7 (stream-K).
+  const bool reg_fits = !grouped && d.fmt == HQ_FMT_INT4 && m <= 16 && ntok <= 16 && !(t && t->cta_group == 2);
+  if (cfg.variant == 3 && !reg_fits) cfg.variant = 0;
+  bool use_reg = reg_fits && cfg.variant == 3;
+  if (reg_fits && cfg.variant == 0) {
+    const long long tiles16 = dense_tiles(d, m, 16);
+    const long long waves = (tiles16 + dev.num_sms - 1) / dev.num_sms;
+    const bool exact_whole = (double)tiles16 / (double)(waves * dev.num_sms) >= 0.85;
+    use_reg = m <= 8 || !exact_whole;
+  }
+  if (use_reg) {
+    const long long tiles = (d.n + kTileN - 1) / kTileN;
+    cfg.variant = 3;
+    cfg.ntok = 16;
+    cfg.dp_tiles = 0;
+    cfg.splits = (t && t->split_k > 0) ? (int)std::min<long long>(t->split_k, d.k / kBlockK)
+                                       : reg_splits(dev.num_sms, d);
+    cfg.grid = (int)(tiles * cfg.splits);
+    return cfg;
+  }
   if (grouped) {
     cfg.ntok = ntok;
     cfg.grid = dev.num_sms;
@@ -961,7 +989,8 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
 W4Config w4_plan(const DeviceInfo& dev, const hq_quant_desc& d, int m, bool grouped, const hq_tuning* t) {
   W4Config cfg = w4_plan_rules(dev, d, m, grouped, t);
   // four tile counters per output tile, in the workspace's fixed counter region
-  if (!grouped && cfg.splits != 0 && (size_t)dense_tiles(d, m, cfg.ntok) * 4 * sizeof(int32_t) > kWsCounterBytes)
+  if (!grouped && cfg.splits != 0 && (size_t)dense_tiles(d, m, cfg.ntok) * 4 * sizeof(int32_t) > kWsCounterBytes &&
+      !(cfg.variant == 3 && cfg.splits == 1))
     cfg = w4_whole_tiles(dev, d, m, cfg);
   return cfg;
 }
@@ -981,6 +1010,7 @@ int rescaled_depth(int ntok, int cta_group) {
 }  // namespace
 
 int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg) {
+  if (cfg.variant == 3) return kRegRing;   // the register path's activation ring (codes stream through registers)
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16, mxi4 = d.fmt == HQ_FMT_MXINT4;
   const int kfmt = d.fmt == HQ_FMT_INT3 ? kFmtInt3 : d.fmt == HQ_FMT_INT2 ? kFmtInt2 : d.fmt == HQ_FMT_INT8 ? kFmtInt8 : kFmtInt4;
   if (!mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1) return small_ring_depth(cfg.ntok, kfmt);
@@ -995,6 +1025,12 @@ int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg) {
 }
 
 W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4Config cfg) {
+  if (cfg.variant == 3) {
+    // register path: one CTA per weight tile over the whole K range
+    cfg.splits = 1;
+    cfg.grid = (d.n + kTileN - 1) / kTileN;
+    return cfg;
+  }
   cfg.splits = 0;
   cfg.dp_tiles = 0;
   cfg.cta_group = 1;
@@ -1003,6 +1039,7 @@ W4Config w4_whole_tiles(const DeviceInfo& dev, const hq_quant_desc& d, int m, W4
 }
 
 size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bool grouped) {
+  if (!grouped && cfg.variant == 3) return reg_workspace_bytes(cfg);
   size_t bytes = sizeof(WsHeader);
   if (grouped) return bytes;
   if (cfg.splits == 0) return bytes;  // data parallel: no partial sums
@@ -1014,6 +1051,7 @@ size_t w4_workspace_bytes(const hq_quant_desc& d, int m, const W4Config& cfg, bo
 hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m,
                     void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream, int swiglu) {
   const bool grouped = expert_offsets != nullptr;
+  if (!grouped && cfg.variant == 3) return reg_launch(d, cfg, packed, a, m, c, ws, stream);
   W4Params p{};
   p.packed = static_cast<const uint8_t*>(packed);
   p.c = static_cast<__nv_bfloat16*>(c);

@@ -182,18 +182,23 @@ def test_mxfp4_a16_pack_accepts_the_largest_finite_scale():
 
 
 def test_w4a16_family_formats_share_one_launch_plan():
-    """INT3 and MXFP4 weights run the INT4 kernels' plan: the same workspace
-    for the same shape, token count and tuning (no device needed; the size
-    is computed for a 148-SM part)."""
+    """INT3, INT2 and MXFP4 weights run the INT4 kernels' plan: the same
+    workspace for the same shape, token count and tuning (no device needed;
+    the size is computed for a 148-SM part), except where INT4 runs its
+    register-path kernel (plan kernel 4), which the other formats do not
+    have."""
     for m, t in ((1, None), (16, None), (300, None), (4096, None), (40, hq.Tuning(split_k=3)),
                  (200, hq.Tuning(tile_m=128))):
         d4 = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
         d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, 18432, 7168, 128, 1, 1)
         dx = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4_A16, 18432, 7168, 32, 0, 1)
         d2 = hq.hq_quant_desc_init(hq.HQ_FMT_INT2, 18432, 7168, 128, 0, 1)
-        w = hq.hq_workspace_size(d4, m, t)
-        assert w >= 256 and hq.hq_workspace_size(d3, m, t) == w == hq.hq_workspace_size(dx, m, t)
-        assert hq.hq_workspace_size(d2, m, t) == w
+        w = hq.hq_workspace_size(d3, m, t)
+        assert w >= 256 and hq.hq_workspace_size(dx, m, t) == w == hq.hq_workspace_size(d2, m, t)
+        if hq.hq_plan_describe(d4, m, t).kernel != 4:
+            assert hq.hq_workspace_size(d4, m, t) == w
+        else:
+            assert m <= 16 and hq.hq_plan_describe(d3, m, t).kernel != 4
 
 
 def test_fp4_scale_layout_is_a_bijection():
@@ -241,7 +246,7 @@ def test_gemm_argument_errors_need_no_gpu():
     t = hq.Tuning(tile_m=48)
     assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(t), 256, 1 << 20,
                             None) == hq.HQ_ERR_UNSUPPORTED
-    for bad in (hq.Tuning(variant=3), hq.Tuning(variant=-1), hq.Tuning(stages=-1), hq.Tuning(cta_group=3),
+    for bad in (hq.Tuning(variant=4), hq.Tuning(variant=-1), hq.Tuning(stages=-1), hq.Tuning(cta_group=3),
                 hq.Tuning(cta_group=2, tile_m=128), hq.Tuning(cta_group=2, split_k=2), hq.Tuning(flags=2)):
         assert L_.hq_gemm_w4a16(ctypes.byref(d), 16, 16, 4, 32, ctypes.byref(bad), 256, 1 << 20,
                                 None) == hq.HQ_ERR_UNSUPPORTED
