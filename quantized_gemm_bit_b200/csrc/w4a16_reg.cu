@@ -33,9 +33,17 @@
 //     the SMs in one wave; each CTA writes an fp32 partial tile, and the last
 //     of a tile's CTAs (a counter per tile) adds the partials in slice order
 //     and writes the bf16 output, so results repeat bit for bit.
-// mma.sync is the older tensor-core path; at these sizes the MMAs are a
-// small share of the time (the bound is HBM), and the register path avoids
-// the per-stage chain that the TMEM accumulator needs.
+// mma.sync is the older tensor-core path (on B200 a 16x8x16 MMA issues about
+// every 2.7 SM cycles, near 0.44 PFLOP/s for the GPU); at 1-8 tokens the MMAs
+// are a small share of the time (the bound is the codes' HBM traffic), at
+// 9-16 tokens they start to show.  Measured on B200 (per launch, back to back,
+// M <= 8): warps matter more than loads in flight per warp: two records in
+// flight per warp with four CTAs (16 warps) per SM beat four records with
+// three CTAs (22.4 against 24.5 us at K=7168 N=18432) and six with two
+// (30.1); staging the codes through shared memory with cp.async (three to
+// four records per warp) took 25.6-25.9 us, bulk L2 prefetches of each CTA's
+// whole K slice 25.4, code loads that skip L1 no change, and the in-order
+// activation reads (a 2-way bank conflict, one 16-byte code load) 2 % more.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -47,13 +55,6 @@ namespace hq {
 namespace w4 {
 
 namespace {
-
-// Activation loads: lanes of the upper half of a quad read their 16-byte
-// pieces rotated by two (conflict-free, two 8-byte code loads per chunk), or
-// in order (two lanes of a quad share a bank, one 16-byte code load per chunk).
-constexpr bool kRotate = true;
-// Code loads skip L1 (each byte is read once; keeps L1 free for nothing else to do).
-constexpr bool kCodesNoL1 = false;
 
 template <int NT8>
 struct RegCfg {
@@ -87,19 +88,7 @@ struct RegParams {
 
 __device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
   uint2 v;
-  if (kCodesNoL1)
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  else
-    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-  uint4 v;
-  if (kCodesNoL1)
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  else
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
 }
 __device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
@@ -174,7 +163,7 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   // codes of (T, h): row rw = 32 warp + 16 T + 8 h + g, chunk qd, at byte
   // (qd * 128 + rw) * 16; the upper half of a quad takes the chunk's two
   // 8-byte halves in swapped order (word slot i holds word (i + 2 (qd >> 1)) % 4)
-  const int rot = kRotate ? (qd >> 1) * 8 : 0;
+  const int rot = (qd >> 1) * 8;
   int coff[2][2], row[2][2];
 #pragma unroll
   for (int T = 0; T < 2; ++T)
@@ -195,20 +184,12 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
       for (int T = 0; T < 2; ++T)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (kRotate) {
-            const uint2 lo = ldg_nc_v2(rec + coff[T][h] + rot);
-            const uint2 hi = ldg_nc_v2(rec + coff[T][h] + (8 - rot));
-            wv[u][T][h][0] = lo.x;
-            wv[u][T][h][1] = lo.y;
-            wv[u][T][h][2] = hi.x;
-            wv[u][T][h][3] = hi.y;
-          } else {
-            const uint4 v = ldg_nc_v4(rec + coff[T][h]);
-            wv[u][T][h][0] = v.x;
-            wv[u][T][h][1] = v.y;
-            wv[u][T][h][2] = v.z;
-            wv[u][T][h][3] = v.w;
-          }
+          const uint2 lo = ldg_nc_v2(rec + coff[T][h] + rot);
+          const uint2 hi = ldg_nc_v2(rec + coff[T][h] + (8 - rot));
+          wv[u][T][h][0] = lo.x;
+          wv[u][T][h][1] = lo.y;
+          wv[u][T][h][2] = hi.x;
+          wv[u][T][h][3] = hi.y;
           sc[u][T][h] = ldg_nc_u16(rec + kW4RecCodes + 2 * row[T][h]);
           if (HASZ) zp[u][T][h] = ldg_nc_u8(rec + kW4RecCodes + 256 + row[T][h]);
         }
@@ -253,7 +234,7 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   uint32_t aoff[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int piece = 4 * (qd & 1) + (kRotate ? ((i + 2 * (qd >> 1)) & 3) : i);
+    const int piece = 4 * (qd & 1) + ((i + 2 * (qd >> 1)) & 3);
     aoff[i] = (uint32_t)((qd >> 1) * C::kBox + g * 128 + ((piece ^ g) << 4));
   }
 
