@@ -65,6 +65,7 @@ struct W4Config {
                 // 3: dense INT4 at 1..16 tokens on the register-path kernel
                 // (exact (q - z) weights in mma.sync fragments, splits = K
                 // slices per weight tile, grid = tiles * splits)
+  int reg_tw;   // register path: 16-row MMA tiles per warp (1: grids of fewer CTAs than SMs, else 2)
 };
 
 struct DeviceInfo {
@@ -112,8 +113,10 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
 
 // Register-path W4A16 kernel (INT4 weights, dense, 1..16 tokens; tuning
 // variant 3): the K slices per weight tile that fill the SMs in one wave of
-// kRegCtasPerSm CTAs per SM, its workspace and its launch.
-constexpr int kRegCtasPerSm = 4;
+// reg_ctas_per_sm(2) CTAs per SM, its workspace and its launch.
+// tw = 16-row MMA tiles per warp (CTAs of 128 rows: 8 / tw warps); CTAs
+// resident per SM (registers and shared memory) of that kernel
+constexpr int reg_ctas_per_sm(int tw) { return tw == 1 ? 3 : 4; }
 constexpr int kRegRing = 3;          // activation ring depth (stages of 2 records)
 int reg_splits(int num_sms, const hq_quant_desc& d);
 size_t reg_workspace_bytes(const W4Config& cfg);

@@ -56,9 +56,10 @@ namespace w4 {
 
 namespace {
 
-template <int NT8>
+template <int NT8, int TW_>
 struct RegCfg {
-  static constexpr int kWarps = 4;
+  static constexpr int kTw = TW_;               // 16-row MMA tiles per warp (1 or 2)
+  static constexpr int kWarps = 8 / kTw;        // 128 weight rows per CTA
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kP = 2;                 // records per activation stage = records in flight per warp
   static constexpr int kD = kRegRing;          // activation ring depth (stages)
@@ -68,14 +69,16 @@ struct RegCfg {
   static constexpr int kStage = kP * kRecA;
   static constexpr int kBarOff = kD * kStage;
   static constexpr int kSmem = kBarOff + 2 * kD * 8 + 16 + 1024;  // + 1 KiB for the 1024-byte alignment
-  static constexpr int kNv4 = 2 * NT8;         // float4s per thread in a partial tile
+  static constexpr int kNv4 = kTw * NT8;       // float4s per thread in a partial tile
+  static constexpr int kCtasPerSm = reg_ctas_per_sm(TW_);
   static_assert(kBox % 1024 == 0, "a 128-byte-swizzled box starts on a 1024-byte boundary");
+  static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "kCtasPerSm CTAs fit one SM's shared memory");
 };
 
 struct RegParams {
   const uint8_t* packed;   // record (0, 0)
   __nv_bfloat16* c;        // [m][n]
-  float* partials;         // [grid][kNv4][128 threads] float4
+  float* partials;         // [grid][kNv4][kThreads] float4
   int32_t* counters;       // 4 per weight tile, the first used
   uint32_t* err;
   uint64_t wait_ns;
@@ -122,14 +125,14 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w, int j, uint32_t z2) {
   return bf16x2_sub(lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x43004300u), z2);
 }
 
-// Warp w of the CTA owns rows 32w .. 32w+31 of the 128-row weight tile: MMA
-// tile T (0, 1) row g (lane / 4) is weight row 32w + 16T + g, row g + 8 is
-// 32w + 16T + 8 + g.  Lane quad position qd (lane % 4) holds the 32-K chunk qd
-// of each record for those rows.
-template <int NT8, bool HASZ>
-__global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
+// Warp w of the CTA owns rows 16 TW w .. 16 TW (w + 1) - 1 of the 128-row
+// weight tile (TW = 1 or 2): MMA tile T row g (lane / 4) is weight
+// row 16 TW w + 16T + g, row g + 8 is 16 TW w + 16T + 8 + g.  Lane quad
+// position qd (lane % 4) holds the 32-K chunk qd of each record for those rows.
+template <int NT8, bool HASZ, int TWT>
+__global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::kCtasPerSm)
     w4a16_reg_kernel(const __grid_constant__ CUtensorMap tmap_a, const RegParams p) {
-  using C = RegCfg<NT8>;
+  using C = RegCfg<NT8, TWT>;
   constexpr int P = C::kP;
   constexpr int D = C::kD;
 
@@ -164,24 +167,25 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   // (qd * 128 + rw) * 16; the upper half of a quad takes the chunk's two
   // 8-byte halves in swapped order (word slot i holds word (i + 2 (qd >> 1)) % 4)
   const int rot = (qd >> 1) * 8;
-  int coff[2][2], row[2][2];
+  constexpr int TW = C::kTw;
+  int coff[TW][2], row[TW][2];
 #pragma unroll
-  for (int T = 0; T < 2; ++T)
+  for (int T = 0; T < TW; ++T)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      row[T][h] = 32 * warp + 16 * T + 8 * h + g;
+      row[T][h] = 16 * TW * warp + 16 * T + 8 * h + g;
       coff[T][h] = (qd * 128 + row[T][h]) * 16;
     }
   const uint8_t* rec0 = p.packed + ((size_t)tile * p.k_blocks + kb0) * (size_t)p.rec_bytes;
 
-  uint32_t wv[P][2][2][4];  // [record slot][T][h][word slot]
-  uint32_t sc[P][2][2];     // fp16 scale bits of row (T, h)
-  uint32_t zp[P][2][2];     // zero point of row (T, h) (HASZ)
+  uint32_t wv[P][TW][2][4];  // [record slot][T][h][word slot]
+  uint32_t sc[P][TW][2];     // fp16 scale bits of row (T, h)
+  uint32_t zp[P][TW][2];     // zero point of row (T, h) (HASZ)
   auto load_rec = [&](int u, int r) {
     if (r < nrec) {
       const uint8_t* rec = rec0 + (size_t)r * p.rec_bytes;
 #pragma unroll
-      for (int T = 0; T < 2; ++T)
+      for (int T = 0; T < TW; ++T)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint2 lo = ldg_nc_v2(rec + coff[T][h] + rot);
@@ -238,9 +242,9 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
     aoff[i] = (uint32_t)((qd >> 1) * C::kBox + g * 128 + ((piece ^ g) << 4));
   }
 
-  float acc[2][NT8][4];
+  float acc[TW][NT8][4];
 #pragma unroll
-  for (int T = 0; T < 2; ++T)
+  for (int T = 0; T < TW; ++T)
 #pragma unroll
     for (int t = 0; t < NT8; ++t)
 #pragma unroll
@@ -270,14 +274,14 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
     for (int u = 0; u < P; ++u) {
       const int r = j * P + u;
       if (r < nrec) {
-        uint32_t z2[2][2];
+        uint32_t z2[TW][2];
 #pragma unroll
-        for (int T = 0; T < 2; ++T)
+        for (int T = 0; T < TW; ++T)
 #pragma unroll
           for (int h = 0; h < 2; ++h) z2[T][h] = HASZ ? (0x43004300u | zp[u][T][h] | (zp[u][T][h] << 16)) : 0x43084308u;
-        float d[2][NT8][4];
+        float d[TW][NT8][4];
 #pragma unroll
-        for (int T = 0; T < 2; ++T)
+        for (int T = 0; T < TW; ++T)
 #pragma unroll
           for (int t = 0; t < NT8; ++t)
 #pragma unroll
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-            for (int T = 0; T < 2; ++T) {
+            for (int T = 0; T < TW; ++T) {
               const uint32_t a0 = code_pair(wv[u][T][0][i], 2 * hh, z2[T][0]);
               const uint32_t a1 = code_pair(wv[u][T][1][i], 2 * hh, z2[T][1]);
               const uint32_t a2 = code_pair(wv[u][T][0][i], 2 * hh + 1, z2[T][0]);
@@ -303,7 +307,7 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
           }
         }
 #pragma unroll
-        for (int T = 0; T < 2; ++T) {
+        for (int T = 0; T < TW; ++T) {
           const float s0 = __half2float(__ushort_as_half((unsigned short)sc[u][T][0]));
           const float s1 = __half2float(__ushort_as_half((unsigned short)sc[u][T][1]));
 #pragma unroll
@@ -327,9 +331,9 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   }
 
   // ---- output: feature tile * 128 + row, token 8t + 2 qd + e
-  auto store = [&](float (&v)[2][NT8][4]) {
+  auto store = [&](float (&v)[TW][NT8][4]) {
 #pragma unroll
-    for (int T = 0; T < 2; ++T)
+    for (int T = 0; T < TW; ++T)
 #pragma unroll
       for (int t = 0; t < NT8; ++t)
 #pragma unroll
@@ -347,7 +351,7 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   // sums the partials in slice order
   float4* mine = reinterpret_cast<float4*>(p.partials) + (size_t)blockIdx.x * C::kNv4 * C::kThreads + threadIdx.x;
 #pragma unroll
-  for (int T = 0; T < 2; ++T)
+  for (int T = 0; T < TW; ++T)
 #pragma unroll
     for (int t = 0; t < NT8; ++t)
       __stcg(mine + (T * NT8 + t) * C::kThreads, make_float4(acc[T][t][0], acc[T][t][1], acc[T][t][2], acc[T][t][3]));
@@ -360,11 +364,11 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   __syncthreads();
   if (!*s_last) return;
   __threadfence();
-  float sum[2][NT8][4];
+  float sum[TW][NT8][4];
   const float4* first = reinterpret_cast<const float4*>(p.partials) +
                         (size_t)tile * p.splits * C::kNv4 * C::kThreads + threadIdx.x;
 #pragma unroll
-  for (int T = 0; T < 2; ++T)
+  for (int T = 0; T < TW; ++T)
 #pragma unroll
     for (int t = 0; t < NT8; ++t) {
       float4 s4 = __ldcg(first + (T * NT8 + t) * C::kThreads);
@@ -384,10 +388,10 @@ __global__ void __launch_bounds__(RegCfg<NT8>::kThreads, kRegCtasPerSm)
   store(sum);
 }
 
-template <int NT8, bool HASZ>
+template <int NT8, bool HASZ, int TWT>
 hq_status reg_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cudaStream_t stream) {
-  auto kern = w4a16_reg_kernel<NT8, HASZ>;
-  const size_t smem = RegCfg<NT8>::kSmem;
+  auto kern = w4a16_reg_kernel<NT8, HASZ, TWT>;
+  const size_t smem = RegCfg<NT8, TWT>::kSmem;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -396,7 +400,7 @@ hq_status reg_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cud
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  return launch_pdl(kern, dim3(grid), dim3(RegCfg<NT8>::kThreads), smem, stream, map, p) == cudaSuccess
+  return launch_pdl(kern, dim3(grid), dim3(RegCfg<NT8, TWT>::kThreads), smem, stream, map, p) == cudaSuccess
              ? HQ_OK
              : HQ_ERR_CUDA;
 }
@@ -407,13 +411,12 @@ hq_status reg_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cud
 using w4::RegParams;
 
 // CTAs per weight tile (K slices) of the register-path plan: the split that
-// fills the SMs best in one wave of kRegCtasPerSm CTAs per SM (a tie goes to
-// more CTAs: more bytes in flight).  kRegCtasPerSm must match the kernel's
-// occupancy (__launch_bounds__ and its shared memory).
+// fills the SMs best in one wave of reg_ctas_per_sm(2) CTAs per SM (a tie
+// goes to more CTAs: more bytes in flight).
 int reg_splits(int num_sms, const hq_quant_desc& d) {
   const long long tiles = (d.n + kTileN - 1) / kTileN;
   const long long kbs = d.k / kBlockK;
-  const long long slots = (long long)num_sms * kRegCtasPerSm;
+  const long long slots = (long long)num_sms * reg_ctas_per_sm(2);
   int best = 1;
   double best_eff = -1.0;
   for (long long s = 1; s <= kbs && tiles * s <= slots; ++s) {
@@ -468,9 +471,16 @@ hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pa
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
   const bool hz = d.has_zero_point != 0;
+  // grids of fewer CTAs than SMs: eight warps of 16 rows per CTA (more warps
+  // on each busy SM); else four warps of 32 rows at four CTAs per SM
+  if (cfg.reg_tw == 1) {
+    if (nt8 == 1)
+      return hz ? w4::reg_launch_t<1, true, 1>(map, p, cfg.grid, stream) : w4::reg_launch_t<1, false, 1>(map, p, cfg.grid, stream);
+    return hz ? w4::reg_launch_t<2, true, 1>(map, p, cfg.grid, stream) : w4::reg_launch_t<2, false, 1>(map, p, cfg.grid, stream);
+  }
   if (nt8 == 1)
-    return hz ? w4::reg_launch_t<1, true>(map, p, cfg.grid, stream) : w4::reg_launch_t<1, false>(map, p, cfg.grid, stream);
-  return hz ? w4::reg_launch_t<2, true>(map, p, cfg.grid, stream) : w4::reg_launch_t<2, false>(map, p, cfg.grid, stream);
+    return hz ? w4::reg_launch_t<1, true, 2>(map, p, cfg.grid, stream) : w4::reg_launch_t<1, false, 2>(map, p, cfg.grid, stream);
+  return hz ? w4::reg_launch_t<2, true, 2>(map, p, cfg.grid, stream) : w4::reg_launch_t<2, false, 2>(map, p, cfg.grid, stream);
 }
 
 }  // namespace hq

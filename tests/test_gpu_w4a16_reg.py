@@ -2,7 +2,7 @@
 INT4 at 1..16 tokens, codes dequantized straight into mma.sync fragments)
 against the fp64 oracle, through the C ABI: full outputs on shapes with
 ragged token counts, ragged N and several K splits, the bench's full-size
-M-sweep shapes (sampled rows), bitwise repeats, counters left at zero,
+M-sweep shapes (every row), bitwise repeats, counters left at zero,
 guard bands, exact zeros, and the plan it reports."""
 
 import numpy as np
@@ -54,11 +54,13 @@ REG = hq.Tuning(variant=3)
 @pytest.mark.parametrize("m,n,k,asym", [
     (1, 128, 128, False), (1, 256, 1024, True), (4, 200, 384, False), (5, 640, 384, True),
     (8, 384, 1152, False), (9, 1000, 640, True), (13, 1152, 2560, False), (16, 1024, 1024, True),
-    (16, 136, 256, False), (3, 9, 512, True),
+    (16, 136, 256, False), (3, 9, 512, True), (7, 4096, 2048, True), (16, 4096, 2048, False),
 ])
 def test_register_path_full_output(m, n, k, asym):
     """One and two 8-token tiles, N not a multiple of 128 (down to one
-    partial tile), K from one record to 20, the library's K split."""
+    partial tile), K from one record to 20, the library's K split; grids
+    below one CTA per SM (eight warps of 16 rows per CTA) and above it (the
+    N=4096 cases: four warps of 32 rows)."""
     d, blob, a, (q, s, z) = make_case(m, n, k, asym, 500 + m + n)
     assert hq.hq_plan_describe(d, m, REG).kernel == 4
     c, _ = run(d, blob, a, m, REG)
