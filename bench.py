@@ -62,25 +62,24 @@ def load_peaks():
 # profiles/traffic_w4a16_sweep.md with the commit it ran on.  The capture
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
-# capture is taken again.  (The fingerprint below is of sources that differ
-# from the captured commit's in comments only.)
-TRAFFIC_COMMIT = "fb566ad"
-TRAFFIC_SOURCES = "a0928f5839a69638"
+# capture is taken again.
+TRAFFIC_COMMIT = "806db2d"
+TRAFFIC_SOURCES = "87fec370729d9ca9"
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 70462720,
-    (4, 7168, 18432): 69294592,
-    (16, 7168, 18432): 69672704,
-    (64, 7168, 18432): 71269120,
-    (256, 7168, 18432): 75859968,
-    (1024, 7168, 18432): 150655488,
-    (4096, 7168, 18432): 343374080,
-    (1, 18432, 7168): 69810432,
-    (4, 18432, 7168): 70138624,
-    (16, 18432, 7168): 70899200,
-    (64, 18432, 7168): 74140928,
-    (256, 18432, 7168): 86837248,
-    (1024, 18432, 7168): 197917440,
-    (4096, 18432, 7168): 711796992,
+    (1, 7168, 18432): 68844032,
+    (4, 7168, 18432): 68222720,
+    (16, 7168, 18432): 69713920,
+    (64, 7168, 18432): 71245312,
+    (256, 7168, 18432): 75831808,
+    (1024, 7168, 18432): 149061120,
+    (4096, 7168, 18432): 355084288,
+    (1, 18432, 7168): 68239104,
+    (4, 18432, 7168): 68381440,
+    (16, 18432, 7168): 68766208,
+    (64, 18432, 7168): 74174720,
+    (256, 18432, 7168): 86867712,
+    (1024, 18432, 7168): 197565952,
+    (4096, 18432, 7168): 713222912,
 }
 
 
