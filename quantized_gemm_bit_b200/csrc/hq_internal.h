@@ -112,13 +112,11 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
                     const float* a_scale, float a_global, int m, void* c, void* ws, cudaStream_t stream);
 
 // Register-path W4A16 kernel (INT4 weights, dense, 1..16 tokens; tuning
-// variant 3): the K slices per weight tile that fill the SMs in one wave of
-// reg_ctas_per_sm(2) CTAs per SM, its workspace and its launch.
-// tw = 16-row MMA tiles per warp (CTAs of 128 rows: 8 / tw warps); CTAs
-// resident per SM (registers and shared memory) of that kernel
-constexpr int reg_ctas_per_sm(int tw) { return tw == 1 ? 3 : 4; }
-constexpr int kRegRing = 3;          // activation ring depth (stages of 2 records)
-int reg_splits(int num_sms, const hq_quant_desc& d);
+// variant 3): CTAs per SM a plan fills (slots) for 8- or 16-token tiles, the
+// K slices per weight tile, its workspace and its launch.
+constexpr int reg_slots_per_sm(int nt8) { return nt8 == 1 ? 3 : 4; }
+constexpr int kRegRing = 3;          // stages of the 8-token kernel's ring (the 16-token kernel: 4)
+int reg_splits(int num_sms, const hq_quant_desc& d, int m);
 size_t reg_workspace_bytes(const W4Config& cfg);
 hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m, void* c,
                      void* ws, cudaStream_t stream);

@@ -861,31 +861,22 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
   cfg.cta_group = 1;
   cfg.variant = t ? t->variant : 0;
   cfg.early_weights = (t && (t->flags & HQ_TUNE_NO_EARLY_WEIGHTS)) ? 0 : 1;
-  // The register-path kernel: dense INT4 at 1..16 tokens, on request
-  // (variant 3); a request that does not apply (more tokens, another
-  // format, MoE) gets the library's choice.  The library's choice takes it
-  // for 1..8 tokens (one 8-token MMA tile), and for 9..16 tokens where the
-  // exact-weight kernel would share K ranges between CTAs (its whole-tile
-  // plan does not fill the SMs).  Measured on B200 (per launch, back to
-  // back): M <= 8, K=7168 N=18432 22.4-22.7 us against 24.5-24.9 for the
-  // exact-weight kernel, K=18432 N=7168 23.7-24.0 against 30.2-30.9;
-  // M=16 27.6 against 25.2 (whole tiles) and 29.1 against 32.7 (stream-K).
+  // The register-path kernel: dense INT4 at 1..16 tokens, the library's
+  // choice there and on request (variant 3); a request that does not apply
+  // (more tokens, another format, MoE) gets the library's choice.  Measured
+  // on B200 (per launch, back to back): K=7168 N=18432 M <= 8 20.8 us, M=16
+  // 24.8, against 24.5 and 25.0 for the exact-weight kernel; K=18432 N=7168
+  // M <= 8 22.9, M=16 26.0, against 30.2 and 32.7.
   const bool reg_fits = !grouped && d.fmt == HQ_FMT_INT4 && m <= 16 && ntok <= 16 && !(t && t->cta_group == 2);
   if (cfg.variant == 3 && !reg_fits) cfg.variant = 0;
-  bool use_reg = reg_fits && cfg.variant == 3;
-  if (reg_fits && cfg.variant == 0) {
-    const long long tiles16 = dense_tiles(d, m, 16);
-    const long long waves = (tiles16 + dev.num_sms - 1) / dev.num_sms;
-    const bool exact_whole = (double)tiles16 / (double)(waves * dev.num_sms) >= 0.85;
-    use_reg = m <= 8 || !exact_whole;
-  }
+  const bool use_reg = reg_fits && (cfg.variant == 0 || cfg.variant == 3);
   if (use_reg) {
     const long long tiles = (d.n + kTileN - 1) / kTileN;
     cfg.variant = 3;
     cfg.ntok = 16;
     cfg.dp_tiles = 0;
     cfg.splits = (t && t->split_k > 0) ? (int)std::min<long long>(t->split_k, d.k / kBlockK)
-                                       : reg_splits(dev.num_sms, d);
+                                       : reg_splits(dev.num_sms, d, m);
     cfg.grid = (int)(tiles * cfg.splits);
     // Grids of fewer CTAs than SMs run eight warps of 16 rows per CTA (more
     // warps on each busy SM): M=16 K=N=1024 (64 CTAs) 8.4 -> 6.5 us on B200;
@@ -1015,7 +1006,7 @@ int rescaled_depth(int ntok, int cta_group) {
 }  // namespace
 
 int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg) {
-  if (cfg.variant == 3) return kRegRing;   // the register path's activation ring (codes stream through registers)
+  if (cfg.variant == 3) return kRegRing;   // the register path's ring of whole-record stages (8-token tiles)
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16, mxi4 = d.fmt == HQ_FMT_MXINT4;
   const int kfmt = d.fmt == HQ_FMT_INT3 ? kFmtInt3 : d.fmt == HQ_FMT_INT2 ? kFmtInt2 : d.fmt == HQ_FMT_INT8 ? kFmtInt8 : kFmtInt4;
   if (!mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1) return small_ring_depth(cfg.ntok, kfmt);

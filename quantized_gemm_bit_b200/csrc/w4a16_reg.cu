@@ -10,40 +10,34 @@
 // and s is applied to each group's fp32 sum.
 //
 // B200 design.  At M <= 16 the launch streams K*N/2 bytes of codes and does
-// almost no arithmetic per byte, so what matters is keeping enough bytes in
-// flight on every SM with as few instructions per byte as possible.  The
-// TMEM path (a TMA stage -> unpacking warps -> tcgen05.st -> an MMA warp ->
-// scale warps) pays a chain of mbarrier handshakes per stage; here every warp
-// is its own pipeline with no handshake on the weight path:
-//   * each warp owns 32 weight rows (two 16-row MMA tiles) of a 128-row tile
-//     and a K range, and keeps kP records (128 K each) of its codes in flight
-//     in registers, loaded with plain coalesced global loads (a warp's load
-//     covers whole 128-byte lines of the packed record);
-//   * codes become bf16 (q - z) in registers and feed mma.sync m16n8k16
-//     directly (weights as the 16-row A side, tokens as the 8-wide B side,
-//     one or two 8-token tiles); each group's fp32 result is scaled into a
-//     running fp32 sum;
-//   * activations, shared by the CTA's four warps, are staged by TMA (128-byte
-//     swizzle) in a small shared-memory ring, one mbarrier pair per stage of
-//     kP records.  Lanes 8 bytes apart in K would meet in one bank; lanes of
-//     the upper half of a quad read their four 16-byte pieces in an order
-//     rotated by two, and load their code words in the same rotated order,
-//     which makes every activation load conflict-free;
+// little arithmetic per byte, so what matters is keeping enough bytes in
+// flight on every SM and few instructions per byte.  The TMEM path (a TMA
+// stage -> unpacking warps -> tcgen05.st -> an MMA warp -> scale warps) pays
+// a chain of mbarrier handshakes per stage; here the warps that convert the
+// codes also issue the MMAs, from registers:
+//   * each CTA owns one 128-row weight tile and a K slice; one thread copies
+//     whole records (codes, scales, zero points: one bulk copy per stage) and
+//     their activation boxes (TMA, 128-byte swizzle) into a small ring of
+//     shared-memory stages, one full and one empty mbarrier per stage;
+//   * each warp owns 32 rows (two 16-row MMA tiles; 16 rows for grids below
+//     one CTA per SM), reads its codes with ldmatrix (conflict-free, see
+//     below), turns them into the exact bf16 (q - z) in registers and feeds
+//     mma.sync m16n8k16 (weights = the 16-row A side, tokens = one or two
+//     8-wide B tiles); each group's fp32 result is scaled into a running
+//     fp32 sum;
 //   * the K range of a tile is split over a few CTAs so that the grid fills
-//     the SMs in one wave; each CTA writes an fp32 partial tile, and the last
-//     of a tile's CTAs (a counter per tile) adds the partials in slice order
-//     and writes the bf16 output, so results repeat bit for bit.
+//     the SMs; each CTA writes an fp32 partial tile, and the last of a tile's
+//     CTAs (a counter per tile) adds the partials in slice order and writes
+//     the bf16 output, so results repeat bit for bit.
 // mma.sync is the older tensor-core path (on B200 a 16x8x16 MMA issues about
 // every 2.7 SM cycles, near 0.44 PFLOP/s for the GPU); at 1-8 tokens the MMAs
-// are a small share of the time (the bound is the codes' HBM traffic), at
-// 9-16 tokens they start to show.  Measured on B200 (per launch, back to back,
-// M <= 8): warps matter more than loads in flight per warp: two records in
-// flight per warp with four CTAs (16 warps) per SM beat four records with
-// three CTAs (22.4 against 24.5 us at K=7168 N=18432) and six with two
-// (30.1); staging the codes through shared memory with cp.async (three to
-// four records per warp) took 25.6-25.9 us, bulk L2 prefetches of each CTA's
-// whole K slice 25.4, code loads that skip L1 no change, and the in-order
-// activation reads (a 2-way bank conflict, one 16-byte code load) 2 % more.
+// are a small share of the time, at 9-16 they start to show.  Measured on
+// B200 (per launch, back to back, M <= 8, K=7168 N=18432): this layout 20.8
+// us; codes loaded by each warp straight from global memory into registers
+// (two records in flight per warp, no shared-memory hop) 22.4 us at best
+// (four records at three CTAs per SM 24.5, six at two 30.1); the same through
+// a per-warp cp.async ring 25.6-25.9; bulk L2 prefetches of each CTA's slice
+// 25.4.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -56,24 +50,6 @@ namespace w4 {
 
 namespace {
 
-template <int NT8, int TW_>
-struct RegCfg {
-  static constexpr int kTw = TW_;               // 16-row MMA tiles per warp (1 or 2)
-  static constexpr int kWarps = 8 / kTw;        // 128 weight rows per CTA
-  static constexpr int kThreads = 32 * kWarps;
-  static constexpr int kP = 2;                 // records per activation stage = records in flight per warp
-  static constexpr int kD = kRegRing;          // activation ring depth (stages)
-  static constexpr int kRows = 8 * NT8;        // tokens in the activation box
-  static constexpr int kBox = kRows * 128;     // one 64-K box: kRows rows of 128 bytes
-  static constexpr int kRecA = 2 * kBox;       // one record's activations
-  static constexpr int kStage = kP * kRecA;
-  static constexpr int kBarOff = kD * kStage;
-  static constexpr int kSmem = kBarOff + 2 * kD * 8 + 16 + 1024;  // + 1 KiB for the 1024-byte alignment
-  static constexpr int kNv4 = kTw * NT8;       // float4s per thread in a partial tile
-  static constexpr int kCtasPerSm = reg_ctas_per_sm(TW_);
-  static_assert(kBox % 1024 == 0, "a 128-byte-swizzled box starts on a 1024-byte boundary");
-  static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "kCtasPerSm CTAs fit one SM's shared memory");
-};
 
 struct RegParams {
   const uint8_t* packed;   // record (0, 0)
@@ -89,19 +65,14 @@ struct RegParams {
   int early_weights;       // load the first records' codes before the previous kernel has completed
 };
 
-__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ uint32_t ldg_nc_u16(const void* p) {
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
   uint16_t v;
-  asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint32_t ldg_nc_u8(const void* p) {
-  uint16_t v;
-  asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(v) : "l"(p));
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -125,16 +96,51 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w, int j, uint32_t z2) {
   return bf16x2_sub(lop3_and_or(w >> (4 * j), 0x000F000Fu, 0x43004300u), z2);
 }
 
-// Warp w of the CTA owns rows 16 TW w .. 16 TW (w + 1) - 1 of the 128-row
-// weight tile (TW = 1 or 2): MMA tile T row g (lane / 4) is weight
-// row 16 TW w + 16T + g, row g + 8 is 16 TW w + 16T + 8 + g.  Lane quad
-// position qd (lane % 4) holds the 32-K chunk qd of each record for those rows.
+// Whole records reach shared memory by one bulk copy per stage (long
+// contiguous reads, no registers held for loads in flight); each warp reads
+// its codes back with ldmatrix.  In the packed record, the
+// 16-byte chunk c of rows r .. r+7 is one 128-byte run, so an 8x8 b16
+// "matrix" of ldmatrix is chunk c of 8 consecutive rows, and lane (g, qd)
+// receives word qd of row g's chunk: exactly the quad distribution of the MMA
+// fragment, with no bank conflict.  Word qd of chunk c holds K = 32c + 8qd ..
+// +7, so lane (g, qd) reads activations K = 32c + 8qd .. +7 of its token; the
+// token of MMA column n is sigma(n) = (n >> 1) | ((n & 1) << 2), which puts
+// the two tokens of every 8-lane phase 4 rows apart under the 128-byte swizzle
+// and makes those reads conflict-free too.
+template <int NT8, int TW_>
+struct RegCfg {
+  static constexpr int kTw = TW_;
+  static constexpr int kWarps = 8 / kTw;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kP = NT8 == 2 ? 1 : 2;          // records per stage
+  static constexpr int kD = NT8 == 2 ? 4 : 3;          // stages
+  static constexpr int kRows = 8 * NT8;
+  static constexpr int kBox = kRows * 128;
+  static constexpr int kRecA = 2 * kBox;
+  static constexpr int kWBytes = (kP * kRecMax + 1023) / 1024 * 1024;   // codes, scales, zero points
+  static constexpr int kStage = kWBytes + kP * kRecA;
+  static constexpr int kBarOff = kD * kStage;
+  static constexpr int kSmem = kBarOff + 2 * kD * 8 + 16 + 1024;
+  static constexpr int kNv4 = kTw * NT8;
+  static constexpr int kCtasPerSm = 3;
+  static_assert(kBox % 1024 == 0 && kWBytes % 1024 == 0 && kStage % 1024 == 0, "1024-byte aligned boxes");
+  static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "kCtasPerSm CTAs fit one SM's shared memory");
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ int col_token(int n) { return (n >> 1) | ((n & 1) << 2); }
+
 template <int NT8, bool HASZ, int TWT>
 __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::kCtasPerSm)
     w4a16_reg_kernel(const __grid_constant__ CUtensorMap tmap_a, const RegParams p) {
   using C = RegCfg<NT8, TWT>;
   constexpr int P = C::kP;
   constexpr int D = C::kD;
+  constexpr int TW = C::kTw;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,6 +156,7 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
   const int kb1 = (int)((long long)(slice + 1) * p.k_blocks / p.splits);
   const int nrec = kb1 - kb0;
   const int nstage = (nrec + P - 1) / P;
+  const uint8_t* rec0 = p.packed + ((size_t)tile * p.k_blocks + kb0) * (size_t)p.rec_bytes;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < D; ++i) {
@@ -161,86 +168,63 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
     pdl_launch_dependents();
     prefetch_tensormap(&tmap_a);
   }
+  __syncthreads();  // barriers initialised
 
-  // ---- this thread's places in a record
-  // codes of (T, h): row rw = 32 warp + 16 T + 8 h + g, chunk qd, at byte
-  // (qd * 128 + rw) * 16; the upper half of a quad takes the chunk's two
-  // 8-byte halves in swapped order (word slot i holds word (i + 2 (qd >> 1)) % 4)
-  const int rot = (qd >> 1) * 8;
-  constexpr int TW = C::kTw;
-  int coff[TW][2], row[TW][2];
+  // stage x: records x*P .. of the slice; weights (one bulk copy) and the
+  // activations' boxes complete on full[x % D]; one thread
+  const uint64_t pol_w = policy_evict_first();
+  auto stage_bytes = [&](int x) { return (uint32_t)(min(P, nrec - x * P) * (p.rec_bytes + C::kRecA)); };
+  auto issue_weights = [&](int x) {
+    const int nr = min(P, nrec - x * P);
+    bulk_g2s(smem + (x % D) * C::kStage, rec0 + (size_t)x * P * p.rec_bytes, (uint32_t)(nr * p.rec_bytes),
+             &full[x % D], pol_w);
+  };
+  auto issue_acts = [&](int x) {
+    const int nr = min(P, nrec - x * P);
+    uint8_t* dst = smem + (x % D) * C::kStage + C::kWBytes;
+    for (int u = 0; u < nr; ++u) {
+      const int kx = (kb0 + x * P + u) * kBlockK;
+      tma_load_2d(dst + u * C::kRecA, &tmap_a, kx, 0, &full[x % D]);
+      tma_load_2d(dst + u * C::kRecA + C::kBox, &tmap_a, kx + 64, 0, &full[x % D]);
+    }
+  };
+  // Phase 1: the first stages' weights before the previous kernel has
+  // completed (no kernel on the stream writes them), unless the caller said
+  // otherwise; their activations after griddepcontrol.wait.
+  const int npre = min(D, nstage);
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < npre; ++x) {
+      mbar_arrive_expect_tx(&full[x], stage_bytes(x));
+      if (p.early_weights) issue_weights(x);
+    }
+  }
+  pdl_wait();   // activations, outputs, partials and counters may be in use until here
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < npre; ++x) {
+      if (!p.early_weights) issue_weights(x);
+      issue_acts(x);
+    }
+  }
+  int issued = npre;
+
+  int row[TW][2];
 #pragma unroll
   for (int T = 0; T < TW; ++T)
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      row[T][h] = 16 * TW * warp + 16 * T + 8 * h + g;
-      coff[T][h] = (qd * 128 + row[T][h]) * 16;
-    }
-  const uint8_t* rec0 = p.packed + ((size_t)tile * p.k_blocks + kb0) * (size_t)p.rec_bytes;
-
-  uint32_t wv[P][TW][2][4];  // [record slot][T][h][word slot]
-  uint32_t sc[P][TW][2];     // fp16 scale bits of row (T, h)
-  uint32_t zp[P][TW][2];     // zero point of row (T, h) (HASZ)
-  auto load_rec = [&](int u, int r) {
-    if (r < nrec) {
-      const uint8_t* rec = rec0 + (size_t)r * p.rec_bytes;
-#pragma unroll
-      for (int T = 0; T < TW; ++T)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint2 lo = ldg_nc_v2(rec + coff[T][h] + rot);
-          const uint2 hi = ldg_nc_v2(rec + coff[T][h] + (8 - rot));
-          wv[u][T][h][0] = lo.x;
-          wv[u][T][h][1] = lo.y;
-          wv[u][T][h][2] = hi.x;
-          wv[u][T][h][3] = hi.y;
-          sc[u][T][h] = ldg_nc_u16(rec + kW4RecCodes + 2 * row[T][h]);
-          if (HASZ) zp[u][T][h] = ldg_nc_u8(rec + kW4RecCodes + 256 + row[T][h]);
-        }
-    }
-  };
-
-  // Phase 1: the first records' codes (no kernel on the stream writes them)
-  // before the previous kernel has completed, unless the caller said otherwise.
-  if (p.early_weights) {
-#pragma unroll
-    for (int u = 0; u < P; ++u) load_rec(u, u);
-  }
-  __syncthreads();  // barriers initialised
-  pdl_wait();       // activations, outputs, partials and counters may be in use until here
-  if (!p.early_weights) {
-#pragma unroll
-    for (int u = 0; u < P; ++u) load_rec(u, u);
-  }
-
-  auto issue_stage = [&](int x) {  // one thread
-    const int r0 = x * P;
-    const int nr = min(P, nrec - r0);
-    uint64_t* fb = &full[x % D];
-    mbar_arrive_expect_tx(fb, (uint32_t)(nr * C::kRecA));
-    uint8_t* dst = smem + (x % D) * C::kStage;
-    for (int u = 0; u < nr; ++u) {
-      const int kx = (kb0 + r0 + u) * kBlockK;
-      tma_load_2d(dst + u * C::kRecA, &tmap_a, kx, 0, fb);
-      tma_load_2d(dst + u * C::kRecA + C::kBox, &tmap_a, kx + 64, 0, fb);
-    }
-  };
-  int issued = 0;
-  if (warp == 0) {
-    if (lane == 0 && nstage > 0) issue_stage(0);
-    issued = nstage > 0 ? 1 : 0;
-  }
-
-  // activation addresses: token row g + 8t of box (qd >> 1); the 16-byte
-  // piece of word slot i is piece 4 (qd & 1) + ((i + 2 (qd >> 1)) & 3) of the
-  // row, stored at piece index ^ (row & 7) by the 128-byte swizzle
-  const uint32_t sbase = smem_u32(smem);
+    for (int h = 0; h < 2; ++h) row[T][h] = 16 * TW * warp + 16 * T + 8 * h + g;
+  // ldmatrix row addresses: lane L gives row L % 8 of matrix L / 8; TW = 2:
+  // matrix k = (T, h) = (k / 2, k % 2) of one chunk; TW = 1: matrix k =
+  // (h, chunk) = (k % 2, c0 + k / 2) of a chunk pair
+  const int mk = lane >> 3, mi = lane & 7;
+  const uint32_t lds_row = TW == 2 ? (uint32_t)((16 * TW * warp + 16 * (mk >> 1) + 8 * (mk & 1) + mi) * 16)
+                                   : (uint32_t)(((mk >> 1) * 128 + 16 * warp + 8 * (mk & 1) + mi) * 16);
+  // activation reads: token row sigma(g) (+ 8t) of box c >> 1, piece 4 (c & 1) + qd
+  const int tg = col_token(g);
   uint32_t aoff[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int piece = 4 * (qd & 1) + ((i + 2 * (qd >> 1)) & 3);
-    aoff[i] = (uint32_t)((qd >> 1) * C::kBox + g * 128 + ((piece ^ g) << 4));
-  }
+  for (int c = 0; c < 4; ++c)
+    aoff[c] = (uint32_t)((c >> 1) * C::kBox + tg * 128 + (((4 * (c & 1) + qd) ^ tg) << 4));
+  const uint32_t sbase = smem_u32(smem);
 
   float acc[TW][NT8][4];
 #pragma unroll
@@ -252,15 +236,19 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
 
   bool ok = true;
   for (int j = 0; j < nstage; ++j) {
-    // the producer refills the slot of stage j + 1, freed at the end of stage j + 1 - D
-    if (warp == 0 && j + 1 < nstage) {
-      const int x = j + 1;
-      if (x >= D && !hq_wait_warp(&empty[x % D], ((x / D) - 1) & 1, p.wait_ns, s_abort)) {
+    // the producer refills the slot of stage j + D - 1, freed at the end of stage j - 1
+    if (warp == 0 && j >= 1 && j + D - 1 < nstage) {
+      const int x = j + D - 1;
+      if (!hq_wait_warp(&empty[x % D], ((x / D) - 1) & 1, p.wait_ns, s_abort)) {
         if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
         ok = false;
         break;
       }
-      if (lane == 0) issue_stage(x);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[x % D], stage_bytes(x));
+        issue_weights(x);
+        issue_acts(x);
+      }
       __syncwarp();
       issued = x + 1;
     }
@@ -269,16 +257,31 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
       ok = false;
       break;
     }
-    const uint32_t sa = sbase + (uint32_t)((j % D) * C::kStage);
+    const uint32_t st = sbase + (uint32_t)((j % D) * C::kStage);
 #pragma unroll
     for (int u = 0; u < P; ++u) {
       const int r = j * P + u;
       if (r < nrec) {
+        const uint32_t wrec = st + (uint32_t)(u * p.rec_bytes);
+        uint32_t w[TW][2][4];   // word qd of chunk c of row (T, h)
+        if (TW == 2) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ldsm_x4(wrec + lds_row + c * 2048, w[0][0][c], w[0][1][c], w[TW - 1][0][c], w[TW - 1][1][c]);
+        } else {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            ldsm_x4(wrec + lds_row + cc * 4096, w[0][0][2 * cc], w[0][1][2 * cc], w[0][0][2 * cc + 1], w[0][1][2 * cc + 1]);
+        }
         uint32_t z2[TW][2];
+        float s[TW][2];
 #pragma unroll
         for (int T = 0; T < TW; ++T)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) z2[T][h] = HASZ ? (0x43004300u | zp[u][T][h] | (zp[u][T][h] << 16)) : 0x43084308u;
+          for (int h = 0; h < 2; ++h) {
+            s[T][h] = __half2float(__ushort_as_half((unsigned short)lds_u16(wrec + kW4RecCodes + 2 * row[T][h])));
+            const uint32_t z = HASZ ? lds_u8(wrec + kW4RecCodes + 256 + row[T][h]) : 8u;
+            z2[T][h] = 0x43004300u | z | (z << 16);
+          }
         float d[TW][NT8][4];
 #pragma unroll
         for (int T = 0; T < TW; ++T)
@@ -286,20 +289,20 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
           for (int t = 0; t < NT8; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e) d[T][t][e] = 0.f;
-        const uint32_t ra = sa + (uint32_t)(u * C::kRecA);
+        const uint32_t ra = st + (uint32_t)(C::kWBytes + u * C::kRecA);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int c = 0; c < 4; ++c) {
           uint4 b[NT8];
 #pragma unroll
-          for (int t = 0; t < NT8; ++t) b[t] = lds128(ra + aoff[i] + t * 8 * 128);
+          for (int t = 0; t < NT8; ++t) b[t] = lds128(ra + aoff[c] + t * 8 * 128);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
             for (int T = 0; T < TW; ++T) {
-              const uint32_t a0 = code_pair(wv[u][T][0][i], 2 * hh, z2[T][0]);
-              const uint32_t a1 = code_pair(wv[u][T][1][i], 2 * hh, z2[T][1]);
-              const uint32_t a2 = code_pair(wv[u][T][0][i], 2 * hh + 1, z2[T][0]);
-              const uint32_t a3 = code_pair(wv[u][T][1][i], 2 * hh + 1, z2[T][1]);
+              const uint32_t a0 = code_pair(w[T][0][c], 2 * hh, z2[T][0]);
+              const uint32_t a1 = code_pair(w[T][1][c], 2 * hh, z2[T][1]);
+              const uint32_t a2 = code_pair(w[T][0][c], 2 * hh + 1, z2[T][0]);
+              const uint32_t a3 = code_pair(w[T][1][c], 2 * hh + 1, z2[T][1]);
 #pragma unroll
               for (int t = 0; t < NT8; ++t)
                 mma_16816(d[T][t], a0, a1, a2, a3, hh ? b[t].z : b[t].x, hh ? b[t].w : b[t].y);
@@ -307,19 +310,15 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
           }
         }
 #pragma unroll
-        for (int T = 0; T < TW; ++T) {
-          const float s0 = __half2float(__ushort_as_half((unsigned short)sc[u][T][0]));
-          const float s1 = __half2float(__ushort_as_half((unsigned short)sc[u][T][1]));
+        for (int T = 0; T < TW; ++T)
 #pragma unroll
           for (int t = 0; t < NT8; ++t) {
-            acc[T][t][0] = fmaf(s0, d[T][t][0], acc[T][t][0]);
-            acc[T][t][1] = fmaf(s0, d[T][t][1], acc[T][t][1]);
-            acc[T][t][2] = fmaf(s1, d[T][t][2], acc[T][t][2]);
-            acc[T][t][3] = fmaf(s1, d[T][t][3], acc[T][t][3]);
+            acc[T][t][0] = fmaf(s[T][0], d[T][t][0], acc[T][t][0]);
+            acc[T][t][1] = fmaf(s[T][0], d[T][t][1], acc[T][t][1]);
+            acc[T][t][2] = fmaf(s[T][1], d[T][t][2], acc[T][t][2]);
+            acc[T][t][3] = fmaf(s[T][1], d[T][t][3], acc[T][t][3]);
           }
-        }
       }
-      load_rec(u, r + P);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[j % D]);
@@ -330,7 +329,7 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
     for (int x = issued > D ? issued - D : 0; x < issued; ++x) hq_wait(&full[x % D], (x / D) & 1, p.wait_ns, nullptr);
   }
 
-  // ---- output: feature tile * 128 + row, token 8t + 2 qd + e
+  // ---- output: feature tile * 128 + row, token 8t + sigma(2 qd + (e & 1))
   auto store = [&](float (&v)[TW][NT8][4]) {
 #pragma unroll
     for (int T = 0; T < TW; ++T)
@@ -339,7 +338,7 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int f = tile * kTileN + row[T][e >> 1];
-          const int tok = 8 * t + 2 * qd + (e & 1);
+          const int tok = 8 * t + col_token(2 * qd + (e & 1));
           if (f < p.n && tok < p.m) p.c[(size_t)tok * p.n + f] = __float2bfloat16_rn(v[T][t][e]);
         }
   };
@@ -347,8 +346,6 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
     store(acc);
     return;
   }
-  // K split over p.splits CTAs: fp32 partial tile, the last CTA of the tile
-  // sums the partials in slice order
   float4* mine = reinterpret_cast<float4*>(p.partials) + (size_t)blockIdx.x * C::kNv4 * C::kThreads + threadIdx.x;
 #pragma unroll
   for (int T = 0; T < TW; ++T)
@@ -391,16 +388,16 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
 template <int NT8, bool HASZ, int TWT>
 hq_status reg_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cudaStream_t stream) {
   auto kern = w4a16_reg_kernel<NT8, HASZ, TWT>;
-  const size_t smem = RegCfg<NT8, TWT>::kSmem;
+  using C = RegCfg<NT8, TWT>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess)
       return HQ_ERR_CUDA;
     attr_set[dev] = true;
   }
-  return launch_pdl(kern, dim3(grid), dim3(RegCfg<NT8, TWT>::kThreads), smem, stream, map, p) == cudaSuccess
+  return launch_pdl(kern, dim3(grid), dim3(C::kThreads), (size_t)C::kSmem, stream, map, p) == cudaSuccess
              ? HQ_OK
              : HQ_ERR_CUDA;
 }
@@ -410,25 +407,17 @@ hq_status reg_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cud
 
 using w4::RegParams;
 
-// CTAs per weight tile (K slices) of the register-path plan: the split that
-// fills the SMs best in one wave of reg_ctas_per_sm(2) CTAs per SM (a tie
-// goes to more CTAs: more bytes in flight).
-int reg_splits(int num_sms, const hq_quant_desc& d) {
+// CTAs per weight tile (K slices) of the register-path plan: the largest
+// split whose grid fits reg_slots_per_sm CTAs per SM (more CTAs, more bytes in
+// flight; one record per CTA at least).  Measured on B200 (back to back,
+// per launch): K=18432 N=7168 M=1 at 4..10 slices 31.9 / 26.8 / 24.8 / 22.9
+// / 26.6 / 25.5 us (7 best: 392 CTAs); M=16 41.1 .. 26.0 (10 best: 560 CTAs);
+// K=7168 N=18432 M=1 26.0 / 20.8 / 24.5 at 2 / 3 / 4, M=16 32.4 / 29.5 / 24.8.
+int reg_splits(int num_sms, const hq_quant_desc& d, int m) {
   const long long tiles = (d.n + kTileN - 1) / kTileN;
   const long long kbs = d.k / kBlockK;
-  const long long slots = (long long)num_sms * reg_ctas_per_sm(2);
-  int best = 1;
-  double best_eff = -1.0;
-  for (long long s = 1; s <= kbs && tiles * s <= slots; ++s) {
-    const long long units = tiles * s;
-    const long long waves = (units + num_sms - 1) / num_sms;
-    const double eff = (double)units / (double)(waves * num_sms);
-    if (eff >= best_eff - 1e-9) {
-      best_eff = eff;
-      best = (int)s;
-    }
-  }
-  return best;
+  const long long slots = (long long)num_sms * reg_slots_per_sm(m <= 8 ? 1 : 2);
+  return (int)std::max<long long>(1, std::min<long long>(kbs, slots / tiles));
 }
 
 size_t reg_workspace_bytes(const W4Config& cfg) {
@@ -472,7 +461,7 @@ hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pa
   if (cr != CUDA_SUCCESS) return HQ_ERR_CUDA;
   const bool hz = d.has_zero_point != 0;
   // grids of fewer CTAs than SMs: eight warps of 16 rows per CTA (more warps
-  // on each busy SM); else four warps of 32 rows at four CTAs per SM
+  // on each busy SM); else four warps of 32 rows
   if (cfg.reg_tw == 1) {
     if (nt8 == 1)
       return hz ? w4::reg_launch_t<1, true, 1>(map, p, cfg.grid, stream) : w4::reg_launch_t<1, false, 1>(map, p, cfg.grid, stream);

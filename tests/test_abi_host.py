@@ -444,15 +444,20 @@ def test_split_plans_fit_the_workspace_counter_region():
     every scratch area starts past the region."""
     header, region = 256, 256 << 10
     d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
-    t = hq.Tuning(tile_m=16, split_k=2)
+    t = hq.Tuning(tile_m=16, split_k=2, variant=2)
     p = hq.hq_plan_describe(d, 16, t)
     assert p.split == 2 and p.workspace_bytes == header + region + p.grid * 2 * 16 * 128 * 4
+    # the register path (M <= 16): one 8 KiB fp32 partial tile per CTA
+    pr = hq.hq_plan_describe(d, 16, hq.Tuning(split_k=2, variant=3))
+    assert (pr.kernel, pr.split, pr.grid) == (4, 2, 2 * 144)
+    assert pr.workspace_bytes == header + region + pr.grid * 8192
     assert hq.hq_plan_describe(d, 16 * 113, t).split == 2          # 16272 tiles
     big = hq.hq_plan_describe(d, 16 * 114, t)                      # 16416 tiles
     assert (big.split, big.workspace_bytes) == (0, header)
     dm = hq.hq_quant_desc_init(hq.HQ_FMT_MXFP4, 18432, 7168, 32, 0, 1)
-    assert hq.hq_plan_describe(dm, 16 * 56, t).split == 2          # 8064 tiles
-    assert hq.hq_plan_describe(dm, 16 * 57, t).split == 0          # 8208 tiles
+    tb = hq.Tuning(tile_m=16, split_k=2)
+    assert hq.hq_plan_describe(dm, 16 * 56, tb).split == 2         # 8064 tiles
+    assert hq.hq_plan_describe(dm, 16 * 57, tb).split == 0         # 8208 tiles
     dn = hq.hq_quant_desc_init(hq.HQ_FMT_NVFP4, 8192, 8192, 16, 0, 1)
     pn = hq.hq_plan_describe(dn, 8192)
     assert pn.split == 0 and pn.workspace_bytes > header + region  # re-laid scales past the region
@@ -483,7 +488,7 @@ def test_tuning_table_entry_changes_the_plan():
     table restores the rules.  The workspace size follows the plan."""
     d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, 18432, 7168, 128, 0, 1)
     base16 = hq.hq_plan_describe(d, 16)
-    assert (base16.tile_m, base16.kernel, base16.from_table) == (16, 2, 0)
+    assert (base16.tile_m, base16.kernel, base16.from_table) == (16, 4, 0)      # the register path
     assert base16.stages == base16.ring_stages >= 2
     base64 = hq.hq_plan_describe(d, 64)
     entry = {"fmt": hq.HQ_FMT_INT4, "n": 18432, "k": 7168, "num_experts": 1, "m_min": 1, "m_max": 32,
