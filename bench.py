@@ -63,23 +63,23 @@ def load_peaks():
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
 # capture is taken again.
-TRAFFIC_COMMIT = "806db2d"
-TRAFFIC_SOURCES = "87fec370729d9ca9"
+TRAFFIC_COMMIT = "0f71beb"
+TRAFFIC_SOURCES = "0550bd8b50abcf58"
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 68844032,
-    (4, 7168, 18432): 68222720,
-    (16, 7168, 18432): 69713920,
-    (64, 7168, 18432): 71245312,
-    (256, 7168, 18432): 75831808,
-    (1024, 7168, 18432): 149061120,
-    (4096, 7168, 18432): 355084288,
-    (1, 18432, 7168): 68239104,
-    (4, 18432, 7168): 68381440,
-    (16, 18432, 7168): 68766208,
-    (64, 18432, 7168): 74174720,
-    (256, 18432, 7168): 86867712,
-    (1024, 18432, 7168): 197565952,
-    (4096, 18432, 7168): 713222912,
+    (1, 7168, 18432): 68518400,
+    (4, 7168, 18432): 68257280,
+    (16, 7168, 18432): 68399104,
+    (64, 7168, 18432): 71279360,
+    (256, 7168, 18432): 75675648,
+    (1024, 7168, 18432): 152192512,
+    (4096, 7168, 18432): 404947712,
+    (1, 18432, 7168): 68235520,
+    (4, 18432, 7168): 68338944,
+    (16, 18432, 7168): 68763136,
+    (64, 18432, 7168): 73953792,
+    (256, 18432, 7168): 86066944,
+    (1024, 18432, 7168): 203194880,
+    (4096, 18432, 7168): 715784960,
 }
 
 
