@@ -196,7 +196,7 @@ hq_status hq_tuning_table_set(const hq_tuning_entry* entries, int32_t count);
 typedef struct {
   int32_t kernel;      /* 1: W4A16 weights rescaled to bf16, 2: W4A16 exact weights, 3: block-scaled,
                           4: W4A16 register path (exact weights in mma.sync fragments)              */
-  int32_t tile_m;      /* token tile                                                                 */
+  int32_t tile_m;      /* token tile (the register path: 8 or 16, one or two 8-token MMA tiles)       */
   int32_t grid;        /* CTAs                                                                       */
   int32_t split;       /* 0: whole tiles; >0: tiles share their K range (stream-K or a K split)      */
   int32_t whole_tiles; /* dense W4A16 split plans: tiles run whole before the shared tail            */

@@ -115,7 +115,7 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
 // variant 3): CTAs per SM a plan fills (slots) for 8- or 16-token tiles, the
 // K slices per weight tile, its workspace and its launch.
 constexpr int reg_slots_per_sm(int nt8) { return nt8 == 1 ? 3 : 4; }
-constexpr int kRegRing = 3;          // stages of the 8-token kernel's ring (the 16-token kernel: 4)
+constexpr int kRegRing8 = 3, kRegRing16 = 4;   // stages of the 8- and 16-token kernels' rings
 int reg_splits(int num_sms, const hq_quant_desc& d, int m);
 size_t reg_workspace_bytes(const W4Config& cfg);
 hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m, void* c,

@@ -873,7 +873,7 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
   if (use_reg) {
     const long long tiles = (d.n + kTileN - 1) / kTileN;
     cfg.variant = 3;
-    cfg.ntok = 16;
+    cfg.ntok = m <= 8 ? 8 : 16;   // one or two 8-token MMA tiles
     cfg.dp_tiles = 0;
     cfg.splits = (t && t->split_k > 0) ? (int)std::min<long long>(t->split_k, d.k / kBlockK)
                                        : reg_splits(dev.num_sms, d, m);
@@ -1006,7 +1006,7 @@ int rescaled_depth(int ntok, int cta_group) {
 }  // namespace
 
 int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg) {
-  if (cfg.variant == 3) return kRegRing;   // the register path's ring of whole-record stages (8-token tiles)
+  if (cfg.variant == 3) return cfg.ntok == 8 ? kRegRing8 : kRegRing16;   // the register path's ring of whole-record stages
   const bool mx = d.fmt == HQ_FMT_MXFP4_A16, mxi4 = d.fmt == HQ_FMT_MXINT4;
   const int kfmt = d.fmt == HQ_FMT_INT3 ? kFmtInt3 : d.fmt == HQ_FMT_INT2 ? kFmtInt2 : d.fmt == HQ_FMT_INT8 ? kFmtInt8 : kFmtInt4;
   if (!mx && !mxi4 && cfg.ntok <= 64 && cfg.variant != 1) return small_ring_depth(cfg.ntok, kfmt);

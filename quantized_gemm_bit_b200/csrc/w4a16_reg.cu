@@ -113,7 +113,7 @@ struct RegCfg {
   static constexpr int kWarps = 8 / kTw;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kP = NT8 == 2 ? 1 : 2;          // records per stage
-  static constexpr int kD = NT8 == 2 ? 4 : 3;          // stages
+  static constexpr int kD = NT8 == 2 ? kRegRing16 : kRegRing8;   // stages
   static constexpr int kRows = 8 * NT8;
   static constexpr int kBox = kRows * 128;
   static constexpr int kRecA = 2 * kBox;
