@@ -517,7 +517,7 @@ hq_status hq_plan_describe(const hq_quant_desc* d, int32_t m, const hq_tuning* t
     const bool mx = d->fmt == HQ_FMT_MXFP4_A16 || d->fmt == HQ_FMT_MXINT4;
     p.tile_m = cfg.ntok;
     p.grid = cfg.grid;
-    const bool reg = !grouped && cfg.variant == 3;
+    const bool reg = cfg.variant == 3;
     p.split = grouped ? 0 : cfg.splits == 0 || (reg && cfg.splits == 1) ? 0 : cfg.splits;
     p.whole_tiles = grouped ? 0 : cfg.dp_tiles;
     p.kernel = reg ? 4 : (!mx && cfg.ntok <= 64 && cfg.variant != 1) ? 2 : 1;

@@ -116,10 +116,18 @@ hq_status bs_launch(const hq_quant_desc& d, const BsConfig& cfg, const void* pac
 // K slices per weight tile, its workspace and its launch.
 constexpr int reg_slots_per_sm(int nt8) { return nt8 == 1 ? 3 : 4; }
 constexpr int kRegRing8 = 3, kRegRing16 = 4;   // stages of the 8- and 16-token kernels' rings
+constexpr bool kRegGroupedDefault = true;       // grouped MoE: the library's choice at <= 8 tokens per expert
 int reg_splits(int num_sms, const hq_quant_desc& d, int m);
 size_t reg_workspace_bytes(const W4Config& cfg);
 hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a, int m, void* c,
                      void* ws, cudaStream_t stream);
+// Grouped MoE on the register path: persistent CTAs (reg_grouped_ctas_per_sm
+// per SM) over 8- or 16-token units (cfg.ntok); swiglu: gated gate+up
+// weights, h written.
+constexpr int reg_grouped_ctas_per_sm(int nt8) { return nt8 == 1 ? 3 : 2; }
+hq_status reg_launch_grouped(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a,
+                             int total_rows, void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream,
+                             int swiglu);
 
 // Ring depth (SMEM pipeline stages) of the kernel a plan launches.
 int w4_ring_depth(const hq_quant_desc& d, const W4Config& cfg);

@@ -868,7 +868,7 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
   // 24.8, against 24.5 and 25.0 for the exact-weight kernel; K=18432 N=7168
   // M <= 8 22.9, M=16 26.0, against 30.2 and 32.7.
   const bool reg_fits = !grouped && d.fmt == HQ_FMT_INT4 && m <= 16 && ntok <= 16 && !(t && t->cta_group == 2);
-  if (cfg.variant == 3 && !reg_fits) cfg.variant = 0;
+  if (cfg.variant == 3 && !reg_fits && !grouped) cfg.variant = 0;
   const bool use_reg = reg_fits && (cfg.variant == 0 || cfg.variant == 3);
   if (use_reg) {
     const long long tiles = (d.n + kTileN - 1) / kTileN;
@@ -886,6 +886,26 @@ W4Config w4_plan_rules(const DeviceInfo& dev, const hq_quant_desc& d, int m, boo
     return cfg;
   }
   if (grouped) {
+    // The register path for INT4 experts of a few tokens each, on request
+    // (variant 3) or by default when a typical expert's rows fit 8 tokens:
+    // 8- or 16-token units over the whole K range on persistent CTAs.
+    // Measured on B200 (256 experts, top-8, hidden 7168, intermediate 2048):
+    // T=64 gate+up 778 us and down 419 against 868 and 452 for the
+    // exact-weight grouped kernel; T=1024 (32 rows per expert) three times
+    // slower, so only the few-token case takes it.
+    const double avg = (double)m / std::max(1, d.num_experts);
+    const double want = avg + 2.0 * std::sqrt(avg);
+    const bool reg_ok = d.fmt == HQ_FMT_INT4 && d.num_experts <= kMaxExperts && !(t && t->cta_group == 2) &&
+                        !(t && t->tile_m && t->tile_m != 8 && t->tile_m != 16);
+    if (reg_ok && (cfg.variant == 3 || (cfg.variant == 0 && kRegGroupedDefault && want <= 8.0))) {
+      cfg.variant = 3;
+      cfg.ntok = (t && t->tile_m) ? t->tile_m : want <= 8.0 ? 8 : 16;
+      cfg.splits = 0;
+      cfg.grid = dev.num_sms * reg_grouped_ctas_per_sm(cfg.ntok / 8);
+      cfg.reg_tw = 2;
+      return cfg;
+    }
+    if (cfg.variant == 3) cfg.variant = 0;
     cfg.ntok = ntok;
     cfg.grid = dev.num_sms;
     return cfg;
@@ -1049,6 +1069,7 @@ hq_status w4_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pac
                     void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream, int swiglu) {
   const bool grouped = expert_offsets != nullptr;
   if (!grouped && cfg.variant == 3) return reg_launch(d, cfg, packed, a, m, c, ws, stream);
+  if (grouped && cfg.variant == 3) return reg_launch_grouped(d, cfg, packed, a, m, c, expert_offsets, ws, stream, swiglu);
   W4Params p{};
   p.packed = static_cast<const uint8_t*>(packed);
   p.c = static_cast<__nv_bfloat16*>(c);

@@ -61,8 +61,20 @@ struct RegParams {
   int m, n;
   int k_blocks;
   int rec_bytes;
-  int splits;              // CTAs per weight tile (K slices)
+  int splits;              // CTAs per weight tile (K slices); grouped: 1
   int early_weights;       // load the first records' codes before the previous kernel has completed
+  // grouped MoE: experts back to back in the blob, rows of A / C sorted by expert
+  const int32_t* expert_offsets;
+  uint64_t expert_bytes;
+  int num_experts;
+  int n_tiles;
+};
+
+// One grouped unit: weight tile nt of one expert over the whole K range, for
+// token rows [row0, row0 + rows) of A.
+struct RegUnit {
+  const uint8_t* rec0;
+  int row0, rows, nt;
 };
 
 __device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
@@ -133,6 +145,68 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "r"(addr));
 }
 __device__ __forceinline__ int col_token(int n) { return (n >> 1) | ((n & 1) << 2); }
+
+// One 128-K record of a warp's rows: codes (ldmatrix from the record at
+// `wrec`), scales and zero points from shared memory, activations from the
+// record's boxes at `ra`; the group's fp32 sum scaled into acc.
+template <int NT8, bool HASZ, int TW>
+__device__ __forceinline__ void reg_record(uint32_t wrec, uint32_t ra, uint32_t lds_row, const uint32_t (&aoff)[4],
+                                           const int (&row)[TW][2], float (&acc)[TW][NT8][4]) {
+  uint32_t w[TW][2][4];   // word qd of chunk c of row (T, h)
+  if (TW == 2) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) ldsm_x4(wrec + lds_row + c * 2048, w[0][0][c], w[0][1][c], w[TW - 1][0][c], w[TW - 1][1][c]);
+  } else {
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc)
+      ldsm_x4(wrec + lds_row + cc * 4096, w[0][0][2 * cc], w[0][1][2 * cc], w[0][0][2 * cc + 1], w[0][1][2 * cc + 1]);
+  }
+  uint32_t z2[TW][2];
+  float s[TW][2];
+#pragma unroll
+  for (int T = 0; T < TW; ++T)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      s[T][h] = __half2float(__ushort_as_half((unsigned short)lds_u16(wrec + kW4RecCodes + 2 * row[T][h])));
+      const uint32_t z = HASZ ? lds_u8(wrec + kW4RecCodes + 256 + row[T][h]) : 8u;
+      z2[T][h] = 0x43004300u | z | (z << 16);
+    }
+  float d[TW][NT8][4];
+#pragma unroll
+  for (int T = 0; T < TW; ++T)
+#pragma unroll
+    for (int t = 0; t < NT8; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[T][t][e] = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 b[NT8];
+#pragma unroll
+    for (int t = 0; t < NT8; ++t) b[t] = lds128(ra + aoff[c] + t * 8 * 128);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+      for (int T = 0; T < TW; ++T) {
+        const uint32_t a0 = code_pair(w[T][0][c], 2 * hh, z2[T][0]);
+        const uint32_t a1 = code_pair(w[T][1][c], 2 * hh, z2[T][1]);
+        const uint32_t a2 = code_pair(w[T][0][c], 2 * hh + 1, z2[T][0]);
+        const uint32_t a3 = code_pair(w[T][1][c], 2 * hh + 1, z2[T][1]);
+#pragma unroll
+        for (int t = 0; t < NT8; ++t)
+          mma_16816(d[T][t], a0, a1, a2, a3, hh ? b[t].z : b[t].x, hh ? b[t].w : b[t].y);
+      }
+    }
+  }
+#pragma unroll
+  for (int T = 0; T < TW; ++T)
+#pragma unroll
+    for (int t = 0; t < NT8; ++t) {
+      acc[T][t][0] = fmaf(s[T][0], d[T][t][0], acc[T][t][0]);
+      acc[T][t][1] = fmaf(s[T][0], d[T][t][1], acc[T][t][1]);
+      acc[T][t][2] = fmaf(s[T][1], d[T][t][2], acc[T][t][2]);
+      acc[T][t][3] = fmaf(s[T][1], d[T][t][3], acc[T][t][3]);
+    }
+}
 
 template <int NT8, bool HASZ, int TWT>
 __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::kCtasPerSm)
@@ -261,64 +335,9 @@ __global__ void __launch_bounds__(RegCfg<NT8, TWT>::kThreads, RegCfg<NT8, TWT>::
 #pragma unroll
     for (int u = 0; u < P; ++u) {
       const int r = j * P + u;
-      if (r < nrec) {
-        const uint32_t wrec = st + (uint32_t)(u * p.rec_bytes);
-        uint32_t w[TW][2][4];   // word qd of chunk c of row (T, h)
-        if (TW == 2) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) ldsm_x4(wrec + lds_row + c * 2048, w[0][0][c], w[0][1][c], w[TW - 1][0][c], w[TW - 1][1][c]);
-        } else {
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-            ldsm_x4(wrec + lds_row + cc * 4096, w[0][0][2 * cc], w[0][1][2 * cc], w[0][0][2 * cc + 1], w[0][1][2 * cc + 1]);
-        }
-        uint32_t z2[TW][2];
-        float s[TW][2];
-#pragma unroll
-        for (int T = 0; T < TW; ++T)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            s[T][h] = __half2float(__ushort_as_half((unsigned short)lds_u16(wrec + kW4RecCodes + 2 * row[T][h])));
-            const uint32_t z = HASZ ? lds_u8(wrec + kW4RecCodes + 256 + row[T][h]) : 8u;
-            z2[T][h] = 0x43004300u | z | (z << 16);
-          }
-        float d[TW][NT8][4];
-#pragma unroll
-        for (int T = 0; T < TW; ++T)
-#pragma unroll
-          for (int t = 0; t < NT8; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) d[T][t][e] = 0.f;
-        const uint32_t ra = st + (uint32_t)(C::kWBytes + u * C::kRecA);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint4 b[NT8];
-#pragma unroll
-          for (int t = 0; t < NT8; ++t) b[t] = lds128(ra + aoff[c] + t * 8 * 128);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-            for (int T = 0; T < TW; ++T) {
-              const uint32_t a0 = code_pair(w[T][0][c], 2 * hh, z2[T][0]);
-              const uint32_t a1 = code_pair(w[T][1][c], 2 * hh, z2[T][1]);
-              const uint32_t a2 = code_pair(w[T][0][c], 2 * hh + 1, z2[T][0]);
-              const uint32_t a3 = code_pair(w[T][1][c], 2 * hh + 1, z2[T][1]);
-#pragma unroll
-              for (int t = 0; t < NT8; ++t)
-                mma_16816(d[T][t], a0, a1, a2, a3, hh ? b[t].z : b[t].x, hh ? b[t].w : b[t].y);
-            }
-          }
-        }
-#pragma unroll
-        for (int T = 0; T < TW; ++T)
-#pragma unroll
-          for (int t = 0; t < NT8; ++t) {
-            acc[T][t][0] = fmaf(s[T][0], d[T][t][0], acc[T][t][0]);
-            acc[T][t][1] = fmaf(s[T][0], d[T][t][1], acc[T][t][1]);
-            acc[T][t][2] = fmaf(s[T][1], d[T][t][2], acc[T][t][2]);
-            acc[T][t][3] = fmaf(s[T][1], d[T][t][3], acc[T][t][3]);
-          }
-      }
+      if (r < nrec)
+        reg_record<NT8, HASZ, TW>(st + (uint32_t)(u * p.rec_bytes), st + (uint32_t)(C::kWBytes + u * C::kRecA),
+                                  lds_row, aoff, row, acc);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[j % D]);
@@ -402,6 +421,231 @@ hq_status reg_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cud
              : HQ_ERR_CUDA;
 }
 
+// Grouped MoE on the register path: persistent CTAs walk (expert, weight
+// tile, 8*NT8-token tile) units built on the device from the expert row
+// offsets, each over the whole K range (four warps of 32 rows).  One thread
+// streams the units' stages through the ring without a gap between units;
+// the warps finish a unit with its stores.  SW: weights in the gated gate+up
+// row order, whose 32-row groups put a warp's 16 gate rows in its MMA tile 0
+// and the matching up rows in tile 1, so each thread writes
+// h = silu(gate) * up for its features directly.
+template <int NT8>
+struct RegGrpCfg {
+  using C = RegCfg<NT8, 2>;
+  static constexpr int kTabOff = C::kBarOff + 128;
+  static constexpr int kSmem = kTabOff + 2 * (kMaxExperts + 1) * 4 + 1024;
+  static constexpr int kCtasPerSm = reg_grouped_ctas_per_sm(NT8);
+  static_assert(kCtasPerSm * (kSmem + 1024) <= 228 * 1024, "kCtasPerSm CTAs fit one SM's shared memory");
+};
+
+template <int NT8, bool HASZ, bool SW>
+__global__ void __launch_bounds__(128, RegGrpCfg<NT8>::kCtasPerSm)
+    w4a16_reg_grouped_kernel(const __grid_constant__ CUtensorMap tmap_a, const RegParams p) {
+  using C = RegCfg<NT8, 2>;
+  using G = RegGrpCfg<NT8>;
+  constexpr int P = C::kP;
+  constexpr int D = C::kD;
+  constexpr int TW = 2;
+  constexpr int NTOK = 8 * NT8;
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + D;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(empty + D);
+  int* s_total = const_cast<int*>(s_abort + 1);
+  int* s_off = reinterpret_cast<int*>(smem + G::kTabOff);   // [num_experts + 1]
+  int* s_prefix = s_off + (kMaxExperts + 1);                 // [num_experts + 1]
+
+  const int warp = (int)(threadIdx.x >> 5), lane = (int)(threadIdx.x & 31);
+  const int g = lane >> 2, qd = lane & 3;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < D; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], C::kWarps);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+    pdl_launch_dependents();
+    prefetch_tensormap(&tmap_a);
+  }
+  pdl_wait();   // the expert offsets, activations and outputs may be in use until here
+  const int E = p.num_experts;
+  for (int i = (int)threadIdx.x; i <= E; i += (int)blockDim.x) s_off[i] = p.expert_offsets[i];
+  __syncthreads();   // barriers initialised, offsets loaded
+  if (threadIdx.x == 0) {
+    int total = 0;
+    bool bad = s_off[0] != 0 || s_off[E] != p.m;
+    for (int e = 0; e < E; ++e) {
+      s_prefix[e] = total;
+      int rows = s_off[e + 1] - s_off[e];
+      if (rows < 0) { bad = true; rows = 0; }
+      total += ((rows + NTOK - 1) / NTOK) * p.n_tiles;
+    }
+    s_prefix[E] = total;
+    if (bad) {
+      atomicCAS(p.err, 0u, (uint32_t)HQ_ERR_DEVICE_BAD_OFFSETS);
+      total = 0;
+    }
+    *s_total = total;
+  }
+  __syncthreads();
+
+  auto get_unit = [&](int idx, RegUnit& x) -> bool {
+    const int u = (int)blockIdx.x + idx * (int)gridDim.x;
+    if (u >= *s_total) return false;
+    // the expert e with prefix[e] <= u < prefix[e + 1] (empty experts share
+    // their prefix with the next one, so the largest such e has rows)
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_prefix[mid] <= u) lo = mid; else hi = mid;
+    }
+    const int rows_e = s_off[lo + 1] - s_off[lo];
+    const int mtiles = (rows_e + NTOK - 1) / NTOK;
+    const int local = u - s_prefix[lo];
+    const int mt = local % mtiles;
+    x.nt = local / mtiles;
+    x.rec0 = p.packed + (size_t)lo * p.expert_bytes + (size_t)x.nt * p.k_blocks * (size_t)p.rec_bytes;
+    x.row0 = s_off[lo] + mt * NTOK;
+    x.rows = min(NTOK, s_off[lo + 1] - x.row0);
+    return true;
+  };
+  const int nrec = p.k_blocks;
+  const int nstage = (nrec + P - 1) / P;
+
+  // ---- producer state (thread 0): the next stage to issue
+  const uint64_t pol_w = policy_evict_first();
+  RegUnit pu{};
+  int pidx = 0, psj = 0;
+  bool pmore = false;
+  int issued = 0;
+  auto issue_next = [&](int X) {   // stage psj of unit pu into ring stage X
+    const int r0 = psj * P, nr = min(P, nrec - r0);
+    uint64_t* fb = &full[X % D];
+    uint8_t* dst = smem + (X % D) * C::kStage;
+    mbar_arrive_expect_tx(fb, (uint32_t)(nr * (p.rec_bytes + C::kRecA)));
+    bulk_g2s(dst, pu.rec0 + (size_t)r0 * p.rec_bytes, (uint32_t)(nr * p.rec_bytes), fb, pol_w);
+    for (int u = 0; u < nr; ++u) {
+      const int kx = (r0 + u) * kBlockK;
+      tma_load_2d(dst + C::kWBytes + u * C::kRecA, &tmap_a, kx, pu.row0, fb);
+      tma_load_2d(dst + C::kWBytes + u * C::kRecA + C::kBox, &tmap_a, kx + 64, pu.row0, fb);
+    }
+    if (++psj == nstage) {
+      psj = 0;
+      pmore = get_unit(++pidx, pu);
+    }
+  };
+  if (threadIdx.x == 0) {
+    pmore = get_unit(0, pu);
+    while (issued < D && pmore) issue_next(issued++);
+  }
+
+  int row[TW][2];
+#pragma unroll
+  for (int T = 0; T < TW; ++T)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) row[T][h] = 32 * warp + 16 * T + 8 * h + g;
+  const int mk = lane >> 3, mi = lane & 7;
+  const uint32_t lds_row = (uint32_t)((32 * warp + 16 * (mk >> 1) + 8 * (mk & 1) + mi) * 16);
+  const int tg = col_token(g);
+  uint32_t aoff[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    aoff[c] = (uint32_t)((c >> 1) * C::kBox + tg * 128 + (((4 * (c & 1) + qd) ^ tg) << 4));
+  const uint32_t sbase = smem_u32(smem);
+
+  float acc[TW][NT8][4];
+  auto zero = [&]() {
+#pragma unroll
+    for (int T = 0; T < TW; ++T)
+#pragma unroll
+      for (int t = 0; t < NT8; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[T][t][e] = 0.f;
+  };
+  zero();
+  RegUnit cu{};
+  int cidx = 0, csj = 0;
+  bool cmore = get_unit(0, cu);
+  bool ok = true;
+  for (int X = 0; cmore; ++X) {
+    // ring stage X + D - 1 reuses the slot of stage X - 1
+    if (warp == 0 && X >= 1) {
+      const bool more = __shfl_sync(0xffffffffu, (lane == 0 && pmore && issued == X + D - 1) ? 1 : 0, 0) != 0;
+      if (more) {
+        if (!hq_wait_warp(&empty[(X - 1) % D], ((X - 1) / D) & 1, p.wait_ns, s_abort)) {
+          if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+          ok = false;
+          break;
+        }
+        if (lane == 0) issue_next(issued++);
+        __syncwarp();
+      }
+    }
+    if (!hq_wait_warp(&full[X % D], (X / D) & 1, p.wait_ns, s_abort)) {
+      if (lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const uint32_t st = sbase + (uint32_t)((X % D) * C::kStage);
+#pragma unroll
+    for (int u = 0; u < P; ++u) {
+      if (csj * P + u < nrec)
+        reg_record<NT8, HASZ, TW>(st + (uint32_t)(u * p.rec_bytes), st + (uint32_t)(C::kWBytes + u * C::kRecA),
+                                  lds_row, aoff, row, acc);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[X % D]);
+    if (++csj < nstage) continue;
+    // ---- the unit's output: token row0 + 8t + sigma(2 qd + (e & 1))
+#pragma unroll
+    for (int t = 0; t < NT8; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = 8 * t + col_token(2 * qd + (e & 1));
+        if (tok >= cu.rows) continue;
+        const size_t r = (size_t)(cu.row0 + tok);
+        if constexpr (SW) {
+          const int hc = p.n >> 1;
+          const int f = cu.nt * (kTileN / 2) + 16 * warp + 8 * (e >> 1) + g;
+          const float gv = acc[0][t][e], uv = acc[1][t][e];
+          if (f < hc) p.c[r * hc + f] = __float2bfloat16_rn(__fdividef(gv, 1.f + __expf(-gv)) * uv);
+        } else {
+#pragma unroll
+          for (int T = 0; T < TW; ++T) {
+            const int f = cu.nt * kTileN + row[T][e >> 1];
+            if (f < p.n) p.c[r * p.n + f] = __float2bfloat16_rn(acc[T][t][e]);
+          }
+        }
+      }
+    zero();
+    csj = 0;
+    cmore = get_unit(++cidx, cu);
+  }
+  if (!ok && lane == 0) raise_error(p.err, s_abort, HQ_ERR_DEVICE_TIMEOUT);
+  if (warp == 0 && lane == 0 && *s_abort) {
+    // let every copy already issued land before the CTA exits
+    for (int X = issued > D ? issued - D : 0; X < issued; ++X) hq_wait(&full[X % D], (X / D) & 1, p.wait_ns, nullptr);
+  }
+}
+
+template <int NT8, bool HASZ, bool SW>
+hq_status reg_grouped_launch_t(const CUtensorMap& map, const RegParams& p, int grid, cudaStream_t stream) {
+  auto kern = w4a16_reg_grouped_kernel<NT8, HASZ, SW>;
+  using G = RegGrpCfg<NT8>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem) != cudaSuccess)
+      return HQ_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  return launch_pdl(kern, dim3(grid), dim3(128), (size_t)G::kSmem, stream, map, p) == cudaSuccess ? HQ_OK
+                                                                                                  : HQ_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace w4
 
@@ -470,6 +714,49 @@ hq_status reg_launch(const hq_quant_desc& d, const W4Config& cfg, const void* pa
   if (nt8 == 1)
     return hz ? w4::reg_launch_t<1, true, 2>(map, p, cfg.grid, stream) : w4::reg_launch_t<1, false, 2>(map, p, cfg.grid, stream);
   return hz ? w4::reg_launch_t<2, true, 2>(map, p, cfg.grid, stream) : w4::reg_launch_t<2, false, 2>(map, p, cfg.grid, stream);
+}
+
+hq_status reg_launch_grouped(const hq_quant_desc& d, const W4Config& cfg, const void* packed, const void* a,
+                             int total_rows, void* c, const int32_t* expert_offsets, void* ws, cudaStream_t stream,
+                             int swiglu) {
+  if (d.fmt != HQ_FMT_INT4 || d.num_experts < 2 || d.num_experts > w4::kMaxExperts || total_rows < 1)
+    return HQ_ERR_UNSUPPORTED;
+  if (cfg.ntok != 8 && cfg.ntok != 16) return HQ_ERR_INVALID_ARG;
+  RegParams p{};
+  p.packed = static_cast<const uint8_t*>(packed);
+  p.c = static_cast<__nv_bfloat16*>(c);
+  p.err = static_cast<uint32_t*>(ws);
+  p.wait_ns = kDefaultWaitNs;
+  p.m = total_rows;
+  p.n = d.n;
+  p.k_blocks = d.k / kBlockK;
+  p.rec_bytes = w4_record_bytes(d.has_zero_point != 0);
+  p.splits = 1;
+  p.expert_offsets = expert_offsets;
+  p.n_tiles = (d.n + kTileN - 1) / kTileN;
+  p.expert_bytes = (uint64_t)p.n_tiles * p.k_blocks * p.rec_bytes;
+  p.num_experts = d.num_experts;
+  CUtensorMap map;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return HQ_ERR_CUDA;
+  cuuint64_t dims[2] = {(cuuint64_t)d.k, (cuuint64_t)total_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d.k * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)cfg.ntok};
+  cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return HQ_ERR_CUDA;
+  const bool hz = d.has_zero_point != 0;
+  const int grid = cfg.grid;
+  if (cfg.ntok == 8) {
+    if (swiglu)
+      return hz ? w4::reg_grouped_launch_t<1, true, true>(map, p, grid, stream) : w4::reg_grouped_launch_t<1, false, true>(map, p, grid, stream);
+    return hz ? w4::reg_grouped_launch_t<1, true, false>(map, p, grid, stream) : w4::reg_grouped_launch_t<1, false, false>(map, p, grid, stream);
+  }
+  if (swiglu)
+    return hz ? w4::reg_grouped_launch_t<2, true, true>(map, p, grid, stream) : w4::reg_grouped_launch_t<2, false, true>(map, p, grid, stream);
+  return hz ? w4::reg_grouped_launch_t<2, true, false>(map, p, grid, stream) : w4::reg_grouped_launch_t<2, false, false>(map, p, grid, stream);
 }
 
 }  // namespace hq

@@ -470,11 +470,17 @@ def test_grouped_token_tile_rule():
     """Grouped GEMMs: the token tile covers a typical expert's rows (avg +
     2 sd of Poisson(avg) rows per expert); above 128 it is 256 only for K of
     at least 4096 and at most 511 experts (the 256-token tile's output
-    transposes sit beside the expert tables), else 128."""
+    transposes sit beside the expert tables), else 128.  INT4 experts whose
+    typical rows fit 8 tokens run on the register path (8-token units)."""
+    def plan(n, k, e, rows, fmt=hq.HQ_FMT_INT4):
+        d = hq.hq_quant_desc_init(fmt, n, k, 128, 0, e)
+        return hq.hq_plan_describe(d, rows)
     def tile(n, k, e, rows):
-        d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, 0, e)
-        return hq.hq_plan_describe(d, rows).tile_m
-    assert tile(4096, 7168, 256, 64 * 8) == 16          # T=64, top-8 of 256: 2 rows per expert
+        return plan(n, k, e, rows).tile_m
+    p64 = plan(4096, 7168, 256, 64 * 8)                 # T=64, top-8 of 256: 2 rows per expert
+    assert (p64.kernel, p64.tile_m, p64.grid) == (4, 8, 148 * 3)
+    p64i3 = plan(4096, 7168, 256, 64 * 8, hq.HQ_FMT_INT3)   # INT3: no register path, 16-token tiles
+    assert (p64i3.kernel, p64i3.tile_m) == (2, 16)
     assert tile(4096, 7168, 256, 1024 * 8) == 64        # 32 rows per expert
     assert tile(4096, 7168, 256, 8192 * 8) == 256       # 256 rows per expert, long K
     assert tile(7168, 2048, 256, 8192 * 8) == 128       # short K

@@ -105,7 +105,7 @@ def _grouped(desc, blob, a_sorted, off, rows, n, tuning=None):
 
 
 @pytest.mark.parametrize("tile_m,variant", [(0, 0), (16, 0), (32, 0), (64, 0), (128, 0), (256, 0), (16, 2), (32, 2),
-                                            (64, 2)])
+                                            (64, 2), (0, 3), (16, 3)])
 def test_grouped_reduced_config_full_output(tile_m, variant):
     e, n, k, t, topk = 8, 256, 512, 40, 2
     q, s, _ = synth.w4a16_weights(n, k, 128, False, seed=5000, experts=e)
@@ -322,7 +322,8 @@ def _layer_oracle(x_bits, logits, q1, s1, q2, s2, k, e, inter, fused=False):
 @pytest.mark.parametrize("tile_m,variant,fmt", [(0, 0, hq.HQ_FMT_INT4), (16, 0, hq.HQ_FMT_INT4),
                                                 (64, 0, hq.HQ_FMT_INT4), (128, 0, hq.HQ_FMT_INT4),
                                                 (256, 0, hq.HQ_FMT_INT4), (32, 1, hq.HQ_FMT_INT4),
-                                                (0, 0, hq.HQ_FMT_INT3), (0, 0, hq.HQ_FMT_MXFP4_A16)])
+                                                (0, 0, hq.HQ_FMT_INT3), (0, 0, hq.HQ_FMT_MXFP4_A16),
+                                                (0, 3, hq.HQ_FMT_INT4), (16, 3, hq.HQ_FMT_INT4)])
 def test_grouped_swiglu_fused_reduced_config(tile_m, variant, fmt):
     """Gate+up grouped GEMM with the SwiGLU epilogue (weights packed in the
     gated row order) against the oracle's fp64 gate and up values: 8

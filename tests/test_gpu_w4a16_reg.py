@@ -3,15 +3,18 @@ INT4 at 1..16 tokens, codes dequantized straight into mma.sync fragments)
 against the fp64 oracle, through the C ABI: full outputs on shapes with
 ragged token counts, ragged N and several K splits, the bench's full-size
 M-sweep shapes (every row), bitwise repeats, counters left at zero,
-guard bands, exact zeros, and the plan it reports."""
+guard bands, exact zeros, and the plan it reports; the grouped MoE GEMM on
+the same path (8- and 16-token units, experts of many tokens, empty
+experts, the fused SwiGLU epilogue)."""
 
 import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import check_gemm, workspace
+from gpu_helpers import check_gemm, check_swiglu, workspace
 from oracle import formats as F
 from oracle import gemm as G
+from oracle import moe as R
 from quantized_gemm_bit_b200 import hq, synth
 from quantized_gemm_bit_b200.build import build
 
@@ -142,3 +145,62 @@ def test_register_path_request_that_does_not_apply():
     check_gemm(c, G.w4a16_ref(_bits(a), q, s, z, 128), k, "reg request m=17")
     d3 = hq.hq_quant_desc_init(hq.HQ_FMT_INT3, n, k, 128, 0, 1)
     assert hq.hq_plan_describe(d3, 8, REG).kernel != 4
+
+
+def _moe_case(e, t, topk, n, k, asym, seed, heavy=None, gated=False):
+    q, s, z = synth.w4a16_weights(n, k, 128, asym, seed, experts=e)
+    d = hq.hq_quant_desc_init(hq.HQ_FMT_INT4, n, k, 128, int(asym), e)
+    pack = hq.hq_pack_weights_gated if gated else hq.hq_pack_weights
+    blob = torch.from_numpy(pack(d, q, s, z)).to(DEV)
+    logits = synth.router_logits(t, e, seed=seed + 1)
+    logits[:, 1] = -100.0                      # expert 1 never chosen: an empty group
+    if heavy is not None:
+        logits[:heavy, 2] = 100.0              # expert 2 takes `heavy` rows: several token tiles
+    ids = R.topk_by_logit(logits.numpy(), topk)
+    _, off, src = R.permute(ids, e)
+    a = synth.bf16_normal(t, k, seed=seed + 2)
+    a_sorted = R.gather_rows(_bits(a), src, topk)
+    a_dev = torch.from_numpy(a_sorted.view(np.int16)).view(torch.bfloat16).to(DEV)
+    off_dev = torch.from_numpy(off.astype(np.int32)).to(DEV)
+    zn = None if z is None else z.numpy()
+    return d, blob, a_sorted, a_dev, off, off_dev, (q.numpy(), s.numpy(), zn)
+
+
+@pytest.mark.parametrize("e,t,topk,tile_m,asym,heavy", [
+    (16, 24, 2, 0, False, None), (16, 24, 2, 0, True, 21), (16, 24, 2, 16, True, 40), (64, 7, 4, 0, False, None),
+])
+def test_register_path_grouped_full_output(e, t, topk, tile_m, asym, heavy):
+    """Grouped MoE on the register path: 8-token units (a few rows per
+    expert) and 16-token units (tile_m=16), an expert whose rows span
+    several units, an empty expert, ragged N."""
+    n, k = 384, 1024
+    d, blob, a_sorted, a_dev, off, off_dev, (q, s, z) = _moe_case(e, t, topk, n, k, asym, 7000 + e + t,
+                                                                  None if heavy is None else min(heavy, t))
+    tuning = hq.Tuning(tile_m=tile_m, variant=3)
+    plan = hq.hq_plan_describe(d, t * topk, tuning)
+    assert plan.kernel == 4 and plan.tile_m == (16 if tile_m == 16 else 8)
+    rows = t * topk
+    c = torch.full((rows, n), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, rows, tuning))
+    hq.hq_grouped_gemm_moe(d, blob, a_dev, off_dev, rows, c, ws, tuning)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    _, ref = G.grouped_w4a16_ref(a_sorted, off, q, s, z, 128)
+    check_gemm(c, ref, k, f"reg grouped e={e} t={t} tile_m={tile_m} asym={asym} heavy={heavy}")
+
+
+@pytest.mark.parametrize("tile_m,heavy", [(0, None), (0, 12), (16, 20)])
+def test_register_path_grouped_swiglu(tile_m, heavy):
+    """Gate+up on the register path with the SwiGLU epilogue (gated row
+    order: each warp's gate and up rows of the same features)."""
+    e, t, topk, inter, k = 16, 24, 2, 192, 1024
+    n = 2 * inter
+    d, blob, a_sorted, a_dev, off, off_dev, (q, s, z) = _moe_case(e, t, topk, n, k, True, 7100, heavy, gated=True)
+    tuning = hq.Tuning(tile_m=tile_m, variant=3)
+    assert hq.hq_plan_describe(d, t * topk, tuning).kernel == 4
+    rows = t * topk
+    h = torch.full((rows, inter), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ws = workspace(hq.hq_workspace_size(d, rows, tuning))
+    hq.hq_grouped_gemm_moe_swiglu(d, blob, a_dev, off_dev, rows, h, ws, tuning)
+    assert hq.hq_check_device_status(ws) == hq.HQ_OK
+    _, gu = G.grouped_w4a16_ref(a_sorted, off, q, s, z, 128)
+    check_swiglu(h, gu, inter, k, f"reg grouped swiglu tile_m={tile_m} heavy={heavy}")
