@@ -63,26 +63,23 @@ def load_peaks():
 # holds for the kernel sources it ran (TRAFFIC_SOURCES, a fingerprint of
 # csrc/ and include/): once they change, `traffic` reads null until the
 # capture is taken again.
-TRAFFIC_COMMIT = "0f71beb"
-# sources since the capture differ only in the plan the library reports
-# (hq_plan_describe: the register path's token tile and ring depth) and in
-# the names of two constants; the kernels are the same
-TRAFFIC_SOURCES = "8c40a856c98394c1"
+TRAFFIC_COMMIT = "da1bb90"
+TRAFFIC_SOURCES = "df35bf2c2cb72083"
 TRAFFIC_BYTES = {
-    (1, 7168, 18432): 68518400,
-    (4, 7168, 18432): 68257280,
-    (16, 7168, 18432): 68399104,
-    (64, 7168, 18432): 71279360,
-    (256, 7168, 18432): 75675648,
-    (1024, 7168, 18432): 152192512,
-    (4096, 7168, 18432): 404947712,
-    (1, 18432, 7168): 68235520,
-    (4, 18432, 7168): 68338944,
-    (16, 18432, 7168): 68763136,
-    (64, 18432, 7168): 73953792,
-    (256, 18432, 7168): 86066944,
-    (1024, 18432, 7168): 203194880,
-    (4096, 18432, 7168): 715784960,
+    (1, 7168, 18432): 68638976,
+    (4, 7168, 18432): 68249856,
+    (16, 7168, 18432): 68398592,
+    (64, 7168, 18432): 71147008,
+    (256, 7168, 18432): 75643648,
+    (1024, 7168, 18432): 158340864,
+    (4096, 7168, 18432): 422855936,
+    (1, 18432, 7168): 68249344,
+    (4, 18432, 7168): 68308480,
+    (16, 18432, 7168): 68766208,
+    (64, 18432, 7168): 74269440,
+    (256, 18432, 7168): 85654528,
+    (1024, 18432, 7168): 199288832,
+    (4096, 18432, 7168): 710096640,
 }
 
 
