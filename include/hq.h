@@ -151,11 +151,16 @@ typedef struct {
  *              go to the tensor core and each 128-K group's scale is
  *              applied to its fp32 group sum (no rounding of w or s);
  *              larger tiles as 1.  INT4, INT3 and INT2 weights.
- *              3 = dense INT4 GEMMs of 1 to 16 tokens: the register-path
- *              kernel (codes dequantized straight into mma.sync register
- *              fragments, exact (q - z) with each group's scale applied to
- *              its fp32 sum, as 2); split_k = CTAs per weight tile (0: the
- *              library's split).  Other calls run the library's choice.
+ *              3 = the register-path kernels (whole records staged in
+ *              shared memory by bulk copies, codes read with ldmatrix into
+ *              mma.sync register fragments, exact (q - z) with each group's
+ *              scale applied to its fp32 sum, as 2), INT4 weights only:
+ *              dense GEMMs of 1 to 16 tokens (split_k = CTAs per weight
+ *              tile, 0: the library's split) and grouped MoE GEMMs in 8- or
+ *              16-token units (tile_m 16 forces 16).  The library's choice
+ *              for dense INT4 at 1 to 16 tokens and for grouped INT4 whose
+ *              typical expert rows fit 8 tokens.  Other calls run the
+ *              library's choice.
  *              Block-scaled GEMMs: 0.                                     */
 typedef struct {
   int32_t tile_m, tile_n, tile_k, stages, split_k, cta_group, variant;

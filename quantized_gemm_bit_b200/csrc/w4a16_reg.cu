@@ -28,7 +28,10 @@
 //   * the K range of a tile is split over a few CTAs so that the grid fills
 //     the SMs; each CTA writes an fp32 partial tile, and the last of a tile's
 //     CTAs (a counter per tile) adds the partials in slice order and writes
-//     the bf16 output, so results repeat bit for bit.
+//     the bf16 output, so results repeat bit for bit;
+//   * grouped MoE (experts of a few tokens): persistent CTAs walk (expert,
+//     weight tile, token tile) units over the whole K range, the ring
+//     streaming across units (w4a16_reg_grouped_kernel, below).
 // mma.sync is the older tensor-core path (on B200 a 16x8x16 MMA issues about
 // every 2.7 SM cycles, near 0.44 PFLOP/s for the GPU); at 1-8 tokens the MMAs
 // are a small share of the time, at 9-16 they start to show.  Measured on
